@@ -1,0 +1,334 @@
+"""CPU oracle for the quantised-matmul sum-check prover -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference arm may import this package. The product path (the CUDA library
+and its binding in ``sum_check_prover_b200``) never imports it and shares no
+code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, single-threaded, every field
+operation an ``unsigned __int128`` product or sum reduced with ``% P``). This
+module only builds that file with gcc and marshals numpy arrays through
+ctypes. The one piece of logic here is wiring a workload's linked sites
+(an operand that is another site's output) on the host.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+P = 0xFFFFFFFF00000001
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "oracle.c"
+_LIB = _HERE / "liboracle.so"
+_lib = None
+
+REASONS = {
+    0: "accept",
+    1: "format",
+    2: "claim",
+    3: "mm_round",
+    4: "mm_final",
+    5: "mm_A",
+    6: "mm_B",
+    7: "root_rem",
+    8: "root_clamp",
+    9: "gkr_round",
+    10: "gkr_final",
+    11: "leaf_P",
+    12: "leaf_Q",
+    13: "leaf_open",
+    14: "args",
+}
+
+
+def build(force: bool = False) -> Path:
+    """Compile oracle.c into liboracle.so with gcc (no GPU needed)."""
+    if force or not _LIB.exists() or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB.with_suffix(f".so.{os.getpid()}")
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(tmp), str(_SRC)])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Site(C.Structure):
+    _fields_ = [("w", C.c_void_p), ("scales", C.c_void_p), ("xt", C.c_void_p),
+                ("w_bits", C.c_int32), ("M", C.c_int32), ("K", C.c_int32), ("N", C.c_int32),
+                ("k_shift", C.c_int32), ("pad", C.c_int32)]
+
+
+class _Wit(C.Structure):
+    _fields_ = [("q", C.c_void_p), ("r", C.c_void_p), ("y", C.c_void_p)]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = C.CDLL(str(_LIB))
+        u64, vp = C.c_uint64, C.c_void_p
+        for nm in ("orc_fadd", "orc_fsub", "orc_fmul", "orc_fpow"):
+            getattr(L, nm).restype = u64
+            getattr(L, nm).argtypes = [u64, u64]
+        L.orc_finv.restype = u64
+        L.orc_finv.argtypes = [u64]
+        L.orc_fint.restype = u64
+        L.orc_fint.argtypes = [C.c_int64]
+        L.orc_sha256.argtypes = [vp, u64, vp]
+        L.orc_tree_digest.argtypes = [vp, u64, vp]
+        L.orc_tx_new.restype = vp
+        L.orc_tx_new.argtypes = [u64]
+        L.orc_tx_free.argtypes = [vp]
+        L.orc_tx_state.argtypes = [vp, vp]
+        L.orc_tx_absorb_h.argtypes = [vp, C.c_char_p, vp, u64]
+        L.orc_tx_squeeze_h.restype = u64
+        L.orc_tx_squeeze_h.argtypes = [vp, C.c_char_p]
+        L.orc_eq_table.argtypes = [vp, C.c_int, vp]
+        L.orc_mle_eval.restype = u64
+        L.orc_mle_eval.argtypes = [vp, u64, vp, C.c_int]
+        L.orc_lagrange.restype = u64
+        L.orc_lagrange.argtypes = [vp, C.c_int, u64]
+        L.orc_witness.restype = C.c_int
+        L.orc_witness.argtypes = [C.POINTER(_Site), vp, vp, vp]
+        L.orc_partial_w.argtypes = [C.POINTER(_Site), vp, C.c_int, vp]
+        L.orc_partial_x.argtypes = [C.POINTER(_Site), vp, C.c_int, vp]
+        L.orc_partial_rows.argtypes = [vp, C.c_int, vp, C.c_int, C.c_int, vp, C.c_int, vp]
+        L.orc_claim.restype = u64
+        L.orc_claim.argtypes = [vp, vp, C.c_int, C.c_int, C.c_int, vp, C.c_int, vp, C.c_int]
+        L.orc_prove.restype = C.c_int
+        L.orc_prove.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64,
+                                C.POINTER(u64), vp, C.POINTER(u64)]
+        L.orc_verify.restype = C.c_int
+        L.orc_verify.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp]
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _u64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.uint64))
+
+
+def log2_ceil(n: int) -> int:
+    v = 0
+    while (1 << v) < n:
+        v += 1
+    return v
+
+
+# ---- primitives -----------------------------------------------------------
+
+def fadd(a, b): return lib().orc_fadd(a, b)
+def fsub(a, b): return lib().orc_fsub(a, b)
+def fmul(a, b): return lib().orc_fmul(a, b)
+def fpow(a, e): return lib().orc_fpow(a, e)
+def finv(a): return lib().orc_finv(a)
+def fint(v): return lib().orc_fint(int(v))
+
+
+def sha256(data: bytes) -> bytes:
+    out = C.create_string_buffer(32)
+    buf = C.create_string_buffer(bytes(data), len(data) or 1)
+    lib().orc_sha256(buf, len(data), out)
+    return out.raw
+
+
+def tree_digest(data) -> bytes:
+    b = np.frombuffer(bytes(data), dtype=np.uint8) if isinstance(data, (bytes, bytearray)) else \
+        np.ascontiguousarray(data).view(np.uint8).reshape(-1)
+    out = C.create_string_buffer(32)
+    lib().orc_tree_digest(_ptr(b) if b.size else None, b.size, out)
+    return out.raw
+
+
+class Transcript:
+    def __init__(self, seed: int):
+        self._h = lib().orc_tx_new(seed)
+
+    def absorb(self, label: str, data: bytes):
+        buf = C.create_string_buffer(bytes(data), len(data) or 1)
+        lib().orc_tx_absorb_h(self._h, label.encode(), buf, len(data))
+
+    def squeeze(self, label: str) -> int:
+        return lib().orc_tx_squeeze_h(self._h, label.encode())
+
+    def state(self) -> bytes:
+        out = C.create_string_buffer(32)
+        lib().orc_tx_state(self._h, out)
+        return out.raw
+
+    def __del__(self):
+        if getattr(self, "_h", None) and _lib is not None:
+            _lib.orc_tx_free(self._h)
+            self._h = None
+
+
+def eq_table(z) -> np.ndarray:
+    z = _u64(z)
+    out = np.zeros(1 << len(z), dtype=np.uint64)
+    lib().orc_eq_table(_ptr(z) if len(z) else None, len(z), _ptr(out))
+    return out
+
+
+def mle_eval(vals, z) -> int:
+    vals, z = _u64(vals), _u64(z)
+    return lib().orc_mle_eval(_ptr(vals), len(vals), _ptr(z) if len(z) else None, len(z))
+
+
+def lagrange(g, x: int) -> int:
+    g = _u64(g)
+    return lib().orc_lagrange(_ptr(g), len(g), x)
+
+
+# ---- sites ----------------------------------------------------------------
+
+def _csite(s, keep: list) -> _Site:
+    w = np.ascontiguousarray(s.w)
+    xt = np.ascontiguousarray(s.xt)
+    sc = None if s.scales is None else np.ascontiguousarray(s.scales)
+    keep.extend([w, xt, sc])
+    return _Site(_ptr(w), _ptr(sc), _ptr(xt), s.w_bits, s.M, s.K, s.N, s.k_shift, 0)
+
+
+def witness(s):
+    """(q, r, y) of one site, each N x M (token-major)."""
+    q = np.zeros((s.N, s.M), dtype=np.int32)
+    r = np.zeros((s.N, s.M), dtype=np.int32)
+    y = np.zeros((s.N, s.M), dtype=np.int8)
+    keep = []
+    cs = _csite(s, keep)
+    rc = lib().orc_witness(C.byref(cs), _ptr(q), _ptr(r), _ptr(y))
+    if rc != 0:
+        raise ValueError("accumulator exceeds 31 bits for this site")
+    return q, r, y
+
+
+def partial_w(s, z) -> np.ndarray:
+    z = _u64(z)
+    out = np.zeros(1 << log2_ceil(s.K), dtype=np.uint64)
+    keep = []
+    cs = _csite(s, keep)
+    lib().orc_partial_w(C.byref(cs), _ptr(z) if len(z) else None, len(z), _ptr(out))
+    return out
+
+
+def partial_x(s, z) -> np.ndarray:
+    z = _u64(z)
+    out = np.zeros(1 << log2_ceil(s.K), dtype=np.uint64)
+    keep = []
+    cs = _csite(s, keep)
+    lib().orc_partial_x(C.byref(cs), _ptr(z) if len(z) else None, len(z), _ptr(out))
+    return out
+
+
+def partial_rows(mat, bits: int, scales, rows: int, cols: int, z) -> np.ndarray:
+    z = _u64(z)
+    mat = np.ascontiguousarray(mat)
+    sc = None if scales is None else np.ascontiguousarray(scales)
+    out = np.zeros(1 << log2_ceil(cols), dtype=np.uint64)
+    lib().orc_partial_rows(_ptr(mat), bits, _ptr(sc), rows, cols, _ptr(z) if len(z) else None,
+                           len(z), _ptr(out))
+    return out
+
+
+def claim(q, r, M, N, k, zr, zc) -> int:
+    q = np.ascontiguousarray(q, dtype=np.int32)
+    r = np.ascontiguousarray(r, dtype=np.int32)
+    zr, zc = _u64(zr), _u64(zc)
+    return lib().orc_claim(_ptr(q), _ptr(r), M, N, k, _ptr(zr) if len(zr) else None, len(zr),
+                           _ptr(zc) if len(zc) else None, len(zc))
+
+
+# ---- workloads --------------------------------------------------------------
+
+class Resolved:
+    """A workload's sites with every linked operand materialised, plus the witness."""
+
+    def __init__(self, sites, wits, groups):
+        self.sites = sites
+        self.wits = wits
+        self.groups = groups
+
+
+def resolve(wl) -> Resolved:
+    """Compute every site's witness in stage order, placing grouped outputs into
+    their shared buffers and reading linked operands out of earlier outputs."""
+    import copy
+    sites = [copy.copy(s) for s in wl.sites]
+    groups = {g: {"q": np.zeros(shp, np.int32), "r": np.zeros(shp, np.int32), "y": np.zeros(shp, np.int8)}
+              for g, shp in wl.groups.items()}
+    wits = [None] * len(sites)
+
+    def out_buffer(idx):
+        s = sites[idx]
+        if s.out_group is not None:
+            return groups[s.out_group[0]]["y"].reshape(-1), 0
+        return wits[idx][2].reshape(-1), 0
+
+    for stage in sorted({s.stage for s in sites}):
+        for i, s in enumerate(sites):
+            if s.stage != stage:
+                continue
+            if s.w_link is not None:
+                src, off = out_buffer(s.w_link[0])
+                s.w = src[off + s.w_link[1]: off + s.w_link[1] + s.M * s.K].reshape(s.M, s.K).copy()
+            if s.xt_link is not None:
+                src, off = out_buffer(s.xt_link[0])
+                s.xt = src[off + s.xt_link[1]: off + s.xt_link[1] + s.N * s.K].reshape(s.N, s.K).copy()
+            q, r, y = witness(s)
+            if s.out_group is not None:
+                g = groups[s.out_group[0]]
+                o = s.out_group[1]
+                n = s.M * s.N
+                g["q"].reshape(-1)[o:o + n] = q.reshape(-1)
+                g["r"].reshape(-1)[o:o + n] = r.reshape(-1)
+                g["y"].reshape(-1)[o:o + n] = y.reshape(-1)
+            wits[i] = (q, r, y)
+    return Resolved(sites, wits, groups)
+
+
+def _marshal(sites, wits, keep):
+    n = len(sites)
+    cs = (_Site * n)()
+    cw = (_Wit * n)()
+    for i, (s, w) in enumerate(zip(sites, wits)):
+        cs[i] = _csite(s, keep)
+        q, r, y = (np.ascontiguousarray(a) for a in w)
+        keep.extend([q, r, y])
+        cw[i] = _Wit(_ptr(q), _ptr(r), _ptr(y))
+    return cs, cw
+
+
+def prove(seed: int, sites, wits):
+    """Full proof. Returns (proof bytes, [state after commit, after matmul, after lookup], matmul section length)."""
+    keep = []
+    cs, cw = _marshal(sites, wits, keep)
+    n = C.c_uint64(0)
+    off = C.c_uint64(0)
+    states = C.create_string_buffer(96)
+    rc = lib().orc_prove(seed, cs, len(sites), cw, None, 0, C.byref(n), states, C.byref(off))
+    if rc not in (0, -2):
+        raise ValueError(f"orc_prove rejected the statement ({rc})")
+    buf = np.zeros(max(1, n.value), dtype=np.uint8)
+    rc = lib().orc_prove(seed, cs, len(sites), cw, _ptr(buf), n.value, C.byref(n), states, C.byref(off))
+    if rc != 0:
+        raise ValueError(f"orc_prove failed ({rc})")
+    st = states.raw
+    return buf[: n.value].tobytes(), [st[0:32], st[32:64], st[64:96]], off.value
+
+
+def verify(seed: int, sites, wits, proof: bytes):
+    """Returns (reason_name, detail) -- reason 'accept' for a valid proof."""
+    keep = []
+    cs, cw = _marshal(sites, wits, keep)
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    rc = lib().orc_verify(seed, cs, len(sites), cw, _ptr(pb), len(proof), _ptr(det))
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

@@ -1,0 +1,1169 @@
+/*
+ * oracle.c -- reference prover and verifier for the quantised-matmul sum-check
+ * with LogUp rescale/clamp lookups.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the slow, obviously-correct CPU
+ * statement of what the CUDA library computes. Only the test-suite, the smoke
+ * check and the benchmark's CPU-baseline / reference arm load it. It shares no
+ * code, header, table or helper with the CUDA library: the library must reach
+ * the same bytes on its own.
+ *
+ * Style rules kept on purpose: single-threaded; every field operation is
+ * (unsigned __int128 arithmetic) % P; every sum is the plain loop of its
+ * definition; no blocking, fusion or reordering.
+ *
+ * Sources (page title, section):
+ *  - "How fast can FlashProve go", 2 Background: the prover commits the
+ *    intermediate values; sum-check reduces each polynomial operation (the
+ *    matmuls) to claims on committed values and weights; non-polynomial steps
+ *    (rescale, clamp) are proven by lookups; Fiat-Shamir makes each challenge
+ *    a hash of everything sent so far.
+ *  - same page, 3.1 Committing intermediate values: a rescale
+ *    g = round(g_hat / 2^k) is proven by committing the remainder
+ *    r = g_hat - 2^k g, using 2^k g + r in place of g_hat in the matmul
+ *    sum-check, and looking r up to show it is small; the field is Goldilocks
+ *    2^64 - 2^32 + 1.
+ *  - same page, 2 Background and 2.1 Batching: many claims are merged into one
+ *    (here: random linear combination of per-matmul claims).
+ *  - same page, 4 Tighter Rooflines: a lookup compares a product over the keys
+ *    with one over the table; the key side is a binary tree whose every level
+ *    is proven with sum-check.
+ *  - "Towards Proving Frontier-Scale LLM Inference", How the prover works /
+ *    The proof system: lookups by logarithmic derivatives (LogUp), whose
+ *    fractions we sum in the same binary tree.
+ * Every point the pages leave open (transcript encoding, bit order, rounding
+ * tie, table layout, batching of the two lookups) follows the protocol
+ * specification written out in the repository's design notes; the choices
+ * are repeated next to the code that makes them.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef uint64_t u64;
+typedef uint32_t u32;
+typedef unsigned __int128 u128;
+
+#define ORC_P 0xFFFFFFFF00000001ull
+
+/* ------------------------------------------------------------------------ */
+/* Goldilocks field: canonical representatives in [0, P).                    */
+/* ------------------------------------------------------------------------ */
+
+u64 orc_fadd(u64 a, u64 b) { return (u64)(((u128)a + (u128)b) % ORC_P); }
+u64 orc_fsub(u64 a, u64 b) { return (u64)(((u128)a + (u128)ORC_P - (u128)(b % ORC_P)) % ORC_P); }
+u64 orc_fmul(u64 a, u64 b) { return (u64)(((u128)a * (u128)b) % ORC_P); }
+
+u64 orc_fpow(u64 a, u64 e) {
+    u64 r = 1, b = a % ORC_P;
+    while (e) {
+        if (e & 1) r = orc_fmul(r, b);
+        b = orc_fmul(b, b);
+        e >>= 1;
+    }
+    return r;
+}
+
+/* Fermat: a^(P-2) is the inverse of a non-zero a. */
+u64 orc_finv(u64 a) { return orc_fpow(a, ORC_P - 2); }
+
+/* A signed integer lifted into the field: v mod P in [0, P). */
+u64 orc_fint(int64_t v) {
+    if (v >= 0) return (u64)v % ORC_P;
+    u64 mag = (u64)(-(v + 1)) + 1u; /* |v| without overflow */
+    return orc_fsub(0, mag % ORC_P);
+}
+
+/* ------------------------------------------------------------------------ */
+/* SHA-256, written from FIPS 180-4 (sections 4.1.2, 4.2.2, 5.1.1, 6.2).      */
+/* ------------------------------------------------------------------------ */
+
+static const u32 SHA_K[64] = {
+    0x428a2f98, 0x71374491, 0xb5c0fbcf, 0xe9b5dba5, 0x3956c25b, 0x59f111f1, 0x923f82a4, 0xab1c5ed5,
+    0xd807aa98, 0x12835b01, 0x243185be, 0x550c7dc3, 0x72be5d74, 0x80deb1fe, 0x9bdc06a7, 0xc19bf174,
+    0xe49b69c1, 0xefbe4786, 0x0fc19dc6, 0x240ca1cc, 0x2de92c6f, 0x4a7484aa, 0x5cb0a9dc, 0x76f988da,
+    0x983e5152, 0xa831c66d, 0xb00327c8, 0xbf597fc7, 0xc6e00bf3, 0xd5a79147, 0x06ca6351, 0x14292967,
+    0x27b70a85, 0x2e1b2138, 0x4d2c6dfc, 0x53380d13, 0x650a7354, 0x766a0abb, 0x81c2c92e, 0x92722c85,
+    0xa2bfe8a1, 0xa81a664b, 0xc24b8b70, 0xc76c51a3, 0xd192e819, 0xd6990624, 0xf40e3585, 0x106aa070,
+    0x19a4c116, 0x1e376c08, 0x2748774c, 0x34b0bcb5, 0x391c0cb3, 0x4ed8aa4a, 0x5b9cca4f, 0x682e6ff3,
+    0x748f82ee, 0x78a5636f, 0x84c87814, 0x8cc70208, 0x90befffa, 0xa4506ceb, 0xbef9a3f7, 0xc67178f2};
+
+typedef struct {
+    u32 h[8];
+    uint8_t buf[64];
+    u64 total; /* bytes fed so far */
+    u32 fill;  /* bytes waiting in buf */
+} sha_ctx;
+
+static u32 rotr32(u32 x, int n) { return (x >> n) | (x << (32 - n)); }
+
+static void sha_compress(u32 h[8], const uint8_t blk[64]) {
+    u32 w[64];
+    for (int t = 0; t < 16; t++)
+        w[t] = ((u32)blk[4 * t] << 24) | ((u32)blk[4 * t + 1] << 16) | ((u32)blk[4 * t + 2] << 8) |
+               (u32)blk[4 * t + 3];
+    for (int t = 16; t < 64; t++) {
+        u32 s0 = rotr32(w[t - 15], 7) ^ rotr32(w[t - 15], 18) ^ (w[t - 15] >> 3);
+        u32 s1 = rotr32(w[t - 2], 17) ^ rotr32(w[t - 2], 19) ^ (w[t - 2] >> 10);
+        w[t] = w[t - 16] + s0 + w[t - 7] + s1;
+    }
+    u32 a = h[0], b = h[1], c = h[2], d = h[3], e = h[4], f = h[5], g = h[6], hh = h[7];
+    for (int t = 0; t < 64; t++) {
+        u32 S1 = rotr32(e, 6) ^ rotr32(e, 11) ^ rotr32(e, 25);
+        u32 ch = (e & f) ^ (~e & g);
+        u32 T1 = hh + S1 + ch + SHA_K[t] + w[t];
+        u32 S0 = rotr32(a, 2) ^ rotr32(a, 13) ^ rotr32(a, 22);
+        u32 mj = (a & b) ^ (a & c) ^ (b & c);
+        u32 T2 = S0 + mj;
+        hh = g; g = f; f = e; e = d + T1; d = c; c = b; b = a; a = T1 + T2;
+    }
+    h[0] += a; h[1] += b; h[2] += c; h[3] += d; h[4] += e; h[5] += f; h[6] += g; h[7] += hh;
+}
+
+static void sha_init(sha_ctx* c) {
+    static const u32 H0[8] = {0x6a09e667, 0xbb67ae85, 0x3c6ef372, 0xa54ff53a,
+                              0x510e527f, 0x9b05688c, 0x1f83d9ab, 0x5be0cd19};
+    memcpy(c->h, H0, sizeof H0);
+    c->total = 0;
+    c->fill = 0;
+}
+
+static void sha_update(sha_ctx* c, const void* data, u64 n) {
+    const uint8_t* p = (const uint8_t*)data;
+    c->total += n;
+    while (n > 0) {
+        u32 take = 64 - c->fill;
+        if (take > n) take = (u32)n;
+        memcpy(c->buf + c->fill, p, take);
+        c->fill += take;
+        p += take;
+        n -= take;
+        if (c->fill == 64) {
+            sha_compress(c->h, c->buf);
+            c->fill = 0;
+        }
+    }
+}
+
+static void sha_final(sha_ctx* c, uint8_t out[32]) {
+    u64 bits = c->total * 8u;
+    uint8_t one = 0x80, zero = 0;
+    sha_update(c, &one, 1);
+    while (c->fill != 56) sha_update(c, &zero, 1);
+    uint8_t lenb[8];
+    for (int i = 0; i < 8; i++) lenb[i] = (uint8_t)(bits >> (56 - 8 * i));
+    sha_update(c, lenb, 8);
+    for (int i = 0; i < 8; i++) {
+        out[4 * i] = (uint8_t)(c->h[i] >> 24);
+        out[4 * i + 1] = (uint8_t)(c->h[i] >> 16);
+        out[4 * i + 2] = (uint8_t)(c->h[i] >> 8);
+        out[4 * i + 3] = (uint8_t)(c->h[i]);
+    }
+}
+
+void orc_sha256(const void* data, u64 n, uint8_t out[32]) {
+    sha_ctx c;
+    sha_init(&c);
+    sha_update(&c, data, n);
+    sha_final(&c, out);
+}
+
+static void put_le(uint8_t* p, u64 v, int nbytes) {
+    for (int i = 0; i < nbytes; i++) p[i] = (uint8_t)(v >> (8 * i));
+}
+
+static u64 get_le(const uint8_t* p, int nbytes) {
+    u64 v = 0;
+    for (int i = 0; i < nbytes; i++) v |= (u64)p[i] << (8 * i);
+    return v;
+}
+
+/*
+ * Tree digest of a byte string (binds the committed buffers into the
+ * transcript; the pages' commitment scheme itself is out of scope).
+ *   level 0: SHA-256 of each 1024-byte chunk (the last one may be short; an
+ *            empty string has one empty chunk);
+ *   level l+1: SHA-256 of each run of up to 32 consecutive level-l digests;
+ *   until one digest is left; result = SHA-256(u64le(len) || that digest).
+ */
+#define ORC_CHUNK 1024u
+void orc_tree_digest(const void* data, u64 len, uint8_t out[32]) {
+    const uint8_t* p = (const uint8_t*)data;
+    u64 cnt = len == 0 ? 1 : (len + ORC_CHUNK - 1) / ORC_CHUNK;
+    uint8_t* lv = (uint8_t*)malloc(cnt * 32);
+    for (u64 c = 0; c < cnt; c++) {
+        u64 off = c * ORC_CHUNK;
+        u64 n = len - off < ORC_CHUNK ? len - off : ORC_CHUNK;
+        if (len == 0) n = 0;
+        orc_sha256(p + off, n, lv + 32 * c);
+    }
+    while (cnt > 1) {
+        u64 nc = (cnt + 31) / 32;
+        uint8_t* nx = (uint8_t*)malloc(nc * 32);
+        for (u64 g = 0; g < nc; g++) {
+            u64 m = cnt - 32 * g < 32 ? cnt - 32 * g : 32;
+            orc_sha256(lv + 32 * 32 * g, 32 * m, nx + 32 * g);
+        }
+        free(lv);
+        lv = nx;
+        cnt = nc;
+    }
+    uint8_t fin[40];
+    put_le(fin, len, 8);
+    memcpy(fin + 8, lv, 32);
+    orc_sha256(fin, 40, out);
+    free(lv);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Fiat-Shamir transcript ("How fast can FlashProve go", 2 Background: each   */
+/* challenge hashes everything the prover sent; SHA-256 instead of BLAKE2b).  */
+/*   state0 = SHA256("FPSC-v1" || u64le(seed))                                */
+/*   absorb: state = SHA256(state || u32le(|label|) || label || u64le(n) || data) */
+/*   squeeze: h = SHA256(state || "sq" || u32le(|label|) || label || u32le(ctr)) */
+/*            for ctr = 0, 1, ...; the first h whose low 8 bytes (LE) are < P  */
+/*            becomes the state and that value the challenge.                 */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    uint8_t st[32];
+} orc_tx;
+
+void orc_tx_init(orc_tx* t, u64 seed) {
+    uint8_t b[15];
+    memcpy(b, "FPSC-v1", 7);
+    put_le(b + 7, seed, 8);
+    orc_sha256(b, 15, t->st);
+}
+
+void orc_tx_absorb(orc_tx* t, const char* label, const void* data, u64 n) {
+    sha_ctx c;
+    uint8_t l4[4], l8[8];
+    u32 ll = (u32)strlen(label);
+    sha_init(&c);
+    sha_update(&c, t->st, 32);
+    put_le(l4, ll, 4);
+    sha_update(&c, l4, 4);
+    sha_update(&c, label, ll);
+    put_le(l8, n, 8);
+    sha_update(&c, l8, 8);
+    sha_update(&c, data, n);
+    sha_final(&c, t->st);
+}
+
+u64 orc_tx_squeeze(orc_tx* t, const char* label) {
+    u32 ll = (u32)strlen(label);
+    for (u32 ctr = 0;; ctr++) {
+        sha_ctx c;
+        uint8_t l4[4], c4[4], h[32];
+        sha_init(&c);
+        sha_update(&c, t->st, 32);
+        sha_update(&c, "sq", 2);
+        put_le(l4, ll, 4);
+        sha_update(&c, l4, 4);
+        sha_update(&c, label, ll);
+        put_le(c4, ctr, 4);
+        sha_update(&c, c4, 4);
+        sha_final(&c, h);
+        u64 v = get_le(h, 8);
+        if (v < ORC_P) {
+            memcpy(t->st, h, 32);
+            return v;
+        }
+    }
+}
+
+/* ctypes-facing transcript handle */
+void* orc_tx_new(u64 seed) {
+    orc_tx* t = (orc_tx*)malloc(sizeof(orc_tx));
+    orc_tx_init(t, seed);
+    return t;
+}
+void orc_tx_free(void* t) { free(t); }
+void orc_tx_state(const void* t, uint8_t out[32]) { memcpy(out, ((const orc_tx*)t)->st, 32); }
+void orc_tx_absorb_h(void* t, const char* label, const void* d, u64 n) { orc_tx_absorb((orc_tx*)t, label, d, n); }
+u64 orc_tx_squeeze_h(void* t, const char* label) { return orc_tx_squeeze((orc_tx*)t, label); }
+
+/* ------------------------------------------------------------------------ */
+/* Multilinear extensions. A vector of length 2^v is indexed by             */
+/* x = sum_b x_b 2^(v-b): the first coordinate z_1 of a point binds the MSB. */
+/* eq(z, x) = prod_b (z_b x_b + (1 - z_b)(1 - x_b)).                          */
+/* ------------------------------------------------------------------------ */
+
+int orc_log2_ceil(u64 n) {
+    int v = 0;
+    while (((u64)1 << v) < n) v++;
+    return v;
+}
+
+/* eq table by doubling: start [1]; step b maps entry j to 2j (times 1 - z_b)
+ * and 2j+1 (times z_b), so z_1 ends up on the most significant bit. */
+void orc_eq_table(const u64* z, int v, u64* out) {
+    out[0] = 1;
+    for (int b = 0; b < v; b++) {
+        u64 len = (u64)1 << b;
+        for (u64 j = len; j-- > 0;) {
+            u64 o = out[j];
+            out[2 * j] = orc_fmul(o, orc_fsub(1, z[b]));
+            out[2 * j + 1] = orc_fmul(o, z[b]);
+        }
+    }
+}
+
+/* MLE of vals (length n, zero-padded to 2^v) at z: sum_x eq(z, x) vals[x]. */
+u64 orc_mle_eval(const u64* vals, u64 n, const u64* z, int v) {
+    u64 sz = (u64)1 << v;
+    u64* e = (u64*)malloc(sz * sizeof(u64));
+    orc_eq_table(z, v, e);
+    u64 acc = 0;
+    for (u64 x = 0; x < n && x < sz; x++) acc = orc_fadd(acc, orc_fmul(e[x], vals[x]));
+    free(e);
+    return acc;
+}
+
+/* Evaluate the polynomial of degree npts-1 through (i, g[i]), i = 0..npts-1, at x. */
+u64 orc_lagrange(const u64* g, int npts, u64 x) {
+    u64 acc = 0;
+    for (int i = 0; i < npts; i++) {
+        u64 num = 1, den = 1;
+        for (int j = 0; j < npts; j++) {
+            if (j == i) continue;
+            num = orc_fmul(num, orc_fsub(x, (u64)j));
+            den = orc_fmul(den, orc_fsub((u64)i, (u64)j));
+        }
+        acc = orc_fadd(acc, orc_fmul(g[i], orc_fmul(num, orc_finv(den))));
+    }
+    return acc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Sites: one matrix product Y = W . X per site.                              */
+/*   W: M x K, int8, or int4 packed two per byte along K (low nibble = even   */
+/*      k, two's complement, ceil(K/2) bytes per row); optional int8 scales  */
+/*      per 64-column group: W_eff[i][k] = S[i][k/64] * w[i][k].             */
+/*   X: stored transposed, xt = N x K int8 (token-major).                    */
+/*   outputs q, r (int32) and y (int8), stored N x M (token-major).          */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const void* w;
+    const int8_t* scales;
+    const int8_t* xt;
+    int32_t w_bits, M, K, N, k_shift, pad;
+} orc_site;
+
+typedef struct {
+    int32_t* q;
+    int32_t* r;
+    int8_t* y;
+} orc_wit;
+
+static int64_t w_eff(const orc_site* s, int i, int k) {
+    int64_t w;
+    if (s->w_bits == 8) {
+        w = ((const int8_t*)s->w)[(u64)i * s->K + k];
+    } else {
+        const uint8_t* row = (const uint8_t*)s->w + (u64)i * ((s->K + 1) / 2);
+        int nib = (k & 1) ? (row[k / 2] >> 4) : (row[k / 2] & 15);
+        w = nib >= 8 ? nib - 16 : nib;
+    }
+    if (s->scales) w *= s->scales[(u64)i * ((s->K + 63) / 64) + k / 64];
+    return w;
+}
+
+static int64_t floordiv_pow2(int64_t a, int k) {
+    int64_t d = (int64_t)1 << k;
+    int64_t q = a / d;
+    if (a % d != 0 && a < 0) q -= 1;
+    return q;
+}
+
+/* Witness of one site ("How fast can FlashProve go", 3.1): Y = W_eff . X in
+ * integers; q = floor((Y + 2^(k-1)) / 2^k) (round half up), r = Y - 2^k q,
+ * y = clamp(q, -128, 127). Returns 0, or -1 if some |Y| needs more than 31
+ * bits (the accepted input domain). */
+int orc_witness(const orc_site* s, int32_t* q, int32_t* r, int8_t* y) {
+    int M = s->M, K = s->K, N = s->N, k = s->k_shift;
+    int64_t* wrow = (int64_t*)malloc(sizeof(int64_t) * (K > 0 ? K : 1));
+    int bad = 0;
+    for (int i = 0; i < M; i++) {
+        for (int kk = 0; kk < K; kk++) wrow[kk] = w_eff(s, i, kk);
+        for (int j = 0; j < N; j++) {
+            const int8_t* xr = s->xt + (u64)j * K;
+            int64_t acc = 0;
+            for (int kk = 0; kk < K; kk++) acc += wrow[kk] * (int64_t)xr[kk];
+            if (acc > 2147483647LL || acc < -2147483648LL) bad = 1;
+            int64_t qq = floordiv_pow2(acc + ((int64_t)1 << (k - 1)), k);
+            int64_t rr = acc - (qq << k);
+            u64 o = (u64)j * M + i;
+            q[o] = (int32_t)qq;
+            r[o] = (int32_t)rr;
+            y[o] = (int8_t)(qq < -128 ? -128 : (qq > 127 ? 127 : qq));
+        }
+    }
+    free(wrow);
+    return bad ? -1 : 0;
+}
+
+/* A_s[k] = sum_i eq(z, i) W_eff[i][k] for k < K, zero up to 2^ceil(log2 K).
+ * z has ceil(log2 M) coordinates. */
+void orc_partial_w(const orc_site* s, const u64* z, int v, u64* out) {
+    u64 Kp = (u64)1 << orc_log2_ceil((u64)s->K);
+    u64* e = (u64*)malloc(sizeof(u64) << v);
+    orc_eq_table(z, v, e);
+    for (u64 k = 0; k < Kp; k++) out[k] = 0;
+    for (int i = 0; i < s->M; i++)
+        for (int k = 0; k < s->K; k++) out[k] = orc_fadd(out[k], orc_fmul(e[i], orc_fint(w_eff(s, i, k))));
+    free(e);
+}
+
+/* B_s[k] = sum_j eq(z, j) X[k][j] = sum_j eq(z, j) xt[j][k]; z has ceil(log2 N) coordinates. */
+void orc_partial_x(const orc_site* s, const u64* z, int v, u64* out) {
+    u64 Kp = (u64)1 << orc_log2_ceil((u64)s->K);
+    u64* e = (u64*)malloc(sizeof(u64) << v);
+    orc_eq_table(z, v, e);
+    for (u64 k = 0; k < Kp; k++) out[k] = 0;
+    for (int j = 0; j < s->N; j++)
+        for (int k = 0; k < s->K; k++)
+            out[k] = orc_fadd(out[k], orc_fmul(e[j], orc_fint(s->xt[(u64)j * s->K + k])));
+    free(e);
+}
+
+/* Generic row contraction used by the library's partial-evaluation entry
+ * point: out[c] = sum_{i<rows} eq(z, i) (S[i][c/64] *) mat[i][c]. */
+void orc_partial_rows(const void* mat, int bits, const int8_t* scales, int rows, int cols,
+                      const u64* z, int v, u64* out) {
+    orc_site s;
+    memset(&s, 0, sizeof s);
+    s.w = mat;
+    s.w_bits = bits;
+    s.scales = scales;
+    s.M = rows;
+    s.K = cols;
+    orc_partial_w(&s, z, v, out);
+}
+
+/* Output claim c = sum_{i,j} eq(zr, i) eq(zc, j) (2^k q[i,j] + r[i,j]): the MLE
+ * of Y = 2^k q + r at (zr, zc), row bits first ("How fast can FlashProve go", 3.1). */
+u64 orc_claim(const int32_t* q, const int32_t* r, int M, int N, int k, const u64* zr, int vr,
+              const u64* zc, int vc) {
+    u64* er = (u64*)malloc(sizeof(u64) << vr);
+    u64* ec = (u64*)malloc(sizeof(u64) << vc);
+    orc_eq_table(zr, vr, er);
+    orc_eq_table(zc, vc, ec);
+    u64 two_k = orc_fint((int64_t)1 << k);
+    u64 acc = 0;
+    for (int i = 0; i < M; i++)
+        for (int j = 0; j < N; j++) {
+            u64 o = (u64)j * M + i;
+            u64 yv = orc_fadd(orc_fmul(two_k, orc_fint(q[o])), orc_fint(r[o]));
+            acc = orc_fadd(acc, orc_fmul(orc_fmul(er[i], ec[j]), yv));
+        }
+    free(er);
+    free(ec);
+    return acc;
+}
+
+/* Direct MLE of W_eff (padded to 2^vr x 2^n) at (zr, rho): sum_{i,k} eq eq W. */
+static u64 mle_w_direct(const orc_site* s, const u64* zr, int vr, const u64* rho, int n) {
+    u64* er = (u64*)malloc(sizeof(u64) << vr);
+    u64* ek = (u64*)malloc(sizeof(u64) << n);
+    orc_eq_table(zr, vr, er);
+    orc_eq_table(rho, n, ek);
+    u64 acc = 0;
+    for (int i = 0; i < s->M; i++)
+        for (int k = 0; k < s->K; k++)
+            acc = orc_fadd(acc, orc_fmul(orc_fmul(er[i], ek[k]), orc_fint(w_eff(s, i, k))));
+    free(er);
+    free(ek);
+    return acc;
+}
+
+/* Direct MLE of X (padded) at (rho, zc), K bits first then N bits. */
+static u64 mle_x_direct(const orc_site* s, const u64* rho, int n, const u64* zc, int vc) {
+    u64* ek = (u64*)malloc(sizeof(u64) << n);
+    u64* ec = (u64*)malloc(sizeof(u64) << vc);
+    orc_eq_table(rho, n, ek);
+    orc_eq_table(zc, vc, ec);
+    u64 acc = 0;
+    for (int k = 0; k < s->K; k++)
+        for (int j = 0; j < s->N; j++)
+            acc = orc_fadd(acc, orc_fmul(orc_fmul(ek[k], ec[j]), orc_fint(s->xt[(u64)j * s->K + k])));
+    free(ek);
+    free(ec);
+    return acc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Proof byte buffer: every prover message is appended (u64 LE field        */
+/* elements, u32 LE multiplicities) and absorbed under its label.            */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    uint8_t* p;
+    u64 cap, len;
+    int overflow;
+} pbuf;
+
+static void pb_put(pbuf* b, const void* d, u64 n) {
+    if (b->len + n > b->cap) {
+        b->overflow = 1;
+    } else if (n) {
+        memcpy(b->p + b->len, d, n);
+    }
+    b->len += n;
+}
+
+/* send field elements: append and absorb */
+static void send_fe(orc_tx* t, pbuf* b, const char* label, const u64* v, u64 n) {
+    uint8_t* tmp = (uint8_t*)malloc(8 * (n ? n : 1));
+    for (u64 i = 0; i < n; i++) put_le(tmp + 8 * i, v[i], 8);
+    pb_put(b, tmp, 8 * n);
+    orc_tx_absorb(t, label, tmp, 8 * n);
+    free(tmp);
+}
+
+/* send a multiplicity table: the raw u32 LE words go into the proof, their
+ * tree digest into the transcript. */
+static void send_mult(orc_tx* t, pbuf* b, const char* label, const u32* m, u64 n) {
+    uint8_t* tmp = (uint8_t*)malloc(4 * n);
+    uint8_t dg[32];
+    for (u64 i = 0; i < n; i++) put_le(tmp + 4 * i, m[i], 4);
+    pb_put(b, tmp, 4 * n);
+    orc_tree_digest(tmp, 4 * n, dg);
+    orc_tx_absorb(t, label, dg, 32);
+    free(tmp);
+}
+
+static u64 site_w_bytes(const orc_site* s) {
+    return (u64)s->M * (s->w_bits == 4 ? (u64)((s->K + 1) / 2) : (u64)s->K);
+}
+
+/* Witness commitment into the transcript: per site, in site order, absorb
+ * "site" with D(W) || D(S) || D(X) || D(q) || D(r) || D(y) (D = tree digest of
+ * the stored bytes; D(S) of an empty string when there are no scales). */
+static void absorb_sites(orc_tx* t, const orc_site* sites, int ns, const orc_wit* wit) {
+    for (int s = 0; s < ns; s++) {
+        const orc_site* st = &sites[s];
+        uint8_t d[192];
+        u64 mn = (u64)st->M * st->N;
+        orc_tree_digest(st->w, site_w_bytes(st), d);
+        orc_tree_digest(st->scales, st->scales ? (u64)st->M * ((st->K + 63) / 64) : 0, d + 32);
+        orc_tree_digest(st->xt, (u64)st->N * st->K, d + 64);
+        orc_tree_digest(wit[s].q, 4 * mn, d + 96);
+        orc_tree_digest(wit[s].r, 4 * mn, d + 128);
+        orc_tree_digest(wit[s].y, mn, d + 160);
+        orc_tx_absorb(t, "site", d, 192);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Matmul sum-check with batched claims.                                     */
+/* vM = max ceil(log2 M_s), vN = max ceil(log2 N_s), n = max ceil(log2 K_s); */
+/* r_row (vM), r_col (vN) squeezed; site s uses their first m_s / nn_s       */
+/* coordinates. c_s sent; if more than one site, rho_s squeezed (else 1).    */
+/* Round t over padded length-2^n vectors A_s, B_s: g(X) at X = 0, 1, 2 of   */
+/* sum_s rho_s sum_b A_s(X, b) B_s(X, b); then r_t and the MSB fold.         */
+/* Finally the per-site A_s(rho), B_s(rho).                                  */
+/* ------------------------------------------------------------------------ */
+
+static int site_dims(const orc_site* sites, int ns, int* vM, int* vN, int* n) {
+    *vM = *vN = *n = 0;
+    for (int s = 0; s < ns; s++) {
+        int a = orc_log2_ceil((u64)sites[s].M), b = orc_log2_ceil((u64)sites[s].N),
+            c = orc_log2_ceil((u64)sites[s].K);
+        if (a > *vM) *vM = a;
+        if (b > *vN) *vN = b;
+        if (c > *n) *n = c;
+    }
+    return 0;
+}
+
+static void mm_prove(orc_tx* t, pbuf* pb, const orc_site* sites, int ns, const orc_wit* wit) {
+    int vM, vN, n;
+    site_dims(sites, ns, &vM, &vN, &n);
+    u64* rr = (u64*)malloc(sizeof(u64) * (vM + 1));
+    u64* rc = (u64*)malloc(sizeof(u64) * (vN + 1));
+    for (int i = 0; i < vM; i++) rr[i] = orc_tx_squeeze(t, "r_row");
+    for (int i = 0; i < vN; i++) rc[i] = orc_tx_squeeze(t, "r_col");
+
+    u64* c = (u64*)malloc(sizeof(u64) * ns);
+    for (int s = 0; s < ns; s++) {
+        int ms = orc_log2_ceil((u64)sites[s].M), nn = orc_log2_ceil((u64)sites[s].N);
+        c[s] = orc_claim(wit[s].q, wit[s].r, sites[s].M, sites[s].N, sites[s].k_shift, rr, ms, rc, nn);
+    }
+    send_fe(t, pb, "claims", c, (u64)ns);
+
+    u64* rho = (u64*)malloc(sizeof(u64) * ns);
+    if (ns == 1)
+        rho[0] = 1;
+    else
+        for (int s = 0; s < ns; s++) rho[s] = orc_tx_squeeze(t, "rho");
+
+    u64 L = (u64)1 << n;
+    u64** A = (u64**)malloc(sizeof(u64*) * ns);
+    u64** B = (u64**)malloc(sizeof(u64*) * ns);
+    for (int s = 0; s < ns; s++) {
+        int ms = orc_log2_ceil((u64)sites[s].M), nn = orc_log2_ceil((u64)sites[s].N);
+        A[s] = (u64*)calloc(L, sizeof(u64));
+        B[s] = (u64*)calloc(L, sizeof(u64));
+        orc_partial_w(&sites[s], rr, ms, A[s]);
+        orc_partial_x(&sites[s], rc, nn, B[s]);
+    }
+
+    for (int t_ = 0; t_ < n; t_++) {
+        u64 h = L >> 1;
+        u64 g[3] = {0, 0, 0};
+        for (int s = 0; s < ns; s++) {
+            u64 g0 = 0, g1 = 0, g2 = 0;
+            for (u64 b = 0; b < h; b++) {
+                u64 a0 = A[s][b], a1 = A[s][h + b], b0 = B[s][b], b1 = B[s][h + b];
+                u64 a2 = orc_fsub(orc_fmul(2, a1), a0), b2 = orc_fsub(orc_fmul(2, b1), b0);
+                g0 = orc_fadd(g0, orc_fmul(a0, b0));
+                g1 = orc_fadd(g1, orc_fmul(a1, b1));
+                g2 = orc_fadd(g2, orc_fmul(a2, b2));
+            }
+            g[0] = orc_fadd(g[0], orc_fmul(rho[s], g0));
+            g[1] = orc_fadd(g[1], orc_fmul(rho[s], g1));
+            g[2] = orc_fadd(g[2], orc_fmul(rho[s], g2));
+        }
+        send_fe(t, pb, "sc_round", g, 3);
+        u64 r = orc_tx_squeeze(t, "sc_chal");
+        for (int s = 0; s < ns; s++)
+            for (u64 b = 0; b < h; b++) {
+                A[s][b] = orc_fadd(A[s][b], orc_fmul(r, orc_fsub(A[s][h + b], A[s][b])));
+                B[s][b] = orc_fadd(B[s][b], orc_fmul(r, orc_fsub(B[s][h + b], B[s][b])));
+            }
+        L = h;
+    }
+    u64* fin = (u64*)malloc(sizeof(u64) * 2 * ns);
+    for (int s = 0; s < ns; s++) {
+        fin[2 * s] = A[s][0];
+        fin[2 * s + 1] = B[s][0];
+    }
+    send_fe(t, pb, "sc_final", fin, 2 * (u64)ns);
+    for (int s = 0; s < ns; s++) {
+        free(A[s]);
+        free(B[s]);
+    }
+    free(A); free(B); free(fin); free(rho); free(c); free(rr); free(rc);
+}
+
+/* ------------------------------------------------------------------------ */
+/* LogUp lookups of the rescale remainders and of the clamp pairs.           */
+/* Table 0 (remainder range): t_j = j - 2^(k-1), j < 2^k; key = r.           */
+/* Table 1 (clamp, also bounds q to 16 bits): t_j = v_j + gamma clamp(v_j),  */
+/*   v_j = j - 2^15, j < 2^16; key = q + gamma y.                            */
+/* Keys: every site's outputs in storage order, sites concatenated, padded  */
+/* to 2^v (v >= 1) with the neutral key 0 (r = 0; q = y = 0).                */
+/* Key side as a binary tree of fractions: leaves (1, alpha - f); parent     */
+/* (pL qR + pR qL, qL qR) of children 2x, 2x+1. The two trees have the same  */
+/* shape and are proven together, layer by layer, in one sum-check whose    */
+/* terms are combined with powers of lambda.                                 */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    u64 nk;       /* real keys */
+    int v;        /* tree depth */
+    int k;        /* rescale shift */
+    int64_t* fr;  /* remainder keys (padded) */
+    int64_t* fq;  /* q component (padded) */
+    int64_t* fy;  /* y component (padded) */
+} orc_keys;
+
+static int keys_build(const orc_site* sites, int ns, const orc_wit* wit, orc_keys* K) {
+    u64 nk = 0;
+    int k = sites[0].k_shift;
+    for (int s = 0; s < ns; s++) {
+        nk += (u64)sites[s].M * sites[s].N;
+        if (sites[s].k_shift != k) return -1;
+    }
+    int v = orc_log2_ceil(nk);
+    if (v < 1) v = 1;
+    u64 L = (u64)1 << v;
+    K->nk = nk;
+    K->v = v;
+    K->k = k;
+    K->fr = (int64_t*)calloc(L, sizeof(int64_t));
+    K->fq = (int64_t*)calloc(L, sizeof(int64_t));
+    K->fy = (int64_t*)calloc(L, sizeof(int64_t));
+    u64 o = 0;
+    for (int s = 0; s < ns; s++) {
+        u64 mn = (u64)sites[s].M * sites[s].N;
+        for (u64 e = 0; e < mn; e++, o++) {
+            K->fr[o] = wit[s].r[e];
+            K->fq[o] = wit[s].q[e];
+            K->fy[o] = wit[s].y[e];
+        }
+    }
+    return 0;
+}
+
+static void keys_free(orc_keys* K) {
+    free(K->fr);
+    free(K->fq);
+    free(K->fy);
+}
+
+/* Multiplicities, counted by the key's table index; a key outside a table's
+ * range is counted nowhere (its lookup then fails at the verifier). */
+static void mult_rem(const orc_keys* K, u32* m) {
+    u64 T = (u64)1 << K->k, L = (u64)1 << K->v;
+    int64_t half = (int64_t)1 << (K->k - 1);
+    memset(m, 0, T * sizeof(u32));
+    for (u64 i = 0; i < L; i++) {
+        int64_t j = K->fr[i] + half;
+        if (j >= 0 && (u64)j < T) m[j]++;
+    }
+}
+
+static void mult_clamp(const orc_keys* K, u32* m) {
+    u64 L = (u64)1 << K->v;
+    memset(m, 0, 65536 * sizeof(u32));
+    for (u64 i = 0; i < L; i++) {
+        int64_t j = K->fq[i] + 32768;
+        if (j >= 0 && j < 65536) m[j]++;
+    }
+}
+
+static u64 key_field(const orc_keys* K, int tab, u64 i, u64 gamma) {
+    if (tab == 0) return orc_fint(K->fr[i]);
+    return orc_fadd(orc_fint(K->fq[i]), orc_fmul(gamma, orc_fint(K->fy[i])));
+}
+
+/* layers[d] has 2^d nodes; P at [0], Q at [1]. */
+typedef struct {
+    u64** P;
+    u64** Q;
+    int v;
+} orc_tree;
+
+static void tree_build(const orc_keys* K, int tab, u64 alpha, u64 gamma, orc_tree* T) {
+    int v = K->v;
+    T->v = v;
+    T->P = (u64**)malloc(sizeof(u64*) * (v + 1));
+    T->Q = (u64**)malloc(sizeof(u64*) * (v + 1));
+    u64 L = (u64)1 << v;
+    T->P[v] = (u64*)malloc(L * sizeof(u64));
+    T->Q[v] = (u64*)malloc(L * sizeof(u64));
+    for (u64 i = 0; i < L; i++) {
+        T->P[v][i] = 1;
+        T->Q[v][i] = orc_fsub(alpha, key_field(K, tab, i, gamma));
+    }
+    for (int d = v - 1; d >= 0; d--) {
+        u64 n = (u64)1 << d;
+        T->P[d] = (u64*)malloc(n * sizeof(u64));
+        T->Q[d] = (u64*)malloc(n * sizeof(u64));
+        for (u64 x = 0; x < n; x++) {
+            u64 pl = T->P[d + 1][2 * x], pr = T->P[d + 1][2 * x + 1];
+            u64 ql = T->Q[d + 1][2 * x], qr = T->Q[d + 1][2 * x + 1];
+            T->P[d][x] = orc_fadd(orc_fmul(pl, qr), orc_fmul(pr, ql));
+            T->Q[d][x] = orc_fmul(ql, qr);
+        }
+    }
+}
+
+static void tree_free(orc_tree* T) {
+    for (int d = 0; d <= T->v; d++) {
+        free(T->P[d]);
+        free(T->Q[d]);
+    }
+    free(T->P);
+    free(T->Q);
+}
+
+/* the summand of one layer: sum over tables tau of
+ * lambda^(2 tau) (pL qR + pR qL + lambda qL qR) */
+static u64 layer_F(const u64 v8[8], u64 lam, u64 lam2) {
+    u64 acc = 0, w = 1;
+    for (int tau = 0; tau < 2; tau++) {
+        const u64* x = v8 + 4 * tau; /* pL, pR, qL, qR */
+        u64 f = orc_fadd(orc_fadd(orc_fmul(x[0], x[3]), orc_fmul(x[1], x[2])),
+                         orc_fmul(lam, orc_fmul(x[2], x[3])));
+        acc = orc_fadd(acc, orc_fmul(w, f));
+        w = lam2;
+    }
+    return acc;
+}
+
+static void lu_prove(orc_tx* t, pbuf* pb, const orc_site* sites, int ns, const orc_wit* wit) {
+    orc_keys K;
+    keys_build(sites, ns, wit, &K);
+    int v = K.v;
+    u64 Trem = (u64)1 << K.k;
+    u32* mr = (u32*)malloc(Trem * sizeof(u32));
+    u32* mc = (u32*)malloc(65536 * sizeof(u32));
+
+    mult_rem(&K, mr);
+    send_mult(t, pb, "logup_m_rem", mr, Trem);
+    u64 gamma = orc_tx_squeeze(t, "logup_gamma");
+    mult_clamp(&K, mc);
+    send_mult(t, pb, "logup_m_clamp", mc, 65536);
+    u64 alpha[2];
+    alpha[0] = orc_tx_squeeze(t, "logup_alpha");
+    alpha[1] = orc_tx_squeeze(t, "logup_alpha");
+
+    orc_tree T[2];
+    tree_build(&K, 0, alpha[0], gamma, &T[0]);
+    tree_build(&K, 1, alpha[1], gamma, &T[1]);
+
+    /* layer 1 (two nodes per tree) is sent in the clear */
+    u64 l1[8];
+    for (int tau = 0; tau < 2; tau++) {
+        l1[4 * tau + 0] = T[tau].P[1][0];
+        l1[4 * tau + 1] = T[tau].P[1][1];
+        l1[4 * tau + 2] = T[tau].Q[1][0];
+        l1[4 * tau + 3] = T[tau].Q[1][1];
+    }
+    send_fe(t, pb, "gkr_l1", l1, 8);
+    u64 mu = orc_tx_squeeze(t, "gkr_mu");
+    u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
+    z[0] = mu;
+
+    for (int d = 1; d < v; d++) {
+        u64 lam = orc_tx_squeeze(t, "gkr_lambda");
+        u64 lam2 = orc_fmul(lam, lam);
+        u64 n = (u64)1 << d;
+        /* vectors: for tau: pL, pR, qL, qR (children of layer d in layer d+1), then eq(z, .) */
+        u64* V[9];
+        for (int i = 0; i < 9; i++) V[i] = (u64*)malloc(n * sizeof(u64));
+        for (int tau = 0; tau < 2; tau++)
+            for (u64 x = 0; x < n; x++) {
+                V[4 * tau + 0][x] = T[tau].P[d + 1][2 * x];
+                V[4 * tau + 1][x] = T[tau].P[d + 1][2 * x + 1];
+                V[4 * tau + 2][x] = T[tau].Q[d + 1][2 * x];
+                V[4 * tau + 3][x] = T[tau].Q[d + 1][2 * x + 1];
+            }
+        orc_eq_table(z, d, V[8]);
+        u64 L = n;
+        u64* rho = (u64*)malloc(sizeof(u64) * d);
+        for (int r = 0; r < d; r++) {
+            u64 h = L >> 1;
+            u64 g[4] = {0, 0, 0, 0};
+            for (u64 b = 0; b < h; b++)
+                for (u64 X = 0; X < 4; X++) {
+                    u64 ev[9];
+                    for (int i = 0; i < 9; i++)
+                        ev[i] = orc_fadd(V[i][b], orc_fmul(X, orc_fsub(V[i][h + b], V[i][b])));
+                    g[X] = orc_fadd(g[X], orc_fmul(ev[8], layer_F(ev, lam, lam2)));
+                }
+            send_fe(t, pb, "gkr_round", g, 4);
+            rho[r] = orc_tx_squeeze(t, "gkr_chal");
+            for (int i = 0; i < 9; i++)
+                for (u64 b = 0; b < h; b++)
+                    V[i][b] = orc_fadd(V[i][b], orc_fmul(rho[r], orc_fsub(V[i][h + b], V[i][b])));
+            L = h;
+        }
+        u64 fin[8];
+        for (int i = 0; i < 8; i++) fin[i] = V[i][0];
+        send_fe(t, pb, "gkr_final", fin, 8);
+        mu = orc_tx_squeeze(t, "gkr_mu");
+        for (int r = 0; r < d; r++) z[r] = rho[r];
+        z[d] = mu;
+        for (int i = 0; i < 9; i++) free(V[i]);
+        free(rho);
+    }
+
+    /* leaf claims: MLEs of the padded r, q, y key columns at z (v coords) */
+    u64 Lk = (u64)1 << v;
+    u64* col = (u64*)malloc(Lk * sizeof(u64));
+    u64 leaf[3];
+    for (u64 i = 0; i < Lk; i++) col[i] = orc_fint(K.fr[i]);
+    leaf[0] = orc_mle_eval(col, Lk, z, v);
+    for (u64 i = 0; i < Lk; i++) col[i] = orc_fint(K.fq[i]);
+    leaf[1] = orc_mle_eval(col, Lk, z, v);
+    for (u64 i = 0; i < Lk; i++) col[i] = orc_fint(K.fy[i]);
+    leaf[2] = orc_mle_eval(col, Lk, z, v);
+    send_fe(t, pb, "leaf", leaf, 3);
+
+    free(col);
+    free(z);
+    tree_free(&T[0]);
+    tree_free(&T[1]);
+    free(mr);
+    free(mc);
+    keys_free(&K);
+}
+
+/*
+ * Full prover. Writes the proof (matmul section, then lookup section) and the
+ * transcript state after each stage (commit, matmul, lookup) into states[96].
+ * sec_off[0] = byte length of the matmul section. Returns 0, -1 on bad input,
+ * -2 if the proof buffer is too small (*len then holds the size needed).
+ */
+int orc_prove(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, uint8_t* proof, u64 cap,
+              u64* len, uint8_t states[96], u64* sec_off) {
+    if (ns < 1) return -1;
+    for (int s = 0; s < ns; s++)
+        if (sites[s].M < 1 || sites[s].N < 1 || sites[s].K < 1 || sites[s].k_shift < 1 ||
+            sites[s].k_shift > 30 || (sites[s].w_bits != 4 && sites[s].w_bits != 8) ||
+            sites[s].k_shift != sites[0].k_shift)
+            return -1;
+    orc_tx t;
+    pbuf pb = {proof, cap, 0, 0};
+    orc_tx_init(&t, seed);
+    absorb_sites(&t, sites, ns, wit);
+    memcpy(states, t.st, 32);
+    mm_prove(&t, &pb, sites, ns, wit);
+    memcpy(states + 32, t.st, 32);
+    *sec_off = pb.len;
+    lu_prove(&t, &pb, sites, ns, wit);
+    memcpy(states + 64, t.st, 32);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Verifier. Replays the transcript from the witness it holds (standing in   */
+/* for the openings of the committed values and weights) and checks every   */
+/* protocol relation. Integer facts of the witness (Y = 2^k q + r, ranges,   */
+/* y = clamp(q)) are NOT checked directly: only the protocol may reject.     */
+/* Returns 0 on accept or a reason code; detail[0..1] locate the failure.    */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_FORMAT = 1,       /* truncated proof, trailing bytes or non-canonical element */
+    REJ_CLAIM = 2,        /* c_s differs from the committed output's MLE */
+    REJ_MM_ROUND = 3,     /* matmul sum-check round: g(0) + g(1) != claim */
+    REJ_MM_FINAL = 4,     /* last matmul claim != sum_s rho_s A_s B_s */
+    REJ_MM_A = 5,         /* A_s(rho) != W_s MLE */
+    REJ_MM_B = 6,         /* B_s(rho) != X_s MLE */
+    REJ_ROOT_REM = 7,     /* remainder lookup: key fraction != table fraction */
+    REJ_ROOT_CLAMP = 8,   /* clamp lookup: key fraction != table fraction */
+    REJ_GKR_ROUND = 9,    /* layer sum-check round inconsistent */
+    REJ_GKR_FINAL = 10,   /* layer end: eq * F != claim */
+    REJ_LEAF_P = 11,      /* leaf numerator MLE != 1 */
+    REJ_LEAF_Q = 12,      /* leaf denominator != alpha - key MLE */
+    REJ_LEAF_OPEN = 13,   /* leaf column claims != committed columns' MLE */
+    REJ_ARGS = 14         /* statement malformed */
+};
+
+typedef struct {
+    const uint8_t* p;
+    u64 len, pos;
+    int bad;
+} prd;
+
+static void rd_fe(orc_tx* t, prd* r, const char* label, u64* out, u64 n) {
+    if (r->bad || r->pos + 8 * n > r->len) {
+        r->bad = 1;
+        for (u64 i = 0; i < n; i++) out[i] = 0;
+        return;
+    }
+    const uint8_t* src = r->p + r->pos;
+    for (u64 i = 0; i < n; i++) {
+        out[i] = get_le(src + 8 * i, 8);
+        if (out[i] >= ORC_P) r->bad = 1;
+    }
+    orc_tx_absorb(t, label, src, 8 * n);
+    r->pos += 8 * n;
+}
+
+static void rd_mult(orc_tx* t, prd* r, const char* label, u32* out, u64 n) {
+    if (r->bad || r->pos + 4 * n > r->len) {
+        r->bad = 1;
+        memset(out, 0, 4 * n);
+        return;
+    }
+    const uint8_t* src = r->p + r->pos;
+    uint8_t dg[32];
+    for (u64 i = 0; i < n; i++) out[i] = (u32)get_le(src + 4 * i, 4);
+    orc_tree_digest(src, 4 * n, dg);
+    orc_tx_absorb(t, label, dg, 32);
+    r->pos += 4 * n;
+}
+
+#define FAIL(code, a, b)         \
+    do {                         \
+        rc = (code);             \
+        detail[0] = (a);         \
+        detail[1] = (b);         \
+        goto done;               \
+    } while (0)
+
+static int mm_verify(orc_tx* t, prd* rd, const orc_site* sites, int ns, const orc_wit* wit,
+                     int64_t* detail) {
+    int rc = 0, vM, vN, n;
+    site_dims(sites, ns, &vM, &vN, &n);
+    u64* rr = (u64*)malloc(sizeof(u64) * (vM + 1));
+    u64* rc_ = (u64*)malloc(sizeof(u64) * (vN + 1));
+    u64* c = (u64*)malloc(sizeof(u64) * ns);
+    u64* rho = (u64*)malloc(sizeof(u64) * ns);
+    u64* pt = (u64*)malloc(sizeof(u64) * (n + 1));
+    u64* fin = (u64*)malloc(sizeof(u64) * 2 * ns);
+    for (int i = 0; i < vM; i++) rr[i] = orc_tx_squeeze(t, "r_row");
+    for (int i = 0; i < vN; i++) rc_[i] = orc_tx_squeeze(t, "r_col");
+    rd_fe(t, rd, "claims", c, (u64)ns);
+    if (rd->bad) FAIL(REJ_FORMAT, 0, 0);
+    for (int s = 0; s < ns; s++) {
+        int ms = orc_log2_ceil((u64)sites[s].M), nn = orc_log2_ceil((u64)sites[s].N);
+        u64 want = orc_claim(wit[s].q, wit[s].r, sites[s].M, sites[s].N, sites[s].k_shift, rr, ms, rc_, nn);
+        if (want != c[s]) FAIL(REJ_CLAIM, s, 0);
+    }
+    if (ns == 1)
+        rho[0] = 1;
+    else
+        for (int s = 0; s < ns; s++) rho[s] = orc_tx_squeeze(t, "rho");
+    u64 claim = 0;
+    for (int s = 0; s < ns; s++) claim = orc_fadd(claim, orc_fmul(rho[s], c[s]));
+    for (int r = 0; r < n; r++) {
+        u64 g[3];
+        rd_fe(t, rd, "sc_round", g, 3);
+        if (rd->bad) FAIL(REJ_FORMAT, 1, r);
+        if (orc_fadd(g[0], g[1]) != claim) FAIL(REJ_MM_ROUND, r, 0);
+        pt[r] = orc_tx_squeeze(t, "sc_chal");
+        claim = orc_lagrange(g, 3, pt[r]);
+    }
+    rd_fe(t, rd, "sc_final", fin, 2 * (u64)ns);
+    if (rd->bad) FAIL(REJ_FORMAT, 2, 0);
+    {
+        u64 acc = 0;
+        for (int s = 0; s < ns; s++) acc = orc_fadd(acc, orc_fmul(rho[s], orc_fmul(fin[2 * s], fin[2 * s + 1])));
+        if (acc != claim) FAIL(REJ_MM_FINAL, 0, 0);
+    }
+    for (int s = 0; s < ns; s++) {
+        int ms = orc_log2_ceil((u64)sites[s].M), nn = orc_log2_ceil((u64)sites[s].N);
+        if (mle_w_direct(&sites[s], rr, ms, pt, n) != fin[2 * s]) FAIL(REJ_MM_A, s, 0);
+        if (mle_x_direct(&sites[s], pt, n, rc_, nn) != fin[2 * s + 1]) FAIL(REJ_MM_B, s, 0);
+    }
+done:
+    free(rr); free(rc_); free(c); free(rho); free(pt); free(fin);
+    return rc;
+}
+
+/* fraction sum over a table: sum_j m_j / (alpha - t_j), kept as (num, den) */
+static void table_fraction(const u32* m, u64 T, int tab, int k, u64 alpha, u64 gamma, u64* num, u64* den) {
+    u64 P = 0, Q = 1;
+    for (u64 j = 0; j < T; j++) {
+        u64 tj;
+        if (tab == 0) {
+            tj = orc_fint((int64_t)j - ((int64_t)1 << (k - 1)));
+        } else {
+            int64_t vj = (int64_t)j - 32768;
+            int64_t cj = vj < -128 ? -128 : (vj > 127 ? 127 : vj);
+            tj = orc_fadd(orc_fint(vj), orc_fmul(gamma, orc_fint(cj)));
+        }
+        u64 d = orc_fsub(alpha, tj);
+        /* P/Q + m/d = (P d + m Q) / (Q d) */
+        P = orc_fadd(orc_fmul(P, d), orc_fmul((u64)m[j], Q));
+        Q = orc_fmul(Q, d);
+    }
+    *num = P;
+    *den = Q;
+}
+
+static int lu_verify(orc_tx* t, prd* rd, const orc_site* sites, int ns, const orc_wit* wit,
+                     int64_t* detail) {
+    int rc = 0;
+    orc_keys K;
+    if (keys_build(sites, ns, wit, &K) != 0) {
+        detail[0] = detail[1] = 0;
+        return REJ_ARGS;
+    }
+    int v = K.v;
+    u64 Trem = (u64)1 << K.k;
+    u32* mr = (u32*)malloc(Trem * sizeof(u32));
+    u32* mc = (u32*)malloc(65536 * sizeof(u32));
+    u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
+    u64* rho = (u64*)malloc(sizeof(u64) * (v + 1));
+    u64* col = NULL;
+
+    rd_mult(t, rd, "logup_m_rem", mr, Trem);
+    u64 gamma = orc_tx_squeeze(t, "logup_gamma");
+    rd_mult(t, rd, "logup_m_clamp", mc, 65536);
+    if (rd->bad) FAIL(REJ_FORMAT, 3, 0);
+    u64 alpha[2];
+    alpha[0] = orc_tx_squeeze(t, "logup_alpha");
+    alpha[1] = orc_tx_squeeze(t, "logup_alpha");
+
+    u64 l1[8];
+    rd_fe(t, rd, "gkr_l1", l1, 8);
+    if (rd->bad) FAIL(REJ_FORMAT, 4, 0);
+    for (int tau = 0; tau < 2; tau++) {
+        const u64* x = l1 + 4 * tau; /* p(0), p(1), q(0), q(1) */
+        u64 P0 = orc_fadd(orc_fmul(x[0], x[3]), orc_fmul(x[1], x[2]));
+        u64 Q0 = orc_fmul(x[2], x[3]);
+        u64 PT, QT;
+        table_fraction(tau == 0 ? mr : mc, tau == 0 ? Trem : 65536, tau, K.k, alpha[tau], gamma, &PT, &QT);
+        if (Q0 == 0 || orc_fmul(P0, QT) != orc_fmul(Q0, PT)) FAIL(tau == 0 ? REJ_ROOT_REM : REJ_ROOT_CLAMP, 0, 0);
+    }
+    u64 mu = orc_tx_squeeze(t, "gkr_mu");
+    u64 cP[2], cQ[2];
+    for (int tau = 0; tau < 2; tau++) {
+        const u64* x = l1 + 4 * tau;
+        cP[tau] = orc_fadd(x[0], orc_fmul(mu, orc_fsub(x[1], x[0])));
+        cQ[tau] = orc_fadd(x[2], orc_fmul(mu, orc_fsub(x[3], x[2])));
+    }
+    z[0] = mu;
+    for (int d = 1; d < v; d++) {
+        u64 lam = orc_tx_squeeze(t, "gkr_lambda");
+        u64 lam2 = orc_fmul(lam, lam), lam3 = orc_fmul(lam2, lam);
+        u64 claim = orc_fadd(orc_fadd(cP[0], orc_fmul(lam, cQ[0])),
+                             orc_fadd(orc_fmul(lam2, cP[1]), orc_fmul(lam3, cQ[1])));
+        for (int r = 0; r < d; r++) {
+            u64 g[4];
+            rd_fe(t, rd, "gkr_round", g, 4);
+            if (rd->bad) FAIL(REJ_FORMAT, 5, d);
+            if (orc_fadd(g[0], g[1]) != claim) FAIL(REJ_GKR_ROUND, d, r);
+            rho[r] = orc_tx_squeeze(t, "gkr_chal");
+            claim = orc_lagrange(g, 4, rho[r]);
+        }
+        u64 fin[8];
+        rd_fe(t, rd, "gkr_final", fin, 8);
+        if (rd->bad) FAIL(REJ_FORMAT, 6, d);
+        /* eq(z, rho) in closed form */
+        u64 e = 1;
+        for (int r = 0; r < d; r++)
+            e = orc_fmul(e, orc_fadd(orc_fmul(z[r], rho[r]),
+                                     orc_fmul(orc_fsub(1, z[r]), orc_fsub(1, rho[r]))));
+        if (orc_fmul(e, layer_F(fin, lam, lam2)) != claim) FAIL(REJ_GKR_FINAL, d, 0);
+        mu = orc_tx_squeeze(t, "gkr_mu");
+        for (int tau = 0; tau < 2; tau++) {
+            const u64* x = fin + 4 * tau;
+            cP[tau] = orc_fadd(x[0], orc_fmul(mu, orc_fsub(x[1], x[0])));
+            cQ[tau] = orc_fadd(x[2], orc_fmul(mu, orc_fsub(x[3], x[2])));
+        }
+        for (int r = 0; r < d; r++) z[r] = rho[r];
+        z[d] = mu;
+    }
+    u64 leaf[3];
+    rd_fe(t, rd, "leaf", leaf, 3);
+    if (rd->bad) FAIL(REJ_FORMAT, 7, 0);
+    if (cP[0] != 1 || cP[1] != 1) FAIL(REJ_LEAF_P, 0, 0);
+    if (cQ[0] != orc_fsub(alpha[0], leaf[0])) FAIL(REJ_LEAF_Q, 0, 0);
+    if (cQ[1] != orc_fsub(alpha[1], orc_fadd(leaf[1], orc_fmul(gamma, leaf[2])))) FAIL(REJ_LEAF_Q, 1, 0);
+    {
+        u64 Lk = (u64)1 << v;
+        col = (u64*)malloc(Lk * sizeof(u64));
+        for (u64 i = 0; i < Lk; i++) col[i] = orc_fint(K.fr[i]);
+        if (orc_mle_eval(col, Lk, z, v) != leaf[0]) FAIL(REJ_LEAF_OPEN, 0, 0);
+        for (u64 i = 0; i < Lk; i++) col[i] = orc_fint(K.fq[i]);
+        if (orc_mle_eval(col, Lk, z, v) != leaf[1]) FAIL(REJ_LEAF_OPEN, 1, 0);
+        for (u64 i = 0; i < Lk; i++) col[i] = orc_fint(K.fy[i]);
+        if (orc_mle_eval(col, Lk, z, v) != leaf[2]) FAIL(REJ_LEAF_OPEN, 2, 0);
+    }
+done:
+    free(col); free(mr); free(mc); free(z); free(rho);
+    keys_free(&K);
+    return rc;
+}
+
+int orc_verify(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, const uint8_t* proof, u64 len,
+               int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (ns < 1) return REJ_ARGS;
+    for (int s = 0; s < ns; s++)
+        if (sites[s].M < 1 || sites[s].N < 1 || sites[s].K < 1 || sites[s].k_shift < 1 ||
+            sites[s].k_shift > 30 || sites[s].k_shift != sites[0].k_shift)
+            return REJ_ARGS;
+    orc_tx t;
+    prd rd = {proof, len, 0, 0};
+    orc_tx_init(&t, seed);
+    absorb_sites(&t, sites, ns, wit);
+    int rc = mm_verify(&t, &rd, sites, ns, wit, detail);
+    if (rc) return rc;
+    rc = lu_verify(&t, &rd, sites, ns, wit, detail);
+    if (rc) return rc;
+    if (rd.pos != rd.len) return REJ_FORMAT;
+    return 0;
+}

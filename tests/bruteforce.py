@@ -1,0 +1,326 @@
+"""Brute-force restatement of the proof, for tiny statements only.
+
+Independent of ``oracle/`` (and of the CUDA library): Python integers for the
+field, ``hashlib`` for SHA-256, numpy only for integer matrix products. Every
+prover message is computed straight from its definition -- each multilinear
+extension is evaluated by summing eq(point, x) f(x) over the whole hypercube,
+and each round polynomial by summing the summand over the unbound variables --
+instead of by folding vectors as the oracle does. The two must produce the same
+bytes; a dropped term, a wrong index, sign or bit order in either shows up.
+
+Cost is exponential on purpose: keep M, K, N and the key count in the tens.
+"""
+
+from __future__ import annotations
+
+import hashlib
+import struct
+
+import numpy as np
+
+P = 0xFFFFFFFF00000001
+
+
+def sha(b: bytes) -> bytes:
+    return hashlib.sha256(b).digest()
+
+
+def tree_digest(data: bytes) -> bytes:
+    n = len(data)
+    lv = [sha(data[i:i + 1024]) for i in range(0, n, 1024)] or [sha(b"")]
+    while len(lv) > 1:
+        lv = [sha(b"".join(lv[i:i + 32])) for i in range(0, len(lv), 32)]
+    return sha(struct.pack("<Q", n) + lv[0])
+
+
+class Tx:
+    def __init__(self, seed: int):
+        self.st = sha(b"FPSC-v1" + struct.pack("<Q", seed))
+
+    def absorb(self, label: str, data: bytes):
+        lb = label.encode()
+        self.st = sha(self.st + struct.pack("<I", len(lb)) + lb + struct.pack("<Q", len(data)) + data)
+
+    def squeeze(self, label: str) -> int:
+        lb = label.encode()
+        ctr = 0
+        while True:
+            h = sha(self.st + b"sq" + struct.pack("<I", len(lb)) + lb + struct.pack("<I", ctr))
+            v = int.from_bytes(h[:8], "little")
+            if v < P:
+                self.st = h
+                return v
+            ctr += 1
+
+
+def log2c(n: int) -> int:
+    v = 0
+    while (1 << v) < n:
+        v += 1
+    return v
+
+
+def eq_point(z, x: int) -> int:
+    """eq(z, x) with z_1 on the most significant bit of x (closed-form product)."""
+    v = len(z)
+    acc = 1
+    for b in range(v):
+        bit = (x >> (v - 1 - b)) & 1
+        acc = acc * (z[b] if bit else (1 - z[b])) % P
+    return acc
+
+
+def mle(vals, z) -> int:
+    """sum over the whole hypercube of eq(z, x) vals[x] (vals zero-padded)."""
+    v = len(z)
+    return sum(eq_point(z, x) * (int(vals[x]) % P) for x in range(min(len(vals), 1 << v))) % P
+
+
+def mle2(mat, zrow, zcol) -> int:
+    """MLE of a 2-D array (row bits first) by the double hypercube sum."""
+    R, Cc = mat.shape
+    acc = 0
+    for i in range(min(R, 1 << len(zrow))):
+        ei = eq_point(zrow, i)
+        for j in range(min(Cc, 1 << len(zcol))):
+            acc += ei * eq_point(zcol, j) * (int(mat[i, j]) % P)
+    return acc % P
+
+
+def weights(site) -> np.ndarray:
+    """W_eff as an int64 M x K array."""
+    if site.w_bits == 8:
+        w = site.w.astype(np.int64)
+    else:
+        b = site.w.astype(np.int64)
+        lo, hi = b & 15, b >> 4
+        full = np.empty((site.M, 2 * b.shape[1]), np.int64)
+        full[:, 0::2], full[:, 1::2] = lo, hi
+        w = np.where(full >= 8, full - 16, full)[:, :site.K]
+    if site.scales is not None:
+        cols = np.arange(site.K) // 64
+        w = w * site.scales.astype(np.int64)[:, cols]
+    return w
+
+
+def fe_bytes(vals) -> bytes:
+    return b"".join(struct.pack("<Q", int(v) % P) for v in vals)
+
+
+def prove(seed: int, sites, wits) -> bytes:
+    """The whole proof (matmul section then lookup section), by definition."""
+    tx = Tx(seed)
+    out = bytearray()
+
+    def send(label, vals):
+        b = fe_bytes(vals)
+        out.extend(b)
+        tx.absorb(label, b)
+
+    for s, (q, r, y) in zip(sites, wits):
+        sc = b"" if s.scales is None else s.scales.tobytes()
+        d = tree_digest(s.w.tobytes()) + tree_digest(sc) + tree_digest(s.xt.tobytes()) + \
+            tree_digest(q.astype("<i4").tobytes()) + tree_digest(r.astype("<i4").tobytes()) + \
+            tree_digest(y.astype(np.int8).tobytes())
+        tx.absorb("site", d)
+
+    # ---- matmul sum-check ----
+    vM = max(log2c(s.M) for s in sites)
+    vN = max(log2c(s.N) for s in sites)
+    n = max(log2c(s.K) for s in sites)
+    rr = [tx.squeeze("r_row") for _ in range(vM)]
+    rc = [tx.squeeze("r_col") for _ in range(vN)]
+    Ws = [weights(s) for s in sites]
+    Xs = [s.xt.astype(np.int64).T for s in sites]          # K x N
+    claims = []
+    for s, (q, r, y) in zip(sites, wits):
+        Yq = (q.astype(np.int64) << s.k_shift) + r.astype(np.int64)   # N x M
+        claims.append(mle2(Yq.T, rr[:log2c(s.M)], rc[:log2c(s.N)]))
+    send("claims", claims)
+    rho = [1] if len(sites) == 1 else [tx.squeeze("rho") for _ in sites]
+
+    def A_at(si, pt):   # W~_s(r_row, pt)
+        return mle2(Ws[si], rr[:log2c(sites[si].M)], pt)
+
+    def B_at(si, pt):   # X~_s(pt, r_col)
+        return mle2(Xs[si], pt, rc[:log2c(sites[si].N)])
+
+    chal = []
+    for t in range(n):
+        g = []
+        for X in range(3):
+            acc = 0
+            rest = n - t - 1
+            for b in range(1 << rest):
+                tail = [(b >> (rest - 1 - i)) & 1 for i in range(rest)]
+                pt = chal + [X] + tail
+                for si in range(len(sites)):
+                    acc += rho[si] * A_at(si, pt) * B_at(si, pt)
+            g.append(acc % P)
+        send("sc_round", g)
+        chal.append(tx.squeeze("sc_chal"))
+    fin = []
+    for si in range(len(sites)):
+        fin += [A_at(si, chal), B_at(si, chal)]
+    send("sc_final", fin)
+
+    # ---- LogUp ----
+    k = sites[0].k_shift
+    fr = np.concatenate([w[1].reshape(-1) for w in wits]).astype(np.int64)
+    fq = np.concatenate([w[0].reshape(-1) for w in wits]).astype(np.int64)
+    fy = np.concatenate([w[2].reshape(-1) for w in wits]).astype(np.int64)
+    v = max(1, log2c(len(fr)))
+    L = 1 << v
+    pad = L - len(fr)
+    fr, fq, fy = (np.concatenate([a, np.zeros(pad, np.int64)]) for a in (fr, fq, fy))
+
+    m_rem = np.zeros(1 << k, np.int64)
+    for x in fr:
+        j = x + (1 << (k - 1))
+        if 0 <= j < (1 << k):
+            m_rem[j] += 1
+    b = m_rem.astype("<u4").tobytes()
+    out.extend(b)
+    tx.absorb("logup_m_rem", tree_digest(b))
+    gamma = tx.squeeze("logup_gamma")
+    m_cl = np.zeros(1 << 16, np.int64)
+    for x in fq:
+        j = x + 32768
+        if 0 <= j < 65536:
+            m_cl[j] += 1
+    b = m_cl.astype("<u4").tobytes()
+    out.extend(b)
+    tx.absorb("logup_m_clamp", tree_digest(b))
+    alpha = [tx.squeeze("logup_alpha"), tx.squeeze("logup_alpha")]
+
+    keys = [[int(x) % P for x in fr], [(int(a) + gamma * int(c)) % P for a, c in zip(fq, fy)]]
+    layers = []  # per table: list over depth d of (P list, Q list)
+    for tau in range(2):
+        Pl = [[1] * L]
+        Ql = [[(alpha[tau] - f) % P for f in keys[tau]]]
+        for _ in range(v):
+            p, q_ = Pl[0], Ql[0]
+            Pl.insert(0, [(p[2 * x] * q_[2 * x + 1] + p[2 * x + 1] * q_[2 * x]) % P for x in range(len(p) // 2)])
+            Ql.insert(0, [q_[2 * x] * q_[2 * x + 1] % P for x in range(len(p) // 2)])
+        layers.append((Pl, Ql))
+
+    l1 = []
+    for tau in range(2):
+        Pl, Ql = layers[tau]
+        l1 += [Pl[1][0], Pl[1][1], Ql[1][0], Ql[1][1]]
+    send("gkr_l1", l1)
+    z = [tx.squeeze("gkr_mu")]
+
+    def kids(tau, d):
+        Pl, Ql = layers[tau]
+        Pc, Qc = Pl[d + 1], Ql[d + 1]
+        return ([Pc[2 * x] for x in range(1 << d)], [Pc[2 * x + 1] for x in range(1 << d)],
+                [Qc[2 * x] for x in range(1 << d)], [Qc[2 * x + 1] for x in range(1 << d)])
+
+    for d in range(1, v):
+        lam = tx.squeeze("gkr_lambda")
+        vecs = kids(0, d) + kids(1, d)
+        rho_l = []
+        for t in range(d):
+            g = []
+            for X in range(4):
+                acc = 0
+                rest = d - t - 1
+                for bb in range(1 << rest):
+                    tail = [(bb >> (rest - 1 - i)) & 1 for i in range(rest)]
+                    pt = rho_l + [X] + tail
+                    e = 1
+                    for zi, pi in zip(z, pt):
+                        e = e * (zi * pi + (1 - zi) * (1 - pi)) % P
+                    ev = [mle(vv, pt) for vv in vecs]
+                    F = 0
+                    for tau in range(2):
+                        pL, pR, qL, qR = ev[4 * tau:4 * tau + 4]
+                        F += pow(lam, 2 * tau, P) * (pL * qR + pR * qL + lam * qL * qR)
+                    acc += e * F
+                g.append(acc % P)
+            send("gkr_round", g)
+            rho_l.append(tx.squeeze("gkr_chal"))
+        send("gkr_final", [mle(vv, rho_l) for vv in vecs])
+        z = rho_l + [tx.squeeze("gkr_mu")]
+
+    send("leaf", [mle(fr, z), mle(fq, z), mle(fy, z)])
+    return bytes(out)
+
+
+def site_digests(sites, wits) -> list:
+    out = []
+    for s, (q, r, y) in zip(sites, wits):
+        sc = b"" if s.scales is None else s.scales.tobytes()
+        out.append(tree_digest(s.w.tobytes()) + tree_digest(sc) + tree_digest(s.xt.tobytes()) +
+                   tree_digest(q.astype("<i4").tobytes()) + tree_digest(r.astype("<i4").tobytes()) +
+                   tree_digest(y.astype(np.int8).tobytes()))
+    return out
+
+
+class _Reader:
+    def __init__(self, proof: bytes, tx: Tx):
+        self.b, self.pos, self.tx = proof, 0, tx
+
+    def fe(self, label: str, n: int):
+        raw = self.b[self.pos:self.pos + 8 * n]
+        assert len(raw) == 8 * n, "proof truncated"
+        self.pos += 8 * n
+        self.tx.absorb(label, raw)
+        return [int.from_bytes(raw[8 * i:8 * i + 8], "little") for i in range(n)]
+
+    def mult(self, label: str, n: int):
+        raw = self.b[self.pos:self.pos + 4 * n]
+        assert len(raw) == 4 * n, "proof truncated"
+        self.pos += 4 * n
+        self.tx.absorb(label, tree_digest(raw))
+        return np.frombuffer(raw, dtype="<u4").astype(np.int64)
+
+
+def walk(seed: int, sites, wits, proof: bytes) -> dict:
+    """Replay the transcript over a proof's bytes (no message is recomputed):
+    returns every challenge and message, and the final transcript state."""
+    tx = Tx(seed)
+    for d in site_digests(sites, wits):
+        tx.absorb("site", d)
+    rd = _Reader(proof, tx)
+    out = {}
+    vM = max(log2c(s.M) for s in sites)
+    vN = max(log2c(s.N) for s in sites)
+    n = max(log2c(s.K) for s in sites)
+    out["r_row"] = [tx.squeeze("r_row") for _ in range(vM)]
+    out["r_col"] = [tx.squeeze("r_col") for _ in range(vN)]
+    out["claims"] = rd.fe("claims", len(sites))
+    out["rho"] = [1] if len(sites) == 1 else [tx.squeeze("rho") for _ in sites]
+    out["mm_rounds"], out["mm_chal"] = [], []
+    for _ in range(n):
+        out["mm_rounds"].append(rd.fe("sc_round", 3))
+        out["mm_chal"].append(tx.squeeze("sc_chal"))
+    out["mm_final"] = rd.fe("sc_final", 2 * len(sites))
+    out["state_mm"] = tx.st
+    k = sites[0].k_shift
+    nk = sum(s.M * s.N for s in sites)
+    v = max(1, log2c(nk))
+    out["v"] = v
+    out["m_rem"] = rd.mult("logup_m_rem", 1 << k)
+    out["gamma"] = tx.squeeze("logup_gamma")
+    out["m_clamp"] = rd.mult("logup_m_clamp", 1 << 16)
+    out["alpha"] = [tx.squeeze("logup_alpha"), tx.squeeze("logup_alpha")]
+    out["l1"] = rd.fe("gkr_l1", 8)
+    z = [tx.squeeze("gkr_mu")]
+    out["layers"] = []
+    for d in range(1, v):
+        lam = tx.squeeze("gkr_lambda")
+        rounds, chal = [], []
+        for _ in range(d):
+            rounds.append(rd.fe("gkr_round", 4))
+            chal.append(tx.squeeze("gkr_chal"))
+        fin = rd.fe("gkr_final", 8)
+        mu = tx.squeeze("gkr_mu")
+        out["layers"].append(dict(lam=lam, rounds=rounds, chal=chal, final=fin, z_in=list(z), mu=mu))
+        z = chal + [mu]
+    out["z_leaf"] = z
+    out["leaf"] = rd.fe("leaf", 3)
+    out["consumed"] = rd.pos
+    out["state"] = tx.st
+    return out
