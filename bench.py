@@ -1,0 +1,345 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 sum-check prover for quantised matrix products.
+
+One step = one whole proof of one synthetic statement: witness + commitment
+(fp_commit_witness), batched matmul sum-check (sumcheck_prove_matmul) and the
+LogUp rescale/clamp proof (logup_prove_rescale), from a fresh transcript.
+Default workload: one projection, W 4096x4096 int4, X 4096x512 int8
+activations ~ round(N(0,32)), rescale by 2^12 (8.6e9 MACs).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). value = proved MACs/s of the whole job with
+inputs resident in HBM; e2e = the same through the public API with the
+activations copied from pinned host memory and the layer output read back
+every step; roofline = the kernel with the largest device time, from a
+profiled pass of identical steps (CUDA events around every launch on its
+stream); cpu_baseline = the CPU oracle timed on this host.
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "proved matmul MACs/s and sum-check Melem/s at 1 B200; HBM GB/s vs peak"
+UNIT = "MAC/s"
+CONFIG = 2
+FLUSH_BYTES = 512 << 20  # > 126 MB L2
+
+# kernel -> source file (traffic counters are valid only for the source they were taken on)
+KSRC = {"witness_gemm": "witness.cu", "digest_leaf": "digest.cu", "digest_node": "digest.cu",
+        "digest_final": "digest.cu", "eq_build": "mle.cu", "partial_acc": "mle.cu", "partial_fin": "mle.cu",
+        "claim": "mle.cu", "sc_round": "sumcheck.cu", "sc_final": "sumcheck.cu", "hist": "logup.cu",
+        "keys_gather": "logup.cu", "tree_leaf": "logup.cu", "tree_up": "logup.cu", "gkr_round": "logup.cu",
+        "gkr_final": "logup.cu", "leaf_eval": "logup.cu", "reduce": "mle.cu"}
+
+
+def src_hash(kernel: str) -> str:
+    f = ROOT / "sum_check_prover_b200" / "csrc" / KSRC.get(kernel, "")
+    h = hashlib.sha256()
+    for p in [f, *sorted((ROOT / "sum_check_prover_b200" / "csrc").glob("*.cuh"))]:
+        if p.is_file():
+            h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def peaks() -> dict:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "src": "fallback"}
+
+
+def sumcheck_elems(wl) -> int:
+    """Initial hypercube sizes of every sum-check instance in one proof."""
+    n = max((s.K - 1).bit_length() for s in wl.sites)
+    mm = len(wl.sites) * (1 << n)
+    nk = wl.n_keys
+    v = max(1, (nk - 1).bit_length())
+    return mm + 2 * ((1 << v) - 2)
+
+
+class Clocks:
+    """nvidia-smi samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def start(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.f.read())) if len(r) >= 9]
+        self.f.close()
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, r[5:9]):
+                if val.strip().lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    """The CPU oracle as it stands, on a bounded sample of the same workload."""
+    world, rank, local = dist()
+    if rank != 0:
+        return
+    import oracle
+    import workloads
+    rows = args.ref_rows
+    wl = workloads.build(CONFIG, seed=args.seed, M=rows)
+    macs = wl.macs
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        R = oracle.resolve(wl)
+        proof, states, _ = oracle.prove(args.seed, R.sites, R.wits)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    per = statistics.mean(times)
+    value = macs / per
+    sample = (f"projection with W {rows}x4096 int4 (rows sampled from the 4096x4096 statement), X 4096x512, "
+              f"k=12: witness + full proof per step, single thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
+            "config": {"workload": "projection W 4096x4096 int4, X 4096x512 int8 N(0,32), k=12", "sample_rows": rows},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist()
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as td
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                              device_id=torch.device(f"cuda:{local}"))
+        pg = td
+
+    import sum_check_prover_b200 as fp
+    import workloads
+    from workloads import device
+
+    dev = torch.device(f"cuda:{local}")
+    # every rank proves its own independent statement (weak scaling, no data-path collective)
+    wl = workloads.build(CONFIG, seed=args.seed + rank)
+    macs = wl.macs
+    elems = sumcheck_elems(wl)
+    ctx = fp.Context(local)
+    stages, keep = device.upload(wl, f"cuda:{local}")
+    device.weight_digests(ctx, stages)  # offline weight commitment: not part of a proof
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(seed):
+        return fp.prove(ctx, seed, stages, stream)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    proof_len = 0
+    for i in range(args.warmup):
+        proof, states, status = step(args.seed + i)
+        proof_len = len(proof)
+        assert status == 0
+    torch.cuda.synchronize()
+
+    # ---- timed pass: value --------------------------------------------------------
+    clocks = Clocks(local)
+    barrier()
+    torch.cuda.synchronize()
+    n0 = ctx.launches()
+    clocks.start()
+    times = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)  # L2 flush between timed steps, outside the event pair
+        e0.record(stream)
+        step(args.seed + 100 + i)
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    clk = clocks.stop()
+    torch.cuda.synchronize()
+    barrier()
+    launches = ctx.launches() - n0
+    total_ms = sum(times)
+    if pg is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * macs * args.steps / (total_ms / 1e3)
+
+    # ---- profiled pass: per-kernel device time and algorithmic bytes -----------------
+    ctx.set_profiling(True)
+    for i in range(args.prof_steps):
+        flush.fill_(i & 0xFF)
+        step(args.seed + 200 + i)
+    torch.cuda.synchronize()
+    stats = ctx.kernel_stats()
+    ctx.set_profiling(False)
+    kern = {k: {"launches": v[0] / args.prof_steps, "ms": v[1] / args.prof_steps,
+                "GBps": (v[2] / (v[1] * 1e-3) / 1e9) if v[1] > 0 else None} for k, v in stats.items()}
+    dom = max(stats.items(), key=lambda kv: kv[1][1])
+    pk = peaks()
+    dname, (dl, dms, dbytes) = dom
+    avg_ms = dms / dl
+    traffic = None
+    tf = ROOT / "profiles" / "traffic.json"
+    if tf.exists():
+        t = json.loads(tf.read_text()).get(dname)
+        if t and t.get("src") == src_hash(dname) and t.get("workload") == "projection":
+            traffic = t.get("bytes_per_launch")
+    if dname == "witness_gemm":
+        flops = 2.0 * macs / (dl / args.prof_steps)
+        peak = pk["bf16_tflops"] * 2.0
+        achieved = flops / (avg_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": traffic, "kernel": dname,
+                "peak_note": f"int8 = {pk['src']} bf16 x 2 (nominal int8/bf16 ratio)"}
+    else:
+        achieved = (dbytes / dl) / (avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "kernel": dname,
+                "avg_launch_us": avg_ms * 1e3, "bytes_per_launch": dbytes / dl,
+                "peak_note": f"{pk['src']} copy bandwidth"}
+
+    # ---- e2e pass: activations from pinned host memory, layer output read back ----------
+    flat = [d for st in stages for d in st]
+    host_x = [(d, d.xt.cpu().pin_memory()) for d in flat]
+    host_y = [(d, torch.empty(d.y.shape, dtype=torch.int8).pin_memory()) for d in flat]
+    h2d = sum(x.numel() for _, x in host_x)
+    d2h = sum(y.numel() for _, y in host_y) + proof_len
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e0.record(stream)
+        for d, x in host_x:
+            d.xt.copy_(x, non_blocking=True)
+        step(args.seed + 300 + i)
+        for d, y in host_y:
+            y.copy_(d.y, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = sum(e2e_ms)
+    if pg is not None:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_value = world * macs * args.steps / (e2e_total / 1e3)
+
+    # ---- CPU baseline: the oracle on this host (rank 0, one GPU only) ------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        t0 = time.perf_counter()
+        R = oracle.resolve(wl)
+        oracle.prove(args.seed, R.sites, R.wits)
+        dt = time.perf_counter() - t0
+        cpu = {"value": macs / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": "the whole statement once (witness + proof), single-threaded C", "seconds": dt}
+
+    ctx.close()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "u64", "data": "synthetic",
+                "config": {"workload": "projection W 4096x4096 int4, X 4096x512 int8 N(0,32), k=12",
+                           "M": 4096, "K": 4096, "N": 512, "macs_per_step": macs,
+                           "l2": "flushed between timed steps (512 MiB write)",
+                           "parallelism": f"{world} independent statements, one per GPU"},
+                "sumcheck_melem_s": world * elems * args.steps / (total_ms / 1e3) / 1e6,
+                "sumcheck_elems_per_step": elems,
+                "roofline": roof,
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches,
+                "clocks": clk,
+                "kernels": kern,
+                "proof_bytes": proof_len}
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--prof-steps", type=int, default=3)
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 1:
+        args.warmup = 1
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

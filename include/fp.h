@@ -1,0 +1,209 @@
+/*
+ * fp.h -- C ABI of libfp: a sum-check prover for the fixed-point quantised
+ * matrix products of a transformer layer, over the Goldilocks field
+ * p = 2^64 - 2^32 + 1, with the rescale and clamp of every product proven by
+ * LogUp lookups. Hand-written CUDA for sm_100a (NVIDIA B200).
+ *
+ * What is proven (page "How fast can FlashProve go"):
+ *  - 2 Background: the prover commits every intermediate value; sum-check
+ *    reduces each polynomial operation (here Y = W.X) to claims on committed
+ *    values and weights; non-polynomial steps (rescale, clamp) are proven by
+ *    lookups; Fiat-Shamir makes every challenge a hash of all messages so far.
+ *  - 3.1 Committing intermediate values: a rescale q = round(Y / 2^k) commits
+ *    the remainder r = Y - 2^k q; the matmul sum-check uses 2^k q + r in place
+ *    of Y and a lookup shows that r is small. Field: Goldilocks.
+ *  - 2 / 2.1 Batching: many claims are merged into one (random linear
+ *    combination of the per-matmul claims).
+ *  - 4 Tighter Rooflines: a lookup's key side is a binary tree, every level
+ *    proven by sum-check. Page "Towards Proving Frontier-Scale LLM Inference",
+ *    The proof system: lookups by logarithmic derivatives (LogUp), whose
+ *    fractions fill that tree.
+ * The exact byte-level protocol (transcript encoding, tree digest, message
+ * order, bit order, rounding tie) is specified in the repository's design
+ * notes and implemented independently by the CPU oracle.
+ *
+ * Conventions for every entry point:
+ *  - Pointers documented "device" are CUDA device pointers on the context's
+ *    device (e.g. torch tensors' data_ptr()); "host" pointers are ordinary
+ *    host memory. The caller owns every buffer it passes; the library never
+ *    frees or retains them past the call.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Kernels run on it; every call returns only after its results
+ *    (transcript updates, proof bytes) are on the host.
+ *  - Scratch memory comes from a per-context device arena that grows on
+ *    demand (cudaMalloc) and is released by fp_ctx_destroy.
+ *  - Return value: FP_OK (0), a positive warning, or a negative FP_ERR_*
+ *    code; fp_last_error(ctx) describes the last failure. No exception or
+ *    signal crosses the ABI. After FP_ERR_CUDA the context should be
+ *    destroyed.
+ *  - A context or transcript must not be used from two threads at once.
+ */
+#ifndef FP_H_
+#define FP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP_OK 0
+#define FP_WARN_KEYS_OUTSIDE_TABLE 1 /* proof written; some key lies outside its table (the verifier will reject) */
+#define FP_ERR_ARG -1                /* null pointer, bad enum value, buffer too small */
+#define FP_ERR_SHAPE -2              /* dimensions out of the accepted domain */
+#define FP_ERR_CUDA -3               /* a CUDA call failed */
+#define FP_ERR_TIMEOUT -4            /* a bounded wait on the device ran out */
+#define FP_ERR_OOM -5                /* device or pinned-host allocation failed */
+
+typedef struct fp_ctx fp_ctx;
+typedef struct fp_tx fp_tx;
+
+/*
+ * One matrix product Y = W . X ("site").
+ *  w       device. W, M x K row-major. w_bits = 8: int8, K bytes per row.
+ *          w_bits = 4: two's-complement nibbles packed two per byte along K,
+ *          low nibble = even k, ceil(K/2) bytes per row (an odd K leaves the
+ *          last high nibble zero).
+ *  scales  device, nullable. int8 group scales, M x ceil(K/64) row-major:
+ *          W_eff[i][k] = scales[i][k/64] * W[i][k].
+ *  xt      device. X stored token-major: X^T as N x K row-major int8.
+ *  q, r, y device, N x M row-major (token-major): q, r int32, y int8.
+ *          Outputs of fp_commit_witness, inputs of the two provers.
+ *  k_shift rescale exponent k, 1 <= k <= 20 (same for all sites of a call to
+ *          logup_prove_rescale).
+ *  w_digest host, nullable: 64 bytes D(W) || D(scales) computed once offline
+ *          with fp_digest (weights committed in advance, page "FlashProve: How
+ *          AI Answers Become Provable...", What FlashProve actually proves:
+ *          offline commitment). NULL makes fp_commit_witness hash W itself
+ *          (operands that are activations, e.g. attention's Q or V).
+ * Accepted domain: 1 <= M, N <= 2^24, 1 <= K <= 2^20, and the worst-case
+ * |Y| = max|W_eff| * 128 * K must stay below 2^31 (int32 accumulation exact),
+ * e.g. K < 16384 for int4 with scales. Violations return FP_ERR_SHAPE.
+ */
+typedef struct {
+    const void* w;
+    const int8_t* scales;
+    const int8_t* xt;
+    int32_t* q;
+    int32_t* r;
+    int8_t* y;
+    int32_t w_bits;
+    int32_t M, K, N;
+    int32_t k_shift;
+    const uint8_t* w_digest;
+} fp_site;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int fp_version(void);
+
+/* Create a context on CUDA device `device`; NULL on failure. */
+fp_ctx* fp_ctx_create(int device);
+void fp_ctx_destroy(fp_ctx* ctx);
+/* Message of the last failure on this context (static storage, valid until the next call). */
+const char* fp_last_error(const fp_ctx* ctx);
+
+/*
+ * Host Fiat-Shamir transcript ("How fast can FlashProve go", 2 Background:
+ * each challenge is a hash of everything the prover has sent; SHA-256 here).
+ *   state0 = SHA256("FPSC-v1" || u64le(seed))
+ *   absorb:  state = SHA256(state || u32le(|label|) || label || u64le(n) || data)
+ *   squeeze: h = SHA256(state || "sq" || u32le(|label|) || label || u32le(ctr)),
+ *            ctr = 0, 1, ...; the first h whose low 8 bytes (little-endian)
+ *            are < p becomes the state, that value the challenge.
+ * fp_tx_squeeze draws n challenges in order into out[0..n).
+ */
+fp_tx* fp_tx_create(uint64_t seed);
+void fp_tx_destroy(fp_tx* tx);
+int fp_tx_absorb(fp_tx* tx, const char* label, const void* data, size_t n);
+int fp_tx_squeeze(fp_tx* tx, const char* label, uint64_t* out, size_t n);
+int fp_tx_state(const fp_tx* tx, uint8_t out[32]);
+
+/*
+ * Tree digest of a device byte buffer: SHA-256 of every 1 KiB chunk, then of
+ * every run of up to 32 consecutive digests until one is left, finally
+ * SHA256(u64le(nbytes) || top). out: host, 32 bytes. dev may be NULL when
+ * nbytes == 0.
+ */
+int fp_digest(fp_ctx* ctx, const void* dev, size_t nbytes, uint8_t out[32], void* stream);
+
+/*
+ * Witness and commitment of `nsites` products ("How fast can FlashProve go",
+ * 3.1). For every site: Y = W_eff . X (exact int32 accumulation),
+ * q = floor((Y + 2^(k-1)) / 2^k) (round half up), r = Y - 2^k q,
+ * y = clamp(q, -128, 127), written to the site's q, r, y. Then, in site order,
+ * absorbs "site" with D(W) || D(scales) || D(xt) || D(q) || D(r) || D(y) into tx.
+ * Sites whose operands are other sites' outputs are committed by a later call,
+ * after the call that produced them.
+ */
+int fp_commit_witness(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites, void* stream);
+
+/*
+ * Multilinear partial evaluation: contracts the rows of a rows x cols matrix
+ * with eq(point, .) ("How fast can FlashProve go", 2 Background and 4: the
+ * matmul sum-check's weight decode), out[c] = sum_i eq(point, i) * M_eff[i][c]
+ * for c < cols, 0 for cols <= c < 2^ceil(log2 cols).
+ *  mat     device; bits = 4 (packed as fp_site.w) or 8 (int8), row-major.
+ *  scales  device, nullable: per-64-column int8 scales, rows x ceil(cols/64).
+ *  point   host, npoint = ceil(log2 rows) canonical field elements; its first
+ *          coordinate binds the most significant row-index bit.
+ *  out     device, 2^ceil(log2 cols) canonical u64.
+ * W~(r_i, .) is mle_partial_eval(W); X~(., r_j) is mle_partial_eval(xt).
+ */
+int mle_partial_eval(fp_ctx* ctx, const void* mat, int bits, const int8_t* scales, int rows, int cols,
+                     const uint64_t* point, int npoint, uint64_t* out, void* stream);
+
+/*
+ * Matmul sum-check over all sites with claims batched by a random linear
+ * combination ("How fast can FlashProve go", 2 and 2.1). Squeezes r_row, r_col;
+ * sends the claims c_s = MLE of 2^k q + r at (r_row, r_col); squeezes rho_s
+ * (more than one site); runs n = max ceil(log2 K) degree-2 rounds, each
+ * sending g(0), g(1), g(2) and folding by the squeezed challenge; sends
+ * A_s(rho), B_s(rho). Proof bytes (u64 little-endian field elements):
+ *   nsites claims | n x 3 round values | 2 x nsites final values.
+ * proof: host buffer; *proof_len: capacity in, bytes written out. Too small:
+ * FP_ERR_ARG with the size needed in *proof_len and tx untouched.
+ */
+int sumcheck_prove_matmul(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites, uint8_t* proof,
+                          size_t* proof_len, void* stream);
+
+/*
+ * LogUp proof of every site's rescale remainder and clamp ("How fast can
+ * FlashProve go", 3.1 and 4; "Towards Proving Frontier-Scale LLM Inference",
+ * The proof system). Keys: all outputs in storage order, sites concatenated,
+ * padded to 2^v (v >= 1) with 0. Remainder table t_j = j - 2^(k-1) (2^k rows);
+ * clamp table t_j = v_j + gamma clamp(v_j), v_j = j - 2^15 (2^16 rows).
+ * Proof bytes: m_rem (2^k u32) | m_clamp (2^16 u32) | layer-one values (8 u64)
+ * | for d = 1..v-1: d x 4 round values, 8 final values | 3 leaf values.
+ * Returns FP_WARN_KEYS_OUTSIDE_TABLE (proof still written) when some r or q
+ * falls outside its table. proof / proof_len as for sumcheck_prove_matmul.
+ */
+int logup_prove_rescale(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites, uint8_t* proof,
+                        size_t* proof_len, void* stream);
+
+/* Proof section sizes in bytes for a statement (no GPU work). */
+int fp_proof_size(const fp_site* sites, int nsites, size_t* matmul_bytes, size_t* logup_bytes);
+
+/*
+ * Per-kernel timing: while profiling is on (fp_ctx_set_profiling(ctx, 1), which
+ * also clears the counters), every launch of the library on this context is
+ * bracketed by CUDA events on its stream. fp_kernel_stats fills up to `cap`
+ * records {kernel id, launches, total device ms, algorithmic bytes moved} and
+ * returns the number of kernels seen; names come from fp_kernel_name(id).
+ */
+typedef struct {
+    int32_t kernel;
+    int32_t launches;
+    double ms;
+    double bytes;
+} fp_kernel_stat;
+int fp_ctx_set_profiling(fp_ctx* ctx, int on);
+/* Number of kernels the library has launched on this context since its creation. */
+int64_t fp_ctx_launches(const fp_ctx* ctx);
+int fp_kernel_stats(fp_ctx* ctx, fp_kernel_stat* out, int cap);
+const char* fp_kernel_name(int kernel);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP_H_ */

@@ -1,0 +1,270 @@
+"""Python binding of libfp, the B200 sum-check prover for quantised matrix products.
+
+Argument marshalling only: every step of the proof runs in the CUDA library
+(``libfp.so``, built in-tree by ``sum_check_prover_b200.build``). PyTorch is
+used by callers for device memory and streams; this module only passes
+``data_ptr()`` values and host buffers through the C ABI declared in
+``include/fp.h``. It fails loudly when the library is missing: there is no
+CPU fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+from pathlib import Path
+from typing import Optional, Sequence
+
+__all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P"]
+
+P = 0xFFFFFFFF00000001
+LIB_PATH = Path(__file__).resolve().with_name("libfp.so")
+
+FP_OK = 0
+FP_WARN_KEYS_OUTSIDE_TABLE = 1
+
+
+class FpError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libfp error {code}: {msg}")
+        self.code = code
+
+
+class _Site(C.Structure):
+    _fields_ = [("w", C.c_void_p), ("scales", C.c_void_p), ("xt", C.c_void_p),
+                ("q", C.c_void_p), ("r", C.c_void_p), ("y", C.c_void_p),
+                ("w_bits", C.c_int32), ("M", C.c_int32), ("K", C.c_int32), ("N", C.c_int32),
+                ("k_shift", C.c_int32), ("w_digest", C.c_void_p)]
+
+
+class _KStat(C.Structure):
+    _fields_ = [("kernel", C.c_int32), ("launches", C.c_int32), ("ms", C.c_double), ("bytes", C.c_double)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libfp.so (raises ImportError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise ImportError(f"{LIB_PATH} is missing: build it with sum_check_prover_b200.build.build() (nvcc, sm_100a)")
+    L = C.CDLL(str(LIB_PATH))
+    vp, i32, u64, sz = C.c_void_p, C.c_int, C.c_uint64, C.c_size_t
+    L.fp_version.restype = i32
+    L.fp_ctx_create.restype = vp
+    L.fp_ctx_create.argtypes = [i32]
+    L.fp_ctx_destroy.argtypes = [vp]
+    L.fp_last_error.restype = C.c_char_p
+    L.fp_last_error.argtypes = [vp]
+    L.fp_tx_create.restype = vp
+    L.fp_tx_create.argtypes = [u64]
+    L.fp_tx_destroy.argtypes = [vp]
+    L.fp_tx_absorb.argtypes = [vp, C.c_char_p, vp, sz]
+    L.fp_tx_squeeze.argtypes = [vp, C.c_char_p, C.POINTER(u64), sz]
+    L.fp_tx_state.argtypes = [vp, vp]
+    L.fp_digest.argtypes = [vp, vp, sz, vp, vp]
+    L.fp_commit_witness.argtypes = [vp, vp, C.POINTER(_Site), i32, vp]
+    L.mle_partial_eval.argtypes = [vp, vp, i32, vp, i32, i32, C.POINTER(u64), i32, vp, vp]
+    L.sumcheck_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
+    L.logup_prove_rescale.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
+    L.fp_proof_size.argtypes = [C.POINTER(_Site), i32, C.POINTER(sz), C.POINTER(sz)]
+    L.fp_ctx_set_profiling.argtypes = [vp, i32]
+    L.fp_ctx_launches.restype = C.c_int64
+    L.fp_ctx_launches.argtypes = [vp]
+    L.fp_kernel_stats.argtypes = [vp, C.POINTER(_KStat), i32]
+    L.fp_kernel_name.restype = C.c_char_p
+    L.fp_kernel_name.argtypes = [i32]
+    _lib = L
+    return L
+
+
+def kernel_names() -> list:
+    L = lib()
+    out, k = [], 0
+    while True:
+        nm = L.fp_kernel_name(k).decode()
+        if nm == "?":
+            return out
+        out.append(nm)
+        k += 1
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return int(t.data_ptr()) if hasattr(t, "data_ptr") else int(t)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        try:
+            import torch
+            return int(torch.cuda.current_stream().cuda_stream)
+        except Exception:
+            return None
+    return int(getattr(stream, "cuda_stream", stream))
+
+
+class SiteDesc:
+    """One product Y = W . X: device tensors (anything with data_ptr()) and sizes.
+
+    w: M x K int8, or M x ceil(K/2) packed int4 bytes; scales: M x ceil(K/64) int8 or None;
+    xt: N x K int8 (token-major X); q, r: N x M int32; y: N x M int8.
+    w_digest: 64 bytes from Context.digest(w) + Context.digest(scales), or None.
+    """
+
+    def __init__(self, w, xt, q, r, y, M, K, N, w_bits, k_shift, scales=None, w_digest: Optional[bytes] = None):
+        self.w, self.xt, self.q, self.r, self.y, self.scales = w, xt, q, r, y, scales
+        self.M, self.K, self.N, self.w_bits, self.k_shift = int(M), int(K), int(N), int(w_bits), int(k_shift)
+        self.w_digest = w_digest
+
+
+def _sites(sites: Sequence[SiteDesc]):
+    n = len(sites)
+    arr = (_Site * n)()
+    keep = []
+    for i, s in enumerate(sites):
+        dg = None
+        if s.w_digest is not None:
+            b = C.create_string_buffer(bytes(s.w_digest), 64)
+            keep.append(b)
+            dg = C.addressof(b)
+        arr[i] = _Site(_ptr(s.w), _ptr(s.scales), _ptr(s.xt), _ptr(s.q), _ptr(s.r), _ptr(s.y),
+                       s.w_bits, s.M, s.K, s.N, s.k_shift, dg)
+    return arr, keep
+
+
+class Transcript:
+    """Host Fiat-Shamir transcript (SHA-256), owned by the library."""
+
+    def __init__(self, seed: int):
+        self._L = lib()
+        self.h = self._L.fp_tx_create(seed)
+
+    def absorb(self, label: str, data: bytes):
+        buf = C.create_string_buffer(bytes(data), max(1, len(data)))
+        self._L.fp_tx_absorb(self.h, label.encode(), buf, len(data))
+
+    def squeeze(self, label: str, n: int = 1) -> list:
+        out = (C.c_uint64 * max(1, n))()
+        self._L.fp_tx_squeeze(self.h, label.encode(), out, n)
+        return list(out[:n])
+
+    def state(self) -> bytes:
+        out = C.create_string_buffer(32)
+        self._L.fp_tx_state(self.h, out)
+        return out.raw
+
+    def close(self):
+        if self.h:
+            self._L.fp_tx_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class Context:
+    """A prover context on one CUDA device (scratch arenas, timing)."""
+
+    def __init__(self, device: int = 0):
+        self._L = lib()
+        self.h = self._L.fp_ctx_create(device)
+        if not self.h:
+            raise FpError(-3, f"fp_ctx_create({device}) failed (no usable CUDA device?)")
+
+    def _check(self, rc: int, what: str) -> int:
+        if rc < 0:
+            raise FpError(rc, f"{what}: {self._L.fp_last_error(self.h).decode()}")
+        return rc
+
+    def close(self):
+        if self.h:
+            self._L.fp_ctx_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def digest(self, dev, nbytes: int, stream=None) -> bytes:
+        out = C.create_string_buffer(32)
+        self._check(self._L.fp_digest(self.h, _ptr(dev), nbytes, out, _stream(stream)), "fp_digest")
+        return out.raw
+
+    def commit_witness(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
+        arr, keep = _sites(sites)
+        self._check(self._L.fp_commit_witness(self.h, tx.h, arr, len(sites), _stream(stream)), "fp_commit_witness")
+
+    def partial_eval(self, mat, bits: int, scales, rows: int, cols: int, point: Sequence[int], out, stream=None):
+        pt = (C.c_uint64 * max(1, len(point)))(*[int(p) for p in point])
+        self._check(self._L.mle_partial_eval(self.h, _ptr(mat), bits, _ptr(scales), rows, cols, pt, len(point),
+                                             _ptr(out), _stream(stream)), "mle_partial_eval")
+
+    def proof_size(self, sites: Sequence[SiteDesc]):
+        arr, keep = _sites(sites)
+        a, b = C.c_size_t(0), C.c_size_t(0)
+        self._check(self._L.fp_proof_size(arr, len(sites), C.byref(a), C.byref(b)), "fp_proof_size")
+        return a.value, b.value
+
+    def prove_matmul(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None) -> bytes:
+        arr, keep = _sites(sites)
+        mm, _ = self.proof_size(sites)
+        buf = C.create_string_buffer(max(1, mm))
+        n = C.c_size_t(mm)
+        self._check(self._L.sumcheck_prove_matmul(self.h, tx.h, arr, len(sites), buf, C.byref(n), _stream(stream)),
+                    "sumcheck_prove_matmul")
+        return buf.raw[: n.value]
+
+    def prove_logup(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
+        """Returns (proof bytes, status): status 1 means some key lies outside its table."""
+        arr, keep = _sites(sites)
+        _, lu = self.proof_size(sites)
+        buf = C.create_string_buffer(max(1, lu))
+        n = C.c_size_t(lu)
+        rc = self._check(self._L.logup_prove_rescale(self.h, tx.h, arr, len(sites), buf, C.byref(n),
+                                                     _stream(stream)), "logup_prove_rescale")
+        return buf.raw[: n.value], rc
+
+    def set_profiling(self, on: bool):
+        self._check(self._L.fp_ctx_set_profiling(self.h, 1 if on else 0), "fp_ctx_set_profiling")
+
+    def launches(self) -> int:
+        """Kernels launched by the library on this context so far."""
+        return int(self._L.fp_ctx_launches(self.h))
+
+    def kernel_stats(self) -> dict:
+        """{kernel name: (launches, total ms, algorithmic bytes)} since the last reset."""
+        cap = 64
+        arr = (_KStat * cap)()
+        n = self._check(self._L.fp_kernel_stats(self.h, arr, cap), "fp_kernel_stats")
+        out = {}
+        for i in range(min(n, cap)):
+            out[self._L.fp_kernel_name(arr[i].kernel).decode()] = (arr[i].launches, arr[i].ms, arr[i].bytes)
+        return out
+
+
+def prove(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], stream=None):
+    """Prove a layer: commit every stage's witness in order (a later stage may read
+    an earlier stage's outputs), then the batched matmul sum-check over all sites,
+    then the LogUp rescale/clamp proof. Returns (proof bytes, transcript states after
+    commit / matmul / lookup, lookup status)."""
+    tx = Transcript(seed)
+    try:
+        for st in stages:
+            ctx.commit_witness(tx, st, stream)
+        sites = [s for st in stages for s in st]
+        s0 = tx.state()
+        mm = ctx.prove_matmul(tx, sites, stream)
+        s1 = tx.state()
+        lu, status = ctx.prove_logup(tx, sites, stream)
+        return mm + lu, [s0, s1, tx.state()], status
+    finally:
+        tx.close()

@@ -1,0 +1,363 @@
+// Context, errors, scratch arena, timing hooks, statement checks and the small
+// entry points (digest, witness commitment, partial evaluation).
+#include <stdio.h>
+#include <string.h>
+
+#include "fp_internal.h"
+
+int fp_version(void) { return 100; }
+
+int fp_fail(fp_ctx* c, int code, const std::string& msg) {
+    if (c) c->err = msg;
+    return code;
+}
+
+int fp_cuda_check(fp_ctx* c, cudaError_t e, const char* what) {
+    return fp_fail(c, FP_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+int fp_log2_ceil(uint64_t n) {
+    int v = 0;
+    while ((1ull << v) < n) v++;
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// context
+// ---------------------------------------------------------------------------
+
+fp_ctx* fp_ctx_create(int device) {
+    fp_ctx* c = new fp_ctx();
+    c->device = device;
+    if (cudaSetDevice(device) != cudaSuccess) {
+        delete c;
+        return nullptr;
+    }
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) {
+        delete c;
+        return nullptr;
+    }
+    c->num_sms = prop.multiProcessorCount;
+    c->host.pinned_host = true;
+    c->dig_host.pinned_host = true;
+    if (cudaMalloc(&c->tickets, 4096) != cudaSuccess || cudaMemset(c->tickets, 0, 4096) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
+        delete c;
+        return nullptr;
+    }
+    return c;
+}
+
+void fp_ctx_destroy(fp_ctx* c) {
+    if (!c) return;
+    cudaSetDevice(c->device);
+    cudaDeviceSynchronize();
+    for (auto& p : c->ev_live) {
+        cudaEventDestroy(p.a);
+        cudaEventDestroy(p.b);
+    }
+    for (auto e : c->ev_free) cudaEventDestroy(e);
+    if (c->dev.p) cudaFree(c->dev.p);
+    if (c->dig.p) cudaFree(c->dig.p);
+    if (c->host.p) cudaFreeHost(c->host.p);
+    if (c->dig_host.p) cudaFreeHost(c->dig_host.p);
+    if (c->tickets) cudaFree(c->tickets);
+    delete c;
+}
+
+const char* fp_last_error(const fp_ctx* c) { return c ? c->err.c_str() : "null context"; }
+
+int fp_reserve(fp_ctx* c, FpArena& a, size_t bytes) {
+    bytes = fp_align_up(bytes, 1 << 20);
+    if (bytes <= a.cap) return FP_OK;
+    FP_CUDA(c, cudaDeviceSynchronize());
+    if (a.p) {
+        if (a.pinned_host)
+            cudaFreeHost(a.p);
+        else
+            cudaFree(a.p);
+    }
+    a.p = nullptr;
+    a.cap = 0;
+    a.top = 0;
+    cudaError_t e = a.pinned_host ? cudaMallocHost((void**)&a.p, bytes) : cudaMalloc((void**)&a.p, bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        a.p = nullptr;
+        return fp_fail(c, FP_ERR_OOM, std::string(a.pinned_host ? "pinned host" : "device") +
+                                          " scratch allocation of " + std::to_string(bytes) + " bytes failed");
+    }
+    a.cap = bytes;
+    return FP_OK;
+}
+
+void* fp_alloc(FpArena& a, size_t bytes) {
+    size_t off = fp_align_up(a.top, 256);
+    if (off + bytes > a.cap) return nullptr;
+    a.top = off + bytes;
+    return a.p + off;
+}
+
+// ---------------------------------------------------------------------------
+// timing hooks
+// ---------------------------------------------------------------------------
+
+static cudaEvent_t ev_get(fp_ctx* c) {
+    if (!c->ev_free.empty()) {
+        cudaEvent_t e = c->ev_free.back();
+        c->ev_free.pop_back();
+        return e;
+    }
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    return e;
+}
+
+void fp_tic(fp_ctx* c, cudaStream_t s, int kernel, double bytes, int* slot) {
+    *slot = -1;
+    c->launches++;
+    if (!c->profiling) return;
+    FpEvPair p;
+    p.a = ev_get(c);
+    p.b = ev_get(c);
+    p.kernel = kernel;
+    p.bytes = bytes;
+    cudaEventRecord(p.a, s);
+    c->ev_live.push_back(p);
+    *slot = (int)c->ev_live.size() - 1;
+}
+
+void fp_toc(fp_ctx* c, cudaStream_t s, int slot) {
+    if (slot < 0) return;
+    cudaEventRecord(c->ev_live[slot].b, s);
+}
+
+static void stats_resolve(fp_ctx* c) {
+    for (auto& p : c->ev_live) {
+        cudaEventSynchronize(p.b);
+        float ms = 0.f;
+        cudaEventElapsedTime(&ms, p.a, p.b);
+        c->stats[p.kernel].launches += 1;
+        c->stats[p.kernel].ms += ms;
+        c->stats[p.kernel].bytes += p.bytes;
+        c->ev_free.push_back(p.a);
+        c->ev_free.push_back(p.b);
+    }
+    c->ev_live.clear();
+}
+
+void fp_stats_reset(fp_ctx* c) {
+    stats_resolve(c);
+    for (auto& s : c->stats) s = FpKStat();
+}
+
+int fp_ctx_set_profiling(fp_ctx* c, int on) {
+    if (!c) return FP_ERR_ARG;
+    stats_resolve(c);
+    c->profiling = on ? 1 : 0;
+    for (auto& s : c->stats) s = FpKStat();
+    return FP_OK;
+}
+
+int64_t fp_ctx_launches(const fp_ctx* c) { return c ? c->launches : -1; }
+
+int fp_kernel_stats(fp_ctx* c, fp_kernel_stat* out, int cap) {
+    if (!c || (cap > 0 && !out)) return FP_ERR_ARG;
+    stats_resolve(c);
+    int n = 0;
+    for (int k = 0; k < K_COUNT; k++) {
+        if (c->stats[k].launches == 0) continue;
+        if (n < cap) {
+            out[n].kernel = k;
+            out[n].launches = c->stats[k].launches;
+            out[n].ms = c->stats[k].ms;
+            out[n].bytes = c->stats[k].bytes;
+        }
+        n++;
+    }
+    return n;
+}
+
+const char* fp_kernel_name(int k) {
+    static const char* names[K_COUNT] = {
+        "witness_gemm", "digest_leaf", "digest_node", "digest_final", "eq_build", "partial_acc",
+        "partial_fin", "claim", "sc_round", "sc_final", "hist", "keys_gather", "tree_leaf",
+        "tree_up", "gkr_round", "gkr_final", "leaf_eval", "reduce"};
+    return (k >= 0 && k < K_COUNT) ? names[k] : "?";
+}
+
+// ---------------------------------------------------------------------------
+// statement checks
+// ---------------------------------------------------------------------------
+
+int fp_check_sites(fp_ctx* c, const fp_site* sites, int nsites, bool need_witness) {
+    if (!sites || nsites < 1) return fp_fail(c, FP_ERR_SHAPE, "need at least one site");
+    for (int s = 0; s < nsites; s++) {
+        const fp_site& t = sites[s];
+        char buf[160];
+        if (t.w_bits != 4 && t.w_bits != 8) {
+            snprintf(buf, sizeof buf, "site %d: w_bits must be 4 or 8", s);
+            return fp_fail(c, FP_ERR_ARG, buf);
+        }
+        if (t.M < 1 || t.N < 1 || t.K < 1 || t.M > (1 << 24) || t.N > (1 << 24) || t.K > (1 << 20)) {
+            snprintf(buf, sizeof buf, "site %d: dims %d x %d x %d outside [1, 2^24] x [1, 2^20] x [1, 2^24]", s,
+                     t.M, t.K, t.N);
+            return fp_fail(c, FP_ERR_SHAPE, buf);
+        }
+        if (t.k_shift < 1 || t.k_shift > 20) {
+            snprintf(buf, sizeof buf, "site %d: k_shift %d outside [1, 20]", s, t.k_shift);
+            return fp_fail(c, FP_ERR_SHAPE, buf);
+        }
+        // worst-case |Y| < 2^31 keeps the int32 accumulation exact
+        double wmax = (t.w_bits == 4 ? 8.0 : 128.0) * (t.scales ? 128.0 : 1.0);
+        if (wmax * 128.0 * (double)t.K >= 2147483648.0) {
+            snprintf(buf, sizeof buf, "site %d: K = %d can overflow the int32 accumulator", s, t.K);
+            return fp_fail(c, FP_ERR_SHAPE, buf);
+        }
+        if (!t.w || !t.xt) {
+            snprintf(buf, sizeof buf, "site %d: null operand", s);
+            return fp_fail(c, FP_ERR_ARG, buf);
+        }
+        if (need_witness && (!t.q || !t.r || !t.y)) {
+            snprintf(buf, sizeof buf, "site %d: null witness buffer", s);
+            return fp_fail(c, FP_ERR_ARG, buf);
+        }
+    }
+    return FP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// transcript entry points
+// ---------------------------------------------------------------------------
+
+fp_tx* fp_tx_create(uint64_t seed) {
+    fp_tx* t = new fp_tx();
+    uint8_t b[15];
+    memcpy(b, "FPSC-v1", 7);
+    for (int i = 0; i < 8; i++) b[7 + i] = (uint8_t)(seed >> (8 * i));
+    FpSha256 h;
+    h.update(b, 15);
+    h.final(t->st);
+    return t;
+}
+
+void fp_tx_destroy(fp_tx* t) { delete t; }
+
+int fp_tx_absorb(fp_tx* t, const char* label, const void* data, size_t n) {
+    if (!t || !label || (n && !data)) return FP_ERR_ARG;
+    fp_tx_absorb_raw(t, label, data, n);
+    return FP_OK;
+}
+
+int fp_tx_squeeze(fp_tx* t, const char* label, uint64_t* out, size_t n) {
+    if (!t || !label || (n && !out)) return FP_ERR_ARG;
+    for (size_t i = 0; i < n; i++) out[i] = fp_tx_squeeze_one(t, label);
+    return FP_OK;
+}
+
+int fp_tx_state(const fp_tx* t, uint8_t out[32]) {
+    if (!t || !out) return FP_ERR_ARG;
+    memcpy(out, t->st, 32);
+    return FP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// digest, witness, partial evaluation
+// ---------------------------------------------------------------------------
+
+int fp_digest(fp_ctx* c, const void* dev, size_t nbytes, uint8_t out[32], void* stream) {
+    if (!c || !out || (nbytes && !dev)) return fp_fail(c, FP_ERR_ARG, "fp_digest: null argument");
+    FP_CUDA(c, cudaSetDevice(c->device));
+    FpDigestJob j{(const uint8_t*)dev, (uint64_t)nbytes};
+    return fp_digest_many(c, &j, 1, out, (cudaStream_t)stream);
+}
+
+int fp_commit_witness(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, void* stream) {
+    if (!c || !tx) return fp_fail(c, FP_ERR_ARG, "fp_commit_witness: null context or transcript");
+    int rc = fp_check_sites(c, sites, nsites, true);
+    if (rc) return rc;
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t s = (cudaStream_t)stream;
+    fp_reset(c->dev);
+    rc = fp_launch_witness(c, sites, nsites, s);
+    if (rc) return rc;
+    // digests: W and scales only where no offline digest is given
+    std::vector<FpDigestJob> jobs;
+    std::vector<int> where;  // job -> (site * 6 + slot)
+    for (int i = 0; i < nsites; i++) {
+        const fp_site& t = sites[i];
+        uint64_t mn = (uint64_t)t.M * t.N;
+        uint64_t wb = (uint64_t)t.M * (t.w_bits == 4 ? (uint64_t)((t.K + 1) / 2) : (uint64_t)t.K);
+        uint64_t sb = t.scales ? (uint64_t)t.M * ((t.K + 63) / 64) : 0;
+        if (!t.w_digest) {
+            jobs.push_back({(const uint8_t*)t.w, wb});
+            where.push_back(6 * i + 0);
+            jobs.push_back({(const uint8_t*)t.scales, sb});
+            where.push_back(6 * i + 1);
+        }
+        jobs.push_back({(const uint8_t*)t.xt, (uint64_t)t.N * t.K});
+        where.push_back(6 * i + 2);
+        jobs.push_back({(const uint8_t*)t.q, 4 * mn});
+        where.push_back(6 * i + 3);
+        jobs.push_back({(const uint8_t*)t.r, 4 * mn});
+        where.push_back(6 * i + 4);
+        jobs.push_back({(const uint8_t*)t.y, mn});
+        where.push_back(6 * i + 5);
+    }
+    std::vector<uint8_t> dg(32 * jobs.size());
+    rc = fp_digest_many(c, jobs.data(), (int)jobs.size(), dg.data(), s);
+    if (rc) return rc;
+    std::vector<uint8_t> rec(192 * (size_t)nsites);
+    for (int i = 0; i < nsites; i++)
+        if (sites[i].w_digest) memcpy(&rec[192 * i], sites[i].w_digest, 64);
+    for (size_t j = 0; j < jobs.size(); j++) memcpy(&rec[32 * where[j]], &dg[32 * j], 32);
+    for (int i = 0; i < nsites; i++) fp_tx_absorb_raw(tx, "site", &rec[192 * i], 192);
+    return FP_OK;
+}
+
+int mle_partial_eval(fp_ctx* c, const void* mat, int bits, const int8_t* scales, int rows, int cols,
+                     const uint64_t* point, int npoint, uint64_t* out, void* stream) {
+    if (!c || !mat || !out || (npoint && !point)) return fp_fail(c, FP_ERR_ARG, "mle_partial_eval: null argument");
+    if (bits != 4 && bits != 8) return fp_fail(c, FP_ERR_ARG, "mle_partial_eval: bits must be 4 or 8");
+    if (rows < 1 || cols < 1 || rows > (1 << 24) || cols > (1 << 24))
+        return fp_fail(c, FP_ERR_SHAPE, "mle_partial_eval: dims outside [1, 2^24]");
+    if (npoint != fp_log2_ceil((uint64_t)rows) || npoint > 32)
+        return fp_fail(c, FP_ERR_SHAPE, "mle_partial_eval: npoint must be ceil(log2 rows)");
+    for (int i = 0; i < npoint; i++)
+        if (point[i] >= 0xFFFFFFFF00000001ull) return fp_fail(c, FP_ERR_ARG, "mle_partial_eval: point not canonical");
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t s = (cudaStream_t)stream;
+    int rc = fp_reserve(c, c->dev, ((size_t)8 << npoint) + fp_partial_rows_scratch(rows, cols) + (1 << 20));
+    if (rc) return rc;
+    fp_reset(c->dev);
+    uint64_t* eq = (uint64_t*)fp_alloc(c->dev, (size_t)8 << npoint);
+    FpPoint z;
+    z.v = npoint;
+    for (int i = 0; i < npoint; i++) z.z[i] = point[i];
+    rc = fp_eq_table(c, z, eq, s);
+    if (rc) return rc;
+    rc = fp_partial_rows(c, mat, bits, scales, rows, cols, eq, out, 1ll << fp_log2_ceil((uint64_t)cols), s);
+    if (rc) return rc;
+    FP_CUDA(c, cudaStreamSynchronize(s));
+    return FP_OK;
+}
+
+int fp_proof_size(const fp_site* sites, int nsites, size_t* mm, size_t* lu) {
+    if (!sites || nsites < 1 || !mm || !lu) return FP_ERR_ARG;
+    int n = 0;
+    uint64_t nk = 0;
+    for (int s = 0; s < nsites; s++) {
+        if (sites[s].K < 1 || sites[s].M < 1 || sites[s].N < 1) return FP_ERR_SHAPE;
+        int a = fp_log2_ceil((uint64_t)sites[s].K);
+        if (a > n) n = a;
+        nk += (uint64_t)sites[s].M * sites[s].N;
+    }
+    int v = fp_log2_ceil(nk);
+    if (v < 1) v = 1;
+    *mm = 8 * (size_t)nsites + 24 * (size_t)n + 16 * (size_t)nsites;
+    size_t l = 4 * ((size_t)1 << sites[0].k_shift) + 4 * 65536 + 64 + 24;
+    for (int d = 1; d < v; d++) l += 32 * (size_t)d + 64;
+    *lu = l;
+    return FP_OK;
+}

@@ -1,0 +1,135 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/fp.h"
+#include "fp_sha256.cuh"
+
+// ---------------------------------------------------------------------------
+// kernels known to the per-kernel timing table
+// ---------------------------------------------------------------------------
+enum FpKernel {
+    K_GEMM = 0,
+    K_DIGEST_LEAF,
+    K_DIGEST_NODE,
+    K_DIGEST_FINAL,
+    K_EQ_BUILD,
+    K_PARTIAL_ACC,
+    K_PARTIAL_FIN,
+    K_CLAIM,
+    K_SC_ROUND,
+    K_SC_FINAL,
+    K_HIST,
+    K_KEYS_GATHER,
+    K_TREE_LEAF,
+    K_TREE_UP,
+    K_GKR_ROUND,
+    K_GKR_FINAL,
+    K_LEAF_EVAL,
+    K_REDUCE,
+    K_COUNT
+};
+
+struct FpKStat {
+    int launches = 0;
+    double ms = 0.0;
+    double bytes = 0.0;
+};
+
+// a pair of events around one launch, resolved lazily
+struct FpEvPair {
+    cudaEvent_t a, b;
+    int kernel;
+    double bytes;
+};
+
+// A growable block carved by a bump allocator. Growing it frees the old block,
+// so every entry point reserves what it needs before handing out pointers.
+struct FpArena {
+    char* p = nullptr;
+    size_t cap = 0;
+    size_t top = 0;
+    bool pinned_host = false;
+};
+
+struct fp_ctx {
+    int device = 0;
+    int num_sms = 148;
+    std::string err;
+    FpArena dev;       // device scratch of the current entry point
+    FpArena dig;       // device scratch of the digest kernels (independent of dev)
+    FpArena host;      // pinned host staging of the current entry point
+    FpArena dig_host;  // pinned host staging of the digest path
+    // small persistent device block: reduction tickets (kept zero between launches)
+    unsigned int* tickets = nullptr;
+    // timing
+    int profiling = 0;
+    int64_t launches = 0;  // every kernel launch of the library on this context
+    std::vector<FpEvPair> ev_live;
+    std::vector<cudaEvent_t> ev_free;
+    FpKStat stats[K_COUNT];
+};
+
+struct fp_tx {
+    uint8_t st[32];
+};
+
+// ---- helpers (api.cu) ------------------------------------------------------
+int fp_fail(fp_ctx* c, int code, const std::string& msg);
+int fp_cuda_check(fp_ctx* c, cudaError_t e, const char* what);
+#define FP_CUDA(c, call)                                  \
+    do {                                                  \
+        cudaError_t e__ = (call);                         \
+        if (e__ != cudaSuccess) return fp_cuda_check(c, e__, #call); \
+    } while (0)
+
+// arenas: reserve (may reallocate, contents and pointers lost), then alloc
+// 256-byte aligned blocks; reset at the start of every public call.
+int fp_reserve(fp_ctx* c, FpArena& a, size_t bytes);
+void* fp_alloc(FpArena& a, size_t bytes);
+static inline void fp_reset(FpArena& a) { a.top = 0; }
+
+// timing hooks around a launch (no-ops unless profiling)
+void fp_tic(fp_ctx* c, cudaStream_t s, int kernel, double bytes, int* slot);
+void fp_toc(fp_ctx* c, cudaStream_t s, int slot);
+void fp_stats_reset(fp_ctx* c);
+
+// transcript (transcript.cu)
+void fp_tx_absorb_raw(fp_tx* t, const char* label, const void* data, uint64_t n);
+uint64_t fp_tx_squeeze_one(fp_tx* t, const char* label);
+
+// statement checks shared by the entry points (api.cu)
+int fp_check_sites(fp_ctx* c, const fp_site* sites, int nsites, bool need_witness);
+int fp_log2_ceil(uint64_t n);
+
+// digests of device buffers (digest.cu): out is host, 32 bytes per job
+struct FpDigestJob {
+    const uint8_t* ptr;
+    uint64_t len;
+};
+int fp_digest_many(fp_ctx* c, const FpDigestJob* jobs, int njobs, uint8_t* out, cudaStream_t s);
+
+// witness (witness.cu)
+int fp_launch_witness(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t s);
+
+// MLE building blocks (mle.cu)
+struct FpPoint {
+    uint64_t z[32];
+    int v;
+};
+int fp_eq_table(fp_ctx* c, const FpPoint& z, uint64_t* out, cudaStream_t s);
+// out[c] = sum_{i<rows} eq[i] M_eff[i][c]; eq device (rows entries); out device (cols_pad)
+// out has out_len >= cols entries; entries past cols are zeroed
+int fp_partial_rows(fp_ctx* c, const void* mat, int bits, const int8_t* scales, int rows, int cols,
+                    const uint64_t* eq, uint64_t* out, int64_t out_len, cudaStream_t s);
+size_t fp_partial_rows_scratch(int rows, int cols);
+size_t fp_claims_scratch(const fp_site* sites, int nsites);
+// per-site output claims into dev_out[s]
+int fp_claims(fp_ctx* c, const fp_site* sites, int nsites, const uint64_t* const* eq_rows,
+              const uint64_t* const* eq_cols, uint64_t* dev_out, cudaStream_t s);
+
+static inline size_t fp_align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

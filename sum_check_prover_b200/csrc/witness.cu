@@ -1,0 +1,353 @@
+// Witness of the quantised matrix products ("How fast can FlashProve go", 3.1):
+// Y = W_eff . X with exact int32 accumulation on the tensor cores, then the
+// rescale q = floor((Y + 2^(k-1)) / 2^k), the committed remainder
+// r = Y - 2^k q and the clamp y = clamp(q, -128, 127), fused into the epilogue.
+//
+// D = Y^T (tokens x output rows) is computed as Xt . W^T so that both
+// operands are K-contiguous (token-major activations, row-major weights).
+// int4 weights are expanded to int8 in registers while building fragments;
+// per-64 group scales multiply each k-tile's partial product (one k-tile is
+// one scale group).
+//
+// Tile 128 tokens x 128 rows x 64 k, 8 warps (2 x 4), warp tile 64 x 32,
+// mma.sync m16n8k32 s8.s8.s32, 3-stage cp.async pipeline. All sites of a call
+// share one launch per operand variant (grouped GEMM over a tile list).
+#include <vector>
+
+#include "fp_internal.h"
+
+namespace {
+
+constexpr int BM = 128;  // tokens (rows of D)
+constexpr int BN = 128;  // output rows i (columns of D)
+constexpr int BK = 64;
+constexpr int STAGES = 3;
+constexpr int THREADS = 256;
+constexpr int A_PITCH = 80;               // bytes per smem row of the Xt tile (64 + 16 pad)
+constexpr int B8_PITCH = 80;              // int8 W tile
+constexpr int B4_PITCH = 48;              // int4 W tile (32 + 16 pad)
+constexpr int A_STAGE = BM * A_PITCH;     // 10240
+constexpr int B_STAGE = BN * B8_PITCH;    // 10240 (int4 uses the first BN * 48)
+
+struct SiteDev {
+    const uint8_t* w;
+    const int8_t* scales;
+    const int8_t* xt;
+    int32_t* q;
+    int32_t* r;
+    int8_t* y;
+    int32_t M, K, N, k_shift;
+    int32_t tiles_i, tiles_j;
+    int64_t tile_base;  // first tile index of this site in the launch
+};
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int src_bytes) {
+    uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void mma_s8(int32_t (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// four packed nibbles (k0..k0+3, low nibble first) -> four int8 in one word
+__device__ __forceinline__ uint32_t nib4_to_s8x4(uint32_t v16) {
+    uint32_t lo = v16 & 0x0F0Fu;
+    uint32_t hi = (v16 >> 4) & 0x0F0Fu;
+    uint32_t w = __byte_perm(lo, hi, 0x5140);
+    return w | ((w & 0x08080808u) * 0x1Eu);  // sign-extend bit 3 of every byte
+}
+
+__device__ __forceinline__ int find_site(const SiteDev* sites, int nsites, int64_t t) {
+    int lo = 0, hi = nsites - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (sites[mid].tile_base <= t)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+// Load one k-tile of Xt (BM x BK) and W (BN x BK) into a stage.
+template <bool W4, bool ALIGNED>
+__device__ __forceinline__ void load_tile(const SiteDev& S, int j0, int i0, int k0, uint8_t* sa, uint8_t* sb) {
+    const int tid = threadIdx.x;
+    if (ALIGNED) {
+        // Xt: 128 rows x 4 chunks of 16 bytes
+#pragma unroll
+        for (int c = tid; c < BM * 4; c += THREADS) {
+            int row = c >> 2, ch = c & 3;
+            int j = j0 + row, k = k0 + ch * 16;
+            bool ok = (j < S.N) && (k < S.K);
+            const int8_t* src = ok ? S.xt + (int64_t)j * S.K + k : S.xt;
+            cp_async16(sa + row * A_PITCH + ch * 16, src, ok ? 16 : 0);
+        }
+        if (W4) {
+            const int pitch = (S.K + 1) >> 1;
+#pragma unroll
+            for (int c = tid; c < BN * 2; c += THREADS) {
+                int row = c >> 1, ch = c & 1;
+                int i = i0 + row, kb = (k0 >> 1) + ch * 16;
+                bool ok = (i < S.M) && (kb < pitch);
+                const uint8_t* src = ok ? S.w + (int64_t)i * pitch + kb : S.w;
+                cp_async16(sb + row * B4_PITCH + ch * 16, src, ok ? 16 : 0);
+            }
+        } else {
+#pragma unroll
+            for (int c = tid; c < BN * 4; c += THREADS) {
+                int row = c >> 2, ch = c & 3;
+                int i = i0 + row, k = k0 + ch * 16;
+                bool ok = (i < S.M) && (k < S.K);
+                const uint8_t* src = ok ? S.w + (int64_t)i * S.K + k : S.w;
+                cp_async16(sb + row * B8_PITCH + ch * 16, src, ok ? 16 : 0);
+            }
+        }
+    } else {
+        // generic path: byte loads with full bounds checks
+        for (int c = tid; c < BM * BK; c += THREADS) {
+            int row = c / BK, kk = c % BK;
+            int j = j0 + row, k = k0 + kk;
+            sa[row * A_PITCH + kk] = (j < S.N && k < S.K) ? (uint8_t)S.xt[(int64_t)j * S.K + k] : 0;
+        }
+        if (W4) {
+            const int pitch = (S.K + 1) >> 1;
+            for (int c = tid; c < BN * (BK / 2); c += THREADS) {
+                int row = c / (BK / 2), kb = c % (BK / 2);
+                int i = i0 + row, k = k0 + 2 * kb;
+                uint8_t v = 0;
+                if (i < S.M && k < S.K) {
+                    v = S.w[(int64_t)i * pitch + (k >> 1)];
+                    if (k + 1 >= S.K) v &= 0x0F;
+                }
+                sb[row * B4_PITCH + kb] = v;
+            }
+        } else {
+            for (int c = tid; c < BN * BK; c += THREADS) {
+                int row = c / BK, kk = c % BK;
+                int i = i0 + row, k = k0 + kk;
+                sb[row * B8_PITCH + kk] = (i < S.M && k < S.K) ? S.w[(int64_t)i * S.K + k] : 0;
+            }
+        }
+    }
+}
+
+template <bool W4, bool SCALED, bool ALIGNED>
+__global__ void __launch_bounds__(THREADS, 1)
+    witness_gemm_kernel(const SiteDev* __restrict__ sites, int nsites) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * A_STAGE;
+
+    const int64_t tile = blockIdx.x;
+    const int s = find_site(sites, nsites, tile);
+    const SiteDev S = sites[s];
+    const int64_t lt = tile - S.tile_base;
+    const int j0 = (int)(lt / S.tiles_i) * BM;
+    const int i0 = (int)(lt % S.tiles_i) * BN;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int wj = (warp >> 2) * 64;  // warp's token offset in the tile
+    const int wi = (warp & 3) * 32;   // warp's row offset in the tile
+
+    int32_t acc[4][4][4];
+    int32_t tot[4][4][4];  // scaled running total (dead code without scales)
+#pragma unroll
+    for (int a = 0; a < 4; a++)
+#pragma unroll
+        for (int b = 0; b < 4; b++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) acc[a][b][e] = tot[a][b][e] = 0;
+
+    const int nk = (S.K + BK - 1) / BK;
+    const int G = (S.K + 63) / 64;
+
+    if (ALIGNED) {
+#pragma unroll
+        for (int st = 0; st < STAGES - 1; st++) {
+            if (st < nk) load_tile<W4, true>(S, j0, i0, st * BK, sA + st * A_STAGE, sB + st * B_STAGE);
+            cp_async_commit();
+        }
+    }
+
+    for (int kt = 0; kt < nk; kt++) {
+        uint8_t* a_st;
+        uint8_t* b_st;
+        if (ALIGNED) {
+            cp_async_wait<STAGES - 2>();
+            __syncthreads();
+            int nxt = kt + STAGES - 1;
+            if (nxt < nk)
+                load_tile<W4, true>(S, j0, i0, nxt * BK, sA + (nxt % STAGES) * A_STAGE, sB + (nxt % STAGES) * B_STAGE);
+            cp_async_commit();
+            a_st = sA + (kt % STAGES) * A_STAGE;
+            b_st = sB + (kt % STAGES) * B_STAGE;
+        } else {
+            __syncthreads();
+            load_tile<W4, false>(S, j0, i0, kt * BK, sA, sB);
+            __syncthreads();
+            a_st = sA;
+            b_st = sB;
+        }
+
+#pragma unroll
+        for (int ks = 0; ks < 2; ks++) {
+            uint32_t af[4][4];
+            uint32_t bf[4][2];
+#pragma unroll
+            for (int mt = 0; mt < 4; mt++) {
+                const uint8_t* base = a_st + (wj + mt * 16 + g) * A_PITCH + ks * 32 + 4 * t;
+                af[mt][0] = *reinterpret_cast<const uint32_t*>(base);
+                af[mt][1] = *reinterpret_cast<const uint32_t*>(base + 8 * A_PITCH);
+                af[mt][2] = *reinterpret_cast<const uint32_t*>(base + 16);
+                af[mt][3] = *reinterpret_cast<const uint32_t*>(base + 8 * A_PITCH + 16);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; nt++) {
+                const int row = wi + nt * 8 + g;
+                if (W4) {
+                    const uint8_t* base = b_st + row * B4_PITCH + ks * 16 + 2 * t;
+                    bf[nt][0] = nib4_to_s8x4(*reinterpret_cast<const uint16_t*>(base));
+                    bf[nt][1] = nib4_to_s8x4(*reinterpret_cast<const uint16_t*>(base + 8));
+                } else {
+                    const uint8_t* base = b_st + row * B8_PITCH + ks * 32 + 4 * t;
+                    bf[nt][0] = *reinterpret_cast<const uint32_t*>(base);
+                    bf[nt][1] = *reinterpret_cast<const uint32_t*>(base + 16);
+                }
+            }
+#pragma unroll
+            for (int mt = 0; mt < 4; mt++)
+#pragma unroll
+                for (int nt = 0; nt < 4; nt++) mma_s8(acc[mt][nt], af[mt], bf[nt]);
+        }
+
+        if (SCALED) {
+            // this k-tile is scale group kt: tot += S[i][kt] * acc, then restart acc
+#pragma unroll
+            for (int nt = 0; nt < 4; nt++) {
+                const int ia = i0 + wi + nt * 8 + 2 * t;
+                int32_t s0 = (ia < S.M) ? (int32_t)S.scales[(int64_t)ia * G + kt] : 0;
+                int32_t s1 = (ia + 1 < S.M) ? (int32_t)S.scales[(int64_t)(ia + 1) * G + kt] : 0;
+#pragma unroll
+                for (int mt = 0; mt < 4; mt++) {
+                    tot[mt][nt][0] += s0 * acc[mt][nt][0];
+                    tot[mt][nt][1] += s1 * acc[mt][nt][1];
+                    tot[mt][nt][2] += s0 * acc[mt][nt][2];
+                    tot[mt][nt][3] += s1 * acc[mt][nt][3];
+                    acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0;
+                }
+            }
+        }
+    }
+    if (ALIGNED) cp_async_wait<0>();
+
+    // epilogue: rescale, remainder, clamp; D[j][i] -> q, r, y at [j * M + i]
+    const int k = S.k_shift;
+    const int64_t half = (int64_t)1 << (k - 1);
+#pragma unroll
+    for (int mt = 0; mt < 4; mt++)
+#pragma unroll
+        for (int nt = 0; nt < 4; nt++)
+#pragma unroll
+            for (int hh = 0; hh < 2; hh++) {
+                const int j = j0 + wj + mt * 16 + g + 8 * hh;
+                const int i = i0 + wi + nt * 8 + 2 * t;
+                if (j >= S.N) continue;
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                    if (i + e >= S.M) continue;
+                    int32_t Y = SCALED ? tot[mt][nt][2 * hh + e] : acc[mt][nt][2 * hh + e];
+                    int64_t qq = ((int64_t)Y + half) >> k;  // arithmetic shift = floor division
+                    int64_t rr = (int64_t)Y - (qq << k);
+                    int64_t o = (int64_t)j * S.M + i + e;
+                    S.q[o] = (int32_t)qq;
+                    S.r[o] = (int32_t)rr;
+                    S.y[o] = (int8_t)(qq < -128 ? -128 : (qq > 127 ? 127 : qq));
+                }
+            }
+}
+
+template <bool W4, bool SCALED, bool ALIGNED>
+int launch_variant(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
+    if (list.empty()) return FP_OK;
+    std::vector<SiteDev> h(list.size());
+    int64_t tiles = 0;
+    double bytes = 0;
+    for (size_t s = 0; s < list.size(); s++) {
+        const fp_site& t = list[s];
+        SiteDev& d = h[s];
+        d.w = (const uint8_t*)t.w;
+        d.scales = t.scales;
+        d.xt = t.xt;
+        d.q = t.q;
+        d.r = t.r;
+        d.y = t.y;
+        d.M = t.M;
+        d.K = t.K;
+        d.N = t.N;
+        d.k_shift = t.k_shift;
+        d.tiles_i = (t.M + BN - 1) / BN;
+        d.tiles_j = (t.N + BM - 1) / BM;
+        d.tile_base = tiles;
+        tiles += (int64_t)d.tiles_i * d.tiles_j;
+        bytes += (double)t.M * (W4 ? (t.K + 1) / 2 : t.K) + (double)t.N * t.K + 9.0 * t.M * t.N;
+    }
+    size_t sz = sizeof(SiteDev) * h.size();
+    SiteDev* dsites = (SiteDev*)fp_alloc(c->dev, sz);
+    char* hst = (char*)fp_alloc(c->host, sz);
+    if (!dsites || !hst) return fp_fail(c, FP_ERR_OOM, "witness: scratch exhausted");
+    memcpy(hst, h.data(), sz);
+    FP_CUDA(c, cudaMemcpyAsync(dsites, hst, sz, cudaMemcpyHostToDevice, st));
+    const int smem = STAGES * (A_STAGE + B_STAGE);
+    auto kern = witness_gemm_kernel<W4, SCALED, ALIGNED>;
+    FP_CUDA(c, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    int slot;
+    fp_tic(c, st, K_GEMM, bytes, &slot);
+    kern<<<(unsigned)tiles, THREADS, smem, st>>>(dsites, (int)h.size());
+    fp_toc(c, st, slot);
+    FP_CUDA(c, cudaGetLastError());
+    return FP_OK;
+}
+
+}  // namespace
+
+int fp_launch_witness(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st) {
+    // group sites by kernel variant
+    std::vector<fp_site> v[8];
+    for (int s = 0; s < nsites; s++) {
+        const fp_site& t = sites[s];
+        bool w4 = t.w_bits == 4, sc = t.scales != nullptr;
+        size_t pitch = w4 ? (size_t)(t.K + 1) / 2 : (size_t)t.K;
+        bool al = ((uintptr_t)t.w % 16 == 0) && ((uintptr_t)t.xt % 16 == 0) && (pitch % 16 == 0) &&
+                  (t.K % 16 == 0) && (!w4 || t.K % 32 == 0);
+        v[(w4 ? 4 : 0) + (sc ? 2 : 0) + (al ? 1 : 0)].push_back(t);
+    }
+    size_t need = 0;
+    for (int i = 0; i < 8; i++) need += fp_align_up(sizeof(SiteDev) * v[i].size(), 256) + 256;
+    int rc = fp_reserve(c, c->dev, need + (1 << 20));
+    if (rc) return rc;
+    rc = fp_reserve(c, c->host, need + (1 << 20));
+    if (rc) return rc;
+    fp_reset(c->dev);
+    fp_reset(c->host);
+    if ((rc = launch_variant<false, false, false>(c, v[0], st))) return rc;
+    if ((rc = launch_variant<false, false, true>(c, v[1], st))) return rc;
+    if ((rc = launch_variant<false, true, false>(c, v[2], st))) return rc;
+    if ((rc = launch_variant<false, true, true>(c, v[3], st))) return rc;
+    if ((rc = launch_variant<true, false, false>(c, v[4], st))) return rc;
+    if ((rc = launch_variant<true, false, true>(c, v[5], st))) return rc;
+    if ((rc = launch_variant<true, true, false>(c, v[6], st))) return rc;
+    if ((rc = launch_variant<true, true, true>(c, v[7], st))) return rc;
+    return FP_OK;
+}

@@ -51,6 +51,8 @@ class Site:
     # Sites whose outputs live inside one shared N x M buffer: (group, offset).
     out_group: Optional[tuple] = None
     stage: int = 0
+    # W is a committed weight (digested once, offline) rather than an activation
+    w_is_weight: bool = True
 
     @property
     def macs(self) -> int:
@@ -199,14 +201,14 @@ def _attn_dense(seed: int, d=5120, nq=40, nkv=8, hd=128, B=64, ctx=2048, ffn=163
     for b in range(B):
         for kv in range(nkv):
             sites.append(Site(f"ot.{b}.{kv}", hd, ctx, g, 8, k, w=vt[b, kv], xt=pr[b, kv],
-                              out_group=("attn_out", b * d + kv * g * hd)))
+                              out_group=("attn_out", b * d + kv * g * hd), w_is_weight=False))
     sites.append(Site("gate", ffn, d, B, 4, k, w=int4_packed(_rng(seed, 4), ffn, d), xt=m))
     sites.append(Site("up", ffn, d, B, 4, k, w=int4_packed(_rng(seed, 5), ffn, d), xt=m))
     sites.append(Site("down", d, ffn, B, 4, k, w=int4_packed(_rng(seed, 6), d, ffn), xt=h))
     for b in range(B):
         for kv in range(nkv):
             sites.append(Site(f"s.{b}.{kv}", g, hd, ctx, 8, k, xt=kc[b, kv],
-                              w_link=(qi, b * nq * hd + kv * g * hd), stage=1))
+                              w_link=(qi, b * nq * hd + kv * g * hd), stage=1, w_is_weight=False))
     sites.append(Site("wo", d, nq * hd, B, 4, k, w=int4_packed(_rng(seed, 7), d, nq * hd),
                       xt_link=(first_o, 0), stage=1))
     return Workload("attn_dense", seed, sites, groups={"attn_out": (B, nq * hd)},
