@@ -328,7 +328,7 @@ int mle_partial_eval(fp_ctx* c, const void* mat, int bits, const int8_t* scales,
         if (point[i] >= 0xFFFFFFFF00000001ull) return fp_fail(c, FP_ERR_ARG, "mle_partial_eval: point not canonical");
     FP_CUDA(c, cudaSetDevice(c->device));
     cudaStream_t s = (cudaStream_t)stream;
-    int rc = fp_reserve(c, c->dev, ((size_t)8 << npoint) + fp_partial_rows_scratch(rows, cols) + (1 << 20));
+    int rc = fp_reserve(c, c->dev, ((size_t)8 << npoint) + fp_partial_rows_scratch(c, rows, cols) + (1 << 20));
     if (rc) return rc;
     fp_reset(c->dev);
     uint64_t* eq = (uint64_t*)fp_alloc(c->dev, (size_t)8 << npoint);

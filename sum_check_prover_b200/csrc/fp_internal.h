@@ -126,7 +126,7 @@ int fp_eq_table(fp_ctx* c, const FpPoint& z, uint64_t* out, cudaStream_t s);
 // out has out_len >= cols entries; entries past cols are zeroed
 int fp_partial_rows(fp_ctx* c, const void* mat, int bits, const int8_t* scales, int rows, int cols,
                     const uint64_t* eq, uint64_t* out, int64_t out_len, cudaStream_t s);
-size_t fp_partial_rows_scratch(int rows, int cols);
+size_t fp_partial_rows_scratch(const fp_ctx* c, int rows, int cols);
 size_t fp_claims_scratch(const fp_site* sites, int nsites);
 // per-site output claims into dev_out[s]
 int fp_claims(fp_ctx* c, const fp_site* sites, int nsites, const uint64_t* const* eq_rows,

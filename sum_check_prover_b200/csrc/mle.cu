@@ -216,8 +216,20 @@ int fp_eq_table(fp_ctx* c, const FpPoint& z, uint64_t* out, cudaStream_t s) {
     return FP_OK;
 }
 
-size_t fp_partial_rows_scratch(int rows, int cols) {
-    int splits = (rows + PR_ROWS_PER_SPLIT_MAX - 1) / PR_ROWS_PER_SPLIT_MAX;
+// row splits of the partial evaluation: about two waves of blocks, every
+// split short enough for the exact 64-bit column sums
+static int pr_rows_per_split(int num_sms, int rows, int cols) {
+    int col_blocks = (cols + PR_THREADS * PR_COLS - 1) / (PR_THREADS * PR_COLS);
+    int want_splits = (2 * num_sms * 4 + col_blocks - 1) / col_blocks;
+    int rps = (rows + want_splits - 1) / want_splits;
+    if (rps < 64) rps = 64;
+    if (rps > PR_ROWS_PER_SPLIT_MAX) rps = PR_ROWS_PER_SPLIT_MAX;
+    return rps;
+}
+
+size_t fp_partial_rows_scratch(const fp_ctx* c, int rows, int cols) {
+    int rps = pr_rows_per_split(c->num_sms, rows, cols);
+    int splits = (rows + rps - 1) / rps;
     return fp_align_up((size_t)8 * splits * cols, 256) + 512;
 }
 
@@ -225,13 +237,9 @@ int fp_partial_rows(fp_ctx* c, const void* mat, int bits, const int8_t* scales, 
                     const uint64_t* eq, uint64_t* out, int64_t out_len, cudaStream_t s) {
     const bool w4 = bits == 4, sc = scales != nullptr;
     const int64_t pitch = w4 ? (cols + 1) / 2 : cols;
-    // rows per split: keep the row-split grid near two waves of the GPU
-    int col_blocks = (cols + PR_THREADS * PR_COLS - 1) / (PR_THREADS * PR_COLS);
-    int want_splits = (2 * c->num_sms * 4 + col_blocks - 1) / col_blocks;
-    int rps = (rows + want_splits - 1) / want_splits;
-    if (rps < 64) rps = 64;
-    if (rps > PR_ROWS_PER_SPLIT_MAX) rps = PR_ROWS_PER_SPLIT_MAX;
-    int splits = (rows + rps - 1) / rps;
+    const int col_blocks = (cols + PR_THREADS * PR_COLS - 1) / (PR_THREADS * PR_COLS);
+    const int rps = pr_rows_per_split(c->num_sms, rows, cols);
+    const int splits = (rows + rps - 1) / rps;
     uint64_t* part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * splits * cols);
     uint64_t* esum = (uint64_t*)fp_alloc(c->dev, 256);
     if (!part || !esum) return fp_fail(c, FP_ERR_OOM, "partial evaluation: scratch exhausted");

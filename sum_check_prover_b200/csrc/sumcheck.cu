@@ -134,8 +134,8 @@ int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites
     need += 4 * fp_align_up(vec, 256);
     size_t pr = 0;
     for (int s = 0; s < nsites; s++)
-        pr = std::max(pr, std::max(fp_partial_rows_scratch(sites[s].M, sites[s].K),
-                                   fp_partial_rows_scratch(sites[s].N, sites[s].K)));
+        pr = std::max(pr, std::max(fp_partial_rows_scratch(c, sites[s].M, sites[s].K),
+                                   fp_partial_rows_scratch(c, sites[s].N, sites[s].K)));
     need += pr;
     const int max_blocks = 4 * c->num_sms;
     need += fp_align_up((size_t)8 * 3 * max_blocks, 256) + fp_align_up(8 * (size_t)nsites, 256) * 3 + (1 << 16);
