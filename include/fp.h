@@ -154,6 +154,34 @@ int mle_partial_eval(fp_ctx* ctx, const void* mat, int bits, const int8_t* scale
                      const uint64_t* point, int npoint, uint64_t* out, void* stream);
 
 /*
+ * mle_partial_eval without any device allocation. The pages have no
+ * counterpart: this entry point exists for callers that must not allocate
+ * device memory -- code running inside a host callback or an allocator hook,
+ * under a memory pool that forbids out-of-band cudaMalloc, or in a process that
+ * has already reserved all device memory. It takes no fp_ctx (creating one
+ * allocates) and calls no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * Same arguments and result as mle_partial_eval; `out` (device) receives
+ * 2^ceil(log2 cols) values. Scratch is a fixed 16 MiB device array inside the
+ * library (held on every GPU that loads it until the process exits), which
+ * limits the shape: ceil(rows / 1024) * cols must not exceed 2^21, and
+ * npoint <= 24. Larger shapes return FP_ERR_SHAPE; bad pointers or bits
+ * FP_ERR_ARG; a CUDA failure FP_ERR_CUDA. The kernels are queued on `stream`
+ * and the call returns without waiting: the result is ready when the stream
+ * reaches that point.
+ *
+ * The first call on each device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. Every call on a device shares the one scratch
+ * array and leaves its contents behind; each call overwrites every entry it
+ * reads, so nothing needs clearing, but calls whose kernels overlap on the GPU
+ * (different streams of the same device) race on the array and must be
+ * ordered by the caller.
+ */
+int mle_partial_eval_noalloc(const void* mat, int bits, const int8_t* scales, int rows, int cols,
+                             const uint64_t* point, int npoint, uint64_t* out, void* stream);
+
+/*
  * Matmul sum-check over all sites with claims batched by a random linear
  * combination ("How fast can FlashProve go", 2 and 2.1). Squeezes r_row, r_col;
  * sends the claims c_s = MLE of 2^k q + r at (r_row, r_col); squeezes rho_s
