@@ -206,6 +206,7 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     n0 = ctx.launches()
+    hw0 = ctx.host_stats()
     clocks.start()
     times = []
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -220,6 +221,9 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     launches = ctx.launches() - n0
+    hw1 = ctx.host_stats()
+    host_waits = (hw1[0] - hw0[0]) / args.steps
+    host_wait_ms = (hw1[1] - hw0[1]) * 1e3 / args.steps
     total_ms = sum(times)
     if pg is not None:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -313,6 +317,8 @@ def run_ours(args):
                 "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches,
+                "host_round_trips_per_step": host_waits,
+                "host_wait_ms_per_step": host_wait_ms,
                 "clocks": clk,
                 "kernels": kern,
                 "proof_bytes": proof_len}

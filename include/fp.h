@@ -209,6 +209,15 @@ int sumcheck_prove_matmul(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsit
 int logup_prove_rescale(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites, uint8_t* proof,
                         size_t* proof_len, void* stream);
 
+/*
+ * Self-test of the bounded device waits. The sum-check kernels stay resident
+ * across rounds and wait (a bounded number of polls) for each Fiat-Shamir
+ * challenge from the host. This call launches a kernel that waits for a
+ * challenge nobody posts: after about a second it gives up and flags the
+ * mailbox, and the call returns FP_ERR_TIMEOUT. The context stays usable.
+ */
+int fp_session_selftest(fp_ctx* ctx, void* stream);
+
 /* Proof section sizes in bytes for a statement (no GPU work). */
 int fp_proof_size(const fp_site* sites, int nsites, size_t* matmul_bytes, size_t* logup_bytes);
 
@@ -226,8 +235,15 @@ typedef struct {
     double bytes;
 } fp_kernel_stat;
 int fp_ctx_set_profiling(fp_ctx* ctx, int on);
+/* While profiling is on (and when the process runs under an injected profiler,
+ * or with FP_STEPPED=1 in the environment) every sum-check round is its own
+ * kernel launch, so that each launch can be timed; otherwise one resident kernel
+ * runs all rounds of a sum-check. Both produce the same proof bytes. */
 /* Number of kernels the library has launched on this context since its creation. */
 int64_t fp_ctx_launches(const fp_ctx* ctx);
+/* Host side of the round exchanges since the context was created:
+ * out[0] = waits for a device result, out[1] = seconds spent waiting. */
+int fp_host_stats(const fp_ctx* ctx, double out[2]);
 int fp_kernel_stats(fp_ctx* ctx, fp_kernel_stat* out, int cap);
 const char* fp_kernel_name(int kernel);
 

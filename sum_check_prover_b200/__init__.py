@@ -71,6 +71,8 @@ def lib():
     L.logup_prove_rescale.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
     L.fp_proof_size.argtypes = [C.POINTER(_Site), i32, C.POINTER(sz), C.POINTER(sz)]
     L.fp_ctx_set_profiling.argtypes = [vp, i32]
+    L.fp_session_selftest.argtypes = [vp, vp]
+    L.fp_host_stats.argtypes = [vp, C.POINTER(C.c_double)]
     L.fp_ctx_launches.restype = C.c_int64
     L.fp_ctx_launches.argtypes = [vp]
     L.fp_kernel_stats.argtypes = [vp, C.POINTER(_KStat), i32]
@@ -235,6 +237,16 @@ class Context:
 
     def set_profiling(self, on: bool):
         self._check(self._L.fp_ctx_set_profiling(self.h, 1 if on else 0), "fp_ctx_set_profiling")
+
+    def session_selftest(self, stream=None) -> int:
+        """Run the bounded-wait self-test; returns the status code (FP_ERR_TIMEOUT = -4 expected)."""
+        return int(self._L.fp_session_selftest(self.h, _stream(stream)))
+
+    def host_stats(self):
+        """(waits for a device result, seconds spent waiting) since the context was created."""
+        out = (C.c_double * 2)()
+        self._check(self._L.fp_host_stats(self.h, out), "fp_host_stats")
+        return int(out[0]), float(out[1])
 
     def launches(self) -> int:
         """Kernels launched by the library on this context so far."""

@@ -1,7 +1,13 @@
 // Context, errors, scratch arena, timing hooks, statement checks and the small
 // entry points (digest, witness commitment, partial evaluation).
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
+
+#include <emmintrin.h>
+
+#include <atomic>
+#include <chrono>
 
 #include "fp_internal.h"
 
@@ -26,6 +32,21 @@ int fp_log2_ceil(uint64_t n) {
 // context
 // ---------------------------------------------------------------------------
 
+// True when a kernel-replaying profiler has injected itself into this process
+// (its injection libraries are mapped, or CUDA's injection hook is set).
+static bool profiler_injected() {
+    const char* inj = getenv("CUDA_INJECTION64_PATH");
+    if (inj && inj[0]) return true;
+    FILE* f = fopen("/proc/self/maps", "r");
+    if (!f) return false;
+    char line[1024];
+    bool found = false;
+    while (!found && fgets(line, sizeof line, f))
+        found = strstr(line, "InjectionTarget") || strstr(line, "TreeLauncherTarget") || strstr(line, "cuda-injection");
+    fclose(f);
+    return found;
+}
+
 fp_ctx* fp_ctx_create(int device) {
     fp_ctx* c = new fp_ctx();
     c->device = device;
@@ -42,10 +63,24 @@ fp_ctx* fp_ctx_create(int device) {
     c->host.pinned_host = true;
     c->dig_host.pinned_host = true;
     if (cudaMalloc(&c->tickets, 4096) != cudaSuccess || cudaMemset(c->tickets, 0, 4096) != cudaSuccess ||
-        cudaDeviceSynchronize() != cudaSuccess) {
+        cudaMalloc(&c->relay, sizeof(FpRelay)) != cudaSuccess ||
+        cudaMemset(c->relay, 0, sizeof(FpRelay)) != cudaSuccess ||
+        cudaHostAlloc((void**)&c->mb, sizeof(FpMailbox), cudaHostAllocMapped) != cudaSuccess ||
+        cudaHostGetDevicePointer((void**)&c->mb_dev, c->mb, 0) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        if (c->tickets) cudaFree(c->tickets);
+        if (c->relay) cudaFree(c->relay);
+        if (c->mb) cudaFreeHost(c->mb);
         delete c;
         return nullptr;
     }
+    memset((void*)c->mb, 0, sizeof(FpMailbox));
+    // A profiler that replays kernels holds the host inside the launch call, so
+    // a kernel that waits for the host's challenges could never be answered:
+    // under an injected profiler (or FP_STEPPED=1) every round is its own launch.
+    const char* st = getenv("FP_STEPPED");
+    c->stepped_env = profiler_injected() || (st && st[0] == '1');
+    c->stepped = c->stepped_env;
     return c;
 }
 
@@ -63,8 +98,106 @@ void fp_ctx_destroy(fp_ctx* c) {
     if (c->host.p) cudaFreeHost(c->host.p);
     if (c->dig_host.p) cudaFreeHost(c->dig_host.p);
     if (c->tickets) cudaFree(c->tickets);
+    if (c->relay) cudaFree(c->relay);
+    if (c->mb) cudaFreeHost(c->mb);
     delete c;
 }
+
+// ---------------------------------------------------------------------------
+// persistent-kernel handshake (host side)
+// ---------------------------------------------------------------------------
+
+uint64_t fp_seq_reserve(fp_ctx* c, uint64_t n) {
+    uint64_t base = c->seq;
+    c->seq += n;
+    return base;
+}
+
+// Reset the relay before a persistent launch and clear stale mailbox errors.
+int fp_session_begin(fp_ctx* c, cudaStream_t s) {
+    c->mb->err = 0;
+    fp_session_expect(c, 0);
+    FP_CUDA(c, cudaMemsetAsync(c->relay, 0, sizeof(FpRelay), s));
+    return FP_OK;
+}
+
+int fp_session_wait(fp_ctx* c, uint64_t seq, cudaStream_t s) {
+    (void)seq;
+    const volatile FpMailbox* mb = c->mb;
+    const int n = c->res_n;
+    using clk = std::chrono::steady_clock;
+    const auto t0 = clk::now();
+    auto next_query = t0 + std::chrono::milliseconds(2);
+    c->host_waits++;
+    for (uint64_t spin = 0;; spin++) {
+        bool full = true;
+        for (int i = 0; i < n; i++) full = full && (mb->res[i] != kEmpty);
+        if (full) {
+            std::atomic_thread_fence(std::memory_order_acquire);
+            c->host_wait_s += std::chrono::duration<double>(clk::now() - t0).count();
+            return FP_OK;
+        }
+        if ((spin & 255) != 255) continue;
+        if (mb->err) return fp_fail(c, FP_ERR_TIMEOUT, "a persistent kernel stopped waiting for the host");
+        const auto now = clk::now();
+        if (now < next_query) continue;
+        // the device may have failed: look at the stream every couple of milliseconds
+        next_query = now + std::chrono::milliseconds(2);
+        cudaError_t q = cudaStreamQuery(s);
+        if (q != cudaErrorNotReady) {
+            bool done = true;
+            for (int i = 0; i < n; i++) done = done && (mb->res[i] != kEmpty);
+            if (done) continue;
+            if (q != cudaSuccess) return fp_cuda_check(c, q, "persistent kernel");
+            return fp_fail(c, FP_ERR_TIMEOUT, "a persistent kernel ended without publishing");
+        }
+        if (std::chrono::duration<double>(now - t0).count() > 30.0)
+            return fp_fail(c, FP_ERR_TIMEOUT, "no answer from the device within 30 s");
+    }
+}
+
+// Empty the n result slots the next publish will fill (before posting the challenge that triggers it).
+void fp_session_expect(fp_ctx* c, int n) {
+    volatile FpMailbox* mb = c->mb;
+    for (int i = 0; i < 16; i++) mb->res[i] = kEmpty;
+    c->res_n = n;
+}
+
+// Waits (bounded) for a challenge that is never posted, then reports it.
+__global__ void session_selftest_kernel(FpMailbox* mb, FpRelay* rl, uint64_t seq, uint32_t limit) {
+    uint64_t chal;
+    if (session_wait(mb, rl, seq, chal, limit) && threadIdx.x == 0) session_publish(mb, &chal, 1, seq);
+}
+
+int fp_session_selftest(fp_ctx* c, void* stream) {
+    if (!c) return FP_ERR_ARG;
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t s = (cudaStream_t)stream;
+    int rc = fp_session_begin(c, s);
+    if (rc) return rc;
+    const uint64_t seq = fp_seq_reserve(c, 1) + 1;  // nobody posts this challenge
+    fp_session_expect(c, 1);
+    // 2^20 polls: about a second before the kernel gives up
+    session_selftest_kernel<<<2, 64, 0, s>>>(c->mb_dev, c->relay, seq, 1u << 20);
+    FP_CUDA(c, cudaGetLastError());
+    rc = fp_session_wait(c, seq, s);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fp_cuda_check(c, e, "session self-test");
+    c->mb->err = 0;
+    return rc;
+}
+
+// Answer with a challenge: the second value first, then {chal, seq} in one
+// aligned 16-byte store, so the device's 16-byte read sees both or neither.
+void fp_session_post2(fp_ctx* c, uint64_t seq, uint64_t chal, uint64_t chal2) {
+    volatile FpMailbox* mb = c->mb;
+    mb->chal2 = chal2;
+    std::atomic_signal_fence(std::memory_order_seq_cst);
+    _mm_store_si128((__m128i*)(&mb->chal), _mm_set_epi64x((long long)seq, (long long)chal));
+    std::atomic_thread_fence(std::memory_order_release);
+}
+
+void fp_session_post(fp_ctx* c, uint64_t seq, uint64_t chal) { fp_session_post2(c, seq, chal, 0); }
 
 const char* fp_last_error(const fp_ctx* c) { return c ? c->err.c_str() : "null context"; }
 
@@ -156,11 +289,20 @@ int fp_ctx_set_profiling(fp_ctx* c, int on) {
     if (!c) return FP_ERR_ARG;
     stats_resolve(c);
     c->profiling = on ? 1 : 0;
+    // per-kernel timing brackets each round's launch, so profiling runs stepped
+    c->stepped = c->profiling || c->stepped_env;
     for (auto& s : c->stats) s = FpKStat();
     return FP_OK;
 }
 
 int64_t fp_ctx_launches(const fp_ctx* c) { return c ? c->launches : -1; }
+
+int fp_host_stats(const fp_ctx* c, double out[2]) {
+    if (!c || !out) return FP_ERR_ARG;
+    out[0] = (double)c->host_waits;
+    out[1] = c->host_wait_s;
+    return FP_OK;
+}
 
 int fp_kernel_stats(fp_ctx* c, fp_kernel_stat* out, int cap) {
     if (!c || (cap > 0 && !out)) return FP_ERR_ARG;
@@ -328,16 +470,14 @@ int mle_partial_eval(fp_ctx* c, const void* mat, int bits, const int8_t* scales,
         if (point[i] >= 0xFFFFFFFF00000001ull) return fp_fail(c, FP_ERR_ARG, "mle_partial_eval: point not canonical");
     FP_CUDA(c, cudaSetDevice(c->device));
     cudaStream_t s = (cudaStream_t)stream;
-    int rc = fp_reserve(c, c->dev, ((size_t)8 << npoint) + fp_partial_rows_scratch(c, rows, cols) + (1 << 20));
+    FpPeJob job{mat, bits, scales, rows, cols, point, npoint, out, 1ll << fp_log2_ceil((uint64_t)cols)};
+    int rc = fp_reserve(c, c->dev, fp_partial_scratch(c, &job, 1) + (1 << 16));
+    if (rc) return rc;
+    rc = fp_reserve(c, c->host, fp_partial_host_scratch(&job, 1) + (1 << 16));
     if (rc) return rc;
     fp_reset(c->dev);
-    uint64_t* eq = (uint64_t*)fp_alloc(c->dev, (size_t)8 << npoint);
-    FpPoint z;
-    z.v = npoint;
-    for (int i = 0; i < npoint; i++) z.z[i] = point[i];
-    rc = fp_eq_table(c, z, eq, s);
-    if (rc) return rc;
-    rc = fp_partial_rows(c, mat, bits, scales, rows, cols, eq, out, 1ll << fp_log2_ceil((uint64_t)cols), s);
+    fp_reset(c->host);
+    rc = fp_partial_many(c, &job, 1, s);
     if (rc) return rc;
     FP_CUDA(c, cudaStreamSynchronize(s));
     return FP_OK;

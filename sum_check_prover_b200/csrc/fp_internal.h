@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "../../include/fp.h"
+#include "fp_session.cuh"
 #include "fp_sha256.cuh"
 
 // ---------------------------------------------------------------------------
@@ -66,9 +67,21 @@ struct fp_ctx {
     FpArena dig_host;  // pinned host staging of the digest path
     // small persistent device block: reduction tickets (kept zero between launches)
     unsigned int* tickets = nullptr;
+    // persistent-kernel handshake: mailbox in mapped pinned host memory, relay on the device
+    FpMailbox* mb = nullptr;      // host view
+    FpMailbox* mb_dev = nullptr;  // device view of the same memory
+    FpRelay* relay = nullptr;
+    uint64_t seq = 1;             // next sequence number to hand out (the empty mailbox holds 0)
+    int res_n = 0;                // result slots the next publish fills
+    // stepped: launch the sum-check kernels once per round instead of once per
+    // sum-check (under a kernel-replaying profiler, and while profiling)
+    int stepped = 0;
+    int stepped_env = 0;
     // timing
     int profiling = 0;
     int64_t launches = 0;  // every kernel launch of the library on this context
+    int64_t host_waits = 0;   // host waits for a device result (sum-check rounds)
+    double host_wait_s = 0;   // host seconds spent in those waits
     std::vector<FpEvPair> ev_live;
     std::vector<cudaEvent_t> ev_free;
     FpKStat stats[K_COUNT];
@@ -98,6 +111,17 @@ void fp_tic(fp_ctx* c, cudaStream_t s, int kernel, double bytes, int* slot);
 void fp_toc(fp_ctx* c, cudaStream_t s, int slot);
 void fp_stats_reset(fp_ctx* c);
 
+// persistent-kernel handshake (api.cu). seq_reserve hands out n consecutive
+// sequence numbers and returns the base; wait blocks until the device published
+// seq (bounded: FP_ERR_TIMEOUT, FP_ERR_CUDA if the kernel died); post answers
+// with a challenge.
+uint64_t fp_seq_reserve(fp_ctx* c, uint64_t n);
+int fp_session_wait(fp_ctx* c, uint64_t seq, cudaStream_t s);
+void fp_session_post(fp_ctx* c, uint64_t seq, uint64_t chal);
+void fp_session_expect(fp_ctx* c, int n);
+void fp_session_post2(fp_ctx* c, uint64_t seq, uint64_t chal, uint64_t chal2);
+int fp_session_begin(fp_ctx* c, cudaStream_t s);
+
 // transcript (transcript.cu)
 void fp_tx_absorb_raw(fp_tx* t, const char* label, const void* data, uint64_t n);
 uint64_t fp_tx_squeeze_one(fp_tx* t, const char* label);
@@ -123,10 +147,22 @@ struct FpPoint {
 };
 int fp_eq_table(fp_ctx* c, const FpPoint& z, uint64_t* out, cudaStream_t s);
 // out[c] = sum_{i<rows} eq[i] M_eff[i][c]; eq device (rows entries); out device (cols_pad)
-// out has out_len >= cols entries; entries past cols are zeroed
-int fp_partial_rows(fp_ctx* c, const void* mat, int bits, const int8_t* scales, int rows, int cols,
-                    const uint64_t* eq, uint64_t* out, int64_t out_len, cudaStream_t s);
-size_t fp_partial_rows_scratch(const fp_ctx* c, int rows, int cols);
+// Row contractions out[c] = sum_{i<rows} eq(z, i) M_eff[i][c], many per launch
+// (partial.cu). z is host memory (v = ceil(log2 rows) coordinates); out is
+// device memory with out_len >= cols entries, the ones past cols zeroed.
+struct FpPeJob {
+    const void* mat;
+    int bits;
+    const int8_t* scales;
+    int rows, cols;
+    const uint64_t* z;
+    int v;
+    uint64_t* out;
+    int64_t out_len;
+};
+size_t fp_partial_scratch(const fp_ctx* c, const FpPeJob* jobs, int njobs);
+size_t fp_partial_host_scratch(const FpPeJob* jobs, int njobs);
+int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s);
 size_t fp_claims_scratch(const fp_site* sites, int nsites);
 // per-site output claims into dev_out[s]
 int fp_claims(fp_ctx* c, const fp_site* sites, int nsites, const uint64_t* const* eq_rows,

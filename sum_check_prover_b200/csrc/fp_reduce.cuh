@@ -27,10 +27,12 @@ __device__ __forceinline__ void block_sum_gl(uint64_t (&v)[NV]) {
     }
 }
 
-// Every block contributes v; returns true in the last block, whose warp 0 then
-// holds the grid totals in v. part needs NV * gridDim.x entries.
+// The first `nblocks` blocks contribute v; returns true in the last of them to
+// finish, whose warp 0 then holds the totals in v. part needs NV * nblocks
+// entries; *ticket must be zero on entry and is zero again on return.
 template <int NV>
-__device__ __forceinline__ bool grid_sum_gl(uint64_t (&v)[NV], uint64_t* part, unsigned int* ticket) {
+__device__ __forceinline__ bool grid_sum_gl_n(uint64_t (&v)[NV], uint64_t* part, unsigned int* ticket,
+                                              unsigned int nblocks) {
     __shared__ bool am_last;
     block_sum_gl<NV>(v);
     if (threadIdx.x == 0) {
@@ -38,7 +40,7 @@ __device__ __forceinline__ bool grid_sum_gl(uint64_t (&v)[NV], uint64_t* part, u
         for (int k = 0; k < NV; k++) part[(size_t)blockIdx.x * NV + k] = v[k];
         __threadfence();
         unsigned int t = atomicAdd(ticket, 1u);
-        am_last = (t == gridDim.x - 1);
+        am_last = (t == nblocks - 1);
     }
     __syncthreads();
     if (!am_last) return false;
@@ -46,7 +48,7 @@ __device__ __forceinline__ bool grid_sum_gl(uint64_t (&v)[NV], uint64_t* part, u
     uint64_t acc[NV];
 #pragma unroll
     for (int k = 0; k < NV; k++) acc[k] = 0;
-    for (unsigned b = threadIdx.x; b < gridDim.x; b += blockDim.x)
+    for (unsigned b = threadIdx.x; b < nblocks; b += blockDim.x)
 #pragma unroll
         for (int k = 0; k < NV; k++) acc[k] = gl_add(acc[k], __ldcg(part + (size_t)b * NV + k));
     block_sum_gl<NV>(acc);
@@ -54,4 +56,10 @@ __device__ __forceinline__ bool grid_sum_gl(uint64_t (&v)[NV], uint64_t* part, u
     for (int k = 0; k < NV; k++) v[k] = acc[k];
     if (threadIdx.x == 0) *ticket = 0u;
     return true;
+}
+
+// Every block of the grid contributes v (see grid_sum_gl_n).
+template <int NV>
+__device__ __forceinline__ bool grid_sum_gl(uint64_t (&v)[NV], uint64_t* part, unsigned int* ticket) {
+    return grid_sum_gl_n<NV>(v, part, ticket, gridDim.x);
 }

@@ -77,6 +77,10 @@ __host__ __device__ __forceinline__ void fp_sha_init(uint32_t h[8]) {
     for (int i = 0; i < 8; i++) h[i] = h0[i];
 }
 
+// Host compression of n 64-byte blocks; uses the CPU's SHA extensions when it
+// has them (defined in transcript.cu).
+void fp_sha256_host_blocks(uint32_t h[8], const uint8_t* p, size_t n);
+
 // Host-side incremental hasher (transcript and small host digests).
 struct FpSha256 {
     uint32_t h[8];
@@ -86,13 +90,7 @@ struct FpSha256 {
 
     FpSha256() { fp_sha_init(h); }
 
-    void block(const uint8_t* p) {
-        uint32_t m[16];
-        for (int i = 0; i < 16; i++)
-            m[i] = ((uint32_t)p[4 * i] << 24) | ((uint32_t)p[4 * i + 1] << 16) | ((uint32_t)p[4 * i + 2] << 8) |
-                   (uint32_t)p[4 * i + 3];
-        fp_sha_compress(h, m);
-    }
+    void block(const uint8_t* p) { fp_sha256_host_blocks(h, p, 1); }
 
     void update(const void* data, uint64_t n) {
         const uint8_t* p = (const uint8_t*)data;
@@ -109,10 +107,11 @@ struct FpSha256 {
                 fill = 0;
             }
         }
-        while (n >= 64) {
-            block(p);
-            p += 64;
-            n -= 64;
+        if (n >= 64) {
+            const size_t nb = n / 64;
+            fp_sha256_host_blocks(h, p, nb);
+            p += 64 * nb;
+            n -= 64 * nb;
         }
         if (n) {
             memcpy(buf, p, n);

@@ -21,10 +21,12 @@
 // table is kept in place too (E_t[b] = E_(t-1)[b] + E_(t-1)[b + h]).
 #include <string.h>
 
+#include <algorithm>
 #include <vector>
 
 #include "fp_internal.h"
 #include "fp_reduce.cuh"
+#include "fp_session.cuh"
 
 namespace {
 
@@ -144,27 +146,67 @@ struct TreeLayer {
     uint64_t* Q[2];
 };
 
-// layer v-1 from the leaves: p = qL + qR (leaf numerators are 1), q = qL qR
-__global__ void tree_leaf_kernel(KeySrc K, Chal C, TreeLayer out, int64_t n) {
-    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
-        uint64_t l0, l1, r0, r1;
-        leaf_den(K, C, 2 * x, l0, l1);
-        leaf_den(K, C, 2 * x + 1, r0, r1);
-        out.P[0][x] = gl_add(l0, r0);
-        out.Q[0][x] = gl_mul(l0, r0);
-        out.P[1][x] = gl_add(l1, r1);
-        out.Q[1][x] = gl_mul(l1, r1);
-    }
-}
+// Up to kTreeLevels layers per launch. Block b takes 2^levels consecutive
+// nodes of layer L0 (the leaves when KEYS, else a stored layer) and builds its
+// subtree down to one node of layer L0 - levels in shared memory, writing
+// every layer it passes to global memory. Parent of children 2x, 2x+1:
+// (pL qR + pR qL, qL qR); at the leaves p = 1, so the first level is (qL + qR, qL qR).
+constexpr int kTreeLevels = 10;
 
-__global__ void tree_up_kernel(TreeLayer in, TreeLayer out, int64_t n) {
-    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
+struct TreeOut {
+    TreeLayer lay[kTreeLevels];  // lay[l]: layer L0 - 1 - l
+};
+
+template <bool KEYS>
+__global__ void __launch_bounds__(512) tree_chunk_kernel(KeySrc K, Chal C, TreeLayer in, TreeOut out, int levels) {
+    extern __shared__ uint64_t sm[];  // [2 buffers][4 values: P0 Q0 P1 Q1][n1]
+    const int n1 = 1 << (levels - 1);
+    uint64_t* buf[2] = {sm, sm + 4 * n1};
+    for (int x = threadIdx.x; x < n1; x += blockDim.x) {
+        const int64_t gx = (int64_t)blockIdx.x * n1 + x;
+        uint64_t P[2], Q[2];
+        if (KEYS) {
+            uint64_t l0, l1, r0, r1;
+            leaf_den(K, C, 2 * gx, l0, l1);
+            leaf_den(K, C, 2 * gx + 1, r0, r1);
+            P[0] = gl_add(l0, r0);
+            Q[0] = gl_mul(l0, r0);
+            P[1] = gl_add(l1, r1);
+            Q[1] = gl_mul(l1, r1);
+        } else {
+#pragma unroll
+            for (int tau = 0; tau < 2; tau++) {
+                const ulonglong2 p = reinterpret_cast<const ulonglong2*>(in.P[tau])[gx];
+                const ulonglong2 q = reinterpret_cast<const ulonglong2*>(in.Q[tau])[gx];
+                P[tau] = gl_add(gl_mul(p.x, q.y), gl_mul(p.y, q.x));
+                Q[tau] = gl_mul(q.x, q.y);
+            }
+        }
 #pragma unroll
         for (int tau = 0; tau < 2; tau++) {
-            const ulonglong2 p = reinterpret_cast<const ulonglong2*>(in.P[tau])[x];
-            const ulonglong2 q = reinterpret_cast<const ulonglong2*>(in.Q[tau])[x];
-            out.P[tau][x] = gl_add(gl_mul(p.x, q.y), gl_mul(p.y, q.x));
-            out.Q[tau][x] = gl_mul(q.x, q.y);
+            out.lay[0].P[tau][gx] = P[tau];
+            out.lay[0].Q[tau][gx] = Q[tau];
+            buf[0][(2 * tau) * n1 + x] = P[tau];
+            buf[0][(2 * tau + 1) * n1 + x] = Q[tau];
+        }
+    }
+    for (int l = 1; l < levels; l++) {
+        __syncthreads();
+        const int nl = n1 >> l;
+        const uint64_t* src = buf[(l - 1) & 1];
+        uint64_t* dst = buf[l & 1];
+        for (int x = threadIdx.x; x < nl; x += blockDim.x) {
+            const int64_t gx = (int64_t)blockIdx.x * nl + x;
+#pragma unroll
+            for (int tau = 0; tau < 2; tau++) {
+                const uint64_t pl = src[(2 * tau) * n1 + 2 * x], pr = src[(2 * tau) * n1 + 2 * x + 1];
+                const uint64_t ql = src[(2 * tau + 1) * n1 + 2 * x], qr = src[(2 * tau + 1) * n1 + 2 * x + 1];
+                const uint64_t P = gl_add(gl_mul(pl, qr), gl_mul(pr, ql)), Q = gl_mul(ql, qr);
+                out.lay[l].P[tau][gx] = P;
+                out.lay[l].Q[tau][gx] = Q;
+                dst[(2 * tau) * n1 + x] = P;
+                dst[(2 * tau + 1) * n1 + x] = Q;
+            }
         }
     }
 }
@@ -187,25 +229,33 @@ __global__ void l1_from_layer_kernel(TreeLayer one, uint64_t* out) {
     }
 }
 
-// ---- layer sum-check rounds ----------------------------------------------------
+// ---- layer sum-check: one persistent kernel per layer ---------------------------------
 
-struct GkrArgs {
-    // pair vectors (x: left child, y: right child); LEAF layers have no p vectors
+struct GkrLayer {
+    // pair vectors (x: left child, y: right child), folded in place; the leaf
+    // layer has no p vectors (all ones) and folds its q pairs into a buffer
     ulonglong2* pp[2];
     ulonglong2* qq[2];
-    const ulonglong2* src_pp[2];  // round 1 / round 2 source when not from keys
-    const ulonglong2* src_qq[2];
-    uint64_t* E;
-    uint64_t* state;  // [0] = eq(z_<t, rho_<t)
+    uint64_t* E;       // suffix eq table, kept in place
     KeySrc keys;
     Chal chal;
-    FpPoint z;        // the layer's point (d coordinates)
-    int d, t;
-    int64_t h;        // pairs this round: 2^(d - t)
-    uint64_t rprev, lam;
+    // Challenge points by layer parity: layer d reads its point from zin
+    // (z_1..z_(d-1) = the previous layer's round challenges, z_d = mu written
+    // by this layer's first launch) and writes its own round challenges to
+    // zout, which is the next layer's zin. lam[0] keeps lambda for later launches.
+    uint64_t* zin;
+    uint64_t* zout;
+    uint64_t* lam;
+    int d;
+    int threads;       // threads per block (<= LU_THREADS)
+    int grid;          // blocks launched (all co-resident)
+    int per_block;     // pairs one block covers in a round
+    uint64_t seq0;     // {mu, lambda} arrive as challenge seq0; round t publishes seq0 + t
+    int t_begin;       // rounds run by this launch: [t_begin, t_end]; t_end > d includes
+    int t_end;         // the final values (one launch per layer, or one per round)
 };
 
-// F(X) of one pair position for the two tables
+// F at one pair position for both tables: sum_tau lambda^(2 tau) (pL qR + pR qL + lambda qL qR)
 template <bool LEAF>
 __device__ __forceinline__ uint64_t layer_F(const uint64_t (&pl)[2], const uint64_t (&pr)[2], const uint64_t (&ql)[2],
                                             const uint64_t (&qr)[2], uint64_t lam, uint64_t lam2) {
@@ -219,22 +269,22 @@ __device__ __forceinline__ uint64_t layer_F(const uint64_t (&pl)[2], const uint6
     return gl_add(f[0], gl_mul(lam2, f[1]));
 }
 
-// Source pair at position x of the layer's initial vectors.
-template <bool KEYS>
-__device__ __forceinline__ void src_pair(const GkrArgs& A, int64_t x, ulonglong2 (&pp)[2], ulonglong2 (&qq)[2]) {
-    if (KEYS) {
+// pair x of the layer's current vectors: from the key columns, or from pp/qq
+template <bool LEAF>
+__device__ __forceinline__ void layer_pair(const GkrLayer& A, bool from_keys, int64_t x, ulonglong2 (&pp)[2],
+                                           ulonglong2 (&qq)[2]) {
+    if (LEAF && from_keys) {
         uint64_t l0, l1, r0, r1;
         leaf_den(A.keys, A.chal, 2 * x, l0, l1);
         leaf_den(A.keys, A.chal, 2 * x + 1, r0, r1);
-        pp[0] = make_ulonglong2(1, 1);
-        pp[1] = make_ulonglong2(1, 1);
         qq[0] = make_ulonglong2(l0, r0);
         qq[1] = make_ulonglong2(l1, r1);
+        pp[0] = pp[1] = make_ulonglong2(1, 1);
     } else {
 #pragma unroll
         for (int tau = 0; tau < 2; tau++) {
-            pp[tau] = A.src_pp[tau][x];
-            qq[tau] = A.src_qq[tau][x];
+            pp[tau] = LEAF ? make_ulonglong2(1, 1) : __ldcg(A.pp[tau] + x);
+            qq[tau] = __ldcg(A.qq[tau] + x);
         }
     }
 }
@@ -243,68 +293,48 @@ __device__ __forceinline__ ulonglong2 fold2(ulonglong2 a, ulonglong2 b, uint64_t
     return make_ulonglong2(gl_fold(a.x, b.x, r), gl_fold(a.y, b.y, r));
 }
 
-// MODE 0: round 1 (no fold). MODE 1: fold from the source (round 2).
-// MODE 2: fold in place in pp/qq (round >= 3). KEYS: the source is the key columns.
-template <bool LEAF, bool KEYS, int MODE>
-__global__ void __launch_bounds__(LU_THREADS) gkr_round_kernel(GkrArgs A, uint64_t* part, unsigned int* ticket,
-                                                               uint64_t* __restrict__ gout) {
-    uint64_t acc[3] = {0, 0, 0};
-    const int64_t h = A.h;
-    const uint64_t lam2 = gl_mul(A.lam, A.lam);
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)gridDim.x * blockDim.x) {
-        ulonglong2 c0p[2], c0q[2], c1p[2], c1q[2];  // current pairs at b and b + h
+// Round t of layer d over the pairs b < h handled by this block.
+// t == 1: the vectors as they are. t >= 2: fold the previous round's vectors
+// (length 4h) by rprev first and store the folded halves in place.
+template <bool LEAF>
+__device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* zs, int t, int64_t h, unsigned active,
+                                            uint64_t rprev, uint64_t lam, uint64_t lam2, uint64_t (&acc)[3]) {
+    const bool from_keys = LEAF && t <= 2;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
+        ulonglong2 c0p[2], c0q[2], c1p[2], c1q[2];
         uint64_t e;
-        if (MODE == 0) {
-            src_pair<KEYS>(A, b, c0p, c0q);
-            src_pair<KEYS>(A, b + h, c1p, c1q);
+        if (t == 1) {
+            layer_pair<LEAF>(A, from_keys, b, c0p, c0q);
+            layer_pair<LEAF>(A, from_keys, b + h, c1p, c1q);
             // E_1[b] = eq(z_2..z_d, b)
             e = 1;
             const int nb = A.d - 1;
-            for (int i = 0; i < nb; i++) e = gl_mul(e, gl_eq1(A.z.z[1 + i], (int)((b >> (nb - 1 - i)) & 1)));
+            for (int i = 0; i < nb; i++) e = gl_mul(e, gl_eq1(zs[1 + i], (int)((b >> (nb - 1 - i)) & 1)));
             if (A.d > 1) A.E[b] = e;
         } else {
             ulonglong2 s0p[2], s0q[2], s1p[2], s1q[2], s2p[2], s2q[2], s3p[2], s3q[2];
-            if (MODE == 1) {
-                src_pair<KEYS>(A, b, s0p, s0q);
-                src_pair<KEYS>(A, b + h, s1p, s1q);
-                src_pair<KEYS>(A, b + 2 * h, s2p, s2q);
-                src_pair<KEYS>(A, b + 3 * h, s3p, s3q);
-            } else {
-#pragma unroll
-                for (int tau = 0; tau < 2; tau++) {
-                    if (!LEAF) {
-                        s0p[tau] = A.pp[tau][b];
-                        s1p[tau] = A.pp[tau][b + h];
-                        s2p[tau] = A.pp[tau][b + 2 * h];
-                        s3p[tau] = A.pp[tau][b + 3 * h];
-                    } else {
-                        s0p[tau] = s1p[tau] = s2p[tau] = s3p[tau] = make_ulonglong2(1, 1);
-                    }
-                    s0q[tau] = A.qq[tau][b];
-                    s1q[tau] = A.qq[tau][b + h];
-                    s2q[tau] = A.qq[tau][b + 2 * h];
-                    s3q[tau] = A.qq[tau][b + 3 * h];
-                }
-            }
+            layer_pair<LEAF>(A, from_keys, b, s0p, s0q);
+            layer_pair<LEAF>(A, from_keys, b + h, s1p, s1q);
+            layer_pair<LEAF>(A, from_keys, b + 2 * h, s2p, s2q);
+            layer_pair<LEAF>(A, from_keys, b + 3 * h, s3p, s3q);
 #pragma unroll
             for (int tau = 0; tau < 2; tau++) {
                 if (LEAF) {
                     c0p[tau] = c1p[tau] = make_ulonglong2(1, 1);
                 } else {
-                    c0p[tau] = fold2(s0p[tau], s2p[tau], A.rprev);
-                    c1p[tau] = fold2(s1p[tau], s3p[tau], A.rprev);
+                    c0p[tau] = fold2(s0p[tau], s2p[tau], rprev);
+                    c1p[tau] = fold2(s1p[tau], s3p[tau], rprev);
                     A.pp[tau][b] = c0p[tau];
                     A.pp[tau][b + h] = c1p[tau];
                 }
-                c0q[tau] = fold2(s0q[tau], s2q[tau], A.rprev);
-                c1q[tau] = fold2(s1q[tau], s3q[tau], A.rprev);
+                c0q[tau] = fold2(s0q[tau], s2q[tau], rprev);
+                c1q[tau] = fold2(s1q[tau], s3q[tau], rprev);
                 A.qq[tau][b] = c0q[tau];
                 A.qq[tau][b + h] = c1q[tau];
             }
-            e = gl_add(A.E[b], A.E[b + h]);
+            e = gl_add(__ldcg(A.E + b), __ldcg(A.E + b + h));
             A.E[b] = e;
         }
-        // h(X) at X = 0, 1, 2
         uint64_t pl[2], pr[2], ql[2], qr[2];
 #pragma unroll
         for (int X = 0; X < 3; X++) {
@@ -321,53 +351,93 @@ __global__ void __launch_bounds__(LU_THREADS) gkr_round_kernel(GkrArgs A, uint64
                     qr[tau] = gl_sub(gl_add(c1q[tau].y, c1q[tau].y), c0q[tau].y);
                 }
             }
-            acc[X] = gl_add(acc[X], gl_mul(e, layer_F<LEAF>(pl, pr, ql, qr, A.lam, lam2)));
-        }
-    }
-    if (grid_sum_gl<3>(acc, part, ticket) && threadIdx.x == 0) {
-        // prefix eq(z_<t, rho_<t), updated with the previous round's challenge
-        uint64_t pre = 1;
-        if (A.t > 1) {
-            const uint64_t zp = A.z.z[A.t - 2];
-            pre = gl_mul(A.state[0], gl_add(gl_mul(zp, A.rprev), gl_mul(gl_sub(1, zp), gl_sub(1, A.rprev))));
-        }
-        A.state[0] = pre;
-        const uint64_t zt = A.z.z[A.t - 1];
-        // h(3) from the third finite difference of a quadratic
-        const uint64_t h3 = gl_add(gl_sub(gl_mul(3, acc[2]), gl_mul(3, acc[1])), acc[0]);
-        const uint64_t hv[4] = {acc[0], acc[1], acc[2], h3};
-        const uint64_t one_m = gl_sub(1, zt), slope = gl_sub(gl_add(zt, zt), 1);  // eq(z_t, X) = (1 - z_t) + X (2 z_t - 1)
-#pragma unroll
-        for (int X = 0; X < 4; X++) {
-            const uint64_t ex = gl_add(one_m, gl_mul((uint64_t)X, slope));
-            gout[X] = gl_mul(pre, gl_mul(ex, hv[X]));
+            acc[X] = gl_add(acc[X], gl_mul(e, layer_F<LEAF>(pl, pr, ql, qr, lam, lam2)));
         }
     }
 }
 
-// The eight child values at the layer's last challenge.
-template <bool LEAF, bool KEYS>
-__global__ void gkr_final_kernel(GkrArgs A, uint64_t rlast, uint64_t* out) {
-    if (threadIdx.x != 0) return;
-    ulonglong2 p0[2], q0[2], p1[2], q1[2];
-    if (KEYS) {
-        src_pair<true>(A, 0, p0, q0);
-        src_pair<true>(A, 1, p1, q1);
-    } else {
-#pragma unroll
-        for (int tau = 0; tau < 2; tau++) {
-            p0[tau] = LEAF ? make_ulonglong2(1, 1) : A.pp[tau][0];
-            p1[tau] = LEAF ? make_ulonglong2(1, 1) : A.pp[tau][1];
-            q0[tau] = A.qq[tau][0];
-            q1[tau] = A.qq[tau][1];
+// Rounds [t_begin, t_end] of one layer (t_end > d: and its final child values).
+template <bool LEAF>
+__global__ void __launch_bounds__(LU_THREADS) gkr_layer_kernel(GkrLayer A, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
+    __shared__ uint64_t zs[32];
+    __shared__ uint64_t s_lam;
+    const int d = A.d;
+    if (A.t_begin == 1) {
+        // the layer's own challenges: mu (last point coordinate) and lambda
+        uint64_t mu, lam;
+        if (!session_wait2(mb, rl, A.seq0, mu, lam)) return;
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < d - 1; i++) zs[i] = __ldcg(A.zin + i);
+            zs[d - 1] = mu;
+            s_lam = lam;
+            if (blockIdx.x == 0) {
+                A.zin[d - 1] = mu;
+                A.lam[0] = lam;
+            }
+        }
+    } else if (threadIdx.x == 0) {
+        for (int i = 0; i < d; i++) zs[i] = __ldcg(A.zin + i);
+        s_lam = __ldcg(A.lam);
+    }
+    __syncthreads();
+    const uint64_t lam = s_lam, lam2 = gl_mul(lam, lam);
+    // eq(z_<t, rho_<t) of the rounds before this launch (their challenges are in zout)
+    uint64_t pre = 1, rprev = 0;
+    for (int i = 1; i + 1 < A.t_begin && i <= d; i++) {
+        const uint64_t r = __ldcg(A.zout + i - 1);
+        pre = gl_mul(pre, gl_add(gl_mul(zs[i - 1], r), gl_mul(gl_sub(1, zs[i - 1]), gl_sub(1, r))));
+    }
+    for (int t = A.t_begin; t <= d && t <= A.t_end; t++) {
+        if (t > 1) {
+            if (!session_wait(mb, rl, A.seq0 + t - 1, rprev)) return;
+            const uint64_t zp = zs[t - 2];
+            pre = gl_mul(pre, gl_add(gl_mul(zp, rprev), gl_mul(gl_sub(1, zp), gl_sub(1, rprev))));
+            if (blockIdx.x == 0 && threadIdx.x == 0) A.zout[t - 2] = rprev;
+        }
+        const int64_t h = 1ll << (d - t);
+        int64_t want = (h + A.per_block - 1) / A.per_block;
+        const unsigned active = (unsigned)(want < 1 ? 1 : (want > A.grid ? A.grid : want));
+        if (blockIdx.x >= active) return;  // this block has no pairs in this or any later round
+        uint64_t acc[3] = {0, 0, 0};
+        layer_round<LEAF>(A, zs, t, h, active, rprev, lam, lam2, acc);
+        bool last;
+        if (active == 1) {
+            block_sum_gl<3>(acc);
+            last = true;
+        } else {
+            last = grid_sum_gl_n<3>(acc, part, &rl->ticket, active);
+        }
+        if (last && threadIdx.x == 0) {
+            // g(X) = eq(z_<t, rho_<t) eq(z_t, X) h(X); h has degree 2, h(3) by finite differences
+            const uint64_t zt = zs[t - 1];
+            const uint64_t one_m = gl_sub(1, zt), slope = gl_sub(gl_add(zt, zt), 1);
+            const uint64_t e2 = gl_add(one_m, gl_add(slope, slope)), e3 = gl_add(e2, slope);
+            const uint64_t h3 = gl_add(gl_sub(gl_add(gl_add(acc[2], acc[2]), acc[2]), gl_add(gl_add(acc[1], acc[1]), acc[1])), acc[0]);
+            uint64_t g[4];
+            g[0] = gl_mul(pre, gl_mul(one_m, acc[0]));
+            g[1] = gl_mul(pre, gl_mul(zt, acc[1]));
+            g[2] = gl_mul(pre, gl_mul(e2, acc[2]));
+            g[3] = gl_mul(pre, gl_mul(e3, h3));
+            session_publish(mb, g, 4, A.seq0 + t);
         }
     }
+    // only block 0 is left: fold the last pair by the last challenge
+    if (A.t_end <= d || blockIdx.x != 0) return;
+    if (!session_wait(mb, rl, A.seq0 + d, rprev)) return;
+    if (threadIdx.x == 0) {
+        A.zout[d - 1] = rprev;
+        ulonglong2 p0[2], q0[2], p1[2], q1[2];
+        layer_pair<LEAF>(A, LEAF && d == 1, 0, p0, q0);
+        layer_pair<LEAF>(A, LEAF && d == 1, 1, p1, q1);
+        uint64_t out[8];
 #pragma unroll
-    for (int tau = 0; tau < 2; tau++) {
-        out[4 * tau + 0] = gl_fold(p0[tau].x, p1[tau].x, rlast);
-        out[4 * tau + 1] = gl_fold(p0[tau].y, p1[tau].y, rlast);
-        out[4 * tau + 2] = gl_fold(q0[tau].x, q1[tau].x, rlast);
-        out[4 * tau + 3] = gl_fold(q0[tau].y, q1[tau].y, rlast);
+        for (int tau = 0; tau < 2; tau++) {
+            out[4 * tau + 0] = gl_fold(p0[tau].x, p1[tau].x, rprev);
+            out[4 * tau + 1] = gl_fold(p0[tau].y, p1[tau].y, rprev);
+            out[4 * tau + 2] = gl_fold(q0[tau].x, q1[tau].x, rprev);
+            out[4 * tau + 3] = gl_fold(q0[tau].y, q1[tau].y, rprev);
+        }
+        session_publish(mb, out, 8, A.seq0 + d + 1);
     }
 }
 
@@ -444,7 +514,7 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
     need += fp_align_up((size_t)8 << (v >= 2 ? v - 2 : 0), 256);              // suffix eq table
     const int lo_bits = v / 2;
     need += fp_align_up((size_t)8 << lo_bits, 256) + fp_align_up((size_t)8 << (v - lo_bits), 256);
-    need += fp_align_up((size_t)8 * 3 * 8 * c->num_sms, 256) + 4096;
+    need += fp_align_up((size_t)8 * 3 * 16 * c->num_sms, 256) + 3 * 512 + 8192;
     if ((rc = fp_reserve(c, c->dev, need + (1 << 20)))) return rc;
     if ((rc = fp_reserve(c, c->host, 4 * (size_t)T + 4 * 65536 + 4096 + sizeof(GatherSite) * nsites))) return rc;
     fp_reset(c->dev);
@@ -535,24 +605,37 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
     if (v >= 2)
         for (int tau = 0; tau < 2; tau++) leafq[tau] = (ulonglong2*)fp_alloc(c->dev, (size_t)16 << (v - 2));
     uint64_t* E = (uint64_t*)fp_alloc(c->dev, (size_t)8 << (v >= 2 ? v - 2 : 0));
-    uint64_t* part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * 3 * 8 * c->num_sms);
-    uint64_t* small = (uint64_t*)fp_alloc(c->dev, 256);  // [0..8) outputs, [16] state
+    uint64_t* part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * 3 * 16 * c->num_sms);
+    uint64_t* small = (uint64_t*)fp_alloc(c->dev, 256);  // [0..8) outputs
+    uint64_t* zb[3] = {(uint64_t*)fp_alloc(c->dev, 8 * 64), (uint64_t*)fp_alloc(c->dev, 8 * 64),
+                       (uint64_t*)fp_alloc(c->dev, 8 * 64)};
     uint64_t* hsmall = (uint64_t*)fp_alloc(c->host, 256);
-    if (!part || !small || !hsmall || !E) return fp_fail(c, FP_ERR_OOM, "logup: scratch exhausted");
+    if (!part || !small || !hsmall || !E || !zb[2]) return fp_fail(c, FP_ERR_OOM, "logup: scratch exhausted");
 
     if (v >= 2) {
-        int slot;
-        const int64_t n = L / 2;
-        fp_tic(c, st, K_TREE_LEAF, 9.0 * L + 32.0 * n, &slot);
-        tree_leaf_kernel<<<grid_for(c, n, 256), 256, 0, st>>>(K, C, lay[v - 1], n);
-        fp_toc(c, st, slot);
-        FP_CUDA(c, cudaGetLastError());
-        for (int d = v - 2; d >= 1; d--) {
-            const int64_t nn = 1ll << d;
-            fp_tic(c, st, K_TREE_UP, 64.0 * nn + 32.0 * nn, &slot);
-            tree_up_kernel<<<grid_for(c, nn, 256), 256, 0, st>>>(lay[d + 1], lay[d], nn);
+        // layers v-1 .. 1, kTreeLevels per launch
+        int L0 = v;
+        while (L0 > 1) {
+            const int levels = std::min(kTreeLevels, L0 - 1);
+            TreeOut to;
+            memset(&to, 0, sizeof to);
+            for (int l = 0; l < levels; l++) to.lay[l] = lay[L0 - 1 - l];
+            const unsigned blocks = 1u << (L0 - levels);
+            const int n1 = 1 << (levels - 1);
+            const int threads = std::min(512, n1);
+            const size_t smem = (size_t)8 * 8 * n1;
+            const double nodes = (double)(1ll << (L0 - 1)) * 2.0;
+            int slot;
+            if (L0 == v) {
+                fp_tic(c, st, K_TREE_LEAF, 9.0 * (double)(1ll << L0) + 32.0 * nodes, &slot);
+                tree_chunk_kernel<true><<<blocks, threads, smem, st>>>(K, C, lay[L0 - 1], to, levels);
+            } else {
+                fp_tic(c, st, K_TREE_UP, 32.0 * (double)(1ll << L0) + 32.0 * nodes, &slot);
+                tree_chunk_kernel<false><<<blocks, threads, smem, st>>>(K, C, lay[L0], to, levels);
+            }
             fp_toc(c, st, slot);
             FP_CUDA(c, cudaGetLastError());
+            L0 -= levels;
         }
         int s2;
         fp_tic(c, st, K_REDUCE, 64.0, &s2);
@@ -574,10 +657,14 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
     z.v = 1;
     z.z[0] = fp_tx_squeeze_one(tx, "gkr_mu");
 
-    // ---- layer sum-checks ----
+    // ---- layer sum-checks: one resident kernel per layer, all queued up front ----
+    int occ[2] = {0, 0};
+    FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[0], gkr_layer_kernel<false>, LU_THREADS, 0));
+    FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[1], gkr_layer_kernel<true>, LU_THREADS, 0));
+    std::vector<GkrLayer> layers(v > 1 ? v - 1 : 0);
     for (int d = 1; d <= v - 1; d++) {
         const bool leaf = (d == v - 1);
-        GkrArgs A;
+        GkrLayer& A = layers[d - 1];
         memset(&A, 0, sizeof A);
         for (int tau = 0; tau < 2; tau++) {
             if (leaf) {
@@ -587,65 +674,84 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
                 A.pp[tau] = reinterpret_cast<ulonglong2*>(lay[d + 1].P[tau]);
                 A.qq[tau] = reinterpret_cast<ulonglong2*>(lay[d + 1].Q[tau]);
             }
-            A.src_pp[tau] = A.pp[tau];
-            A.src_qq[tau] = A.qq[tau];
         }
         A.E = E;
-        A.state = small + 16;
         A.keys = K;
         A.chal = C;
-        A.z = z;
+        A.zin = zb[d & 1];
+        A.zout = zb[(d + 1) & 1];
+        A.lam = zb[2];
         A.d = d;
-        A.lam = fp_tx_squeeze_one(tx, "gkr_lambda");
-        std::vector<uint64_t> rho(d);
-        uint64_t rprev = 0;
-        for (int t = 1; t <= d; t++) {
-            A.t = t;
-            A.h = 1ll << (d - t);
-            A.rprev = rprev;
-            const int mode = t == 1 ? 0 : (t == 2 ? 1 : 2);
-            const int blocks = grid_for(c, A.h, LU_THREADS);
-            double bytes = (leaf ? 36.0 : 128.0) * A.h * (mode == 0 ? 1 : 2) + (mode ? 24.0 * A.h : 8.0 * A.h);
-            int slot;
-            fp_tic(c, st, K_GKR_ROUND, bytes, &slot);
-            if (leaf) {
-                if (mode == 0) gkr_round_kernel<true, true, 0><<<blocks, LU_THREADS, 0, st>>>(A, part, c->tickets, small);
-                else if (mode == 1) gkr_round_kernel<true, true, 1><<<blocks, LU_THREADS, 0, st>>>(A, part, c->tickets, small);
-                else gkr_round_kernel<true, false, 2><<<blocks, LU_THREADS, 0, st>>>(A, part, c->tickets, small);
-            } else {
-                if (mode == 0) gkr_round_kernel<false, false, 0><<<blocks, LU_THREADS, 0, st>>>(A, part, c->tickets, small);
-                else if (mode == 1) gkr_round_kernel<false, false, 1><<<blocks, LU_THREADS, 0, st>>>(A, part, c->tickets, small);
-                else gkr_round_kernel<false, false, 2><<<blocks, LU_THREADS, 0, st>>>(A, part, c->tickets, small);
-            }
-            fp_toc(c, st, slot);
-            FP_CUDA(c, cudaGetLastError());
-            FP_CUDA(c, cudaMemcpyAsync(hsmall, small, 32, cudaMemcpyDeviceToHost, st));
-            FP_CUDA(c, cudaStreamSynchronize(st));
-            for (int i = 0; i < 4; i++) put_le(proof + pos + 8 * i, hsmall[i], 8);
-            fp_tx_absorb_raw(tx, "gkr_round", proof + pos, 32);
-            pos += 32;
-            rprev = rho[t - 1] = fp_tx_squeeze_one(tx, "gkr_chal");
-        }
-        int slot;
-        fp_tic(c, st, K_GKR_FINAL, 128.0, &slot);
-        if (leaf) {
-            if (d == 1) gkr_final_kernel<true, true><<<1, 32, 0, st>>>(A, rprev, small);
-            else gkr_final_kernel<true, false><<<1, 32, 0, st>>>(A, rprev, small);
-        } else {
-            gkr_final_kernel<false, false><<<1, 32, 0, st>>>(A, rprev, small);
-        }
-        fp_toc(c, st, slot);
-        FP_CUDA(c, cudaGetLastError());
-        FP_CUDA(c, cudaMemcpyAsync(hsmall, small, 64, cudaMemcpyDeviceToHost, st));
-        FP_CUDA(c, cudaStreamSynchronize(st));
-        for (int i = 0; i < 8; i++) put_le(proof + pos + 8 * i, hsmall[i], 8);
-        fp_tx_absorb_raw(tx, "gkr_final", proof + pos, 64);
-        pos += 64;
-        const uint64_t mu = fp_tx_squeeze_one(tx, "gkr_mu");
-        for (int t = 0; t < d; t++) z.z[t] = rho[t];
-        z.z[d] = mu;
-        z.v = d + 1;
+        const int64_t h1 = 1ll << (d - 1);
+        // small layers: fewer threads, so single-block rounds reduce over fewer warps
+        A.threads = (int)std::min<int64_t>(LU_THREADS, std::max<int64_t>(64, h1));
+        A.per_block = A.threads * 4;
+        const int64_t want = (h1 + A.per_block - 1) / A.per_block;
+        const int cap = std::max(1, occ[leaf ? 1 : 0]) * c->num_sms;
+        A.grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
+        A.seq0 = fp_seq_reserve(c, d + 2);
     }
+    if ((rc = fp_session_begin(c, st))) return rc;
+    if (!c->stepped) {
+        for (int d = 1; d <= v - 1; d++) {
+            GkrLayer& A = layers[d - 1];
+            A.t_begin = 1;
+            A.t_end = d + 1;
+            void* args[] = {&A, &c->mb_dev, &c->relay, &part};
+            const bool leaf = (d == v - 1);
+            int slot;
+            fp_tic(c, st, K_GKR_ROUND, (leaf ? 36.0 : 128.0) * (double)(1ll << d), &slot);
+            FP_CUDA(c, cudaLaunchCooperativeKernel(leaf ? (const void*)gkr_layer_kernel<true>
+                                                        : (const void*)gkr_layer_kernel<false>,
+                                                   dim3(A.grid), dim3(A.threads), args, 0, st));
+            fp_toc(c, st, slot);
+        }
+    }
+    uint64_t mu = z.z[0];
+    for (int d = 1; d <= v - 1; d++) {
+        GkrLayer A = layers[d - 1];
+        const bool leaf = (d == v - 1);
+        const void* kern = leaf ? (const void*)gkr_layer_kernel<true> : (const void*)gkr_layer_kernel<false>;
+        const uint64_t lam = fp_tx_squeeze_one(tx, "gkr_lambda");
+        fp_session_expect(c, d >= 1 ? 4 : 8);
+        fp_session_post2(c, A.seq0, mu, lam);
+        for (int t = 1; t <= d + 1; t++) {
+            if (c->stepped) {
+                // one launch per round (its challenge is already in the mailbox), then the final values
+                A.t_begin = A.t_end = t;
+                void* args[] = {&A, &c->mb_dev, &c->relay, &part};
+                const int64_t h = t <= d ? 1ll << (d - t) : 0;
+                int slot;
+                if (t <= d)
+                    fp_tic(c, st, K_GKR_ROUND, (leaf && t <= 2 ? 36.0 : 128.0) * h * (t == 1 ? 1 : 2) + 24.0 * h, &slot);
+                else
+                    fp_tic(c, st, K_GKR_FINAL, 128.0, &slot);
+                FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(t <= d ? A.grid : 1), dim3(A.threads), args, 0, st));
+                fp_toc(c, st, slot);
+            }
+            if ((rc = fp_session_wait(c, A.seq0 + t, st))) return rc;
+            if (t <= d) {
+                for (int i = 0; i < 4; i++) put_le(proof + pos + 8 * i, c->mb->res[i], 8);
+                fp_tx_absorb_raw(tx, "gkr_round", proof + pos, 32);
+                pos += 32;
+                fp_session_expect(c, t < d ? 4 : 8);  // the last challenge triggers the final values
+                fp_session_post(c, A.seq0 + t, fp_tx_squeeze_one(tx, "gkr_chal"));
+            } else {
+                for (int i = 0; i < 8; i++) put_le(proof + pos + 8 * i, c->mb->res[i], 8);
+                fp_tx_absorb_raw(tx, "gkr_final", proof + pos, 64);
+                pos += 64;
+                mu = fp_tx_squeeze_one(tx, "gkr_mu");
+            }
+        }
+    }
+    // the leaf point: the last layer's round challenges, then its mu
+    if (v >= 2) {
+        FP_CUDA(c, cudaMemcpyAsync(hsmall, zb[v & 1], 8 * (size_t)(v - 1), cudaMemcpyDeviceToHost, st));
+        FP_CUDA(c, cudaStreamSynchronize(st));
+        for (int i = 0; i < v - 1; i++) z.z[i] = hsmall[i];
+    }
+    z.z[v - 1] = mu;
+    z.v = v;
 
     // ---- leaf claims ----
     {

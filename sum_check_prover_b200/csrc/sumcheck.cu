@@ -14,64 +14,107 @@
 // pass; warp shuffles + a block tree + the last block finish the sums.
 #include <string.h>
 
+#include <algorithm>
 #include <map>
 #include <vector>
 
 #include "fp_internal.h"
 #include "fp_reduce.cuh"
+#include "fp_session.cuh"
 
 namespace {
 
 constexpr int SC_THREADS = 256;
 
-// Round t of the matmul sum-check over `nsites` site vectors of current length
-// 2*half. FOLD: the inputs have length 4*half per site (round t-1's vectors)
-// and are folded by rprev first, the folded halves being written to out.
-template <bool FOLD, bool MULTI>
-__global__ void __launch_bounds__(SC_THREADS)
-    sc_round_kernel(const uint64_t* __restrict__ Ain, const uint64_t* __restrict__ Bin, uint64_t* __restrict__ Aout,
-                    uint64_t* __restrict__ Bout, int64_t half, int logh, int64_t npairs, uint64_t rprev,
-                    const uint64_t* __restrict__ rho, uint64_t* part, unsigned int* ticket,
-                    uint64_t* __restrict__ gout) {
-    uint64_t acc[3] = {0, 0, 0};
-    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < npairs; p += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t s = p >> logh, b = p & (half - 1);
-        uint64_t a0, a1, b0, b1;
-        if (FOLD) {
-            const int64_t bi = s * 4 * half + b;
-            a0 = gl_fold(Ain[bi], Ain[bi + 2 * half], rprev);
-            a1 = gl_fold(Ain[bi + half], Ain[bi + 3 * half], rprev);
-            b0 = gl_fold(Bin[bi], Bin[bi + 2 * half], rprev);
-            b1 = gl_fold(Bin[bi + half], Bin[bi + 3 * half], rprev);
-            const int64_t bo = s * 2 * half + b;
-            Aout[bo] = a0;
-            Aout[bo + half] = a1;
-            Bout[bo] = b0;
-            Bout[bo + half] = b1;
+struct ScArgs {
+    uint64_t* A[2];  // ping-pong vectors; A[0], B[0] hold the partial evaluations (site stride 2^n)
+    uint64_t* B[2];
+    const uint64_t* rho;
+    uint64_t* fin;   // 2 * nsites final values
+    int nsites, n;
+    int grid, per_block;
+    uint64_t seq0;   // round t publishes seq0 + t and waits for challenge seq0 + t
+    int t_begin, t_end;  // rounds run by this launch; t_end > n includes the final values
+};
+
+// All n rounds of the matmul sum-check, then the final values, in one launch.
+// Round t pairs (b, b + half) of every site; from round 2 on the inputs are the
+// previous round's vectors (length 4 half per site), folded by the previous
+// challenge on the fly, the folded halves going to the other buffer.
+template <bool MULTI>
+__global__ void __launch_bounds__(SC_THREADS) sc_session_kernel(ScArgs P, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
+    uint64_t rprev = 0;
+    for (int t = P.t_begin; t <= P.n && t <= P.t_end; t++) {
+        if (t > 1 && !session_wait(mb, rl, P.seq0 + t - 1, rprev)) return;
+        const int logh = P.n - t;
+        const int64_t half = 1ll << logh;
+        const int64_t npairs = (int64_t)P.nsites * half;
+        int64_t want = (npairs + P.per_block - 1) / P.per_block;
+        const unsigned active = (unsigned)(want < 1 ? 1 : (want > P.grid ? P.grid : want));
+        if (blockIdx.x >= active) return;
+        const bool fold = t > 1;
+        const uint64_t* Ain = fold ? P.A[t & 1] : P.A[0];
+        const uint64_t* Bin = fold ? P.B[t & 1] : P.B[0];
+        uint64_t* Aout = P.A[1 - (t & 1)];
+        uint64_t* Bout = P.B[1 - (t & 1)];
+        uint64_t acc[3] = {0, 0, 0};
+        for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < npairs; p += (int64_t)active * blockDim.x) {
+            const int64_t s = p >> logh, b = p & (half - 1);
+            uint64_t a0, a1, b0, b1;
+            if (fold) {
+                const int64_t bi = s * 4 * half + b;
+                a0 = gl_fold(__ldcg(Ain + bi), __ldcg(Ain + bi + 2 * half), rprev);
+                a1 = gl_fold(__ldcg(Ain + bi + half), __ldcg(Ain + bi + 3 * half), rprev);
+                b0 = gl_fold(__ldcg(Bin + bi), __ldcg(Bin + bi + 2 * half), rprev);
+                b1 = gl_fold(__ldcg(Bin + bi + half), __ldcg(Bin + bi + 3 * half), rprev);
+                const int64_t bo = s * 2 * half + b;
+                Aout[bo] = a0;
+                Aout[bo + half] = a1;
+                Bout[bo] = b0;
+                Bout[bo + half] = b1;
+            } else {
+                const int64_t bi = s * 2 * half + b;
+                a0 = __ldcg(Ain + bi);
+                a1 = __ldcg(Ain + bi + half);
+                b0 = __ldcg(Bin + bi);
+                b1 = __ldcg(Bin + bi + half);
+            }
+            const uint64_t a2 = gl_sub(gl_add(a1, a1), a0);
+            const uint64_t b2 = gl_sub(gl_add(b1, b1), b0);
+            uint64_t t0 = gl_mul(a0, b0), t1 = gl_mul(a1, b1), t2 = gl_mul(a2, b2);
+            if (MULTI) {
+                const uint64_t rs = P.rho[s];
+                t0 = gl_mul(t0, rs);
+                t1 = gl_mul(t1, rs);
+                t2 = gl_mul(t2, rs);
+            }
+            acc[0] = gl_add(acc[0], t0);
+            acc[1] = gl_add(acc[1], t1);
+            acc[2] = gl_add(acc[2], t2);
+        }
+        bool last;
+        if (active == 1) {
+            block_sum_gl<3>(acc);
+            last = true;
         } else {
-            const int64_t bi = s * 2 * half + b;
-            a0 = Ain[bi];
-            a1 = Ain[bi + half];
-            b0 = Bin[bi];
-            b1 = Bin[bi + half];
+            last = grid_sum_gl_n<3>(acc, part, &rl->ticket, active);
         }
-        const uint64_t a2 = gl_sub(gl_add(a1, a1), a0);
-        const uint64_t b2 = gl_sub(gl_add(b1, b1), b0);
-        uint64_t t0 = gl_mul(a0, b0), t1 = gl_mul(a1, b1), t2 = gl_mul(a2, b2);
-        if (MULTI) {
-            const uint64_t rs = rho[s];
-            t0 = gl_mul(t0, rs);
-            t1 = gl_mul(t1, rs);
-            t2 = gl_mul(t2, rs);
-        }
-        acc[0] = gl_add(acc[0], t0);
-        acc[1] = gl_add(acc[1], t1);
-        acc[2] = gl_add(acc[2], t2);
+        if (last && threadIdx.x == 0) session_publish(mb, acc, 3, P.seq0 + t);
     }
-    if (grid_sum_gl<3>(acc, part, ticket) && threadIdx.x == 0) {
-        gout[0] = acc[0];
-        gout[1] = acc[1];
-        gout[2] = acc[2];
+    if (P.t_end <= P.n || blockIdx.x != 0) return;
+    if (!session_wait(mb, rl, P.seq0 + P.n, rprev)) return;
+    // the round-n vectors (length 2 per site) sit in A[0] when n == 1, else in the round's output buffer
+    const uint64_t* Af = P.n == 1 ? P.A[0] : P.A[1 - (P.n & 1)];
+    const uint64_t* Bf = P.n == 1 ? P.B[0] : P.B[1 - (P.n & 1)];
+    for (int s = threadIdx.x; s < P.nsites; s += blockDim.x) {
+        P.fin[2 * s] = gl_fold(__ldcg(Af + 2 * s), __ldcg(Af + 2 * s + 1), rprev);
+        P.fin[2 * s + 1] = gl_fold(__ldcg(Bf + 2 * s), __ldcg(Bf + 2 * s + 1), rprev);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const uint64_t done = 0;
+        session_publish(mb, &done, 1, P.seq0 + P.n + 1);
     }
 }
 
@@ -132,16 +175,19 @@ int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites
     need += fp_claims_scratch(sites, nsites);
     const size_t vec = (size_t)8 * nsites * L;
     need += 4 * fp_align_up(vec, 256);
-    size_t pr = 0;
-    for (int s = 0; s < nsites; s++)
-        pr = std::max(pr, std::max(fp_partial_rows_scratch(c, sites[s].M, sites[s].K),
-                                   fp_partial_rows_scratch(c, sites[s].N, sites[s].K)));
-    need += pr;
-    const int max_blocks = 4 * c->num_sms;
-    need += fp_align_up((size_t)8 * 3 * max_blocks, 256) + fp_align_up(8 * (size_t)nsites, 256) * 3 + (1 << 16);
+    // partial-evaluation jobs (points filled in once squeezed)
+    std::vector<FpPeJob> pe(2 * (size_t)nsites);
+    for (int s = 0; s < nsites; s++) {
+        pe[2 * s] = FpPeJob{sites[s].w, sites[s].w_bits, sites[s].scales, sites[s].M, sites[s].K, nullptr,
+                            fp_log2_ceil((uint64_t)sites[s].M), nullptr, L};
+        pe[2 * s + 1] = FpPeJob{sites[s].xt, 8, nullptr, sites[s].N, sites[s].K, nullptr,
+                                fp_log2_ceil((uint64_t)sites[s].N), nullptr, L};
+    }
+    need += fp_partial_scratch(c, pe.data(), (int)pe.size());
+    need += fp_align_up((size_t)8 * 3 * 16 * c->num_sms, 256) + fp_align_up(8 * (size_t)nsites, 256) * 3 + (1 << 16);
     if ((rc = fp_reserve(c, c->dev, need))) return rc;
     if ((rc = fp_reserve(c, c->host, fp_align_up(sizeof(uint64_t) * (4 * (size_t)nsites + 64), 256) + 8192 +
-                                         (size_t)160 * nsites)))
+                                         (size_t)160 * nsites + fp_partial_host_scratch(pe.data(), (int)pe.size()))))
         return rc;
     fp_reset(c->dev);
     fp_reset(c->host);
@@ -192,63 +238,86 @@ int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites
     memcpy(hrho, rho.data(), 8 * (size_t)nsites);
     FP_CUDA(c, cudaMemcpyAsync(drho, hrho, 8 * (size_t)nsites, cudaMemcpyHostToDevice, st));
 
-    // ---- partial evaluations A_s = W~_s(r_row, .), B_s = X~_s(., r_col) ----
+    // ---- partial evaluations A_s = W~_s(r_row, .), B_s = X~_s(., r_col), one launch ----
     uint64_t* bufA[2] = {(uint64_t*)fp_alloc(c->dev, vec), (uint64_t*)fp_alloc(c->dev, vec)};
     uint64_t* bufB[2] = {(uint64_t*)fp_alloc(c->dev, vec), (uint64_t*)fp_alloc(c->dev, vec)};
-    const size_t mark = c->dev.top;
+    if (!bufA[0] || !bufB[0]) return fp_fail(c, FP_ERR_OOM, "sumcheck: scratch exhausted");
     for (int s = 0; s < nsites; s++) {
-        c->dev.top = mark;  // partial-evaluation scratch is reused site after site
-        if ((rc = fp_partial_rows(c, sites[s].w, sites[s].w_bits, sites[s].scales, sites[s].M, sites[s].K, er[s],
-                                  bufA[0] + (size_t)s * L, L, st)))
-            return rc;
-        c->dev.top = mark;
-        if ((rc = fp_partial_rows(c, sites[s].xt, 8, nullptr, sites[s].N, sites[s].K, ec[s],
-                                  bufB[0] + (size_t)s * L, L, st)))
-            return rc;
+        pe[2 * s].z = zr.z;
+        pe[2 * s].out = bufA[0] + (size_t)s * L;
+        pe[2 * s + 1].z = zc.z;
+        pe[2 * s + 1].out = bufB[0] + (size_t)s * L;
     }
-    c->dev.top = mark + pr;
-    uint64_t* part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * 3 * max_blocks);
+    if ((rc = fp_partial_many(c, pe.data(), (int)pe.size(), st))) return rc;
+    uint64_t* part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * 3 * 16 * c->num_sms);
     uint64_t* dg = (uint64_t*)fp_alloc(c->dev, 64);
     uint64_t* dfin = (uint64_t*)fp_alloc(c->dev, 16 * (size_t)nsites);
     if (!bufA[1] || !bufB[1] || !part || !dg || !dfin) return fp_fail(c, FP_ERR_OOM, "sumcheck: scratch exhausted");
 
-    // ---- rounds ----
-    int cur = 0;
-    uint64_t rprev = 0;
-    for (int t = 1; t <= n; t++) {
-        const int64_t half = 1ll << (n - t);
-        const int64_t npairs = (int64_t)nsites * half;
-        int blocks = (int)std::min<int64_t>(max_blocks, (npairs + SC_THREADS - 1) / SC_THREADS);
-        const bool fold = t > 1;
-        const int nxt = fold ? 1 - cur : cur;
-        double bytes = fold ? 48.0 * npairs : 32.0 * npairs;
-        int slot;
-        fp_tic(c, st, K_SC_ROUND, bytes, &slot);
-#define SC_LAUNCH(F, M)                                                                                    \
-    sc_round_kernel<F, M><<<blocks, SC_THREADS, 0, st>>>(bufA[cur], bufB[cur], bufA[nxt], bufB[nxt], half, \
-                                                         n - t, npairs, rprev, drho, part, c->tickets, dg)
-        if (fold) {
-            if (nsites > 1) SC_LAUNCH(true, true); else SC_LAUNCH(true, false);
-        } else {
-            if (nsites > 1) SC_LAUNCH(false, true); else SC_LAUNCH(false, false);
+    // ---- rounds: one persistent kernel ----
+    if (n > 0) {
+        int occ = 0;
+        if (nsites > 1)
+            FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, sc_session_kernel<true>, SC_THREADS, 0));
+        else
+            FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, sc_session_kernel<false>, SC_THREADS, 0));
+        ScArgs P;
+        P.A[0] = bufA[0];
+        P.A[1] = bufA[1];
+        P.B[0] = bufB[0];
+        P.B[1] = bufB[1];
+        P.rho = drho;
+        P.fin = dfin;
+        P.nsites = nsites;
+        P.n = n;
+        P.per_block = SC_THREADS * 4;
+        const int64_t want = ((int64_t)nsites * (L / 2) + P.per_block - 1) / P.per_block;
+        P.grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)std::max(1, occ) * c->num_sms));
+        P.seq0 = fp_seq_reserve(c, n + 2);
+        if ((rc = fp_session_begin(c, st))) return rc;
+        fp_session_expect(c, 3);  // round 1 publishes without a challenge
+        void* args[] = {&P, &c->mb_dev, &c->relay, &part};
+        const void* kern = nsites > 1 ? (const void*)sc_session_kernel<true> : (const void*)sc_session_kernel<false>;
+        if (!c->stepped) {
+            P.t_begin = 1;
+            P.t_end = n + 1;
+            int slot;
+            fp_tic(c, st, K_SC_ROUND, 32.0 * nsites * L + 48.0 * nsites * L / 2, &slot);
+            FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(P.grid), dim3(SC_THREADS), args, 0, st));
+            fp_toc(c, st, slot);
         }
-#undef SC_LAUNCH
+        for (int t = 1; t <= n; t++) {
+            if (c->stepped) {
+                P.t_begin = P.t_end = t;
+                const double pairs = (double)nsites * (double)(1ll << (n - t));
+                int slot;
+                fp_tic(c, st, K_SC_ROUND, t == 1 ? 32.0 * pairs : 48.0 * pairs, &slot);
+                FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(P.grid), dim3(SC_THREADS), args, 0, st));
+                fp_toc(c, st, slot);
+            }
+            if ((rc = fp_session_wait(c, P.seq0 + t, st))) return rc;
+            uint64_t g[3] = {c->mb->res[0], c->mb->res[1], c->mb->res[2]};
+            put_u64s(proof + pos, g, 3);
+            fp_tx_absorb_raw(tx, "sc_round", proof + pos, 24);
+            pos += 24;
+            fp_session_expect(c, t < n ? 3 : 1);  // the last challenge triggers the final values
+            fp_session_post(c, P.seq0 + t, fp_tx_squeeze_one(tx, "sc_chal"));
+        }
+        if (c->stepped) {
+            P.t_begin = P.t_end = n + 1;
+            int slot;
+            fp_tic(c, st, K_SC_FINAL, 32.0 * nsites, &slot);
+            FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(1), dim3(SC_THREADS), args, 0, st));
+            fp_toc(c, st, slot);
+        }
+        if ((rc = fp_session_wait(c, P.seq0 + n + 1, st))) return rc;
+    } else {
+        int slot;
+        fp_tic(c, st, K_SC_FINAL, 32.0 * nsites, &slot);
+        sc_final_kernel<<<(nsites + 127) / 128, 128, 0, st>>>(bufA[0], bufB[0], nsites, 1, 0, dfin);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
-        cur = nxt;
-        FP_CUDA(c, cudaMemcpyAsync(hbuf, dg, 24, cudaMemcpyDeviceToHost, st));
-        FP_CUDA(c, cudaStreamSynchronize(st));
-        put_u64s(proof + pos, hbuf, 3);
-        fp_tx_absorb_raw(tx, "sc_round", proof + pos, 24);
-        pos += 24;
-        rprev = fp_tx_squeeze_one(tx, "sc_chal");
     }
-    // ---- final evaluations ----
-    int slot;
-    fp_tic(c, st, K_SC_FINAL, 32.0 * nsites, &slot);
-    sc_final_kernel<<<(nsites + 127) / 128, 128, 0, st>>>(bufA[cur], bufB[cur], nsites, n > 0 ? 2 : 1, rprev, dfin);
-    fp_toc(c, st, slot);
-    FP_CUDA(c, cudaGetLastError());
     FP_CUDA(c, cudaMemcpyAsync(hbuf, dfin, 16 * (size_t)nsites, cudaMemcpyDeviceToHost, st));
     FP_CUDA(c, cudaStreamSynchronize(st));
     put_u64s(proof + pos, hbuf, 2 * (size_t)nsites);

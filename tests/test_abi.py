@@ -81,3 +81,21 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(fp, "_lib", None)
     with pytest.raises(ImportError):
         fp.lib()
+
+
+def test_portable_sha_path_matches_oracle(L):
+    """The host transcript uses the CPU's SHA extensions when present; the
+    portable compression (forced here) must give the same states."""
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, '.'); import sum_check_prover_b200 as fp, oracle; "
+            "a, b = fp.Transcript(7), oracle.Transcript(7)\n"
+            "for i in range(300):\n"
+            "    d = bytes((i * 37 + j) % 256 for j in range(i % 190))\n"
+            "    a.absorb('l%d' % (i % 5), d); b.absorb('l%d' % (i % 5), d)\n"
+            "    assert a.squeeze('c')[0] == b.squeeze('c')\n"
+            "assert a.state() == b.state(); print('ok')")
+    import os
+    env = dict(os.environ, FP_NO_SHANI="1")
+    r = subprocess.run([sys.executable, "-c", code], cwd=str(ROOT), env=env, capture_output=True, text=True)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stderr

@@ -210,3 +210,21 @@ def test_argument_errors(env):
     with pytest.raises(fp.FpError):
         ctx.prove_logup(tx, [d, mix])
     tx.close()
+
+
+def test_stepped_and_resident_rounds_give_the_same_proof(env):
+    torch, fp, ctx = env
+    wl = workloads.build(3, seed=8, small=True)
+    a = run_gpu(env, wl, 8)[0]
+    ctx.set_profiling(True)        # profiling launches every round separately
+    b = run_gpu(env, wl, 8)[0]
+    stats = ctx.kernel_stats()
+    ctx.set_profiling(False)
+    assert a == b
+    assert stats["gkr_round"][0] > 20 and stats["sc_round"][0] >= 8
+
+
+def test_bounded_wait_times_out_and_context_survives(env):
+    torch, fp, ctx = env
+    assert ctx.session_selftest() == -4      # FP_ERR_TIMEOUT, reported, not hung
+    check_against_oracle(env, workloads.build(1), 0)
