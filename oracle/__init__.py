@@ -104,6 +104,8 @@ def lib():
                                 C.POINTER(u64), vp, C.POINTER(u64)]
         L.orc_verify.restype = C.c_int
         L.orc_verify.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp]
+        L.orc_verify_opts.restype = C.c_int
+        L.orc_verify_opts.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp, vp, C.c_int]
         _lib = L
     return _lib
 
@@ -324,11 +326,20 @@ def prove(seed: int, sites, wits):
     return buf[: n.value].tobytes(), [st[0:32], st[32:64], st[64:96]], off.value
 
 
-def verify(seed: int, sites, wits, proof: bytes):
-    """Returns (reason_name, detail) -- reason 'accept' for a valid proof."""
+def verify(seed: int, sites, wits, proof: bytes, site_mask=None, skip_leaf_open: bool = False):
+    """Returns (reason_name, detail) -- reason 'accept' for a valid proof.
+
+    site_mask (optional, one flag per site) limits the direct recomputation of
+    claims and of W/X evaluations to the flagged sites; skip_leaf_open skips the
+    recomputation of the key columns' MLEs. Every other check always runs."""
     keep = []
     cs, cw = _marshal(sites, wits, keep)
     pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
     det = np.zeros(2, dtype=np.int64)
-    rc = lib().orc_verify(seed, cs, len(sites), cw, _ptr(pb), len(proof), _ptr(det))
+    if site_mask is None and not skip_leaf_open:
+        rc = lib().orc_verify(seed, cs, len(sites), cw, _ptr(pb), len(proof), _ptr(det))
+    else:
+        mask = None if site_mask is None else np.ascontiguousarray(np.asarray(site_mask, dtype=np.uint8))
+        rc = lib().orc_verify_opts(seed, cs, len(sites), cw, _ptr(pb), len(proof), _ptr(det), _ptr(mask),
+                                   4 if skip_leaf_open else 0)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

@@ -981,6 +981,15 @@ static void rd_mult(orc_tx* t, prd* r, const char* label, u32* out, u64 n) {
         goto done;               \
     } while (0)
 
+/* Verification options for statements too large to check in full: a site
+ * whose mask entry is 0 skips the direct recomputation of its claim and of its
+ * A/B evaluations (every other check still runs); VERIFY_SKIP_LEAF_OPEN skips
+ * recomputing the key columns' MLEs. NULL mask and flags 0 = full verification. */
+#define VERIFY_SKIP_LEAF_OPEN 4
+static const uint8_t* g_site_mask = NULL;
+static int g_verify_flags = 0;
+static int site_checked(int s) { return g_site_mask == NULL || g_site_mask[s]; }
+
 static int mm_verify(orc_tx* t, prd* rd, const orc_site* sites, int ns, const orc_wit* wit,
                      int64_t* detail) {
     int rc = 0, vM, vN, n;
@@ -996,6 +1005,7 @@ static int mm_verify(orc_tx* t, prd* rd, const orc_site* sites, int ns, const or
     rd_fe(t, rd, "claims", c, (u64)ns);
     if (rd->bad) FAIL(REJ_FORMAT, 0, 0);
     for (int s = 0; s < ns; s++) {
+        if (!site_checked(s)) continue;
         int ms = orc_log2_ceil((u64)sites[s].M), nn = orc_log2_ceil((u64)sites[s].N);
         u64 want = orc_claim(wit[s].q, wit[s].r, sites[s].M, sites[s].N, sites[s].k_shift, rr, ms, rc_, nn);
         if (want != c[s]) FAIL(REJ_CLAIM, s, 0);
@@ -1022,6 +1032,7 @@ static int mm_verify(orc_tx* t, prd* rd, const orc_site* sites, int ns, const or
         if (acc != claim) FAIL(REJ_MM_FINAL, 0, 0);
     }
     for (int s = 0; s < ns; s++) {
+        if (!site_checked(s)) continue;
         int ms = orc_log2_ceil((u64)sites[s].M), nn = orc_log2_ceil((u64)sites[s].N);
         if (mle_w_direct(&sites[s], rr, ms, pt, n) != fin[2 * s]) FAIL(REJ_MM_A, s, 0);
         if (mle_x_direct(&sites[s], pt, n, rc_, nn) != fin[2 * s + 1]) FAIL(REJ_MM_B, s, 0);
@@ -1132,7 +1143,7 @@ static int lu_verify(orc_tx* t, prd* rd, const orc_site* sites, int ns, const or
     if (cP[0] != 1 || cP[1] != 1) FAIL(REJ_LEAF_P, 0, 0);
     if (cQ[0] != orc_fsub(alpha[0], leaf[0])) FAIL(REJ_LEAF_Q, 0, 0);
     if (cQ[1] != orc_fsub(alpha[1], orc_fadd(leaf[1], orc_fmul(gamma, leaf[2])))) FAIL(REJ_LEAF_Q, 1, 0);
-    {
+    if (!(g_verify_flags & VERIFY_SKIP_LEAF_OPEN)) {
         u64 Lk = (u64)1 << v;
         col = (u64*)malloc(Lk * sizeof(u64));
         for (u64 i = 0; i < Lk; i++) col[i] = orc_fint(K.fr[i]);
@@ -1148,8 +1159,18 @@ done:
     return rc;
 }
 
+int orc_verify_opts(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, const uint8_t* proof, u64 len,
+                    int64_t detail[2], const uint8_t* site_mask, int flags);
+
 int orc_verify(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, const uint8_t* proof, u64 len,
                int64_t detail[2]) {
+    return orc_verify_opts(seed, sites, ns, wit, proof, len, detail, NULL, 0);
+}
+
+int orc_verify_opts(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, const uint8_t* proof, u64 len,
+                    int64_t detail[2], const uint8_t* site_mask, int flags) {
+    g_site_mask = site_mask;
+    g_verify_flags = flags;
     detail[0] = detail[1] = 0;
     if (ns < 1) return REJ_ARGS;
     for (int s = 0; s < ns; s++)
