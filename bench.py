@@ -42,7 +42,7 @@ FLUSH_BYTES = 512 << 20  # > 126 MB L2
 
 # kernel -> source file (traffic counters are valid only for the source they were taken on)
 KSRC = {"witness_gemm": "witness.cu", "digest_leaf": "digest.cu", "digest_node": "digest.cu",
-        "digest_final": "digest.cu", "eq_build": "mle.cu", "partial_acc": "mle.cu", "partial_fin": "mle.cu",
+        "digest_final": "digest.cu", "eq_build": "mle.cu", "partial_acc": "partial.cu", "partial_fin": "partial.cu",
         "claim": "mle.cu", "sc_round": "sumcheck.cu", "sc_final": "sumcheck.cu", "hist": "logup.cu",
         "keys_gather": "logup.cu", "tree_leaf": "logup.cu", "tree_up": "logup.cu", "gkr_round": "logup.cu",
         "gkr_final": "logup.cu", "leaf_eval": "logup.cu", "reduce": "mle.cu"}
@@ -118,6 +118,69 @@ class Clocks:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr") -> dict:
+    """Kernel rooflines at HBM scale (inputs well above the 126 MB L2), from a
+    profiled pass: every round is its own launch, timed with CUDA events.
+
+    sc_round: matmul sum-check rounds over 2 x 2^26-element vectors (64 sites,
+      W 1 x 2^20 int4, one token); round 1 reads A and B, later rounds fold
+      in place of the next evaluation (read 4, write 2 values per pair).
+    partial_acc: eq-weighted row contraction of a 16384 x 16384 int4 matrix.
+    gkr_round: LogUp layer rounds over 2^26 keys (one 8192 x 64 x 8192 int8 site).
+    """
+    import workloads
+    from workloads import device
+    pk = peaks()
+    out = {}
+
+    def measure(name, kernel, fn, big=1 << 28):
+        ctx.set_profiling(True)
+        fn()  # warm: module loading and arena growth stay out of the numbers
+        torch.cuda.synchronize()
+        ctx.set_profiling(True)  # resets the per-kernel counters
+        fn()
+        torch.cuda.synchronize()
+        log = [r for r in ctx.kernel_log() if r[0] == kernel]
+        ctx.set_profiling(False)
+        # the HBM-scale launches (>= 256 MB of algorithmic traffic); the small
+        # rounds at the end of a sum-check are latency, not bandwidth
+        sel = [r for r in log if r[2] >= big]
+        ms = sum(r[1] for r in sel)
+        by = sum(r[2] for r in sel)
+        gbs = by / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
+        out[name] = {"kernel": kernel, "launches": len(sel), "ms": ms, "bytes": by, "GBps": gbs,
+                     "frac": gbs / pk["hbm_gbs"], "peak": pk["hbm_gbs"],
+                     "per_launch": [[round(r[1], 4), r[2]] for r in sel],
+                     "all_launches": len(log), "all_ms": sum(r[1] for r in log)}
+
+    which = set(which.split(","))
+    if "sc" in which:
+        sites = [workloads.random_site(900 + i, 1, 1 << 20, 1, 4, 12) for i in range(64)]
+        st, keep = device.upload(workloads.Workload("sc", 0, sites), dev)
+        device.weight_digests(ctx, st)
+        measure("sc_round_2^26", "sc_round", lambda: fp.prove(ctx, 1, st))
+        del st, keep
+
+    if "pe" in which:
+        rows = cols = 16384
+        rng = __import__("numpy").random.default_rng(3)
+        mat = torch.from_numpy(workloads.int4_packed(rng, rows, cols)).to(dev)
+        outv = torch.empty(cols, dtype=torch.int64, device=dev)
+        z = [int(x) for x in rng.integers(0, fp.P, size=14, dtype="uint64")]
+        measure("partial_eval_int4_16384^2", "partial_acc",
+                lambda: ctx.partial_eval(mat, 4, None, rows, cols, z, outv), big=1 << 26)
+        del mat, outv
+
+    if "gkr" in which:
+        s = workloads.random_site(77, 8192, 64, 8192, 8, 12)
+        st, keep = device.upload(workloads.Workload("gkr", 0, [s]), dev)
+        device.weight_digests(ctx, st)
+        measure("gkr_round_2^26_keys", "gkr_round", lambda: fp.prove(ctx, 2, st))
+        del st, keep
+    torch.cuda.empty_cache()
+    return out
 
 
 def dist():
@@ -224,6 +287,7 @@ def run_ours(args):
     hw1 = ctx.host_stats()
     host_waits = (hw1[0] - hw0[0]) / args.steps
     host_wait_ms = (hw1[1] - hw0[1]) * 1e3 / args.steps
+    host_turn_us = (hw1[2] - hw0[2]) * 1e6 / max(1.0, hw1[0] - hw0[0])
     total_ms = sum(times)
     if pg is not None:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -302,6 +366,10 @@ def run_ours(args):
         cpu = {"value": macs / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "the whole statement once (witness + proof), single-threaded C", "seconds": dt}
 
+    micro = None
+    if rank == 0 and world == 1 and not args.no_micro:
+        micro = run_micro(fp, torch, ctx, f"cuda:{local}")
+
     ctx.close()
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -318,9 +386,11 @@ def run_ours(args):
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches,
                 "host_round_trips_per_step": host_waits,
+                "host_turnaround_us_per_round": host_turn_us,
                 "host_wait_ms_per_step": host_wait_ms,
                 "clocks": clk,
                 "kernels": kern,
+                "microbench": micro,
                 "proof_bytes": proof_len}
         print(json.dumps(line), flush=True)
     if pg is not None:
@@ -338,7 +408,18 @@ def main():
     ap.add_argument("--prof-steps", type=int, default=3)
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-micro", action="store_true")
+    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr", default=None,
+                    help="run only the HBM-scale kernel measurements (comma list of sc, pe, gkr)")
     args = ap.parse_args()
+    if args.micro_only:
+        import torch
+
+        import sum_check_prover_b200 as fp
+        ctx = fp.Context(0)
+        print(json.dumps({"microbench": run_micro(fp, torch, ctx, "cuda:0", args.micro_only)}))
+        ctx.close()
+        return
     if args.warmup < 1:
         args.warmup = 1
     if args.impl == "reference":

@@ -242,9 +242,23 @@ int fp_ctx_set_profiling(fp_ctx* ctx, int on);
 /* Number of kernels the library has launched on this context since its creation. */
 int64_t fp_ctx_launches(const fp_ctx* ctx);
 /* Host side of the round exchanges since the context was created:
- * out[0] = waits for a device result, out[1] = seconds spent waiting. */
-int fp_host_stats(const fp_ctx* ctx, double out[2]);
+ * out[0] = waits for a device result, out[1] = seconds spent waiting,
+ * out[2] = seconds from a result's arrival to the next challenge posted (the
+ * host's own share of a round: hashing and bookkeeping), out[3] = the longest
+ * such turnaround in seconds. */
+int fp_host_stats(const fp_ctx* ctx, double out[4]);
 int fp_kernel_stats(fp_ctx* ctx, fp_kernel_stat* out, int cap);
+/* Per-launch records of the same timing, in launch order: {kernel id, 0, device
+ * ms of that launch, its algorithmic bytes}. Copies up to `cap` records into
+ * `out` (host memory owned by the caller) and returns how many there are;
+ * cleared by fp_ctx_set_profiling. */
+typedef struct {
+    int32_t kernel;
+    int32_t reserved;
+    double ms;
+    double bytes;
+} fp_launch_rec;
+int64_t fp_kernel_log(fp_ctx* ctx, fp_launch_rec* out, int64_t cap);
 const char* fp_kernel_name(int kernel);
 
 #ifdef __cplusplus

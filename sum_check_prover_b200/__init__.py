@@ -40,6 +40,10 @@ class _KStat(C.Structure):
     _fields_ = [("kernel", C.c_int32), ("launches", C.c_int32), ("ms", C.c_double), ("bytes", C.c_double)]
 
 
+class _LRec(C.Structure):
+    _fields_ = [("kernel", C.c_int32), ("reserved", C.c_int32), ("ms", C.c_double), ("bytes", C.c_double)]
+
+
 _lib = None
 
 
@@ -76,6 +80,8 @@ def lib():
     L.fp_ctx_launches.restype = C.c_int64
     L.fp_ctx_launches.argtypes = [vp]
     L.fp_kernel_stats.argtypes = [vp, C.POINTER(_KStat), i32]
+    L.fp_kernel_log.restype = C.c_int64
+    L.fp_kernel_log.argtypes = [vp, C.POINTER(_LRec), C.c_int64]
     L.fp_kernel_name.restype = C.c_char_p
     L.fp_kernel_name.argtypes = [i32]
     _lib = L
@@ -243,14 +249,22 @@ class Context:
         return int(self._L.fp_session_selftest(self.h, _stream(stream)))
 
     def host_stats(self):
-        """(waits for a device result, seconds spent waiting) since the context was created."""
-        out = (C.c_double * 2)()
+        """(waits for a device result, seconds spent waiting, seconds from results to the
+        next posted challenge, longest such turnaround) since the context was created."""
+        out = (C.c_double * 4)()
         self._check(self._L.fp_host_stats(self.h, out), "fp_host_stats")
-        return int(out[0]), float(out[1])
+        return int(out[0]), float(out[1]), float(out[2]), float(out[3])
 
     def launches(self) -> int:
         """Kernels launched by the library on this context so far."""
         return int(self._L.fp_ctx_launches(self.h))
+
+    def kernel_log(self) -> list:
+        """[(kernel name, device ms, algorithmic bytes)] per timed launch, in launch order."""
+        n = self._check(self._L.fp_kernel_log(self.h, None, 0), "fp_kernel_log")
+        arr = (_LRec * max(1, n))()
+        n = self._check(self._L.fp_kernel_log(self.h, arr, n), "fp_kernel_log")
+        return [(self._L.fp_kernel_name(r.kernel).decode(), r.ms, r.bytes) for r in arr[:n]]
 
     def kernel_stats(self) -> dict:
         """{kernel name: (launches, total ms, algorithmic bytes)} since the last reset."""

@@ -116,6 +116,7 @@ uint64_t fp_seq_reserve(fp_ctx* c, uint64_t n) {
 // Reset the relay before a persistent launch and clear stale mailbox errors.
 int fp_session_begin(fp_ctx* c, cudaStream_t s) {
     c->mb->err = 0;
+    c->t_result = -1;
     fp_session_expect(c, 0);
     FP_CUDA(c, cudaMemsetAsync(c->relay, 0, sizeof(FpRelay), s));
     return FP_OK;
@@ -134,7 +135,9 @@ int fp_session_wait(fp_ctx* c, uint64_t seq, cudaStream_t s) {
         for (int i = 0; i < n; i++) full = full && (mb->res[i] != kEmpty);
         if (full) {
             std::atomic_thread_fence(std::memory_order_acquire);
-            c->host_wait_s += std::chrono::duration<double>(clk::now() - t0).count();
+            const auto t1 = clk::now();
+            c->host_wait_s += std::chrono::duration<double>(t1 - t0).count();
+            c->t_result = std::chrono::duration<double>(t1.time_since_epoch()).count();
             return FP_OK;
         }
         if ((spin & 255) != 255) continue;
@@ -195,6 +198,13 @@ void fp_session_post2(fp_ctx* c, uint64_t seq, uint64_t chal, uint64_t chal2) {
     std::atomic_signal_fence(std::memory_order_seq_cst);
     _mm_store_si128((__m128i*)(&mb->chal), _mm_set_epi64x((long long)seq, (long long)chal));
     std::atomic_thread_fence(std::memory_order_release);
+    if (c->t_result >= 0) {
+        const double dt =
+            std::chrono::duration<double>(std::chrono::steady_clock::now().time_since_epoch()).count() - c->t_result;
+        c->host_turn_s += dt;
+        if (dt > c->host_turn_max) c->host_turn_max = dt;
+        c->t_result = -1;
+    }
 }
 
 void fp_session_post(fp_ctx* c, uint64_t seq, uint64_t chal) { fp_session_post2(c, seq, chal, 0); }
@@ -274,6 +284,7 @@ static void stats_resolve(fp_ctx* c) {
         c->stats[p.kernel].launches += 1;
         c->stats[p.kernel].ms += ms;
         c->stats[p.kernel].bytes += p.bytes;
+        c->log.push_back(fp_launch_rec{p.kernel, 0, (double)ms, p.bytes});
         c->ev_free.push_back(p.a);
         c->ev_free.push_back(p.b);
     }
@@ -283,6 +294,7 @@ static void stats_resolve(fp_ctx* c) {
 void fp_stats_reset(fp_ctx* c) {
     stats_resolve(c);
     for (auto& s : c->stats) s = FpKStat();
+    c->log.clear();
 }
 
 int fp_ctx_set_profiling(fp_ctx* c, int on) {
@@ -292,6 +304,7 @@ int fp_ctx_set_profiling(fp_ctx* c, int on) {
     // per-kernel timing brackets each round's launch, so profiling runs stepped
     c->stepped = c->profiling || c->stepped_env;
     for (auto& s : c->stats) s = FpKStat();
+    c->log.clear();
     return FP_OK;
 }
 
@@ -301,6 +314,8 @@ int fp_host_stats(const fp_ctx* c, double out[2]) {
     if (!c || !out) return FP_ERR_ARG;
     out[0] = (double)c->host_waits;
     out[1] = c->host_wait_s;
+    out[2] = c->host_turn_s;
+    out[3] = c->host_turn_max;
     return FP_OK;
 }
 
@@ -318,6 +333,14 @@ int fp_kernel_stats(fp_ctx* c, fp_kernel_stat* out, int cap) {
         }
         n++;
     }
+    return n;
+}
+
+int64_t fp_kernel_log(fp_ctx* c, fp_launch_rec* out, int64_t cap) {
+    if (!c || (cap > 0 && !out)) return FP_ERR_ARG;
+    stats_resolve(c);
+    const int64_t n = (int64_t)c->log.size();
+    for (int64_t i = 0; i < n && i < cap; i++) out[i] = c->log[i];
     return n;
 }
 

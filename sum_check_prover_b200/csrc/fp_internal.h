@@ -82,9 +82,13 @@ struct fp_ctx {
     int64_t launches = 0;  // every kernel launch of the library on this context
     int64_t host_waits = 0;   // host waits for a device result (sum-check rounds)
     double host_wait_s = 0;   // host seconds spent in those waits
+    double host_turn_s = 0;   // host seconds from a result's arrival to the next posted challenge
+    double host_turn_max = 0;
+    double t_result = -1;     // arrival time of the last result (steady clock seconds), -1: none pending
     std::vector<FpEvPair> ev_live;
     std::vector<cudaEvent_t> ev_free;
     FpKStat stats[K_COUNT];
+    std::vector<fp_launch_rec> log;  // every timed launch since profiling was switched on
 };
 
 struct fp_tx {

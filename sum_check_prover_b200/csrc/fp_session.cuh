@@ -130,4 +130,11 @@ __device__ __forceinline__ void session_publish(FpMailbox* mb, const uint64_t* v
     for (int i = 0; i < n; i++) mb->res[i] = v[i];
 }
 
+template <int N>
+__device__ __forceinline__ void session_publish(FpMailbox* mb, const uint64_t (&v)[N], uint64_t seq) {
+    (void)seq;
+#pragma unroll
+    for (int i = 0; i < N; i++) mb->res[i] = v[i];
+}
+
 #endif

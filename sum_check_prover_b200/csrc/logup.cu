@@ -58,7 +58,7 @@ __device__ __forceinline__ void leaf_den(const KeySrc& K, const Chal& C, int64_t
     int32_t r, q, y;
     key_at(K, i, r, q, y);
     d0 = gl_sub(C.alpha0, gl_from_i64(r));
-    d1 = gl_sub(C.alpha1, gl_add(gl_from_i64(q), gl_mul(C.gamma, gl_from_i64(y))));
+    d1 = gl_sub(C.alpha1, gl_add(gl_from_i64(q), gl_mul_small(C.gamma, y)));
 }
 
 // ---- histograms --------------------------------------------------------------
@@ -255,18 +255,19 @@ struct GkrLayer {
     int t_end;         // the final values (one launch per layer, or one per round)
 };
 
-// F at one pair position for both tables: sum_tau lambda^(2 tau) (pL qR + pR qL + lambda qL qR)
+// F at one pair position for both tables: sum_tau lambda^(2 tau) (pL qR + pR qL + lambda qL qR),
+// each table's term as pL qR + qL (pR + lambda qR) (qR + qL (1 + lambda qR) when p = 1),
+// weakly reduced (it only feeds the product with the eq weight)
 template <bool LEAF>
 __device__ __forceinline__ uint64_t layer_F(const uint64_t (&pl)[2], const uint64_t (&pr)[2], const uint64_t (&ql)[2],
                                             const uint64_t (&qr)[2], uint64_t lam, uint64_t lam2) {
     uint64_t f[2];
 #pragma unroll
     for (int tau = 0; tau < 2; tau++) {
-        const uint64_t qq = gl_mul(ql[tau], qr[tau]);
-        const uint64_t cross = LEAF ? gl_add(qr[tau], ql[tau]) : gl_add(gl_mul(pl[tau], qr[tau]), gl_mul(pr[tau], ql[tau]));
-        f[tau] = gl_add(cross, gl_mul(lam, qq));
+        const uint64_t u = gl_add(LEAF ? 1ull : pr[tau], gl_mul_weak(lam, qr[tau]));
+        f[tau] = gl_muladd_weak(ql[tau], u, LEAF ? qr[tau] : gl_mul_weak(pl[tau], qr[tau]));
     }
-    return gl_add(f[0], gl_mul(lam2, f[1]));
+    return gl_muladd_weak(lam2, f[1], f[0]);
 }
 
 // pair x of the layer's current vectors: from the key columns, or from pp/qq
@@ -290,15 +291,58 @@ __device__ __forceinline__ void layer_pair(const GkrLayer& A, bool from_keys, in
 }
 
 __device__ __forceinline__ ulonglong2 fold2(ulonglong2 a, ulonglong2 b, uint64_t r) {
-    return make_ulonglong2(gl_fold(a.x, b.x, r), gl_fold(a.y, b.y, r));
+    return make_ulonglong2(gl_fold_fast(a.x, b.x, r), gl_fold_fast(a.y, b.y, r));
 }
 
 // Round t of layer d over the pairs b < h handled by this block.
 // t == 1: the vectors as they are. t >= 2: fold the previous round's vectors
 // (length 4h) by rprev first and store the folded halves in place.
+// eq(z_2..z_d, b) of round one, from three shared-memory tables over chunks
+// of b's bits (most significant first, widths w0 >= w1 >= w2 >= 0, each at
+// most 10; a table of width 0 is the single entry 1). Every entry is a
+// product of at most 10 factors, built once per block; each pair then costs
+// two multiplications.
+constexpr int kEqChunk = 10;
+
+struct EqChunks {
+    int w0, w1, w2;
+};
+
+__device__ __forceinline__ EqChunks eq_chunks_build(uint64_t* tab, const uint64_t* zs, int d) {
+    const int nb = d - 1;  // coordinates z_2..z_d, i.e. zs[1..d-1]
+    EqChunks C;
+    C.w0 = nb < kEqChunk ? nb : kEqChunk;
+    C.w1 = nb - C.w0 < kEqChunk ? nb - C.w0 : kEqChunk;
+    C.w2 = nb - C.w0 - C.w1;
+    const int n0 = 1 << C.w0, n1 = 1 << C.w1, n2 = 1 << C.w2;
+    for (int x = threadIdx.x; x < n0 + n1 + n2; x += blockDim.x) {
+        int w, first, y;
+        if (x < n0) {
+            w = C.w0; first = 1; y = x;
+        } else if (x < n0 + n1) {
+            w = C.w1; first = 1 + C.w0; y = x - n0;
+        } else {
+            w = C.w2; first = 1 + C.w0 + C.w1; y = x - n0 - n1;
+        }
+        uint64_t e = 1;
+        for (int i = 0; i < w; i++) e = gl_mul(e, gl_eq1(zs[first + i], (y >> (w - 1 - i)) & 1));
+        tab[x] = e;
+    }
+    __syncthreads();
+    return C;
+}
+
+__device__ __forceinline__ uint64_t eq_chunks_at(const EqChunks& C, const uint64_t* tab, int64_t b) {
+    const int64_t i2 = b & ((1 << C.w2) - 1);
+    const int64_t i1 = (b >> C.w2) & ((1 << C.w1) - 1);
+    const int64_t i0 = b >> (C.w1 + C.w2);
+    return gl_canon(gl_mul_weak(gl_mul_weak(tab[i0], tab[(1 << C.w0) + i1]), tab[(1 << C.w0) + (1 << C.w1) + i2]));
+}
+
 template <bool LEAF>
-__device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* zs, int t, int64_t h, unsigned active,
-                                            uint64_t rprev, uint64_t lam, uint64_t lam2, uint64_t (&acc)[3]) {
+__device__ __forceinline__ void layer_round(const GkrLayer& A, const EqChunks& EC, const uint64_t* eq_tab, int t,
+                                            int64_t h, unsigned active, uint64_t rprev, uint64_t lam, uint64_t lam2,
+                                            bool need1, GlAcc (&acc)[3]) {
     const bool from_keys = LEAF && t <= 2;
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
         ulonglong2 c0p[2], c0q[2], c1p[2], c1q[2];
@@ -306,10 +350,7 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* z
         if (t == 1) {
             layer_pair<LEAF>(A, from_keys, b, c0p, c0q);
             layer_pair<LEAF>(A, from_keys, b + h, c1p, c1q);
-            // E_1[b] = eq(z_2..z_d, b)
-            e = 1;
-            const int nb = A.d - 1;
-            for (int i = 0; i < nb; i++) e = gl_mul(e, gl_eq1(zs[1 + i], (int)((b >> (nb - 1 - i)) & 1)));
+            e = eq_chunks_at(EC, eq_tab, b);  // E_1[b] = eq(z_2..z_d, b)
             if (A.d > 1) A.E[b] = e;
         } else {
             ulonglong2 s0p[2], s0q[2], s1p[2], s1q[2], s2p[2], s2q[2], s3p[2], s3q[2];
@@ -335,32 +376,40 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* z
             e = gl_add(__ldcg(A.E + b), __ldcg(A.E + b + h));
             A.E[b] = e;
         }
+        // h(0) and h(2) always; h(1) only when z_t = 0 (otherwise the host takes it
+        // from the running claim). Products with the eq weight are summed exactly.
         uint64_t pl[2], pr[2], ql[2], qr[2];
 #pragma unroll
-        for (int X = 0; X < 3; X++) {
+        for (int tau = 0; tau < 2; tau++) {
+            pl[tau] = c0p[tau].x; pr[tau] = c0p[tau].y; ql[tau] = c0q[tau].x; qr[tau] = c0q[tau].y;
+        }
+        acc[0].mac(e, layer_F<LEAF>(pl, pr, ql, qr, lam, lam2));
+        if (need1) {
 #pragma unroll
             for (int tau = 0; tau < 2; tau++) {
-                if (X == 0) {
-                    pl[tau] = c0p[tau].x; pr[tau] = c0p[tau].y; ql[tau] = c0q[tau].x; qr[tau] = c0q[tau].y;
-                } else if (X == 1) {
-                    pl[tau] = c1p[tau].x; pr[tau] = c1p[tau].y; ql[tau] = c1q[tau].x; qr[tau] = c1q[tau].y;
-                } else {
-                    pl[tau] = gl_sub(gl_add(c1p[tau].x, c1p[tau].x), c0p[tau].x);
-                    pr[tau] = gl_sub(gl_add(c1p[tau].y, c1p[tau].y), c0p[tau].y);
-                    ql[tau] = gl_sub(gl_add(c1q[tau].x, c1q[tau].x), c0q[tau].x);
-                    qr[tau] = gl_sub(gl_add(c1q[tau].y, c1q[tau].y), c0q[tau].y);
-                }
+                pl[tau] = c1p[tau].x; pr[tau] = c1p[tau].y; ql[tau] = c1q[tau].x; qr[tau] = c1q[tau].y;
             }
-            acc[X] = gl_add(acc[X], gl_mul(e, layer_F<LEAF>(pl, pr, ql, qr, lam, lam2)));
+            acc[2].mac(e, layer_F<LEAF>(pl, pr, ql, qr, lam, lam2));
         }
+#pragma unroll
+        for (int tau = 0; tau < 2; tau++) {
+            if (!LEAF) {
+                pl[tau] = gl_add(gl_sub(c1p[tau].x, c0p[tau].x), c1p[tau].x);
+                pr[tau] = gl_add(gl_sub(c1p[tau].y, c0p[tau].y), c1p[tau].y);
+            }
+            ql[tau] = gl_add(gl_sub(c1q[tau].x, c0q[tau].x), c1q[tau].x);
+            qr[tau] = gl_add(gl_sub(c1q[tau].y, c0q[tau].y), c1q[tau].y);
+        }
+        acc[1].mac(e, layer_F<LEAF>(pl, pr, ql, qr, lam, lam2));
     }
 }
 
 // Rounds [t_begin, t_end] of one layer (t_end > d: and its final child values).
 template <bool LEAF>
-__global__ void __launch_bounds__(LU_THREADS) gkr_layer_kernel(GkrLayer A, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
+__global__ void __launch_bounds__(LU_THREADS, 2) gkr_layer_kernel(GkrLayer A, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
     __shared__ uint64_t zs[32];
     __shared__ uint64_t s_lam;
+    __shared__ uint64_t eq_tab[3 << kEqChunk];
     const int d = A.d;
     if (A.t_begin == 1) {
         // the layer's own challenges: mu (last point coordinate) and lambda
@@ -381,25 +430,21 @@ __global__ void __launch_bounds__(LU_THREADS) gkr_layer_kernel(GkrLayer A, FpMai
     }
     __syncthreads();
     const uint64_t lam = s_lam, lam2 = gl_mul(lam, lam);
-    // eq(z_<t, rho_<t) of the rounds before this launch (their challenges are in zout)
-    uint64_t pre = 1, rprev = 0;
-    for (int i = 1; i + 1 < A.t_begin && i <= d; i++) {
-        const uint64_t r = __ldcg(A.zout + i - 1);
-        pre = gl_mul(pre, gl_add(gl_mul(zs[i - 1], r), gl_mul(gl_sub(1, zs[i - 1]), gl_sub(1, r))));
-    }
+    uint64_t rprev = 0;
     for (int t = A.t_begin; t <= d && t <= A.t_end; t++) {
         if (t > 1) {
             if (!session_wait(mb, rl, A.seq0 + t - 1, rprev)) return;
-            const uint64_t zp = zs[t - 2];
-            pre = gl_mul(pre, gl_add(gl_mul(zp, rprev), gl_mul(gl_sub(1, zp), gl_sub(1, rprev))));
             if (blockIdx.x == 0 && threadIdx.x == 0) A.zout[t - 2] = rprev;
         }
         const int64_t h = 1ll << (d - t);
         int64_t want = (h + A.per_block - 1) / A.per_block;
         const unsigned active = (unsigned)(want < 1 ? 1 : (want > A.grid ? A.grid : want));
         if (blockIdx.x >= active) return;  // this block has no pairs in this or any later round
-        uint64_t acc[3] = {0, 0, 0};
-        layer_round<LEAF>(A, zs, t, h, active, rprev, lam, lam2, acc);
+        EqChunks EC{0, 0, 0};
+        if (t == 1) EC = eq_chunks_build(eq_tab, zs, d);
+        GlAcc sums[3];
+        layer_round<LEAF>(A, EC, eq_tab, t, h, active, rprev, lam, lam2, zs[t - 1] == 0, sums);
+        uint64_t acc[3] = {sums[0].value(), sums[1].value(), sums[2].value()};
         bool last;
         if (active == 1) {
             block_sum_gl<3>(acc);
@@ -407,19 +452,9 @@ __global__ void __launch_bounds__(LU_THREADS) gkr_layer_kernel(GkrLayer A, FpMai
         } else {
             last = grid_sum_gl_n<3>(acc, part, &rl->ticket, active);
         }
-        if (last && threadIdx.x == 0) {
-            // g(X) = eq(z_<t, rho_<t) eq(z_t, X) h(X); h has degree 2, h(3) by finite differences
-            const uint64_t zt = zs[t - 1];
-            const uint64_t one_m = gl_sub(1, zt), slope = gl_sub(gl_add(zt, zt), 1);
-            const uint64_t e2 = gl_add(one_m, gl_add(slope, slope)), e3 = gl_add(e2, slope);
-            const uint64_t h3 = gl_add(gl_sub(gl_add(gl_add(acc[2], acc[2]), acc[2]), gl_add(gl_add(acc[1], acc[1]), acc[1])), acc[0]);
-            uint64_t g[4];
-            g[0] = gl_mul(pre, gl_mul(one_m, acc[0]));
-            g[1] = gl_mul(pre, gl_mul(zt, acc[1]));
-            g[2] = gl_mul(pre, gl_mul(e2, acc[2]));
-            g[3] = gl_mul(pre, gl_mul(e3, h3));
-            session_publish(mb, g, 4, A.seq0 + t);
-        }
+        // {h(0), h(2), h(1) or 0} of h(X) = sum_b eq(z_>t, b) F(rho_<t, X, b); the host
+        // forms g(X) = eq(z_<t, rho_<t) eq(z_t, X) h(X)
+        if (last && threadIdx.x == 0) session_publish(mb, acc, A.seq0 + t);
     }
     // only block 0 is left: fold the last pair by the last challenge
     if (A.t_end <= d || blockIdx.x != 0) return;
@@ -461,6 +496,17 @@ __global__ void __launch_bounds__(LU_THREADS) leaf_eval_kernel(KeySrc K, const u
         out[1] = acc[1];
         out[2] = acc[2];
     }
+}
+
+// Algorithmic bytes of round t of a layer with h pairs: the pair vectors
+// (p and q of both tables, 16 B per pair entry; the leaf layer has only q and
+// reads its first two rounds from the keys, 9 B per key), read at 2 (t = 1)
+// or 4 positions and written at 2, plus the suffix eq table.
+double gkr_round_bytes(bool leaf, int t, double h) {
+    const double entry = leaf ? 32.0 : 64.0;  // one position of all pair vectors
+    if (t == 1) return (leaf ? 4 * 9.0 : 2 * entry) * h + 8.0 * h;
+    if (leaf && t == 2) return 8 * 9.0 * h + 2 * entry * h + 24.0 * h;
+    return 4 * entry * h + 2 * entry * h + 24.0 * h;
 }
 
 void put_le(uint8_t* p, uint64_t v, int nb) {
@@ -699,21 +745,66 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
             A.t_end = d + 1;
             void* args[] = {&A, &c->mb_dev, &c->relay, &part};
             const bool leaf = (d == v - 1);
+            double bytes = 0;
+            for (int t = 1; t <= d; t++) bytes += gkr_round_bytes(leaf, t, (double)(1ll << (d - t)));
             int slot;
-            fp_tic(c, st, K_GKR_ROUND, (leaf ? 36.0 : 128.0) * (double)(1ll << d), &slot);
+            fp_tic(c, st, K_GKR_ROUND, bytes, &slot);
             FP_CUDA(c, cudaLaunchCooperativeKernel(leaf ? (const void*)gkr_layer_kernel<true>
                                                         : (const void*)gkr_layer_kernel<false>,
                                                    dim3(A.grid), dim3(A.threads), args, 0, st));
             fp_toc(c, st, slot);
         }
     }
+    // The host assembles each round polynomial g(X) = pre eq(z_t, X) h(X) from the
+    // device's h(0), h(2): g(1) follows from the running claim (g(0) + g(1) = claim),
+    // h(1) = g(1) / (pre z_t) gives g(3) through h(3) = h(0) - 3 h(1) + 3 h(2).
+    // The next claim is g(rho_t) (Lagrange on the nodes 0..3).
+    static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
+    auto lagrange4 = [](const uint64_t g[4], uint64_t r) {
+        const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2), r3 = gl_sub(r, 3);
+        const uint64_t l0 = gl_sub(0, gl_mul(gl_mul(r1, r2), gl_mul(r3, inv6)));
+        const uint64_t l1 = gl_mul(gl_mul(r, r2), gl_mul(r3, inv2));
+        const uint64_t l2 = gl_sub(0, gl_mul(gl_mul(r, r1), gl_mul(r3, inv2)));
+        const uint64_t l3 = gl_mul(gl_mul(r, r1), gl_mul(r2, inv6));
+        return gl_add(gl_add(gl_mul(g[0], l0), gl_mul(g[1], l1)), gl_add(gl_mul(g[2], l2), gl_mul(g[3], l3)));
+    };
+    uint64_t prev[8];  // the two-node layer's values, then each layer's child values at its point
+    memcpy(prev, hsmall, sizeof prev);
+    std::vector<uint64_t> zpt, rhos, zinv;
     uint64_t mu = z.z[0];
     for (int d = 1; d <= v - 1; d++) {
         GkrLayer A = layers[d - 1];
         const bool leaf = (d == v - 1);
         const void* kern = leaf ? (const void*)gkr_layer_kernel<true> : (const void*)gkr_layer_kernel<false>;
         const uint64_t lam = fp_tx_squeeze_one(tx, "gkr_lambda");
-        fp_session_expect(c, d >= 1 ? 4 : 8);
+        // point (previous rounds' challenges, mu) and claim sum_tau lam^(2 tau) (p~_tau + lam q~_tau)
+        zpt = rhos;
+        zpt.push_back(mu);
+        rhos.clear();
+        uint64_t claim = 0, lp = 1;
+        for (int tau = 0; tau < 2; tau++) {
+            const uint64_t pz = gl_fold(prev[4 * tau], prev[4 * tau + 1], mu);
+            const uint64_t qz = gl_fold(prev[4 * tau + 2], prev[4 * tau + 3], mu);
+            claim = gl_add(claim, gl_mul(lp, gl_add(pz, gl_mul(lam, qz))));
+            lp = gl_mul(lam, lam);
+        }
+        // 1 / z_t for every coordinate at once (zero coordinates are left to the device)
+        zinv.assign(d, 0);
+        {
+            uint64_t run = 1;
+            for (int i = 0; i < d; i++) {
+                zinv[i] = run;
+                if (zpt[i]) run = gl_mul(run, zpt[i]);
+            }
+            uint64_t inv = gl_inv(run);
+            for (int i = d - 1; i >= 0; i--) {
+                if (!zpt[i]) continue;
+                zinv[i] = gl_mul(zinv[i], inv);
+                inv = gl_mul(inv, zpt[i]);
+            }
+        }
+        uint64_t pre = 1;
+        fp_session_expect(c, 3);
         fp_session_post2(c, A.seq0, mu, lam);
         for (int t = 1; t <= d + 1; t++) {
             if (c->stepped) {
@@ -723,7 +814,7 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
                 const int64_t h = t <= d ? 1ll << (d - t) : 0;
                 int slot;
                 if (t <= d)
-                    fp_tic(c, st, K_GKR_ROUND, (leaf && t <= 2 ? 36.0 : 128.0) * h * (t == 1 ? 1 : 2) + 24.0 * h, &slot);
+                    fp_tic(c, st, K_GKR_ROUND, gkr_round_bytes(leaf, t, (double)h), &slot);
                 else
                     fp_tic(c, st, K_GKR_FINAL, 128.0, &slot);
                 FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(t <= d ? A.grid : 1), dim3(A.threads), args, 0, st));
@@ -731,13 +822,30 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
             }
             if ((rc = fp_session_wait(c, A.seq0 + t, st))) return rc;
             if (t <= d) {
-                for (int i = 0; i < 4; i++) put_le(proof + pos + 8 * i, c->mb->res[i], 8);
+                const uint64_t h0 = c->mb->res[0], h2 = c->mb->res[1], h1 = c->mb->res[2];
+                const uint64_t zt = zpt[t - 1];
+                const uint64_t ph0 = gl_mul(pre, h0), ph2 = gl_mul(pre, h2);
+                uint64_t g[4];
+                g[0] = gl_mul(gl_sub(1, zt), ph0);
+                g[1] = gl_sub(claim, g[0]);
+                const uint64_t ph1 = zt ? gl_mul(g[1], zinv[t - 1]) : gl_mul(pre, h1);
+                g[2] = gl_mul(gl_sub(gl_add(zt, gl_add(zt, zt)), 1), ph2);                  // eq(z_t, 2) = 3 z_t - 1
+                const uint64_t ph3 = gl_add(gl_sub(ph0, gl_add(ph1, gl_add(ph1, ph1))), gl_add(ph2, gl_add(ph2, ph2)));
+                g[3] = gl_mul(gl_sub(gl_add(gl_add(zt, zt), gl_add(zt, gl_add(zt, zt))), 2), ph3);  // 5 z_t - 2
+                for (int i = 0; i < 4; i++) put_le(proof + pos + 8 * i, g[i], 8);
                 fp_tx_absorb_raw(tx, "gkr_round", proof + pos, 32);
                 pos += 32;
-                fp_session_expect(c, t < d ? 4 : 8);  // the last challenge triggers the final values
-                fp_session_post(c, A.seq0 + t, fp_tx_squeeze_one(tx, "gkr_chal"));
+                fp_session_expect(c, t < d ? 3 : 8);  // the last challenge triggers the final values
+                const uint64_t r = fp_tx_squeeze_one(tx, "gkr_chal");
+                fp_session_post(c, A.seq0 + t, r);
+                claim = lagrange4(g, r);
+                pre = gl_mul(pre, gl_add(gl_mul(zt, r), gl_mul(gl_sub(1, zt), gl_sub(1, r))));
+                rhos.push_back(r);
             } else {
-                for (int i = 0; i < 8; i++) put_le(proof + pos + 8 * i, c->mb->res[i], 8);
+                for (int i = 0; i < 8; i++) {
+                    prev[i] = c->mb->res[i];
+                    put_le(proof + pos + 8 * i, prev[i], 8);
+                }
                 fp_tx_absorb_raw(tx, "gkr_final", proof + pos, 64);
                 pos += 64;
                 mu = fp_tx_squeeze_one(tx, "gkr_mu");
@@ -745,11 +853,7 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
         }
     }
     // the leaf point: the last layer's round challenges, then its mu
-    if (v >= 2) {
-        FP_CUDA(c, cudaMemcpyAsync(hsmall, zb[v & 1], 8 * (size_t)(v - 1), cudaMemcpyDeviceToHost, st));
-        FP_CUDA(c, cudaStreamSynchronize(st));
-        for (int i = 0; i < v - 1; i++) z.z[i] = hsmall[i];
-    }
+    for (int i = 0; i < v - 1; i++) z.z[i] = rhos[i];
     z.z[v - 1] = mu;
     z.v = v;
 

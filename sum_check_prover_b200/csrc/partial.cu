@@ -41,8 +41,9 @@ struct PeJob {
 };
 
 constexpr int PE_THREADS = 256;              // 8 warps share the block's columns, split its rows
-constexpr int PE_COLS = 16;                  // columns per lane
-constexpr int PE_BLOCK_COLS = 32 * PE_COLS;  // 512 columns per block
+constexpr int PE_COLS = 8;                   // columns per lane: one 32-bit (int4) or 64-bit (int8) load per row
+constexpr int PE_BLOCK_COLS = 32 * PE_COLS;  // 256 columns per block
+constexpr int PE_UNROLL = 8;                 // rows whose loads a warp issues before using any of them
 constexpr int PE_MAX_ROWS = 256;             // 256 rows x 2^32 x 2^15 < 2^64: the sums stay exact
 
 __device__ __forceinline__ uint64_t fold_lohi(uint64_t lo, uint64_t hi) {
@@ -62,7 +63,7 @@ __device__ __forceinline__ int find_job(const PeJob* jobs, int njobs, int64_t b)
 }
 
 template <bool W4, bool SCALED>
-__global__ void __launch_bounds__(PE_THREADS) partial_many_kernel(const PeJob* __restrict__ jobs, int njobs) {
+__global__ void __launch_bounds__(PE_THREADS, 3) partial_many_kernel(const PeJob* __restrict__ jobs, int njobs) {
     __shared__ uint64_t eqs[PE_MAX_ROWS];
     __shared__ uint64_t red[2][8][PE_BLOCK_COLS / 2];
     __shared__ uint64_t wsum[8];
@@ -96,50 +97,68 @@ __global__ void __launch_bounds__(PE_THREADS) partial_many_kernel(const PeJob* _
     uint64_t lo[PE_COLS], hi[PE_COLS];
 #pragma unroll
     for (int c = 0; c < PE_COLS; c++) lo[c] = hi[c] = 0;
-    if (col0 < J.cols) {
+    if (col0 < J.cols && J.aligned) {
+        // u = M_eff + off >= 0 from the stored bits: an int4 nibble n holds w = n - 16 [n >= 8],
+        // so n ^ 8 = w + 8; an int8 byte b gives b ^ 0x80 = w + 128. With a scale s,
+        // w s + off = (n ^ 8) s + (off - 8 s) (int4) or (b ^ 0x80) s + (off - 128 s) (int8).
+        const uint8_t* base = J.mat + (int64_t)r0 * pitch + (W4 ? (col0 >> 1) : col0);
+        for (int kb = warp; kb < nr; kb += (PE_THREADS / 32) * PE_UNROLL) {
+            uint32_t wv[PE_UNROLL][W4 ? 1 : 2];
+            int32_t sv[PE_UNROLL];
+            uint64_t ev[PE_UNROLL];
+#pragma unroll
+            for (int u = 0; u < PE_UNROLL; u++) {
+                const int k = kb + (PE_THREADS / 32) * u;
+                const bool in = k < nr;
+                const uint8_t* rp = base + (int64_t)(in ? k : 0) * pitch;
+                if (W4) {
+                    wv[u][0] = in ? __ldcs(reinterpret_cast<const uint32_t*>(rp)) : 0u;
+                } else {
+                    const uint2 q = in ? __ldcs(reinterpret_cast<const uint2*>(rp)) : make_uint2(0, 0);
+                    wv[u][0] = q.x;
+                    wv[u][W4 ? 0 : 1] = q.y;
+                }
+                sv[u] = SCALED && in ? (int32_t)__ldg(J.scales + (int64_t)(r0 + k) * G + (col0 >> 6)) : 1;
+                ev[u] = in ? eqs[k] : 0ull;  // rows past the end weigh nothing
+            }
+#pragma unroll
+            for (int u = 0; u < PE_UNROLL; u++) {
+                const uint32_t el = (uint32_t)ev[u], eh = (uint32_t)(ev[u] >> 32);
+                const int32_t sc = sv[u];
+                const uint32_t base_u = SCALED ? (uint32_t)((int32_t)off - (W4 ? 8 : 128) * sc) : 0u;
+#pragma unroll
+                for (int c = 0; c < PE_COLS; c++) {
+                    uint32_t n;
+                    if (W4)
+                        n = ((wv[u][0] ^ 0x88888888u) >> (4 * c)) & 15u;
+                    else
+                        n = ((wv[u][c >> 2] ^ 0x80808080u) >> (8 * (c & 3))) & 255u;
+                    const uint32_t uu = SCALED ? n * (uint32_t)sc + base_u : n;
+                    lo[c] += (uint64_t)el * uu;
+                    hi[c] += (uint64_t)eh * uu;
+                }
+            }
+        }
+    } else if (col0 < J.cols) {
         for (int k = warp; k < nr; k += PE_THREADS / 32) {
             const int64_t i = r0 + k;
             const uint64_t e = eqs[k];
             const uint32_t el = (uint32_t)e, eh = (uint32_t)(e >> 32);
-            int32_t w[PE_COLS];
-            if (J.aligned) {
-                // 16 columns never straddle a 64-column scale group
-                const int32_t sc = SCALED ? (int32_t)__ldg(J.scales + i * G + (col0 >> 6)) : 1;
-                if (W4) {
-                    const uint2 q = __ldg(reinterpret_cast<const uint2*>(J.mat + i * pitch + (col0 >> 1)));
-                    const uint64_t bb = ((uint64_t)q.y << 32) | q.x;
-#pragma unroll
-                    for (int c = 0; c < PE_COLS; c++) {
-                        const int n = (int)((bb >> (4 * c)) & 15);
-                        w[c] = (n >= 8 ? n - 16 : n) * sc;
-                    }
-                } else {
-                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(J.mat + i * pitch + col0));
-                    const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                    for (int c = 0; c < PE_COLS; c++) w[c] = (int32_t)(int8_t)(wd[c >> 2] >> (8 * (c & 3))) * sc;
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < PE_COLS; c++) {
-                    const int cc = col0 + c;
-                    int x = 0;
-                    if (cc < J.cols) {
-                        if (W4) {
-                            const uint8_t bt = J.mat[i * pitch + (cc >> 1)];
-                            const int n = (cc & 1) ? (bt >> 4) : (bt & 15);
-                            x = n >= 8 ? n - 16 : n;
-                        } else {
-                            x = (int8_t)J.mat[i * pitch + cc];
-                        }
-                        if (SCALED) x *= (int32_t)__ldg(J.scales + i * G + (cc >> 6));
-                    }
-                    w[c] = x;
-                }
-            }
 #pragma unroll
             for (int c = 0; c < PE_COLS; c++) {
-                const uint32_t u = (uint32_t)(w[c] + (int32_t)off);
+                const int cc = col0 + c;
+                int x = 0;
+                if (cc < J.cols) {
+                    if (W4) {
+                        const uint8_t bt = J.mat[i * pitch + (cc >> 1)];
+                        const int n = (cc & 1) ? (bt >> 4) : (bt & 15);
+                        x = n >= 8 ? n - 16 : n;
+                    } else {
+                        x = (int8_t)J.mat[i * pitch + cc];
+                    }
+                    if (SCALED) x *= (int32_t)__ldg(J.scales + i * G + (cc >> 6));
+                }
+                const uint32_t u = (uint32_t)(x + (int32_t)off);
                 lo[c] += (uint64_t)el * u;
                 hi[c] += (uint64_t)eh * u;
             }
@@ -236,8 +255,9 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         d.v = q.v;
         pe_plan(c->num_sms, q.rows, q.cols, d.col_blocks, d.rows_per_block, d.splits);
         const int64_t pitch = q.bits == 4 ? (q.cols + 1) / 2 : q.cols;
+        // the fast path loads 4 (int4) or 8 (int8) bytes per lane and row
         d.aligned = ((uintptr_t)q.mat % 16 == 0) && (q.cols % PE_COLS == 0) &&
-                    (q.bits == 4 ? (pitch % 8 == 0) : (pitch % 16 == 0));
+                    (q.bits == 4 ? (pitch % 4 == 0) : (pitch % 8 == 0));
         d.pad = 0;
         d.first_block = 0;
         d.part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * d.splits * q.cols);

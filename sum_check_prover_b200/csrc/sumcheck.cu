@@ -42,7 +42,7 @@ struct ScArgs {
 // previous round's vectors (length 4 half per site), folded by the previous
 // challenge on the fly, the folded halves going to the other buffer.
 template <bool MULTI>
-__global__ void __launch_bounds__(SC_THREADS) sc_session_kernel(ScArgs P, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
+__global__ void __launch_bounds__(SC_THREADS, 3) sc_session_kernel(ScArgs P, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
     uint64_t rprev = 0;
     for (int t = P.t_begin; t <= P.n && t <= P.t_end; t++) {
         if (t > 1 && !session_wait(mb, rl, P.seq0 + t - 1, rprev)) return;
@@ -53,20 +53,40 @@ __global__ void __launch_bounds__(SC_THREADS) sc_session_kernel(ScArgs P, FpMail
         const unsigned active = (unsigned)(want < 1 ? 1 : (want > P.grid ? P.grid : want));
         if (blockIdx.x >= active) return;
         const bool fold = t > 1;
-        const uint64_t* Ain = fold ? P.A[t & 1] : P.A[0];
-        const uint64_t* Bin = fold ? P.B[t & 1] : P.B[0];
-        uint64_t* Aout = P.A[1 - (t & 1)];
-        uint64_t* Bout = P.B[1 - (t & 1)];
-        uint64_t acc[3] = {0, 0, 0};
-        for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < npairs; p += (int64_t)active * blockDim.x) {
+        // ping-pong by round parity (selects, not a dynamic index into the parameter struct)
+        const bool odd = t & 1;
+        const uint64_t* Ain = (fold && odd) ? P.A[1] : P.A[0];
+        const uint64_t* Bin = (fold && odd) ? P.B[1] : P.B[0];
+        uint64_t* Aout = odd ? P.A[0] : P.A[1];
+        uint64_t* Bout = odd ? P.B[0] : P.B[1];
+        // each block takes a contiguous range of pairs (its threads stride through it, so
+        // loads stay coalesced and a thread meets few site boundaries): products are
+        // summed exactly per site and weighted by rho_s once per site
+        const int64_t chunk = ((npairs + active - 1) / active + blockDim.x - 1) / blockDim.x * blockDim.x;
+        const int64_t pbeg = (int64_t)blockIdx.x * chunk;
+        const int64_t pend = pbeg + chunk < npairs ? pbeg + chunk : npairs;
+        GlAcc s0, s2;               // current site's sums of A(0)B(0) and A(2)B(2)
+        GlAcc w0, w2;               // rho-weighted sums over finished sites (MULTI)
+        int64_t scur = -1;
+        for (int64_t p = pbeg + threadIdx.x; p < pend; p += blockDim.x) {
             const int64_t s = p >> logh, b = p & (half - 1);
+            if (MULTI && s != scur) {
+                if (scur >= 0) {
+                    const uint64_t rs = __ldg(P.rho + scur);
+                    w0.mac(s0.value(), rs);
+                    w2.mac(s2.value(), rs);
+                    s0 = GlAcc();
+                    s2 = GlAcc();
+                }
+                scur = s;
+            }
             uint64_t a0, a1, b0, b1;
             if (fold) {
                 const int64_t bi = s * 4 * half + b;
-                a0 = gl_fold(__ldcg(Ain + bi), __ldcg(Ain + bi + 2 * half), rprev);
-                a1 = gl_fold(__ldcg(Ain + bi + half), __ldcg(Ain + bi + 3 * half), rprev);
-                b0 = gl_fold(__ldcg(Bin + bi), __ldcg(Bin + bi + 2 * half), rprev);
-                b1 = gl_fold(__ldcg(Bin + bi + half), __ldcg(Bin + bi + 3 * half), rprev);
+                a0 = gl_fold_fast(__ldcg(Ain + bi), __ldcg(Ain + bi + 2 * half), rprev);
+                a1 = gl_fold_fast(__ldcg(Ain + bi + half), __ldcg(Ain + bi + 3 * half), rprev);
+                b0 = gl_fold_fast(__ldcg(Bin + bi), __ldcg(Bin + bi + 2 * half), rprev);
+                b1 = gl_fold_fast(__ldcg(Bin + bi + half), __ldcg(Bin + bi + 3 * half), rprev);
                 const int64_t bo = s * 2 * half + b;
                 Aout[bo] = a0;
                 Aout[bo + half] = a1;
@@ -79,33 +99,40 @@ __global__ void __launch_bounds__(SC_THREADS) sc_session_kernel(ScArgs P, FpMail
                 b0 = __ldcg(Bin + bi);
                 b1 = __ldcg(Bin + bi + half);
             }
-            const uint64_t a2 = gl_sub(gl_add(a1, a1), a0);
-            const uint64_t b2 = gl_sub(gl_add(b1, b1), b0);
-            uint64_t t0 = gl_mul(a0, b0), t1 = gl_mul(a1, b1), t2 = gl_mul(a2, b2);
-            if (MULTI) {
-                const uint64_t rs = P.rho[s];
-                t0 = gl_mul(t0, rs);
-                t1 = gl_mul(t1, rs);
-                t2 = gl_mul(t2, rs);
+            // g(0) and g(2); the host takes g(1) from the running claim. The value at 2 only
+            // feeds a product, so it may stay weakly reduced.
+            const uint64_t a2 = gl_add(gl_sub(a1, a0), a1);
+            const uint64_t b2 = gl_add(gl_sub(b1, b0), b1);
+            s0.mac(a0, b0);
+            s2.mac(a2, b2);
+        }
+        uint64_t acc[2];
+        if (MULTI) {
+            if (scur >= 0) {
+                const uint64_t rs = __ldg(P.rho + scur);
+                w0.mac(s0.value(), rs);
+                w2.mac(s2.value(), rs);
             }
-            acc[0] = gl_add(acc[0], t0);
-            acc[1] = gl_add(acc[1], t1);
-            acc[2] = gl_add(acc[2], t2);
+            acc[0] = w0.value();
+            acc[1] = w2.value();
+        } else {
+            acc[0] = s0.value();
+            acc[1] = s2.value();
         }
         bool last;
         if (active == 1) {
-            block_sum_gl<3>(acc);
+            block_sum_gl<2>(acc);
             last = true;
         } else {
-            last = grid_sum_gl_n<3>(acc, part, &rl->ticket, active);
+            last = grid_sum_gl_n<2>(acc, part, &rl->ticket, active);
         }
-        if (last && threadIdx.x == 0) session_publish(mb, acc, 3, P.seq0 + t);
+        if (last && threadIdx.x == 0) session_publish(mb, acc, P.seq0 + t);
     }
     if (P.t_end <= P.n || blockIdx.x != 0) return;
     if (!session_wait(mb, rl, P.seq0 + P.n, rprev)) return;
     // the round-n vectors (length 2 per site) sit in A[0] when n == 1, else in the round's output buffer
-    const uint64_t* Af = P.n == 1 ? P.A[0] : P.A[1 - (P.n & 1)];
-    const uint64_t* Bf = P.n == 1 ? P.B[0] : P.B[1 - (P.n & 1)];
+    const uint64_t* Af = (P.n == 1 || (P.n & 1)) ? P.A[0] : P.A[1];
+    const uint64_t* Bf = (P.n == 1 || (P.n & 1)) ? P.B[0] : P.B[1];
     for (int s = threadIdx.x; s < P.nsites; s += blockDim.x) {
         P.fin[2 * s] = gl_fold(__ldcg(Af + 2 * s), __ldcg(Af + 2 * s + 1), rprev);
         P.fin[2 * s + 1] = gl_fold(__ldcg(Bf + 2 * s), __ldcg(Bf + 2 * s + 1), rprev);
@@ -225,6 +252,7 @@ int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites
     FP_CUDA(c, cudaMemcpyAsync(hbuf, dclaims, 8 * (size_t)nsites, cudaMemcpyDeviceToHost, st));
     FP_CUDA(c, cudaStreamSynchronize(st));
     size_t pos = 0;
+    std::vector<uint64_t> hclaims(hbuf, hbuf + nsites);
     put_u64s(proof + pos, hbuf, nsites);
     fp_tx_absorb_raw(tx, "claims", proof + pos, 8 * (size_t)nsites);
     pos += 8 * (size_t)nsites;
@@ -275,14 +303,19 @@ int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites
         P.grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)std::max(1, occ) * c->num_sms));
         P.seq0 = fp_seq_reserve(c, n + 2);
         if ((rc = fp_session_begin(c, st))) return rc;
-        fp_session_expect(c, 3);  // round 1 publishes without a challenge
+        static const uint64_t inv2 = gl_inv(2);
+        uint64_t claim = 0;  // sum_s rho_s c_s, then g_t(r_t) after each round
+        for (int s = 0; s < nsites; s++) claim = gl_add(claim, gl_mul(rho[s], hclaims[s]));
+        fp_session_expect(c, 2);  // round 1 publishes without a challenge
         void* args[] = {&P, &c->mb_dev, &c->relay, &part};
         const void* kern = nsites > 1 ? (const void*)sc_session_kernel<true> : (const void*)sc_session_kernel<false>;
         if (!c->stepped) {
             P.t_begin = 1;
             P.t_end = n + 1;
             int slot;
-            fp_tic(c, st, K_SC_ROUND, 32.0 * nsites * L + 48.0 * nsites * L / 2, &slot);
+            // round 1 reads A, B (16 B per element); each later round reads 4 and writes 2 values of
+            // both vectors per pair (96 B), over S L / 2^t pairs: 64 S L bytes in all
+            fp_tic(c, st, K_SC_ROUND, 64.0 * nsites * L, &slot);
             FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(P.grid), dim3(SC_THREADS), args, 0, st));
             fp_toc(c, st, slot);
         }
@@ -291,17 +324,23 @@ int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites
                 P.t_begin = P.t_end = t;
                 const double pairs = (double)nsites * (double)(1ll << (n - t));
                 int slot;
-                fp_tic(c, st, K_SC_ROUND, t == 1 ? 32.0 * pairs : 48.0 * pairs, &slot);
+                fp_tic(c, st, K_SC_ROUND, t == 1 ? 32.0 * pairs : 96.0 * pairs, &slot);
                 FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(P.grid), dim3(SC_THREADS), args, 0, st));
                 fp_toc(c, st, slot);
             }
             if ((rc = fp_session_wait(c, P.seq0 + t, st))) return rc;
-            uint64_t g[3] = {c->mb->res[0], c->mb->res[1], c->mb->res[2]};
+            // g(1) = claim - g(0); the next claim is g(r) (Lagrange on the nodes 0, 1, 2)
+            uint64_t g[3] = {c->mb->res[0], 0, c->mb->res[1]};
+            g[1] = gl_sub(claim, g[0]);
             put_u64s(proof + pos, g, 3);
             fp_tx_absorb_raw(tx, "sc_round", proof + pos, 24);
             pos += 24;
-            fp_session_expect(c, t < n ? 3 : 1);  // the last challenge triggers the final values
-            fp_session_post(c, P.seq0 + t, fp_tx_squeeze_one(tx, "sc_chal"));
+            fp_session_expect(c, t < n ? 2 : 1);  // the last challenge triggers the final values
+            const uint64_t r = fp_tx_squeeze_one(tx, "sc_chal");
+            fp_session_post(c, P.seq0 + t, r);
+            const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2);
+            claim = gl_add(gl_add(gl_mul(g[0], gl_mul(gl_mul(r1, r2), inv2)), gl_sub(0, gl_mul(g[1], gl_mul(r, r2)))),
+                           gl_mul(g[2], gl_mul(gl_mul(r, r1), inv2)));
         }
         if (c->stepped) {
             P.t_begin = P.t_end = n + 1;
