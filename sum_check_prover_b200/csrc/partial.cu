@@ -11,11 +11,19 @@
 // Lo + 2^32 Hi - off * (sum of the block's eq values). int4 nibbles are
 // unpacked in registers.
 //
-// All contractions of a call go into one launch per operand variant (a job
-// list; the MoE layer has hundreds of sites): a block owns 512 columns x up
-// to 256 rows of one job, its 8 warps split the rows, and their sums meet in
-// shared memory. eq(z, i) for the block's rows is computed in the block from
-// the point, so no eq table is materialised.
+// Tensor-core path (matrices whose rows hold whole 32-byte warp slices): the
+// field weights are split into 8 byte limbs, e = sum_l e_l 2^(8 l), and
+// C[l][c] = sum_i e_l[i] u[i][c] is an exact u8 x u8 -> s32 matrix product
+// (mma m16n8k32, limbs as the A rows, matrix rows as K, columns as N). Each
+// lane loads one 32-bit word from each of 4 consecutive rows and transposes
+// the 4 x 4 bytes with byte permutes into B fragments; int4 nibbles split into
+// two fragments. The limbs are recombined mod p once per block. With scales,
+// the weight of row i in column group g is e_i s[i][g] (a warp's columns lie
+// in one group), so the unsigned operand stays w + off.
+//
+// All contractions of a call go into one launch per kernel variant (a job
+// list; the MoE layer has hundreds of sites). eq(z, i) for the block's rows
+// is computed in the block from the point, so no eq table is materialised.
 #include <string.h>
 
 #include <algorithm>
@@ -45,6 +53,27 @@ constexpr int PE_COLS = 8;                   // columns per lane: one 32-bit (in
 constexpr int PE_BLOCK_COLS = 32 * PE_COLS;  // 256 columns per block
 constexpr int PE_UNROLL = 8;                 // rows whose loads a warp issues before using any of them
 constexpr int PE_MAX_ROWS = 256;             // 256 rows x 2^32 x 2^15 < 2^64: the sums stay exact
+
+__device__ __forceinline__ void mma_u8(uint32_t (&c)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    // A rows 8..15 (a1, a3) are zero: only 8 limbs; their outputs are discarded
+    uint32_t d2, d3;
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};\n"
+        : "=r"(c[0]), "=r"(c[1]), "=r"(d2), "=r"(d3)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]), "r"(0u), "r"(0u));
+    (void)d2;
+    (void)d3;
+}
+
+// rows w[0..3] -> t[j] = byte j of each row (row r in byte r)
+__device__ __forceinline__ void transpose4x4(const uint32_t* w, uint32_t* t) {
+    const uint32_t x0 = __byte_perm(w[0], w[1], 0x5140), x1 = __byte_perm(w[0], w[1], 0x7362);
+    const uint32_t x2 = __byte_perm(w[2], w[3], 0x5140), x3 = __byte_perm(w[2], w[3], 0x7362);
+    t[0] = __byte_perm(x0, x2, 0x5410);
+    t[1] = __byte_perm(x0, x2, 0x7632);
+    t[2] = __byte_perm(x1, x3, 0x5410);
+    t[3] = __byte_perm(x1, x3, 0x7632);
+}
 
 __device__ __forceinline__ uint64_t fold_lohi(uint64_t lo, uint64_t hi) {
     return gl_add(gl_canon(lo), gl_mul_2_32(gl_canon(hi)));
@@ -189,6 +218,160 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_many_kernel(const PeJob
     }
 }
 
+// Tensor-core partial evaluation. A warp owns 32 bytes of every row (64 int4 or
+// 32 int8 columns); 8 warps side by side, up to tc_rows<SCALED>() rows per block.
+//
+// eq(z, i) of the block's rows comes from two small tables: with i = 32 m + n,
+// eq(z, i) = H[m - m0] T[n], H over the high coordinates of the block's row
+// groups and T over the last five coordinates; one product per row.
+template <bool SCALED>
+__host__ __device__ constexpr int tc_rows() {
+    return SCALED ? 256 : 2048;  // exact s32 sums: 2048 x 255 x 255 < 2^31
+}
+
+template <bool W4, bool SCALED>
+__global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* __restrict__ jobs, int njobs) {
+    constexpr int WCOLS = W4 ? 64 : 32;
+    constexpr int NG = W4 ? 8 : 4;  // mma column groups per lane
+    constexpr int ROWS = tc_rows<SCALED>();
+    // limb l of row k's weight: one table for all warps, or one per warp (scaled: the weight
+    // depends on the warp's column group)
+    __shared__ __align__(16) uint8_t et[SCALED ? 8 : 1][8][ROWS];
+    __shared__ uint64_t eqs[SCALED ? ROWS : 1];
+    __shared__ uint64_t htab[ROWS / 32], ttab[32];
+    __shared__ uint64_t wsum[8];
+    __shared__ uint32_t red[8][64 * 8];  // per warp: [column][limb]
+    const PeJob J = jobs[find_job(jobs, njobs, blockIdx.x)];
+    const int64_t lb = blockIdx.x - J.first_block;
+    const int cb = (int)(lb % J.col_blocks), split = (int)(lb / J.col_blocks);
+    const int r0 = split * J.rows_per_block;  // a multiple of 32
+    const int nr = min(J.rows_per_block, J.rows - r0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+    const int wc0 = (cb * (PE_THREADS / 32) + warp) * WCOLS;
+    const bool wactive = wc0 < J.cols;
+    const int64_t pitch = W4 ? J.cols / 2 : J.cols;
+    const int G = (J.cols + 63) / 64;
+
+    // the two eq tables (v < 5: T covers every coordinate and H is the single entry 1)
+    const int tb = J.v < 5 ? J.v : 5;  // coordinates in T (the last tb of z)
+    const int hb = J.v - tb;
+    const int ngroups = (nr + 31) >> 5;
+    for (int x = threadIdx.x; x < ngroups + 32; x += PE_THREADS) {
+        uint64_t e = 1;
+        if (x < ngroups) {
+            const uint64_t m = (uint64_t)(r0 >> 5) + x;  // row group: the rows' high bits
+            for (int b = 0; b < hb; b++) e = gl_mul(e, gl_eq1(J.z[b], (int)((m >> (hb - 1 - b)) & 1)));
+            htab[x] = e;
+        } else {
+            const int n = x - ngroups;
+            for (int b = 0; b < tb; b++) e = gl_mul(e, gl_eq1(J.z[hb + b], (n >> (tb - 1 - b)) & 1));
+            ttab[n] = e;
+        }
+    }
+    __syncthreads();
+    uint64_t es = 0;  // sum of the weights this warp's columns see
+    if (!SCALED) {
+        for (int k = threadIdx.x; k < ROWS; k += PE_THREADS) {
+            // with v < 5 the rows are i = n < 2^v and H = {1}
+            const uint64_t e = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
+#pragma unroll
+            for (int l = 0; l < 8; l++) et[0][l][k] = (uint8_t)(e >> (8 * l));
+            es = gl_add(es, e);
+        }
+        es = warp_sum_gl(es);
+        if (lane == 0) wsum[warp] = es;
+        __syncthreads();
+        es = 0;
+#pragma unroll
+        for (int w = 0; w < PE_THREADS / 32; w++) es = gl_add(es, wsum[w]);
+    } else {
+        for (int k = threadIdx.x; k < ROWS; k += PE_THREADS) eqs[k] = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
+        __syncthreads();
+        const int g = wc0 / 64;
+        for (int k = lane; k < ROWS; k += 32) {
+            uint64_t e = 0;
+            if (wactive && k < nr) e = gl_mul_small(eqs[k], (int32_t)__ldg(J.scales + (int64_t)(r0 + k) * G + g));
+#pragma unroll
+            for (int l = 0; l < 8; l++) et[warp][l][k] = (uint8_t)(e >> (8 * l));
+            es = gl_add(es, e);
+        }
+        es = warp_sum_gl(es);
+        __syncwarp();
+    }
+
+    uint32_t acc[NG][2];
+#pragma unroll
+    for (int g = 0; g < NG; g++) acc[g][0] = acc[g][1] = 0;
+    if (wactive) {
+        // lane reads word gid of the warp's 32-byte slice, rows tig*4 + r and 16 + tig*4 + r of each 32-row chunk
+        const uint8_t* base = J.mat + (int64_t)(r0 + tig * 4) * pitch + (W4 ? wc0 / 2 : wc0) + 4 * gid;
+        const uint8_t* lp = &et[SCALED ? warp : 0][gid][0];
+        auto load_chunk = [&](uint32_t (&w)[8], int ch) {
+            const uint8_t* p = base + (int64_t)ch * pitch;
+            if (ch + 32 <= nr) {
+#pragma unroll
+                for (int q = 0; q < 8; q++)
+                    w[q] = __ldcs(reinterpret_cast<const unsigned int*>(p + ((q >> 2) * 16 + (q & 3)) * pitch));
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    const int row = ch + (q >> 2) * 16 + tig * 4 + (q & 3);
+                    w[q] = row < nr ? __ldcs(reinterpret_cast<const unsigned int*>(
+                                          p + ((q >> 2) * 16 + (q & 3)) * pitch))
+                                    : 0u;
+                }
+            }
+        };
+        uint32_t cur[8], nxt[8];
+        load_chunk(cur, 0);
+        for (int ch = 0; ch < nr; ch += 32) {
+            if (ch + 32 < nr) load_chunk(nxt, ch + 32);
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lp + ch + tig * 4);
+            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lp + ch + 16 + tig * 4);
+            uint32_t t0[4], t1[4];
+            transpose4x4(cur, t0);
+            transpose4x4(cur + 4, t1);
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                if (W4) {
+                    // u = nibble ^ 8 = w + 8: low nibbles are even columns, high nibbles odd ones
+                    const uint32_t x0 = t0[j] ^ 0x88888888u, x1 = t1[j] ^ 0x88888888u;
+                    mma_u8(acc[2 * j], a0, a2, x0 & 0x0F0F0F0Fu, x1 & 0x0F0F0F0Fu);
+                    mma_u8(acc[2 * j + 1], a0, a2, (x0 >> 4) & 0x0F0F0F0Fu, (x1 >> 4) & 0x0F0F0F0Fu);
+                } else {
+                    // u = byte ^ 0x80 = w + 128
+                    mma_u8(acc[j], a0, a2, t0[j] ^ 0x80808080u, t1[j] ^ 0x80808080u);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 8; q++) cur[q] = nxt[q];
+        }
+    }
+    // C[limb gid][n = 2 tig + e] of group j (and nibble parity) belongs to column
+    // 2 (4 n + j) + parity (int4) or 4 n + j (int8) of the warp's slice
+    if (!wactive) return;
+#pragma unroll
+    for (int g = 0; g < NG; g++) {
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int n = 2 * tig + e;
+            const int col = W4 ? 2 * (4 * n + (g >> 1)) + (g & 1) : 4 * n + g;
+            red[warp][col * 8 + gid] = acc[g][e];
+        }
+    }
+    __syncwarp();
+    const uint32_t off = W4 ? 8u : 128u;
+    const uint64_t corr = gl_mul(off, es);
+    for (int c = lane; c < WCOLS; c += 32) {
+        const int gc = wc0 + c;
+        if (gc >= J.cols) break;
+        GlAcc a;
+#pragma unroll
+        for (int l = 0; l < 8; l++) a.mac(red[warp][c * 8 + l], 1ull << (8 * l));
+        J.part[(int64_t)split * J.cols + gc] = gl_sub(a.value(), corr);
+    }
+}
+
 // out[c] = sum over the splits of part[split][c] (c < cols), 0 up to out_len; job blockIdx.y
 __global__ void partial_fin_kernel(const PeJob* __restrict__ jobs) {
     const PeJob J = jobs[blockIdx.y];
@@ -204,15 +387,33 @@ __global__ void partial_fin_kernel(const PeJob* __restrict__ jobs) {
     }
 }
 
-// About two waves of 8-warp blocks, at most PE_MAX_ROWS rows per block.
-void pe_plan(int num_sms, int rows, int cols, int& col_blocks, int& rpb, int& splits) {
-    col_blocks = (cols + PE_BLOCK_COLS - 1) / PE_BLOCK_COLS;
-    int want = (2 * num_sms + col_blocks - 1) / col_blocks;
+// About `waves` blocks per SM, at most max_rows rows per block (a multiple of 8, or of 32 on the
+// tensor-core path).
+void pe_plan_shape(int num_sms, int rows, int cols, int block_cols, int max_rows, int row_step, int waves,
+                   int& col_blocks, int& rpb, int& splits) {
+    col_blocks = (cols + block_cols - 1) / block_cols;
+    int want = (waves * num_sms + col_blocks - 1) / col_blocks;
     rpb = (rows + want - 1) / want;
-    rpb = (rpb + 7) / 8 * 8;
-    if (rpb < 8) rpb = 8;
-    if (rpb > PE_MAX_ROWS) rpb = PE_MAX_ROWS;
+    rpb = (rpb + row_step - 1) / row_step * row_step;
+    if (rpb < row_step) rpb = row_step;
+    if (rpb > max_rows) rpb = max_rows;
     splits = (rows + rpb - 1) / rpb;
+}
+
+// The tensor-core path needs whole 32-byte warp slices in every row, read as 32-bit words.
+bool pe_tc_ok(const FpPeJob& q) {
+    const int64_t pitch = q.bits == 4 ? (q.cols + 1) / 2 : q.cols;
+    return ((uintptr_t)q.mat % 4 == 0) && (q.cols % (q.bits == 4 ? 64 : 32) == 0) && (pitch % 4 == 0);
+}
+
+void pe_plan(int num_sms, const FpPeJob& q, bool& tc, int& col_blocks, int& rpb, int& splits) {
+    tc = pe_tc_ok(q);
+    // tensor-core blocks: three fit an SM; about two rounds of them keep the tail short
+    if (tc)
+        pe_plan_shape(num_sms, q.rows, q.cols, (PE_THREADS / 32) * (q.bits == 4 ? 64 : 32),
+                      q.scales ? tc_rows<true>() : tc_rows<false>(), 32, 6, col_blocks, rpb, splits);
+    else
+        pe_plan_shape(num_sms, q.rows, q.cols, PE_BLOCK_COLS, PE_MAX_ROWS, 8, 2, col_blocks, rpb, splits);
 }
 
 }  // namespace
@@ -221,7 +422,8 @@ size_t fp_partial_scratch(const fp_ctx* c, const FpPeJob* jobs, int njobs) {
     size_t need = 4 * fp_align_up(sizeof(PeJob) * (size_t)njobs, 256) + 4096;
     for (int j = 0; j < njobs; j++) {
         int cbk, rpb, sp;
-        pe_plan(c->num_sms, jobs[j].rows, jobs[j].cols, cbk, rpb, sp);
+        bool tc;
+        pe_plan(c->num_sms, jobs[j], tc, cbk, rpb, sp);
         need += fp_align_up((size_t)8 * sp * jobs[j].cols, 256) + fp_align_up(8 * (size_t)std::max(1, jobs[j].v), 256);
     }
     return need;
@@ -236,7 +438,7 @@ size_t fp_partial_host_scratch(const FpPeJob* jobs, int njobs) {
 int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
     if (njobs <= 0) return FP_OK;
     std::vector<PeJob> h(njobs);
-    std::vector<int> order[4];
+    std::vector<int> order[8];  // (tensor-core path, int4, scaled)
     size_t zt = 0;
     for (int j = 0; j < njobs; j++) zt += (size_t)jobs[j].v;
     uint64_t* hz = (uint64_t*)fp_alloc(c->host, 8 * (zt + 1));
@@ -253,7 +455,8 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         d.rows = q.rows;
         d.cols = q.cols;
         d.v = q.v;
-        pe_plan(c->num_sms, q.rows, q.cols, d.col_blocks, d.rows_per_block, d.splits);
+        bool tc;
+        pe_plan(c->num_sms, q, tc, d.col_blocks, d.rows_per_block, d.splits);
         const int64_t pitch = q.bits == 4 ? (q.cols + 1) / 2 : q.cols;
         // the fast path loads 4 (int4) or 8 (int8) bytes per lane and row
         d.aligned = ((uintptr_t)q.mat % 16 == 0) && (q.cols % PE_COLS == 0) &&
@@ -265,10 +468,10 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         if (q.v) memcpy(hz + zo, q.z, 8 * (size_t)q.v);
         d.z = dz + zo;
         zo += (size_t)q.v;
-        order[(q.bits == 4 ? 2 : 0) + (q.scales ? 1 : 0)].push_back(j);
+        order[(tc ? 4 : 0) + (q.bits == 4 ? 2 : 0) + (q.scales ? 1 : 0)].push_back(j);
     }
     FP_CUDA(c, cudaMemcpyAsync(dz, hz, 8 * (zt + 1), cudaMemcpyHostToDevice, s));
-    for (int var = 0; var < 4; var++) {
+    for (int var = 0; var < 8; var++) {
         if (order[var].empty()) continue;
         std::vector<PeJob> g;
         int64_t blocks = 0;
@@ -294,6 +497,10 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         if (var == 1) partial_many_kernel<false, true><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
         if (var == 2) partial_many_kernel<true, false><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
         if (var == 3) partial_many_kernel<true, true><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
+        if (var == 4) partial_tc_kernel<false, false><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
+        if (var == 5) partial_tc_kernel<false, true><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
+        if (var == 6) partial_tc_kernel<true, false><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
+        if (var == 7) partial_tc_kernel<true, true><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
         fp_toc(c, s, slot);
         FP_CUDA(c, cudaGetLastError());
     }

@@ -87,6 +87,8 @@ PE_SHAPES = [
     # rows, cols, bits, scales
     (1, 1, 8, False), (5, 37, 8, False), (64, 4096, 4, False), (300, 257, 4, False), (129, 1000, 4, True),
     (4096, 512, 8, False), (17, 96, 8, True), (2000, 2048, 4, True), (3, 7, 4, False), (16384, 64, 4, False),
+    # whole 32-byte row slices (the tensor-core path): ragged row chunks, several scale groups
+    (1000, 192, 4, True), (33, 32, 8, False), (257, 640, 8, True), (31, 64, 4, False), (300, 1536, 8, False),
 ]
 
 
