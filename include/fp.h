@@ -222,8 +222,8 @@ int fp_session_selftest(fp_ctx* ctx, void* stream);
 int fp_proof_size(const fp_site* sites, int nsites, size_t* matmul_bytes, size_t* logup_bytes);
 
 /*
- * Per-kernel timing: while profiling is on (fp_ctx_set_profiling(ctx, 1), which
- * also clears the counters), every launch of the library on this context is
+ * Per-kernel timing: while profiling is on (fp_ctx_set_profiling(ctx, 1) or 2,
+ * which also clears the counters), every launch of the library on this context is
  * bracketed by CUDA events on its stream. fp_kernel_stats fills up to `cap`
  * records {kernel id, launches, total device ms, algorithmic bytes moved} and
  * returns the number of kernels seen; names come from fp_kernel_name(id).
@@ -235,10 +235,12 @@ typedef struct {
     double bytes;
 } fp_kernel_stat;
 int fp_ctx_set_profiling(fp_ctx* ctx, int on);
-/* While profiling is on (and when the process runs under an injected profiler,
+/* With profiling level 1 (and when the process runs under an injected profiler,
  * or with FP_STEPPED=1 in the environment) every sum-check round is its own
  * kernel launch, so that each launch can be timed; otherwise one resident kernel
- * runs all rounds of a sum-check. Both produce the same proof bytes. */
+ * runs all rounds of a sum-check, and level 2 times those launches as they run
+ * (host exchanges included). Both modes produce the same proof bytes. 0 turns
+ * timing off; other values are FP_ERR_ARG. */
 /* Number of kernels the library has launched on this context since its creation. */
 int64_t fp_ctx_launches(const fp_ctx* ctx);
 /* Host side of the round exchanges since the context was created:

@@ -241,8 +241,11 @@ class Context:
                                                      _stream(stream)), "logup_prove_rescale")
         return buf.raw[: n.value], rc
 
-    def set_profiling(self, on: bool):
-        self._check(self._L.fp_ctx_set_profiling(self.h, 1 if on else 0), "fp_ctx_set_profiling")
+    def set_profiling(self, on):
+        """False/0: off; True/1: one launch per sum-check round, each timed; 2: time the
+        production (resident) launches as they run."""
+        level = 2 if on == 2 else (1 if on else 0)
+        self._check(self._L.fp_ctx_set_profiling(self.h, level), "fp_ctx_set_profiling")
 
     def session_selftest(self, stream=None) -> int:
         """Run the bounded-wait self-test; returns the status code (FP_ERR_TIMEOUT = -4 expected)."""

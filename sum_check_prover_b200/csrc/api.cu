@@ -81,6 +81,8 @@ fp_ctx* fp_ctx_create(int device) {
     const char* st = getenv("FP_STEPPED");
     c->stepped_env = profiler_injected() || (st && st[0] == '1');
     c->stepped = c->stepped_env;
+    const char* tg = getenv("FP_TCGEN05");
+    c->tc_gemm = tg && tg[0] == '1';
     return c;
 }
 
@@ -298,11 +300,12 @@ void fp_stats_reset(fp_ctx* c) {
 }
 
 int fp_ctx_set_profiling(fp_ctx* c, int on) {
-    if (!c) return FP_ERR_ARG;
+    if (!c || on < 0 || on > 2) return FP_ERR_ARG;
     stats_resolve(c);
-    c->profiling = on ? 1 : 0;
-    // per-kernel timing brackets each round's launch, so profiling runs stepped
-    c->stepped = c->profiling || c->stepped_env;
+    // 1: every round is its own launch, timed alone; 2: launches as in production
+    // (resident sum-check kernels, whose time then includes the host exchanges)
+    c->profiling = on == 1 ? 1 : on == 2 ? 2 : 0;
+    c->stepped = c->profiling == 1 || c->stepped_env;
     for (auto& s : c->stats) s = FpKStat();
     c->log.clear();
     return FP_OK;
@@ -445,6 +448,7 @@ int fp_commit_witness(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, vo
     FP_CUDA(c, cudaSetDevice(c->device));
     cudaStream_t s = (cudaStream_t)stream;
     fp_reset(c->dev);
+    c->mb->err = 0;
     rc = fp_launch_witness(c, sites, nsites, s);
     if (rc) return rc;
     // digests: W and scales only where no offline digest is given
@@ -473,6 +477,8 @@ int fp_commit_witness(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, vo
     std::vector<uint8_t> dg(32 * jobs.size());
     rc = fp_digest_many(c, jobs.data(), (int)jobs.size(), dg.data(), s);
     if (rc) return rc;
+    if (c->mb->err)  // the digests synchronised the stream
+        return fp_fail(c, FP_ERR_TIMEOUT, "witness GEMM: a tensor-core completion wait ran out");
     std::vector<uint8_t> rec(192 * (size_t)nsites);
     for (int i = 0; i < nsites; i++)
         if (sites[i].w_digest) memcpy(&rec[192 * i], sites[i].w_digest, 64);

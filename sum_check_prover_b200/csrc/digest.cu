@@ -45,18 +45,29 @@ __device__ void sha_bytes(const uint8_t* p, uint32_t n, bool aligned16, uint32_t
     fp_sha_init(h);
     uint32_t nfull = n / 64;
     uint32_t m[16];
-    for (uint32_t b = 0; b < nfull; b++) {
-        const uint8_t* q = p + 64 * b;
-        if (aligned16) {
+    if (aligned16 && nfull) {
+        // the next block's loads are in flight while this block is compressed
+        uint4 nx[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) nx[i] = __ldg(reinterpret_cast<const uint4*>(p) + i);
+        for (uint32_t b = 0; b < nfull; b++) {
 #pragma unroll
             for (int i = 0; i < 4; i++) {
-                uint4 v = __ldg(reinterpret_cast<const uint4*>(q) + i);
-                m[4 * i + 0] = bswap32(v.x);
-                m[4 * i + 1] = bswap32(v.y);
-                m[4 * i + 2] = bswap32(v.z);
-                m[4 * i + 3] = bswap32(v.w);
+                m[4 * i + 0] = bswap32(nx[i].x);
+                m[4 * i + 1] = bswap32(nx[i].y);
+                m[4 * i + 2] = bswap32(nx[i].z);
+                m[4 * i + 3] = bswap32(nx[i].w);
             }
-        } else {
+            if (b + 1 < nfull) {
+#pragma unroll
+                for (int i = 0; i < 4; i++) nx[i] = __ldg(reinterpret_cast<const uint4*>(p + 64 * (b + 1)) + i);
+            }
+            fp_sha_compress(h, m);
+        }
+    }
+    for (uint32_t b = 0; b < nfull && !aligned16; b++) {
+        const uint8_t* q = p + 64 * b;
+        {
 #pragma unroll
             for (int i = 0; i < 16; i++)
                 m[i] = ((uint32_t)q[4 * i] << 24) | ((uint32_t)q[4 * i + 1] << 16) | ((uint32_t)q[4 * i + 2] << 8) |
@@ -99,9 +110,18 @@ __device__ void sha_words(const uint32_t* w, uint32_t nw, uint32_t h[8]) {
     fp_sha_init(h);
     uint32_t m[16];
     uint32_t nfull = nw / 16;
+    uint32_t nx[16];
+    if (nfull) {
+#pragma unroll
+        for (int i = 0; i < 16; i++) nx[i] = __ldcg(w + i);
+    }
     for (uint32_t b = 0; b < nfull; b++) {
 #pragma unroll
-        for (int i = 0; i < 16; i++) m[i] = w[16 * b + i];
+        for (int i = 0; i < 16; i++) m[i] = nx[i];
+        if (b + 1 < nfull) {
+#pragma unroll
+            for (int i = 0; i < 16; i++) nx[i] = __ldcg(w + 16 * (b + 1) + i);
+        }
         fp_sha_compress(h, m);
     }
     uint32_t tail = nw - 16 * nfull;  // 0 or 8

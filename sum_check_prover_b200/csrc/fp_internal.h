@@ -77,6 +77,8 @@ struct fp_ctx {
     // sum-check (under a kernel-replaying profiler, and while profiling)
     int stepped = 0;
     int stepped_env = 0;
+    // witness GEMM on the tcgen05 tensor-core path (FP_TCGEN05=0 selects the mma.sync kernel)
+    int tc_gemm = 0;
     // timing
     int profiling = 0;
     int64_t launches = 0;  // every kernel launch of the library on this context

@@ -61,6 +61,20 @@ __device__ __forceinline__ void leaf_den(const KeySrc& K, const Chal& C, int64_t
     d1 = gl_sub(C.alpha1, gl_add(gl_from_i64(q), gl_mul_small(C.gamma, y)));
 }
 
+// The same with alpha1 - gamma y taken from a 256-entry table (index y + 128)
+__device__ __forceinline__ void leaf_den_tab(const KeySrc& K, const Chal& C, const uint64_t* ytab, int64_t i,
+                                             uint64_t& d0, uint64_t& d1) {
+    int32_t r, q, y;
+    key_at(K, i, r, q, y);
+    d0 = gl_sub(C.alpha0, gl_from_i64(r));
+    d1 = gl_sub(ytab[y + 128], gl_from_i64(q));
+}
+
+// ytab[y + 128] = alpha1 - gamma y for every int8 y (one block fills it)
+__device__ __forceinline__ void leaf_ytab_build(const Chal& C, uint64_t* ytab) {
+    for (int j = threadIdx.x; j < 256; j += blockDim.x) ytab[j] = gl_sub(C.alpha1, gl_mul_small(C.gamma, j - 128));
+}
+
 // ---- histograms --------------------------------------------------------------
 
 constexpr int HIST_WIN = 1 << 14;  // q in [-2^14, 2^14) counted in shared memory
@@ -272,12 +286,12 @@ __device__ __forceinline__ uint64_t layer_F(const uint64_t (&pl)[2], const uint6
 
 // pair x of the layer's current vectors: from the key columns, or from pp/qq
 template <bool LEAF>
-__device__ __forceinline__ void layer_pair(const GkrLayer& A, bool from_keys, int64_t x, ulonglong2 (&pp)[2],
-                                           ulonglong2 (&qq)[2]) {
+__device__ __forceinline__ void layer_pair(const GkrLayer& A, const uint64_t* ytab, bool from_keys, int64_t x,
+                                           ulonglong2 (&pp)[2], ulonglong2 (&qq)[2]) {
     if (LEAF && from_keys) {
         uint64_t l0, l1, r0, r1;
-        leaf_den(A.keys, A.chal, 2 * x, l0, l1);
-        leaf_den(A.keys, A.chal, 2 * x + 1, r0, r1);
+        leaf_den_tab(A.keys, A.chal, ytab, 2 * x, l0, l1);
+        leaf_den_tab(A.keys, A.chal, ytab, 2 * x + 1, r0, r1);
         qq[0] = make_ulonglong2(l0, r0);
         qq[1] = make_ulonglong2(l1, r1);
         pp[0] = pp[1] = make_ulonglong2(1, 1);
@@ -340,7 +354,8 @@ __device__ __forceinline__ uint64_t eq_chunks_at(const EqChunks& C, const uint64
 }
 
 template <bool LEAF>
-__device__ __forceinline__ void layer_round(const GkrLayer& A, const EqChunks& EC, const uint64_t* eq_tab, int t,
+__device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* ytab, const EqChunks& EC,
+                                            const uint64_t* eq_tab, int t,
                                             int64_t h, unsigned active, uint64_t rprev, uint64_t lam, uint64_t lam2,
                                             bool need1, GlAcc (&acc)[3]) {
     const bool from_keys = LEAF && t <= 2;
@@ -348,16 +363,16 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const EqChunks& E
         ulonglong2 c0p[2], c0q[2], c1p[2], c1q[2];
         uint64_t e;
         if (t == 1) {
-            layer_pair<LEAF>(A, from_keys, b, c0p, c0q);
-            layer_pair<LEAF>(A, from_keys, b + h, c1p, c1q);
+            layer_pair<LEAF>(A, ytab, from_keys, b, c0p, c0q);
+            layer_pair<LEAF>(A, ytab, from_keys, b + h, c1p, c1q);
             e = eq_chunks_at(EC, eq_tab, b);  // E_1[b] = eq(z_2..z_d, b)
             if (A.d > 1) A.E[b] = e;
         } else {
             ulonglong2 s0p[2], s0q[2], s1p[2], s1q[2], s2p[2], s2q[2], s3p[2], s3q[2];
-            layer_pair<LEAF>(A, from_keys, b, s0p, s0q);
-            layer_pair<LEAF>(A, from_keys, b + h, s1p, s1q);
-            layer_pair<LEAF>(A, from_keys, b + 2 * h, s2p, s2q);
-            layer_pair<LEAF>(A, from_keys, b + 3 * h, s3p, s3q);
+            layer_pair<LEAF>(A, ytab, from_keys, b, s0p, s0q);
+            layer_pair<LEAF>(A, ytab, from_keys, b + h, s1p, s1q);
+            layer_pair<LEAF>(A, ytab, from_keys, b + 2 * h, s2p, s2q);
+            layer_pair<LEAF>(A, ytab, from_keys, b + 3 * h, s3p, s3q);
 #pragma unroll
             for (int tau = 0; tau < 2; tau++) {
                 if (LEAF) {
@@ -404,13 +419,102 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const EqChunks& E
     }
 }
 
+// The rest of a layer once one block holds all its pairs (h <= kTailPairs): the
+// pair vectors move to shared memory (folded there by each new challenge) and
+// each (pair, table, evaluation point) is its own task, so a round is a few
+// short dependency chains per thread instead of one long one.
+constexpr int kTailPairs = 128;
+
+template <bool LEAF>
+__device__ __forceinline__ void layer_tail(const GkrLayer& A, const uint64_t* ytab, const uint64_t* zs,
+                                           const EqChunks& EC, const uint64_t* eq_tab, int t0, uint64_t rprev,
+                                           uint64_t lam, uint64_t lam2, FpMailbox* mb, FpRelay* rl) {
+    __shared__ uint64_t S[8][2 * kTailPairs];  // position x: p0L p0R q0L q0R p1L p1R q1L q1R
+    __shared__ uint64_t Et[kTailPairs];
+    const int d = A.d;
+    int h = 1 << (d - t0);
+    const bool from_keys = LEAF && t0 <= 2;
+    for (int x = threadIdx.x; x < 2 * h; x += blockDim.x) {
+        ulonglong2 pp[2], qq[2];
+        layer_pair<LEAF>(A, ytab, from_keys, x, pp, qq);
+        if (t0 > 1) {
+            ulonglong2 p2[2], q2[2];
+            layer_pair<LEAF>(A, ytab, from_keys, x + 2 * h, p2, q2);
+#pragma unroll
+            for (int tau = 0; tau < 2; tau++) {
+                if (!LEAF) pp[tau] = fold2(pp[tau], p2[tau], rprev);
+                qq[tau] = fold2(qq[tau], q2[tau], rprev);
+            }
+        }
+#pragma unroll
+        for (int tau = 0; tau < 2; tau++) {
+            S[4 * tau + 0][x] = pp[tau].x;
+            S[4 * tau + 1][x] = pp[tau].y;
+            S[4 * tau + 2][x] = qq[tau].x;
+            S[4 * tau + 3][x] = qq[tau].y;
+        }
+    }
+    for (int b = threadIdx.x; b < h; b += blockDim.x)
+        Et[b] = t0 == 1 ? eq_chunks_at(EC, eq_tab, b) : gl_add(__ldcg(A.E + b), __ldcg(A.E + b + h));
+    __syncthreads();
+    for (int t = t0; t <= d; t++) {
+        if (t > t0) {
+            if (!session_wait(mb, rl, A.seq0 + t - 1, rprev)) return;
+            if (threadIdx.x == 0) A.zout[t - 2] = rprev;
+            h >>= 1;
+            // fold the most significant position bit: x < 2h takes x + 2h (p stays 1 on the leaf layer)
+            for (int i = threadIdx.x; i < 8 * 2 * h; i += blockDim.x) {
+                const int c = i / (2 * h), x = i - c * (2 * h);
+                if (LEAF && (c & 2) == 0) continue;
+                S[c][x] = gl_fold_fast(S[c][x], S[c][x + 2 * h], rprev);
+            }
+            for (int b = threadIdx.x; b < h; b += blockDim.x) Et[b] = gl_add(Et[b], Et[b + h]);
+            __syncthreads();
+        }
+        const int nx = zs[t - 1] == 0 ? 3 : 2;  // X = 0, 2 (and 1 when z_t = 0)
+        GlAcc acc0, acc2, acc1;  // by evaluation point (separate variables: no dynamic indexing)
+        for (int task = threadIdx.x; task < h * 2 * nx; task += blockDim.x) {
+            const int b = task % h, rest = task / h, tau = rest & 1, xi = rest >> 1;
+            uint64_t v[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const uint64_t c0 = S[4 * tau + k][b], c1 = S[4 * tau + k][b + h];
+                v[k] = xi == 0 ? c0 : xi == 1 ? gl_add(gl_sub(c1, c0), c1) : c1;
+            }
+            // v = pL, pR, qL, qR at X
+            const uint64_t u = gl_add(LEAF ? 1ull : v[1], gl_mul_weak(lam, v[3]));
+            uint64_t f = gl_muladd_weak(v[2], u, LEAF ? v[3] : gl_mul_weak(v[0], v[3]));
+            if (tau) f = gl_mul_weak(lam2, f);
+            if (xi == 0)
+                acc0.mac(Et[b], f);
+            else if (xi == 1)
+                acc2.mac(Et[b], f);
+            else
+                acc1.mac(Et[b], f);
+        }
+        uint64_t out[3] = {acc0.value(), acc2.value(), acc1.value()};
+        block_sum_gl<3>(out);
+        if (threadIdx.x == 0) session_publish(mb, out, A.seq0 + t);
+    }
+    if (!session_wait(mb, rl, A.seq0 + d, rprev)) return;
+    if (threadIdx.x == 0) {
+        A.zout[d - 1] = rprev;
+        uint64_t out[8];
+#pragma unroll
+        for (int c = 0; c < 8; c++) out[c] = gl_fold(S[c][0], S[c][1], rprev);
+        session_publish(mb, out, A.seq0 + d + 1);
+    }
+}
+
 // Rounds [t_begin, t_end] of one layer (t_end > d: and its final child values).
 template <bool LEAF>
 __global__ void __launch_bounds__(LU_THREADS, 2) gkr_layer_kernel(GkrLayer A, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
     __shared__ uint64_t zs[32];
     __shared__ uint64_t s_lam;
     __shared__ uint64_t eq_tab[3 << kEqChunk];
+    __shared__ uint64_t ytab[LEAF ? 256 : 1];
     const int d = A.d;
+    if (LEAF) leaf_ytab_build(A.chal, ytab);  // visible after the first barrier below
     if (A.t_begin == 1) {
         // the layer's own challenges: mu (last point coordinate) and lambda
         uint64_t mu, lam;
@@ -442,8 +546,13 @@ __global__ void __launch_bounds__(LU_THREADS, 2) gkr_layer_kernel(GkrLayer A, Fp
         if (blockIdx.x >= active) return;  // this block has no pairs in this or any later round
         EqChunks EC{0, 0, 0};
         if (t == 1) EC = eq_chunks_build(eq_tab, zs, d);
+        if (active == 1 && h <= kTailPairs && A.t_end > d) {
+            // one block left, and this launch runs to the end of the layer
+            layer_tail<LEAF>(A, ytab, zs, EC, eq_tab, t, rprev, lam, lam2, mb, rl);
+            return;
+        }
         GlAcc sums[3];
-        layer_round<LEAF>(A, EC, eq_tab, t, h, active, rprev, lam, lam2, zs[t - 1] == 0, sums);
+        layer_round<LEAF>(A, ytab, EC, eq_tab, t, h, active, rprev, lam, lam2, zs[t - 1] == 0, sums);
         uint64_t acc[3] = {sums[0].value(), sums[1].value(), sums[2].value()};
         bool last;
         if (active == 1) {
@@ -462,8 +571,8 @@ __global__ void __launch_bounds__(LU_THREADS, 2) gkr_layer_kernel(GkrLayer A, Fp
     if (threadIdx.x == 0) {
         A.zout[d - 1] = rprev;
         ulonglong2 p0[2], q0[2], p1[2], q1[2];
-        layer_pair<LEAF>(A, LEAF && d == 1, 0, p0, q0);
-        layer_pair<LEAF>(A, LEAF && d == 1, 1, p1, q1);
+        layer_pair<LEAF>(A, ytab, LEAF && d == 1, 0, p0, q0);
+        layer_pair<LEAF>(A, ytab, LEAF && d == 1, 1, p1, q1);
         uint64_t out[8];
 #pragma unroll
         for (int tau = 0; tau < 2; tau++) {

@@ -365,10 +365,15 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
     for (int c = lane; c < WCOLS; c += 32) {
         const int gc = wc0 + c;
         if (gc >= J.cols) break;
-        GlAcc a;
-#pragma unroll
-        for (int l = 0; l < 8; l++) a.mac(red[warp][c * 8 + l], 1ull << (8 * l));
-        J.part[(int64_t)split * J.cols + gc] = gl_sub(a.value(), corr);
+        // sum_l C_l 2^(8 l) with every C_l < 2^31: limbs 0..4 fit 64 bits, limbs 5..7 form
+        // (C5 + 2^8 C6 + 2^16 C7) 2^40 (< 2^88)
+        const uint32_t* C = &red[warp][c * 8];
+        uint64_t lo = (uint64_t)C[0] + ((uint64_t)C[1] << 8) + ((uint64_t)C[2] << 16) + ((uint64_t)C[3] << 24) +
+                      ((uint64_t)C[4] << 32);
+        const uint64_t up = (uint64_t)C[5] + ((uint64_t)C[6] << 8) + ((uint64_t)C[7] << 16);
+        uint64_t hi = up >> 24;
+        asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, 0;" : "+l"(lo), "+l"(hi) : "l"(up << 40));
+        J.part[(int64_t)split * J.cols + gc] = gl_sub(gl_canon(gl_reduce_weak(lo, hi)), corr);
     }
 }
 

@@ -278,6 +278,278 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
 }
 
+
+// ---- tensor-core (tcgen05) variant -------------------------------------------------
+//
+// D = Xt . W^T for unscaled sites on the 5th-generation tensor cores: one CTA per
+// 128-token x 256-row tile, the accumulator (128 lanes x 256 columns of s32) in
+// tensor memory, operands in shared memory in the K-major core-matrix layout
+// (8 rows x 16 bytes per core matrix; element (row, byte kb) at
+// (row / 8) * 1024 + (kb / 16) * 128 + (row % 8) * 16 + kb % 16 within a
+// 128-byte-deep k-tile). Each thread prefetches its part of the next k-tile
+// into registers (int4 weights expand to int8 on the way to shared memory);
+// one thread issues the four K = 32 MMAs of a k-tile and commits them to that
+// stage's mbarrier, which frees the stage three tiles later. The epilogue
+// reads the accumulator with tcgen05.ld and applies the rescale / clamp.
+constexpr int TC_BM = 128;   // tokens: MMA M, tensor-memory lanes
+constexpr int TC_BN = 256;   // weight rows: MMA N, tensor-memory columns
+constexpr int TC_BK = 128;   // bytes of K per stage
+constexpr int TC_STAGES = 3;
+constexpr int TC_THREADS = 256;
+constexpr int TC_A_BYTES = TC_BM * TC_BK;  // 16 KB
+constexpr int TC_B_BYTES = TC_BN * TC_BK;  // 32 KB
+constexpr int TC_SMEM = TC_STAGES * (TC_A_BYTES + TC_B_BYTES) + 1024;
+constexpr uint32_t TC_WAIT_LIMIT = 1u << 24;  // mbarrier polls before the kernel gives up
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// shared-memory matrix descriptor: K-major, no swizzle, core matrices 128 B apart along K
+// (leading byte offset) and 1024 B apart along M / N (stride byte offset)
+__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46);
+}
+
+// instruction descriptor: s32 accumulator, s8 x s8, both K-major, N = 256, M = 128
+constexpr uint32_t TC_IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_BN >> 3) << 17) |
+                              ((uint32_t)(TC_BM >> 4) << 24);
+
+__device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
+    for (uint32_t it = 0; it < TC_WAIT_LIMIT; it++) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
+template <bool W4>
+struct TcRegs {
+    uint4 a[4];              // 4 chunks of 16 B of the Xt tile
+    uint4 b[W4 ? 4 : 8];     // 4 packed (int4) or 8 (int8) chunks of the W tile
+};
+
+template <bool W4>
+__device__ __forceinline__ void tc_fetch(const SiteDev& S, int j0, int i0, int k0, TcRegs<W4>& R) {
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+        const int c = tid + TC_THREADS * u, row = c >> 3, kk = c & 7;
+        const int j = j0 + row, k = k0 + kk * 16;
+        R.a[u] = (j < S.N && k < S.K) ? __ldcs(reinterpret_cast<const uint4*>(S.xt + (int64_t)j * S.K + k))
+                                      : make_uint4(0, 0, 0, 0);
+    }
+    if (W4) {
+        const int pitch = S.K >> 1;
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int c = tid + TC_THREADS * u, row = c >> 2, kq = c & 3;
+            const int i = i0 + row, k = k0 + kq * 32;
+            R.b[u] = (i < S.M && k < S.K) ? __ldg(reinterpret_cast<const uint4*>(S.w + (int64_t)i * pitch + (k >> 1)))
+                                          : make_uint4(0, 0, 0, 0);
+        }
+    } else {
+#pragma unroll
+        for (int u = 0; u < (W4 ? 4 : 8); u++) {
+            const int c = tid + TC_THREADS * u, row = c >> 3, kk = c & 7;
+            const int i = i0 + row, k = k0 + kk * 16;
+            R.b[u] = (i < S.M && k < S.K) ? __ldg(reinterpret_cast<const uint4*>(S.w + (int64_t)i * S.K + k))
+                                          : make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t tc_off(int row, int kk) { return (row >> 3) * 1024 + kk * 128 + (row & 7) * 16; }
+
+template <bool W4>
+__device__ __forceinline__ void tc_store(const TcRegs<W4>& R, uint8_t* sa, uint8_t* sb) {
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+        const int c = tid + TC_THREADS * u;
+        *reinterpret_cast<uint4*>(sa + tc_off(c >> 3, c & 7)) = R.a[u];
+    }
+    if (W4) {
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int c = tid + TC_THREADS * u, row = c >> 2, kq = c & 3;
+            // 32 nibbles (low nibble first) -> 32 int8 in two 16-byte chunks
+            const uint32_t w[4] = {R.b[u].x, R.b[u].y, R.b[u].z, R.b[u].w};
+            uint32_t o[8];
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                o[2 * q] = nib4_to_s8x4(w[q] & 0xFFFFu);
+                o[2 * q + 1] = nib4_to_s8x4(w[q] >> 16);
+            }
+            *reinterpret_cast<uint4*>(sb + tc_off(row, 2 * kq)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(sb + tc_off(row, 2 * kq + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+    } else {
+#pragma unroll
+        for (int u = 0; u < (W4 ? 4 : 8); u++) {
+            const int c = tid + TC_THREADS * u;
+            *reinterpret_cast<uint4*>(sb + tc_off(c >> 3, c & 7)) = R.b[u];
+        }
+    }
+}
+
+__device__ __forceinline__ void tc_store_out(const SiteDev& S, int j, int i, int32_t Y) {
+    const int k = S.k_shift;
+    const int64_t qq = ((int64_t)Y + ((int64_t)1 << (k - 1))) >> k;
+    const int64_t o = (int64_t)j * S.M + i;
+    S.q[o] = (int32_t)qq;
+    S.r[o] = (int32_t)((int64_t)Y - (qq << k));
+    S.y[o] = (int8_t)(qq < -128 ? -128 : (qq > 127 ? 127 : qq));
+}
+
+template <bool W4>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    witness_tc_kernel(const SiteDev* __restrict__ sites, int nsites, volatile uint64_t* err) {
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte aligned operand stages
+    uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
+    __shared__ __align__(8) uint64_t mbar[TC_STAGES];
+    __shared__ uint32_t tmem_base;
+    __shared__ int s_fail;
+
+    const int64_t tile = blockIdx.x;
+    const SiteDev S = sites[find_site(sites, nsites, tile)];
+    const int64_t lt = tile - S.tile_base;
+    const int j0 = (int)(lt / S.tiles_i) * TC_BM;
+    const int i0 = (int)(lt % S.tiles_i) * TC_BN;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        s_fail = 0;
+#pragma unroll
+        for (int st = 0; st < TC_STAGES; st++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&mbar[st])));
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::);
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;\n" ::"r"(smem_addr(&tmem_base)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
+    const uint32_t tmem = tmem_base;
+
+    const int nk = (S.K + TC_BK - 1) / TC_BK;
+    TcRegs<W4> R;
+    tc_fetch<W4>(S, j0, i0, 0, R);
+    for (int kt = 0; kt < nk; kt++) {
+        const int st = kt % TC_STAGES;
+        // the stage is free once the MMAs of tile kt - TC_STAGES (its previous use) are done;
+        // every thread waits, and the block leaves the loop together if any wait ran out
+        const bool late = kt >= TC_STAGES && !tc_wait(smem_addr(&mbar[st]), (uint32_t)((kt / TC_STAGES - 1) & 1));
+        if (__syncthreads_or(late)) {
+            if (tid == 0) s_fail = 1;
+            break;
+        }
+        tc_store<W4>(R, sA + st * TC_A_BYTES, sB + st * TC_B_BYTES);
+        if (kt + 1 < nk) tc_fetch<W4>(S, j0, i0, (kt + 1) * TC_BK, R);
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic stores -> tensor-core reads
+        asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
+        __syncthreads();
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
+        if (tid == 0) {
+            const uint32_t a0 = smem_addr(sA + st * TC_A_BYTES), b0 = smem_addr(sB + st * TC_B_BYTES);
+#pragma unroll
+            for (int kc = 0; kc < TC_BK / 32; kc++) {
+                const uint32_t en = (kt > 0 || kc > 0) ? 1u : 0u;
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+                    "l"(tc_desc(a0 + kc * 256)), "l"(tc_desc(b0 + kc * 256)), "r"(TC_IDESC), "r"(en));
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                smem_addr(&mbar[st])));
+        }
+    }
+    // all MMAs done: the last tile's commit completes after every earlier one
+    const int last = nk - 1;
+    __syncthreads();
+    const bool done = !s_fail && tc_wait(smem_addr(&mbar[last % TC_STAGES]), (uint32_t)((last / TC_STAGES) & 1));
+    const bool ok = !__syncthreads_or(!done);  // the same answer in every thread (tcgen05.ld is warp-wide)
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
+    if (ok) {
+        // warp w reads lanes 32 (w % 4) .. + 31 (tokens) and columns 128 (w / 4) .. + 127 (weight rows)
+        const int j = j0 + 32 * (warp & 3) + lane;
+        const int cbase = 128 * (warp >> 2);
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 16) {
+            uint32_t v[16];
+            const uint32_t a = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(cbase + c0);
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                : "r"(a));
+            asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+            const int i = i0 + cbase + c0;
+            if (j < S.N) {
+#pragma unroll
+                for (int e = 0; e < 16; e++)
+                    if (i + e < S.M) tc_store_out(S, j, i + e, (int32_t)v[e]);
+            }
+        }
+    } else if (tid == 0) {
+        *err = 3;  // a tensor-core wait ran out
+        __threadfence_system();
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
+    __syncthreads();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;\n" ::"r"(tmem));
+}
+
+template <bool W4>
+int launch_tc(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
+    if (list.empty()) return FP_OK;
+    std::vector<SiteDev> h(list.size());
+    int64_t tiles = 0;
+    double bytes = 0;
+    for (size_t s = 0; s < list.size(); s++) {
+        const fp_site& t = list[s];
+        SiteDev& d = h[s];
+        d.w = (const uint8_t*)t.w;
+        d.scales = t.scales;
+        d.xt = t.xt;
+        d.q = t.q;
+        d.r = t.r;
+        d.y = t.y;
+        d.M = t.M;
+        d.K = t.K;
+        d.N = t.N;
+        d.k_shift = t.k_shift;
+        d.tiles_i = (t.M + TC_BN - 1) / TC_BN;
+        d.tiles_j = (t.N + TC_BM - 1) / TC_BM;
+        d.tile_base = tiles;
+        tiles += (int64_t)d.tiles_i * d.tiles_j;
+        bytes += (double)t.M * (W4 ? t.K / 2 : t.K) + (double)t.N * t.K + 9.0 * t.M * t.N;
+    }
+    size_t sz = sizeof(SiteDev) * h.size();
+    SiteDev* dsites = (SiteDev*)fp_alloc(c->dev, sz);
+    char* hst = (char*)fp_alloc(c->host, sz);
+    if (!dsites || !hst) return fp_fail(c, FP_ERR_OOM, "witness: scratch exhausted");
+    memcpy(hst, h.data(), sz);
+    FP_CUDA(c, cudaMemcpyAsync(dsites, hst, sz, cudaMemcpyHostToDevice, st));
+    auto kern = witness_tc_kernel<W4>;
+    FP_CUDA(c, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM));
+    int slot;
+    fp_tic(c, st, K_GEMM, bytes, &slot);
+    kern<<<(unsigned)tiles, TC_THREADS, TC_SMEM, st>>>(dsites, (int)h.size(), &c->mb_dev->err);
+    fp_toc(c, st, slot);
+    FP_CUDA(c, cudaGetLastError());
+    return FP_OK;
+}
+
 template <bool W4, bool SCALED, bool ALIGNED>
 int launch_variant(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
     if (list.empty()) return FP_OK;
@@ -323,24 +595,31 @@ int launch_variant(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st)
 }  // namespace
 
 int fp_launch_witness(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st) {
-    // group sites by kernel variant
-    std::vector<fp_site> v[8];
+    // group sites by kernel variant: unscaled sites with 16-byte rows go to the tensor-core
+    // (tcgen05) kernel, the rest to the mma.sync kernel
+    std::vector<fp_site> v[8], tcv[2];
     for (int s = 0; s < nsites; s++) {
         const fp_site& t = sites[s];
         bool w4 = t.w_bits == 4, sc = t.scales != nullptr;
         size_t pitch = w4 ? (size_t)(t.K + 1) / 2 : (size_t)t.K;
         bool al = ((uintptr_t)t.w % 16 == 0) && ((uintptr_t)t.xt % 16 == 0) && (pitch % 16 == 0) &&
                   (t.K % 16 == 0) && (!w4 || t.K % 32 == 0);
-        v[(w4 ? 4 : 0) + (sc ? 2 : 0) + (al ? 1 : 0)].push_back(t);
+        if (al && !sc && c->tc_gemm)
+            tcv[w4 ? 1 : 0].push_back(t);
+        else
+            v[(w4 ? 4 : 0) + (sc ? 2 : 0) + (al ? 1 : 0)].push_back(t);
     }
     size_t need = 0;
     for (int i = 0; i < 8; i++) need += fp_align_up(sizeof(SiteDev) * v[i].size(), 256) + 256;
+    for (int i = 0; i < 2; i++) need += fp_align_up(sizeof(SiteDev) * tcv[i].size(), 256) + 256;
     int rc = fp_reserve(c, c->dev, need + (1 << 20));
     if (rc) return rc;
     rc = fp_reserve(c, c->host, need + (1 << 20));
     if (rc) return rc;
     fp_reset(c->dev);
     fp_reset(c->host);
+    if ((rc = launch_tc<false>(c, tcv[0], st))) return rc;
+    if ((rc = launch_tc<true>(c, tcv[1], st))) return rc;
     if ((rc = launch_variant<false, false, false>(c, v[0], st))) return rc;
     if ((rc = launch_variant<false, false, true>(c, v[1], st))) return rc;
     if ((rc = launch_variant<false, true, false>(c, v[2], st))) return rc;
