@@ -78,7 +78,7 @@ struct fp_ctx {
     int stepped = 0;
     int stepped_env = 0;
     // witness GEMM on the tcgen05 tensor-core path (FP_TCGEN05=0 selects the mma.sync kernel)
-    int tc_gemm = 0;
+    int tc_gemm = 1;
     // timing
     int profiling = 0;
     int64_t launches = 0;  // every kernel launch of the library on this context

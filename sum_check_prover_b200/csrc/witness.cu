@@ -282,24 +282,32 @@ __global__ void __launch_bounds__(THREADS, 1)
 // ---- tensor-core (tcgen05) variant -------------------------------------------------
 //
 // D = Xt . W^T for unscaled sites on the 5th-generation tensor cores: one CTA per
-// 128-token x 256-row tile, the accumulator (128 lanes x 256 columns of s32) in
+// 128-token x BN-row tile, the accumulator (128 lanes x BN columns of s32) in
 // tensor memory, operands in shared memory in the K-major core-matrix layout
 // (8 rows x 16 bytes per core matrix; element (row, byte kb) at
 // (row / 8) * 1024 + (kb / 16) * 128 + (row % 8) * 16 + kb % 16 within a
-// 128-byte-deep k-tile). Each thread prefetches its part of the next k-tile
-// into registers (int4 weights expand to int8 on the way to shared memory);
-// one thread issues the four K = 32 MMAs of a k-tile and commits them to that
-// stage's mbarrier, which frees the stage three tiles later. The epilogue
-// reads the accumulator with tcgen05.ld and applies the rescale / clamp.
+// 128-byte-deep k-tile). cp.async fills stage kt % S two tiles before use;
+// int4 weights land packed in the upper half of their stage and are expanded
+// to int8 in place just before the MMAs. One thread issues the four K = 32 MMAs
+// of a k-tile and commits them to the stage's mbarrier; a stage is refilled
+// once the MMAs two tiles back are done, so the tensor core always has the
+// next tile queued. The epilogue reads the accumulator with tcgen05.ld and
+// applies the rescale / clamp.
 constexpr int TC_BM = 128;   // tokens: MMA M, tensor-memory lanes
-constexpr int TC_BN = 256;   // weight rows: MMA N, tensor-memory columns
 constexpr int TC_BK = 128;   // bytes of K per stage
-constexpr int TC_STAGES = 3;
 constexpr int TC_THREADS = 256;
 constexpr int TC_A_BYTES = TC_BM * TC_BK;  // 16 KB
-constexpr int TC_B_BYTES = TC_BN * TC_BK;  // 32 KB
-constexpr int TC_SMEM = TC_STAGES * (TC_A_BYTES + TC_B_BYTES) + 1024;
 constexpr uint32_t TC_WAIT_LIMIT = 1u << 24;  // mbarrier polls before the kernel gives up
+
+template <int BN>
+struct TcCfg {
+    static constexpr int B_BYTES = BN * TC_BK;
+    static constexpr int STAGES = BN == 256 ? 4 : 6;
+    static constexpr int SMEM = STAGES * (TC_A_BYTES + B_BYTES) + 1024;
+    // s32 accumulator, s8 x s8, both K-major, N = BN, M = 128
+    static constexpr uint32_t IDESC =
+        (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(TC_BM >> 4) << 24);
+};
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -309,10 +317,6 @@ __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
            ((uint64_t)1 << 46);
 }
-
-// instruction descriptor: s32 accumulator, s8 x s8, both K-major, N = 256, M = 128
-constexpr uint32_t TC_IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TC_BN >> 3) << 17) |
-                              ((uint32_t)(TC_BM >> 4) << 24);
 
 __device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
     for (uint32_t it = 0; it < TC_WAIT_LIMIT; it++) {
@@ -327,94 +331,115 @@ __device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
     return false;
 }
 
-template <bool W4>
-struct TcRegs {
-    uint4 a[4];              // 4 chunks of 16 B of the Xt tile
-    uint4 b[W4 ? 4 : 8];     // 4 packed (int4) or 8 (int8) chunks of the W tile
-};
-
-template <bool W4>
-__device__ __forceinline__ void tc_fetch(const SiteDev& S, int j0, int i0, int k0, TcRegs<W4>& R) {
-    const int tid = threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < 4; u++) {
-        const int c = tid + TC_THREADS * u, row = c >> 3, kk = c & 7;
-        const int j = j0 + row, k = k0 + kk * 16;
-        R.a[u] = (j < S.N && k < S.K) ? __ldcs(reinterpret_cast<const uint4*>(S.xt + (int64_t)j * S.K + k))
-                                      : make_uint4(0, 0, 0, 0);
-    }
-    if (W4) {
-        const int pitch = S.K >> 1;
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const int c = tid + TC_THREADS * u, row = c >> 2, kq = c & 3;
-            const int i = i0 + row, k = k0 + kq * 32;
-            R.b[u] = (i < S.M && k < S.K) ? __ldg(reinterpret_cast<const uint4*>(S.w + (int64_t)i * pitch + (k >> 1)))
-                                          : make_uint4(0, 0, 0, 0);
-        }
-    } else {
-#pragma unroll
-        for (int u = 0; u < (W4 ? 4 : 8); u++) {
-            const int c = tid + TC_THREADS * u, row = c >> 3, kk = c & 7;
-            const int i = i0 + row, k = k0 + kk * 16;
-            R.b[u] = (i < S.M && k < S.K) ? __ldg(reinterpret_cast<const uint4*>(S.w + (int64_t)i * S.K + k))
-                                          : make_uint4(0, 0, 0, 0);
-        }
-    }
-}
-
 __device__ __forceinline__ uint32_t tc_off(int row, int kk) { return (row >> 3) * 1024 + kk * 128 + (row & 7) * 16; }
 
-template <bool W4>
-__device__ __forceinline__ void tc_store(const TcRegs<W4>& R, uint8_t* sa, uint8_t* sb) {
+// cp.async of k-tile k0 into a stage (zero fill outside the matrices)
+template <bool W4, int BN>
+__device__ __forceinline__ void tc_issue(const SiteDev& S, int j0, int i0, int k0, uint8_t* sa, uint8_t* sb) {
     const int tid = threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < 4; u++) {
-        const int c = tid + TC_THREADS * u;
-        *reinterpret_cast<uint4*>(sa + tc_off(c >> 3, c & 7)) = R.a[u];
+    for (int u = 0; u < TC_A_BYTES / 16 / TC_THREADS; u++) {
+        const int c = tid + TC_THREADS * u, row = c >> 3, kk = c & 7;
+        const int j = j0 + row, k = k0 + kk * 16;
+        const bool ok = j < S.N && k < S.K;
+        cp_async16(sa + tc_off(row, kk), ok ? S.xt + (int64_t)j * S.K + k : S.xt, ok ? 16 : 0);
     }
     if (W4) {
+        // packed rows (64 bytes of the k-tile each) in the stage's upper half
+        const int pitch = S.K >> 1;
+        uint8_t* pk = sb + TcCfg<BN>::B_BYTES / 2;
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
+        for (int u = 0; u < BN * 4 / TC_THREADS; u++) {
             const int c = tid + TC_THREADS * u, row = c >> 2, kq = c & 3;
-            // 32 nibbles (low nibble first) -> 32 int8 in two 16-byte chunks
-            const uint32_t w[4] = {R.b[u].x, R.b[u].y, R.b[u].z, R.b[u].w};
-            uint32_t o[8];
-#pragma unroll
-            for (int q = 0; q < 4; q++) {
-                o[2 * q] = nib4_to_s8x4(w[q] & 0xFFFFu);
-                o[2 * q + 1] = nib4_to_s8x4(w[q] >> 16);
-            }
-            *reinterpret_cast<uint4*>(sb + tc_off(row, 2 * kq)) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4*>(sb + tc_off(row, 2 * kq + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+            const int i = i0 + row, k = k0 + kq * 32;
+            const bool ok = i < S.M && k < S.K;
+            cp_async16(pk + row * 64 + kq * 16, ok ? S.w + (int64_t)i * pitch + (k >> 1) : S.w, ok ? 16 : 0);
         }
     } else {
 #pragma unroll
-        for (int u = 0; u < (W4 ? 4 : 8); u++) {
-            const int c = tid + TC_THREADS * u;
-            *reinterpret_cast<uint4*>(sb + tc_off(c >> 3, c & 7)) = R.b[u];
+        for (int u = 0; u < BN * 8 / TC_THREADS; u++) {
+            const int c = tid + TC_THREADS * u, row = c >> 3, kk = c & 7;
+            const int i = i0 + row, k = k0 + kk * 16;
+            const bool ok = i < S.M && k < S.K;
+            cp_async16(sb + tc_off(row, kk), ok ? S.w + (int64_t)i * S.K + k : S.w, ok ? 16 : 0);
         }
     }
 }
 
-__device__ __forceinline__ void tc_store_out(const SiteDev& S, int j, int i, int32_t Y) {
-    const int k = S.k_shift;
-    const int64_t qq = ((int64_t)Y + ((int64_t)1 << (k - 1))) >> k;
-    const int64_t o = (int64_t)j * S.M + i;
-    S.q[o] = (int32_t)qq;
-    S.r[o] = (int32_t)((int64_t)Y - (qq << k));
-    S.y[o] = (int8_t)(qq < -128 ? -128 : (qq > 127 ? 127 : qq));
+// int4 stage: packed upper half -> int8 core-matrix layout (read everything first, then write)
+template <int BN>
+__device__ __forceinline__ void tc_expand(uint8_t* sb) {
+    const int tid = threadIdx.x;
+    const uint8_t* pk = sb + TcCfg<BN>::B_BYTES / 2;
+    uint4 v[BN * 4 / TC_THREADS];
+#pragma unroll
+    for (int u = 0; u < BN * 4 / TC_THREADS; u++) {
+        const int c = tid + TC_THREADS * u;
+        v[u] = *reinterpret_cast<const uint4*>(pk + (c >> 2) * 64 + (c & 3) * 16);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < BN * 4 / TC_THREADS; u++) {
+        const int c = tid + TC_THREADS * u, row = c >> 2, kq = c & 3;
+        // 32 nibbles (low nibble first) -> 32 int8 in two 16-byte chunks
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t o[8];
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            o[2 * q] = nib4_to_s8x4(w[q] & 0xFFFFu);
+            o[2 * q + 1] = nib4_to_s8x4(w[q] >> 16);
+        }
+        *reinterpret_cast<uint4*>(sb + tc_off(row, 2 * kq)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(sb + tc_off(row, 2 * kq + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+    }
 }
 
-template <bool W4>
+// q, r, y of 16 consecutive weight rows i..i+15 of token j
+__device__ __forceinline__ void tc_store16(const SiteDev& S, int j, int i, const uint32_t (&v)[16]) {
+    const int k = S.k_shift;
+    const int64_t half = (int64_t)1 << (k - 1);
+    int32_t q[16], r[16];
+    uint32_t y[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int e = 0; e < 16; e++) {
+        const int64_t Y = (int32_t)v[e];
+        const int64_t qq = (Y + half) >> k;
+        q[e] = (int32_t)qq;
+        r[e] = (int32_t)(Y - (qq << k));
+        const int32_t yc = qq < -128 ? -128 : (qq > 127 ? 127 : (int32_t)qq);
+        y[e >> 2] |= ((uint32_t)yc & 0xFFu) << (8 * (e & 3));
+    }
+    const int64_t o = (int64_t)j * S.M + i;
+    const bool vec = i + 16 <= S.M && ((reinterpret_cast<uintptr_t>(S.q + o) | reinterpret_cast<uintptr_t>(S.r + o) |
+                                        reinterpret_cast<uintptr_t>(S.y + o)) & 15) == 0;
+    if (vec) {
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+            *reinterpret_cast<int4*>(S.q + o + e) = make_int4(q[e], q[e + 1], q[e + 2], q[e + 3]);
+            *reinterpret_cast<int4*>(S.r + o + e) = make_int4(r[e], r[e + 1], r[e + 2], r[e + 3]);
+        }
+        *reinterpret_cast<uint4*>(S.y + o) = make_uint4(y[0], y[1], y[2], y[3]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; e++) {
+            if (i + e >= S.M) break;
+            S.q[o + e] = q[e];
+            S.r[o + e] = r[e];
+            S.y[o + e] = (int8_t)(y[e >> 2] >> (8 * (e & 3)));
+        }
+    }
+}
+
+template <bool W4, int BN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     witness_tc_kernel(const SiteDev* __restrict__ sites, int nsites, volatile uint64_t* err) {
+    using C = TcCfg<BN>;
+    constexpr int ST = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
-    // 1024-byte aligned operand stages
     uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     uint8_t* sA = smem;
-    uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
-    __shared__ __align__(8) uint64_t mbar[TC_STAGES];
+    uint8_t* sB = smem + ST * TC_A_BYTES;
+    __shared__ __align__(8) uint64_t mbar[ST];
     __shared__ uint32_t tmem_base;
     __shared__ int s_fail;
 
@@ -422,69 +447,77 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const SiteDev S = sites[find_site(sites, nsites, tile)];
     const int64_t lt = tile - S.tile_base;
     const int j0 = (int)(lt / S.tiles_i) * TC_BM;
-    const int i0 = (int)(lt % S.tiles_i) * TC_BN;
+    const int i0 = (int)(lt % S.tiles_i) * BN;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nk = (S.K + TC_BK - 1) / TC_BK;
 
     if (tid == 0) {
         s_fail = 0;
 #pragma unroll
-        for (int st = 0; st < TC_STAGES; st++)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&mbar[st])));
+        for (int st = 0; st < ST; st++) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&mbar[st])));
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::);
     }
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;\n" ::"r"(smem_addr(&tmem_base)));
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_addr(&tmem_base)),
+                     "n"(BN));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+    }
+    // prologue: tiles 0 .. ST-3 in flight (prefetch distance ST - 2)
+#pragma unroll
+    for (int t = 0; t < ST - 2; t++) {
+        if (t < nk) tc_issue<W4, BN>(S, j0, i0, t * TC_BK, sA + t * TC_A_BYTES, sB + t * C::B_BYTES);
+        cp_async_commit();
     }
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
     const uint32_t tmem = tmem_base;
 
-    const int nk = (S.K + TC_BK - 1) / TC_BK;
-    TcRegs<W4> R;
-    tc_fetch<W4>(S, j0, i0, 0, R);
     for (int kt = 0; kt < nk; kt++) {
-        const int st = kt % TC_STAGES;
-        // the stage is free once the MMAs of tile kt - TC_STAGES (its previous use) are done;
-        // every thread waits, and the block leaves the loop together if any wait ran out
-        const bool late = kt >= TC_STAGES && !tc_wait(smem_addr(&mbar[st]), (uint32_t)((kt / TC_STAGES - 1) & 1));
+        const int st = kt % ST;
+        // refill the stage of tile kt + ST - 2; its previous tile (kt - 2) must be done with it
+        const int nt = kt + ST - 2, ns = nt % ST;
+        const bool late = nt < nk && kt >= 2 && !tc_wait(smem_addr(&mbar[ns]), (uint32_t)(((kt - 2) / ST) & 1));
         if (__syncthreads_or(late)) {
             if (tid == 0) s_fail = 1;
             break;
         }
-        tc_store<W4>(R, sA + st * TC_A_BYTES, sB + st * TC_B_BYTES);
-        if (kt + 1 < nk) tc_fetch<W4>(S, j0, i0, (kt + 1) * TC_BK, R);
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic stores -> tensor-core reads
+        if (nt < nk) tc_issue<W4, BN>(S, j0, i0, nt * TC_BK, sA + ns * TC_A_BYTES, sB + ns * C::B_BYTES);
+        cp_async_commit();
+        cp_async_wait<ST - 2>();  // tile kt has landed (this thread's copies)
+        __syncthreads();
+        if (W4) tc_expand<BN>(sB + st * C::B_BYTES);
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic writes -> tensor-core reads
         asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
         __syncthreads();
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
         if (tid == 0) {
-            const uint32_t a0 = smem_addr(sA + st * TC_A_BYTES), b0 = smem_addr(sB + st * TC_B_BYTES);
+            const uint32_t a0 = smem_addr(sA + st * TC_A_BYTES), b0 = smem_addr(sB + st * C::B_BYTES);
 #pragma unroll
             for (int kc = 0; kc < TC_BK / 32; kc++) {
                 const uint32_t en = (kt > 0 || kc > 0) ? 1u : 0u;
                 asm volatile(
                     "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                     "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-                    "l"(tc_desc(a0 + kc * 256)), "l"(tc_desc(b0 + kc * 256)), "r"(TC_IDESC), "r"(en));
+                    "l"(tc_desc(a0 + kc * 256)), "l"(tc_desc(b0 + kc * 256)), "r"(C::IDESC), "r"(en));
             }
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
                 smem_addr(&mbar[st])));
         }
     }
+    cp_async_wait<0>();
     // all MMAs done: the last tile's commit completes after every earlier one
     const int last = nk - 1;
     __syncthreads();
-    const bool done = !s_fail && tc_wait(smem_addr(&mbar[last % TC_STAGES]), (uint32_t)((last / TC_STAGES) & 1));
+    const bool done = !s_fail && tc_wait(smem_addr(&mbar[last % ST]), (uint32_t)((last / ST) & 1));
     const bool ok = !__syncthreads_or(!done);  // the same answer in every thread (tcgen05.ld is warp-wide)
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
     if (ok) {
-        // warp w reads lanes 32 (w % 4) .. + 31 (tokens) and columns 128 (w / 4) .. + 127 (weight rows)
+        // warp w reads lanes 32 (w % 4) .. + 31 (tokens) and the (w / 4)-th half of the columns
         const int j = j0 + 32 * (warp & 3) + lane;
-        const int cbase = 128 * (warp >> 2);
+        const int cbase = (BN / 2) * (warp >> 2);
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 16) {
+        for (int c0 = 0; c0 < BN / 2; c0 += 16) {
             uint32_t v[16];
             const uint32_t a = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(cbase + c0);
             asm volatile(
@@ -494,11 +527,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 : "r"(a));
             asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
             const int i = i0 + cbase + c0;
-            if (j < S.N) {
-#pragma unroll
-                for (int e = 0; e < 16; e++)
-                    if (i + e < S.M) tc_store_out(S, j, i + e, (int32_t)v[e]);
-            }
+            if (j < S.N && i < S.M) tc_store16(S, j, i, v);
         }
     } else if (tid == 0) {
         *err = 3;  // a tensor-core wait ran out
@@ -506,12 +535,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
     __syncthreads();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;\n" ::"r"(tmem));
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "n"(BN));
 }
 
-template <bool W4>
-int launch_tc(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
-    if (list.empty()) return FP_OK;
+template <bool W4, int BN>
+int launch_tc_bn(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
     std::vector<SiteDev> h(list.size());
     int64_t tiles = 0;
     double bytes = 0;
@@ -528,7 +556,7 @@ int launch_tc(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
         d.K = t.K;
         d.N = t.N;
         d.k_shift = t.k_shift;
-        d.tiles_i = (t.M + TC_BN - 1) / TC_BN;
+        d.tiles_i = (t.M + BN - 1) / BN;
         d.tiles_j = (t.N + TC_BM - 1) / TC_BM;
         d.tile_base = tiles;
         tiles += (int64_t)d.tiles_i * d.tiles_j;
@@ -540,14 +568,23 @@ int launch_tc(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
     if (!dsites || !hst) return fp_fail(c, FP_ERR_OOM, "witness: scratch exhausted");
     memcpy(hst, h.data(), sz);
     FP_CUDA(c, cudaMemcpyAsync(dsites, hst, sz, cudaMemcpyHostToDevice, st));
-    auto kern = witness_tc_kernel<W4>;
-    FP_CUDA(c, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM));
+    auto kern = witness_tc_kernel<W4, BN>;
+    FP_CUDA(c, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM));
     int slot;
     fp_tic(c, st, K_GEMM, bytes, &slot);
-    kern<<<(unsigned)tiles, TC_THREADS, TC_SMEM, st>>>(dsites, (int)h.size(), &c->mb_dev->err);
+    kern<<<(unsigned)tiles, TC_THREADS, TcCfg<BN>::SMEM, st>>>(dsites, (int)h.size(), &c->mb_dev->err);
     fp_toc(c, st, slot);
     FP_CUDA(c, cudaGetLastError());
     return FP_OK;
+}
+
+// 256-row tiles when they still give every SM a tile, 128-row tiles otherwise
+template <bool W4>
+int launch_tc(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
+    if (list.empty()) return FP_OK;
+    int64_t wide = 0;
+    for (const fp_site& t : list) wide += (int64_t)((t.M + 255) / 256) * ((t.N + TC_BM - 1) / TC_BM);
+    return wide >= c->num_sms ? launch_tc_bn<W4, 256>(c, list, st) : launch_tc_bn<W4, 128>(c, list, st);
 }
 
 template <bool W4, bool SCALED, bool ALIGNED>

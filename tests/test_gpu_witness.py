@@ -3,7 +3,7 @@ against a plain numpy definition: int64 matrix product, floor division with
 round-half-up, remainder, clamp ("How fast can FlashProve go", 3.1).
 
 The tcgen05 kernel takes unscaled sites whose rows are whole 16-byte chunks
-(128-token x 256-row tiles, 128-byte k-tiles); the mma.sync kernel takes the
+(128-token x 128- or 256-row tiles, 128-byte k-tiles); the mma.sync kernel takes the
 rest, or every site when the context is created with FP_TCGEN05=0. Shapes
 cover partial tiles in every dimension, K below and across k-tiles, and one
 or many tiles per site.
@@ -22,6 +22,8 @@ SHAPES = [
     (300, 128, 200, 8, False), (256, 256, 128, 4, False), (513, 96, 130, 4, False), (64, 16, 1, 8, False),
     (1000, 4096, 77, 4, False), (40, 32, 300, 4, False), (257, 160, 129, 8, False), (256, 1024, 512, 4, False),
     (129, 64, 64, 4, True), (77, 48, 33, 8, False), (33, 40, 17, 8, False),
+    # enough 256-row tiles to fill the GPU: the tcgen05 kernel's N = 256 variant
+    (4096, 256, 1280, 4, False), (2048, 128, 2560, 8, False),
 ]
 
 
