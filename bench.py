@@ -120,7 +120,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr") -> dict:
+def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
     """Kernel rooflines at HBM scale (inputs well above the 126 MB L2), from a
     profiled pass: every round is its own launch, timed with CUDA events.
 
@@ -129,6 +129,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr") -> dict:
       in place of the next evaluation (read 4, write 2 values per pair).
     partial_acc: eq-weighted row contraction of a 16384 x 16384 int4 matrix.
     gkr_round: LogUp layer rounds over 2^26 keys (one 8192 x 64 x 8192 int8 site).
+    witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
+      epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
     import workloads
     from workloads import device
@@ -172,6 +174,28 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr") -> dict:
         measure("partial_eval_int4_16384^2", "partial_acc",
                 lambda: ctx.partial_eval(mat, 4, None, rows, cols, z, outv), big=1 << 26)
         del mat, outv
+
+    if "gemm" in which:
+        # witness GEMM of an FFN-sized site on the tensor cores (2 x MACs integer ops)
+        site = workloads.random_site(55, 14336, 4096, 4096, 4, 12)
+        st, keep = device.upload(workloads.Workload("gemm", 0, [site]), dev)
+        device.weight_digests(ctx, st)
+        tx = fp.Transcript(0)
+        ctx.commit_witness(tx, st[0])
+        torch.cuda.synchronize()
+        ctx.set_profiling(True)
+        for _ in range(3):
+            ctx.commit_witness(tx, st[0])
+        torch.cuda.synchronize()
+        n, ms, by = ctx.kernel_stats()["witness_gemm"]
+        ctx.set_profiling(False)
+        tx.close()
+        tops = 2.0 * site.macs / (ms / n * 1e-3) / 1e12
+        peak = pk["bf16_tflops"] * 2.0
+        out["witness_gemm_14336x4096x4096_int4"] = {"kernel": "witness_gemm", "launches": n, "ms": ms / n,
+                                                    "TOPS": tops, "frac": tops / peak, "peak": peak,
+                                                    "peak_note": "int8 = measured bf16 x 2 (nominal ratio)"}
+        del st, keep
 
     if "gkr" in which:
         s = workloads.random_site(77, 8192, 64, 8192, 8, 12)
@@ -437,8 +461,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-micro", action="store_true")
-    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr", default=None,
-                    help="run only the HBM-scale kernel measurements (comma list of sc, pe, gkr)")
+    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm", default=None,
+                    help="run only the kernel measurements at scale (comma list of sc, pe, gkr, gemm)")
     args = ap.parse_args()
     if args.micro_only:
         import torch

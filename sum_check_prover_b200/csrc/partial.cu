@@ -24,6 +24,8 @@
 // All contractions of a call go into one launch per kernel variant (a job
 // list; the MoE layer has hundreds of sites). eq(z, i) for the block's rows
 // is computed in the block from the point, so no eq table is materialised.
+#include <cuda.h>  // CUtensorMap and its enums; the encoder is fetched through the runtime
+#include <cudaTypedefs.h>
 #include <string.h>
 
 #include <algorithm>
@@ -46,6 +48,9 @@ struct PeJob {
     int32_t aligned;
     int32_t pad;
     int64_t first_block;
+    // tensor-core path: the matrix as a 2-D byte tensor (rows x pitch), 32-row x 128-byte
+    // boxes with 128-byte swizzle, read by TMA from this device copy of the job
+    alignas(64) CUtensorMap tmap;
 };
 
 constexpr int PE_THREADS = 256;              // 8 warps share the block's columns, split its rows
@@ -54,15 +59,34 @@ constexpr int PE_BLOCK_COLS = 32 * PE_COLS;  // 256 columns per block
 constexpr int PE_UNROLL = 8;                 // rows whose loads a warp issues before using any of them
 constexpr int PE_MAX_ROWS = 256;             // 256 rows x 2^32 x 2^15 < 2^64: the sums stay exact
 
-__device__ __forceinline__ void mma_u8(uint32_t (&c)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-    // A rows 8..15 (a1, a3) are zero: only 8 limbs; their outputs are discarded
-    uint32_t d2, d3;
+// D (16 columns x 8 limbs) += A (16 columns x 32 rows of the matrix) . B (32 rows x 8 limbs)
+__device__ __forceinline__ void mma_u8(uint32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};\n"
-        : "=r"(c[0]), "=r"(c[1]), "=r"(d2), "=r"(d3)
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]), "r"(0u), "r"(0u));
-    (void)d2;
-    (void)d3;
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---- TMA pipeline (shared-memory stages filled by cp.async.bulk.tensor, tracked by mbarriers) ----
+constexpr int PE_STAGES = 6;               // 32-row chunks in flight per block
+constexpr int PE_STAGE = 2 * 32 * 128;     // one chunk: two 32 x 128-byte boxes
+constexpr int PE_DYN = PE_STAGES * PE_STAGE + 1024;  // + alignment slack
+constexpr uint32_t PE_WAIT_LIMIT = 1u << 24;
+
+__device__ __forceinline__ uint32_t pe_saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool pe_wait(uint32_t mbar, uint32_t parity) {
+    for (uint32_t it = 0; it < PE_WAIT_LIMIT; it++) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
 }
 
 // rows w[0..3] -> t[j] = byte j of each row (row r in byte r)
@@ -232,7 +256,7 @@ __host__ __device__ constexpr int tc_rows() {
 template <bool W4, bool SCALED>
 __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* __restrict__ jobs, int njobs) {
     constexpr int WCOLS = W4 ? 64 : 32;
-    constexpr int NG = W4 ? 8 : 4;  // mma column groups per lane
+    constexpr int NG = W4 ? 4 : 2;  // MMAs per 32-row chunk: 16 columns each
     constexpr int ROWS = tc_rows<SCALED>();
     // limb l of row k's weight: one table for all warps, or one per warp (scaled: the weight
     // depends on the warp's column group)
@@ -240,16 +264,26 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
     __shared__ uint64_t eqs[SCALED ? ROWS : 1];
     __shared__ uint64_t htab[ROWS / 32], ttab[32];
     __shared__ uint64_t wsum[8];
-    __shared__ uint32_t red[8][64 * 8];  // per warp: [column][limb]
-    const PeJob J = jobs[find_job(jobs, njobs, blockIdx.x)];
+    __shared__ __align__(8) uint64_t full[PE_STAGES], empty[PE_STAGES];
+    extern __shared__ uint8_t dyn_raw[];  // PE_STAGES chunks (1024-byte aligned); then the per-warp sums
+    uint8_t* stg = dyn_raw + ((1024 - (pe_saddr(dyn_raw) & 1023)) & 1023);
+    uint32_t(*red)[64 * 8] = reinterpret_cast<uint32_t(*)[64 * 8]>(stg);
+    const int jidx = find_job(jobs, njobs, blockIdx.x);
+    const PeJob J = jobs[jidx];
     const int64_t lb = blockIdx.x - J.first_block;
     const int cb = (int)(lb % J.col_blocks), split = (int)(lb / J.col_blocks);
     const int r0 = split * J.rows_per_block;  // a multiple of 32
     const int nr = min(J.rows_per_block, J.rows - r0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
     const int wc0 = (cb * (PE_THREADS / 32) + warp) * WCOLS;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < PE_STAGES; st++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(pe_saddr(&full[st])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(pe_saddr(&empty[st])), "r"(PE_THREADS / 32));
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::);
+    }  // visible after the barrier that follows the eq tables
     const bool wactive = wc0 < J.cols;
-    const int64_t pitch = W4 ? J.cols / 2 : J.cols;
     const int G = (J.cols + 63) / 64;
 
     // the two eq tables (v < 5: T covers every coordinate and H is the single entry 1)
@@ -299,64 +333,90 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
         __syncwarp();
     }
 
-    uint32_t acc[NG][2];
+    uint32_t acc[NG][4];
 #pragma unroll
-    for (int g = 0; g < NG; g++) acc[g][0] = acc[g][1] = 0;
-    if (wactive) {
-        // lane reads word gid of the warp's 32-byte slice, rows tig*4 + r and 16 + tig*4 + r of each 32-row chunk
-        const uint8_t* base = J.mat + (int64_t)(r0 + tig * 4) * pitch + (W4 ? wc0 / 2 : wc0) + 4 * gid;
-        const uint8_t* lp = &et[SCALED ? warp : 0][gid][0];
-        auto load_chunk = [&](uint32_t (&w)[8], int ch) {
-            const uint8_t* p = base + (int64_t)ch * pitch;
-            if (ch + 32 <= nr) {
+    for (int g = 0; g < NG; g++) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0;
+    {
+        // Thread 0 streams 32-row chunks of the block's 256-byte column slice into the stages, two
+        // TMA boxes (32 rows x 128 bytes, 128-byte swizzle) per chunk; every warp waits for a chunk,
+        // takes its 32-byte slice (word gid of rows tig*4 + r and 16 + tig*4 + r), and releases the
+        // stage. Rows past the block are read too: their eq limbs are zero.
+        const int nch = (nr + 31) >> 5;
+        const CUtensorMap* tm = &jobs[jidx].tmap;
+        auto produce = [&](int i) {
+            const int st = i % PE_STAGES;
+            const uint32_t fb = pe_saddr(&full[st]);
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(fb), "r"(PE_STAGE) : "memory");
 #pragma unroll
-                for (int q = 0; q < 8; q++)
-                    w[q] = __ldcs(reinterpret_cast<const unsigned int*>(p + ((q >> 2) * 16 + (q & 3)) * pitch));
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; q++) {
-                    const int row = ch + (q >> 2) * 16 + tig * 4 + (q & 3);
-                    w[q] = row < nr ? __ldcs(reinterpret_cast<const unsigned int*>(
-                                          p + ((q >> 2) * 16 + (q & 3)) * pitch))
-                                    : 0u;
-                }
-            }
+            for (int half = 0; half < 2; half++)
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+                    "[%4];\n" ::"r"(pe_saddr(stg + st * PE_STAGE + half * (PE_STAGE / 2))),
+                    "l"(tm), "r"(cb * 256 + half * 128), "r"(r0 + 32 * i), "r"(fb)
+                    : "memory");
         };
-        uint32_t cur[8], nxt[8];
-        load_chunk(cur, 0);
-        for (int ch = 0; ch < nr; ch += 32) {
-            if (ch + 32 < nr) load_chunk(nxt, ch + 32);
-            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(lp + ch + tig * 4);
-            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(lp + ch + 16 + tig * 4);
+        if (threadIdx.x == 0) {
+            asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(tm) : "memory");
+            for (int i = 0; i < PE_STAGES && i < nch; i++) produce(i);
+        }
+        const uint8_t* lp = &et[SCALED ? warp : 0][gid][0];
+        // the lane's word within its 128-byte half of the chunk (warps 0-3: bytes 0..127 of the
+        // slice, warps 4-7: 128..255); 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r % 8)
+        const int hoff = (warp >> 2) * (PE_STAGE / 2), bb = (warp & 3) * 32 + gid * 4;
+        for (int i = 0; i < nch; i++) {
+            const int st = i % PE_STAGES;
+            const uint32_t par = (uint32_t)((i / PE_STAGES) & 1);
+            const bool got = pe_wait(pe_saddr(&full[st]), par);
+            uint32_t cur[8];
+            const uint8_t* sp = stg + st * PE_STAGE + hoff;
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const int row = (q >> 2) * 16 + tig * 4 + (q & 3);
+                cur[q] = *reinterpret_cast<const uint32_t*>(sp + row * 128 + ((((bb >> 4) ^ (row & 7))) << 4) + (bb & 15));
+            }
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(pe_saddr(&empty[st])) : "memory");
+            if (threadIdx.x == 0 && i + PE_STAGES < nch) {
+                // every warp has its words of chunk i: refill the stage with chunk i + PE_STAGES
+                if (pe_wait(pe_saddr(&empty[st]), par)) produce(i + PE_STAGES);
+            }
+            __syncwarp();  // the MMAs below are warp-wide
+            // a stalled copy leaves this block's sums wrong, not hung (the same decision in every lane)
+            if (!__all_sync(0xffffffffu, got) || !wactive) continue;
+            const int ch = 32 * i;
+            // B: limb gid of rows tig*4 .. +3 and 16 + tig*4 .. +3
+            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(lp + ch + tig * 4);
+            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(lp + ch + 16 + tig * 4);
             uint32_t t0[4], t1[4];
             transpose4x4(cur, t0);
             transpose4x4(cur + 4, t1);
+            // A rows (columns of the matrix) gid and gid + 8 of MMA g: int4, byte j = g of the
+            // lane's word, low nibble (w + 8 = nibble ^ 8) in row gid, high nibble in row gid + 8;
+            // int8, bytes 2g and 2g + 1 (w + 128 = byte ^ 0x80)
 #pragma unroll
-            for (int j = 0; j < 4; j++) {
+            for (int g = 0; g < NG; g++) {
                 if (W4) {
-                    // u = nibble ^ 8 = w + 8: low nibbles are even columns, high nibbles odd ones
-                    const uint32_t x0 = t0[j] ^ 0x88888888u, x1 = t1[j] ^ 0x88888888u;
-                    mma_u8(acc[2 * j], a0, a2, x0 & 0x0F0F0F0Fu, x1 & 0x0F0F0F0Fu);
-                    mma_u8(acc[2 * j + 1], a0, a2, (x0 >> 4) & 0x0F0F0F0Fu, (x1 >> 4) & 0x0F0F0F0Fu);
+                    const uint32_t x0 = t0[g] ^ 0x88888888u, x1 = t1[g] ^ 0x88888888u;
+                    mma_u8(acc[g], x0 & 0x0F0F0F0Fu, (x0 >> 4) & 0x0F0F0F0Fu, x1 & 0x0F0F0F0Fu, (x1 >> 4) & 0x0F0F0F0Fu,
+                           b0, b1);
                 } else {
-                    // u = byte ^ 0x80 = w + 128
-                    mma_u8(acc[j], a0, a2, t0[j] ^ 0x80808080u, t1[j] ^ 0x80808080u);
+                    mma_u8(acc[g], t0[2 * g] ^ 0x80808080u, t0[2 * g + 1] ^ 0x80808080u, t1[2 * g] ^ 0x80808080u,
+                           t1[2 * g + 1] ^ 0x80808080u, b0, b1);
                 }
             }
-#pragma unroll
-            for (int q = 0; q < 8; q++) cur[q] = nxt[q];
         }
     }
-    // C[limb gid][n = 2 tig + e] of group j (and nibble parity) belongs to column
-    // 2 (4 n + j) + parity (int4) or 4 n + j (int8) of the warp's slice
+    __syncthreads();  // every warp is done with the stages, which now hold the sums
+    // D[m][n] of MMA g: m = gid -> column 2 (4 gid + g) (int4) or 4 gid + 2 g (int8), m = gid + 8 ->
+    // the next column; n = 2 tig + e -> limb. c0, c1 hold m = gid, c2, c3 m = gid + 8.
     if (!wactive) return;
 #pragma unroll
     for (int g = 0; g < NG; g++) {
+        const int col = W4 ? 2 * (4 * gid + g) : 4 * gid + 2 * g;
 #pragma unroll
         for (int e = 0; e < 2; e++) {
-            const int n = 2 * tig + e;
-            const int col = W4 ? 2 * (4 * n + (g >> 1)) + (g & 1) : 4 * n + g;
-            red[warp][col * 8 + gid] = acc[g][e];
+            red[warp][col * 8 + 2 * tig + e] = acc[g][e];
+            red[warp][(col + 1) * 8 + 2 * tig + e] = acc[g][2 + e];
         }
     }
     __syncwarp();
@@ -392,6 +452,14 @@ __global__ void partial_fin_kernel(const PeJob* __restrict__ jobs) {
     }
 }
 
+template <bool W4, bool SCALED>
+cudaError_t pe_tc_launch(const PeJob* dj, int n, int64_t blocks, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(partial_tc_kernel<W4, SCALED>, cudaFuncAttributeMaxDynamicSharedMemorySize, PE_DYN);
+    if (e != cudaSuccess) return e;
+    partial_tc_kernel<W4, SCALED><<<(unsigned)blocks, PE_THREADS, PE_DYN, s>>>(dj, n);
+    return cudaGetLastError();
+}
+
 // About `waves` blocks per SM, at most max_rows rows per block (a multiple of 8, or of 32 on the
 // tensor-core path).
 void pe_plan_shape(int num_sms, int rows, int cols, int block_cols, int max_rows, int row_step, int waves,
@@ -405,10 +473,44 @@ void pe_plan_shape(int num_sms, int rows, int cols, int block_cols, int max_rows
     splits = (rows + rpb - 1) / rpb;
 }
 
-// The tensor-core path needs whole 32-byte warp slices in every row, read as 32-bit words.
+// cuTensorMapEncodeTiled through the runtime (no link-time dependency on the driver library)
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            p = nullptr;
+        }
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// The matrix as a 2-D byte tensor for TMA: 32-row x 128-byte boxes, 128-byte swizzle, zero fill
+bool pe_make_tmap(const FpPeJob& q, CUtensorMap* tm) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tmap_encoder();
+    if (!enc) return false;
+    const cuuint64_t pitch = q.bits == 4 ? (cuuint64_t)(q.cols + 1) / 2 : (cuuint64_t)q.cols;
+    const cuuint64_t dims[2] = {pitch, (cuuint64_t)q.rows};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {128, 32}, estr[2] = {1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(q.mat), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tensor-core path needs whole 32-byte warp slices in every row and a matrix that TMA can
+// read (16-byte aligned base and row pitch).
 bool pe_tc_ok(const FpPeJob& q) {
     const int64_t pitch = q.bits == 4 ? (q.cols + 1) / 2 : q.cols;
-    return ((uintptr_t)q.mat % 4 == 0) && (q.cols % (q.bits == 4 ? 64 : 32) == 0) && (pitch % 4 == 0);
+    return ((uintptr_t)q.mat % 16 == 0) && (q.cols % (q.bits == 4 ? 64 : 32) == 0) && (pitch % 16 == 0) &&
+           tmap_encoder() != nullptr;
+}
+
+void pe_plan_cuda_core(int num_sms, const FpPeJob& q, int& col_blocks, int& rpb, int& splits) {
+    pe_plan_shape(num_sms, q.rows, q.cols, PE_BLOCK_COLS, PE_MAX_ROWS, 8, 2, col_blocks, rpb, splits);
 }
 
 void pe_plan(int num_sms, const FpPeJob& q, bool& tc, int& col_blocks, int& rpb, int& splits) {
@@ -462,6 +564,11 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         d.v = q.v;
         bool tc;
         pe_plan(c->num_sms, q, tc, d.col_blocks, d.rows_per_block, d.splits);
+        memset(&d.tmap, 0, sizeof d.tmap);
+        if (tc && !pe_make_tmap(q, &d.tmap)) {  // no tensor map: the CUDA-core kernel
+            tc = false;
+            pe_plan_cuda_core(c->num_sms, q, d.col_blocks, d.rows_per_block, d.splits);
+        }
         const int64_t pitch = q.bits == 4 ? (q.cols + 1) / 2 : q.cols;
         // the fast path loads 4 (int4) or 8 (int8) bytes per lane and row
         d.aligned = ((uintptr_t)q.mat % 16 == 0) && (q.cols % PE_COLS == 0) &&
@@ -502,10 +609,11 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         if (var == 1) partial_many_kernel<false, true><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
         if (var == 2) partial_many_kernel<true, false><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
         if (var == 3) partial_many_kernel<true, true><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
-        if (var == 4) partial_tc_kernel<false, false><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
-        if (var == 5) partial_tc_kernel<false, true><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
-        if (var == 6) partial_tc_kernel<true, false><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
-        if (var == 7) partial_tc_kernel<true, true><<<(unsigned)blocks, PE_THREADS, 0, s>>>(dj, n);
+        static_assert(PE_STAGES * PE_STAGE >= 8 * 64 * 8 * 4, "the stages must hold the per-warp sums");
+        if (var == 4) FP_CUDA(c, (pe_tc_launch<false, false>(dj, n, blocks, s)));
+        if (var == 5) FP_CUDA(c, (pe_tc_launch<false, true>(dj, n, blocks, s)));
+        if (var == 6) FP_CUDA(c, (pe_tc_launch<true, false>(dj, n, blocks, s)));
+        if (var == 7) FP_CUDA(c, (pe_tc_launch<true, true>(dj, n, blocks, s)));
         fp_toc(c, s, slot);
         FP_CUDA(c, cudaGetLastError());
     }
