@@ -127,7 +127,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
     sc_round: matmul sum-check rounds over 2 x 2^26-element vectors (64 sites,
       W 1 x 2^20 int4, one token); round 1 reads A and B, later rounds fold
       in place of the next evaluation (read 4, write 2 values per pair).
-    partial_acc: eq-weighted row contraction of a 16384 x 16384 int4 matrix.
+    partial_acc: eq-weighted row contraction of a 16384 x 16384 int4 matrix (the
+      weight side) and of a 16384 x 16384 int8 matrix (the activation side).
     gkr_round: LogUp layer rounds over 2^26 keys (one 8192 x 64 x 8192 int8 site).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
@@ -173,6 +174,10 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
         z = [int(x) for x in rng.integers(0, fp.P, size=14, dtype="uint64")]
         measure("partial_eval_int4_16384^2", "partial_acc",
                 lambda: ctx.partial_eval(mat, 4, None, rows, cols, z, outv), big=1 << 26)
+        del mat
+        mat = torch.from_numpy(workloads.int8_uniform(rng, (rows, cols))).to(dev)
+        measure("partial_eval_int8_16384^2", "partial_acc",
+                lambda: ctx.partial_eval(mat, 8, None, rows, cols, z, outv), big=1 << 26)
         del mat, outv
 
     if "gemm" in which:
