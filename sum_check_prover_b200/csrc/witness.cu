@@ -334,12 +334,25 @@ __device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
 __device__ __forceinline__ uint32_t tc_off(int row, int kk) { return (row >> 3) * 1024 + kk * 128 + (row & 7) * 16; }
 
 // cp.async of k-tile k0 into a stage (zero fill outside the matrices)
+// 16-byte chunk c of a k-tile -> (row, k chunk): eight consecutive lanes take eight consecutive
+// rows of one k chunk, i.e. one whole 128-byte core matrix, so shared-memory writes do not
+// collide on banks (global reads stay whole 32-byte sectors: four k chunks of a row per warp)
+__device__ __forceinline__ void tc_chunk(int c, int& row, int& kk) {
+    row = (c & 7) | ((c >> 6) << 3);
+    kk = (c >> 3) & 7;
+}
+
+// packed int4 staging: row r's 16-byte chunk kq at r * 64 + (kq ^ ((r >> 1) & 3)) * 16, so
+// that eight consecutive rows of one chunk hit different banks
+__device__ __forceinline__ uint32_t tc_pk_off(int row, int kq) { return row * 64 + ((kq ^ ((row >> 1) & 3)) << 4); }
+
 template <bool W4, int BN>
 __device__ __forceinline__ void tc_issue(const SiteDev& S, int j0, int i0, int k0, uint8_t* sa, uint8_t* sb) {
     const int tid = threadIdx.x;
 #pragma unroll
     for (int u = 0; u < TC_A_BYTES / 16 / TC_THREADS; u++) {
-        const int c = tid + TC_THREADS * u, row = c >> 3, kk = c & 7;
+        int row, kk;
+        tc_chunk(tid + TC_THREADS * u, row, kk);
         const int j = j0 + row, k = k0 + kk * 16;
         const bool ok = j < S.N && k < S.K;
         cp_async16(sa + tc_off(row, kk), ok ? S.xt + (int64_t)j * S.K + k : S.xt, ok ? 16 : 0);
@@ -353,12 +366,13 @@ __device__ __forceinline__ void tc_issue(const SiteDev& S, int j0, int i0, int k
             const int c = tid + TC_THREADS * u, row = c >> 2, kq = c & 3;
             const int i = i0 + row, k = k0 + kq * 32;
             const bool ok = i < S.M && k < S.K;
-            cp_async16(pk + row * 64 + kq * 16, ok ? S.w + (int64_t)i * pitch + (k >> 1) : S.w, ok ? 16 : 0);
+            cp_async16(pk + tc_pk_off(row, kq), ok ? S.w + (int64_t)i * pitch + (k >> 1) : S.w, ok ? 16 : 0);
         }
     } else {
 #pragma unroll
         for (int u = 0; u < BN * 8 / TC_THREADS; u++) {
-            const int c = tid + TC_THREADS * u, row = c >> 3, kk = c & 7;
+            int row, kk;
+            tc_chunk(tid + TC_THREADS * u, row, kk);
             const int i = i0 + row, k = k0 + kk * 16;
             const bool ok = i < S.M && k < S.K;
             cp_async16(sb + tc_off(row, kk), ok ? S.w + (int64_t)i * S.K + k : S.w, ok ? 16 : 0);
@@ -366,7 +380,8 @@ __device__ __forceinline__ void tc_issue(const SiteDev& S, int j0, int i0, int k
     }
 }
 
-// int4 stage: packed upper half -> int8 core-matrix layout (read everything first, then write)
+// int4 stage: packed upper half -> int8 core-matrix layout (read everything first, then write);
+// lane l takes row l % 8 of its group, so both the reads and the writes are bank-conflict free
 template <int BN>
 __device__ __forceinline__ void tc_expand(uint8_t* sb) {
     const int tid = threadIdx.x;
@@ -374,13 +389,13 @@ __device__ __forceinline__ void tc_expand(uint8_t* sb) {
     uint4 v[BN * 4 / TC_THREADS];
 #pragma unroll
     for (int u = 0; u < BN * 4 / TC_THREADS; u++) {
-        const int c = tid + TC_THREADS * u;
-        v[u] = *reinterpret_cast<const uint4*>(pk + (c >> 2) * 64 + (c & 3) * 16);
+        const int c = tid + TC_THREADS * u, row = (c & 7) | ((c >> 5) << 3), kq = (c >> 3) & 3;
+        v[u] = *reinterpret_cast<const uint4*>(pk + tc_pk_off(row, kq));
     }
     __syncthreads();
 #pragma unroll
     for (int u = 0; u < BN * 4 / TC_THREADS; u++) {
-        const int c = tid + TC_THREADS * u, row = c >> 2, kq = c & 3;
+        const int c = tid + TC_THREADS * u, row = (c & 7) | ((c >> 5) << 3), kq = (c >> 3) & 3;
         // 32 nibbles (low nibble first) -> 32 int8 in two 16-byte chunks
         const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
         uint32_t o[8];
