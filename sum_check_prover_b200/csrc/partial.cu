@@ -304,8 +304,9 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
     }
     __syncthreads();
     uint64_t es = 0;  // sum of the weights this warp's columns see
+    const int kend = (nr + 31) & ~31;  // whole chunks: positions past nr read zero limbs
     if (!SCALED) {
-        for (int k = threadIdx.x; k < ROWS; k += PE_THREADS) {
+        for (int k = threadIdx.x; k < kend; k += PE_THREADS) {
             // with v < 5 the rows are i = n < 2^v and H = {1}
             const uint64_t e = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
 #pragma unroll
@@ -319,10 +320,10 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
 #pragma unroll
         for (int w = 0; w < PE_THREADS / 32; w++) es = gl_add(es, wsum[w]);
     } else {
-        for (int k = threadIdx.x; k < ROWS; k += PE_THREADS) eqs[k] = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
+        for (int k = threadIdx.x; k < kend; k += PE_THREADS) eqs[k] = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
         __syncthreads();
         const int g = wc0 / 64;
-        for (int k = lane; k < ROWS; k += 32) {
+        for (int k = lane; k < kend; k += 32) {
             uint64_t e = 0;
             if (wactive && k < nr) e = gl_mul_small(eqs[k], (int32_t)__ldg(J.scales + (int64_t)(r0 + k) * G + g));
 #pragma unroll

@@ -299,11 +299,16 @@ constexpr int TC_THREADS = 256;
 constexpr int TC_A_BYTES = TC_BM * TC_BK;  // 16 KB
 constexpr uint32_t TC_WAIT_LIMIT = 1u << 24;  // mbarrier polls before the kernel gives up
 
-template <int BN>
+// Shared-memory plan: a ring of STAGES k-tiles of A (and of B for int8 weights; for int4 weights
+// a ring of packed tiles plus a double buffer of expanded int8 B tiles), within 224 KB
+template <bool W4, int BN>
 struct TcCfg {
-    static constexpr int B_BYTES = BN * TC_BK;
-    static constexpr int STAGES = BN == 256 ? 4 : 6;
-    static constexpr int SMEM = STAGES * (TC_A_BYTES + B_BYTES) + 1024;
+    static constexpr int B_BYTES = BN * TC_BK;      // an int8 B tile
+    static constexpr int PK_BYTES = BN * TC_BK / 2;  // a packed int4 B tile
+    static constexpr int RING = W4 ? TC_A_BYTES + PK_BYTES : TC_A_BYTES + B_BYTES;
+    static constexpr int FIXED = W4 ? 2 * B_BYTES : 0;
+    static constexpr int STAGES = (224 * 1024 - FIXED) / RING;
+    static constexpr int SMEM = STAGES * RING + FIXED + 1024;
     // s32 accumulator, s8 x s8, both K-major, N = BN, M = 128
     static constexpr uint32_t IDESC =
         (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(TC_BM >> 4) << 24);
@@ -348,6 +353,7 @@ __device__ __forceinline__ uint32_t tc_pk_off(int row, int kq) { return row * 64
 
 template <bool W4, int BN>
 __device__ __forceinline__ void tc_issue(const SiteDev& S, int j0, int i0, int k0, uint8_t* sa, uint8_t* sb) {
+    // sb: the int8 B tile, or (int4) the packed tile
     const int tid = threadIdx.x;
 #pragma unroll
     for (int u = 0; u < TC_A_BYTES / 16 / TC_THREADS; u++) {
@@ -358,9 +364,9 @@ __device__ __forceinline__ void tc_issue(const SiteDev& S, int j0, int i0, int k
         cp_async16(sa + tc_off(row, kk), ok ? S.xt + (int64_t)j * S.K + k : S.xt, ok ? 16 : 0);
     }
     if (W4) {
-        // packed rows (64 bytes of the k-tile each) in the stage's upper half
+        // packed rows: 64 bytes of the k-tile each
         const int pitch = S.K >> 1;
-        uint8_t* pk = sb + TcCfg<BN>::B_BYTES / 2;
+        uint8_t* pk = sb;
 #pragma unroll
         for (int u = 0; u < BN * 4 / TC_THREADS; u++) {
             const int c = tid + TC_THREADS * u, row = c >> 2, kq = c & 3;
@@ -380,19 +386,17 @@ __device__ __forceinline__ void tc_issue(const SiteDev& S, int j0, int i0, int k
     }
 }
 
-// int4 stage: packed upper half -> int8 core-matrix layout (read everything first, then write);
-// lane l takes row l % 8 of its group, so both the reads and the writes are bank-conflict free
+// int4: a packed tile -> the int8 core-matrix layout of an expanded B buffer; lane l takes
+// row l % 8 of its group, so both the reads and the writes are bank-conflict free
 template <int BN>
-__device__ __forceinline__ void tc_expand(uint8_t* sb) {
+__device__ __forceinline__ void tc_expand(const uint8_t* pk, uint8_t* sb) {
     const int tid = threadIdx.x;
-    const uint8_t* pk = sb + TcCfg<BN>::B_BYTES / 2;
     uint4 v[BN * 4 / TC_THREADS];
 #pragma unroll
     for (int u = 0; u < BN * 4 / TC_THREADS; u++) {
         const int c = tid + TC_THREADS * u, row = (c & 7) | ((c >> 5) << 3), kq = (c >> 3) & 3;
         v[u] = *reinterpret_cast<const uint4*>(pk + tc_pk_off(row, kq));
     }
-    __syncthreads();
 #pragma unroll
     for (int u = 0; u < BN * 4 / TC_THREADS; u++) {
         const int c = tid + TC_THREADS * u, row = (c & 7) | ((c >> 5) << 3), kq = (c >> 3) & 3;
@@ -448,12 +452,14 @@ __device__ __forceinline__ void tc_store16(const SiteDev& S, int j, int i, const
 template <bool W4, int BN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     witness_tc_kernel(const SiteDev* __restrict__ sites, int nsites, volatile uint64_t* err) {
-    using C = TcCfg<BN>;
+    using C = TcCfg<W4, BN>;
     constexpr int ST = C::STAGES;
+    constexpr int SBT = W4 ? C::PK_BYTES : C::B_BYTES;  // ring slot of the B side
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     uint8_t* sA = smem;
-    uint8_t* sB = smem + ST * TC_A_BYTES;
+    uint8_t* sB = smem + ST * TC_A_BYTES;  // int8 B tiles, or packed int4 tiles
+    uint8_t* sX = sB + ST * SBT;            // int4: two expanded B tiles
     __shared__ __align__(8) uint64_t mbar[ST];
     __shared__ uint32_t tmem_base;
     __shared__ int s_fail;
@@ -480,7 +486,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // prologue: tiles 0 .. ST-3 in flight (prefetch distance ST - 2)
 #pragma unroll
     for (int t = 0; t < ST - 2; t++) {
-        if (t < nk) tc_issue<W4, BN>(S, j0, i0, t * TC_BK, sA + t * TC_A_BYTES, sB + t * C::B_BYTES);
+        if (t < nk) tc_issue<W4, BN>(S, j0, i0, t * TC_BK, sA + t * TC_A_BYTES, sB + t * SBT);
         cp_async_commit();
     }
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
@@ -491,23 +497,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int kt = 0; kt < nk; kt++) {
         const int st = kt % ST;
         // refill the stage of tile kt + ST - 2; its previous tile (kt - 2) must be done with it
+        // (for int4 this also frees the expanded buffer that tile kt is about to use)
         const int nt = kt + ST - 2, ns = nt % ST;
-        const bool late = nt < nk && kt >= 2 && !tc_wait(smem_addr(&mbar[ns]), (uint32_t)(((kt - 2) / ST) & 1));
+        const bool late = (W4 || nt < nk) && kt >= 2 && !tc_wait(smem_addr(&mbar[ns]), (uint32_t)(((kt - 2) / ST) & 1));
         if (__syncthreads_or(late)) {
             if (tid == 0) s_fail = 1;
             break;
         }
-        if (nt < nk) tc_issue<W4, BN>(S, j0, i0, nt * TC_BK, sA + ns * TC_A_BYTES, sB + ns * C::B_BYTES);
+        if (nt < nk) tc_issue<W4, BN>(S, j0, i0, nt * TC_BK, sA + ns * TC_A_BYTES, sB + ns * SBT);
         cp_async_commit();
         cp_async_wait<ST - 2>();  // tile kt has landed (this thread's copies)
         __syncthreads();
-        if (W4) tc_expand<BN>(sB + st * C::B_BYTES);
+        uint8_t* bt = W4 ? sX + (kt & 1) * C::B_BYTES : sB + st * SBT;  // the B tile the MMAs read
+        if (W4) tc_expand<BN>(sB + st * SBT, bt);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic writes -> tensor-core reads
         asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
         __syncthreads();
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
         if (tid == 0) {
-            const uint32_t a0 = smem_addr(sA + st * TC_A_BYTES), b0 = smem_addr(sB + st * C::B_BYTES);
+            const uint32_t a0 = smem_addr(sA + st * TC_A_BYTES), b0 = smem_addr(bt);
 #pragma unroll
             for (int kc = 0; kc < TC_BK / 32; kc++) {
                 const uint32_t en = (kt > 0 || kc > 0) ? 1u : 0u;
@@ -584,10 +592,10 @@ int launch_tc_bn(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
     memcpy(hst, h.data(), sz);
     FP_CUDA(c, cudaMemcpyAsync(dsites, hst, sz, cudaMemcpyHostToDevice, st));
     auto kern = witness_tc_kernel<W4, BN>;
-    FP_CUDA(c, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM));
+    FP_CUDA(c, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<W4, BN>::SMEM));
     int slot;
     fp_tic(c, st, K_GEMM, bytes, &slot);
-    kern<<<(unsigned)tiles, TC_THREADS, TcCfg<BN>::SMEM, st>>>(dsites, (int)h.size(), &c->mb_dev->err);
+    kern<<<(unsigned)tiles, TC_THREADS, TcCfg<W4, BN>::SMEM, st>>>(dsites, (int)h.size(), &c->mb_dev->err);
     fp_toc(c, st, slot);
     FP_CUDA(c, cudaGetLastError());
     return FP_OK;
