@@ -283,10 +283,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 //
 // D = Xt . W^T for unscaled sites on the 5th-generation tensor cores: one CTA per
 // 128-token x BN-row tile, the accumulator (128 lanes x BN columns of s32) in
-// tensor memory, operands in shared memory in the K-major core-matrix layout
-// (8 rows x 16 bytes per core matrix; element (row, byte kb) at
-// (row / 8) * 1024 + (kb / 16) * 128 + (row % 8) * 16 + kb % 16 within a
-// 128-byte-deep k-tile). cp.async fills stage kt % S two tiles before use;
+// tensor memory, operands in shared memory in the K-major layout with the
+// 128-byte swizzle (a k-tile is 128 bytes deep: row r at (r / 8) * 1024 +
+// (r % 8) * 128, its 16-byte chunk c at chunk position c ^ (r % 8)); the four
+// K = 32 MMAs of a k-tile start 32 bytes apart inside the swizzle atom. cp.async fills stage kt % S two tiles before use;
 // int4 weights land packed in the upper half of their stage and are expanded
 // to int8 in place just before the MMAs. One thread issues the four K = 32 MMAs
 // of a k-tile and commits them to the stage's mbarrier; a stage is refilled
@@ -316,11 +316,11 @@ struct TcCfg {
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-// shared-memory matrix descriptor: K-major, no swizzle, core matrices 128 B apart along K
-// (leading byte offset) and 1024 B apart along M / N (stride byte offset)
+// shared-memory matrix descriptor: K-major with the 128-byte swizzle (8-row x 128-byte atoms,
+// 1024 B apart along M / N: the stride byte offset; the leading byte offset is unused), version 1
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46);
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
 __device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
@@ -336,12 +336,16 @@ __device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
     return false;
 }
 
-__device__ __forceinline__ uint32_t tc_off(int row, int kk) { return (row >> 3) * 1024 + kk * 128 + (row & 7) * 16; }
+// byte offset of 16-byte chunk kk of row `row` in a 128-byte-deep k-tile: row r of 8-row atom
+// r / 8 at (r / 8) * 1024 + (r % 8) * 128, chunk kk stored at chunk position kk ^ (r % 8)
+__device__ __forceinline__ uint32_t tc_off(int row, int kk) {
+    return (row >> 3) * 1024 + (row & 7) * 128 + ((kk ^ (row & 7)) << 4);
+}
 
 // cp.async of k-tile k0 into a stage (zero fill outside the matrices)
 // 16-byte chunk c of a k-tile -> (row, k chunk): eight consecutive lanes take eight consecutive
-// rows of one k chunk, i.e. one whole 128-byte core matrix, so shared-memory writes do not
-// collide on banks (global reads stay whole 32-byte sectors: four k chunks of a row per warp)
+// rows of one k chunk, which the swizzle spreads over all 32 banks (global reads stay whole
+// 32-byte sectors: four k chunks of a row per warp)
 __device__ __forceinline__ void tc_chunk(int c, int& row, int& kk) {
     row = (c & 7) | ((c >> 6) << 3);
     kk = (c >> 3) & 7;
@@ -386,7 +390,7 @@ __device__ __forceinline__ void tc_issue(const SiteDev& S, int j0, int i0, int k
     }
 }
 
-// int4: a packed tile -> the int8 core-matrix layout of an expanded B buffer; lane l takes
+// int4: a packed tile -> the swizzled int8 layout of an expanded B buffer; lane l takes
 // row l % 8 of its group, so both the reads and the writes are bank-conflict free
 template <int BN>
 __device__ __forceinline__ void tc_expand(const uint8_t* pk, uint8_t* sb) {
@@ -522,7 +526,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 asm volatile(
                     "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                     "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-                    "l"(tc_desc(a0 + kc * 256)), "l"(tc_desc(b0 + kc * 256)), "r"(C::IDESC), "r"(en));
+                    "l"(tc_desc(a0 + kc * 32)), "l"(tc_desc(b0 + kc * 32)), "r"(C::IDESC), "r"(en));
             }
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
                 smem_addr(&mbar[st])));
