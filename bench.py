@@ -75,7 +75,8 @@ def sumcheck_elems(wl) -> int:
 
 
 class Clocks:
-    """nvidia-smi samples during the timed region."""
+    """SM clock and clock-event reasons sampled every 2 ms during the timed region (NVML
+    from a thread, read-only queries; nvidia-smi every 200 ms when NVML is unavailable)."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -85,8 +86,50 @@ class Clocks:
         self.index = index
         self.proc = None
         self.f = None
+        self.nvml = None
+        self.samples = []
+        self.stop_flag = False
+        self.thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _poll(self):
+        nv = self.nvml
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        while not self.stop_flag:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = (nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                      if hasattr(nv, "nvmlDeviceGetCurrentClocksEventReasons")
+                      else nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h))
+                self.samples.append((mhz, [k for k, v in bits.items() if rs & v]))
+            except Exception:
+                pass
+            self.started.set()
+            time.sleep(0.002)
 
     def start(self):
+        if self.nvml is not None:
+            import threading
+
+            self.samples = []
+            self.stop_flag = False
+            self.started = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            self.started.wait(timeout=5)
+            self.samples = []  # the region starts now
+            return
         try:
             self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
@@ -96,6 +139,14 @@ class Clocks:
             self.proc = None
 
     def stop(self) -> dict:
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            self.thread = None
+            sm = [m for m, _ in self.samples]
+            reasons = sorted({r for _, rs in self.samples for r in rs})
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                    "samples": len(sm), "reasons": reasons, "source": "nvml, every 2 ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
@@ -117,7 +168,7 @@ class Clocks:
                 if val.strip().lower().startswith("active"):
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
 def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
