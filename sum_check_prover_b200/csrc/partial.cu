@@ -13,13 +13,15 @@
 //
 // Tensor-core path (matrices whose rows hold whole 32-byte warp slices): the
 // field weights are split into 8 byte limbs, e = sum_l e_l 2^(8 l), and
-// C[l][c] = sum_i e_l[i] u[i][c] is an exact u8 x u8 -> s32 matrix product
-// (mma m16n8k32, limbs as the A rows, matrix rows as K, columns as N). Each
-// lane loads one 32-bit word from each of 4 consecutive rows and transposes
-// the 4 x 4 bytes with byte permutes into B fragments; int4 nibbles split into
-// two fragments. The limbs are recombined mod p once per block. With scales,
-// the weight of row i in column group g is e_i s[i][g] (a warp's columns lie
-// in one group), so the unsigned operand stays w + off.
+// C[c][l] = sum_i u[i][c] e_l[i] is an exact 8-bit -> s32 matrix product
+// (mma m16n8k32: 16 matrix columns as the A rows, matrix rows as K, limbs as
+// N). TMA streams 32-row chunks into shared memory; each warp takes its 32-byte
+// slice with transposing ldmatrix loads, which hand it A fragments directly.
+// int8 bytes enter as signed operands; an int4 byte b ^ 0x88 =
+// 16 (w_odd + 8) + (w_even + 8) enters whole and as its low nibble, and the
+// odd column is the difference over 16. The limbs are recombined mod p once
+// per block. With scales, the weight of row i in column group g is
+// e_i s[i][g] (a warp's columns lie in one group).
 //
 // All contractions of a call go into one launch per kernel variant (a job
 // list; the MoE layer has hundreds of sites). eq(z, i) for the block's rows
@@ -68,6 +70,26 @@ __device__ __forceinline__ void mma_u8(uint32_t (&c)[4], uint32_t a0, uint32_t a
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D (16 columns x 8 limbs) += A (signed bytes) . B (unsigned limbs)
+__device__ __forceinline__ void mma_s8u8(uint32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two 16 x 16-byte matrices (rows named by lanes 0-15 and 16-31), transposed on the way in: the
+// lane gets, per matrix, column gid of rows 4 tig .. 4 tig + 3 and column gid + 8 of the same rows
+// (four bytes per register, row 4 tig in the low byte): the m16n8k32 A fragment of a row-major
+// (K rows x 16 columns) tile.
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t (&f)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(f[0]), "=r"(f[1]), "=r"(f[2]), "=r"(f[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
 // ---- TMA pipeline (shared-memory stages filled by cp.async.bulk.tensor, tracked by mbarriers) ----
 constexpr int PE_STAGES = 6;               // 32-row chunks in flight per block
 constexpr int PE_STAGE = 2 * 32 * 128;     // one chunk: two 32 x 128-byte boxes
@@ -87,16 +109,6 @@ __device__ __forceinline__ bool pe_wait(uint32_t mbar, uint32_t parity) {
         if (ok) return true;
     }
     return false;
-}
-
-// rows w[0..3] -> t[j] = byte j of each row (row r in byte r)
-__device__ __forceinline__ void transpose4x4(const uint32_t* w, uint32_t* t) {
-    const uint32_t x0 = __byte_perm(w[0], w[1], 0x5140), x1 = __byte_perm(w[0], w[1], 0x7362);
-    const uint32_t x2 = __byte_perm(w[2], w[3], 0x5140), x3 = __byte_perm(w[2], w[3], 0x7362);
-    t[0] = __byte_perm(x0, x2, 0x5410);
-    t[1] = __byte_perm(x0, x2, 0x7632);
-    t[2] = __byte_perm(x1, x3, 0x5410);
-    t[3] = __byte_perm(x1, x3, 0x7632);
 }
 
 __device__ __forceinline__ uint64_t fold_lohi(uint64_t lo, uint64_t hi) {
@@ -340,12 +352,11 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
     {
         // Thread 0 streams 32-row chunks of the block's 256-byte column slice into the stages, two
         // TMA boxes (32 rows x 128 bytes, 128-byte swizzle) per chunk; every warp waits for a chunk,
-        // takes its 32-byte slice (word gid of rows tig*4 + r and 16 + tig*4 + r), and releases the
+        // loads its 32-byte slice as two transposed 32 x 16-byte A fragments, and releases the
         // stage. Rows past the block are read too: their eq limbs are zero.
         const int nch = (nr + 31) >> 5;
         const CUtensorMap* tm = &jobs[jidx].tmap;
-        auto produce = [&](int i) {
-            const int st = i % PE_STAGES;
+        auto produce = [&](int i, int st) {
             const uint32_t fb = pe_saddr(&full[st]);
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(fb), "r"(PE_STAGE) : "memory");
 #pragma unroll
@@ -358,82 +369,102 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
         };
         if (threadIdx.x == 0) {
             asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(tm) : "memory");
-            for (int i = 0; i < PE_STAGES && i < nch; i++) produce(i);
+            for (int i = 0; i < PE_STAGES && i < nch; i++) produce(i, i);
         }
         const uint8_t* lp = &et[SCALED ? warp : 0][gid][0];
-        // the lane's word within its 128-byte half of the chunk (warps 0-3: bytes 0..127 of the
-        // slice, warps 4-7: 128..255); 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r % 8)
-        const int hoff = (warp >> 2) * (PE_STAGE / 2), bb = (warp & 3) * 32 + gid * 4;
+        // ldmatrix row addresses: lane L names row L of the chunk (lanes 0-15 the first 16 x 16-byte
+        // matrix, lanes 16-31 the second); the warp's slice is 16-byte chunks c0 and c0 + 1 of its
+        // 128-byte half, and 128-byte swizzle puts chunk c of row r at c ^ (r % 8)
+        const int c0 = (warp & 3) * 2;
+        const uint32_t hoff = (uint32_t)((warp >> 2) * (PE_STAGE / 2) + lane * 128);
+        const uint32_t o0 = hoff + ((c0 ^ (lane & 7)) << 4), o1 = hoff + (((c0 + 1) ^ (lane & 7)) << 4);
+        const uint32_t sbase = pe_saddr(stg);
+        int st = 0;
+        uint32_t par = 0;
         for (int i = 0; i < nch; i++) {
-            const int st = i % PE_STAGES;
-            const uint32_t par = (uint32_t)((i / PE_STAGES) & 1);
             const bool got = pe_wait(pe_saddr(&full[st]), par);
-            uint32_t cur[8];
-            const uint8_t* sp = stg + st * PE_STAGE + hoff;
-#pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const int row = (q >> 2) * 16 + tig * 4 + (q & 3);
-                cur[q] = *reinterpret_cast<const uint32_t*>(sp + row * 128 + ((((bb >> 4) ^ (row & 7))) << 4) + (bb & 15));
-            }
+            __syncwarp();  // ldmatrix is warp-wide
+            // f[h][0..3]: the A fragment of bytes 16 h .. 16 h + 15 of the slice: f[h][0] holds byte
+            // column gid of rows 4 tig .. 4 tig + 3, f[h][1] column gid + 8, f[h][2], f[h][3] the same
+            // for rows 16 + 4 tig ..
+            uint32_t f[2][4];
+            const uint32_t sp = sbase + (uint32_t)(st * PE_STAGE);
+            ldsm_x2_trans(f[0], sp + o0);
+            ldsm_x2_trans(f[1], sp + o1);
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(pe_saddr(&empty[st])) : "memory");
             if (threadIdx.x == 0 && i + PE_STAGES < nch) {
-                // every warp has its words of chunk i: refill the stage with chunk i + PE_STAGES
-                if (pe_wait(pe_saddr(&empty[st]), par)) produce(i + PE_STAGES);
+                // every warp has its fragments of chunk i: refill the stage with chunk i + PE_STAGES
+                if (pe_wait(pe_saddr(&empty[st]), par)) produce(i + PE_STAGES, st);
             }
             __syncwarp();  // the MMAs below are warp-wide
+            const int ch = 32 * i;
+            if (++st == PE_STAGES) {
+                st = 0;
+                par ^= 1u;
+            }
             // a stalled copy leaves this block's sums wrong, not hung (the same decision in every lane)
             if (!__all_sync(0xffffffffu, got) || !wactive) continue;
-            const int ch = 32 * i;
             // B: limb gid of rows tig*4 .. +3 and 16 + tig*4 .. +3
             const uint32_t b0 = *reinterpret_cast<const uint32_t*>(lp + ch + tig * 4);
             const uint32_t b1 = *reinterpret_cast<const uint32_t*>(lp + ch + 16 + tig * 4);
-            uint32_t t0[4], t1[4];
-            transpose4x4(cur, t0);
-            transpose4x4(cur + 4, t1);
-            // A rows (columns of the matrix) gid and gid + 8 of MMA g: int4, byte j = g of the
-            // lane's word, low nibble (w + 8 = nibble ^ 8) in row gid, high nibble in row gid + 8;
-            // int8, bytes 2g and 2g + 1 (w + 128 = byte ^ 0x80)
 #pragma unroll
-            for (int g = 0; g < NG; g++) {
+            for (int h = 0; h < 2; h++) {
                 if (W4) {
-                    const uint32_t x0 = t0[g] ^ 0x88888888u, x1 = t1[g] ^ 0x88888888u;
-                    mma_u8(acc[g], x0 & 0x0F0F0F0Fu, (x0 >> 4) & 0x0F0F0F0Fu, x1 & 0x0F0F0F0Fu, (x1 >> 4) & 0x0F0F0F0Fu,
-                           b0, b1);
+                    // byte ^ 0x88 = 16 (w_odd + 8) + (w_even + 8): the whole byte (P) and its low
+                    // nibble (Q) give both columns, the odd one as (P - Q) / 16
+                    uint32_t x[4], lo[4];
+#pragma unroll
+                    for (int r = 0; r < 4; r++) {
+                        x[r] = f[h][r] ^ 0x88888888u;
+                        lo[r] = x[r] & 0x0F0F0F0Fu;
+                    }
+                    mma_u8(acc[2 * h], x[0], x[1], x[2], x[3], b0, b1);
+                    mma_u8(acc[2 * h + 1], lo[0], lo[1], lo[2], lo[3], b0, b1);
                 } else {
-                    mma_u8(acc[g], t0[2 * g] ^ 0x80808080u, t0[2 * g + 1] ^ 0x80808080u, t1[2 * g] ^ 0x80808080u,
-                           t1[2 * g + 1] ^ 0x80808080u, b0, b1);
+                    mma_s8u8(acc[h], f[h][0], f[h][1], f[h][2], f[h][3], b0, b1);
                 }
             }
         }
     }
     __syncthreads();  // every warp is done with the stages, which now hold the sums
-    // D[m][n] of MMA g: m = gid -> column 2 (4 gid + g) (int4) or 4 gid + 2 g (int8), m = gid + 8 ->
-    // the next column; n = 2 tig + e -> limb. c0, c1 hold m = gid, c2, c3 m = gid + 8.
+    // D[m][n]: m = byte column of the 16-byte half h (m = gid in c0, c1; gid + 8 in c2, c3),
+    // n = 2 tig + e = limb. int4: byte b holds columns 2 b (low nibble) and 2 b + 1.
     if (!wactive) return;
 #pragma unroll
-    for (int g = 0; g < NG; g++) {
-        const int col = W4 ? 2 * (4 * gid + g) : 4 * gid + 2 * g;
+    for (int h = 0; h < 2; h++) {
 #pragma unroll
         for (int e = 0; e < 2; e++) {
-            red[warp][col * 8 + 2 * tig + e] = acc[g][e];
-            red[warp][(col + 1) * 8 + 2 * tig + e] = acc[g][2 + e];
+#pragma unroll
+            for (int hm = 0; hm < 2; hm++) {
+                const int byte = 16 * h + gid + 8 * hm;
+                const int limb = 2 * tig + e;
+                if (W4) {
+                    const uint32_t P = acc[2 * h][2 * hm + e], Q = acc[2 * h + 1][2 * hm + e];
+                    red[warp][(2 * byte) * 8 + limb] = Q;
+                    red[warp][(2 * byte + 1) * 8 + limb] = (P - Q) >> 4;
+                } else {
+                    red[warp][byte * 8 + limb] = acc[h][2 * hm + e];
+                }
+            }
         }
     }
     __syncwarp();
-    const uint32_t off = W4 ? 8u : 128u;
-    const uint64_t corr = gl_mul(off, es);
+    // int4 sums are of w + 8 (corrected by 8 times the weight sum); int8 limb sums are signed
+    // (s8 matrix bytes): each is read with 2^31 added, and the added 2^31 sum_l 2^(8 l) is removed
+    const uint64_t corr = W4 ? gl_mul(8u, es) : gl_mul(1ull << 31, 0x0101010101010101ull);
+    const uint32_t flip = W4 ? 0u : 0x80000000u;
     for (int c = lane; c < WCOLS; c += 32) {
         const int gc = wc0 + c;
         if (gc >= J.cols) break;
-        // sum_l C_l 2^(8 l) with every C_l < 2^31: limbs 0..4 fit 64 bits, limbs 5..7 form
-        // (C5 + 2^8 C6 + 2^16 C7) 2^40 (< 2^88)
+        // sum_l C_l 2^(8 l) for C_l < 2^32: a = limbs 0..3, b = limbs 4..7 (each < 2^57), a + 2^32 b
         const uint32_t* C = &red[warp][c * 8];
-        uint64_t lo = (uint64_t)C[0] + ((uint64_t)C[1] << 8) + ((uint64_t)C[2] << 16) + ((uint64_t)C[3] << 24) +
-                      ((uint64_t)C[4] << 32);
-        const uint64_t up = (uint64_t)C[5] + ((uint64_t)C[6] << 8) + ((uint64_t)C[7] << 16);
-        uint64_t hi = up >> 24;
-        asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, 0;" : "+l"(lo), "+l"(hi) : "l"(up << 40));
+        const uint64_t a = (uint64_t)(C[0] ^ flip) + ((uint64_t)(C[1] ^ flip) << 8) + ((uint64_t)(C[2] ^ flip) << 16) +
+                           ((uint64_t)(C[3] ^ flip) << 24);
+        const uint64_t bq = (uint64_t)(C[4] ^ flip) + ((uint64_t)(C[5] ^ flip) << 8) + ((uint64_t)(C[6] ^ flip) << 16) +
+                            ((uint64_t)(C[7] ^ flip) << 24);
+        uint64_t lo = a, hi = bq >> 32;
+        asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, 0;" : "+l"(lo), "+l"(hi) : "l"(bq << 32));
         J.part[(int64_t)split * J.cols + gc] = gl_sub(gl_canon(gl_reduce_weak(lo, hi)), corr);
     }
 }
