@@ -60,6 +60,7 @@ constexpr int PE_COLS = 8;                   // columns per lane: one 32-bit (in
 constexpr int PE_BLOCK_COLS = 32 * PE_COLS;  // 256 columns per block
 constexpr int PE_UNROLL = 8;                 // rows whose loads a warp issues before using any of them
 constexpr int PE_MAX_ROWS = 256;             // 256 rows x 2^32 x 2^15 < 2^64: the sums stay exact
+constexpr int PE_TC_THREADS = PE_THREADS + 32;  // tensor-core path: 8 consumer warps and a TMA producer warp
 
 // D (16 columns x 8 limbs) += A (16 columns x 32 rows of the matrix) . B (32 rows x 8 limbs)
 __device__ __forceinline__ void mma_u8(uint32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -97,6 +98,9 @@ constexpr int PE_DYN = PE_STAGES * PE_STAGE + 1024;  // + alignment slack
 constexpr uint32_t PE_WAIT_LIMIT = 1u << 24;
 
 __device__ __forceinline__ uint32_t pe_saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// barrier 1 among the 8 consumer warps only (the producer warp never joins it)
+__device__ __forceinline__ void pe_consumers_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(PE_THREADS) : "memory"); }
 
 __device__ __forceinline__ bool pe_wait(uint32_t mbar, uint32_t parity) {
     for (uint32_t it = 0; it < PE_WAIT_LIMIT; it++) {
@@ -266,7 +270,7 @@ __host__ __device__ constexpr int tc_rows() {
 }
 
 template <bool W4, bool SCALED>
-__global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* __restrict__ jobs, int njobs) {
+__global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJob* __restrict__ jobs, int njobs) {
     constexpr int WCOLS = W4 ? 64 : 32;
     constexpr int NG = W4 ? 4 : 2;  // MMAs per 32-row chunk: 16 columns each
     constexpr int ROWS = tc_rows<SCALED>();
@@ -294,7 +298,39 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
             asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(pe_saddr(&empty[st])), "r"(PE_THREADS / 32));
         }
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::);
-    }  // visible after the barrier that follows the eq tables
+    }
+    __syncthreads();  // the barriers are initialised
+    const int nch = (nr + 31) >> 5;
+    if (warp == PE_THREADS / 32) {
+        // producer warp: one lane streams the block's 32-row chunks of its 256-byte column slice into
+        // the stages, two TMA boxes (32 rows x 128 bytes, 128-byte swizzle) per chunk, each stage once
+        // the consumer warps have released the chunk it held. Rows past the block are read too: their
+        // eq limbs are zero. A release that never comes ends the stream (the consumers' waits then
+        // run out too: wrong sums, no hang).
+        if (lane == 0) {
+            const CUtensorMap* tm = &jobs[jidx].tmap;
+            asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(tm) : "memory");
+            int st = 0;
+            uint32_t par = 0;
+            for (int i = 0; i < nch; i++) {
+                if (i >= PE_STAGES && !pe_wait(pe_saddr(&empty[st]), par ^ 1u)) break;
+                const uint32_t fb = pe_saddr(&full[st]);
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(fb), "r"(PE_STAGE) : "memory");
+#pragma unroll
+                for (int half = 0; half < 2; half++)
+                    asm volatile(
+                        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+                        "%3}], [%4];\n" ::"r"(pe_saddr(stg + st * PE_STAGE + half * (PE_STAGE / 2))),
+                        "l"(tm), "r"(cb * 256 + half * 128), "r"(r0 + 32 * i), "r"(fb)
+                        : "memory");
+                if (++st == PE_STAGES) {
+                    st = 0;
+                    par ^= 1u;
+                }
+            }
+        }
+        return;
+    }
     const bool wactive = wc0 < J.cols;
     const int G = (J.cols + 63) / 64;
 
@@ -314,7 +350,7 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
             ttab[n] = e;
         }
     }
-    __syncthreads();
+    pe_consumers_sync();
     uint64_t es = 0;  // sum of the weights this warp's columns see
     const int kend = (nr + 31) & ~31;  // whole chunks: positions past nr read zero limbs
     if (!SCALED) {
@@ -327,13 +363,13 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
         }
         es = warp_sum_gl(es);
         if (lane == 0) wsum[warp] = es;
-        __syncthreads();
+        pe_consumers_sync();
         es = 0;
 #pragma unroll
         for (int w = 0; w < PE_THREADS / 32; w++) es = gl_add(es, wsum[w]);
     } else {
         for (int k = threadIdx.x; k < kend; k += PE_THREADS) eqs[k] = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
-        __syncthreads();
+        pe_consumers_sync();
         const int g = wc0 / 64;
         for (int k = lane; k < kend; k += 32) {
             uint64_t e = 0;
@@ -350,27 +386,8 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
 #pragma unroll
     for (int g = 0; g < NG; g++) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0;
     {
-        // Thread 0 streams 32-row chunks of the block's 256-byte column slice into the stages, two
-        // TMA boxes (32 rows x 128 bytes, 128-byte swizzle) per chunk; every warp waits for a chunk,
-        // loads its 32-byte slice as two transposed 32 x 16-byte A fragments, and releases the
-        // stage. Rows past the block are read too: their eq limbs are zero.
-        const int nch = (nr + 31) >> 5;
-        const CUtensorMap* tm = &jobs[jidx].tmap;
-        auto produce = [&](int i, int st) {
-            const uint32_t fb = pe_saddr(&full[st]);
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(fb), "r"(PE_STAGE) : "memory");
-#pragma unroll
-            for (int half = 0; half < 2; half++)
-                asm volatile(
-                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-                    "[%4];\n" ::"r"(pe_saddr(stg + st * PE_STAGE + half * (PE_STAGE / 2))),
-                    "l"(tm), "r"(cb * 256 + half * 128), "r"(r0 + 32 * i), "r"(fb)
-                    : "memory");
-        };
-        if (threadIdx.x == 0) {
-            asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(tm) : "memory");
-            for (int i = 0; i < PE_STAGES && i < nch; i++) produce(i, i);
-        }
+        // every warp waits for a chunk, loads its 32-byte slice as two transposed 32 x 16-byte A
+        // fragments, and releases the stage
         const uint8_t* lp = &et[SCALED ? warp : 0][gid][0];
         // ldmatrix row addresses: lane L names row L of the chunk (lanes 0-15 the first 16 x 16-byte
         // matrix, lanes 16-31 the second); the warp's slice is 16-byte chunks c0 and c0 + 1 of its
@@ -393,11 +410,6 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
             ldsm_x2_trans(f[1], sp + o1);
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(pe_saddr(&empty[st])) : "memory");
-            if (threadIdx.x == 0 && i + PE_STAGES < nch) {
-                // every warp has its fragments of chunk i: refill the stage with chunk i + PE_STAGES
-                if (pe_wait(pe_saddr(&empty[st]), par)) produce(i + PE_STAGES, st);
-            }
-            __syncwarp();  // the MMAs below are warp-wide
             const int ch = 32 * i;
             if (++st == PE_STAGES) {
                 st = 0;
@@ -427,7 +439,7 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_tc_kernel(const PeJob* 
             }
         }
     }
-    __syncthreads();  // every warp is done with the stages, which now hold the sums
+    pe_consumers_sync();  // every consumer warp is done with the stages, which now hold the sums
     // D[m][n]: m = byte column of the 16-byte half h (m = gid in c0, c1; gid + 8 in c2, c3),
     // n = 2 tig + e = limb. int4: byte b holds columns 2 b (low nibble) and 2 b + 1.
     if (!wactive) return;
@@ -488,12 +500,12 @@ template <bool W4, bool SCALED>
 cudaError_t pe_tc_launch(const PeJob* dj, int n, int64_t blocks, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(partial_tc_kernel<W4, SCALED>, cudaFuncAttributeMaxDynamicSharedMemorySize, PE_DYN);
     if (e != cudaSuccess) return e;
-    partial_tc_kernel<W4, SCALED><<<(unsigned)blocks, PE_THREADS, PE_DYN, s>>>(dj, n);
+    partial_tc_kernel<W4, SCALED><<<(unsigned)blocks, PE_TC_THREADS, PE_DYN, s>>>(dj, n);
     return cudaGetLastError();
 }
 
-// About `waves` blocks per SM, at most max_rows rows per block (a multiple of 8, or of 32 on the
-// tensor-core path).
+// About `waves` blocks per SM, at most max_rows rows per block (a multiple of row_step): the
+// CUDA-core fallback for a job whose tensor map could not be made.
 void pe_plan_shape(int num_sms, int rows, int cols, int block_cols, int max_rows, int row_step, int waves,
                    int& col_blocks, int& rpb, int& splits) {
     col_blocks = (cols + block_cols - 1) / block_cols;
@@ -545,24 +557,69 @@ void pe_plan_cuda_core(int num_sms, const FpPeJob& q, int& col_blocks, int& rpb,
     pe_plan_shape(num_sms, q.rows, q.cols, PE_BLOCK_COLS, PE_MAX_ROWS, 8, 2, col_blocks, rpb, splits);
 }
 
-void pe_plan(int num_sms, const FpPeJob& q, bool& tc, int& col_blocks, int& rpb, int& splits) {
-    tc = pe_tc_ok(q);
-    // tensor-core blocks: three fit an SM; about two rounds of them keep the tail short
-    if (tc)
-        pe_plan_shape(num_sms, q.rows, q.cols, (PE_THREADS / 32) * (q.bits == 4 ? 64 : 32),
-                      q.scales ? tc_rows<true>() : tc_rows<false>(), 32, 6, col_blocks, rpb, splits);
-    else
-        pe_plan_shape(num_sms, q.rows, q.cols, PE_BLOCK_COLS, PE_MAX_ROWS, 8, 2, col_blocks, rpb, splits);
+struct PePlan {
+    bool tc;
+    int col_blocks, rpb, splits;
+};
+
+int pe_variant(bool tc, const FpPeJob& q) { return (tc ? 4 : 0) + (q.bits == 4 ? 2 : 0) + (q.scales ? 1 : 0); }
+
+// Every job of a call is planned together: the jobs of one kernel variant share one grid, so one
+// row count per block is chosen for all of them, the smallest (a multiple of the row step, at most
+// the exact-sum limit) that keeps the whole grid within about `waves` blocks per SM. A lone large
+// matrix gets about two rounds of three resident blocks per SM; a batch of many matrices (a MoE
+// layer) gets long blocks instead of many short ones, each of which would pay the block's set-up
+// and its first copy's latency over a few chunks.
+std::vector<PePlan> pe_plan_all(int num_sms, const FpPeJob* jobs, int njobs) {
+    std::vector<PePlan> P(njobs);
+    for (int j = 0; j < njobs; j++) {
+        const FpPeJob& q = jobs[j];
+        P[j].tc = pe_tc_ok(q);
+        const int bc = P[j].tc ? (PE_THREADS / 32) * (q.bits == 4 ? 64 : 32) : PE_BLOCK_COLS;
+        P[j].col_blocks = (q.cols + bc - 1) / bc;
+    }
+    for (int var = 0; var < 8; var++) {
+        const bool tc = var >= 4, scaled = var & 1;
+        const int64_t step = tc ? 32 : 8, cap = tc ? (scaled ? tc_rows<true>() : tc_rows<false>()) : PE_MAX_ROWS;
+        const int64_t target = (int64_t)(tc ? 6 : 2) * num_sms;
+        auto blocks = [&](int64_t R) {
+            int64_t n = 0;
+            for (int j = 0; j < njobs; j++)
+                if (pe_variant(P[j].tc, jobs[j]) == var) n += (int64_t)P[j].col_blocks * ((jobs[j].rows + R - 1) / R);
+            return n;
+        };
+        if (blocks(cap) == 0) continue;  // no job of this variant
+        int64_t lo = 1, hi = cap / step;  // the answer in row steps
+        if (blocks(cap) > target) {
+            lo = hi;
+        } else {
+            while (lo < hi) {
+                const int64_t mid = (lo + hi) / 2;
+                if (blocks(mid * step) <= target)
+                    hi = mid;
+                else
+                    lo = mid + 1;
+            }
+        }
+        const int R = (int)(lo * step);
+        for (int j = 0; j < njobs; j++)
+            if (pe_variant(P[j].tc, jobs[j]) == var) {
+                P[j].rpb = R;
+                P[j].splits = (jobs[j].rows + R - 1) / R;
+            }
+    }
+    return P;
 }
 
 }  // namespace
 
 size_t fp_partial_scratch(const fp_ctx* c, const FpPeJob* jobs, int njobs) {
     size_t need = 4 * fp_align_up(sizeof(PeJob) * (size_t)njobs, 256) + 4096;
+    const std::vector<PePlan> P = pe_plan_all(c->num_sms, jobs, njobs);
     for (int j = 0; j < njobs; j++) {
         int cbk, rpb, sp;
-        bool tc;
-        pe_plan(c->num_sms, jobs[j], tc, cbk, rpb, sp);
+        pe_plan_cuda_core(c->num_sms, jobs[j], cbk, rpb, sp);  // the fallback of a job without a tensor map
+        sp = std::max(sp, P[j].splits);
         need += fp_align_up((size_t)8 * sp * jobs[j].cols, 256) + fp_align_up(8 * (size_t)std::max(1, jobs[j].v), 256);
     }
     return need;
@@ -578,6 +635,7 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
     if (njobs <= 0) return FP_OK;
     std::vector<PeJob> h(njobs);
     std::vector<int> order[8];  // (tensor-core path, int4, scaled)
+    const std::vector<PePlan> P = pe_plan_all(c->num_sms, jobs, njobs);
     size_t zt = 0;
     for (int j = 0; j < njobs; j++) zt += (size_t)jobs[j].v;
     uint64_t* hz = (uint64_t*)fp_alloc(c->host, 8 * (zt + 1));
@@ -594,8 +652,10 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         d.rows = q.rows;
         d.cols = q.cols;
         d.v = q.v;
-        bool tc;
-        pe_plan(c->num_sms, q, tc, d.col_blocks, d.rows_per_block, d.splits);
+        bool tc = P[j].tc;
+        d.col_blocks = P[j].col_blocks;
+        d.rows_per_block = P[j].rpb;
+        d.splits = P[j].splits;
         memset(&d.tmap, 0, sizeof d.tmap);
         if (tc && !pe_make_tmap(q, &d.tmap)) {  // no tensor map: the CUDA-core kernel
             tc = false;
@@ -612,7 +672,7 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         if (q.v) memcpy(hz + zo, q.z, 8 * (size_t)q.v);
         d.z = dz + zo;
         zo += (size_t)q.v;
-        order[(tc ? 4 : 0) + (q.bits == 4 ? 2 : 0) + (q.scales ? 1 : 0)].push_back(j);
+        order[pe_variant(tc, q)].push_back(j);
     }
     FP_CUDA(c, cudaMemcpyAsync(dz, hz, 8 * (zt + 1), cudaMemcpyHostToDevice, s));
     for (int var = 0; var < 8; var++) {
