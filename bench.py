@@ -179,7 +179,9 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
       W 1 x 2^20 int4, one token); round 1 reads A and B, later rounds fold
       in place of the next evaluation (read 4, write 2 values per pair).
     partial_acc: eq-weighted row contraction of a 16384 x 16384 int4 matrix (the
-      weight side) and of a 16384 x 16384 int8 matrix (the activation side).
+      weight side) and of a 16384 x 16384 int8 matrix (the activation side); and
+      the batched weight-side launch of a MoE layer's proof (16 experts of
+      8192 x 5120 / 5120 x 8192 int4 plus the shared expert: 51 matrices, 1.07 GB).
     gkr_round: LogUp layer rounds over 2^26 keys (one 8192 x 64 x 8192 int8 site).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
@@ -230,6 +232,12 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
         measure("partial_eval_int8_16384^2", "partial_acc",
                 lambda: ctx.partial_eval(mat, 8, None, rows, cols, z, outv), big=1 << 26)
         del mat, outv
+        # the weight side of a MoE layer in one batched launch (the prover's own call)
+        wl = workloads.build(5, 0, E=16, T=1024)
+        st, keep = device.upload(wl, dev)
+        device.weight_digests(ctx, st)
+        measure("partial_eval_int4_moe_16x3_experts", "partial_acc", lambda: fp.prove(ctx, 0, st), big=1 << 28)
+        del st, keep, wl
 
     if "gemm" in which:
         # witness GEMM of an FFN-sized site on the tensor cores (2 x MACs integer ops)

@@ -259,25 +259,26 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_many_kernel(const PeJob
 }
 
 // Tensor-core partial evaluation. A warp owns 32 bytes of every row (64 int4 or
-// 32 int8 columns); 8 warps side by side, up to tc_rows<SCALED>() rows per block.
+// 32 int8 columns); 8 warps side by side, up to PE_TC_ROWS rows per block.
 //
 // eq(z, i) of the block's rows comes from two small tables: with i = 32 m + n,
 // eq(z, i) = H[m - m0] T[n], H over the high coordinates of the block's row
-// groups and T over the last five coordinates; one product per row.
-template <bool SCALED>
-__host__ __device__ constexpr int tc_rows() {
-    return SCALED ? 256 : 2048;  // exact s32 sums: 2048 x 255 x 255 < 2^31
-}
+// groups and T over the last five coordinates; one product per row. Without
+// scales every warp reads one limb table of the block's rows; with scales the
+// weight of row i is e_i s[i][g] for the warp's column group g, so each warp
+// forms its chunk's 32 scaled weights as it goes (the scales one chunk ahead).
+constexpr int PE_TC_ROWS = 2048;  // exact s32 sums: 2048 x 255 x 255 < 2^31
 
 template <bool W4, bool SCALED>
 __global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJob* __restrict__ jobs, int njobs) {
     constexpr int WCOLS = W4 ? 64 : 32;
     constexpr int NG = W4 ? 4 : 2;  // MMAs per 32-row chunk: 16 columns each
-    constexpr int ROWS = tc_rows<SCALED>();
-    // limb l of row k's weight: one table for all warps, or one per warp (scaled: the weight
-    // depends on the warp's column group)
-    __shared__ __align__(16) uint8_t et[SCALED ? 8 : 1][8][ROWS];
+    constexpr int ROWS = PE_TC_ROWS;
+    // unscaled: limb l of row k's weight eq(z, i); scaled: eq(z, i) of the block's rows, and per
+    // warp the limbs of the current chunk's scaled weights
+    __shared__ __align__(16) uint8_t et[8][SCALED ? 16 : ROWS];
     __shared__ uint64_t eqs[SCALED ? ROWS : 1];
+    __shared__ __align__(16) uint8_t lt[SCALED ? PE_THREADS / 32 : 1][8][32];
     __shared__ uint64_t htab[ROWS / 32], ttab[32];
     __shared__ uint64_t wsum[8];
     __shared__ __align__(8) uint64_t full[PE_STAGES], empty[PE_STAGES];
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJo
             // with v < 5 the rows are i = n < 2^v and H = {1}
             const uint64_t e = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
 #pragma unroll
-            for (int l = 0; l < 8; l++) et[0][l][k] = (uint8_t)(e >> (8 * l));
+            for (int l = 0; l < 8; l++) et[l][k] = (uint8_t)(e >> (8 * l));
             es = gl_add(es, e);
         }
         es = warp_sum_gl(es);
@@ -370,17 +371,11 @@ __global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJo
     } else {
         for (int k = threadIdx.x; k < kend; k += PE_THREADS) eqs[k] = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
         pe_consumers_sync();
-        const int g = wc0 / 64;
-        for (int k = lane; k < kend; k += 32) {
-            uint64_t e = 0;
-            if (wactive && k < nr) e = gl_mul_small(eqs[k], (int32_t)__ldg(J.scales + (int64_t)(r0 + k) * G + g));
-#pragma unroll
-            for (int l = 0; l < 8; l++) et[warp][l][k] = (uint8_t)(e >> (8 * l));
-            es = gl_add(es, e);
-        }
-        es = warp_sum_gl(es);
-        __syncwarp();
     }
+    // scaled: the scale of row 32 i + lane in the warp's column group, loaded a chunk ahead
+    const int8_t* srow = SCALED ? J.scales + (int64_t)r0 * G + wc0 / 64 : nullptr;
+    int32_t sv = 0;
+    if (SCALED && wactive && lane < nr) sv = (int32_t)__ldg(srow + (int64_t)lane * G);
 
     uint32_t acc[NG][4];
 #pragma unroll
@@ -388,7 +383,7 @@ __global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJo
     {
         // every warp waits for a chunk, loads its 32-byte slice as two transposed 32 x 16-byte A
         // fragments, and releases the stage
-        const uint8_t* lp = &et[SCALED ? warp : 0][gid][0];
+        const uint8_t* lp = &et[gid][0];
         // ldmatrix row addresses: lane L names row L of the chunk (lanes 0-15 the first 16 x 16-byte
         // matrix, lanes 16-31 the second); the warp's slice is 16-byte chunks c0 and c0 + 1 of its
         // 128-byte half, and 128-byte swizzle puts chunk c of row r at c ^ (r % 8)
@@ -418,8 +413,23 @@ __global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJo
             // a stalled copy leaves this block's sums wrong, not hung (the same decision in every lane)
             if (!__all_sync(0xffffffffu, got) || !wactive) continue;
             // B: limb gid of rows tig*4 .. +3 and 16 + tig*4 .. +3
-            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(lp + ch + tig * 4);
-            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(lp + ch + 16 + tig * 4);
+            uint32_t b0, b1;
+            if (SCALED) {
+                // lane r forms row r's weight e s (zero past the block: eqs is zero there) and
+                // spreads its limbs; the warp's previous reads of lt ended before the wait above
+                const int k = ch + lane;
+                const uint64_t w = gl_mul_small(eqs[k], sv);
+                sv = k + 32 < nr ? (int32_t)__ldg(srow + (int64_t)(k + 32) * G) : 0;
+                es = gl_add(es, w);
+#pragma unroll
+                for (int l = 0; l < 8; l++) lt[warp][l][lane] = (uint8_t)(w >> (8 * l));
+                __syncwarp();
+                b0 = *reinterpret_cast<const uint32_t*>(&lt[warp][gid][tig * 4]);
+                b1 = *reinterpret_cast<const uint32_t*>(&lt[warp][gid][16 + tig * 4]);
+            } else {
+                b0 = *reinterpret_cast<const uint32_t*>(lp + ch + tig * 4);
+                b1 = *reinterpret_cast<const uint32_t*>(lp + ch + 16 + tig * 4);
+            }
 #pragma unroll
             for (int h = 0; h < 2; h++) {
                 if (W4) {
@@ -443,6 +453,7 @@ __global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJo
     // D[m][n]: m = byte column of the 16-byte half h (m = gid in c0, c1; gid + 8 in c2, c3),
     // n = 2 tig + e = limb. int4: byte b holds columns 2 b (low nibble) and 2 b + 1.
     if (!wactive) return;
+    if (SCALED) es = warp_sum_gl(es);  // this warp's sum of e s
 #pragma unroll
     for (int h = 0; h < 2; h++) {
 #pragma unroll
@@ -579,8 +590,8 @@ std::vector<PePlan> pe_plan_all(int num_sms, const FpPeJob* jobs, int njobs) {
         P[j].col_blocks = (q.cols + bc - 1) / bc;
     }
     for (int var = 0; var < 8; var++) {
-        const bool tc = var >= 4, scaled = var & 1;
-        const int64_t step = tc ? 32 : 8, cap = tc ? (scaled ? tc_rows<true>() : tc_rows<false>()) : PE_MAX_ROWS;
+        const bool tc = var >= 4;
+        const int64_t step = tc ? 32 : 8, cap = tc ? PE_TC_ROWS : PE_MAX_ROWS;
         const int64_t target = (int64_t)(tc ? 6 : 2) * num_sms;
         auto blocks = [&](int64_t R) {
             int64_t n = 0;
