@@ -298,7 +298,7 @@ int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites
         P.fin = dfin;
         P.nsites = nsites;
         P.n = n;
-        P.per_block = SC_THREADS * 4;
+        P.per_block = SC_THREADS;  // one pair per thread: small rounds spread over more blocks
         const int64_t want = ((int64_t)nsites * (L / 2) + P.per_block - 1) / P.per_block;
         P.grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)std::max(1, occ) * c->num_sms));
         P.seq0 = fp_seq_reserve(c, n + 2);
