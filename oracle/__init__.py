@@ -43,6 +43,10 @@ REASONS = {
     12: "leaf_Q",
     13: "leaf_open",
     14: "args",
+    15: "had_claim",
+    16: "had_round",
+    17: "had_final",
+    18: "had_open",
 }
 
 
@@ -106,6 +110,10 @@ def lib():
         L.orc_verify.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp]
         L.orc_verify_opts.restype = C.c_int
         L.orc_verify_opts.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp, vp, C.c_int]
+        L.orc_had_prove.restype = C.c_int
+        L.orc_had_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
+        L.orc_had_verify.restype = C.c_int
+        L.orc_had_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
         _lib = L
     return _lib
 
@@ -342,4 +350,48 @@ def verify(seed: int, sites, wits, proof: bytes, site_mask=None, skip_leaf_open:
         mask = None if site_mask is None else np.ascontiguousarray(np.asarray(site_mask, dtype=np.uint8))
         rc = lib().orc_verify_opts(seed, cs, len(sites), cw, _ptr(pb), len(proof), _ptr(det), _ptr(mask),
                                    4 if skip_leaf_open else 0)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+# ---- gated product h = s (.) u ------------------------------------------------
+
+def _i8(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int8).reshape(-1))
+
+
+def had_prove(seed: int, s, u):
+    """Sum-check proof that the gated product h = s (.) u has the claimed MLE at the
+    transcript's point (see oracle.c). Returns (proof bytes, transcript state after)."""
+    L = lib()
+    a, b = _i8(s), _i8(u)
+    if a.size != b.size or a.size < 1:
+        raise ValueError("had_prove: s and u need the same length >= 1")
+    out = []
+    for cap in (0, None):
+        tx = L.orc_tx_new(seed)
+        n = C.c_uint64(0)
+        buf = np.zeros(max(1, out[0] if out else 1), dtype=np.uint8)
+        rc = L.orc_had_prove(tx, _ptr(a), _ptr(b), a.size, _ptr(buf) if out else None, out[0] if out else 0,
+                             C.byref(n))
+        st = C.create_string_buffer(32)
+        L.orc_tx_state(tx, st)
+        L.orc_tx_free(tx)
+        if out:
+            if rc != 0:
+                raise ValueError(f"orc_had_prove failed ({rc})")
+            return buf[: n.value].tobytes(), st.raw
+        if rc not in (0, -2):
+            raise ValueError(f"orc_had_prove rejected the statement ({rc})")
+        out.append(n.value)
+
+
+def had_verify(seed: int, s, u, proof: bytes):
+    """Returns (reason_name, detail); 'accept' for a valid proof."""
+    L = lib()
+    a, b = _i8(s), _i8(u)
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_had_verify(tx, _ptr(a), _ptr(b), a.size, _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

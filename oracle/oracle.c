@@ -1188,3 +1188,148 @@ int orc_verify_opts(u64 seed, const orc_site* sites, int ns, const orc_wit* wit,
     if (rd.pos != rd.len) return REJ_FORMAT;
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Gated product h = s (.) u. The pages ("How fast can FlashProve go", 3.1   */
+/* Committing intermediate values, the note on the MLP's hidden values) say  */
+/* the gated product is a plain product that the sum-check handles without   */
+/* committing to it: a claim on h~(z) is reduced to claims on s~(rho) and    */
+/* u~(rho), the two committed factors. The textbook product sum-check over   */
+/* three multilinear vectors, eq(z, .), s and u, degree 3 per round:         */
+/*   absorb "had_site" D(s) || D(u) (the tree digests of the two int8        */
+/*     vectors); squeeze z_1..z_v ("had_z"), v = ceil(log2 n);               */
+/*   send c = sum_x eq(z, x) s(x) u(x) ("had_claim");                         */
+/*   round t = 1..v: send g_t(0), g_t(1), g_t(2), g_t(3) ("had_round"), with  */
+/*     g_t(X) = sum_b E(X, b) S(X, b) U(X, b) over the vectors folded by the  */
+/*     earlier challenges; squeeze rho_t ("had_chal"); fold E, S and U;       */
+/*   send S(rho), U(rho) ("had_final").                                        */
+/* The vectors are zero-padded to 2^v; n = 1 gives v = 0 and no rounds.      */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_HAD_CLAIM = 15,  /* c != h~(z) recomputed from s and u */
+    REJ_HAD_ROUND = 16,  /* g_t(0) + g_t(1) != running claim */
+    REJ_HAD_FINAL = 17,  /* eq(z, rho) S U != claim after the last round */
+    REJ_HAD_OPEN = 18    /* S or U != the committed vector's MLE at rho */
+};
+
+static void had_absorb_site(orc_tx* t, const int8_t* s, const int8_t* u, u64 n) {
+    uint8_t d[64];
+    orc_tree_digest(s, n, d);
+    orc_tree_digest(u, n, d + 32);
+    orc_tx_absorb(t, "had_site", d, 64);
+}
+
+/* the int8 vector as field elements, zero-padded to 2^v */
+static u64* had_lift(const int8_t* a, u64 n, int v) {
+    u64 sz = (u64)1 << v;
+    u64* out = (u64*)calloc(sz, sizeof(u64));
+    for (u64 i = 0; i < n; i++) out[i] = orc_fint(a[i]);
+    return out;
+}
+
+/* Proof into proof[0..cap); *len = bytes needed. Returns 0, -1 on bad input,
+ * -2 if cap is too small. tx is an orc_tx_new handle, advanced in place. */
+int orc_had_prove(void* txh, const int8_t* s, const int8_t* u, u64 n, uint8_t* proof, u64 cap, u64* len) {
+    if (n < 1) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n);
+    u64 sz = (u64)1 << v;
+    pbuf pb = {proof, cap, 0, 0};
+    had_absorb_site(t, s, u, n);
+    u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
+    for (int i = 0; i < v; i++) z[i] = orc_tx_squeeze(t, "had_z");
+    u64* E = (u64*)malloc(sz * sizeof(u64));
+    orc_eq_table(z, v, E);
+    u64* S = had_lift(s, n, v);
+    u64* U = had_lift(u, n, v);
+    u64 c = 0;
+    for (u64 x = 0; x < sz; x++) c = orc_fadd(c, orc_fmul(E[x], orc_fmul(S[x], U[x])));
+    send_fe(t, &pb, "had_claim", &c, 1);
+    u64 L = sz;
+    for (int r = 0; r < v; r++) {
+        u64 h = L >> 1;
+        u64 g[4] = {0, 0, 0, 0};
+        for (u64 b = 0; b < h; b++)
+            for (u64 X = 0; X < 4; X++) {
+                /* each vector's line through (b, b + h) at X */
+                u64 e = orc_fadd(E[b], orc_fmul(X, orc_fsub(E[h + b], E[b])));
+                u64 sx = orc_fadd(S[b], orc_fmul(X, orc_fsub(S[h + b], S[b])));
+                u64 ux = orc_fadd(U[b], orc_fmul(X, orc_fsub(U[h + b], U[b])));
+                g[X] = orc_fadd(g[X], orc_fmul(e, orc_fmul(sx, ux)));
+            }
+        send_fe(t, &pb, "had_round", g, 4);
+        u64 rho = orc_tx_squeeze(t, "had_chal");
+        for (u64 b = 0; b < h; b++) {
+            E[b] = orc_fadd(E[b], orc_fmul(rho, orc_fsub(E[h + b], E[b])));
+            S[b] = orc_fadd(S[b], orc_fmul(rho, orc_fsub(S[h + b], S[b])));
+            U[b] = orc_fadd(U[b], orc_fmul(rho, orc_fsub(U[h + b], U[b])));
+        }
+        L = h;
+    }
+    u64 fin[2] = {S[0], U[0]};
+    send_fe(t, &pb, "had_final", fin, 2);
+    free(z);
+    free(E);
+    free(S);
+    free(U);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+/* Verifier: every round's consistency, the end against eq(z, rho) S U in
+ * closed form, and (standing in for openings of the committed s and u) the
+ * claim c and the final S, U recomputed from the vectors it holds. Returns 0
+ * (accept) or a rejection code; detail[0] = the round of a failed round check. */
+int orc_had_verify(void* txh, const int8_t* s, const int8_t* u, u64 n, const uint8_t* proof, u64 len,
+                   int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (n < 1) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n), rc = 0;
+    u64 sz = (u64)1 << v;
+    prd rd = {proof, len, 0, 0};
+    had_absorb_site(t, s, u, n);
+    u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
+    u64* rho = (u64*)malloc(sizeof(u64) * (v + 1));
+    u64* S = had_lift(s, n, v);
+    u64* U = had_lift(u, n, v);
+    for (int i = 0; i < v; i++) z[i] = orc_tx_squeeze(t, "had_z");
+    u64 c, claim;
+    rd_fe(t, &rd, "had_claim", &c, 1);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    {
+        u64* P = (u64*)malloc(sz * sizeof(u64));
+        for (u64 x = 0; x < sz; x++) P[x] = orc_fmul(S[x], U[x]);
+        u64 want = orc_mle_eval(P, sz, z, v);
+        free(P);
+        if (want != c) FAIL(REJ_HAD_CLAIM, 0, 0);
+    }
+    claim = c;
+    for (int r = 0; r < v; r++) {
+        u64 g[4];
+        rd_fe(t, &rd, "had_round", g, 4);
+        if (rd.bad) FAIL(REJ_FORMAT, r, 0);
+        if (orc_fadd(g[0], g[1]) != claim) FAIL(REJ_HAD_ROUND, r, 0);
+        rho[r] = orc_tx_squeeze(t, "had_chal");
+        claim = orc_lagrange(g, 4, rho[r]);
+    }
+    u64 fin[2];
+    rd_fe(t, &rd, "had_final", fin, 2);
+    if (rd.bad) FAIL(REJ_FORMAT, v, 0);
+    {
+        u64 e = 1;
+        for (int i = 0; i < v; i++)
+            e = orc_fmul(e, orc_fadd(orc_fmul(z[i], rho[i]), orc_fmul(orc_fsub(1, z[i]), orc_fsub(1, rho[i]))));
+        if (orc_fmul(e, orc_fmul(fin[0], fin[1])) != claim) FAIL(REJ_HAD_FINAL, 0, 0);
+    }
+    if (orc_mle_eval(S, sz, rho, v) != fin[0]) FAIL(REJ_HAD_OPEN, 0, 0);
+    if (orc_mle_eval(U, sz, rho, v) != fin[1]) FAIL(REJ_HAD_OPEN, 1, 0);
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(z);
+    free(rho);
+    free(S);
+    free(U);
+    return rc;
+}

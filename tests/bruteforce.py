@@ -324,3 +324,57 @@ def walk(seed: int, sites, wits, proof: bytes) -> dict:
     out["consumed"] = rd.pos
     out["state"] = tx.st
     return out
+
+
+# ---- gated product h = s (.) u ---------------------------------------------------
+
+def eq_ml(z, w) -> int:
+    """eq(z, w) for field points z, w of equal length: prod (z_i w_i + (1 - z_i)(1 - w_i))."""
+    acc = 1
+    for a, b in zip(z, w):
+        acc = acc * ((a * b + (1 - a) * (1 - b)) % P) % P
+    return acc
+
+
+def mle_at(vals, w) -> int:
+    """MLE of vals (zero-padded to 2^len(w)) at a field point w, by the hypercube sum."""
+    v = len(w)
+    acc = 0
+    for x in range(min(len(vals), 1 << v)):
+        bits = [(x >> (v - 1 - b)) & 1 for b in range(v)]
+        acc += eq_ml(w, bits) * (int(vals[x]) % P)
+    return acc % P
+
+
+def had_prove(seed: int, s, u) -> bytes:
+    """The gated-product proof from definitions: every round value is the sum, over the
+    unbound Boolean variables b, of eq(z, (rho, X, b)) s~(rho, X, b) u~(rho, X, b), each
+    MLE evaluated by its own hypercube sum; no vector is folded."""
+    s = [int(x) for x in np.asarray(s).reshape(-1)]
+    u = [int(x) for x in np.asarray(u).reshape(-1)]
+    n = len(s)
+    v = log2c(n)
+    tx = Tx(seed)
+    tx.absorb("had_site", tree_digest(bytes(np.asarray(s, np.int8).tobytes())) +
+              tree_digest(bytes(np.asarray(u, np.int8).tobytes())))
+    z = [tx.squeeze("had_z") for _ in range(v)]
+    c = sum(eq_point(z, x) * s[x] * u[x] for x in range(n)) % P
+    out = fe_bytes([c])
+    tx.absorb("had_claim", fe_bytes([c]))
+    rho = []
+    for t in range(v):
+        rest = v - t - 1
+        g = []
+        for X in range(4):
+            acc = 0
+            for b in range(1 << rest):
+                w = rho + [X] + [(b >> (rest - 1 - i)) & 1 for i in range(rest)]
+                acc += eq_ml(z, w) * mle_at(s, w) * mle_at(u, w)
+            g.append(acc % P)
+        out += fe_bytes(g)
+        tx.absorb("had_round", fe_bytes(g))
+        rho.append(tx.squeeze("had_chal"))
+    fin = [mle_at(s, rho), mle_at(u, rho)]
+    out += fe_bytes(fin)
+    tx.absorb("had_final", fe_bytes(fin))
+    return out
