@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
+def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had") -> dict:
     """Kernel rooflines at HBM scale (inputs well above the 126 MB L2), from a
     profiled pass: every round is its own launch, timed with CUDA events.
 
@@ -183,6 +183,10 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
       the batched weight-side launch of a MoE layer's proof (16 experts of
       8192 x 5120 / 5120 x 8192 int4 plus the shared expert: 51 matrices, 1.07 GB).
     gkr_round: LogUp layer rounds over 2^26 keys (one 8192 x 64 x 8192 int8 site).
+    had_round: gated-product sum-check rounds over two 2^26-entry int8 factors
+      (round 1 reads the int8 factors and writes the eq table, round 2 folds
+      them into field vectors, later rounds read 4 and write 2 values of both
+      factors and fold the eq table: 120 B per pair).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
@@ -260,6 +264,15 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm") -> dict:
                                                     "TOPS": tops, "frac": tops / peak, "peak": peak,
                                                     "peak_note": "int8 = measured bf16 x 2 (nominal ratio)"}
         del st, keep
+
+    if "had" in which:
+        # the gated product of an FFN's hidden tensor, 2^26 entries per factor
+        rng = __import__("numpy").random.default_rng(9)
+        n = 1 << 26
+        sv = torch.from_numpy(rng.integers(-128, 128, n).astype("int8")).to(dev)
+        uv = torch.from_numpy(rng.integers(-128, 128, n).astype("int8")).to(dev)
+        measure("hadamard_round_2^26", "had_round", lambda: ctx.prove_hadamard(fp.Transcript(4), sv, uv))
+        del sv, uv
 
     if "gkr" in which:
         s = workloads.random_site(77, 8192, 64, 8192, 8, 12)
@@ -525,7 +538,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-micro", action="store_true")
-    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm", default=None,
+    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm,had", default=None,
                     help="run only the kernel measurements at scale (comma list of sc, pe, gkr, gemm)")
     args = ap.parse_args()
     if args.micro_only:

@@ -210,6 +210,28 @@ int logup_prove_rescale(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites
                         size_t* proof_len, void* stream);
 
 /*
+ * Sum-check of a gated product h = s (.) u that is never committed ("How fast
+ * can FlashProve go", 3.1 Committing intermediate values: the MLP's gated
+ * product is a plain product, so sum-check handles it without committing to
+ * it). s, u: device int8 vectors of n entries each (for an MLP, the SiLU output
+ * and the up projection, [tokens, hidden] row-major), caller-owned, read only.
+ * Both are zero-padded to 2^v, v = ceil(log2 n). The call continues tx:
+ *   absorb "had_site" D(s) || D(u) (tree digests as fp_digest);
+ *   squeeze z_1..z_v ("had_z"); send c = sum_x eq(z, x) s(x) u(x) ("had_claim");
+ *   round t = 1..v: send g_t(0), g_t(1), g_t(2), g_t(3) ("had_round") with
+ *     g_t(X) = sum over the unbound Boolean b of eq(z, (rho_<t, X, b))
+ *     s~(rho_<t, X, b) u~(rho_<t, X, b); squeeze rho_t ("had_chal");
+ *   send s~(rho), u~(rho) ("had_final").
+ * Proof bytes (u64 LE field elements): c | v x 4 round values | 2 final values,
+ * 8 + 32 v + 16 bytes. The verifier checks g_t(0) + g_t(1) against the running
+ * claim, g_v(rho_v) = eq(z, rho) s~(rho) u~(rho), and the two final values
+ * against openings of s and u. 1 <= n <= 2^30, else FP_ERR_SHAPE; null
+ * arguments FP_ERR_ARG; proof / proof_len as for sumcheck_prove_matmul.
+ */
+int sumcheck_prove_hadamard(fp_ctx* ctx, fp_tx* tx, const int8_t* s, const int8_t* u, int64_t n, uint8_t* proof,
+                            size_t* proof_len, void* stream);
+
+/*
  * Self-test of the bounded device waits. The sum-check kernels stay resident
  * across rounds and wait (a bounded number of polls) for each Fiat-Shamir
  * challenge from the host. This call launches a kernel that waits for a

@@ -73,6 +73,7 @@ def lib():
     L.mle_partial_eval.argtypes = [vp, vp, i32, vp, i32, i32, C.POINTER(u64), i32, vp, vp]
     L.sumcheck_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
     L.logup_prove_rescale.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
+    L.sumcheck_prove_hadamard.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_proof_size.argtypes = [C.POINTER(_Site), i32, C.POINTER(sz), C.POINTER(sz)]
     L.fp_ctx_set_profiling.argtypes = [vp, i32]
     L.fp_session_selftest.argtypes = [vp, vp]
@@ -230,6 +231,22 @@ class Context:
         self._check(self._L.sumcheck_prove_matmul(self.h, tx.h, arr, len(sites), buf, C.byref(n), _stream(stream)),
                     "sumcheck_prove_matmul")
         return buf.raw[: n.value]
+
+    def prove_hadamard(self, tx: Transcript, s, u, stream=None) -> bytes:
+        """Sum-check proof for the gated product of two device int8 tensors of equal size
+        (flattened row-major); continues tx."""
+        n = int(s.numel())
+        if int(u.numel()) != n:
+            raise ValueError("prove_hadamard: s and u differ in size")
+        v = 0
+        while (1 << v) < n:
+            v += 1
+        cap = 8 + 32 * v + 16
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        self._check(self._L.sumcheck_prove_hadamard(self.h, tx.h, _ptr(s), _ptr(u), n, buf, C.byref(ln),
+                                                    _stream(stream)), "sumcheck_prove_hadamard")
+        return buf.raw[: ln.value]
 
     def prove_logup(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
         """Returns (proof bytes, status): status 1 means some key lies outside its table."""

@@ -32,6 +32,9 @@ enum FpKernel {
     K_GKR_FINAL,
     K_LEAF_EVAL,
     K_REDUCE,
+    K_HAD_CLAIM,
+    K_HAD_ROUND,
+    K_HAD_FINAL,
     K_COUNT
 };
 
@@ -175,3 +178,6 @@ int fp_claims(fp_ctx* c, const fp_site* sites, int nsites, const uint64_t* const
               const uint64_t* const* eq_cols, uint64_t* dev_out, cudaStream_t s);
 
 static inline size_t fp_align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// little-endian u64 words into a proof buffer (sumcheck.cu)
+void put_u64s(uint8_t* p, const uint64_t* v, size_t n);

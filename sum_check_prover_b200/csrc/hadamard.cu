@@ -1,0 +1,340 @@
+// Sum-check of the gated product h = s (.) u.
+//
+// "How fast can FlashProve go", 3.1 Committing intermediate values: the MLP's
+// gated product is a plain product, so the prover never commits to it; a
+// sum-check reduces a claim on h~(z) to claims on the committed factors s and
+// u. The statement here is two int8 vectors of n entries (s, u; zero-padded to
+// 2^v):
+//   absorb "had_site" D(s) || D(u); squeeze z_1..z_v ("had_z");
+//   send c = sum_x eq(z, x) s(x) u(x) ("had_claim");
+//   round t = 1..v: send g_t(0..3) ("had_round"); squeeze rho_t ("had_chal");
+//   send S(rho), U(rho) ("had_final").
+// g_t(X) = eq(z_<t, rho_<t) eq(z_t, X) h_t(X) with h_t(X) =
+// sum_b eq(z_>t, b) S(X, b) U(X, b) over the factors folded by rho_<t; h_t has
+// degree 2, so the device returns h_t(0), h_t(1), h_t(2) and the host forms the
+// four values of g_t (h_t(3) = h_t(0) - 3 h_t(1) + 3 h_t(2)). g_t(0) + g_t(1)
+// must equal the running claim; the host checks it on every round.
+//
+// All rounds run in one resident cooperative launch (the handshake of
+// fp_session.cuh). Round 1 reads the int8 factors and writes the suffix eq
+// table E[b] = eq(z_>1, b); round 2 folds the int8 factors by rho_1 into field
+// vectors; later rounds fold those in place (each thread owns positions b,
+// b + h, b + 2h, b + 3h) and sum E in place. One pair per thread per pass.
+#include <string.h>
+
+#include <algorithm>
+
+#include "fp_eqchunks.cuh"
+#include "fp_internal.h"
+#include "fp_reduce.cuh"
+#include "fp_session.cuh"
+
+namespace {
+
+constexpr int HAD_THREADS = 256;
+constexpr int HAD_MAX_V = 30;
+
+struct HadArgs {
+    const int8_t* s;
+    const int8_t* u;
+    int64_t n;
+    uint64_t* S;  // folded factors from round 2 on (2^(v-1) entries each)
+    uint64_t* U;
+    uint64_t* E;  // suffix eq table (2^(v-1) entries)
+    const uint64_t* z;  // device copy of z_1..z_v
+    int v;
+    int grid;
+    int per_block;
+    int pad;
+    uint64_t seq0;  // round t publishes seq0 + t, the final values seq0 + v + 1
+    int t_begin;    // rounds run by this launch: [t_begin, t_end]; t_end > v includes the final values
+    int t_end;
+};
+
+__device__ __forceinline__ uint64_t lift8(int8_t x) { return x < 0 ? GL_P - (uint64_t)(-(int)x) : (uint64_t)x; }
+
+__device__ __forceinline__ uint64_t ld8(const int8_t* a, int64_t i, int64_t n) { return i < n ? lift8(a[i]) : 0ull; }
+
+// X = 2 on the line through (a, b) at 0 and 1
+__device__ __forceinline__ uint64_t at2(uint64_t a, uint64_t b) { return gl_sub(gl_add(b, b), a); }
+
+// c = sum_x eq(z, x) s(x) u(x), eq split as EH[x >> vl] EL[x & (2^vl - 1)]; one partial per block
+__global__ void __launch_bounds__(256) had_claim_kernel(const int8_t* __restrict__ s, const int8_t* __restrict__ u,
+                                                        int64_t n, const uint64_t* __restrict__ EH,
+                                                        const uint64_t* __restrict__ EL, int vl, uint64_t* part,
+                                                        unsigned int* ticket, uint64_t* out) {
+    GlAcc acc;
+    const int64_t mask = (1ll << vl) - 1;
+    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
+        const int p = (int)s[x] * (int)u[x];
+        if (p == 0) continue;
+        const uint64_t e = gl_mul(__ldg(EH + (x >> vl)), __ldg(EL + (x & mask)));
+        acc.mac(e, p < 0 ? GL_P - (uint64_t)(-p) : (uint64_t)p);
+    }
+    uint64_t v[1] = {acc.value()};
+    if (grid_sum_gl<1>(v, part, ticket) && threadIdx.x == 0) *out = v[0];
+}
+
+__global__ void __launch_bounds__(HAD_THREADS, 2) had_session_kernel(HadArgs A, FpMailbox* mb, FpRelay* rl,
+                                                                    uint64_t* part) {
+    __shared__ uint64_t zs[32];
+    __shared__ uint64_t eq_tab[3 << kEqChunk];
+    if (threadIdx.x < A.v) zs[threadIdx.x] = A.z[threadIdx.x];
+    __syncthreads();
+    uint64_t rprev = 0;
+    for (int t = A.t_begin; t <= A.v && t <= A.t_end; t++) {
+        if (t > 1 && !session_wait(mb, rl, A.seq0 + t - 1, rprev)) return;
+        const int64_t h = 1ll << (A.v - t);
+        const int64_t want = (h + A.per_block - 1) / A.per_block;
+        const unsigned active = (unsigned)(want < 1 ? 1 : (want > A.grid ? A.grid : want));
+        if (blockIdx.x >= active) return;  // no pairs for this block in this or any later round
+        EqChunks EC{0, 0, 0};
+        if (t == 1) EC = eq_chunks_build(eq_tab, zs, A.v);
+        GlAcc a0, a1, a2;
+        for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
+            uint64_t s0, s1, u0, u1, e;
+            if (t == 1) {
+                s0 = ld8(A.s, b, A.n);
+                s1 = ld8(A.s, b + h, A.n);
+                u0 = ld8(A.u, b, A.n);
+                u1 = ld8(A.u, b + h, A.n);
+                e = eq_chunks_at(EC, eq_tab, b);  // eq(z_2..z_v, b)
+                if (A.v > 1) A.E[b] = e;
+            } else {
+                if (t == 2) {
+                    // the int8 factors (length 4h) folded by rho_1
+                    s0 = gl_fold_fast(ld8(A.s, b, A.n), ld8(A.s, b + 2 * h, A.n), rprev);
+                    s1 = gl_fold_fast(ld8(A.s, b + h, A.n), ld8(A.s, b + 3 * h, A.n), rprev);
+                    u0 = gl_fold_fast(ld8(A.u, b, A.n), ld8(A.u, b + 2 * h, A.n), rprev);
+                    u1 = gl_fold_fast(ld8(A.u, b + h, A.n), ld8(A.u, b + 3 * h, A.n), rprev);
+                } else {
+                    s0 = gl_fold_fast(__ldcg(A.S + b), __ldcg(A.S + b + 2 * h), rprev);
+                    s1 = gl_fold_fast(__ldcg(A.S + b + h), __ldcg(A.S + b + 3 * h), rprev);
+                    u0 = gl_fold_fast(__ldcg(A.U + b), __ldcg(A.U + b + 2 * h), rprev);
+                    u1 = gl_fold_fast(__ldcg(A.U + b + h), __ldcg(A.U + b + 3 * h), rprev);
+                }
+                A.S[b] = s0;
+                A.S[b + h] = s1;
+                A.U[b] = u0;
+                A.U[b + h] = u1;
+                e = gl_add(__ldcg(A.E + b), __ldcg(A.E + b + h));  // eq(z_>t, b)
+                A.E[b] = e;
+            }
+            a0.mac(e, gl_mul_weak(s0, u0));
+            a1.mac(e, gl_mul_weak(s1, u1));
+            a2.mac(e, gl_mul_weak(at2(s0, s1), at2(u0, u1)));
+        }
+        uint64_t acc[3] = {a0.value(), a1.value(), a2.value()};
+        bool last;
+        if (active == 1) {
+            block_sum_gl<3>(acc);
+            last = true;
+        } else {
+            last = grid_sum_gl_n<3>(acc, part, &rl->ticket, active);
+        }
+        if (last && threadIdx.x == 0) session_publish(mb, acc, A.seq0 + t);  // {h(0), h(1), h(2)}
+    }
+    // block 0 folds the last pair by the last challenge: S(rho), U(rho)
+    if (A.t_end <= A.v || blockIdx.x != 0) return;
+    if (!session_wait(mb, rl, A.seq0 + A.v, rprev)) return;
+    if (threadIdx.x == 0) {
+        uint64_t s0, s1, u0, u1;
+        if (A.v == 1) {
+            s0 = ld8(A.s, 0, A.n);
+            s1 = ld8(A.s, 1, A.n);
+            u0 = ld8(A.u, 0, A.n);
+            u1 = ld8(A.u, 1, A.n);
+        } else {
+            s0 = __ldcg(A.S);
+            s1 = __ldcg(A.S + 1);
+            u0 = __ldcg(A.U);
+            u1 = __ldcg(A.U + 1);
+        }
+        const uint64_t fin[2] = {gl_fold_fast(s0, s1, rprev), gl_fold_fast(u0, u1, rprev)};
+        session_publish(mb, fin, A.seq0 + A.v + 1);
+    }
+}
+
+uint64_t lift_host(int8_t x) { return x < 0 ? GL_P - (uint64_t)(-(int)x) : (uint64_t)x; }
+
+// the degree-3 polynomial through (i, g[i]), i = 0..3, at r
+uint64_t lagrange4(const uint64_t g[4], uint64_t r) {
+    static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
+    const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2), r3 = gl_sub(r, 3);
+    // L0 = -(r-1)(r-2)(r-3)/6, L1 = r(r-2)(r-3)/2, L2 = -r(r-1)(r-3)/2, L3 = r(r-1)(r-2)/6
+    const uint64_t l0 = gl_sub(0, gl_mul(gl_mul(gl_mul(r1, r2), r3), inv6));
+    const uint64_t l1 = gl_mul(gl_mul(gl_mul(r, r2), r3), inv2);
+    const uint64_t l2 = gl_sub(0, gl_mul(gl_mul(gl_mul(r, r1), r3), inv2));
+    const uint64_t l3 = gl_mul(gl_mul(gl_mul(r, r1), r2), inv6);
+    return gl_add(gl_add(gl_mul(g[0], l0), gl_mul(g[1], l1)), gl_add(gl_mul(g[2], l2), gl_mul(g[3], l3)));
+}
+
+}  // namespace
+
+int sumcheck_prove_hadamard(fp_ctx* c, fp_tx* tx, const int8_t* s, const int8_t* u, int64_t n, uint8_t* proof,
+                            size_t* proof_len, void* stream) {
+    if (!c || !tx || !proof_len) return fp_fail(c, FP_ERR_ARG, "sumcheck_prove_hadamard: null argument");
+    if (!s || !u) return fp_fail(c, FP_ERR_ARG, "sumcheck_prove_hadamard: null factor");
+    if (n < 1 || n > (1ll << HAD_MAX_V))
+        return fp_fail(c, FP_ERR_SHAPE, "sumcheck_prove_hadamard: need 1 <= n <= 2^30");
+    const int v = fp_log2_ceil((uint64_t)n);
+    const size_t need_len = 8 + 32 * (size_t)v + 16;
+    if (!proof || *proof_len < need_len) {
+        *proof_len = need_len;
+        return fp_fail(c, FP_ERR_ARG, "sumcheck_prove_hadamard: proof buffer too small");
+    }
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t st = (cudaStream_t)stream;
+    int rc;
+
+    // ---- commit: digests of both factors ----
+    {
+        FpDigestJob jobs[2] = {{(const uint8_t*)s, (uint64_t)n}, {(const uint8_t*)u, (uint64_t)n}};
+        uint8_t d[64];
+        if ((rc = fp_digest_many(c, jobs, 2, d, st))) return rc;  // synchronises the stream
+        fp_tx_absorb_raw(tx, "had_site", d, 64);
+    }
+    FpPoint z;
+    z.v = v;
+    for (int i = 0; i < v; i++) z.z[i] = fp_tx_squeeze_one(tx, "had_z");
+
+    // ---- scratch ----
+    const int vl = v / 2, vh = v - vl;
+    const int64_t half = v > 0 ? 1ll << (v - 1) : 0;
+    int occ = 0;
+    FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, had_session_kernel, HAD_THREADS, 0));
+    const int cap_grid = std::max(1, occ) * c->num_sms;
+    const size_t part_n = (size_t)3 * std::max(cap_grid, 2 * c->num_sms);
+    size_t need = fp_align_up((size_t)8 << vh, 256) + fp_align_up((size_t)8 << vl, 256) +
+                  3 * fp_align_up((size_t)8 * std::max<int64_t>(half, 1), 256) + fp_align_up(8 * part_n, 256) +
+                  fp_align_up(8 * 64, 256) + 4096;
+    if ((rc = fp_reserve(c, c->dev, need))) return rc;
+    if ((rc = fp_reserve(c, c->host, 4096))) return rc;
+    fp_reset(c->dev);
+    fp_reset(c->host);
+    uint64_t* EH = (uint64_t*)fp_alloc(c->dev, (size_t)8 << vh);
+    uint64_t* EL = (uint64_t*)fp_alloc(c->dev, (size_t)8 << vl);
+    uint64_t* S = (uint64_t*)fp_alloc(c->dev, (size_t)8 * std::max<int64_t>(half, 1));
+    uint64_t* U = (uint64_t*)fp_alloc(c->dev, (size_t)8 * std::max<int64_t>(half, 1));
+    uint64_t* E = (uint64_t*)fp_alloc(c->dev, (size_t)8 * std::max<int64_t>(half, 1));
+    uint64_t* part = (uint64_t*)fp_alloc(c->dev, 8 * part_n);
+    uint64_t* small = (uint64_t*)fp_alloc(c->dev, 8 * 64);  // [0] claim, [8..] z
+    uint64_t* hs = (uint64_t*)fp_alloc(c->host, 8 * 64);
+    if (!EH || !EL || !S || !U || !E || !part || !small || !hs)
+        return fp_fail(c, FP_ERR_OOM, "sumcheck_prove_hadamard: scratch exhausted");
+
+    // ---- the claim c = h~(z) ----
+    {
+        FpPoint zh, zl;
+        zh.v = vh;
+        zl.v = vl;
+        for (int i = 0; i < vh; i++) zh.z[i] = z.z[i];
+        for (int i = 0; i < vl; i++) zl.z[i] = z.z[vh + i];
+        if ((rc = fp_eq_table(c, zh, EH, st))) return rc;
+        if ((rc = fp_eq_table(c, zl, EL, st))) return rc;
+        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 2 * (int64_t)c->num_sms));
+        int slot;
+        fp_tic(c, st, K_HAD_CLAIM, 2.0 * (double)n, &slot);
+        had_claim_kernel<<<(unsigned)blocks, 256, 0, st>>>(s, u, n, EH, EL, vl, part, c->tickets, small);
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+        for (int i = 0; i < v; i++) hs[8 + i] = z.z[i];
+        FP_CUDA(c, cudaMemcpyAsync(small + 8, hs + 8, 8 * (size_t)std::max(v, 1), cudaMemcpyHostToDevice, st));
+        FP_CUDA(c, cudaMemcpyAsync(hs, small, 8, cudaMemcpyDeviceToHost, st));
+        FP_CUDA(c, cudaStreamSynchronize(st));
+    }
+    size_t pos = 0;
+    uint64_t claim = hs[0];
+    put_u64s(proof + pos, &claim, 1);
+    fp_tx_absorb_raw(tx, "had_claim", proof + pos, 8);
+    pos += 8;
+
+    uint64_t fin[2];
+    if (v == 0) {
+        int8_t b2[2];
+        FP_CUDA(c, cudaMemcpyAsync(&b2[0], s, 1, cudaMemcpyDeviceToHost, st));
+        FP_CUDA(c, cudaMemcpyAsync(&b2[1], u, 1, cudaMemcpyDeviceToHost, st));
+        FP_CUDA(c, cudaStreamSynchronize(st));
+        fin[0] = lift_host(b2[0]);
+        fin[1] = lift_host(b2[1]);
+    } else {
+        HadArgs A;
+        memset(&A, 0, sizeof A);
+        A.s = s;
+        A.u = u;
+        A.n = n;
+        A.S = S;
+        A.U = U;
+        A.E = E;
+        A.z = small + 8;
+        A.v = v;
+        A.per_block = HAD_THREADS;  // one pair per thread
+        A.grid = (int)std::max<int64_t>(1, std::min<int64_t>((half + A.per_block - 1) / A.per_block, cap_grid));
+        A.seq0 = fp_seq_reserve(c, (uint64_t)v + 2);
+        if ((rc = fp_session_begin(c, st))) return rc;
+        fp_session_expect(c, 3);  // before any launch: round 1 publishes without a challenge
+        void* args[] = {&A, &c->mb_dev, &c->relay, &part};
+        auto round_bytes = [&](int t) {
+            const double pairs = (double)(1ll << (v - t));
+            return t == 1 ? 12.0 * pairs : (t == 2 ? 64.0 * pairs : 120.0 * pairs);
+        };
+        if (!c->stepped) {
+            A.t_begin = 1;
+            A.t_end = v + 1;
+            double bytes = 0;
+            for (int t = 1; t <= v; t++) bytes += round_bytes(t);
+            int slot;
+            fp_tic(c, st, K_HAD_ROUND, bytes, &slot);
+            FP_CUDA(c, cudaLaunchCooperativeKernel((const void*)had_session_kernel, dim3(A.grid), dim3(HAD_THREADS),
+                                                   args, 0, st));
+            fp_toc(c, st, slot);
+        }
+        uint64_t pre = 1;         // eq(z_<t, rho_<t)
+        for (int t = 1; t <= v; t++) {
+            if (c->stepped) {
+                A.t_begin = A.t_end = t;
+                int slot;
+                fp_tic(c, st, K_HAD_ROUND, round_bytes(t), &slot);
+                FP_CUDA(c, cudaLaunchCooperativeKernel((const void*)had_session_kernel, dim3(A.grid),
+                                                       dim3(HAD_THREADS), args, 0, st));
+                fp_toc(c, st, slot);
+            }
+            if ((rc = fp_session_wait(c, A.seq0 + t, st))) return rc;
+            const uint64_t h0 = c->mb->res[0], h1 = c->mb->res[1], h2 = c->mb->res[2];
+            const uint64_t zt = z.z[t - 1];
+            const uint64_t h3 = gl_add(gl_sub(h0, gl_mul(3, h1)), gl_mul(3, h2));
+            uint64_t g[4];
+            g[0] = gl_mul(pre, gl_mul(gl_sub(1, zt), h0));
+            g[1] = gl_mul(pre, gl_mul(zt, h1));
+            g[2] = gl_mul(pre, gl_mul(gl_sub(gl_mul(3, zt), 1), h2));
+            g[3] = gl_mul(pre, gl_mul(gl_sub(gl_mul(5, zt), 2), h3));
+            if (gl_add(g[0], g[1]) != claim)
+                return fp_fail(c, FP_ERR_CUDA, "sumcheck_prove_hadamard: round values inconsistent with the claim");
+            put_u64s(proof + pos, g, 4);
+            fp_tx_absorb_raw(tx, "had_round", proof + pos, 32);
+            pos += 32;
+            fp_session_expect(c, t < v ? 3 : 2);  // the last challenge triggers the final values
+            const uint64_t r = fp_tx_squeeze_one(tx, "had_chal");
+            fp_session_post(c, A.seq0 + t, r);
+            claim = lagrange4(g, r);
+            pre = gl_mul(pre, gl_add(gl_mul(zt, r), gl_mul(gl_sub(1, zt), gl_sub(1, r))));
+        }
+        if (c->stepped) {
+            A.t_begin = A.t_end = v + 1;
+            int slot;
+            fp_tic(c, st, K_HAD_FINAL, 32.0, &slot);
+            FP_CUDA(c, cudaLaunchCooperativeKernel((const void*)had_session_kernel, dim3(1), dim3(HAD_THREADS), args,
+                                                   0, st));
+            fp_toc(c, st, slot);
+        }
+        if ((rc = fp_session_wait(c, A.seq0 + v + 1, st))) return rc;
+        fin[0] = c->mb->res[0];
+        fin[1] = c->mb->res[1];
+        FP_CUDA(c, cudaStreamSynchronize(st));
+    }
+    put_u64s(proof + pos, fin, 2);
+    fp_tx_absorb_raw(tx, "had_final", proof + pos, 16);
+    pos += 16;
+    *proof_len = pos;
+    return FP_OK;
+}

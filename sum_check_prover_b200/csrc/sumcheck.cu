@@ -160,12 +160,12 @@ __global__ void sc_final_kernel(const uint64_t* A, const uint64_t* B, int nsites
     }
 }
 
+}  // namespace
+
 void put_u64s(uint8_t* p, const uint64_t* v, size_t n) {
     for (size_t i = 0; i < n; i++)
         for (int b = 0; b < 8; b++) p[8 * i + b] = (uint8_t)(v[i] >> (8 * b));
 }
-
-}  // namespace
 
 int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, uint8_t* proof, size_t* proof_len,
                           void* stream) {
