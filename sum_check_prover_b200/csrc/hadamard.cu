@@ -55,6 +55,11 @@ __device__ __forceinline__ uint64_t lift8(int8_t x) { return x < 0 ? GL_P - (uin
 
 __device__ __forceinline__ uint64_t ld8(const int8_t* a, int64_t i, int64_t n) { return i < n ? lift8(a[i]) : 0ull; }
 
+__device__ __forceinline__ int ld8i(const int8_t* a, int64_t i, int64_t n) { return i < n ? (int)a[i] : 0; }
+
+// a small signed integer as a field element
+__device__ __forceinline__ uint64_t lifti(int x) { return x < 0 ? GL_P - (uint64_t)(-(int64_t)x) : (uint64_t)x; }
+
 // X = 2 on the line through (a, b) at 0 and 1
 __device__ __forceinline__ uint64_t at2(uint64_t a, uint64_t b) { return gl_sub(gl_add(b, b), a); }
 
@@ -92,34 +97,41 @@ __global__ void __launch_bounds__(HAD_THREADS, 2) had_session_kernel(HadArgs A, 
         if (t == 1) EC = eq_chunks_build(eq_tab, zs, A.v);
         GlAcc a0, a1, a2;
         for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
-            uint64_t s0, s1, u0, u1, e;
             if (t == 1) {
-                s0 = ld8(A.s, b, A.n);
-                s1 = ld8(A.s, b + h, A.n);
-                u0 = ld8(A.u, b, A.n);
-                u1 = ld8(A.u, b + h, A.n);
-                e = eq_chunks_at(EC, eq_tab, b);  // eq(z_2..z_v, b)
+                // the int8 factors as they are: the three products are small integers
+                // (|s u| <= 2^14, |(2 s1 - s0)(2 u1 - u0)| < 2^18)
+                const int s0 = ld8i(A.s, b, A.n), s1 = ld8i(A.s, b + h, A.n);
+                const int u0 = ld8i(A.u, b, A.n), u1 = ld8i(A.u, b + h, A.n);
+                const uint64_t e = eq_chunks_at(EC, eq_tab, b);  // eq(z_2..z_v, b)
                 if (A.v > 1) A.E[b] = e;
-            } else {
-                if (t == 2) {
-                    // the int8 factors (length 4h) folded by rho_1
-                    s0 = gl_fold_fast(ld8(A.s, b, A.n), ld8(A.s, b + 2 * h, A.n), rprev);
-                    s1 = gl_fold_fast(ld8(A.s, b + h, A.n), ld8(A.s, b + 3 * h, A.n), rprev);
-                    u0 = gl_fold_fast(ld8(A.u, b, A.n), ld8(A.u, b + 2 * h, A.n), rprev);
-                    u1 = gl_fold_fast(ld8(A.u, b + h, A.n), ld8(A.u, b + 3 * h, A.n), rprev);
-                } else {
-                    s0 = gl_fold_fast(__ldcg(A.S + b), __ldcg(A.S + b + 2 * h), rprev);
-                    s1 = gl_fold_fast(__ldcg(A.S + b + h), __ldcg(A.S + b + 3 * h), rprev);
-                    u0 = gl_fold_fast(__ldcg(A.U + b), __ldcg(A.U + b + 2 * h), rprev);
-                    u1 = gl_fold_fast(__ldcg(A.U + b + h), __ldcg(A.U + b + 3 * h), rprev);
-                }
-                A.S[b] = s0;
-                A.S[b + h] = s1;
-                A.U[b] = u0;
-                A.U[b + h] = u1;
-                e = gl_add(__ldcg(A.E + b), __ldcg(A.E + b + h));  // eq(z_>t, b)
-                A.E[b] = e;
+                a0.mac(e, lifti(s0 * u0));
+                a1.mac(e, lifti(s1 * u1));
+                a2.mac(e, lifti((2 * s1 - s0) * (2 * u1 - u0)));
+                continue;
             }
+            uint64_t s0, s1, u0, u1;
+            if (t == 2) {
+                // the int8 factors (length 4h) folded by rho_1: a + rho_1 (b - a) with b - a small
+                const int sa = ld8i(A.s, b, A.n), sb = ld8i(A.s, b + 2 * h, A.n);
+                const int sc = ld8i(A.s, b + h, A.n), sd = ld8i(A.s, b + 3 * h, A.n);
+                const int ua = ld8i(A.u, b, A.n), ub = ld8i(A.u, b + 2 * h, A.n);
+                const int uc = ld8i(A.u, b + h, A.n), ud = ld8i(A.u, b + 3 * h, A.n);
+                s0 = gl_add(lifti(sa), gl_mul_small(rprev, sb - sa));
+                s1 = gl_add(lifti(sc), gl_mul_small(rprev, sd - sc));
+                u0 = gl_add(lifti(ua), gl_mul_small(rprev, ub - ua));
+                u1 = gl_add(lifti(uc), gl_mul_small(rprev, ud - uc));
+            } else {
+                s0 = gl_fold_fast(__ldcg(A.S + b), __ldcg(A.S + b + 2 * h), rprev);
+                s1 = gl_fold_fast(__ldcg(A.S + b + h), __ldcg(A.S + b + 3 * h), rprev);
+                u0 = gl_fold_fast(__ldcg(A.U + b), __ldcg(A.U + b + 2 * h), rprev);
+                u1 = gl_fold_fast(__ldcg(A.U + b + h), __ldcg(A.U + b + 3 * h), rprev);
+            }
+            A.S[b] = s0;
+            A.S[b + h] = s1;
+            A.U[b] = u0;
+            A.U[b + h] = u1;
+            const uint64_t e = gl_add(__ldcg(A.E + b), __ldcg(A.E + b + h));  // eq(z_>t, b)
+            A.E[b] = e;
             a0.mac(e, gl_mul_weak(s0, u0));
             a1.mac(e, gl_mul_weak(s1, u1));
             a2.mac(e, gl_mul_weak(at2(s0, s1), at2(u0, u1)));
