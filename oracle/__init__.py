@@ -47,6 +47,10 @@ REASONS = {
     16: "had_round",
     17: "had_final",
     18: "had_open",
+    19: "scl_claim",
+    20: "scl_round",
+    21: "scl_final",
+    22: "scl_open",
 }
 
 
@@ -114,6 +118,10 @@ def lib():
         L.orc_had_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
         L.orc_had_verify.restype = C.c_int
         L.orc_had_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
+        L.orc_scl_prove.restype = C.c_int
+        L.orc_scl_prove.argtypes = [vp, vp, C.c_int, vp, C.c_int, C.c_int, vp, vp, u64, C.POINTER(u64)]
+        L.orc_scl_verify.restype = C.c_int
+        L.orc_scl_verify.argtypes = [vp, vp, C.c_int, vp, C.c_int, C.c_int, vp, vp, u64, vp]
         _lib = L
     return _lib
 
@@ -393,5 +401,48 @@ def had_verify(seed: int, s, u, proof: bytes):
     det = np.zeros(2, dtype=np.int64)
     tx = L.orc_tx_new(seed)
     rc = L.orc_had_verify(tx, _ptr(a), _ptr(b), a.size, _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+# ---- per-group scale reduction: W_eff = S (.) w to claims on w and S ----------------
+
+def scl_prove(seed: int, w, bits: int, scales, M: int, K: int, z):
+    """Sum-check reducing a claim on W_eff~(z) (W_eff[i][k] = S[i][k // 64] w[i][k]) to
+    claims on w and S (see oracle.c). z: vM + vK field elements, row coordinates first.
+    Returns (proof bytes, transcript state after)."""
+    L = lib()
+    wa = np.ascontiguousarray(w)
+    sa = np.ascontiguousarray(np.asarray(scales, dtype=np.int8))
+    za = _u64(z)
+    out = []
+    for _ in range(2):
+        tx = L.orc_tx_new(seed)
+        n = C.c_uint64(0)
+        buf = np.zeros(max(1, out[0] if out else 1), dtype=np.uint8)
+        rc = L.orc_scl_prove(tx, _ptr(wa), bits, _ptr(sa), M, K, _ptr(za), _ptr(buf) if out else None,
+                             out[0] if out else 0, C.byref(n))
+        st = C.create_string_buffer(32)
+        L.orc_tx_state(tx, st)
+        L.orc_tx_free(tx)
+        if out:
+            if rc != 0:
+                raise ValueError(f"orc_scl_prove failed ({rc})")
+            return buf[: n.value].tobytes(), st.raw
+        if rc not in (0, -2):
+            raise ValueError(f"orc_scl_prove rejected the statement ({rc})")
+        out.append(n.value)
+
+
+def scl_verify(seed: int, w, bits: int, scales, M: int, K: int, z, proof: bytes):
+    """Returns (reason_name, detail); 'accept' for a valid proof."""
+    L = lib()
+    wa = np.ascontiguousarray(w)
+    sa = np.ascontiguousarray(np.asarray(scales, dtype=np.int8))
+    za = _u64(z)
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_scl_verify(tx, _ptr(wa), bits, _ptr(sa), M, K, _ptr(za), _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

@@ -1213,6 +1213,68 @@ enum {
     REJ_HAD_OPEN = 18    /* S or U != the committed vector's MLE at rho */
 };
 
+/* The rounds of the textbook product sum-check of E S U over v variables (E,
+ * S, U of length 2^v, folded in place): round r sends g(0..3) under lab_round,
+ * with g(X) = sum_b E(X, b) S(X, b) U(X, b) on each vector's line through
+ * (b, b + h); squeezes rho_r under lab_chal; folds all three. Then sends the
+ * final S(rho), U(rho) under lab_final. */
+static void prod3_rounds(orc_tx* t, pbuf* pb, u64* E, u64* S, u64* U, int v, const char* lab_round,
+                         const char* lab_chal, const char* lab_final) {
+    u64 L = (u64)1 << v;
+    for (int r = 0; r < v; r++) {
+        u64 h = L >> 1;
+        u64 g[4] = {0, 0, 0, 0};
+        for (u64 b = 0; b < h; b++)
+            for (u64 X = 0; X < 4; X++) {
+                /* each vector's line through (b, b + h) at X */
+                u64 e = orc_fadd(E[b], orc_fmul(X, orc_fsub(E[h + b], E[b])));
+                u64 sx = orc_fadd(S[b], orc_fmul(X, orc_fsub(S[h + b], S[b])));
+                u64 ux = orc_fadd(U[b], orc_fmul(X, orc_fsub(U[h + b], U[b])));
+                g[X] = orc_fadd(g[X], orc_fmul(e, orc_fmul(sx, ux)));
+            }
+        send_fe(t, pb, lab_round, g, 4);
+        u64 rho = orc_tx_squeeze(t, lab_chal);
+        for (u64 b = 0; b < h; b++) {
+            E[b] = orc_fadd(E[b], orc_fmul(rho, orc_fsub(E[h + b], E[b])));
+            S[b] = orc_fadd(S[b], orc_fmul(rho, orc_fsub(S[h + b], S[b])));
+            U[b] = orc_fadd(U[b], orc_fmul(rho, orc_fsub(U[h + b], U[b])));
+        }
+        L = h;
+    }
+    u64 fin[2] = {S[0], U[0]};
+    send_fe(t, pb, lab_final, fin, 2);
+}
+
+/* Verifier side of prod3_rounds: each round's g(0) + g(1) against the running
+ * claim (starting at *claim), the next claim g(rho) by Lagrange; returns 0 or
+ * REJ_FORMAT / bad_round with detail[0] = the round. rho (v entries) and fin
+ * (S(rho), U(rho)) are filled in; *claim ends as the last round's g(rho). */
+static int prod3_verify(orc_tx* t, prd* rd, int v, u64* claim, u64* rho, u64 fin[2], const char* lab_round,
+                        const char* lab_chal, const char* lab_final, int bad_round, int64_t* detail) {
+    for (int r = 0; r < v; r++) {
+        u64 g[4];
+        rd_fe(t, rd, lab_round, g, 4);
+        detail[0] = r;
+        if (rd->bad) return REJ_FORMAT;
+        if (orc_fadd(g[0], g[1]) != *claim) return bad_round;
+        rho[r] = orc_tx_squeeze(t, lab_chal);
+        *claim = orc_lagrange(g, 4, rho[r]);
+    }
+    detail[0] = v;
+    rd_fe(t, rd, lab_final, fin, 2);
+    if (rd->bad) return REJ_FORMAT;
+    detail[0] = 0;
+    return 0;
+}
+
+/* eq(z, rho) in closed form */
+static u64 eq_closed(const u64* z, const u64* rho, int v) {
+    u64 e = 1;
+    for (int i = 0; i < v; i++)
+        e = orc_fmul(e, orc_fadd(orc_fmul(z[i], rho[i]), orc_fmul(orc_fsub(1, z[i]), orc_fsub(1, rho[i]))));
+    return e;
+}
+
 static void had_absorb_site(orc_tx* t, const int8_t* s, const int8_t* u, u64 n) {
     uint8_t d[64];
     orc_tree_digest(s, n, d);
@@ -1246,29 +1308,7 @@ int orc_had_prove(void* txh, const int8_t* s, const int8_t* u, u64 n, uint8_t* p
     u64 c = 0;
     for (u64 x = 0; x < sz; x++) c = orc_fadd(c, orc_fmul(E[x], orc_fmul(S[x], U[x])));
     send_fe(t, &pb, "had_claim", &c, 1);
-    u64 L = sz;
-    for (int r = 0; r < v; r++) {
-        u64 h = L >> 1;
-        u64 g[4] = {0, 0, 0, 0};
-        for (u64 b = 0; b < h; b++)
-            for (u64 X = 0; X < 4; X++) {
-                /* each vector's line through (b, b + h) at X */
-                u64 e = orc_fadd(E[b], orc_fmul(X, orc_fsub(E[h + b], E[b])));
-                u64 sx = orc_fadd(S[b], orc_fmul(X, orc_fsub(S[h + b], S[b])));
-                u64 ux = orc_fadd(U[b], orc_fmul(X, orc_fsub(U[h + b], U[b])));
-                g[X] = orc_fadd(g[X], orc_fmul(e, orc_fmul(sx, ux)));
-            }
-        send_fe(t, &pb, "had_round", g, 4);
-        u64 rho = orc_tx_squeeze(t, "had_chal");
-        for (u64 b = 0; b < h; b++) {
-            E[b] = orc_fadd(E[b], orc_fmul(rho, orc_fsub(E[h + b], E[b])));
-            S[b] = orc_fadd(S[b], orc_fmul(rho, orc_fsub(S[h + b], S[b])));
-            U[b] = orc_fadd(U[b], orc_fmul(rho, orc_fsub(U[h + b], U[b])));
-        }
-        L = h;
-    }
-    u64 fin[2] = {S[0], U[0]};
-    send_fe(t, &pb, "had_final", fin, 2);
+    prod3_rounds(t, &pb, E, S, U, v, "had_round", "had_chal", "had_final");
     free(z);
     free(E);
     free(S);
@@ -1306,23 +1346,13 @@ int orc_had_verify(void* txh, const int8_t* s, const int8_t* u, u64 n, const uin
         if (want != c) FAIL(REJ_HAD_CLAIM, 0, 0);
     }
     claim = c;
-    for (int r = 0; r < v; r++) {
-        u64 g[4];
-        rd_fe(t, &rd, "had_round", g, 4);
-        if (rd.bad) FAIL(REJ_FORMAT, r, 0);
-        if (orc_fadd(g[0], g[1]) != claim) FAIL(REJ_HAD_ROUND, r, 0);
-        rho[r] = orc_tx_squeeze(t, "had_chal");
-        claim = orc_lagrange(g, 4, rho[r]);
-    }
     u64 fin[2];
-    rd_fe(t, &rd, "had_final", fin, 2);
-    if (rd.bad) FAIL(REJ_FORMAT, v, 0);
     {
-        u64 e = 1;
-        for (int i = 0; i < v; i++)
-            e = orc_fmul(e, orc_fadd(orc_fmul(z[i], rho[i]), orc_fmul(orc_fsub(1, z[i]), orc_fsub(1, rho[i]))));
-        if (orc_fmul(e, orc_fmul(fin[0], fin[1])) != claim) FAIL(REJ_HAD_FINAL, 0, 0);
+        int64_t d0 = 0;
+        int r2 = prod3_verify(t, &rd, v, &claim, rho, fin, "had_round", "had_chal", "had_final", REJ_HAD_ROUND, &d0);
+        if (r2) FAIL(r2, d0, 0);
     }
+    if (orc_fmul(eq_closed(z, rho, v), orc_fmul(fin[0], fin[1])) != claim) FAIL(REJ_HAD_FINAL, 0, 0);
     if (orc_mle_eval(S, sz, rho, v) != fin[0]) FAIL(REJ_HAD_OPEN, 0, 0);
     if (orc_mle_eval(U, sz, rho, v) != fin[1]) FAIL(REJ_HAD_OPEN, 1, 0);
     if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
@@ -1331,5 +1361,130 @@ done:
     free(rho);
     free(S);
     free(U);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-group scale reduction. A site with per-64-column int8 scales uses     */
+/* W_eff[i][k] = S[i][k / 64] w[i][k]; its matmul sum-check ends with a      */
+/* claim on W_eff~(z), but only w and S are committed. As for the gated     */
+/* product ("How fast can FlashProve go", 3.1: a product that is not        */
+/* committed is reduced by sum-check to claims on its committed factors),   */
+/* the same degree-3 product sum-check runs over x = (i, k) (row bits       */
+/* first; M and K padded to 2^vM and 2^vK) with the factors                 */
+/*   Se(i, k) = S[i][k >> 6] (0 past the M x G scales, G = ceil(K / 64)),    */
+/*   w(i, k)  (0 past M x K),                                                */
+/* at a point z = (z_row, z_col) the caller supplies:                        */
+/*   absorb "scl_site" D(W bytes) || D(S bytes);                             */
+/*   send a = sum_x eq(z, x) Se(x) w(x) ("scl_claim");                        */
+/*   v = vM + vK rounds ("scl_round", "scl_chal"); send Se(rho), w(rho)        */
+/*   ("scl_final").                                                           */
+/* Se does not depend on the six low column bits, so Se~(rho) is            */
+/* S~(rho_row, rho_col_hi), rho_col_hi the first vK - 6 column coordinates  */
+/* (none when vK <= 6): a claim on the committed scales.                    */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_SCL_CLAIM = 19,  /* a != W_eff~(z) recomputed from w and S */
+    REJ_SCL_ROUND = 20,  /* g_t(0) + g_t(1) != running claim */
+    REJ_SCL_FINAL = 21,  /* eq(z, rho) Se w != claim after the last round */
+    REJ_SCL_OPEN = 22    /* Se(rho) != S~(rho_row, rho_col_hi) or w(rho) != w~(rho) */
+};
+
+static int64_t w_raw(const void* w, int bits, int K, u64 i, u64 k) {
+    if (bits == 8) return ((const int8_t*)w)[i * (u64)K + k];
+    const uint8_t* row = (const uint8_t*)w + i * (u64)((K + 1) / 2);
+    int nib = (k & 1) ? (row[k / 2] >> 4) : (row[k / 2] & 15);
+    return nib >= 8 ? nib - 16 : nib;
+}
+
+/* the two factors over the padded 2^(vM + vK) grid */
+static void scl_vectors(const void* w, int bits, const int8_t* sc, int M, int K, int vM, int vK, u64* Se, u64* W) {
+    u64 G = (u64)(K + 63) / 64, cols = (u64)1 << vK;
+    for (u64 i = 0; i < ((u64)1 << vM); i++)
+        for (u64 k = 0; k < cols; k++) {
+            u64 x = i * cols + k;
+            Se[x] = (i < (u64)M && (k >> 6) < G) ? orc_fint(sc[i * G + (k >> 6)]) : 0;
+            W[x] = (i < (u64)M && k < (u64)K) ? orc_fint(w_raw(w, bits, K, i, k)) : 0;
+        }
+}
+
+static void scl_absorb_site(orc_tx* t, const void* w, int bits, const int8_t* sc, int M, int K) {
+    uint8_t d[64];
+    orc_tree_digest(w, (u64)M * (bits == 4 ? (u64)((K + 1) / 2) : (u64)K), d);
+    orc_tree_digest(sc, (u64)M * (u64)((K + 63) / 64), d + 32);
+    orc_tx_absorb(t, "scl_site", d, 64);
+}
+
+static int scl_args_ok(int bits, int M, int K) { return (bits == 4 || bits == 8) && M >= 1 && K >= 1; }
+
+int orc_scl_prove(void* txh, const void* w, int bits, const int8_t* sc, int M, int K, const u64* z, uint8_t* proof,
+                  u64 cap, u64* len) {
+    if (!scl_args_ok(bits, M, K)) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int vM = orc_log2_ceil((u64)M), vK = orc_log2_ceil((u64)K), v = vM + vK;
+    u64 sz = (u64)1 << v;
+    pbuf pb = {proof, cap, 0, 0};
+    scl_absorb_site(t, w, bits, sc, M, K);
+    u64* E = (u64*)malloc(sz * sizeof(u64));
+    u64* Se = (u64*)malloc(sz * sizeof(u64));
+    u64* W = (u64*)malloc(sz * sizeof(u64));
+    orc_eq_table(z, v, E);
+    scl_vectors(w, bits, sc, M, K, vM, vK, Se, W);
+    u64 a = 0;
+    for (u64 x = 0; x < sz; x++) a = orc_fadd(a, orc_fmul(E[x], orc_fmul(Se[x], W[x])));
+    send_fe(t, &pb, "scl_claim", &a, 1);
+    prod3_rounds(t, &pb, E, Se, W, v, "scl_round", "scl_chal", "scl_final");
+    free(E);
+    free(Se);
+    free(W);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+int orc_scl_verify(void* txh, const void* w, int bits, const int8_t* sc, int M, int K, const u64* z,
+                   const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (!scl_args_ok(bits, M, K)) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int vM = orc_log2_ceil((u64)M), vK = orc_log2_ceil((u64)K), v = vM + vK, rc = 0;
+    int vKh = vK > 6 ? vK - 6 : 0;
+    u64 sz = (u64)1 << v, G = (u64)(K + 63) / 64;
+    prd rd = {proof, len, 0, 0};
+    u64* Se = (u64*)malloc(sz * sizeof(u64));
+    u64* W = (u64*)malloc(sz * sizeof(u64));
+    u64* P = (u64*)malloc(sz * sizeof(u64));
+    u64* rho = (u64*)malloc(sizeof(u64) * (v + 1));
+    u64* Sp = (u64*)calloc((u64)1 << (vM + vKh), sizeof(u64));
+    u64* pt = (u64*)malloc(sizeof(u64) * (vM + vKh + 1));
+    scl_absorb_site(t, w, bits, sc, M, K);
+    scl_vectors(w, bits, sc, M, K, vM, vK, Se, W);
+    u64 a, claim, fin[2];
+    rd_fe(t, &rd, "scl_claim", &a, 1);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    for (u64 x = 0; x < sz; x++) P[x] = orc_fmul(Se[x], W[x]);
+    if (orc_mle_eval(P, sz, z, v) != a) FAIL(REJ_SCL_CLAIM, 0, 0);
+    claim = a;
+    {
+        int64_t d0 = 0;
+        int r2 = prod3_verify(t, &rd, v, &claim, rho, fin, "scl_round", "scl_chal", "scl_final", REJ_SCL_ROUND, &d0);
+        if (r2) FAIL(r2, d0, 0);
+    }
+    if (orc_fmul(eq_closed(z, rho, v), orc_fmul(fin[0], fin[1])) != claim) FAIL(REJ_SCL_FINAL, 0, 0);
+    /* openings: the scales at (rho_row, rho_col_hi), the weights at rho */
+    for (u64 i = 0; i < (u64)M; i++)
+        for (u64 g = 0; g < G; g++) Sp[(i << vKh) + g] = orc_fint(sc[i * G + g]);
+    for (int i = 0; i < vM; i++) pt[i] = rho[i];
+    for (int i = 0; i < vKh; i++) pt[vM + i] = rho[vM + i];
+    if (orc_mle_eval(Sp, (u64)1 << (vM + vKh), pt, vM + vKh) != fin[0]) FAIL(REJ_SCL_OPEN, 0, 0);
+    if (orc_mle_eval(W, sz, rho, v) != fin[1]) FAIL(REJ_SCL_OPEN, 1, 0);
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(Se);
+    free(W);
+    free(P);
+    free(rho);
+    free(Sp);
+    free(pt);
     return rc;
 }

@@ -378,3 +378,61 @@ def had_prove(seed: int, s, u) -> bytes:
     out += fe_bytes(fin)
     tx.absorb("had_final", fe_bytes(fin))
     return out
+
+
+# ---- per-group scale reduction -------------------------------------------------
+
+def _prod3_rounds(tx, z, svals, uvals, lab_round, lab_chal, lab_final) -> bytes:
+    """Round values of the product sum-check of eq(z, .) s u from definitions (hypercube sums)."""
+    v = len(z)
+    out = b""
+    rho = []
+    for t in range(v):
+        rest = v - t - 1
+        g = []
+        for X in range(4):
+            acc = 0
+            for b in range(1 << rest):
+                w = rho + [X] + [(b >> (rest - 1 - i)) & 1 for i in range(rest)]
+                acc += eq_ml(z, w) * mle_at(svals, w) * mle_at(uvals, w)
+            g.append(acc % P)
+        out += fe_bytes(g)
+        tx.absorb(lab_round, fe_bytes(g))
+        rho.append(tx.squeeze(lab_chal))
+    fin = [mle_at(svals, rho), mle_at(uvals, rho)]
+    out += fe_bytes(fin)
+    tx.absorb(lab_final, fe_bytes(fin))
+    return out, rho
+
+
+def scale_factors(w, bits: int, scales, M: int, K: int):
+    """Se(i, k) = S[i][k // 64] and w(i, k) over the padded (row bits first) grid, as lists."""
+    vM, vK = log2c(M), log2c(K)
+    G = (K + 63) // 64
+    if bits == 8:
+        wv = np.asarray(w, np.int64)
+    else:
+        b = np.asarray(w, np.int64)
+        full = np.empty((M, 2 * b.shape[1]), np.int64)
+        full[:, 0::2], full[:, 1::2] = b & 15, b >> 4
+        wv = np.where(full >= 8, full - 16, full)[:, :K]
+    sc = np.asarray(scales, np.int64).reshape(M, G)
+    Se, W = [], []
+    for i in range(1 << vM):
+        for k in range(1 << vK):
+            Se.append(int(sc[i, k // 64]) if i < M and k // 64 < G else 0)
+            W.append(int(wv[i, k]) if i < M and k < K else 0)
+    return Se, W
+
+
+def scl_prove(seed: int, w, bits: int, scales, M: int, K: int, z) -> bytes:
+    """The scale reduction's proof from definitions, at the given point z (row coordinates first)."""
+    Se, W = scale_factors(w, bits, scales, M, K)
+    tx = Tx(seed)
+    wb = np.ascontiguousarray(w).tobytes()
+    tx.absorb("scl_site", tree_digest(wb) + tree_digest(np.ascontiguousarray(scales, dtype=np.int8).tobytes()))
+    a = sum(eq_ml(z, [(x >> (len(z) - 1 - i)) & 1 for i in range(len(z))]) * Se[x] * W[x]
+            for x in range(len(Se))) % P
+    tx.absorb("scl_claim", fe_bytes([a]))
+    body, _ = _prod3_rounds(tx, list(z), Se, W, "scl_round", "scl_chal", "scl_final")
+    return fe_bytes([a]) + body
