@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had") -> dict:
+def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl") -> dict:
     """Kernel rooflines at HBM scale (inputs well above the 126 MB L2), from a
     profiled pass: every round is its own launch, timed with CUDA events.
 
@@ -186,7 +186,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had") -> di
     had_round: gated-product sum-check rounds over two 2^26-entry int8 factors
       (round 1 reads the int8 factors and writes the eq table, round 2 folds
       them into field vectors, later rounds read 4 and write 2 values of both
-      factors and fold the eq table: 120 B per pair).
+      factors and fold the eq table: 120 B per pair); and the same rounds reducing a
+      14336 x 4096 int4 weight matrix with per-64 scales to claims on w and S.
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
@@ -273,6 +274,17 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had") -> di
         uv = torch.from_numpy(rng.integers(-128, 128, n).astype("int8")).to(dev)
         measure("hadamard_round_2^26", "had_round", lambda: ctx.prove_hadamard(fp.Transcript(4), sv, uv))
         del sv, uv
+
+    if "scl" in which:
+        # the scale reduction of an FFN gate projection: 14336 x 4096 int4 weights with per-64 scales
+        rng = __import__("numpy").random.default_rng(10)
+        M, K = 14336, 4096
+        wv = torch.from_numpy(workloads.int4_packed(rng, M, K)).to(dev)
+        sv = torch.from_numpy(workloads.group_scales(rng, M, K)).to(dev)
+        pt = [int(x) for x in rng.integers(0, fp.P, size=26, dtype="uint64")]
+        measure("scale_reduction_round_14336x4096", "had_round",
+                lambda: ctx.reduce_scales(fp.Transcript(5), wv, 4, sv, M, K, pt))
+        del wv, sv
 
     if "gkr" in which:
         s = workloads.random_site(77, 8192, 64, 8192, 8, 12)
@@ -538,7 +550,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-micro", action="store_true")
-    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm,had", default=None,
+    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm,had,scl", default=None,
                     help="run only the kernel measurements at scale (comma list of sc, pe, gkr, gemm)")
     args = ap.parse_args()
     if args.micro_only:

@@ -232,6 +232,28 @@ int sumcheck_prove_hadamard(fp_ctx* ctx, fp_tx* tx, const int8_t* s, const int8_
                             size_t* proof_len, void* stream);
 
 /*
+ * Per-group scale reduction: a claim on W_eff~(z), W_eff[i][k] = S[i][k / 64] w[i][k]
+ * (what the matmul sum-check of a site with scales ends with), reduced to claims on
+ * the committed weights w and scales S by the same product sum-check as the gated
+ * product ("How fast can FlashProve go", 3.1: a product that is not committed is
+ * reduced by sum-check to its committed factors). Variables x = (i, k), row bits
+ * first, M and K padded to 2^vM, 2^vK; factors Se(i, k) = S[i][k >> 6] (zero past
+ * the M x ceil(K/64) scales) and w(i, k) (zero past M x K).
+ * w: device, M x K int8 or int4 (two per byte, low nibble = even k, rows of
+ * ceil(K/2) bytes); scales: device, M x ceil(K/64) int8; point: host, vM + vK
+ * canonical field elements (row coordinates first). The call continues tx:
+ *   absorb "scl_site" D(W) || D(S); send a = sum_x eq(z, x) Se(x) w(x) ("scl_claim");
+ *   vM + vK rounds of g(0..3) ("scl_round") and challenges ("scl_chal");
+ *   send Se~(rho), w~(rho) ("scl_final").
+ * Se~(rho) equals S~(rho_row, rho_col_hi), rho_col_hi the first vK - 6 column
+ * coordinates (none when vK <= 6). Proof: 8 + 32 (vM + vK) + 16 bytes.
+ * M, K >= 1 and vM + vK <= 30, else FP_ERR_SHAPE; null or non-canonical
+ * arguments FP_ERR_ARG; proof / proof_len as for sumcheck_prove_matmul.
+ */
+int sumcheck_reduce_scales(fp_ctx* ctx, fp_tx* tx, const void* w, int w_bits, const int8_t* scales, int M, int K,
+                           const uint64_t* point, uint8_t* proof, size_t* proof_len, void* stream);
+
+/*
  * Self-test of the bounded device waits. The sum-check kernels stay resident
  * across rounds and wait (a bounded number of polls) for each Fiat-Shamir
  * challenge from the host. This call launches a kernel that waits for a

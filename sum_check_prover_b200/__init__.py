@@ -74,6 +74,7 @@ def lib():
     L.sumcheck_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
     L.logup_prove_rescale.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
     L.sumcheck_prove_hadamard.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
+    L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, C.POINTER(sz), vp]
     L.fp_proof_size.argtypes = [C.POINTER(_Site), i32, C.POINTER(sz), C.POINTER(sz)]
     L.fp_ctx_set_profiling.argtypes = [vp, i32]
     L.fp_session_selftest.argtypes = [vp, vp]
@@ -246,6 +247,27 @@ class Context:
         ln = C.c_size_t(cap)
         self._check(self._L.sumcheck_prove_hadamard(self.h, tx.h, _ptr(s), _ptr(u), n, buf, C.byref(ln),
                                                     _stream(stream)), "sumcheck_prove_hadamard")
+        return buf.raw[: ln.value]
+
+    def reduce_scales(self, tx: Transcript, w, bits: int, scales, M: int, K: int, point: Sequence[int],
+                      stream=None) -> bytes:
+        """Sum-check reducing a claim on the scaled weights' MLE at point (row coordinates
+        first) to claims on the weights w and the per-64-column scales (device tensors)."""
+        v = 0
+        while (1 << v) < M:
+            v += 1
+        vk = 0
+        while (1 << vk) < K:
+            vk += 1
+        v += vk
+        if len(point) != v:
+            raise ValueError(f"reduce_scales: the point needs {v} coordinates")
+        pt = (C.c_uint64 * max(1, v))(*[int(p) for p in point])
+        cap = 8 + 32 * v + 16
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        self._check(self._L.sumcheck_reduce_scales(self.h, tx.h, _ptr(w), bits, _ptr(scales), M, K, pt, buf,
+                                                   C.byref(ln), _stream(stream)), "sumcheck_reduce_scales")
         return buf.raw[: ln.value]
 
     def prove_logup(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
