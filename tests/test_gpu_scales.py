@@ -84,3 +84,21 @@ def test_ffn_gate_full_size_verified(env):
     pf, _ = _gpu(env, 2, w, bits, sc, M, K, z)
     assert len(pf) == 8 + 32 * 26 + 16
     assert oracle.scl_verify(2, w, bits, sc, M, K, z, pf) == ("accept", (0, 0))
+
+
+def test_argument_errors(env):
+    torch, fp, ctx = env
+    w, sc, z = _site(4, 64, 4, 1)
+    wd = torch.from_numpy(np.ascontiguousarray(w)).cuda()
+    sd = torch.from_numpy(np.ascontiguousarray(sc)).cuda()
+    with pytest.raises(fp.FpError):  # weights are int4 or int8
+        ctx.reduce_scales(fp.Transcript(0), wd, 2, sd, 4, 64, z)
+    with pytest.raises(fp.FpError):  # a coordinate that is not a field element
+        ctx.reduce_scales(fp.Transcript(0), wd, 4, sd, 4, 64, [P] + z[1:])
+    with pytest.raises(ValueError):  # the point has vM + vK coordinates
+        ctx.reduce_scales(fp.Transcript(0), wd, 4, sd, 4, 64, z[:-1])
+    with pytest.raises(fp.FpError):  # M = 0: the binding asks for the 6 column coordinates, the library refuses
+        ctx.reduce_scales(fp.Transcript(0), wd, 4, sd, 0, 64, [1] * 6)
+    # the context is still usable afterwards
+    pf, _ = _gpu(env, 6, w, 4, sc, 4, 64, z)
+    assert pf == oracle.scl_prove(6, w, 4, sc, 4, 64, z)[0]
