@@ -321,6 +321,20 @@ def dist():
     return world, rank, local
 
 
+# The pages' own figures, with their hardware: context for the numbers above, not a target
+# (other hardware, whole-model proofs including commitments, which this path does not build).
+PAGES_CONTEXT = {
+    "flashprove_maverick_h100": "about 100 proved tokens/s for Llama 4 Maverick (4-bit weights, batches of 64 "
+                                "1,024-token requests) on one H100, 111 tokens/s at batch 24 "
+                                "(How fast can FlashProve go; FlashProve: How AI Answers Become Provable)",
+    "layer_rtx5070ti": "3.2-6.1 s prove-to-verify per Maverick-width layer on an RTX 5070 Ti "
+                       "(flashprove-consumer-gpu)",
+    "llama8b_request_h100": "1.0-1.5 h per 4,096 + 512-token Llama-3.1-8B request on one H100, with a "
+                            "different proof system (a Circle STARK over M31) (Towards Proving Frontier-Scale "
+                            "LLM Inference)",
+}
+
+
 def run_reference(args):
     """The CPU oracle as it stands, on a bounded sample of the same workload."""
     world, rank, local = dist()
@@ -532,7 +546,8 @@ def run_ours(args):
                 "kernels": kern,
                 "kernels_stepped": kern_stepped,
                 "microbench": micro,
-                "proof_bytes": proof_len}
+                "proof_bytes": proof_len,
+                "pages_context": PAGES_CONTEXT}
         print(json.dumps(line), flush=True)
     if pg is not None:
         pg.barrier()
