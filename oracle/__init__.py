@@ -51,6 +51,11 @@ REASONS = {
     20: "scl_round",
     21: "scl_final",
     22: "scl_open",
+    23: "silu_root",
+    24: "silu_round",
+    25: "silu_final",
+    26: "silu_leaf",
+    27: "silu_open",
 }
 
 
@@ -58,7 +63,7 @@ def build(force: bool = False) -> Path:
     """Compile oracle.c into liboracle.so with gcc (no GPU needed)."""
     if force or not _LIB.exists() or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
         tmp = _LIB.with_suffix(f".so.{os.getpid()}")
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(tmp), str(_SRC)])
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(tmp), str(_SRC), "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -122,6 +127,12 @@ def lib():
         L.orc_scl_prove.argtypes = [vp, vp, C.c_int, vp, C.c_int, C.c_int, vp, vp, u64, C.POINTER(u64)]
         L.orc_scl_verify.restype = C.c_int
         L.orc_scl_verify.argtypes = [vp, vp, C.c_int, vp, C.c_int, C.c_int, vp, vp, u64, vp]
+        L.orc_silu_q.restype = C.c_int32
+        L.orc_silu_q.argtypes = [C.c_int32]
+        L.orc_silu_prove.restype = C.c_int
+        L.orc_silu_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
+        L.orc_silu_verify.restype = C.c_int
+        L.orc_silu_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
         _lib = L
     return _lib
 
@@ -444,5 +455,53 @@ def scl_verify(seed: int, w, bits: int, scales, M: int, K: int, z, proof: bytes)
     det = np.zeros(2, dtype=np.int64)
     tx = L.orc_tx_new(seed)
     rc = L.orc_scl_verify(tx, _ptr(wa), bits, _ptr(sa), M, K, _ptr(za), _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+# ---- SiLU by lookup -----------------------------------------------------------------
+
+def silu_q(v: int) -> int:
+    """The SiLU table's entry for a 16-bit input read with 8 fractional bits (see oracle.c)."""
+    return int(lib().orc_silu_q(int(v)))
+
+
+def _i16(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int16).reshape(-1))
+
+
+def silu_prove(seed: int, g, s):
+    """LogUp proof that every s_i is the SiLU table's entry for g_i. Returns (proof, state after)."""
+    L = lib()
+    a, b = _i16(g), _i16(s)
+    if a.size != b.size or a.size < 1:
+        raise ValueError("silu_prove: g and s need the same length >= 1")
+    out = []
+    for _ in range(2):
+        tx = L.orc_tx_new(seed)
+        n = C.c_uint64(0)
+        buf = np.zeros(max(1, out[0] if out else 1), dtype=np.uint8)
+        rc = L.orc_silu_prove(tx, _ptr(a), _ptr(b), a.size, _ptr(buf) if out else None, out[0] if out else 0,
+                              C.byref(n))
+        st = C.create_string_buffer(32)
+        L.orc_tx_state(tx, st)
+        L.orc_tx_free(tx)
+        if out:
+            if rc != 0:
+                raise ValueError(f"orc_silu_prove failed ({rc})")
+            return buf[: n.value].tobytes(), st.raw
+        if rc not in (0, -2):
+            raise ValueError(f"orc_silu_prove rejected the statement ({rc})")
+        out.append(n.value)
+
+
+def silu_verify(seed: int, g, s, proof: bytes):
+    """Returns (reason_name, detail); 'accept' for a valid proof."""
+    L = lib()
+    a, b = _i16(g), _i16(s)
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_silu_verify(tx, _ptr(a), _ptr(b), a.size, _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

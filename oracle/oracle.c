@@ -37,6 +37,7 @@
  * are repeated next to the code that makes them.
  */
 #include <stdint.h>
+#include <math.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -1486,5 +1487,238 @@ done:
     free(rho);
     free(Sp);
     free(pt);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* SiLU by lookup. The pages prove non-polynomial steps such as the SiLU by  */
+/* committing their outputs and looking them up ("How fast can FlashProve   */
+/* go", 2 Background; 3.1: the gate's values are 16-bit and the SiLU's      */
+/* output is committed). The table is read over the 16-bit domain           */
+/* v in [-2^15, 2^15) as fixed point with 8 fractional bits:                */
+/*   silu_q(v) = floor(v sigma(v / 256) + 1/2) = floor(v / (1 + e^(-v/256)) + 1/2), */
+/* evaluated in double precision (the table is this formula). One LogUp    */
+/* tree over the keys f_i = g_i + gamma s_i, with the steps of the          */
+/* remainder / clamp lookup:                                                 */
+/*   absorb "silu_site" D(g) || D(s) (int16 little-endian);                  */
+/*   squeeze gamma ("silu_gamma"); keys padded to 2^v (v >= 1) with (0, 0);  */
+/*   m_j = #{keys with g = j - 2^15}; send m (2^16 u32, digest absorbed,     */
+/*   "silu_m"); squeeze alpha ("silu_alpha");                                 */
+/*   tree of leaves (1, alpha - f); send layer one p(0), p(1), q(0), q(1)      */
+/*   ("silu_l1"); squeeze mu ("silu_mu");                                     */
+/*   layers d = 1..v-1: squeeze lambda ("silu_lambda"); sum-check of          */
+/*   eq(z, x)(pL qR + pR qL + lambda qL qR), rounds "silu_round" / "silu_chal";*/
+/*   send pL, pR, qL, qR at rho ("silu_final"); squeeze mu; z = (rho, mu);     */
+/*   send g~(z), s~(z) ("silu_leaf").                                          */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_SILU_ROOT = 23,   /* key fraction != table fraction */
+    REJ_SILU_ROUND = 24,  /* layer sum-check round inconsistent */
+    REJ_SILU_FINAL = 25,  /* layer end: eq * F != claim */
+    REJ_SILU_LEAF = 26,   /* leaf numerator != 1 or denominator != alpha - key */
+    REJ_SILU_OPEN = 27    /* g~(z) or s~(z) != the committed column's MLE */
+};
+
+int32_t orc_silu_q(int32_t v) { return (int32_t)floor((double)v / (1.0 + exp(-(double)v / 256.0)) + 0.5); }
+
+static void silu_absorb_site(orc_tx* t, const int16_t* g, const int16_t* s, u64 n) {
+    uint8_t d[64];
+    uint8_t* b = (uint8_t*)calloc(2 * n, 1);
+    for (u64 i = 0; i < n; i++) put_le(b + 2 * i, (u64)(uint16_t)g[i], 2);
+    orc_tree_digest(b, 2 * n, d);
+    for (u64 i = 0; i < n; i++) put_le(b + 2 * i, (u64)(uint16_t)s[i], 2);
+    orc_tree_digest(b, 2 * n, d + 32);
+    free(b);
+    orc_tx_absorb(t, "silu_site", d, 64);
+}
+
+static void silu_mult(const int16_t* g, u64 n, u64 L, u32* m) {
+    memset(m, 0, 65536 * sizeof(u32));
+    for (u64 i = 0; i < L; i++) m[(i < n ? (int64_t)g[i] : 0) + 32768]++;
+}
+
+/* layers[d] has 2^d nodes */
+static void silu_tree(const int16_t* g, const int16_t* s, u64 n, int v, u64 alpha, u64 gamma, u64** Pd, u64** Qd) {
+    u64 L = (u64)1 << v;
+    Pd[v] = (u64*)malloc(L * sizeof(u64));
+    Qd[v] = (u64*)malloc(L * sizeof(u64));
+    for (u64 i = 0; i < L; i++) {
+        u64 f = i < n ? orc_fadd(orc_fint(g[i]), orc_fmul(gamma, orc_fint(s[i]))) : 0;
+        Pd[v][i] = 1;
+        Qd[v][i] = orc_fsub(alpha, f);
+    }
+    for (int d = v - 1; d >= 0; d--) {
+        u64 c = (u64)1 << d;
+        Pd[d] = (u64*)malloc(c * sizeof(u64));
+        Qd[d] = (u64*)malloc(c * sizeof(u64));
+        for (u64 x = 0; x < c; x++) {
+            Pd[d][x] = orc_fadd(orc_fmul(Pd[d + 1][2 * x], Qd[d + 1][2 * x + 1]),
+                                orc_fmul(Pd[d + 1][2 * x + 1], Qd[d + 1][2 * x]));
+            Qd[d][x] = orc_fmul(Qd[d + 1][2 * x], Qd[d + 1][2 * x + 1]);
+        }
+    }
+}
+
+static u64 silu_F(const u64 x[4], u64 lam) { /* pL qR + pR qL + lambda qL qR */
+    return orc_fadd(orc_fadd(orc_fmul(x[0], x[3]), orc_fmul(x[1], x[2])), orc_fmul(lam, orc_fmul(x[2], x[3])));
+}
+
+/* the padded key columns as field elements, and their MLEs at z */
+static void silu_leaf_values(const int16_t* g, const int16_t* s, u64 n, int v, const u64* z, u64 out[2]) {
+    u64 L = (u64)1 << v;
+    u64* col = (u64*)malloc(L * sizeof(u64));
+    for (u64 i = 0; i < L; i++) col[i] = i < n ? orc_fint(g[i]) : 0;
+    out[0] = orc_mle_eval(col, L, z, v);
+    for (u64 i = 0; i < L; i++) col[i] = i < n ? orc_fint(s[i]) : 0;
+    out[1] = orc_mle_eval(col, L, z, v);
+    free(col);
+}
+
+int orc_silu_prove(void* txh, const int16_t* g, const int16_t* s, u64 n, uint8_t* proof, u64 cap, u64* len) {
+    if (n < 1) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n);
+    if (v < 1) v = 1;
+    u64 L = (u64)1 << v;
+    pbuf pb = {proof, cap, 0, 0};
+    silu_absorb_site(t, g, s, n);
+    u64 gamma = orc_tx_squeeze(t, "silu_gamma");
+    u32* m = (u32*)malloc(65536 * sizeof(u32));
+    silu_mult(g, n, L, m);
+    send_mult(t, &pb, "silu_m", m, 65536);
+    u64 alpha = orc_tx_squeeze(t, "silu_alpha");
+    u64** Pd = (u64**)malloc(sizeof(u64*) * (v + 1));
+    u64** Qd = (u64**)malloc(sizeof(u64*) * (v + 1));
+    silu_tree(g, s, n, v, alpha, gamma, Pd, Qd);
+    u64 l1[4] = {Pd[1][0], Pd[1][1], Qd[1][0], Qd[1][1]};
+    send_fe(t, &pb, "silu_l1", l1, 4);
+    u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
+    z[0] = orc_tx_squeeze(t, "silu_mu");
+    for (int d = 1; d < v; d++) {
+        u64 lam = orc_tx_squeeze(t, "silu_lambda");
+        u64 c = (u64)1 << d;
+        u64* V[5]; /* pL, pR, qL, qR (children of layer d), eq(z, .) */
+        for (int i = 0; i < 5; i++) V[i] = (u64*)malloc(c * sizeof(u64));
+        for (u64 x = 0; x < c; x++) {
+            V[0][x] = Pd[d + 1][2 * x];
+            V[1][x] = Pd[d + 1][2 * x + 1];
+            V[2][x] = Qd[d + 1][2 * x];
+            V[3][x] = Qd[d + 1][2 * x + 1];
+        }
+        orc_eq_table(z, d, V[4]);
+        u64* rho = (u64*)malloc(sizeof(u64) * d);
+        u64 Lr = c;
+        for (int r = 0; r < d; r++) {
+            u64 h = Lr >> 1;
+            u64 gr[4] = {0, 0, 0, 0};
+            for (u64 b = 0; b < h; b++)
+                for (u64 X = 0; X < 4; X++) {
+                    u64 ev[5];
+                    for (int i = 0; i < 5; i++) ev[i] = orc_fadd(V[i][b], orc_fmul(X, orc_fsub(V[i][h + b], V[i][b])));
+                    gr[X] = orc_fadd(gr[X], orc_fmul(ev[4], silu_F(ev, lam)));
+                }
+            send_fe(t, &pb, "silu_round", gr, 4);
+            rho[r] = orc_tx_squeeze(t, "silu_chal");
+            for (int i = 0; i < 5; i++)
+                for (u64 b = 0; b < h; b++) V[i][b] = orc_fadd(V[i][b], orc_fmul(rho[r], orc_fsub(V[i][h + b], V[i][b])));
+            Lr = h;
+        }
+        u64 fin[4] = {V[0][0], V[1][0], V[2][0], V[3][0]};
+        send_fe(t, &pb, "silu_final", fin, 4);
+        u64 mu = orc_tx_squeeze(t, "silu_mu");
+        for (int r = 0; r < d; r++) z[r] = rho[r];
+        z[d] = mu;
+        for (int i = 0; i < 5; i++) free(V[i]);
+        free(rho);
+    }
+    u64 leaf[2];
+    silu_leaf_values(g, s, n, v, z, leaf);
+    send_fe(t, &pb, "silu_leaf", leaf, 2);
+    for (int d = 0; d <= v; d++) {
+        free(Pd[d]);
+        free(Qd[d]);
+    }
+    free(Pd);
+    free(Qd);
+    free(z);
+    free(m);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+int orc_silu_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const uint8_t* proof, u64 len,
+                    int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (n < 1) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n), rc = 0;
+    if (v < 1) v = 1;
+    prd rd = {proof, len, 0, 0};
+    u32* m = (u32*)malloc(65536 * sizeof(u32));
+    u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
+    u64* rho = (u64*)malloc(sizeof(u64) * (v + 1));
+    silu_absorb_site(t, g, s, n);
+    u64 gamma = orc_tx_squeeze(t, "silu_gamma");
+    rd_mult(t, &rd, "silu_m", m, 65536);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    u64 alpha = orc_tx_squeeze(t, "silu_alpha");
+    u64 l1[4];
+    rd_fe(t, &rd, "silu_l1", l1, 4);
+    if (rd.bad) FAIL(REJ_FORMAT, 1, 0);
+    {
+        /* the table side, sum_j m_j / (alpha - t_j) with t_j = v_j + gamma silu_q(v_j) */
+        u64 PT = 0, QT = 1;
+        for (u64 j = 0; j < 65536; j++) {
+            int32_t vj = (int32_t)j - 32768;
+            u64 dj = orc_fsub(alpha, orc_fadd(orc_fint(vj), orc_fmul(gamma, orc_fint(orc_silu_q(vj)))));
+            PT = orc_fadd(orc_fmul(PT, dj), orc_fmul((u64)m[j], QT));
+            QT = orc_fmul(QT, dj);
+        }
+        u64 P0 = orc_fadd(orc_fmul(l1[0], l1[3]), orc_fmul(l1[1], l1[2]));
+        u64 Q0 = orc_fmul(l1[2], l1[3]);
+        if (Q0 == 0 || orc_fmul(P0, QT) != orc_fmul(Q0, PT)) FAIL(REJ_SILU_ROOT, 0, 0);
+    }
+    u64 mu = orc_tx_squeeze(t, "silu_mu");
+    u64 cP = orc_fadd(l1[0], orc_fmul(mu, orc_fsub(l1[1], l1[0])));
+    u64 cQ = orc_fadd(l1[2], orc_fmul(mu, orc_fsub(l1[3], l1[2])));
+    z[0] = mu;
+    for (int d = 1; d < v; d++) {
+        u64 lam = orc_tx_squeeze(t, "silu_lambda");
+        u64 claim = orc_fadd(cP, orc_fmul(lam, cQ));
+        for (int r = 0; r < d; r++) {
+            u64 gr[4];
+            rd_fe(t, &rd, "silu_round", gr, 4);
+            if (rd.bad) FAIL(REJ_FORMAT, 2, d);
+            if (orc_fadd(gr[0], gr[1]) != claim) FAIL(REJ_SILU_ROUND, d, r);
+            rho[r] = orc_tx_squeeze(t, "silu_chal");
+            claim = orc_lagrange(gr, 4, rho[r]);
+        }
+        u64 fin[4];
+        rd_fe(t, &rd, "silu_final", fin, 4);
+        if (rd.bad) FAIL(REJ_FORMAT, 3, d);
+        if (orc_fmul(eq_closed(z, rho, d), silu_F(fin, lam)) != claim) FAIL(REJ_SILU_FINAL, d, 0);
+        mu = orc_tx_squeeze(t, "silu_mu");
+        cP = orc_fadd(fin[0], orc_fmul(mu, orc_fsub(fin[1], fin[0])));
+        cQ = orc_fadd(fin[2], orc_fmul(mu, orc_fsub(fin[3], fin[2])));
+        for (int r = 0; r < d; r++) z[r] = rho[r];
+        z[d] = mu;
+    }
+    u64 leaf[2];
+    rd_fe(t, &rd, "silu_leaf", leaf, 2);
+    if (rd.bad) FAIL(REJ_FORMAT, 4, 0);
+    if (cP != 1) FAIL(REJ_SILU_LEAF, 0, 0);
+    if (cQ != orc_fsub(alpha, orc_fadd(leaf[0], orc_fmul(gamma, leaf[1])))) FAIL(REJ_SILU_LEAF, 1, 0);
+    {
+        u64 want[2];
+        silu_leaf_values(g, s, n, v, z, want);
+        if (want[0] != leaf[0]) FAIL(REJ_SILU_OPEN, 0, 0);
+        if (want[1] != leaf[1]) FAIL(REJ_SILU_OPEN, 1, 0);
+    }
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(m);
+    free(z);
+    free(rho);
     return rc;
 }

@@ -436,3 +436,70 @@ def scl_prove(seed: int, w, bits: int, scales, M: int, K: int, z) -> bytes:
     tx.absorb("scl_claim", fe_bytes([a]))
     body, _ = _prod3_rounds(tx, list(z), Se, W, "scl_round", "scl_chal", "scl_final")
     return fe_bytes([a]) + body
+
+
+# ---- SiLU by lookup ----------------------------------------------------------------
+
+def silu_table_entry(v: int) -> int:
+    """floor(v / (1 + e^(-v / 256)) + 1/2) in double precision: the table's definition."""
+    import math
+    return math.floor(v / (1.0 + math.exp(-v / 256.0)) + 0.5)
+
+
+def silu_prove(seed: int, g, s) -> bytes:
+    """The SiLU lookup's proof from definitions: tree layers by their recurrence, every
+    layer round value a hypercube sum of eq times the layer summand over MLEs (no folding)."""
+    g = [int(x) for x in np.asarray(g).reshape(-1)]
+    s = [int(x) for x in np.asarray(s).reshape(-1)]
+    n = len(g)
+    v = max(1, log2c(n))
+    L = 1 << v
+    gp = g + [0] * (L - n)
+    sp = s + [0] * (L - n)
+    out = bytearray()
+
+    def send(label, vals):
+        b = fe_bytes(vals)
+        out.extend(b)
+        tx.absorb(label, b)
+
+    tx = Tx(seed)
+    tx.absorb("silu_site", tree_digest(np.asarray(g, "<i2").tobytes()) + tree_digest(np.asarray(s, "<i2").tobytes()))
+    gamma = tx.squeeze("silu_gamma")
+    m = np.zeros(1 << 16, np.int64)
+    for x in gp:
+        m[x + 32768] += 1
+    b = m.astype("<u4").tobytes()
+    out.extend(b)
+    tx.absorb("silu_m", tree_digest(b))
+    alpha = tx.squeeze("silu_alpha")
+    Pl = [[1] * L]
+    Ql = [[(alpha - (a + gamma * c)) % P for a, c in zip(gp, sp)]]
+    for _ in range(v):
+        p, q_ = Pl[0], Ql[0]
+        Pl.insert(0, [(p[2 * x] * q_[2 * x + 1] + p[2 * x + 1] * q_[2 * x]) % P for x in range(len(p) // 2)])
+        Ql.insert(0, [q_[2 * x] * q_[2 * x + 1] % P for x in range(len(p) // 2)])
+    send("silu_l1", [Pl[1][0], Pl[1][1], Ql[1][0], Ql[1][1]])
+    z = [tx.squeeze("silu_mu")]
+    for d in range(1, v):
+        lam = tx.squeeze("silu_lambda")
+        Pc, Qc = Pl[d + 1], Ql[d + 1]
+        vecs = ([Pc[2 * x] for x in range(1 << d)], [Pc[2 * x + 1] for x in range(1 << d)],
+                [Qc[2 * x] for x in range(1 << d)], [Qc[2 * x + 1] for x in range(1 << d)])
+        rho_l = []
+        for t in range(d):
+            gr = []
+            for X in range(4):
+                acc = 0
+                rest = d - t - 1
+                for bb in range(1 << rest):
+                    pt = rho_l + [X] + [(bb >> (rest - 1 - i)) & 1 for i in range(rest)]
+                    pL, pR, qL, qR = (mle(vv, pt) for vv in vecs)
+                    acc += eq_ml(z, pt) * (pL * qR + pR * qL + lam * qL * qR)
+                gr.append(acc % P)
+            send("silu_round", gr)
+            rho_l.append(tx.squeeze("silu_chal"))
+        send("silu_final", [mle(vv, rho_l) for vv in vecs])
+        z = rho_l + [tx.squeeze("silu_mu")]
+    send("silu_leaf", [mle(gp, z), mle(sp, z)])
+    return bytes(out)
