@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl") -> dict:
+def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,silu") -> dict:
     """Kernel rooflines at HBM scale (inputs well above the 126 MB L2), from a
     profiled pass: every round is its own launch, timed with CUDA events.
 
@@ -188,6 +188,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl") -
       them into field vectors, later rounds read 4 and write 2 values of both
       factors and fold the eq table: 120 B per pair); and the same rounds reducing a
       14336 x 4096 int4 weight matrix with per-64 scales to claims on w and S.
+    silu_round: the SiLU lookup's layer sum-checks over 2^26 keys (one tree; round 1
+      reads the tree layer's children, later rounds fold them: 80 and 160 B per pair).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
@@ -292,7 +294,24 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl") -
         device.weight_digests(ctx, st)
         measure("gkr_round_2^26_keys", "gkr_round", lambda: fp.prove(ctx, 2, st))
         del st, keep
-    torch.cuda.empty_cache()
+    if "silu" in which:
+        # the SiLU lookup of an FFN's gate values: 2^26 16-bit inputs and their table entries
+        try:
+            np_ = __import__("numpy")
+            rng = np_.random.default_rng(11)
+            tab = fp.silu_table().astype(np_.int16)
+            gv = rng.integers(-32768, 32768, 1 << 26).astype(np_.int16)
+            gd = torch.from_numpy(gv).to(dev)
+            sd = torch.from_numpy(tab[gv.astype(np_.int64) + 32768]).to(dev)
+            measure("silu_lookup_round_2^26", "silu_round", lambda: ctx.prove_silu(fp.Transcript(6), gd, sd))
+            del gd, sd
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["silu_lookup_round_2^26"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+
+    try:
+        torch.cuda.empty_cache()
+    except Exception:
+        pass
     return out
 
 
@@ -565,7 +584,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-micro", action="store_true")
-    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm,had,scl", default=None,
+    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm,had,scl,silu", default=None,
                     help="run only the kernel measurements at scale (comma list of sc, pe, gkr, gemm)")
     args = ap.parse_args()
     if args.micro_only:

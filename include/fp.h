@@ -254,6 +254,35 @@ int sumcheck_reduce_scales(fp_ctx* ctx, fp_tx* tx, const void* w, int w_bits, co
                            const uint64_t* point, uint8_t* proof, size_t* proof_len, void* stream);
 
 /*
+ * SiLU by lookup ("How fast can FlashProve go", 2 Background and 3.1: the SiLU is
+ * not a polynomial, so its committed 16-bit outputs are proven by a lookup). The
+ * table reads a 16-bit input v with 8 fractional bits and stores
+ * silu_q(v) = floor(v / (1 + e^(-v/256)) + 1/2), evaluated in double precision.
+ * g, s: device int16 columns of n entries (the SiLU's inputs and its claimed
+ * outputs), caller-owned, read only. One LogUp-GKR tree over the keys
+ * f = g + gamma s; the call continues tx:
+ *   absorb "silu_site" D(g) || D(s) (int16 little-endian); squeeze gamma
+ *   ("silu_gamma"); keys padded to 2^v (v = max(1, ceil(log2 n))) with (0, 0);
+ *   send m_j = #{keys with g = j - 2^15} (2^16 u32; "silu_m" absorbs their
+ *   digest); squeeze alpha ("silu_alpha"); send layer one p(0), p(1), q(0),
+ *   q(1) ("silu_l1"); squeeze mu ("silu_mu"); for d = 1..v-1: squeeze lambda
+ *   ("silu_lambda"), d rounds of g(0..3) ("silu_round") and challenges
+ *   ("silu_chal") of the sum-check of eq(z, x)(pL qR + pR qL + lambda qL qR),
+ *   the children pL, pR, qL, qR at rho ("silu_final"), squeeze mu; then
+ *   g~(z), s~(z) ("silu_leaf").
+ * Proof bytes: 4 * 2^16 + 32 + sum_{d=1}^{v-1} (32 d + 32) + 16. The verifier
+ * checks the root against sum_j m_j / (alpha - v_j - gamma silu_q(v_j)), every
+ * layer, and the leaf against alpha - (g~ + gamma s~). 1 <= n <= 2^30, else
+ * FP_ERR_SHAPE; null arguments FP_ERR_ARG; proof / proof_len as for
+ * sumcheck_prove_matmul.
+ */
+int logup_prove_silu(fp_ctx* ctx, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
+                     size_t* proof_len, void* stream);
+
+/* The SiLU table's 2^16 entries silu_q(v), v = -2^15 .. 2^15 - 1, into host out (no GPU work). */
+int fp_silu_table(int32_t* out);
+
+/*
  * Self-test of the bounded device waits. The sum-check kernels stay resident
  * across rounds and wait (a bounded number of polls) for each Fiat-Shamir
  * challenge from the host. This call launches a kernel that waits for a

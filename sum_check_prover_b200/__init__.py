@@ -75,6 +75,8 @@ def lib():
     L.logup_prove_rescale.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
     L.sumcheck_prove_hadamard.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, C.POINTER(sz), vp]
+    L.logup_prove_silu.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
+    L.fp_silu_table.argtypes = [vp]
     L.fp_proof_size.argtypes = [C.POINTER(_Site), i32, C.POINTER(sz), C.POINTER(sz)]
     L.fp_ctx_set_profiling.argtypes = [vp, i32]
     L.fp_session_selftest.argtypes = [vp, vp]
@@ -270,6 +272,23 @@ class Context:
                                                    C.byref(ln), _stream(stream)), "sumcheck_reduce_scales")
         return buf.raw[: ln.value]
 
+    def prove_silu(self, tx: Transcript, g, s, stream=None) -> bytes:
+        """LogUp proof that every entry of the device int16 tensor s is the SiLU table's entry
+        for the same entry of g (flattened row-major); continues tx."""
+        n = int(g.numel())
+        if int(s.numel()) != n:
+            raise ValueError("prove_silu: g and s differ in size")
+        v = 0
+        while (1 << v) < n:
+            v += 1
+        v = max(v, 1)
+        cap = 4 * 65536 + 32 + 16 + sum(32 * d + 32 for d in range(1, v))
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        self._check(self._L.logup_prove_silu(self.h, tx.h, _ptr(g), _ptr(s), n, buf, C.byref(ln),
+                                             _stream(stream)), "logup_prove_silu")
+        return buf.raw[: ln.value]
+
     def prove_logup(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
         """Returns (proof bytes, status): status 1 means some key lies outside its table."""
         arr, keep = _sites(sites)
@@ -336,3 +355,13 @@ def prove(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], stream=
         return mm + lu, [s0, s1, tx.state()], status
     finally:
         tx.close()
+
+
+def silu_table():
+    """The SiLU table's 2^16 entries (inputs -2^15 .. 2^15 - 1), as the library computes them."""
+    import numpy as np
+    out = np.zeros(65536, dtype=np.int32)
+    rc = lib().fp_silu_table(out.ctypes.data)
+    if rc != 0:
+        raise FpError(rc, "fp_silu_table")
+    return out

@@ -35,6 +35,10 @@ enum FpKernel {
     K_HAD_CLAIM,
     K_HAD_ROUND,
     K_HAD_FINAL,
+    K_SILU_HIST,
+    K_SILU_TREE,
+    K_SILU_ROUND,
+    K_SILU_LEAF,
     K_COUNT
 };
 

@@ -1,0 +1,461 @@
+// SiLU by lookup: one LogUp-GKR fraction tree over the keys f = g + gamma s.
+//
+// "How fast can FlashProve go", 2 Background and 3.1: the SiLU is not a
+// polynomial, so its 16-bit outputs are committed and proven by a lookup. The
+// table reads a 16-bit input v with 8 fractional bits and stores
+// silu_q(v) = floor(v / (1 + e^(-v/256)) + 1/2) (evaluated in double precision on
+// the host, where the verifier evaluates it too). The statement:
+//   absorb "silu_site" D(g) || D(s) (int16 little-endian); squeeze gamma;
+//   keys padded to 2^v (v >= 1) with (0, 0); m_j = #{keys with g = j - 2^15};
+//   send m (2^16 u32, its digest absorbed as "silu_m"); squeeze alpha;
+//   the fraction tree of leaves (1, alpha - f): send layer one ("silu_l1"),
+//   squeeze mu; layers d = 1..v-1: squeeze lambda, sum-check of
+//   eq(z, x)(pL qR + pR qL + lambda qL qR) over d variables ("silu_round" /
+//   "silu_chal"), send the four child values at rho ("silu_final"), squeeze
+//   mu, z = (rho, mu); send g~(z), s~(z) ("silu_leaf").
+// A layer's round values come as in the product sum-checks: the device returns
+// h(0), h(1), h(2) of h(X) = sum_b eq(z_>t, b) F(X, b) (F has degree 2) and the
+// host multiplies in eq(z_<t, rho_<t) eq(z_t, X), checking g(0) + g(1) against
+// the running claim.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "fp_eqchunks.cuh"
+#include "fp_internal.h"
+#include "fp_reduce.cuh"
+#include "fp_session.cuh"
+
+namespace {
+
+constexpr int SL_THREADS = 256;
+constexpr int SL_MAX_V = 30;
+
+__device__ __forceinline__ uint64_t lift_i(int64_t x) { return x < 0 ? GL_P - (uint64_t)(-x) : (uint64_t)x; }
+
+// m[g + 2^15] += 1 for every entry of g (the padding keys are counted by the host)
+__global__ void silu_hist_kernel(const int16_t* __restrict__ g, int64_t n, uint32_t* __restrict__ m) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        atomicAdd(m + ((int)g[i] + 32768), 1u);
+}
+
+__global__ void silu_add_pad_kernel(uint32_t* m, uint32_t pad) { m[32768] += pad; }
+
+// leaves: P = 1, Q = alpha - (g + gamma s) (zero keys past n)
+__global__ void silu_leaf_kernel(const int16_t* __restrict__ g, const int16_t* __restrict__ s, int64_t n, int64_t L,
+                                 uint64_t alpha, uint64_t gamma, uint64_t* __restrict__ P, uint64_t* __restrict__ Q) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < L; i += (int64_t)gridDim.x * blockDim.x) {
+        uint64_t f = 0;
+        if (i < n) f = gl_add(lift_i(g[i]), gl_mul(gamma, lift_i(s[i])));
+        P[i] = 1;
+        Q[i] = gl_sub(alpha, f);
+    }
+}
+
+// one level up: P'[x] = P[2x] Q[2x+1] + P[2x+1] Q[2x], Q'[x] = Q[2x] Q[2x+1], x < c
+__global__ void silu_level_kernel(const uint64_t* __restrict__ P, const uint64_t* __restrict__ Q, int64_t c,
+                                  uint64_t* __restrict__ Po, uint64_t* __restrict__ Qo) {
+    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < c; x += (int64_t)gridDim.x * blockDim.x) {
+        const uint64_t pl = P[2 * x], pr = P[2 * x + 1], ql = Q[2 * x], qr = Q[2 * x + 1];
+        Po[x] = gl_add(gl_mul(pl, qr), gl_mul(pr, ql));
+        Qo[x] = gl_mul(ql, qr);
+    }
+}
+
+// sum_{x < L} eq(z, x) a(x) for an int16 column a of n entries (zero past n), eq split as
+// EH[x >> vl] EL[x & (2^vl - 1)]
+__global__ void __launch_bounds__(256) silu_mle_kernel(const int16_t* __restrict__ a, int64_t n,
+                                                       const uint64_t* __restrict__ EH, const uint64_t* __restrict__ EL,
+                                                       int vl, uint64_t* part, unsigned int* ticket, uint64_t* out) {
+    GlAcc acc;
+    const int64_t mask = (1ll << vl) - 1;
+    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
+        const int v = a[x];
+        if (v == 0) continue;
+        acc.mac(gl_mul(__ldg(EH + (x >> vl)), __ldg(EL + (x & mask))), lift_i(v));
+    }
+    uint64_t v[1] = {acc.value()};
+    if (grid_sum_gl<1>(v, part, ticket) && threadIdx.x == 0) *out = v[0];
+}
+
+struct LayerArgs {
+    const uint64_t* P;  // tree layer d + 1 (2^(d+1) entries): child x of node b is entry 2 b + x
+    const uint64_t* Q;
+    uint64_t* pl;       // folded children from round 2 on (2^(d-1) entries each)
+    uint64_t* pr;
+    uint64_t* ql;
+    uint64_t* qr;
+    uint64_t* E;        // suffix eq table (2^(d-1) entries)
+    const uint64_t* z;  // device copy of the layer's point z_1..z_d
+    uint64_t lam;
+    int d;
+    int grid;
+    int per_block;
+    int pad;
+    uint64_t seq0;  // round t publishes seq0 + t, the final values seq0 + d + 1
+    int t_begin;    // rounds run by this launch: [t_begin, t_end]; t_end > d includes the final values
+    int t_end;
+};
+
+__device__ __forceinline__ uint64_t at2(uint64_t a, uint64_t b) { return gl_sub(gl_add(b, b), a); }
+
+// pL qR + pR qL + lambda qL qR
+__device__ __forceinline__ uint64_t layer_f(uint64_t a, uint64_t b, uint64_t c, uint64_t e, uint64_t lam) {
+    return gl_add(gl_add(gl_mul(a, e), gl_mul(b, c)), gl_mul(lam, gl_mul(c, e)));
+}
+
+__global__ void __launch_bounds__(SL_THREADS, 2) silu_layer_kernel(LayerArgs A, FpMailbox* mb, FpRelay* rl,
+                                                                  uint64_t* part) {
+    __shared__ uint64_t zs[32];
+    __shared__ uint64_t eq_tab[3 << kEqChunk];
+    if (threadIdx.x < A.d) zs[threadIdx.x] = A.z[threadIdx.x];
+    __syncthreads();
+    uint64_t rprev = 0;
+    for (int t = A.t_begin; t <= A.d && t <= A.t_end; t++) {
+        if (t > 1 && !session_wait(mb, rl, A.seq0 + t - 1, rprev)) return;
+        const int64_t h = 1ll << (A.d - t);
+        const int64_t want = (h + A.per_block - 1) / A.per_block;
+        const unsigned active = (unsigned)(want < 1 ? 1 : (want > A.grid ? A.grid : want));
+        if (blockIdx.x >= active) return;  // no pairs for this block in this or any later round
+        EqChunks EC{0, 0, 0};
+        if (t == 1) EC = eq_chunks_build(eq_tab, zs, A.d);
+        GlAcc a0, a1, a2;
+        for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
+            uint64_t p0, p1, r0, r1, q0, q1, s0, s1, e;  // pL, pR, qL, qR at the pair's two points
+            if (t == 1) {
+                p0 = A.P[2 * b];
+                r0 = A.P[2 * b + 1];
+                q0 = A.Q[2 * b];
+                s0 = A.Q[2 * b + 1];
+                p1 = A.P[2 * (b + h)];
+                r1 = A.P[2 * (b + h) + 1];
+                q1 = A.Q[2 * (b + h)];
+                s1 = A.Q[2 * (b + h) + 1];
+                e = eq_chunks_at(EC, eq_tab, b);  // eq(z_2..z_d, b)
+                if (A.d > 1) A.E[b] = e;
+            } else {
+                if (t == 2) {
+                    // the children vectors (length 4h, read from the tree layer) folded by rho_1
+                    p0 = gl_fold_fast(A.P[2 * b], A.P[2 * (b + 2 * h)], rprev);
+                    r0 = gl_fold_fast(A.P[2 * b + 1], A.P[2 * (b + 2 * h) + 1], rprev);
+                    q0 = gl_fold_fast(A.Q[2 * b], A.Q[2 * (b + 2 * h)], rprev);
+                    s0 = gl_fold_fast(A.Q[2 * b + 1], A.Q[2 * (b + 2 * h) + 1], rprev);
+                    p1 = gl_fold_fast(A.P[2 * (b + h)], A.P[2 * (b + 3 * h)], rprev);
+                    r1 = gl_fold_fast(A.P[2 * (b + h) + 1], A.P[2 * (b + 3 * h) + 1], rprev);
+                    q1 = gl_fold_fast(A.Q[2 * (b + h)], A.Q[2 * (b + 3 * h)], rprev);
+                    s1 = gl_fold_fast(A.Q[2 * (b + h) + 1], A.Q[2 * (b + 3 * h) + 1], rprev);
+                } else {
+                    p0 = gl_fold_fast(__ldcg(A.pl + b), __ldcg(A.pl + b + 2 * h), rprev);
+                    r0 = gl_fold_fast(__ldcg(A.pr + b), __ldcg(A.pr + b + 2 * h), rprev);
+                    q0 = gl_fold_fast(__ldcg(A.ql + b), __ldcg(A.ql + b + 2 * h), rprev);
+                    s0 = gl_fold_fast(__ldcg(A.qr + b), __ldcg(A.qr + b + 2 * h), rprev);
+                    p1 = gl_fold_fast(__ldcg(A.pl + b + h), __ldcg(A.pl + b + 3 * h), rprev);
+                    r1 = gl_fold_fast(__ldcg(A.pr + b + h), __ldcg(A.pr + b + 3 * h), rprev);
+                    q1 = gl_fold_fast(__ldcg(A.ql + b + h), __ldcg(A.ql + b + 3 * h), rprev);
+                    s1 = gl_fold_fast(__ldcg(A.qr + b + h), __ldcg(A.qr + b + 3 * h), rprev);
+                }
+                A.pl[b] = p0;
+                A.pr[b] = r0;
+                A.ql[b] = q0;
+                A.qr[b] = s0;
+                A.pl[b + h] = p1;
+                A.pr[b + h] = r1;
+                A.ql[b + h] = q1;
+                A.qr[b + h] = s1;
+                e = gl_add(__ldcg(A.E + b), __ldcg(A.E + b + h));  // eq(z_>t, b)
+                A.E[b] = e;
+            }
+            a0.mac(e, layer_f(p0, r0, q0, s0, A.lam));
+            a1.mac(e, layer_f(p1, r1, q1, s1, A.lam));
+            a2.mac(e, layer_f(at2(p0, p1), at2(r0, r1), at2(q0, q1), at2(s0, s1), A.lam));
+        }
+        uint64_t acc[3] = {a0.value(), a1.value(), a2.value()};
+        bool last;
+        if (active == 1) {
+            block_sum_gl<3>(acc);
+            last = true;
+        } else {
+            last = grid_sum_gl_n<3>(acc, part, &rl->ticket, active);
+        }
+        if (last && threadIdx.x == 0) session_publish(mb, acc, A.seq0 + t);  // {h(0), h(1), h(2)}
+    }
+    // block 0 folds the last pair of each vector by the last challenge: pL, pR, qL, qR at rho
+    if (A.t_end <= A.d || blockIdx.x != 0) return;
+    if (!session_wait(mb, rl, A.seq0 + A.d, rprev)) return;
+    if (threadIdx.x == 0) {
+        uint64_t fin[4];
+        if (A.d == 1) {
+            fin[0] = gl_fold_fast(A.P[0], A.P[2], rprev);
+            fin[1] = gl_fold_fast(A.P[1], A.P[3], rprev);
+            fin[2] = gl_fold_fast(A.Q[0], A.Q[2], rprev);
+            fin[3] = gl_fold_fast(A.Q[1], A.Q[3], rprev);
+        } else {
+            fin[0] = gl_fold_fast(__ldcg(A.pl), __ldcg(A.pl + 1), rprev);
+            fin[1] = gl_fold_fast(__ldcg(A.pr), __ldcg(A.pr + 1), rprev);
+            fin[2] = gl_fold_fast(__ldcg(A.ql), __ldcg(A.ql + 1), rprev);
+            fin[3] = gl_fold_fast(__ldcg(A.qr), __ldcg(A.qr + 1), rprev);
+        }
+        session_publish(mb, fin, A.seq0 + A.d + 1);
+    }
+}
+
+int64_t silu_q_host(int64_t v) { return (int64_t)floor((double)v / (1.0 + exp(-(double)v / 256.0)) + 0.5); }
+
+// the degree-3 polynomial through (i, g[i]), i = 0..3, at r
+uint64_t lagrange4(const uint64_t g[4], uint64_t r) {
+    static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
+    const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2), r3 = gl_sub(r, 3);
+    const uint64_t l0 = gl_sub(0, gl_mul(gl_mul(gl_mul(r1, r2), r3), inv6));
+    const uint64_t l1 = gl_mul(gl_mul(gl_mul(r, r2), r3), inv2);
+    const uint64_t l2 = gl_sub(0, gl_mul(gl_mul(gl_mul(r, r1), r3), inv2));
+    const uint64_t l3 = gl_mul(gl_mul(gl_mul(r, r1), r2), inv6);
+    return gl_add(gl_add(gl_mul(g[0], l0), gl_mul(g[1], l1)), gl_add(gl_mul(g[2], l2), gl_mul(g[3], l3)));
+}
+
+unsigned grid_of(const fp_ctx* c, int64_t work) {
+    return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
+}
+
+// m (2^16 u32), layer one (4), per layer d = 1..v-1 its d rounds (4 each) and 4 final values, 2 leaf values
+size_t silu_proof_len(int64_t n) {
+    int v = fp_log2_ceil((uint64_t)n);
+    if (v < 1) v = 1;
+    size_t len = 4 * 65536 + 32 + 16;
+    for (int d = 1; d < v; d++) len += 32 * (size_t)d + 32;
+    return len;
+}
+
+}  // namespace
+
+int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
+                     size_t* proof_len, void* stream) {
+    if (!c || !tx || !proof_len) return fp_fail(c, FP_ERR_ARG, "logup_prove_silu: null argument");
+    if (!g || !s) return fp_fail(c, FP_ERR_ARG, "logup_prove_silu: null column");
+    if (n < 1 || n > (1ll << SL_MAX_V)) return fp_fail(c, FP_ERR_SHAPE, "logup_prove_silu: need 1 <= n <= 2^30");
+    const size_t need_len = silu_proof_len(n);
+    if (!proof || *proof_len < need_len) {
+        *proof_len = need_len;
+        return fp_fail(c, FP_ERR_ARG, "logup_prove_silu: proof buffer too small");
+    }
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t st = (cudaStream_t)stream;
+    int rc;
+    int v = fp_log2_ceil((uint64_t)n);
+    if (v < 1) v = 1;
+    const int64_t L = 1ll << v;
+
+    // ---- commit ----
+    {
+        FpDigestJob jobs[2] = {{(const uint8_t*)g, 2 * (uint64_t)n}, {(const uint8_t*)s, 2 * (uint64_t)n}};
+        uint8_t d[64];
+        if ((rc = fp_digest_many(c, jobs, 2, d, st))) return rc;  // synchronises the stream
+        fp_tx_absorb_raw(tx, "silu_site", d, 64);
+    }
+    const uint64_t gamma = fp_tx_squeeze_one(tx, "silu_gamma");
+
+    // ---- scratch: multiplicities, tree layers 1..v, layer vectors, eq tables, reductions ----
+    int occ = 0;
+    FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, silu_layer_kernel, SL_THREADS, 0));
+    const int cap_grid = std::max(1, occ) * c->num_sms;
+    const size_t part_n = (size_t)3 * std::max(cap_grid, 4 * c->num_sms);
+    const int64_t hv = v >= 2 ? 1ll << (v - 2) : 1;  // the largest layer's vectors: 2^(d-1) for d = v - 1
+    const int vl = v / 2, vh = v - vl;
+    size_t need = fp_align_up(4 * 65536, 256) + fp_align_up(8 * part_n, 256) + fp_align_up(8 * 64, 256) +
+                  fp_align_up((size_t)8 << vh, 256) + fp_align_up((size_t)8 << vl, 256) +
+                  5 * fp_align_up((size_t)8 * hv, 256) + 4096;
+    for (int d = 1; d <= v; d++) need += 2 * fp_align_up((size_t)8 << d, 256);
+    if ((rc = fp_reserve(c, c->dev, need))) return rc;
+    if ((rc = fp_reserve(c, c->host, 4 * 65536 + 8192))) return rc;
+    fp_reset(c->dev);
+    fp_reset(c->host);
+    uint32_t* m = (uint32_t*)fp_alloc(c->dev, 4 * 65536);
+    uint64_t* part = (uint64_t*)fp_alloc(c->dev, 8 * part_n);
+    uint64_t* small = (uint64_t*)fp_alloc(c->dev, 8 * 64);  // [0..1] leaf values, [8..] the layer's point
+    uint64_t* EH = (uint64_t*)fp_alloc(c->dev, (size_t)8 << vh);
+    uint64_t* EL = (uint64_t*)fp_alloc(c->dev, (size_t)8 << vl);
+    uint64_t* vecs[5];
+    for (int i = 0; i < 5; i++) vecs[i] = (uint64_t*)fp_alloc(c->dev, (size_t)8 * hv);
+    std::vector<uint64_t*> TP(v + 1, nullptr), TQ(v + 1, nullptr);
+    for (int d = 1; d <= v; d++) {
+        TP[d] = (uint64_t*)fp_alloc(c->dev, (size_t)8 << d);
+        TQ[d] = (uint64_t*)fp_alloc(c->dev, (size_t)8 << d);
+        if (!TP[d] || !TQ[d]) return fp_fail(c, FP_ERR_OOM, "logup_prove_silu: scratch exhausted");
+    }
+    uint8_t* hm = (uint8_t*)fp_alloc(c->host, 4 * 65536);
+    uint64_t* hs = (uint64_t*)fp_alloc(c->host, 8 * 64);
+    if (!m || !part || !small || !EH || !EL || !vecs[4] || !hm || !hs)
+        return fp_fail(c, FP_ERR_OOM, "logup_prove_silu: scratch exhausted");
+
+    // ---- multiplicities ----
+    FP_CUDA(c, cudaMemsetAsync(m, 0, 4 * 65536, st));
+    {
+        int slot;
+        fp_tic(c, st, K_SILU_HIST, 2.0 * (double)n, &slot);
+        silu_hist_kernel<<<grid_of(c, n), 256, 0, st>>>(g, n, m);
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+        if (L > n) silu_add_pad_kernel<<<1, 1, 0, st>>>(m, (uint32_t)(L - n));
+        FP_CUDA(c, cudaGetLastError());
+    }
+    FP_CUDA(c, cudaMemcpyAsync(hm, m, 4 * 65536, cudaMemcpyDeviceToHost, st));
+    uint8_t dm[32];
+    {
+        FpDigestJob job = {(const uint8_t*)m, 4 * 65536ull};
+        if ((rc = fp_digest_many(c, &job, 1, dm, st))) return rc;  // synchronises the stream
+    }
+    size_t pos = 0;
+    memcpy(proof + pos, hm, 4 * 65536);  // device words are little-endian u32
+    pos += 4 * 65536;
+    fp_tx_absorb_raw(tx, "silu_m", dm, 32);
+    const uint64_t alpha = fp_tx_squeeze_one(tx, "silu_alpha");
+
+    // ---- the fraction tree, layers v (leaves) .. 1 ----
+    {
+        int slot;
+        fp_tic(c, st, K_SILU_TREE, 4.0 * (double)n + 32.0 * (double)L, &slot);
+        silu_leaf_kernel<<<grid_of(c, L), 256, 0, st>>>(g, s, n, L, alpha, gamma, TP[v], TQ[v]);
+        FP_CUDA(c, cudaGetLastError());
+        for (int d = v - 1; d >= 1; d--) {
+            silu_level_kernel<<<grid_of(c, 1ll << d), 256, 0, st>>>(TP[d + 1], TQ[d + 1], 1ll << d, TP[d], TQ[d]);
+            FP_CUDA(c, cudaGetLastError());
+        }
+        fp_toc(c, st, slot);
+    }
+    FP_CUDA(c, cudaMemcpyAsync(hs, TP[1], 16, cudaMemcpyDeviceToHost, st));
+    FP_CUDA(c, cudaMemcpyAsync(hs + 2, TQ[1], 16, cudaMemcpyDeviceToHost, st));
+    FP_CUDA(c, cudaStreamSynchronize(st));
+    uint64_t l1[4] = {hs[0], hs[1], hs[2], hs[3]};
+    put_u64s(proof + pos, l1, 4);
+    fp_tx_absorb_raw(tx, "silu_l1", proof + pos, 32);
+    pos += 32;
+    FpPoint z;
+    z.v = 1;
+    z.z[0] = fp_tx_squeeze_one(tx, "silu_mu");
+    uint64_t cP = gl_fold(l1[0], l1[1], z.z[0]), cQ = gl_fold(l1[2], l1[3], z.z[0]);
+
+    // ---- layer sum-checks d = 1 .. v - 1 ----
+    for (int d = 1; d < v; d++) {
+        const uint64_t lam = fp_tx_squeeze_one(tx, "silu_lambda");
+        uint64_t claim = gl_add(cP, gl_mul(lam, cQ));
+        for (int i = 0; i < d; i++) hs[8 + i] = z.z[i];
+        FP_CUDA(c, cudaMemcpyAsync(small + 8, hs + 8, 8 * (size_t)d, cudaMemcpyHostToDevice, st));
+        LayerArgs A;
+        memset(&A, 0, sizeof A);
+        A.P = TP[d + 1];
+        A.Q = TQ[d + 1];
+        A.pl = vecs[0];
+        A.pr = vecs[1];
+        A.ql = vecs[2];
+        A.qr = vecs[3];
+        A.E = vecs[4];
+        A.z = small + 8;
+        A.lam = lam;
+        A.d = d;
+        A.per_block = SL_THREADS;  // one pair per thread
+        const int64_t half = 1ll << (d - 1);
+        A.grid = (int)std::max<int64_t>(1, std::min<int64_t>((half + A.per_block - 1) / A.per_block, cap_grid));
+        A.seq0 = fp_seq_reserve(c, (uint64_t)d + 2);
+        if ((rc = fp_session_begin(c, st))) return rc;
+        fp_session_expect(c, 3);  // before any launch: round 1 publishes without a challenge
+        void* args[] = {&A, &c->mb_dev, &c->relay, &part};
+        auto round_bytes = [&](int t) { return 80.0 * (double)(1ll << (d - t)) * (t == 1 ? 1.0 : 2.0); };
+        if (!c->stepped) {
+            A.t_begin = 1;
+            A.t_end = d + 1;
+            double bytes = 0;
+            for (int t = 1; t <= d; t++) bytes += round_bytes(t);
+            int slot;
+            fp_tic(c, st, K_SILU_ROUND, bytes, &slot);
+            FP_CUDA(c, cudaLaunchCooperativeKernel((const void*)silu_layer_kernel, dim3(A.grid), dim3(SL_THREADS),
+                                                   args, 0, st));
+            fp_toc(c, st, slot);
+        }
+        uint64_t pre = 1;  // eq(z_<t, rho_<t)
+        std::vector<uint64_t> rho(d);
+        for (int t = 1; t <= d; t++) {
+            if (c->stepped) {
+                A.t_begin = A.t_end = t;
+                int slot;
+                fp_tic(c, st, K_SILU_ROUND, round_bytes(t), &slot);
+                FP_CUDA(c, cudaLaunchCooperativeKernel((const void*)silu_layer_kernel, dim3(A.grid),
+                                                       dim3(SL_THREADS), args, 0, st));
+                fp_toc(c, st, slot);
+            }
+            if ((rc = fp_session_wait(c, A.seq0 + t, st))) return rc;
+            const uint64_t h0 = c->mb->res[0], h1 = c->mb->res[1], h2 = c->mb->res[2];
+            const uint64_t zt = z.z[t - 1];
+            const uint64_t h3 = gl_add(gl_sub(h0, gl_mul(3, h1)), gl_mul(3, h2));
+            uint64_t gr[4];
+            gr[0] = gl_mul(pre, gl_mul(gl_sub(1, zt), h0));
+            gr[1] = gl_mul(pre, gl_mul(zt, h1));
+            gr[2] = gl_mul(pre, gl_mul(gl_sub(gl_mul(3, zt), 1), h2));
+            gr[3] = gl_mul(pre, gl_mul(gl_sub(gl_mul(5, zt), 2), h3));
+            if (gl_add(gr[0], gr[1]) != claim)
+                return fp_fail(c, FP_ERR_CUDA, "logup_prove_silu: round values inconsistent with the claim");
+            put_u64s(proof + pos, gr, 4);
+            fp_tx_absorb_raw(tx, "silu_round", proof + pos, 32);
+            pos += 32;
+            fp_session_expect(c, t < d ? 3 : 4);  // the last challenge triggers the four final values
+            const uint64_t r = fp_tx_squeeze_one(tx, "silu_chal");
+            fp_session_post(c, A.seq0 + t, r);
+            rho[t - 1] = r;
+            claim = lagrange4(gr, r);
+            pre = gl_mul(pre, gl_add(gl_mul(zt, r), gl_mul(gl_sub(1, zt), gl_sub(1, r))));
+        }
+        if (c->stepped) {
+            A.t_begin = A.t_end = d + 1;
+            int slot;
+            fp_tic(c, st, K_SILU_ROUND, 64.0, &slot);
+            FP_CUDA(c, cudaLaunchCooperativeKernel((const void*)silu_layer_kernel, dim3(1), dim3(SL_THREADS), args, 0,
+                                                   st));
+            fp_toc(c, st, slot);
+        }
+        if ((rc = fp_session_wait(c, A.seq0 + d + 1, st))) return rc;
+        uint64_t fin[4] = {c->mb->res[0], c->mb->res[1], c->mb->res[2], c->mb->res[3]};
+        FP_CUDA(c, cudaStreamSynchronize(st));
+        put_u64s(proof + pos, fin, 4);
+        fp_tx_absorb_raw(tx, "silu_final", proof + pos, 32);
+        pos += 32;
+        const uint64_t mu = fp_tx_squeeze_one(tx, "silu_mu");
+        cP = gl_fold(fin[0], fin[1], mu);
+        cQ = gl_fold(fin[2], fin[3], mu);
+        for (int i = 0; i < d; i++) z.z[i] = rho[i];
+        z.z[d] = mu;
+        z.v = d + 1;
+    }
+
+    // ---- leaf claims: g~(z), s~(z) over the padded columns ----
+    {
+        FpPoint zh, zl;
+        zh.v = vh;
+        zl.v = vl;
+        for (int i = 0; i < vh; i++) zh.z[i] = z.z[i];
+        for (int i = 0; i < vl; i++) zl.z[i] = z.z[vh + i];
+        if ((rc = fp_eq_table(c, zh, EH, st))) return rc;
+        if ((rc = fp_eq_table(c, zl, EL, st))) return rc;
+        const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 2 * (int64_t)c->num_sms));
+        int slot;
+        fp_tic(c, st, K_SILU_LEAF, 4.0 * (double)n, &slot);
+        silu_mle_kernel<<<blocks, 256, 0, st>>>(g, n, EH, EL, vl, part, c->tickets, small);
+        FP_CUDA(c, cudaGetLastError());
+        silu_mle_kernel<<<blocks, 256, 0, st>>>(s, n, EH, EL, vl, part, c->tickets, small + 1);
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+        FP_CUDA(c, cudaMemcpyAsync(hs, small, 16, cudaMemcpyDeviceToHost, st));
+        FP_CUDA(c, cudaStreamSynchronize(st));
+    }
+    const uint64_t leaf[2] = {hs[0], hs[1]};
+    put_u64s(proof + pos, leaf, 2);
+    fp_tx_absorb_raw(tx, "silu_leaf", proof + pos, 16);
+    pos += 16;
+    *proof_len = pos;
+    return FP_OK;
+}
+
+int fp_silu_table(int32_t* out) {
+    if (!out) return FP_ERR_ARG;
+    for (int64_t v = -32768; v < 32768; v++) out[v + 32768] = (int32_t)silu_q_host(v);
+    return FP_OK;
+}

@@ -99,3 +99,12 @@ def test_portable_sha_path_matches_oracle(L):
     env = dict(os.environ, FP_NO_SHANI="1")
     r = subprocess.run([sys.executable, "-c", code], cwd=str(ROOT), env=env, capture_output=True, text=True)
     assert r.returncode == 0 and "ok" in r.stdout, r.stderr
+
+
+def test_silu_table_matches_oracle(L):
+    # the library's table (host C++) and the oracle's (plain C), each from the formula
+    import numpy as np
+    import sum_check_prover_b200 as fp
+    lib_t = fp.silu_table()
+    ora_t = np.array([oracle.silu_q(v) for v in range(-32768, 32768)], dtype=np.int32)
+    assert np.array_equal(lib_t, ora_t)

@@ -1,0 +1,85 @@
+"""GPU parity of the SiLU lookup through the C ABI.
+
+"How fast can FlashProve go", 2 Background and 3.1: the SiLU's committed
+outputs are proven by a lookup into a 2^16-entry table. The CUDA path (one
+LogUp-GKR tree, resident layer sum-checks with host-assembled round values)
+must give the oracle's proof bytes and transcript state for honest and
+dishonest outputs alike (the oracle's verifier then accepts only the honest
+ones), on ragged sizes, and the same proof in stepped and resident modes.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+
+pytestmark = pytest.mark.gpu
+TABLE = None
+
+
+def table():
+    global TABLE
+    if TABLE is None:
+        TABLE = np.array([oracle.silu_q(v) for v in range(-32768, 32768)], dtype=np.int16)
+    return TABLE
+
+
+@pytest.fixture(scope="module")
+def lib_env():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sum_check_prover_b200 import build
+    build.build()
+    import sum_check_prover_b200 as fp
+    return torch, fp
+
+
+@pytest.fixture
+def env(lib_env):
+    torch, fp = lib_env
+    ctx = fp.Context(0)
+    yield torch, fp, ctx
+    ctx.close()
+
+
+def _cols(n, seed, lo=-32768, hi=32768):
+    rng = np.random.default_rng(seed)
+    g = rng.integers(lo, hi, n).astype(np.int16)
+    return g, table()[g.astype(np.int64) + 32768]
+
+
+def _gpu(env, seed, g, s):
+    torch, fp, ctx = env
+    tx = fp.Transcript(seed)
+    pf = ctx.prove_silu(tx, torch.from_numpy(g).cuda(), torch.from_numpy(s).cuda())
+    torch.cuda.synchronize()
+    return pf, tx.state()
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 8, 13, 300, 1000, 4097, 65537])
+def test_matches_oracle(env, n):
+    g, s = _cols(n, 10 + n)
+    pf, st = _gpu(env, 3, g, s)
+    assert (pf, st) == oracle.silu_prove(3, g, s)
+    if n <= 4097:
+        assert oracle.silu_verify(3, g, s, pf) == ("accept", (0, 0))
+
+
+def test_dishonest_output_same_bytes_rejected(env):
+    g, s = _cols(500, 4, -2000, 2000)
+    s = s.copy()
+    s[123] += 1
+    pf, st = _gpu(env, 7, g, s)
+    assert (pf, st) == oracle.silu_prove(7, g, s)
+    assert oracle.silu_verify(7, g, s, pf)[0] == "silu_root"
+
+
+def test_stepped_and_resident_give_the_same_proof(env):
+    torch, fp, ctx = env
+    g, s = _cols(3000, 5)
+    a = _gpu(env, 1, g, s)
+    ctx.set_profiling(True)
+    b = _gpu(env, 1, g, s)
+    ctx.set_profiling(False)
+    assert a == b
