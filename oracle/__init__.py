@@ -51,11 +51,11 @@ REASONS = {
     20: "scl_round",
     21: "scl_final",
     22: "scl_open",
-    23: "silu_root",
-    24: "silu_round",
-    25: "silu_final",
-    26: "silu_leaf",
-    27: "silu_open",
+    23: "lookup_root",
+    24: "lookup_round",
+    25: "lookup_final",
+    26: "lookup_leaf",
+    27: "lookup_open",
 }
 
 
@@ -133,6 +133,12 @@ def lib():
         L.orc_silu_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
         L.orc_silu_verify.restype = C.c_int
         L.orc_silu_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
+        L.orc_exp_q.restype = C.c_int32
+        L.orc_exp_q.argtypes = [C.c_int32]
+        L.orc_exp_prove.restype = C.c_int
+        L.orc_exp_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
+        L.orc_exp_verify.restype = C.c_int
+        L.orc_exp_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
         _lib = L
     return _lib
 
@@ -470,38 +476,59 @@ def _i16(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a, dtype=np.int16).reshape(-1))
 
 
-def silu_prove(seed: int, g, s):
-    """LogUp proof that every s_i is the SiLU table's entry for g_i. Returns (proof, state after)."""
+def _lookup16_prove(fn, seed: int, g, s):
     L = lib()
     a, b = _i16(g), _i16(s)
     if a.size != b.size or a.size < 1:
-        raise ValueError("silu_prove: g and s need the same length >= 1")
+        raise ValueError("lookup: g and s need the same length >= 1")
     out = []
     for _ in range(2):
         tx = L.orc_tx_new(seed)
         n = C.c_uint64(0)
         buf = np.zeros(max(1, out[0] if out else 1), dtype=np.uint8)
-        rc = L.orc_silu_prove(tx, _ptr(a), _ptr(b), a.size, _ptr(buf) if out else None, out[0] if out else 0,
-                              C.byref(n))
+        rc = fn(tx, _ptr(a), _ptr(b), a.size, _ptr(buf) if out else None, out[0] if out else 0, C.byref(n))
         st = C.create_string_buffer(32)
         L.orc_tx_state(tx, st)
         L.orc_tx_free(tx)
         if out:
             if rc != 0:
-                raise ValueError(f"orc_silu_prove failed ({rc})")
+                raise ValueError(f"lookup prover failed ({rc})")
             return buf[: n.value].tobytes(), st.raw
         if rc not in (0, -2):
-            raise ValueError(f"orc_silu_prove rejected the statement ({rc})")
+            raise ValueError(f"lookup prover rejected the statement ({rc})")
         out.append(n.value)
 
 
-def silu_verify(seed: int, g, s, proof: bytes):
-    """Returns (reason_name, detail); 'accept' for a valid proof."""
+def _lookup16_verify(fn, seed: int, g, s, proof: bytes):
     L = lib()
     a, b = _i16(g), _i16(s)
     pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
     det = np.zeros(2, dtype=np.int64)
     tx = L.orc_tx_new(seed)
-    rc = L.orc_silu_verify(tx, _ptr(a), _ptr(b), a.size, _ptr(pb), len(proof), _ptr(det))
+    rc = fn(tx, _ptr(a), _ptr(b), a.size, _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+def silu_prove(seed: int, g, s):
+    """LogUp proof that every s_i is the SiLU table's entry for g_i. Returns (proof, state after)."""
+    return _lookup16_prove(lib().orc_silu_prove, seed, g, s)
+
+
+def silu_verify(seed: int, g, s, proof: bytes):
+    """Returns (reason_name, detail); 'accept' for a valid proof."""
+    return _lookup16_verify(lib().orc_silu_verify, seed, g, s, proof)
+
+
+def exp_q(v: int) -> int:
+    """The softmax numerator table's entry: floor(511 e^(v / 256) + 1/2) for v <= 0, 511 above."""
+    return int(lib().orc_exp_q(int(v)))
+
+
+def exp_prove(seed: int, g, s):
+    """LogUp proof that every s_i is the exponent table's entry for g_i."""
+    return _lookup16_prove(lib().orc_exp_prove, seed, g, s)
+
+
+def exp_verify(seed: int, g, s, proof: bytes):
+    return _lookup16_verify(lib().orc_exp_verify, seed, g, s, proof)

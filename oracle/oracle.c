@@ -1501,7 +1501,8 @@ done:
 /* tree over the keys f_i = g_i + gamma s_i, with the steps of the          */
 /* remainder / clamp lookup:                                                 */
 /*   absorb "silu_site" D(g) || D(s) (int16 little-endian);                  */
-/*   squeeze gamma ("silu_gamma"); keys padded to 2^v (v >= 1) with (0, 0);  */
+/*   squeeze gamma ("silu_gamma"); keys padded to 2^v (v >= 1) with the      */
+/*   table's own row (0, silu_q(0)) = (0, 0);                                 */
 /*   m_j = #{keys with g = j - 2^15}; send m (2^16 u32, digest absorbed,     */
 /*   "silu_m"); squeeze alpha ("silu_alpha");                                 */
 /*   tree of leaves (1, alpha - f); send layer one p(0), p(1), q(0), q(1)      */
@@ -1522,7 +1523,23 @@ enum {
 
 int32_t orc_silu_q(int32_t v) { return (int32_t)floor((double)v / (1.0 + exp(-(double)v / 256.0)) + 0.5); }
 
-static void silu_absorb_site(orc_tx* t, const int16_t* g, const int16_t* s, u64 n) {
+/* The softmax numerator by lookup (the same pages: the exponential is a lookup table; the
+ * integer softmax of "Towards Proving Frontier-Scale LLM Inference", The arithmetic, has a 9-bit
+ * numerator). Input v = score - row maximum <= 0 with 8 fractional bits:
+ *   exp_q(v) = floor(511 e^(v / 256) + 1/2), and 511 for v > 0 (never reached after the max). */
+int32_t orc_exp_q(int32_t v) { return v >= 0 ? 511 : (int32_t)floor(511.0 * exp((double)v / 256.0) + 0.5); }
+
+/* A lookup of a 16-bit function table: the same argument for every table, only the labels and
+ * (at the verifier) the table differ. */
+typedef struct {
+    const char *site, *gamma, *m, *alpha, *l1, *mu, *lambda, *round, *chal, *fin, *leaf;
+} lk_labels;
+static const lk_labels LK_SILU = {"silu_site", "silu_gamma", "silu_m", "silu_alpha", "silu_l1", "silu_mu",
+                                  "silu_lambda", "silu_round", "silu_chal", "silu_final", "silu_leaf"};
+static const lk_labels LK_EXP = {"exp_site", "exp_gamma", "exp_m", "exp_alpha", "exp_l1", "exp_mu",
+                                 "exp_lambda", "exp_round", "exp_chal", "exp_final", "exp_leaf"};
+
+static void silu_absorb_site(orc_tx* t, const lk_labels* lab, const int16_t* g, const int16_t* s, u64 n) {
     uint8_t d[64];
     uint8_t* b = (uint8_t*)calloc(2 * n, 1);
     for (u64 i = 0; i < n; i++) put_le(b + 2 * i, (u64)(uint16_t)g[i], 2);
@@ -1530,7 +1547,7 @@ static void silu_absorb_site(orc_tx* t, const int16_t* g, const int16_t* s, u64 
     for (u64 i = 0; i < n; i++) put_le(b + 2 * i, (u64)(uint16_t)s[i], 2);
     orc_tree_digest(b, 2 * n, d + 32);
     free(b);
-    orc_tx_absorb(t, "silu_site", d, 64);
+    orc_tx_absorb(t, lab->site, d, 64);
 }
 
 static void silu_mult(const int16_t* g, u64 n, u64 L, u32* m) {
@@ -1539,12 +1556,14 @@ static void silu_mult(const int16_t* g, u64 n, u64 L, u32* m) {
 }
 
 /* layers[d] has 2^d nodes */
-static void silu_tree(const int16_t* g, const int16_t* s, u64 n, int v, u64 alpha, u64 gamma, u64** Pd, u64** Qd) {
+/* padding keys are (0, tab(0)): the table's own row for input 0 */
+static void silu_tree(const int16_t* g, const int16_t* s, u64 n, int v, u64 alpha, u64 gamma, int32_t pad_s, u64** Pd,
+                      u64** Qd) {
     u64 L = (u64)1 << v;
     Pd[v] = (u64*)malloc(L * sizeof(u64));
     Qd[v] = (u64*)malloc(L * sizeof(u64));
     for (u64 i = 0; i < L; i++) {
-        u64 f = i < n ? orc_fadd(orc_fint(g[i]), orc_fmul(gamma, orc_fint(s[i]))) : 0;
+        u64 f = i < n ? orc_fadd(orc_fint(g[i]), orc_fmul(gamma, orc_fint(s[i]))) : orc_fmul(gamma, orc_fint(pad_s));
         Pd[v][i] = 1;
         Qd[v][i] = orc_fsub(alpha, f);
     }
@@ -1565,38 +1584,39 @@ static u64 silu_F(const u64 x[4], u64 lam) { /* pL qR + pR qL + lambda qL qR */
 }
 
 /* the padded key columns as field elements, and their MLEs at z */
-static void silu_leaf_values(const int16_t* g, const int16_t* s, u64 n, int v, const u64* z, u64 out[2]) {
+static void silu_leaf_values(const int16_t* g, const int16_t* s, u64 n, int v, const u64* z, int32_t pad_s, u64 out[2]) {
     u64 L = (u64)1 << v;
     u64* col = (u64*)malloc(L * sizeof(u64));
     for (u64 i = 0; i < L; i++) col[i] = i < n ? orc_fint(g[i]) : 0;
     out[0] = orc_mle_eval(col, L, z, v);
-    for (u64 i = 0; i < L; i++) col[i] = i < n ? orc_fint(s[i]) : 0;
+    for (u64 i = 0; i < L; i++) col[i] = i < n ? orc_fint(s[i]) : orc_fint(pad_s);
     out[1] = orc_mle_eval(col, L, z, v);
     free(col);
 }
 
-int orc_silu_prove(void* txh, const int16_t* g, const int16_t* s, u64 n, uint8_t* proof, u64 cap, u64* len) {
+static int lookup16_prove(void* txh, const lk_labels* lab, int32_t pad_s, const int16_t* g, const int16_t* s, u64 n,
+                          uint8_t* proof, u64 cap, u64* len) {
     if (n < 1) return -1;
     orc_tx* t = (orc_tx*)txh;
     int v = orc_log2_ceil(n);
     if (v < 1) v = 1;
     u64 L = (u64)1 << v;
     pbuf pb = {proof, cap, 0, 0};
-    silu_absorb_site(t, g, s, n);
-    u64 gamma = orc_tx_squeeze(t, "silu_gamma");
+    silu_absorb_site(t, lab, g, s, n);
+    u64 gamma = orc_tx_squeeze(t, lab->gamma);
     u32* m = (u32*)malloc(65536 * sizeof(u32));
     silu_mult(g, n, L, m);
-    send_mult(t, &pb, "silu_m", m, 65536);
-    u64 alpha = orc_tx_squeeze(t, "silu_alpha");
+    send_mult(t, &pb, lab->m, m, 65536);
+    u64 alpha = orc_tx_squeeze(t, lab->alpha);
     u64** Pd = (u64**)malloc(sizeof(u64*) * (v + 1));
     u64** Qd = (u64**)malloc(sizeof(u64*) * (v + 1));
-    silu_tree(g, s, n, v, alpha, gamma, Pd, Qd);
+    silu_tree(g, s, n, v, alpha, gamma, pad_s, Pd, Qd);
     u64 l1[4] = {Pd[1][0], Pd[1][1], Qd[1][0], Qd[1][1]};
-    send_fe(t, &pb, "silu_l1", l1, 4);
+    send_fe(t, &pb, lab->l1, l1, 4);
     u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
-    z[0] = orc_tx_squeeze(t, "silu_mu");
+    z[0] = orc_tx_squeeze(t, lab->mu);
     for (int d = 1; d < v; d++) {
-        u64 lam = orc_tx_squeeze(t, "silu_lambda");
+        u64 lam = orc_tx_squeeze(t, lab->lambda);
         u64 c = (u64)1 << d;
         u64* V[5]; /* pL, pR, qL, qR (children of layer d), eq(z, .) */
         for (int i = 0; i < 5; i++) V[i] = (u64*)malloc(c * sizeof(u64));
@@ -1618,23 +1638,23 @@ int orc_silu_prove(void* txh, const int16_t* g, const int16_t* s, u64 n, uint8_t
                     for (int i = 0; i < 5; i++) ev[i] = orc_fadd(V[i][b], orc_fmul(X, orc_fsub(V[i][h + b], V[i][b])));
                     gr[X] = orc_fadd(gr[X], orc_fmul(ev[4], silu_F(ev, lam)));
                 }
-            send_fe(t, &pb, "silu_round", gr, 4);
-            rho[r] = orc_tx_squeeze(t, "silu_chal");
+            send_fe(t, &pb, lab->round, gr, 4);
+            rho[r] = orc_tx_squeeze(t, lab->chal);
             for (int i = 0; i < 5; i++)
                 for (u64 b = 0; b < h; b++) V[i][b] = orc_fadd(V[i][b], orc_fmul(rho[r], orc_fsub(V[i][h + b], V[i][b])));
             Lr = h;
         }
         u64 fin[4] = {V[0][0], V[1][0], V[2][0], V[3][0]};
-        send_fe(t, &pb, "silu_final", fin, 4);
-        u64 mu = orc_tx_squeeze(t, "silu_mu");
+        send_fe(t, &pb, lab->fin, fin, 4);
+        u64 mu = orc_tx_squeeze(t, lab->mu);
         for (int r = 0; r < d; r++) z[r] = rho[r];
         z[d] = mu;
         for (int i = 0; i < 5; i++) free(V[i]);
         free(rho);
     }
     u64 leaf[2];
-    silu_leaf_values(g, s, n, v, z, leaf);
-    send_fe(t, &pb, "silu_leaf", leaf, 2);
+    silu_leaf_values(g, s, n, v, z, pad_s, leaf);
+    send_fe(t, &pb, lab->leaf, leaf, 2);
     for (int d = 0; d <= v; d++) {
         free(Pd[d]);
         free(Qd[d]);
@@ -1647,8 +1667,8 @@ int orc_silu_prove(void* txh, const int16_t* g, const int16_t* s, u64 n, uint8_t
     return pb.overflow ? -2 : 0;
 }
 
-int orc_silu_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const uint8_t* proof, u64 len,
-                    int64_t detail[2]) {
+static int lookup16_verify(void* txh, const lk_labels* lab, int32_t (*tab)(int32_t), const int16_t* g,
+                           const int16_t* s, u64 n, const uint8_t* proof, u64 len, int64_t detail[2]) {
     detail[0] = detail[1] = 0;
     if (n < 1) return REJ_ARGS;
     orc_tx* t = (orc_tx*)txh;
@@ -1658,20 +1678,20 @@ int orc_silu_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const 
     u32* m = (u32*)malloc(65536 * sizeof(u32));
     u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
     u64* rho = (u64*)malloc(sizeof(u64) * (v + 1));
-    silu_absorb_site(t, g, s, n);
-    u64 gamma = orc_tx_squeeze(t, "silu_gamma");
-    rd_mult(t, &rd, "silu_m", m, 65536);
+    silu_absorb_site(t, lab, g, s, n);
+    u64 gamma = orc_tx_squeeze(t, lab->gamma);
+    rd_mult(t, &rd, lab->m, m, 65536);
     if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
-    u64 alpha = orc_tx_squeeze(t, "silu_alpha");
+    u64 alpha = orc_tx_squeeze(t, lab->alpha);
     u64 l1[4];
-    rd_fe(t, &rd, "silu_l1", l1, 4);
+    rd_fe(t, &rd, lab->l1, l1, 4);
     if (rd.bad) FAIL(REJ_FORMAT, 1, 0);
     {
         /* the table side, sum_j m_j / (alpha - t_j) with t_j = v_j + gamma silu_q(v_j) */
         u64 PT = 0, QT = 1;
         for (u64 j = 0; j < 65536; j++) {
             int32_t vj = (int32_t)j - 32768;
-            u64 dj = orc_fsub(alpha, orc_fadd(orc_fint(vj), orc_fmul(gamma, orc_fint(orc_silu_q(vj)))));
+            u64 dj = orc_fsub(alpha, orc_fadd(orc_fint(vj), orc_fmul(gamma, orc_fint(tab(vj)))));
             PT = orc_fadd(orc_fmul(PT, dj), orc_fmul((u64)m[j], QT));
             QT = orc_fmul(QT, dj);
         }
@@ -1679,39 +1699,39 @@ int orc_silu_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const 
         u64 Q0 = orc_fmul(l1[2], l1[3]);
         if (Q0 == 0 || orc_fmul(P0, QT) != orc_fmul(Q0, PT)) FAIL(REJ_SILU_ROOT, 0, 0);
     }
-    u64 mu = orc_tx_squeeze(t, "silu_mu");
+    u64 mu = orc_tx_squeeze(t, lab->mu);
     u64 cP = orc_fadd(l1[0], orc_fmul(mu, orc_fsub(l1[1], l1[0])));
     u64 cQ = orc_fadd(l1[2], orc_fmul(mu, orc_fsub(l1[3], l1[2])));
     z[0] = mu;
     for (int d = 1; d < v; d++) {
-        u64 lam = orc_tx_squeeze(t, "silu_lambda");
+        u64 lam = orc_tx_squeeze(t, lab->lambda);
         u64 claim = orc_fadd(cP, orc_fmul(lam, cQ));
         for (int r = 0; r < d; r++) {
             u64 gr[4];
-            rd_fe(t, &rd, "silu_round", gr, 4);
+            rd_fe(t, &rd, lab->round, gr, 4);
             if (rd.bad) FAIL(REJ_FORMAT, 2, d);
             if (orc_fadd(gr[0], gr[1]) != claim) FAIL(REJ_SILU_ROUND, d, r);
-            rho[r] = orc_tx_squeeze(t, "silu_chal");
+            rho[r] = orc_tx_squeeze(t, lab->chal);
             claim = orc_lagrange(gr, 4, rho[r]);
         }
         u64 fin[4];
-        rd_fe(t, &rd, "silu_final", fin, 4);
+        rd_fe(t, &rd, lab->fin, fin, 4);
         if (rd.bad) FAIL(REJ_FORMAT, 3, d);
         if (orc_fmul(eq_closed(z, rho, d), silu_F(fin, lam)) != claim) FAIL(REJ_SILU_FINAL, d, 0);
-        mu = orc_tx_squeeze(t, "silu_mu");
+        mu = orc_tx_squeeze(t, lab->mu);
         cP = orc_fadd(fin[0], orc_fmul(mu, orc_fsub(fin[1], fin[0])));
         cQ = orc_fadd(fin[2], orc_fmul(mu, orc_fsub(fin[3], fin[2])));
         for (int r = 0; r < d; r++) z[r] = rho[r];
         z[d] = mu;
     }
     u64 leaf[2];
-    rd_fe(t, &rd, "silu_leaf", leaf, 2);
+    rd_fe(t, &rd, lab->leaf, leaf, 2);
     if (rd.bad) FAIL(REJ_FORMAT, 4, 0);
     if (cP != 1) FAIL(REJ_SILU_LEAF, 0, 0);
     if (cQ != orc_fsub(alpha, orc_fadd(leaf[0], orc_fmul(gamma, leaf[1])))) FAIL(REJ_SILU_LEAF, 1, 0);
     {
         u64 want[2];
-        silu_leaf_values(g, s, n, v, z, want);
+        silu_leaf_values(g, s, n, v, z, tab(0), want);
         if (want[0] != leaf[0]) FAIL(REJ_SILU_OPEN, 0, 0);
         if (want[1] != leaf[1]) FAIL(REJ_SILU_OPEN, 1, 0);
     }
@@ -1721,4 +1741,19 @@ done:
     free(z);
     free(rho);
     return rc;
+}
+
+int orc_silu_prove(void* txh, const int16_t* g, const int16_t* s, u64 n, uint8_t* proof, u64 cap, u64* len) {
+    return lookup16_prove(txh, &LK_SILU, orc_silu_q(0), g, s, n, proof, cap, len);
+}
+int orc_silu_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const uint8_t* proof, u64 len,
+                    int64_t detail[2]) {
+    return lookup16_verify(txh, &LK_SILU, orc_silu_q, g, s, n, proof, len, detail);
+}
+int orc_exp_prove(void* txh, const int16_t* g, const int16_t* s, u64 n, uint8_t* proof, u64 cap, u64* len) {
+    return lookup16_prove(txh, &LK_EXP, orc_exp_q(0), g, s, n, proof, cap, len);
+}
+int orc_exp_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const uint8_t* proof, u64 len,
+                   int64_t detail[2]) {
+    return lookup16_verify(txh, &LK_EXP, orc_exp_q, g, s, n, proof, len, detail);
 }

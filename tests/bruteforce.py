@@ -447,15 +447,21 @@ def silu_table_entry(v: int) -> int:
 
 
 def silu_prove(seed: int, g, s) -> bytes:
-    """The SiLU lookup's proof from definitions: tree layers by their recurrence, every
-    layer round value a hypercube sum of eq times the layer summand over MLEs (no folding)."""
+    """The SiLU lookup's proof from definitions (see lookup16_prove)."""
+    return lookup16_prove(seed, g, s, "silu", silu_table_entry(0))
+
+
+def lookup16_prove(seed: int, g, s, prefix: str, pad_s: int) -> bytes:
+    """A 16-bit function lookup's proof from definitions: tree layers by their recurrence, every
+    layer round value a hypercube sum of eq times the layer summand over MLEs (no folding).
+    The table enters only through its row for input 0, which pads the keys."""
     g = [int(x) for x in np.asarray(g).reshape(-1)]
     s = [int(x) for x in np.asarray(s).reshape(-1)]
     n = len(g)
     v = max(1, log2c(n))
     L = 1 << v
     gp = g + [0] * (L - n)
-    sp = s + [0] * (L - n)
+    sp = s + [pad_s] * (L - n)  # padding keys are the table's row for input 0
     out = bytearray()
 
     def send(label, vals):
@@ -464,25 +470,25 @@ def silu_prove(seed: int, g, s) -> bytes:
         tx.absorb(label, b)
 
     tx = Tx(seed)
-    tx.absorb("silu_site", tree_digest(np.asarray(g, "<i2").tobytes()) + tree_digest(np.asarray(s, "<i2").tobytes()))
-    gamma = tx.squeeze("silu_gamma")
+    tx.absorb(prefix + "_site", tree_digest(np.asarray(g, "<i2").tobytes()) + tree_digest(np.asarray(s, "<i2").tobytes()))
+    gamma = tx.squeeze(prefix + "_gamma")
     m = np.zeros(1 << 16, np.int64)
     for x in gp:
         m[x + 32768] += 1
     b = m.astype("<u4").tobytes()
     out.extend(b)
-    tx.absorb("silu_m", tree_digest(b))
-    alpha = tx.squeeze("silu_alpha")
+    tx.absorb(prefix + "_m", tree_digest(b))
+    alpha = tx.squeeze(prefix + "_alpha")
     Pl = [[1] * L]
     Ql = [[(alpha - (a + gamma * c)) % P for a, c in zip(gp, sp)]]
     for _ in range(v):
         p, q_ = Pl[0], Ql[0]
         Pl.insert(0, [(p[2 * x] * q_[2 * x + 1] + p[2 * x + 1] * q_[2 * x]) % P for x in range(len(p) // 2)])
         Ql.insert(0, [q_[2 * x] * q_[2 * x + 1] % P for x in range(len(p) // 2)])
-    send("silu_l1", [Pl[1][0], Pl[1][1], Ql[1][0], Ql[1][1]])
-    z = [tx.squeeze("silu_mu")]
+    send(prefix + "_l1", [Pl[1][0], Pl[1][1], Ql[1][0], Ql[1][1]])
+    z = [tx.squeeze(prefix + "_mu")]
     for d in range(1, v):
-        lam = tx.squeeze("silu_lambda")
+        lam = tx.squeeze(prefix + "_lambda")
         Pc, Qc = Pl[d + 1], Ql[d + 1]
         vecs = ([Pc[2 * x] for x in range(1 << d)], [Pc[2 * x + 1] for x in range(1 << d)],
                 [Qc[2 * x] for x in range(1 << d)], [Qc[2 * x + 1] for x in range(1 << d)])
@@ -497,9 +503,9 @@ def silu_prove(seed: int, g, s) -> bytes:
                     pL, pR, qL, qR = (mle(vv, pt) for vv in vecs)
                     acc += eq_ml(z, pt) * (pL * qR + pR * qL + lam * qL * qR)
                 gr.append(acc % P)
-            send("silu_round", gr)
-            rho_l.append(tx.squeeze("silu_chal"))
-        send("silu_final", [mle(vv, rho_l) for vv in vecs])
-        z = rho_l + [tx.squeeze("silu_mu")]
-    send("silu_leaf", [mle(gp, z), mle(sp, z)])
+            send(prefix + "_round", gr)
+            rho_l.append(tx.squeeze(prefix + "_chal"))
+        send(prefix + "_final", [mle(vv, rho_l) for vv in vecs])
+        z = rho_l + [tx.squeeze(prefix + "_mu")]
+    send(prefix + "_leaf", [mle(gp, z), mle(sp, z)])
     return bytes(out)

@@ -85,22 +85,22 @@ def test_each_check_fires():
     s_bad = s.copy()
     s_bad[7] += 1
     pf_bad, _ = oracle.silu_prove(2, g, s_bad)
-    assert oracle.silu_verify(2, g, s_bad, pf_bad)[0] == "silu_root"
+    assert oracle.silu_verify(2, g, s_bad, pf_bad)[0] == "lookup_root"
     pf, _ = oracle.silu_prove(2, g, s)
     v = bf.log2c(n)
     off = 4 * 65536  # the multiplicities come first
     l1 = list(struct.unpack("<4Q", pf[off:off + 32]))
-    assert oracle.silu_verify(2, g, s, _put(pf, off, l1[0] + 1))[0] == "silu_root"
+    assert oracle.silu_verify(2, g, s, _put(pf, off, l1[0] + 1))[0] == "lookup_root"
     off += 32
     # layer d has d rounds of 4 values and 4 final values; layer 1's first round value
     g0 = struct.unpack("<Q", pf[off:off + 8])[0]
-    assert oracle.silu_verify(2, g, s, _put(pf, off, g0 + 1)) == ("silu_round", (1, 0))
+    assert oracle.silu_verify(2, g, s, _put(pf, off, g0 + 1)) == ("lookup_round", (1, 0))
     fin = off + 32
     f0 = struct.unpack("<Q", pf[fin:fin + 8])[0]
-    assert oracle.silu_verify(2, g, s, _put(pf, fin, f0 + 1)) == ("silu_final", (1, 0))
+    assert oracle.silu_verify(2, g, s, _put(pf, fin, f0 + 1)) == ("lookup_final", (1, 0))
     leaf = len(pf) - 16
     lg = struct.unpack("<Q", pf[leaf:leaf + 8])[0]
-    assert oracle.silu_verify(2, g, s, _put(pf, leaf, lg + 1))[0] == "silu_leaf"
+    assert oracle.silu_verify(2, g, s, _put(pf, leaf, lg + 1))[0] == "lookup_leaf"
     # the verifier holds other columns than the prover used
     g2 = g.copy()
     g2[0] ^= 2
