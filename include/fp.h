@@ -283,6 +283,22 @@ int logup_prove_silu(fp_ctx* ctx, fp_tx* tx, const int16_t* g, const int16_t* s,
 int fp_silu_table(int32_t* out);
 
 /*
+ * The softmax numerator by lookup ("Towards Proving Frontier-Scale LLM Inference",
+ * The arithmetic: the exponential is a lookup table, the integer softmax has a
+ * 9-bit numerator): the same argument as logup_prove_silu with the labels
+ * "exp_site", "exp_gamma", "exp_m", "exp_alpha", "exp_l1", "exp_mu",
+ * "exp_lambda", "exp_round", "exp_chal", "exp_final", "exp_leaf" and the table
+ * exp_q(v) = floor(511 e^(v/256) + 1/2) for v = score - row maximum <= 0, 511
+ * for v > 0. Keys are padded with the table's row for input 0, (0, 511). Same
+ * arguments, proof layout and errors as logup_prove_silu.
+ */
+int logup_prove_exp(fp_ctx* ctx, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
+                    size_t* proof_len, void* stream);
+
+/* The numerator table's 2^16 entries exp_q(v), v = -2^15 .. 2^15 - 1, into host out (no GPU work). */
+int fp_exp_table(int32_t* out);
+
+/*
  * Self-test of the bounded device waits. The sum-check kernels stay resident
  * across rounds and wait (a bounded number of polls) for each Fiat-Shamir
  * challenge from the host. This call launches a kernel that waits for a

@@ -77,6 +77,8 @@ def lib():
     L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, C.POINTER(sz), vp]
     L.logup_prove_silu.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_silu_table.argtypes = [vp]
+    L.logup_prove_exp.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
+    L.fp_exp_table.argtypes = [vp]
     L.fp_proof_size.argtypes = [C.POINTER(_Site), i32, C.POINTER(sz), C.POINTER(sz)]
     L.fp_ctx_set_profiling.argtypes = [vp, i32]
     L.fp_session_selftest.argtypes = [vp, vp]
@@ -275,9 +277,16 @@ class Context:
     def prove_silu(self, tx: Transcript, g, s, stream=None) -> bytes:
         """LogUp proof that every entry of the device int16 tensor s is the SiLU table's entry
         for the same entry of g (flattened row-major); continues tx."""
+        return self._lookup16(self._L.logup_prove_silu, "prove_silu", tx, g, s, stream)
+
+    def prove_exp(self, tx: Transcript, g, s, stream=None) -> bytes:
+        """As prove_silu, for the softmax numerator table."""
+        return self._lookup16(self._L.logup_prove_exp, "prove_exp", tx, g, s, stream)
+
+    def _lookup16(self, fn, what, tx, g, s, stream):
         n = int(g.numel())
         if int(s.numel()) != n:
-            raise ValueError("prove_silu: g and s differ in size")
+            raise ValueError(f"{what}: g and s differ in size")
         v = 0
         while (1 << v) < n:
             v += 1
@@ -285,8 +294,7 @@ class Context:
         cap = 4 * 65536 + 32 + 16 + sum(32 * d + 32 for d in range(1, v))
         buf = C.create_string_buffer(cap)
         ln = C.c_size_t(cap)
-        self._check(self._L.logup_prove_silu(self.h, tx.h, _ptr(g), _ptr(s), n, buf, C.byref(ln),
-                                             _stream(stream)), "logup_prove_silu")
+        self._check(fn(self.h, tx.h, _ptr(g), _ptr(s), n, buf, C.byref(ln), _stream(stream)), what)
         return buf.raw[: ln.value]
 
     def prove_logup(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
@@ -364,4 +372,14 @@ def silu_table():
     rc = lib().fp_silu_table(out.ctypes.data)
     if rc != 0:
         raise FpError(rc, "fp_silu_table")
+    return out
+
+
+def exp_table():
+    """The softmax numerator table's 2^16 entries, as the library computes them."""
+    import numpy as np
+    out = np.zeros(65536, dtype=np.int32)
+    rc = lib().fp_exp_table(out.ctypes.data)
+    if rc != 0:
+        raise FpError(rc, "fp_exp_table")
     return out

@@ -43,11 +43,12 @@ __global__ void silu_hist_kernel(const int16_t* __restrict__ g, int64_t n, uint3
 
 __global__ void silu_add_pad_kernel(uint32_t* m, uint32_t pad) { m[32768] += pad; }
 
-// leaves: P = 1, Q = alpha - (g + gamma s) (zero keys past n)
+// leaves: P = 1, Q = alpha - (g + gamma s); past n the padding key fpad (the table's row for input 0)
 __global__ void silu_leaf_kernel(const int16_t* __restrict__ g, const int16_t* __restrict__ s, int64_t n, int64_t L,
-                                 uint64_t alpha, uint64_t gamma, uint64_t* __restrict__ P, uint64_t* __restrict__ Q) {
+                                 uint64_t alpha, uint64_t gamma, uint64_t fpad, uint64_t* __restrict__ P,
+                                 uint64_t* __restrict__ Q) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < L; i += (int64_t)gridDim.x * blockDim.x) {
-        uint64_t f = 0;
+        uint64_t f = fpad;
         if (i < n) f = gl_add(lift_i(g[i]), gl_mul(gamma, lift_i(s[i])));
         P[i] = 1;
         Q[i] = gl_sub(alpha, f);
@@ -64,20 +65,24 @@ __global__ void silu_level_kernel(const uint64_t* __restrict__ P, const uint64_t
     }
 }
 
-// sum_{x < L} eq(z, x) a(x) for an int16 column a of n entries (zero past n), eq split as
-// EH[x >> vl] EL[x & (2^vl - 1)]
+// out[0] = sum_{x < n} eq(z, x) a(x) for an int16 column a of n entries, out[1] = sum_{x < n} eq(z, x)
+// (so that a padding value past n adds pad (1 - out[1])); eq split as EH[x >> vl] EL[x & (2^vl - 1)]
 __global__ void __launch_bounds__(256) silu_mle_kernel(const int16_t* __restrict__ a, int64_t n,
                                                        const uint64_t* __restrict__ EH, const uint64_t* __restrict__ EL,
                                                        int vl, uint64_t* part, unsigned int* ticket, uint64_t* out) {
-    GlAcc acc;
+    GlAcc acc, eacc;
     const int64_t mask = (1ll << vl) - 1;
     for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
+        const uint64_t e = gl_mul(__ldg(EH + (x >> vl)), __ldg(EL + (x & mask)));
+        eacc.add(e);
         const int v = a[x];
-        if (v == 0) continue;
-        acc.mac(gl_mul(__ldg(EH + (x >> vl)), __ldg(EL + (x & mask))), lift_i(v));
+        if (v != 0) acc.mac(e, lift_i(v));
     }
-    uint64_t v[1] = {acc.value()};
-    if (grid_sum_gl<1>(v, part, ticket) && threadIdx.x == 0) *out = v[0];
+    uint64_t v[2] = {acc.value(), eacc.value()};
+    if (grid_sum_gl<2>(v, part, ticket) && threadIdx.x == 0) {
+        out[0] = v[0];
+        out[1] = v[1];
+    }
 }
 
 struct LayerArgs {
@@ -203,6 +208,17 @@ __global__ void __launch_bounds__(SL_THREADS, 2) silu_layer_kernel(LayerArgs A, 
 
 int64_t silu_q_host(int64_t v) { return (int64_t)floor((double)v / (1.0 + exp(-(double)v / 256.0)) + 0.5); }
 
+// the softmax numerator: floor(511 e^(v/256) + 1/2) for v = score - row maximum <= 0, 511 above
+int64_t exp_q_host(int64_t v) { return v >= 0 ? 511 : (int64_t)floor(511.0 * exp((double)v / 256.0) + 0.5); }
+
+struct LookupLabels {
+    const char *site, *gamma, *m, *alpha, *l1, *mu, *lambda, *round, *chal, *fin, *leaf;
+};
+const LookupLabels kSiluLabels = {"silu_site", "silu_gamma", "silu_m", "silu_alpha", "silu_l1", "silu_mu",
+                                  "silu_lambda", "silu_round", "silu_chal", "silu_final", "silu_leaf"};
+const LookupLabels kExpLabels = {"exp_site", "exp_gamma", "exp_m", "exp_alpha", "exp_l1", "exp_mu",
+                                 "exp_lambda", "exp_round", "exp_chal", "exp_final", "exp_leaf"};
+
 // the degree-3 polynomial through (i, g[i]), i = 0..3, at r
 uint64_t lagrange4(const uint64_t g[4], uint64_t r) {
     static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
@@ -227,10 +243,10 @@ size_t silu_proof_len(int64_t n) {
     return len;
 }
 
-}  // namespace
-
-int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
-                     size_t* proof_len, void* stream) {
+// One 16-bit function lookup: the argument is the same for every table; the table enters
+// only through its row for input 0 (pad_s = table(0)), which pads the keys, and the labels.
+int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s, const int16_t* g, const int16_t* s,
+                   int64_t n, uint8_t* proof, size_t* proof_len, void* stream) {
     if (!c || !tx || !proof_len) return fp_fail(c, FP_ERR_ARG, "logup_prove_silu: null argument");
     if (!g || !s) return fp_fail(c, FP_ERR_ARG, "logup_prove_silu: null column");
     if (n < 1 || n > (1ll << SL_MAX_V)) return fp_fail(c, FP_ERR_SHAPE, "logup_prove_silu: need 1 <= n <= 2^30");
@@ -251,9 +267,9 @@ int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, i
         FpDigestJob jobs[2] = {{(const uint8_t*)g, 2 * (uint64_t)n}, {(const uint8_t*)s, 2 * (uint64_t)n}};
         uint8_t d[64];
         if ((rc = fp_digest_many(c, jobs, 2, d, st))) return rc;  // synchronises the stream
-        fp_tx_absorb_raw(tx, "silu_site", d, 64);
+        fp_tx_absorb_raw(tx, lab.site, d, 64);
     }
-    const uint64_t gamma = fp_tx_squeeze_one(tx, "silu_gamma");
+    const uint64_t gamma = fp_tx_squeeze_one(tx, lab.gamma);
 
     // ---- scratch: multiplicities, tree layers 1..v, layer vectors, eq tables, reductions ----
     int occ = 0;
@@ -308,14 +324,15 @@ int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, i
     size_t pos = 0;
     memcpy(proof + pos, hm, 4 * 65536);  // device words are little-endian u32
     pos += 4 * 65536;
-    fp_tx_absorb_raw(tx, "silu_m", dm, 32);
-    const uint64_t alpha = fp_tx_squeeze_one(tx, "silu_alpha");
+    fp_tx_absorb_raw(tx, lab.m, dm, 32);
+    const uint64_t alpha = fp_tx_squeeze_one(tx, lab.alpha);
 
     // ---- the fraction tree, layers v (leaves) .. 1 ----
     {
         int slot;
         fp_tic(c, st, K_SILU_TREE, 4.0 * (double)n + 32.0 * (double)L, &slot);
-        silu_leaf_kernel<<<grid_of(c, L), 256, 0, st>>>(g, s, n, L, alpha, gamma, TP[v], TQ[v]);
+        const uint64_t fpad = gl_mul(gamma, pad_s < 0 ? GL_P - (uint64_t)(-pad_s) : (uint64_t)pad_s);
+        silu_leaf_kernel<<<grid_of(c, L), 256, 0, st>>>(g, s, n, L, alpha, gamma, fpad, TP[v], TQ[v]);
         FP_CUDA(c, cudaGetLastError());
         for (int d = v - 1; d >= 1; d--) {
             silu_level_kernel<<<grid_of(c, 1ll << d), 256, 0, st>>>(TP[d + 1], TQ[d + 1], 1ll << d, TP[d], TQ[d]);
@@ -328,16 +345,16 @@ int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, i
     FP_CUDA(c, cudaStreamSynchronize(st));
     uint64_t l1[4] = {hs[0], hs[1], hs[2], hs[3]};
     put_u64s(proof + pos, l1, 4);
-    fp_tx_absorb_raw(tx, "silu_l1", proof + pos, 32);
+    fp_tx_absorb_raw(tx, lab.l1, proof + pos, 32);
     pos += 32;
     FpPoint z;
     z.v = 1;
-    z.z[0] = fp_tx_squeeze_one(tx, "silu_mu");
+    z.z[0] = fp_tx_squeeze_one(tx, lab.mu);
     uint64_t cP = gl_fold(l1[0], l1[1], z.z[0]), cQ = gl_fold(l1[2], l1[3], z.z[0]);
 
     // ---- layer sum-checks d = 1 .. v - 1 ----
     for (int d = 1; d < v; d++) {
-        const uint64_t lam = fp_tx_squeeze_one(tx, "silu_lambda");
+        const uint64_t lam = fp_tx_squeeze_one(tx, lab.lambda);
         uint64_t claim = gl_add(cP, gl_mul(lam, cQ));
         for (int i = 0; i < d; i++) hs[8 + i] = z.z[i];
         FP_CUDA(c, cudaMemcpyAsync(small + 8, hs + 8, 8 * (size_t)d, cudaMemcpyHostToDevice, st));
@@ -395,10 +412,10 @@ int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, i
             if (gl_add(gr[0], gr[1]) != claim)
                 return fp_fail(c, FP_ERR_CUDA, "logup_prove_silu: round values inconsistent with the claim");
             put_u64s(proof + pos, gr, 4);
-            fp_tx_absorb_raw(tx, "silu_round", proof + pos, 32);
+            fp_tx_absorb_raw(tx, lab.round, proof + pos, 32);
             pos += 32;
             fp_session_expect(c, t < d ? 3 : 4);  // the last challenge triggers the four final values
-            const uint64_t r = fp_tx_squeeze_one(tx, "silu_chal");
+            const uint64_t r = fp_tx_squeeze_one(tx, lab.chal);
             fp_session_post(c, A.seq0 + t, r);
             rho[t - 1] = r;
             claim = lagrange4(gr, r);
@@ -416,9 +433,9 @@ int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, i
         uint64_t fin[4] = {c->mb->res[0], c->mb->res[1], c->mb->res[2], c->mb->res[3]};
         FP_CUDA(c, cudaStreamSynchronize(st));
         put_u64s(proof + pos, fin, 4);
-        fp_tx_absorb_raw(tx, "silu_final", proof + pos, 32);
+        fp_tx_absorb_raw(tx, lab.fin, proof + pos, 32);
         pos += 32;
-        const uint64_t mu = fp_tx_squeeze_one(tx, "silu_mu");
+        const uint64_t mu = fp_tx_squeeze_one(tx, lab.mu);
         cP = gl_fold(fin[0], fin[1], mu);
         cQ = gl_fold(fin[2], fin[3], mu);
         for (int i = 0; i < d; i++) z.z[i] = rho[i];
@@ -440,22 +457,42 @@ int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, i
         fp_tic(c, st, K_SILU_LEAF, 4.0 * (double)n, &slot);
         silu_mle_kernel<<<blocks, 256, 0, st>>>(g, n, EH, EL, vl, part, c->tickets, small);
         FP_CUDA(c, cudaGetLastError());
-        silu_mle_kernel<<<blocks, 256, 0, st>>>(s, n, EH, EL, vl, part, c->tickets, small + 1);
+        silu_mle_kernel<<<blocks, 256, 0, st>>>(s, n, EH, EL, vl, part, c->tickets, small + 2);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
-        FP_CUDA(c, cudaMemcpyAsync(hs, small, 16, cudaMemcpyDeviceToHost, st));
+        FP_CUDA(c, cudaMemcpyAsync(hs, small, 32, cudaMemcpyDeviceToHost, st));
         FP_CUDA(c, cudaStreamSynchronize(st));
     }
-    const uint64_t leaf[2] = {hs[0], hs[1]};
+    // the s column past n holds the padding value: it adds pad_s (1 - sum_{x < n} eq(z, x))
+    const uint64_t padf = pad_s < 0 ? GL_P - (uint64_t)(-pad_s) : (uint64_t)pad_s;
+    const uint64_t leaf[2] = {hs[0], gl_add(hs[2], gl_mul(padf, gl_sub(1, hs[3])))};
     put_u64s(proof + pos, leaf, 2);
-    fp_tx_absorb_raw(tx, "silu_leaf", proof + pos, 16);
+    fp_tx_absorb_raw(tx, lab.leaf, proof + pos, 16);
     pos += 16;
     *proof_len = pos;
     return FP_OK;
 }
 
+}  // namespace
+
+int logup_prove_silu(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
+                     size_t* proof_len, void* stream) {
+    return lookup16_prove(c, tx, kSiluLabels, silu_q_host(0), g, s, n, proof, proof_len, stream);
+}
+
+int logup_prove_exp(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
+                    size_t* proof_len, void* stream) {
+    return lookup16_prove(c, tx, kExpLabels, exp_q_host(0), g, s, n, proof, proof_len, stream);
+}
+
 int fp_silu_table(int32_t* out) {
     if (!out) return FP_ERR_ARG;
     for (int64_t v = -32768; v < 32768; v++) out[v + 32768] = (int32_t)silu_q_host(v);
+    return FP_OK;
+}
+
+int fp_exp_table(int32_t* out) {
+    if (!out) return FP_ERR_ARG;
+    for (int64_t v = -32768; v < 32768; v++) out[v + 32768] = (int32_t)exp_q_host(v);
     return FP_OK;
 }

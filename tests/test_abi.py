@@ -108,3 +108,10 @@ def test_silu_table_matches_oracle(L):
     lib_t = fp.silu_table()
     ora_t = np.array([oracle.silu_q(v) for v in range(-32768, 32768)], dtype=np.int32)
     assert np.array_equal(lib_t, ora_t)
+
+
+def test_exp_table_matches_oracle(L):
+    import numpy as np
+    import sum_check_prover_b200 as fp
+    ora_t = np.array([oracle.exp_q(v) for v in range(-32768, 32768)], dtype=np.int32)
+    assert np.array_equal(fp.exp_table(), ora_t)

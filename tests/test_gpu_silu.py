@@ -72,7 +72,31 @@ def test_dishonest_output_same_bytes_rejected(env):
     s[123] += 1
     pf, st = _gpu(env, 7, g, s)
     assert (pf, st) == oracle.silu_prove(7, g, s)
-    assert oracle.silu_verify(7, g, s, pf)[0] == "silu_root"
+    assert oracle.silu_verify(7, g, s, pf)[0] == "lookup_root"
+
+
+EXP = None
+
+
+def exp_cols(n, seed):
+    global EXP
+    if EXP is None:
+        EXP = np.array([oracle.exp_q(v) for v in range(-32768, 32768)], dtype=np.int16)
+    rng = np.random.default_rng(seed)
+    g = rng.integers(-3000, 1, n).astype(np.int16)
+    return g, EXP[g.astype(np.int64) + 32768]
+
+
+@pytest.mark.parametrize("n", [1, 3, 5, 100, 1000, 4097])
+def test_exp_matches_oracle(env, n):
+    # padded sizes exercise the numerator table's padding row (0, 511)
+    torch, fp, ctx = env
+    g, s = exp_cols(n, 20 + n)
+    tx = fp.Transcript(9)
+    pf = ctx.prove_exp(tx, torch.from_numpy(g).cuda(), torch.from_numpy(s).cuda())
+    torch.cuda.synchronize()
+    assert (pf, tx.state()) == oracle.exp_prove(9, g, s)
+    assert oracle.exp_verify(9, g, s, pf) == ("accept", (0, 0))
 
 
 def test_stepped_and_resident_give_the_same_proof(env):
