@@ -18,6 +18,10 @@
  *    proven by sum-check. Page "Towards Proving Frontier-Scale LLM Inference",
  *    The proof system: lookups by logarithmic derivatives (LogUp), whose
  *    fractions fill that tree.
+ *  - 2 and 3.1 again: products that are never committed (the MLP's gated
+ *    product, the per-group scaled weights) are reduced by sum-check to claims
+ *    on their committed factors, and the SiLU and the softmax exponential are
+ *    proven by lookups into 16-bit function tables.
  * The exact byte-level protocol (transcript encoding, tree digest, message
  * order, bit order, rounding tie) is specified in the repository's design
  * notes and implemented independently by the CPU oracle.
