@@ -56,6 +56,10 @@ REASONS = {
     25: "lookup_final",
     26: "lookup_leaf",
     27: "lookup_open",
+    28: "lhi_sum",
+    29: "lhi_round",
+    30: "lhi_final",
+    31: "lhi_open",
 }
 
 
@@ -139,6 +143,10 @@ def lib():
         L.orc_exp_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
         L.orc_exp_verify.restype = C.c_int
         L.orc_exp_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
+        L.orc_lhi_prove.restype = C.c_int
+        L.orc_lhi_prove.argtypes = [vp, vp, u64, C.c_int, vp, u64, C.POINTER(u64)]
+        L.orc_lhi_verify.restype = C.c_int
+        L.orc_lhi_verify.argtypes = [vp, vp, u64, C.c_int, vp, u64, vp]
         _lib = L
     return _lib
 
@@ -532,3 +540,38 @@ def exp_prove(seed: int, g, s):
 
 def exp_verify(seed: int, g, s, proof: bytes):
     return _lookup16_verify(lib().orc_exp_verify, seed, g, s, proof)
+
+
+# ---- the helper-inverse LogUp (the variant to set against the GKR tree) -------------
+
+def lhi_prove(seed: int, r, k: int):
+    """Helper-inverse LogUp proof that every key r_i lies in the remainder table R_k."""
+    L = lib()
+    a = np.ascontiguousarray(np.asarray(r, dtype=np.int32).reshape(-1))
+    out = []
+    for _ in range(2):
+        tx = L.orc_tx_new(seed)
+        n = C.c_uint64(0)
+        buf = np.zeros(max(1, out[0] if out else 1), dtype=np.uint8)
+        rc = L.orc_lhi_prove(tx, _ptr(a), a.size, k, _ptr(buf) if out else None, out[0] if out else 0, C.byref(n))
+        st = C.create_string_buffer(32)
+        L.orc_tx_state(tx, st)
+        L.orc_tx_free(tx)
+        if out:
+            if rc != 0:
+                raise ValueError(f"orc_lhi_prove failed ({rc})")
+            return buf[: n.value].tobytes(), st.raw
+        if rc not in (0, -2):
+            raise ValueError(f"orc_lhi_prove rejected the statement ({rc})")
+        out.append(n.value)
+
+
+def lhi_verify(seed: int, r, k: int, proof: bytes):
+    L = lib()
+    a = np.ascontiguousarray(np.asarray(r, dtype=np.int32).reshape(-1))
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_lhi_verify(tx, _ptr(a), a.size, k, _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

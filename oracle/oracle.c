@@ -1757,3 +1757,187 @@ int orc_exp_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const u
                    int64_t detail[2]) {
     return lookup16_verify(txh, &LK_EXP, orc_exp_q, g, s, n, proof, len, detail);
 }
+
+/* ------------------------------------------------------------------------ */
+/* The helper-inverse LogUp (the lookup argument of "Towards Proving         */
+/* Frontier-Scale LLM Inference", The proof system: LogUp after Haboeck      */
+/* 2022), the variant to set against the GKR fraction tree. For the         */
+/* remainder table R_k = {j - 2^(k-1)} and a key column r (int32, n keys,   */
+/* padded to 2^v, v >= 1, with the key 0):                                  */
+/*   absorb "lhi_site" D(r) (int32 little-endian);                          */
+/*   m_j = #{keys = j - 2^(k-1)}; send m (2^k u32, digest absorbed, "lhi_m"); */
+/*   squeeze alpha ("lhi_alpha"); the helper column h_i = 1 / (alpha - r_i) */
+/*   is committed: absorb "lhi_h" D(h as u64 little-endian);                 */
+/*   squeeze z_1..z_v ("lhi_z") and beta ("lhi_beta");                       */
+/*   send S = sum_i h_i ("lhi_sum");                                         */
+/*   sum-check of F(x) = h(x) + beta eq(z, x) (h(x) (alpha - f(x)) - 1) over  */
+/*   v variables, claim S: rounds g(0..3) ("lhi_round"), "lhi_chal";         */
+/*   send h(rho), f(rho) ("lhi_final").                                       */
+/* The verifier checks S against sum_j m_j / (alpha - t_j), every round, the */
+/* end against h + beta eq(z, rho) (h (alpha - f) - 1), and h(rho), f(rho)   */
+/* against the columns it recomputes (standing in for openings). The        */
+/* zero-check part forces h_i (alpha - f_i) = 1 everywhere (with high        */
+/* probability over z), so S is the key side of the LogUp identity.         */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_LHI_SUM = 28,    /* S != the table side */
+    REJ_LHI_ROUND = 29,  /* g(0) + g(1) != running claim */
+    REJ_LHI_FINAL = 30,  /* the end does not match F at rho */
+    REJ_LHI_OPEN = 31    /* h(rho) or f(rho) != the columns' MLEs */
+};
+
+static void lhi_columns(const int32_t* r, u64 n, int v, u64 alpha, u64* f, u64* h) {
+    u64 L = (u64)1 << v;
+    for (u64 i = 0; i < L; i++) {
+        f[i] = i < n ? orc_fint(r[i]) : 0;
+        h[i] = orc_finv(orc_fsub(alpha, f[i]));
+    }
+}
+
+static void lhi_absorb_h(orc_tx* t, const u64* h, u64 L) {
+    uint8_t* b = (uint8_t*)malloc(8 * L);
+    uint8_t d[32];
+    for (u64 i = 0; i < L; i++) put_le(b + 8 * i, h[i], 8);
+    orc_tree_digest(b, 8 * L, d);
+    free(b);
+    orc_tx_absorb(t, "lhi_h", d, 32);
+}
+
+static void lhi_absorb_site(orc_tx* t, const int32_t* r, u64 n) {
+    uint8_t* b = (uint8_t*)calloc(4 * n, 1);
+    uint8_t d[32];
+    for (u64 i = 0; i < n; i++) put_le(b + 4 * i, (u64)(u32)r[i], 4);
+    orc_tree_digest(b, 4 * n, d);
+    free(b);
+    orc_tx_absorb(t, "lhi_site", d, 32);
+}
+
+static void lhi_mult(const int32_t* r, u64 n, u64 L, int k, u32* m) {
+    u64 T = (u64)1 << k;
+    int64_t half = (int64_t)1 << (k - 1);
+    memset(m, 0, T * sizeof(u32));
+    for (u64 i = 0; i < L; i++) {
+        int64_t j = (i < n ? (int64_t)r[i] : 0) + half;
+        if (j >= 0 && (u64)j < T) m[j]++;
+    }
+}
+
+/* F at one point of the three lines: h + beta e (h (alpha - f) - 1) */
+static u64 lhi_F(u64 h, u64 f, u64 e, u64 alpha, u64 beta) {
+    return orc_fadd(h, orc_fmul(beta, orc_fmul(e, orc_fsub(orc_fmul(h, orc_fsub(alpha, f)), 1))));
+}
+
+int orc_lhi_prove(void* txh, const int32_t* r, u64 n, int k, uint8_t* proof, u64 cap, u64* len) {
+    if (n < 1 || k < 1 || k > 24) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n);
+    if (v < 1) v = 1;
+    u64 L = (u64)1 << v, T = (u64)1 << k;
+    pbuf pb = {proof, cap, 0, 0};
+    lhi_absorb_site(t, r, n);
+    u32* m = (u32*)malloc(T * sizeof(u32));
+    lhi_mult(r, n, L, k, m);
+    send_mult(t, &pb, "lhi_m", m, T);
+    u64 alpha = orc_tx_squeeze(t, "lhi_alpha");
+    u64* f = (u64*)malloc(L * sizeof(u64));
+    u64* h = (u64*)malloc(L * sizeof(u64));
+    u64* E = (u64*)malloc(L * sizeof(u64));
+    u64* z = (u64*)malloc(sizeof(u64) * v);
+    lhi_columns(r, n, v, alpha, f, h);
+    lhi_absorb_h(t, h, L);
+    for (int i = 0; i < v; i++) z[i] = orc_tx_squeeze(t, "lhi_z");
+    u64 beta = orc_tx_squeeze(t, "lhi_beta");
+    u64 S = 0;
+    for (u64 i = 0; i < L; i++) S = orc_fadd(S, h[i]);
+    send_fe(t, &pb, "lhi_sum", &S, 1);
+    orc_eq_table(z, v, E);
+    u64 Lr = L;
+    for (int rd = 0; rd < v; rd++) {
+        u64 hh = Lr >> 1;
+        u64 g[4] = {0, 0, 0, 0};
+        for (u64 b = 0; b < hh; b++)
+            for (u64 X = 0; X < 4; X++) {
+                u64 hx = orc_fadd(h[b], orc_fmul(X, orc_fsub(h[hh + b], h[b])));
+                u64 fx = orc_fadd(f[b], orc_fmul(X, orc_fsub(f[hh + b], f[b])));
+                u64 ex = orc_fadd(E[b], orc_fmul(X, orc_fsub(E[hh + b], E[b])));
+                g[X] = orc_fadd(g[X], lhi_F(hx, fx, ex, alpha, beta));
+            }
+        send_fe(t, &pb, "lhi_round", g, 4);
+        u64 rho = orc_tx_squeeze(t, "lhi_chal");
+        for (u64 b = 0; b < hh; b++) {
+            h[b] = orc_fadd(h[b], orc_fmul(rho, orc_fsub(h[hh + b], h[b])));
+            f[b] = orc_fadd(f[b], orc_fmul(rho, orc_fsub(f[hh + b], f[b])));
+            E[b] = orc_fadd(E[b], orc_fmul(rho, orc_fsub(E[hh + b], E[b])));
+        }
+        Lr = hh;
+    }
+    u64 fin[2] = {h[0], f[0]};
+    send_fe(t, &pb, "lhi_final", fin, 2);
+    free(m);
+    free(f);
+    free(h);
+    free(E);
+    free(z);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+int orc_lhi_verify(void* txh, const int32_t* r, u64 n, int k, const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (n < 1 || k < 1 || k > 24) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n), rc = 0;
+    if (v < 1) v = 1;
+    u64 L = (u64)1 << v, T = (u64)1 << k;
+    prd rd = {proof, len, 0, 0};
+    u32* m = (u32*)malloc(T * sizeof(u32));
+    u64* f = (u64*)malloc(L * sizeof(u64));
+    u64* h = (u64*)malloc(L * sizeof(u64));
+    u64* z = (u64*)malloc(sizeof(u64) * v);
+    u64* rho = (u64*)malloc(sizeof(u64) * v);
+    lhi_absorb_site(t, r, n);
+    rd_mult(t, &rd, "lhi_m", m, T);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    u64 alpha = orc_tx_squeeze(t, "lhi_alpha");
+    lhi_columns(r, n, v, alpha, f, h); /* the verifier holds the key column, so h too */
+    lhi_absorb_h(t, h, L);
+    for (int i = 0; i < v; i++) z[i] = orc_tx_squeeze(t, "lhi_z");
+    u64 beta = orc_tx_squeeze(t, "lhi_beta");
+    u64 S;
+    rd_fe(t, &rd, "lhi_sum", &S, 1);
+    if (rd.bad) FAIL(REJ_FORMAT, 1, 0);
+    {
+        /* the table side: sum_j m_j / (alpha - t_j), t_j = j - 2^(k-1) */
+        u64 P = 0, Q = 1;
+        for (u64 j = 0; j < T; j++) {
+            u64 dj = orc_fsub(alpha, orc_fint((int64_t)j - ((int64_t)1 << (k - 1))));
+            P = orc_fadd(orc_fmul(P, dj), orc_fmul((u64)m[j], Q));
+            Q = orc_fmul(Q, dj);
+        }
+        if (orc_fmul(S, Q) != P) FAIL(REJ_LHI_SUM, 0, 0);
+    }
+    u64 claim = S;
+    for (int i = 0; i < v; i++) {
+        u64 g[4];
+        rd_fe(t, &rd, "lhi_round", g, 4);
+        if (rd.bad) FAIL(REJ_FORMAT, 2, i);
+        if (orc_fadd(g[0], g[1]) != claim) FAIL(REJ_LHI_ROUND, i, 0);
+        rho[i] = orc_tx_squeeze(t, "lhi_chal");
+        claim = orc_lagrange(g, 4, rho[i]);
+    }
+    u64 fin[2];
+    rd_fe(t, &rd, "lhi_final", fin, 2);
+    if (rd.bad) FAIL(REJ_FORMAT, 3, 0);
+    if (lhi_F(fin[0], fin[1], eq_closed(z, rho, v), alpha, beta) != claim) FAIL(REJ_LHI_FINAL, 0, 0);
+    if (orc_mle_eval(h, L, rho, v) != fin[0]) FAIL(REJ_LHI_OPEN, 0, 0);
+    if (orc_mle_eval(f, L, rho, v) != fin[1]) FAIL(REJ_LHI_OPEN, 1, 0);
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(m);
+    free(f);
+    free(h);
+    free(z);
+    free(rho);
+    return rc;
+}

@@ -509,3 +509,53 @@ def lookup16_prove(seed: int, g, s, prefix: str, pad_s: int) -> bytes:
         z = rho_l + [tx.squeeze(prefix + "_mu")]
     send(prefix + "_leaf", [mle(gp, z), mle(sp, z)])
     return bytes(out)
+
+
+# ---- the helper-inverse LogUp -------------------------------------------------------
+
+def lhi_prove(seed: int, r, k: int) -> bytes:
+    """The helper-inverse LogUp proof from definitions: h by Python modular inverses, every
+    round value a hypercube sum of h + beta eq (h (alpha - f) - 1) over MLEs (no folding)."""
+    r = [int(x) for x in np.asarray(r).reshape(-1)]
+    n = len(r)
+    v = max(1, log2c(n))
+    L = 1 << v
+    f = [x % P for x in r] + [0] * (L - n)
+    out = bytearray()
+
+    def send(label, vals):
+        b = fe_bytes(vals)
+        out.extend(b)
+        tx.absorb(label, b)
+
+    tx = Tx(seed)
+    tx.absorb("lhi_site", tree_digest(np.asarray(r, "<i4").tobytes()))
+    m = np.zeros(1 << k, np.int64)
+    for x in r + [0] * (L - n):
+        j = x + (1 << (k - 1))
+        if 0 <= j < (1 << k):
+            m[j] += 1
+    b = m.astype("<u4").tobytes()
+    out.extend(b)
+    tx.absorb("lhi_m", tree_digest(b))
+    alpha = tx.squeeze("lhi_alpha")
+    h = [pow((alpha - x) % P, P - 2, P) for x in f]
+    tx.absorb("lhi_h", tree_digest(b"".join(struct.pack("<Q", x) for x in h)))
+    z = [tx.squeeze("lhi_z") for _ in range(v)]
+    beta = tx.squeeze("lhi_beta")
+    send("lhi_sum", [sum(h) % P])
+    rho = []
+    for t in range(v):
+        rest = v - t - 1
+        g = []
+        for X in range(4):
+            acc = 0
+            for bb in range(1 << rest):
+                w = rho + [X] + [(bb >> (rest - 1 - i)) & 1 for i in range(rest)]
+                hw, fw = mle_at(h, w), mle_at(f, w)
+                acc += hw + beta * eq_ml(z, w) * (hw * (alpha - fw) - 1)
+            g.append(acc % P)
+        send("lhi_round", g)
+        rho.append(tx.squeeze("lhi_chal"))
+    send("lhi_final", [mle_at(h, rho), mle_at(f, rho)])
+    return bytes(out)
