@@ -15,10 +15,11 @@
 // Layer d (point z of d coordinates, challenges lambda): round t sends
 // g(X) = sum_b eq(z, (rho_<t, X, b)) F(rho_<t, X, b) at X = 0..3 with
 // F = sum_tau lambda^(2 tau) (pL qR + pR qL + lambda qL qR)_tau. The kernels
-// compute h(X) = sum_b eq(z_>t, b) F(., X, b) at X = 0, 1, 2 and the last block
-// forms g(X) = eq(z_<t, rho_<t) eq(z_t, X) h(X) (h has degree 2). The vectors are
-// folded in place by the previous challenge in the same pass; the suffix eq
-// table is kept in place too (E_t[b] = E_(t-1)[b] + E_(t-1)[b + h]).
+// compute h(X) = sum_b eq(z_>t, b) F(., X, b) at X = 0 and 2 (and at 1 only when
+// z_t = 0); the host forms g(X) = eq(z_<t, rho_<t) eq(z_t, X) h(X) (h has degree
+// 2), taking g(1) from the running claim. The vectors are folded in place by the
+// previous challenge in the same pass; the suffix eq table is kept in place too
+// (E_t[b] = E_(t-1)[b] + E_(t-1)[b + h]).
 #include <string.h>
 
 #include <algorithm>
@@ -33,7 +34,7 @@ namespace {
 
 constexpr int LU_THREADS = 256;
 // The leaf layer's kernel runs 512-thread blocks (one per SM): its big rounds, read from the key
-// columns, ran about 3% faster so than as two 256-thread blocks per SM.
+// columns, ran about 3% faster that way than as two 256-thread blocks per SM.
 constexpr int LU_LEAF_THREADS = 512;
 
 struct KeySrc {
