@@ -9,9 +9,11 @@
 // The batched claim sum_s rho_s c_s is proven in n = max ceil(log2 K_s)
 // rounds of the degree-2 polynomial g(X) = sum_s rho_s sum_b A_s(X,b) B_s(X,b).
 //
-// One kernel per round: it folds the previous round's vectors by the
-// previous challenge (MSB binding) and evaluates g at 0, 1, 2 in the same
-// pass; warp shuffles + a block tree + the last block finish the sums.
+// All rounds run in one resident cooperative launch (the handshake of
+// fp_session.cuh): each round folds the previous round's vectors by the
+// previous challenge (MSB binding) and evaluates g at 0 and 2 in the same pass
+// (the host takes g(1) from the running claim); warp shuffles, a block tree and
+// the last block to finish reduce the sums. One pair per thread.
 #include <string.h>
 
 #include <algorithm>

@@ -9,9 +9,13 @@
 // per-64 group scales multiply each k-tile's partial product (one k-tile is
 // one scale group).
 //
-// Tile 128 tokens x 128 rows x 64 k, 8 warps (2 x 4), warp tile 64 x 32,
-// mma.sync m16n8k32 s8.s8.s32, 3-stage cp.async pipeline. All sites of a call
-// share one launch per operand variant (grouped GEMM over a tile list).
+// Two kernels. Unscaled sites run on tcgen05 (witness_tc_kernel: kind::i8 MMAs
+// with the accumulator in tensor memory, 128-token x 128- or 256-row tiles,
+// operands in the K-major 128-byte-swizzled layout); sites with scales, and all
+// sites when FP_TCGEN05=0, run the mma.sync kernel: tile 128 tokens x 128 rows x
+// 64 k, 8 warps (2 x 4), warp tile 64 x 32, m16n8k32 s8.s8.s32, 3-stage
+// cp.async pipeline. All sites of a call share one launch per operand variant
+// (grouped GEMM over a tile list).
 #include <vector>
 
 #include "fp_internal.h"
