@@ -147,6 +147,12 @@ def lib():
         L.orc_lhi_prove.argtypes = [vp, vp, u64, C.c_int, vp, u64, C.POINTER(u64)]
         L.orc_lhi_verify.restype = C.c_int
         L.orc_lhi_verify.argtypes = [vp, vp, u64, C.c_int, vp, u64, vp]
+        L.orc_e2_mul.argtypes = [vp, vp, vp]
+        L.orc_e2_inv.argtypes = [vp, vp]
+        L.orc_had2_prove.restype = C.c_int
+        L.orc_had2_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
+        L.orc_had2_verify.restype = C.c_int
+        L.orc_had2_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
         _lib = L
     return _lib
 
@@ -575,3 +581,53 @@ def lhi_verify(seed: int, r, k: int, proof: bytes):
     rc = L.orc_lhi_verify(tx, _ptr(a), a.size, k, _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+# ---- extension-field challenges: F_p[phi] / (phi^2 - 7) -----------------------------
+
+def e2_mul(x, y):
+    a, b, out = _u64(x), _u64(y), np.zeros(2, np.uint64)
+    lib().orc_e2_mul(_ptr(a), _ptr(b), _ptr(out))
+    return int(out[0]), int(out[1])
+
+
+def e2_inv(x):
+    a, out = _u64(x), np.zeros(2, np.uint64)
+    lib().orc_e2_inv(_ptr(a), _ptr(out))
+    return int(out[0]), int(out[1])
+
+
+def had2_prove(seed: int, s, u):
+    """The gated-product sum-check with challenges in the quadratic extension."""
+    return _lookup16_free_prove(lib().orc_had2_prove, seed, _i8(s), _i8(u))
+
+
+def had2_verify(seed: int, s, u, proof: bytes):
+    L = lib()
+    a, b = _i8(s), _i8(u)
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_had2_verify(tx, _ptr(a), _ptr(b), a.size, _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+def _lookup16_free_prove(fn, seed, a, b):
+    L = lib()
+    out = []
+    for _ in range(2):
+        tx = L.orc_tx_new(seed)
+        n = C.c_uint64(0)
+        buf = np.zeros(max(1, out[0] if out else 1), dtype=np.uint8)
+        rc = fn(tx, _ptr(a), _ptr(b), a.size, _ptr(buf) if out else None, out[0] if out else 0, C.byref(n))
+        st = C.create_string_buffer(32)
+        L.orc_tx_state(tx, st)
+        L.orc_tx_free(tx)
+        if out:
+            if rc != 0:
+                raise ValueError(f"prover failed ({rc})")
+            return buf[: n.value].tobytes(), st.raw
+        if rc not in (0, -2):
+            raise ValueError(f"prover rejected the statement ({rc})")
+        out.append(n.value)

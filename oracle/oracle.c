@@ -1941,3 +1941,217 @@ done:
     free(rho);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Extension-field challenges (next row f4): "How fast can FlashProve go",   */
+/* 4 Tighter Rooflines (a note there): for soundness the challenges live in  */
+/* an extension of the Goldilocks field. Here the quadratic extension        */
+/* F_p[phi] / (phi^2 - 7) (7 is not a square mod p), an element a + b phi    */
+/* stored as (a, b) and sent as 16 bytes (a, then b, u64 little-endian); a   */
+/* challenge is two squeezes (a, then b) under its label. First statement:  */
+/* the gated-product sum-check of section "Gated product" with every         */
+/* challenge, claim, round value and final value in the extension:           */
+/*   absorb "had2_site" D(s) || D(u); squeeze z_1..z_v ("had2_z");            */
+/*   send c ("had2_claim"); rounds g(0..3) ("had2_round"), "had2_chal";       */
+/*   send S(rho), U(rho) ("had2_final").                                      */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    u64 a, b;
+} ext2;
+
+static ext2 e2(u64 a, u64 b) { ext2 r = {a, b}; return r; }
+static ext2 e2_add(ext2 x, ext2 y) { return e2(orc_fadd(x.a, y.a), orc_fadd(x.b, y.b)); }
+static ext2 e2_sub(ext2 x, ext2 y) { return e2(orc_fsub(x.a, y.a), orc_fsub(x.b, y.b)); }
+static ext2 e2_mul(ext2 x, ext2 y) { /* (a + b phi)(c + d phi) = ac + 7 bd + (ad + bc) phi */
+    return e2(orc_fadd(orc_fmul(x.a, y.a), orc_fmul(7, orc_fmul(x.b, y.b))),
+              orc_fadd(orc_fmul(x.a, y.b), orc_fmul(x.b, y.a)));
+}
+static ext2 e2_scal(ext2 x, u64 k) { return e2(orc_fmul(x.a, k), orc_fmul(x.b, k)); }
+
+/* ctypes-facing multiplication and inverse (for the pins) */
+void orc_e2_mul(const u64 x[2], const u64 y[2], u64 out[2]) {
+    ext2 r = e2_mul(e2(x[0], x[1]), e2(y[0], y[1]));
+    out[0] = r.a;
+    out[1] = r.b;
+}
+void orc_e2_inv(const u64 x[2], u64 out[2]) { /* 1 / (a + b phi) = (a - b phi) / (a^2 - 7 b^2) */
+    u64 n = orc_fsub(orc_fmul(x[0], x[0]), orc_fmul(7, orc_fmul(x[1], x[1])));
+    u64 ni = orc_finv(n);
+    out[0] = orc_fmul(x[0], ni);
+    out[1] = orc_fsub(0, orc_fmul(x[1], ni));
+}
+
+static ext2 e2_squeeze(orc_tx* t, const char* label) {
+    u64 a = orc_tx_squeeze(t, label);
+    u64 b = orc_tx_squeeze(t, label);
+    return e2(a, b);
+}
+
+static void e2_send(orc_tx* t, pbuf* pb, const char* label, const ext2* v, u64 n) {
+    u64* w = (u64*)malloc(sizeof(u64) * 2 * (n ? n : 1));
+    for (u64 i = 0; i < n; i++) {
+        w[2 * i] = v[i].a;
+        w[2 * i + 1] = v[i].b;
+    }
+    send_fe(t, pb, label, w, 2 * n);
+    free(w);
+}
+
+static void e2_read(orc_tx* t, prd* rd, const char* label, ext2* v, u64 n) {
+    u64* w = (u64*)malloc(sizeof(u64) * 2 * (n ? n : 1));
+    rd_fe(t, rd, label, w, 2 * n);
+    for (u64 i = 0; i < n; i++) v[i] = e2(w[2 * i], w[2 * i + 1]);
+    free(w);
+}
+
+/* eq table of an extension point by doubling (z_1 on the most significant bit) */
+static void e2_eq_table(const ext2* z, int v, ext2* out) {
+    out[0] = e2(1, 0);
+    for (int b = 0; b < v; b++) {
+        u64 len = (u64)1 << b;
+        for (u64 j = len; j-- > 0;) {
+            ext2 o = out[j];
+            out[2 * j] = e2_mul(o, e2_sub(e2(1, 0), z[b]));
+            out[2 * j + 1] = e2_mul(o, z[b]);
+        }
+    }
+}
+
+/* the degree-3 polynomial through (i, g[i]), i = 0..3, at r */
+static ext2 e2_lagrange4(const ext2 g[4], ext2 r) {
+    ext2 acc = e2(0, 0);
+    for (int i = 0; i < 4; i++) {
+        ext2 num = e2(1, 0);
+        int64_t den = 1;
+        for (int j = 0; j < 4; j++) {
+            if (j == i) continue;
+            num = e2_mul(num, e2_sub(r, e2((u64)j, 0)));
+            den *= (int64_t)(i - j);
+        }
+        acc = e2_add(acc, e2_mul(g[i], e2_scal(num, orc_finv(orc_fint(den)))));
+    }
+    return acc;
+}
+
+int orc_had2_prove(void* txh, const int8_t* s, const int8_t* u, u64 n, uint8_t* proof, u64 cap, u64* len) {
+    if (n < 1) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n);
+    u64 sz = (u64)1 << v;
+    pbuf pb = {proof, cap, 0, 0};
+    uint8_t d[64];
+    orc_tree_digest(s, n, d);
+    orc_tree_digest(u, n, d + 32);
+    orc_tx_absorb(t, "had2_site", d, 64);
+    ext2* z = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    for (int i = 0; i < v; i++) z[i] = e2_squeeze(t, "had2_z");
+    ext2* E = (ext2*)malloc(sizeof(ext2) * sz);
+    ext2* S = (ext2*)malloc(sizeof(ext2) * sz);
+    ext2* U = (ext2*)malloc(sizeof(ext2) * sz);
+    e2_eq_table(z, v, E);
+    for (u64 x = 0; x < sz; x++) {
+        S[x] = e2(x < n ? orc_fint(s[x]) : 0, 0);
+        U[x] = e2(x < n ? orc_fint(u[x]) : 0, 0);
+    }
+    ext2 c = e2(0, 0);
+    for (u64 x = 0; x < sz; x++) c = e2_add(c, e2_mul(E[x], e2_mul(S[x], U[x])));
+    e2_send(t, &pb, "had2_claim", &c, 1);
+    u64 L = sz;
+    for (int r = 0; r < v; r++) {
+        u64 h = L >> 1;
+        ext2 g[4] = {e2(0, 0), e2(0, 0), e2(0, 0), e2(0, 0)};
+        for (u64 b = 0; b < h; b++)
+            for (u64 X = 0; X < 4; X++) {
+                ext2 ex = e2_add(E[b], e2_scal(e2_sub(E[h + b], E[b]), X));
+                ext2 sx = e2_add(S[b], e2_scal(e2_sub(S[h + b], S[b]), X));
+                ext2 ux = e2_add(U[b], e2_scal(e2_sub(U[h + b], U[b]), X));
+                g[X] = e2_add(g[X], e2_mul(ex, e2_mul(sx, ux)));
+            }
+        e2_send(t, &pb, "had2_round", g, 4);
+        ext2 rho = e2_squeeze(t, "had2_chal");
+        for (u64 b = 0; b < h; b++) {
+            E[b] = e2_add(E[b], e2_mul(rho, e2_sub(E[h + b], E[b])));
+            S[b] = e2_add(S[b], e2_mul(rho, e2_sub(S[h + b], S[b])));
+            U[b] = e2_add(U[b], e2_mul(rho, e2_sub(U[h + b], U[b])));
+        }
+        L = h;
+    }
+    ext2 fin[2] = {S[0], U[0]};
+    e2_send(t, &pb, "had2_final", fin, 2);
+    free(z);
+    free(E);
+    free(S);
+    free(U);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+/* MLE at an extension point of a base-field vector (zero-padded to 2^v) */
+static ext2 e2_mle(const int8_t* a, u64 n, const ext2* z, int v) {
+    u64 sz = (u64)1 << v;
+    ext2* E = (ext2*)malloc(sizeof(ext2) * sz);
+    e2_eq_table(z, v, E);
+    ext2 acc = e2(0, 0);
+    for (u64 x = 0; x < n && x < sz; x++) acc = e2_add(acc, e2_scal(E[x], orc_fint(a[x])));
+    free(E);
+    return acc;
+}
+
+int orc_had2_verify(void* txh, const int8_t* s, const int8_t* u, u64 n, const uint8_t* proof, u64 len,
+                    int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (n < 1) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n), rc = 0;
+    u64 sz = (u64)1 << v;
+    prd rd = {proof, len, 0, 0};
+    uint8_t d[64];
+    orc_tree_digest(s, n, d);
+    orc_tree_digest(u, n, d + 32);
+    orc_tx_absorb(t, "had2_site", d, 64);
+    ext2* z = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    ext2* rho = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    ext2* E = (ext2*)malloc(sizeof(ext2) * sz);
+    for (int i = 0; i < v; i++) z[i] = e2_squeeze(t, "had2_z");
+    ext2 c, claim;
+    e2_read(t, &rd, "had2_claim", &c, 1);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    {
+        e2_eq_table(z, v, E);
+        ext2 want = e2(0, 0);
+        for (u64 x = 0; x < n; x++) want = e2_add(want, e2_scal(E[x], orc_fmul(orc_fint(s[x]), orc_fint(u[x]))));
+        if (want.a != c.a || want.b != c.b) FAIL(REJ_HAD_CLAIM, 0, 0);
+    }
+    claim = c;
+    for (int r = 0; r < v; r++) {
+        ext2 g[4];
+        e2_read(t, &rd, "had2_round", g, 4);
+        if (rd.bad) FAIL(REJ_FORMAT, r, 0);
+        ext2 s01 = e2_add(g[0], g[1]);
+        if (s01.a != claim.a || s01.b != claim.b) FAIL(REJ_HAD_ROUND, r, 0);
+        rho[r] = e2_squeeze(t, "had2_chal");
+        claim = e2_lagrange4(g, rho[r]);
+    }
+    ext2 fin[2];
+    e2_read(t, &rd, "had2_final", fin, 2);
+    if (rd.bad) FAIL(REJ_FORMAT, v, 0);
+    {
+        ext2 e = e2(1, 0);
+        for (int i = 0; i < v; i++)
+            e = e2_mul(e, e2_add(e2_mul(z[i], rho[i]), e2_mul(e2_sub(e2(1, 0), z[i]), e2_sub(e2(1, 0), rho[i]))));
+        ext2 end = e2_mul(e, e2_mul(fin[0], fin[1]));
+        if (end.a != claim.a || end.b != claim.b) FAIL(REJ_HAD_FINAL, 0, 0);
+    }
+    {
+        ext2 ws = e2_mle(s, n, rho, v), wu = e2_mle(u, n, rho, v);
+        if (ws.a != fin[0].a || ws.b != fin[0].b) FAIL(REJ_HAD_OPEN, 0, 0);
+        if (wu.a != fin[1].a || wu.b != fin[1].b) FAIL(REJ_HAD_OPEN, 1, 0);
+    }
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(z);
+    free(rho);
+    free(E);
+    return rc;
+}

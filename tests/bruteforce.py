@@ -559,3 +559,77 @@ def lhi_prove(seed: int, r, k: int) -> bytes:
         rho.append(tx.squeeze("lhi_chal"))
     send("lhi_final", [mle_at(h, rho), mle_at(f, rho)])
     return bytes(out)
+
+
+# ---- extension-field challenges: F_p[phi] / (phi^2 - 7) -----------------------------
+
+def x_mul(x, y):
+    """(a + b phi)(c + d phi) with phi^2 = 7, as polynomials reduced mod phi^2 - 7."""
+    a, b = x
+    c, d = y
+    return ((a * c + 7 * b * d) % P, (a * d + b * c) % P)
+
+
+def x_add(x, y):
+    return ((x[0] + y[0]) % P, (x[1] + y[1]) % P)
+
+
+def x_eq(z, w):
+    acc = (1, 0)
+    for zi, wi in zip(z, w):
+        one_z, one_w = ((1 - zi[0]) % P, (-zi[1]) % P), ((1 - wi[0]) % P, (-wi[1]) % P)
+        acc = x_mul(acc, x_add(x_mul(zi, wi), x_mul(one_z, one_w)))
+    return acc
+
+
+def x_mle(vals, w):
+    v = len(w)
+    acc = (0, 0)
+    for x in range(min(len(vals), 1 << v)):
+        bits = [((x >> (v - 1 - b)) & 1, 0) for b in range(v)]
+        e = x_eq(w, bits)
+        acc = x_add(acc, (e[0] * (int(vals[x]) % P) % P, e[1] * (int(vals[x]) % P) % P))
+    return acc
+
+
+def had2_prove(seed: int, s, u) -> bytes:
+    """The extension-field gated-product proof from definitions (hypercube sums, no folding)."""
+    s = [int(x) for x in np.asarray(s).reshape(-1)]
+    u = [int(x) for x in np.asarray(u).reshape(-1)]
+    n = len(s)
+    v = log2c(n)
+    tx = Tx(seed)
+    tx.absorb("had2_site", tree_digest(np.asarray(s, np.int8).tobytes()) + tree_digest(np.asarray(u, np.int8).tobytes()))
+    z = []
+    for _ in range(v):
+        a = tx.squeeze("had2_z")
+        z.append((a, tx.squeeze("had2_z")))
+    out = bytearray()
+
+    def send(label, xs):
+        b = fe_bytes([c for x in xs for c in x])
+        out.extend(b)
+        tx.absorb(label, b)
+
+    c = (0, 0)
+    for x in range(n):
+        bits = [((x >> (v - 1 - b)) & 1, 0) for b in range(v)]
+        e = x_eq(z, bits)
+        pr = s[x] * u[x] % P
+        c = x_add(c, (e[0] * pr % P, e[1] * pr % P))
+    send("had2_claim", [c])
+    rho = []
+    for t in range(v):
+        rest = v - t - 1
+        g = []
+        for X in range(4):
+            acc = (0, 0)
+            for bb in range(1 << rest):
+                w = rho + [(X, 0)] + [((bb >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                acc = x_add(acc, x_mul(x_eq(z, w), x_mul(x_mle(s, w), x_mle(u, w))))
+            g.append(acc)
+        send("had2_round", g)
+        a = tx.squeeze("had2_chal")
+        rho.append((a, tx.squeeze("had2_chal")))
+    send("had2_final", [x_mle(s, rho), x_mle(u, rho)])
+    return bytes(out)

@@ -1,0 +1,80 @@
+"""Extension-field challenges in the oracle (next row f4), pinned.
+
+"How fast can FlashProve go", 4 Tighter Rooflines: for soundness the
+challenges are drawn from an extension of the Goldilocks field. The quadratic
+extension F_p[phi] / (phi^2 - 7): the arithmetic is pinned by the field's laws
+(7 is a non-residue, so every nonzero element is invertible), and the
+gated-product sum-check with extension challenges byte for byte against a
+brute-force restatement with its own extension arithmetic (Python integers).
+"""
+
+import random
+import struct
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import bruteforce as bf
+
+P = oracle.P
+
+
+def test_seven_is_not_a_square():
+    assert pow(7, (P - 1) // 2, P) == P - 1
+
+
+def test_arithmetic():
+    rnd = random.Random(4)
+    for _ in range(200):
+        x = (rnd.randrange(P), rnd.randrange(P))
+        y = (rnd.randrange(P), rnd.randrange(P))
+        assert oracle.e2_mul(x, y) == bf.x_mul(x, y)
+        if x != (0, 0):
+            assert oracle.e2_mul(x, oracle.e2_inv(x)) == (1, 0)
+    # phi^2 = 7; the base field embeds as (a, 0)
+    assert oracle.e2_mul((0, 1), (0, 1)) == (7, 0)
+    assert oracle.e2_mul((3, 0), (5, 0)) == (15, 0)
+
+
+def _vecs(n, seed):
+    rng = np.random.default_rng(seed)
+    return rng.integers(-128, 128, n).astype(np.int8), rng.integers(-128, 128, n).astype(np.int8)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 8])
+def test_bytes_match_bruteforce(n):
+    s, u = _vecs(n, n)
+    pf, _ = oracle.had2_prove(2, s, u)
+    assert pf == bf.had2_prove(2, s, u)
+    assert len(pf) == 16 + 64 * bf.log2c(n) + 32
+
+
+@pytest.mark.parametrize("n", [1, 100, 1000])
+def test_honest_proof_accepted(n):
+    s, u = _vecs(n, 9 + n)
+    pf, _ = oracle.had2_prove(3, s, u)
+    assert oracle.had2_verify(3, s, u, pf) == ("accept", (0, 0))
+
+
+def _put(pf, off, val):
+    return pf[:off] + struct.pack("<Q", val % P) + pf[off + 8:]
+
+
+def test_each_check_fires():
+    s, u = _vecs(40, 5)
+    pf, _ = oracle.had2_prove(1, s, u)
+    c_im = struct.unpack("<Q", pf[8:16])[0]
+    assert oracle.had2_verify(1, s, u, _put(pf, 8, c_im + 1))[0] == "had_claim"
+    r0 = 16 + 8  # round 1, g(0)'s second coordinate
+    x = struct.unpack("<Q", pf[r0:r0 + 8])[0]
+    assert oracle.had2_verify(1, s, u, _put(pf, r0, x + 1)) == ("had_round", (0, 0))
+    fo = len(pf) - 32
+    a = struct.unpack("<Q", pf[fo:fo + 8])[0]
+    assert oracle.had2_verify(1, s, u, _put(pf, fo, a + 1))[0] == "had_final"
+    s2 = s.copy()
+    s2[0] ^= 1
+    assert oracle.had2_verify(1, s2, u, pf)[0] != "accept"
+    # the base-field statement is a different one: its proof does not verify here
+    pf_base, _ = oracle.had_prove(1, s, u)
+    assert oracle.had2_verify(1, s, u, pf_base)[0] != "accept"
