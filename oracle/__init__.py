@@ -56,6 +56,8 @@ REASONS = {
     25: "lookup_final",
     26: "lookup_leaf",
     27: "lookup_open",
+    32: "frv_u",
+    33: "frv_row",
     28: "lhi_sum",
     29: "lhi_round",
     30: "lhi_final",
@@ -153,6 +155,10 @@ def lib():
         L.orc_had2_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
         L.orc_had2_verify.restype = C.c_int
         L.orc_had2_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
+        L.orc_frv_prove.restype = C.c_int
+        L.orc_frv_prove.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, C.POINTER(u64)]
+        L.orc_frv_verify.restype = C.c_int
+        L.orc_frv_verify.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, vp]
         _lib = L
     return _lib
 
@@ -631,3 +637,41 @@ def _lookup16_free_prove(fn, seed, a, b):
         if rc not in (0, -2):
             raise ValueError(f"prover rejected the statement ({rc})")
         out.append(n.value)
+
+
+# ---- the Freivalds check of a weight matmul (a comparison statement) ------------------
+
+def frv_prove(seed: int, site, wit):
+    """Freivalds proof of one site: u = X rho^(.) sent after absorbing the site's digests."""
+    L = lib()
+    keep = []
+    cs = _csite(site, keep)
+    q, r, y = (np.ascontiguousarray(a) for a in wit)
+    cw = _Wit(_ptr(q), _ptr(r), _ptr(y))
+    n = C.c_uint64(0)
+    tx = L.orc_tx_new(seed)
+    L.orc_frv_prove(tx, C.byref(cs), C.byref(cw), None, 0, C.byref(n))
+    L.orc_tx_free(tx)
+    buf = np.zeros(max(1, n.value), dtype=np.uint8)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_frv_prove(tx, C.byref(cs), C.byref(cw), _ptr(buf), n.value, C.byref(n))
+    st = C.create_string_buffer(32)
+    L.orc_tx_state(tx, st)
+    L.orc_tx_free(tx)
+    if rc != 0:
+        raise ValueError(f"orc_frv_prove failed ({rc})")
+    return buf[: n.value].tobytes(), st.raw
+
+
+def frv_verify(seed: int, site, wit, proof: bytes):
+    L = lib()
+    keep = []
+    cs = _csite(site, keep)
+    q, r, y = (np.ascontiguousarray(a) for a in wit)
+    cw = _Wit(_ptr(q), _ptr(r), _ptr(y))
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_frv_verify(tx, C.byref(cs), C.byref(cw), _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

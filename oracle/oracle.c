@@ -2155,3 +2155,99 @@ done:
     free(E);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* The Freivalds check of a weight matmul (next row f4, the comparison      */
+/* statement): "Towards Proving Frontier-Scale LLM Inference", The proof     */
+/* system -- instead of recomputing C = A B, check A (B r) = C r for a random */
+/* vector r. Here, for one site Y = W_eff X with Y = 2^k q + r standing in    */
+/* for the unrounded product (the committed witness):                        */
+/*   absorb "frv_site" D(W) || D(S) || D(Xt) || D(q) || D(r);                 */
+/*   squeeze rho ("frv_rho"); the vector over tokens is rho^j, j < N;         */
+/*   send u = X rho^(.) (K values, "frv_u"): u_k = sum_j X[k][j] rho^j.        */
+/* The verifier checks u against X and W_eff u = Y rho^(.) row by row: a     */
+/* wrong witness row makes a nonzero polynomial of degree < N in rho vanish, */
+/* probability below N / p.                                                   */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_FRV_U = 32,   /* u != X rho^(.) */
+    REJ_FRV_ROW = 33  /* (W_eff u)_i != (Y rho^(.))_i; detail[0] = i */
+};
+
+static void frv_absorb(orc_tx* t, const orc_site* s, const orc_wit* w) {
+    uint8_t d[160];
+    u64 mn = (u64)s->M * s->N;
+    uint8_t* qb = (uint8_t*)calloc(4 * mn + 1, 1);
+    uint8_t* rb = (uint8_t*)calloc(4 * mn + 1, 1);
+    for (u64 i = 0; i < mn; i++) {
+        put_le(qb + 4 * i, (u64)(u32)w->q[i], 4);
+        put_le(rb + 4 * i, (u64)(u32)w->r[i], 4);
+    }
+    orc_tree_digest(s->w, site_w_bytes(s), d);
+    orc_tree_digest(s->scales, s->scales ? (u64)s->M * ((s->K + 63) / 64) : 0, d + 32);
+    orc_tree_digest(s->xt, (u64)s->N * s->K, d + 64);
+    orc_tree_digest(qb, 4 * mn, d + 96);
+    orc_tree_digest(rb, 4 * mn, d + 128);
+    free(qb);
+    free(rb);
+    orc_tx_absorb(t, "frv_site", d, 160);
+}
+
+/* u_k = sum_j X[k][j] rho^j, X[k][j] = xt[j][k] */
+static void frv_u(const orc_site* s, u64 rho, u64* u) {
+    for (int k = 0; k < s->K; k++) u[k] = 0;
+    u64 pw = 1;
+    for (int j = 0; j < s->N; j++) {
+        for (int k = 0; k < s->K; k++) u[k] = orc_fadd(u[k], orc_fmul(orc_fint(s->xt[(u64)j * s->K + k]), pw));
+        pw = orc_fmul(pw, rho);
+    }
+}
+
+int orc_frv_prove(void* txh, const orc_site* s, const orc_wit* w, uint8_t* proof, u64 cap, u64* len) {
+    if (s->M < 1 || s->N < 1 || s->K < 1) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    pbuf pb = {proof, cap, 0, 0};
+    frv_absorb(t, s, w);
+    u64 rho = orc_tx_squeeze(t, "frv_rho");
+    u64* u = (u64*)malloc(sizeof(u64) * s->K);
+    frv_u(s, rho, u);
+    send_fe(t, &pb, "frv_u", u, (u64)s->K);
+    free(u);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+int orc_frv_verify(void* txh, const orc_site* s, const orc_wit* w, const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (s->M < 1 || s->N < 1 || s->K < 1) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int rc = 0;
+    prd rd = {proof, len, 0, 0};
+    u64* u = (u64*)malloc(sizeof(u64) * s->K);
+    u64* want = (u64*)malloc(sizeof(u64) * s->K);
+    frv_absorb(t, s, w);
+    u64 rho = orc_tx_squeeze(t, "frv_rho");
+    rd_fe(t, &rd, "frv_u", u, (u64)s->K);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    frv_u(s, rho, want);
+    for (int k = 0; k < s->K; k++)
+        if (u[k] != want[k]) FAIL(REJ_FRV_U, k, 0);
+    for (int i = 0; i < s->M; i++) {
+        u64 lhs = 0, rhs = 0, pw = 1;
+        for (int k = 0; k < s->K; k++) lhs = orc_fadd(lhs, orc_fmul(orc_fint(w_eff(s, i, k)), u[k]));
+        for (int j = 0; j < s->N; j++) {
+            /* Y[i][j] = 2^k q + r, witness stored token-major (N x M) */
+            u64 y = orc_fadd(orc_fmul(orc_fint((int64_t)1 << s->k_shift), orc_fint(w->q[(u64)j * s->M + i])),
+                             orc_fint(w->r[(u64)j * s->M + i]));
+            rhs = orc_fadd(rhs, orc_fmul(y, pw));
+            pw = orc_fmul(pw, rho);
+        }
+        if (lhs != rhs) FAIL(REJ_FRV_ROW, i, 0);
+    }
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(u);
+    free(want);
+    return rc;
+}
