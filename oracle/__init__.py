@@ -159,6 +159,10 @@ def lib():
         L.orc_frv_prove.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, C.POINTER(u64)]
         L.orc_frv_verify.restype = C.c_int
         L.orc_frv_verify.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, vp]
+        L.orc_mm2_prove.restype = C.c_int
+        L.orc_mm2_prove.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, C.POINTER(u64)]
+        L.orc_mm2_verify.restype = C.c_int
+        L.orc_mm2_verify.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, vp]
         _lib = L
     return _lib
 
@@ -643,6 +647,23 @@ def _lookup16_free_prove(fn, seed, a, b):
 
 def frv_prove(seed: int, site, wit):
     """Freivalds proof of one site: u = X rho^(.) sent after absorbing the site's digests."""
+    return _site_prove(lib().orc_frv_prove, seed, site, wit)
+
+
+def frv_verify(seed: int, site, wit, proof: bytes):
+    return _site_verify(lib().orc_frv_verify, seed, site, wit, proof)
+
+
+def mm2_prove(seed: int, site, wit):
+    """The matmul sum-check of one site with challenges in the quadratic extension."""
+    return _site_prove(lib().orc_mm2_prove, seed, site, wit)
+
+
+def mm2_verify(seed: int, site, wit, proof: bytes):
+    return _site_verify(lib().orc_mm2_verify, seed, site, wit, proof)
+
+
+def _site_prove(fn, seed: int, site, wit):
     L = lib()
     keep = []
     cs = _csite(site, keep)
@@ -650,20 +671,20 @@ def frv_prove(seed: int, site, wit):
     cw = _Wit(_ptr(q), _ptr(r), _ptr(y))
     n = C.c_uint64(0)
     tx = L.orc_tx_new(seed)
-    L.orc_frv_prove(tx, C.byref(cs), C.byref(cw), None, 0, C.byref(n))
+    fn(tx, C.byref(cs), C.byref(cw), None, 0, C.byref(n))
     L.orc_tx_free(tx)
     buf = np.zeros(max(1, n.value), dtype=np.uint8)
     tx = L.orc_tx_new(seed)
-    rc = L.orc_frv_prove(tx, C.byref(cs), C.byref(cw), _ptr(buf), n.value, C.byref(n))
+    rc = fn(tx, C.byref(cs), C.byref(cw), _ptr(buf), n.value, C.byref(n))
     st = C.create_string_buffer(32)
     L.orc_tx_state(tx, st)
     L.orc_tx_free(tx)
     if rc != 0:
-        raise ValueError(f"orc_frv_prove failed ({rc})")
+        raise ValueError(f"prover failed ({rc})")
     return buf[: n.value].tobytes(), st.raw
 
 
-def frv_verify(seed: int, site, wit, proof: bytes):
+def _site_verify(fn, seed: int, site, wit, proof: bytes):
     L = lib()
     keep = []
     cs = _csite(site, keep)
@@ -672,6 +693,6 @@ def frv_verify(seed: int, site, wit, proof: bytes):
     pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
     det = np.zeros(2, dtype=np.int64)
     tx = L.orc_tx_new(seed)
-    rc = L.orc_frv_verify(tx, C.byref(cs), C.byref(cw), _ptr(pb), len(proof), _ptr(det))
+    rc = fn(tx, C.byref(cs), C.byref(cw), _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

@@ -2175,8 +2175,8 @@ enum {
     REJ_FRV_ROW = 33  /* (W_eff u)_i != (Y rho^(.))_i; detail[0] = i */
 };
 
-static void frv_absorb(orc_tx* t, const orc_site* s, const orc_wit* w) {
-    uint8_t d[160];
+/* D(W) || D(S) || D(Xt) || D(q) || D(r) of one site */
+static void site_digest160(const orc_site* s, const orc_wit* w, uint8_t d[160]) {
     u64 mn = (u64)s->M * s->N;
     uint8_t* qb = (uint8_t*)calloc(4 * mn + 1, 1);
     uint8_t* rb = (uint8_t*)calloc(4 * mn + 1, 1);
@@ -2191,6 +2191,11 @@ static void frv_absorb(orc_tx* t, const orc_site* s, const orc_wit* w) {
     orc_tree_digest(rb, 4 * mn, d + 128);
     free(qb);
     free(rb);
+}
+
+static void frv_absorb(orc_tx* t, const orc_site* s, const orc_wit* w) {
+    uint8_t d[160];
+    site_digest160(s, w, d);
     orc_tx_absorb(t, "frv_site", d, 160);
 }
 
@@ -2249,5 +2254,169 @@ int orc_frv_verify(void* txh, const orc_site* s, const orc_wit* w, const uint8_t
 done:
     free(u);
     free(want);
+    return rc;
+}
+
+/* The matmul sum-check of one site with extension-field challenges (next    */
+/* row f4): the statement of the matmul section for a single site, every     */
+/* challenge and every sent value in F_p[phi] / (phi^2 - 7):                  */
+/*   absorb "mm2_site" D(W) || D(S) || D(Xt) || D(q) || D(r);                  */
+/*   squeeze r_row (vM coordinates, "mm2_row") and r_col (vN, "mm2_col");      */
+/*   send c = Y~(r_row, r_col), Y = 2^k q + r ("mm2_claim");                   */
+/*   A[k] = W_eff~(r_row, k), B[k] = X~(k, r_col) over K padded to 2^n;         */
+/*   n rounds of g(0), g(1), g(2) of sum_b A(X, b) B(X, b) ("mm2_round"),      */
+/*   "mm2_chal"; send A(rho), B(rho) ("mm2_final").                            */
+
+static ext2 e2_lagrange3(const ext2 g[3], ext2 r) {
+    ext2 acc = e2(0, 0);
+    for (int i = 0; i < 3; i++) {
+        ext2 num = e2(1, 0);
+        int64_t den = 1;
+        for (int j = 0; j < 3; j++) {
+            if (j == i) continue;
+            num = e2_mul(num, e2_sub(r, e2((u64)j, 0)));
+            den *= (int64_t)(i - j);
+        }
+        acc = e2_add(acc, e2_mul(g[i], e2_scal(num, orc_finv(orc_fint(den)))));
+    }
+    return acc;
+}
+
+/* c, A, B of the site at (r_row, r_col); A, B of length 2^n */
+static ext2 mm2_vectors(const orc_site* s, const orc_wit* w, const ext2* zr, int vM, const ext2* zc, int vN, int n,
+                        ext2* A, ext2* B) {
+    u64 Mp = (u64)1 << vM, Np = (u64)1 << vN, L = (u64)1 << n;
+    ext2* er = (ext2*)malloc(sizeof(ext2) * Mp);
+    ext2* ec = (ext2*)malloc(sizeof(ext2) * Np);
+    e2_eq_table(zr, vM, er);
+    e2_eq_table(zc, vN, ec);
+    for (u64 k = 0; k < L; k++) A[k] = B[k] = e2(0, 0);
+    for (int i = 0; i < s->M; i++)
+        for (int k = 0; k < s->K; k++) A[k] = e2_add(A[k], e2_scal(er[i], orc_fint(w_eff(s, i, k))));
+    for (int j = 0; j < s->N; j++)
+        for (int k = 0; k < s->K; k++) B[k] = e2_add(B[k], e2_scal(ec[j], orc_fint(s->xt[(u64)j * s->K + k])));
+    ext2 c = e2(0, 0);
+    for (int i = 0; i < s->M; i++)
+        for (int j = 0; j < s->N; j++) {
+            u64 y = orc_fadd(orc_fmul(orc_fint((int64_t)1 << s->k_shift), orc_fint(w->q[(u64)j * s->M + i])),
+                             orc_fint(w->r[(u64)j * s->M + i]));
+            c = e2_add(c, e2_scal(e2_mul(er[i], ec[j]), y));
+        }
+    free(er);
+    free(ec);
+    return c;
+}
+
+int orc_mm2_prove(void* txh, const orc_site* s, const orc_wit* w, uint8_t* proof, u64 cap, u64* len) {
+    if (s->M < 1 || s->N < 1 || s->K < 1) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int vM = orc_log2_ceil((u64)s->M), vN = orc_log2_ceil((u64)s->N), n = orc_log2_ceil((u64)s->K);
+    u64 L = (u64)1 << n;
+    pbuf pb = {proof, cap, 0, 0};
+    {
+        uint8_t d[160];
+        site_digest160(s, w, d);
+        orc_tx_absorb(t, "mm2_site", d, 160);
+    }
+    ext2* zr = (ext2*)malloc(sizeof(ext2) * (vM + 1));
+    ext2* zc = (ext2*)malloc(sizeof(ext2) * (vN + 1));
+    for (int i = 0; i < vM; i++) zr[i] = e2_squeeze(t, "mm2_row");
+    for (int i = 0; i < vN; i++) zc[i] = e2_squeeze(t, "mm2_col");
+    ext2* A = (ext2*)malloc(sizeof(ext2) * L);
+    ext2* B = (ext2*)malloc(sizeof(ext2) * L);
+    ext2 c = mm2_vectors(s, w, zr, vM, zc, vN, n, A, B);
+    e2_send(t, &pb, "mm2_claim", &c, 1);
+    u64 Lr = L;
+    for (int r = 0; r < n; r++) {
+        u64 h = Lr >> 1;
+        ext2 g[3] = {e2(0, 0), e2(0, 0), e2(0, 0)};
+        for (u64 b = 0; b < h; b++)
+            for (u64 X = 0; X < 3; X++) {
+                ext2 ax = e2_add(A[b], e2_scal(e2_sub(A[h + b], A[b]), X));
+                ext2 bx = e2_add(B[b], e2_scal(e2_sub(B[h + b], B[b]), X));
+                g[X] = e2_add(g[X], e2_mul(ax, bx));
+            }
+        e2_send(t, &pb, "mm2_round", g, 3);
+        ext2 rho = e2_squeeze(t, "mm2_chal");
+        for (u64 b = 0; b < h; b++) {
+            A[b] = e2_add(A[b], e2_mul(rho, e2_sub(A[h + b], A[b])));
+            B[b] = e2_add(B[b], e2_mul(rho, e2_sub(B[h + b], B[b])));
+        }
+        Lr = h;
+    }
+    ext2 fin[2] = {A[0], B[0]};
+    e2_send(t, &pb, "mm2_final", fin, 2);
+    free(zr);
+    free(zc);
+    free(A);
+    free(B);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+/* Verifier: the claim against Y, every round (g(0) + g(1) = claim, the next
+ * claim g(rho) through the nodes 0, 1, 2), the end A(rho) B(rho) = claim, and
+ * A(rho), B(rho) against the MLEs of W_eff and X it recomputes. */
+int orc_mm2_verify(void* txh, const orc_site* s, const orc_wit* w, const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (s->M < 1 || s->N < 1 || s->K < 1) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int vM = orc_log2_ceil((u64)s->M), vN = orc_log2_ceil((u64)s->N), n = orc_log2_ceil((u64)s->K), rc = 0;
+    u64 L = (u64)1 << n;
+    prd rd = {proof, len, 0, 0};
+    {
+        uint8_t d[160];
+        site_digest160(s, w, d);
+        orc_tx_absorb(t, "mm2_site", d, 160);
+    }
+    ext2* zr = (ext2*)malloc(sizeof(ext2) * (vM + 1));
+    ext2* zc = (ext2*)malloc(sizeof(ext2) * (vN + 1));
+    ext2* rho = (ext2*)malloc(sizeof(ext2) * (n + 1));
+    ext2* A = (ext2*)malloc(sizeof(ext2) * L);
+    ext2* B = (ext2*)malloc(sizeof(ext2) * L);
+    ext2* E = (ext2*)malloc(sizeof(ext2) * L);
+    for (int i = 0; i < vM; i++) zr[i] = e2_squeeze(t, "mm2_row");
+    for (int i = 0; i < vN; i++) zc[i] = e2_squeeze(t, "mm2_col");
+    ext2 want = mm2_vectors(s, w, zr, vM, zc, vN, n, A, B);
+    ext2 c, claim;
+    e2_read(t, &rd, "mm2_claim", &c, 1);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    if (c.a != want.a || c.b != want.b) FAIL(REJ_CLAIM, 0, 0);
+    claim = c;
+    for (int r = 0; r < n; r++) {
+        ext2 g[3];
+        e2_read(t, &rd, "mm2_round", g, 3);
+        if (rd.bad) FAIL(REJ_FORMAT, 1, r);
+        ext2 s01 = e2_add(g[0], g[1]);
+        if (s01.a != claim.a || s01.b != claim.b) FAIL(REJ_MM_ROUND, r, 0);
+        rho[r] = e2_squeeze(t, "mm2_chal");
+        claim = e2_lagrange3(g, rho[r]);
+    }
+    ext2 fin[2];
+    e2_read(t, &rd, "mm2_final", fin, 2);
+    if (rd.bad) FAIL(REJ_FORMAT, 2, 0);
+    {
+        ext2 end = e2_mul(fin[0], fin[1]);
+        if (end.a != claim.a || end.b != claim.b) FAIL(REJ_MM_FINAL, 0, 0);
+    }
+    {
+        /* A(rho) = sum_k eq(rho, k) A[k] with A recomputed from W_eff (likewise B from X) */
+        e2_eq_table(rho, n, E);
+        ext2 a = e2(0, 0), b = e2(0, 0);
+        for (u64 k = 0; k < L; k++) {
+            a = e2_add(a, e2_mul(E[k], A[k]));
+            b = e2_add(b, e2_mul(E[k], B[k]));
+        }
+        if (a.a != fin[0].a || a.b != fin[0].b) FAIL(REJ_MM_A, 0, 0);
+        if (b.a != fin[1].a || b.b != fin[1].b) FAIL(REJ_MM_B, 0, 0);
+    }
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(zr);
+    free(zc);
+    free(rho);
+    free(A);
+    free(B);
+    free(E);
     return rc;
 }

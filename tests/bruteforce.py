@@ -633,3 +633,72 @@ def had2_prove(seed: int, s, u) -> bytes:
         rho.append((a, tx.squeeze("had2_chal")))
     send("had2_final", [x_mle(s, rho), x_mle(u, rho)])
     return bytes(out)
+
+
+def mm2_prove(seed: int, site, wit) -> bytes:
+    """The extension-field matmul sum-check of one site from definitions: every MLE a hypercube
+    sum at an extension point, every round value a sum over the unbound variables."""
+    q, r, _ = wit
+    M, K, N, k = site.M, site.K, site.N, site.k_shift
+    vM, vN, n = log2c(M), log2c(N), log2c(K)
+    W = weights(site)                      # M x K
+    X = np.asarray(site.xt, np.int64).T    # K x N
+    Y = ((1 << k) * np.asarray(q, np.int64) + np.asarray(r, np.int64)).T  # M x N
+    tx = Tx(seed)
+    tx.absorb("mm2_site", site_digests([site], [wit])[0][:160])
+
+    def squeeze_ext(label):
+        a = tx.squeeze(label)
+        return (a, tx.squeeze(label))
+
+    zr = [squeeze_ext("mm2_row") for _ in range(vM)]
+    zc = [squeeze_ext("mm2_col") for _ in range(vN)]
+    out = bytearray()
+
+    def send(label, xs):
+        b = fe_bytes([c for x in xs for c in x])
+        out.extend(b)
+        tx.absorb(label, b)
+
+    def bits(x, v):
+        return [((x >> (v - 1 - b)) & 1, 0) for b in range(v)]
+
+    def A_at(pt):  # W_eff~(zr, pt) by the double hypercube sum
+        acc = (0, 0)
+        for i in range(M):
+            ei = x_eq(zr, bits(i, vM))
+            for kk in range(K):
+                e = x_mul(ei, x_eq(pt, bits(kk, n)))
+                acc = x_add(acc, (e[0] * (int(W[i, kk]) % P) % P, e[1] * (int(W[i, kk]) % P) % P))
+        return acc
+
+    def B_at(pt):
+        acc = (0, 0)
+        for j in range(N):
+            ej = x_eq(zc, bits(j, vN))
+            for kk in range(K):
+                e = x_mul(ej, x_eq(pt, bits(kk, n)))
+                acc = x_add(acc, (e[0] * (int(X[kk, j]) % P) % P, e[1] * (int(X[kk, j]) % P) % P))
+        return acc
+
+    c = (0, 0)
+    for i in range(M):
+        for j in range(N):
+            e = x_mul(x_eq(zr, bits(i, vM)), x_eq(zc, bits(j, vN)))
+            y = int(Y[i, j]) % P
+            c = x_add(c, (e[0] * y % P, e[1] * y % P))
+    send("mm2_claim", [c])
+    rho = []
+    for t in range(n):
+        rest = n - t - 1
+        g = []
+        for Xv in range(3):
+            acc = (0, 0)
+            for bb in range(1 << rest):
+                pt = rho + [(Xv, 0)] + [((bb >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                acc = x_add(acc, x_mul(A_at(pt), B_at(pt)))
+            g.append(acc)
+        send("mm2_round", g)
+        rho.append(squeeze_ext("mm2_chal"))
+    send("mm2_final", [A_at(rho), B_at(rho)])
+    return bytes(out)

@@ -78,3 +78,37 @@ def test_each_check_fires():
     # the base-field statement is a different one: its proof does not verify here
     pf_base, _ = oracle.had_prove(1, s, u)
     assert oracle.had2_verify(1, s, u, pf_base)[0] != "accept"
+
+
+# ---- the matmul sum-check over the extension ------------------------------------------
+
+import workloads  # noqa: E402
+
+
+def _site(M, K, N, bits, scales, seed):
+    s = workloads.random_site(seed, M, K, N, bits, 6)
+    if scales:
+        s.scales = workloads.group_scales(np.random.default_rng(seed), M, K)
+    return s, oracle.witness(s)
+
+
+@pytest.mark.parametrize("M,K,N,bits,scales", [(1, 1, 1, 8, False), (2, 4, 3, 8, False), (3, 5, 2, 4, True)])
+def test_mm2_bytes_match_bruteforce(M, K, N, bits, scales):
+    s, w = _site(M, K, N, bits, scales, M * 10 + K)
+    pf, _ = oracle.mm2_prove(4, s, w)
+    assert pf == bf.mm2_prove(4, s, w)
+
+
+@pytest.mark.parametrize("M,K,N,bits,scales", [(17, 100, 9, 4, True), (64, 256, 32, 8, False)])
+def test_mm2_honest_accepted_and_tampering_named(M, K, N, bits, scales):
+    s, w = _site(M, K, N, bits, scales, M + N)
+    pf, _ = oracle.mm2_prove(7, s, w)
+    assert oracle.mm2_verify(7, s, w, pf) == ("accept", (0, 0))
+    fo = len(pf) - 32
+    a = struct.unpack("<Q", pf[fo:fo + 8])[0]
+    assert oracle.mm2_verify(7, s, w, pf[:fo] + struct.pack("<Q", (a + 1) % P) + pf[fo + 8:])[0] == "mm_final"
+    x = struct.unpack("<Q", pf[16:24])[0]  # round 1, g(0)'s first coordinate
+    assert oracle.mm2_verify(7, s, w, pf[:16] + struct.pack("<Q", (x + 1) % P) + pf[24:]) == ("mm_round", (0, 0))
+    q, r, y = (t.copy() for t in w)
+    r[1, 2] += 1
+    assert oracle.mm2_verify(7, s, (q, r, y), pf)[0] != "accept"
