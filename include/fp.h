@@ -236,6 +236,39 @@ int sumcheck_prove_hadamard(fp_ctx* ctx, fp_tx* tx, const int8_t* s, const int8_
                             size_t* proof_len, void* stream);
 
 /*
+ * The gated-product sum-check with challenges in the quadratic extension
+ * F_p[phi]/(phi^2 - 7) ("How fast can FlashProve go", 4, the note on soundness:
+ * challenges from an extension field; 7 is not a square mod p). The statement of
+ * sumcheck_prove_hadamard with every challenge, claim, round value and final value
+ * an extension element a + b phi, sent as a then b (16 bytes) and squeezed as two
+ * base challenges under its label. Same arguments; the call continues tx:
+ *   absorb "had2_site" D(s) || D(u); squeeze z_1..z_v ("had2_z");
+ *   send c ("had2_claim"); round t = 1..v: send g_t(0..3) ("had2_round"),
+ *   squeeze rho_t ("had2_chal"); send s~(rho), u~(rho) ("had2_final").
+ * Proof bytes: 16 + 64 v + 32. Errors as for sumcheck_prove_hadamard.
+ */
+int sumcheck_prove_hadamard_ext2(fp_ctx* ctx, fp_tx* tx, const int8_t* s, const int8_t* u, int64_t n,
+                                 uint8_t* proof, size_t* proof_len, void* stream);
+
+/*
+ * The host half of sumcheck_prove_hadamard_ext2 with its device values supplied
+ * by a callback (no GPU work): it checks the transcript order and the round
+ * polynomials against values computed elsewhere. tx must have absorbed
+ * "had2_site". The callback gets (user, kind, t, in, out) and returns 0, or
+ * nonzero to stop the call with FP_ERR_ARG:
+ *   FP_EXT_START: in = z_1..z_v (2 v words, a then b each), t = v;
+ *   FP_EXT_SINGLE (v = 0 only): out = c, s(0), u(0) (6 words);
+ *   FP_EXT_ROUND: out = h_t(0), h_t(1), h_t(2) (6 words), where
+ *     h_t(X) = sum_b eq(z_>t, b) s~(rho_<t, X, b) u~(rho_<t, X, b);
+ *   FP_EXT_ANSWER: in = rho_t (2 words);
+ *   FP_EXT_FINALS: out = s~(rho), u~(rho) (4 words).
+ * The proof and proof_len are as for sumcheck_prove_hadamard_ext2 (v variables).
+ */
+enum { FP_EXT_START = 0, FP_EXT_SINGLE = 1, FP_EXT_ROUND = 2, FP_EXT_ANSWER = 3, FP_EXT_FINALS = 4 };
+typedef int (*fp_ext_values_fn)(void* user, int kind, int t, const uint64_t* in, uint64_t* out);
+int fp_had2_protocol_drive(fp_tx* tx, int v, fp_ext_values_fn fn, void* user, uint8_t* proof, size_t* proof_len);
+
+/*
  * Per-group scale reduction: a claim on W_eff~(z), W_eff[i][k] = S[i][k / 64] w[i][k]
  * (what the matmul sum-check of a site with scales ends with), reduced to claims on
  * the committed weights w and scales S by the same product sum-check as the gated

@@ -14,7 +14,8 @@ import ctypes as C
 from pathlib import Path
 from typing import Optional, Sequence
 
-__all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P"]
+__all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P",
+           "had2_protocol_drive"]
 
 P = 0xFFFFFFFF00000001
 LIB_PATH = Path(__file__).resolve().with_name("libfp.so")
@@ -74,6 +75,8 @@ def lib():
     L.sumcheck_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
     L.logup_prove_rescale.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
     L.sumcheck_prove_hadamard.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
+    L.sumcheck_prove_hadamard_ext2.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
+    L.fp_had2_protocol_drive.argtypes = [vp, i32, _EXT_VALUES_FN, vp, vp, C.POINTER(sz)]
     L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, C.POINTER(sz), vp]
     L.logup_prove_silu.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_silu_table.argtypes = [vp]
@@ -92,6 +95,45 @@ def lib():
     L.fp_kernel_name.argtypes = [i32]
     _lib = L
     return L
+
+
+# int (*)(void* user, int kind, int t, const uint64_t* in, uint64_t* out)
+_EXT_VALUES_FN = C.CFUNCTYPE(C.c_int, C.c_void_p, C.c_int, C.c_int, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64))
+EXT_START, EXT_SINGLE, EXT_ROUND, EXT_ANSWER, EXT_FINALS = range(5)
+
+
+def had2_protocol_drive(tx: "Transcript", v: int, values) -> bytes:
+    """Run the host half of the extension-field gated-product proof with its device values
+    taken from `values` (no GPU work): values.start(z), values.single() -> (c, s0, u0),
+    values.round(t) -> (h(0), h(1), h(2)), values.answer(t, rho), values.finals() -> (s, u),
+    every extension element a pair (a, b). tx must have absorbed "had2_site"."""
+    L = lib()
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            if kind == EXT_START:
+                values.start([(int(inp[2 * i]), int(inp[2 * i + 1])) for i in range(t)])
+                return 0
+            if kind == EXT_ANSWER:
+                values.answer(t, (int(inp[0]), int(inp[1])))
+                return 0
+            res = {EXT_SINGLE: values.single, EXT_FINALS: values.finals}.get(kind)
+            res = values.round(t) if kind == EXT_ROUND else res()
+            for i, (a, b) in enumerate(res):
+                out[2 * i] = int(a)
+                out[2 * i + 1] = int(b)
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _EXT_VALUES_FN(cb)
+    cap = 16 + 64 * v + 32
+    buf = C.create_string_buffer(cap)
+    ln = C.c_size_t(cap)
+    rc = L.fp_had2_protocol_drive(tx.h, v, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_had2_protocol_drive failed")
+    return buf.raw[: ln.value]
 
 
 def kernel_names() -> list:
@@ -251,6 +293,22 @@ class Context:
         ln = C.c_size_t(cap)
         self._check(self._L.sumcheck_prove_hadamard(self.h, tx.h, _ptr(s), _ptr(u), n, buf, C.byref(ln),
                                                     _stream(stream)), "sumcheck_prove_hadamard")
+        return buf.raw[: ln.value]
+
+    def prove_hadamard_ext2(self, tx: Transcript, s, u, stream=None) -> bytes:
+        """As prove_hadamard, with every challenge and every value sent in the quadratic
+        extension F_p[phi]/(phi^2 - 7) (16 bytes each); continues tx."""
+        n = int(s.numel())
+        if int(u.numel()) != n:
+            raise ValueError("prove_hadamard_ext2: s and u differ in size")
+        v = 0
+        while (1 << v) < n:
+            v += 1
+        cap = 16 + 64 * v + 32
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        self._check(self._L.sumcheck_prove_hadamard_ext2(self.h, tx.h, _ptr(s), _ptr(u), n, buf, C.byref(ln),
+                                                         _stream(stream)), "sumcheck_prove_hadamard_ext2")
         return buf.raw[: ln.value]
 
     def reduce_scales(self, tx: Transcript, w, bits: int, scales, M: int, K: int, point: Sequence[int],

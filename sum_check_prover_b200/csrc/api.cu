@@ -352,7 +352,7 @@ const char* fp_kernel_name(int k) {
         "witness_gemm", "digest_leaf", "digest_node", "digest_final", "eq_build", "partial_acc",
         "partial_fin", "claim", "sc_round", "sc_final", "hist", "keys_gather", "tree_leaf",
         "tree_up", "gkr_round", "gkr_final", "leaf_eval", "reduce", "had_claim", "had_round", "had_final",
-        "silu_hist", "silu_tree", "silu_round", "silu_leaf"};
+        "silu_hist", "silu_tree", "silu_round", "silu_leaf", "had2_round", "had2_final"};
     return (k >= 0 && k < K_COUNT) ? names[k] : "?";
 }
 

@@ -39,6 +39,8 @@ enum FpKernel {
     K_SILU_TREE,
     K_SILU_ROUND,
     K_SILU_LEAF,
+    K_HAD2_ROUND,
+    K_HAD2_FINAL,
     K_COUNT
 };
 

@@ -1,0 +1,156 @@
+"""The host half of the extension-field gated-product proof, without a GPU.
+
+"How fast can FlashProve go", 3.1 (the gated product is proven by sum-check)
+and 4 (the note on soundness: challenges from an extension field). The library
+splits sumcheck_prove_hadamard_ext2 into device round values h_t(0..2) and a
+host half that squeezes the point and the challenges, forms the round
+polynomials g_t(X) = eq(z_<t, rho_<t) eq(z_t, X) h_t(X), takes the claim from
+round 1, checks every later round against the running claim, and writes the
+proof. Here the round values come from a brute-force restatement (every value a
+hypercube sum of MLEs at extension points) and the proof and the transcript
+state must be the oracle's, byte for byte; the extension arithmetic on the
+host side of the library is the same code its kernels use.
+"""
+
+import numpy as np
+import pytest
+
+from tests import bruteforce as bf
+import oracle
+
+P = bf.P
+
+
+@pytest.fixture(scope="module")
+def fp():
+    from sum_check_prover_b200 import build
+    build.build()
+    import sum_check_prover_b200 as m
+    return m
+
+
+class BruteValues:
+    """Device values of the gated-product sum-check by their definitions."""
+
+    def __init__(self, s, u, tamper=None):
+        self.s = [int(x) for x in s]
+        self.u = [int(x) for x in u]
+        self.v = bf.log2c(len(self.s))
+        self.rho = []
+        self.tamper = tamper  # (round, X): add one to that value
+        self.calls = []
+
+    def start(self, z):
+        assert len(z) == self.v
+        self.z = z
+        self.calls.append("start")
+
+    def single(self):
+        self.calls.append("single")
+        c = self.s[0] * self.u[0] % P
+        return [(c, 0), (self.s[0] % P, 0), (self.u[0] % P, 0)]
+
+    def round(self, t):
+        self.calls.append(("round", t))
+        assert len(self.rho) == t - 1
+        rest = self.v - t
+        out = []
+        for X in range(3):
+            acc = (0, 0)
+            for b in range(1 << rest):
+                bits = [((b >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                pt = self.rho + [(X, 0)] + bits
+                e = bf.x_eq(self.z[t:], bits)
+                acc = bf.x_add(acc, bf.x_mul(e, bf.x_mul(bf.x_mle(self.s, pt), bf.x_mle(self.u, pt))))
+            if self.tamper == (t, X):
+                acc = ((acc[0] + 1) % P, acc[1])
+            out.append(acc)
+        return out
+
+    def answer(self, t, rho):
+        self.calls.append(("answer", t))
+        assert t == len(self.rho) + 1
+        self.rho.append(rho)
+
+    def finals(self):
+        self.calls.append("finals")
+        return [bf.x_mle(self.s, self.rho), bf.x_mle(self.u, self.rho)]
+
+
+def _site_tx(fp, seed, s, u):
+    tx = fp.Transcript(seed)
+    tx.absorb("had2_site", bf.tree_digest(np.asarray(s, np.int8).tobytes())
+              + bf.tree_digest(np.asarray(u, np.int8).tobytes()))
+    return tx
+
+
+def _vecs(n, seed):
+    rng = np.random.default_rng(seed)
+    return rng.integers(-128, 128, n).astype(np.int8), rng.integers(-128, 128, n).astype(np.int8)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 8, 13, 16, 27])
+def test_host_half_matches_oracle(fp, n):
+    s, u = _vecs(n, 40 + n)
+    tx = _site_tx(fp, 9, s, u)
+    vals = BruteValues(s, u)
+    pf = fp.had2_protocol_drive(tx, vals.v, vals)
+    want, wst = oracle.had2_prove(9, s, u)
+    assert pf == want
+    assert tx.state() == wst
+    v = vals.v
+    assert len(pf) == 16 + 64 * v + 32
+    if v == 0:
+        assert vals.calls == ["start", "single"]
+    else:
+        assert vals.calls == ["start"] + [c for t in range(1, v + 1) for c in (("round", t), ("answer", t))] + ["finals"]
+
+
+def test_extreme_factors(fp):
+    for a, b in ((-128, -128), (127, -128)):
+        s = np.full(7, a, np.int8)
+        u = np.full(7, b, np.int8)
+        tx = _site_tx(fp, 3, s, u)
+        vals = BruteValues(s, u)
+        assert fp.had2_protocol_drive(tx, vals.v, vals) == oracle.had2_prove(3, s, u)[0]
+
+
+@pytest.mark.parametrize("t,X", [(2, 0), (2, 1), (3, 0)])
+def test_inconsistent_round_is_refused(fp, t, X):
+    # a wrong h_t(0) or h_t(1) from round 2 on breaks g_t(0) + g_t(1) = claim; the host stops
+    s, u = _vecs(8, 5)
+    tx = _site_tx(fp, 1, s, u)
+    with pytest.raises(fp.FpError):
+        fp.had2_protocol_drive(tx, 3, BruteValues(s, u, tamper=(t, X)))
+
+
+def test_wrong_h2_gives_a_proof_the_oracle_rejects(fp):
+    # h_t(2) is not covered by the sum check of that round; the next round's claim (or the
+    # final check) catches it, which is the verifier's job
+    s, u = _vecs(8, 6)
+    tx = _site_tx(fp, 2, s, u)
+    with pytest.raises(fp.FpError):  # round 2 no longer sums to the claim taken from round 1
+        fp.had2_protocol_drive(tx, 3, BruteValues(s, u, tamper=(1, 2)))
+    tx = _site_tx(fp, 2, s, u)
+    pf = fp.had2_protocol_drive(tx, 3, BruteValues(s, u, tamper=(3, 2)))
+    assert oracle.had2_verify(2, s, u, pf)[0] != "accept"
+
+
+def test_callback_errors_and_small_buffers(fp):
+    s, u = _vecs(4, 7)
+
+    class Broken(BruteValues):
+        def round(self, t):
+            raise RuntimeError("no values")
+
+    tx = _site_tx(fp, 0, s, u)
+    with pytest.raises(fp.FpError):
+        fp.had2_protocol_drive(tx, 2, Broken(s, u))
+    import ctypes as C
+    L = fp.lib()
+    ln = C.c_size_t(10)
+    buf = C.create_string_buffer(10)
+    cb = fp._EXT_VALUES_FN(lambda *a: 0)
+    assert L.fp_had2_protocol_drive(fp.Transcript(0).h, 2, cb, None, buf, C.byref(ln)) != 0
+    assert ln.value == 16 + 64 * 2 + 32
+    assert L.fp_had2_protocol_drive(fp.Transcript(0).h, 31, cb, None, buf, C.byref(ln)) != 0
