@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,silu") -> dict:
+def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,silu,had2") -> dict:
     """Kernel rooflines at HBM scale (inputs well above the 126 MB L2), from a
     profiled pass: every round is its own launch, timed with CUDA events.
 
@@ -190,11 +190,14 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,sil
       14336 x 4096 int4 weight matrix with per-64 scales to claims on w and S.
     silu_round: the SiLU lookup's layer sum-checks over 2^26 keys (one tree; round 1
       reads the tree layer's children, later rounds fold them: 80 and 160 B per pair).
+    had2_round: the gated product over 2^26 entries with challenges in the quadratic
+      extension (16-byte vector elements: 120 B per pair in round 2, 240 B later).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
     import workloads
     from workloads import device
+    which = set(which.split(","))  # names, not substrings ("had" is not "had2", "sc" is not "scl")
     pk = peaks()
     out = {}
 
@@ -307,6 +310,18 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,sil
             del gd, sd
         except Exception as e:  # a failure here must not cost the rest of the line
             out["silu_lookup_round_2^26"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    if "had2" in which:
+        # the gated product of the same 2^26-entry factors with extension-field challenges
+        try:
+            rng = __import__("numpy").random.default_rng(9)
+            n = 1 << 26
+            sv = torch.from_numpy(rng.integers(-128, 128, n).astype("int8")).to(dev)
+            uv = torch.from_numpy(rng.integers(-128, 128, n).astype("int8")).to(dev)
+            measure("hadamard_ext2_round_2^26", "had2_round",
+                    lambda: ctx.prove_hadamard_ext2(fp.Transcript(4), sv, uv))
+            del sv, uv
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["hadamard_ext2_round_2^26"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     try:
         torch.cuda.empty_cache()
@@ -584,7 +599,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-micro", action="store_true")
-    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm,had,scl,silu", default=None,
+    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm,had,scl,silu,had2", default=None,
                     help="run only the kernel measurements at scale (comma list of sc, pe, gkr, gemm)")
     args = ap.parse_args()
     if args.micro_only:
