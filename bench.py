@@ -171,7 +171,19 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,silu,had2") -> dict:
+MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi"
+
+
+def micro_names(which) -> set:
+    """The microbench names in a comma-separated list (whole names: "had" is not "had2")."""
+    names = set(which.split(",")) if isinstance(which, str) else set(which)
+    unknown = names - set(MICRO_ALL.split(","))
+    if unknown:
+        raise ValueError(f"unknown microbench names: {sorted(unknown)}")
+    return names
+
+
+def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
     """Kernel rooflines at HBM scale (inputs well above the 126 MB L2), from a
     profiled pass: every round is its own launch, timed with CUDA events.
 
@@ -192,12 +204,13 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,sil
       reads the tree layer's children, later rounds fold them: 80 and 160 B per pair).
     had2_round: the gated product over 2^26 entries with challenges in the quadratic
       extension (16-byte vector elements: 120 B per pair in round 2, 240 B later).
+    lhi_round: the helper-inverse LogUp's sum-check over 2^26 keys of R_12 (round 1 reads
+      the helper column and the keys, later rounds fold both: 104 and 120 B per pair).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
     import workloads
     from workloads import device
-    which = set(which.split(","))  # names, not substrings ("had" is not "had2", "sc" is not "scl")
     pk = peaks()
     out = {}
 
@@ -221,7 +234,7 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,sil
                      "per_launch": [[round(r[1], 4), r[2]] for r in sel],
                      "all_launches": len(log), "all_ms": sum(r[1] for r in log)}
 
-    which = set(which.split(","))
+    which = micro_names(which)
     if "sc" in which:
         sites = [workloads.random_site(900 + i, 1, 1 << 20, 1, 4, 12) for i in range(64)]
         st, keep = device.upload(workloads.Workload("sc", 0, sites), dev)
@@ -322,6 +335,16 @@ def run_micro(fp, torch, ctx, dev: str, which: str = "sc,pe,gkr,gemm,had,scl,sil
             del sv, uv
         except Exception as e:  # a failure here must not cost the rest of the line
             out["hadamard_ext2_round_2^26"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    if "lhi" in which:
+        # the helper-inverse LogUp of 2^26 remainders in R_12 (set against gkr_round's tree)
+        try:
+            rng = __import__("numpy").random.default_rng(12)
+            rv = torch.from_numpy(rng.integers(-2048, 2048, 1 << 26).astype("int32")).to(dev)
+            measure("helper_inverse_round_2^26_keys", "lhi_round",
+                    lambda: ctx.prove_helper_inverse(fp.Transcript(7), rv, 12))
+            del rv
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["helper_inverse_round_2^26_keys"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     try:
         torch.cuda.empty_cache()
@@ -599,7 +622,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-micro", action="store_true")
-    ap.add_argument("--micro-only", nargs="?", const="sc,pe,gkr,gemm,had,scl,silu,had2", default=None,
+    ap.add_argument("--micro-only", nargs="?", const=MICRO_ALL, default=None,
                     help="run only the kernel measurements at scale (comma list of sc, pe, gkr, gemm)")
     args = ap.parse_args()
     if args.micro_only:

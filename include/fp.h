@@ -251,22 +251,36 @@ int sumcheck_prove_hadamard_ext2(fp_ctx* ctx, fp_tx* tx, const int8_t* s, const 
                                  uint8_t* proof, size_t* proof_len, void* stream);
 
 /*
- * The host half of sumcheck_prove_hadamard_ext2 with its device values supplied
- * by a callback (no GPU work): it checks the transcript order and the round
- * polynomials against values computed elsewhere. tx must have absorbed
- * "had2_site". The callback gets (user, kind, t, in, out) and returns 0, or
- * nonzero to stop the call with FP_ERR_ARG:
- *   FP_EXT_START: in = z_1..z_v (2 v words, a then b each), t = v;
- *   FP_EXT_SINGLE (v = 0 only): out = c, s(0), u(0) (6 words);
- *   FP_EXT_ROUND: out = h_t(0), h_t(1), h_t(2) (6 words), where
- *     h_t(X) = sum_b eq(z_>t, b) s~(rho_<t, X, b) u~(rho_<t, X, b);
- *   FP_EXT_ANSWER: in = rho_t (2 words);
- *   FP_EXT_FINALS: out = s~(rho), u~(rho) (4 words).
- * The proof and proof_len are as for sumcheck_prove_hadamard_ext2 (v variables).
+ * Protocol drivers (no GPU work). The host half of a statement (the transcript,
+ * the round polynomials, the running claim, the proof layout) is separate from
+ * the device work that feeds it; a driver runs that host half with its device
+ * values supplied by a callback, so the protocol can be checked against values
+ * computed elsewhere. The callback gets (user, kind, t, in, out) and returns 0,
+ * or nonzero to stop the driver with FP_ERR_ARG. What in and out hold for each
+ * kind is given per driver below. Values are canonical field elements.
  */
-enum { FP_EXT_START = 0, FP_EXT_SINGLE = 1, FP_EXT_ROUND = 2, FP_EXT_ANSWER = 3, FP_EXT_FINALS = 4 };
-typedef int (*fp_ext_values_fn)(void* user, int kind, int t, const uint64_t* in, uint64_t* out);
-int fp_had2_protocol_drive(fp_tx* tx, int v, fp_ext_values_fn fn, void* user, uint8_t* proof, size_t* proof_len);
+enum {
+    FP_VAL_START = 0,   /* the point is known */
+    FP_VAL_SINGLE = 1,  /* a statement without rounds */
+    FP_VAL_ROUND = 2,   /* round t's device values */
+    FP_VAL_ANSWER = 3,  /* round t's challenge */
+    FP_VAL_FINALS = 4,  /* the final values */
+    FP_VAL_COLUMN = 5   /* a committed column is formed: its digest */
+};
+typedef int (*fp_values_fn)(void* user, int kind, int t, const uint64_t* in, uint64_t* out);
+
+/*
+ * The host half of sumcheck_prove_hadamard_ext2 (v variables); tx must have
+ * absorbed "had2_site". Callback kinds:
+ *   FP_VAL_START: in = z_1..z_v (2 v words, a then b each), t = v;
+ *   FP_VAL_SINGLE (v = 0 only): out = c, s(0), u(0) (6 words);
+ *   FP_VAL_ROUND: out = h_t(0), h_t(1), h_t(2) (6 words), where
+ *     h_t(X) = sum_b eq(z_>t, b) s~(rho_<t, X, b) u~(rho_<t, X, b);
+ *   FP_VAL_ANSWER: in = rho_t (2 words);
+ *   FP_VAL_FINALS: out = s~(rho), u~(rho) (4 words).
+ * The proof and proof_len are as for sumcheck_prove_hadamard_ext2.
+ */
+int fp_had2_protocol_drive(fp_tx* tx, int v, fp_values_fn fn, void* user, uint8_t* proof, size_t* proof_len);
 
 /*
  * Per-group scale reduction: a claim on W_eff~(z), W_eff[i][k] = S[i][k / 64] w[i][k]
@@ -315,6 +329,46 @@ int sumcheck_reduce_scales(fp_ctx* ctx, fp_tx* tx, const void* w, int w_bits, co
  */
 int logup_prove_silu(fp_ctx* ctx, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
                      size_t* proof_len, void* stream);
+
+/*
+ * Helper-inverse LogUp on the remainder table R_k = {j - 2^(k-1) : j < 2^k}
+ * ("Towards Proving Frontier-Scale LLM Inference", The proof system: LogUp after
+ * Haboeck 2022, the key side a committed column of inverses checked by one
+ * sum-check; set against the GKR fraction tree of logup_prove_rescale).
+ * r: device int32 key column of n entries (caller-owned, read only); keys are
+ * padded to 2^v (v = max(1, ceil(log2 n))) with 0. The call continues tx:
+ *   absorb "lhi_site" D(r) (int32 little-endian); send m_j = #{keys equal to
+ *   j - 2^(k-1)} (2^k u32, keys outside the table not counted; "lhi_m" absorbs
+ *   their digest); squeeze alpha ("lhi_alpha"); absorb "lhi_h" D(h) for the
+ *   helper column h_i = 1 / (alpha - r_i) (u64 little-endian, 2^v entries);
+ *   squeeze z_1..z_v ("lhi_z") and beta ("lhi_beta"); send S = sum_i h_i
+ *   ("lhi_sum"); v rounds of g(0..3) ("lhi_round") and challenges ("lhi_chal")
+ *   of the sum-check of h(x) + beta eq(z, x) (h(x) (alpha - f(x)) - 1), claim S;
+ *   send h~(rho), f~(rho) ("lhi_final").
+ * Proof bytes: 4 2^k + 8 + 32 v + 16. Returns FP_OK, or 1 when some key lies
+ * outside the table (the proof is still written; it will not verify).
+ * 1 <= k <= 24 and null arguments: FP_ERR_ARG; 1 <= n <= 2^30, else
+ * FP_ERR_SHAPE; proof / proof_len as for sumcheck_prove_matmul.
+ */
+int logup_prove_helper_inverse(fp_ctx* ctx, fp_tx* tx, const int32_t* r, int64_t n, int k, uint8_t* proof,
+                               size_t* proof_len, void* stream);
+
+/*
+ * The host half of logup_prove_helper_inverse from the multiplicities on (v >= 1
+ * variables, table R_k): m (host, 2^k u32) and m_digest (host, 32 bytes: the
+ * digest of m's bytes) are given; tx must have absorbed "lhi_site". Callback
+ * kinds (see the protocol drivers above):
+ *   FP_VAL_COLUMN: in = alpha (1 word); out = D(h) (32 bytes as 4 little-endian words);
+ *   FP_VAL_START: in = z_1..z_v, beta (v + 1 words), t = v;
+ *   FP_VAL_ROUND: out = H_t(0), H_t(1), Q_t(0), Q_t(1), Q_t(2) (5 words) with
+ *     H_t(X) = sum_b h~(rho_<t, X, b) and
+ *     Q_t(X) = sum_b eq(z_>t, b) h~(rho_<t, X, b) (alpha - f~(rho_<t, X, b));
+ *   FP_VAL_ANSWER: in = rho_t (1 word);
+ *   FP_VAL_FINALS: out = h~(rho), f~(rho) (2 words).
+ * The proof and proof_len are as for logup_prove_helper_inverse.
+ */
+int fp_lhi_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uint8_t* m_digest, fp_values_fn fn,
+                          void* user, uint8_t* proof, size_t* proof_len);
 
 /* The SiLU table's 2^16 entries silu_q(v), v = -2^15 .. 2^15 - 1, into host out (no GPU work). */
 int fp_silu_table(int32_t* out);

@@ -15,7 +15,7 @@ from pathlib import Path
 from typing import Optional, Sequence
 
 __all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P",
-           "had2_protocol_drive"]
+           "had2_protocol_drive", "lhi_protocol_drive"]
 
 P = 0xFFFFFFFF00000001
 LIB_PATH = Path(__file__).resolve().with_name("libfp.so")
@@ -76,7 +76,9 @@ def lib():
     L.logup_prove_rescale.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
     L.sumcheck_prove_hadamard.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.sumcheck_prove_hadamard_ext2.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
-    L.fp_had2_protocol_drive.argtypes = [vp, i32, _EXT_VALUES_FN, vp, vp, C.POINTER(sz)]
+    L.fp_had2_protocol_drive.argtypes = [vp, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
+    L.logup_prove_helper_inverse.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
+    L.fp_lhi_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, C.POINTER(sz), vp]
     L.logup_prove_silu.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_silu_table.argtypes = [vp]
@@ -98,8 +100,8 @@ def lib():
 
 
 # int (*)(void* user, int kind, int t, const uint64_t* in, uint64_t* out)
-_EXT_VALUES_FN = C.CFUNCTYPE(C.c_int, C.c_void_p, C.c_int, C.c_int, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64))
-EXT_START, EXT_SINGLE, EXT_ROUND, EXT_ANSWER, EXT_FINALS = range(5)
+_VALUES_FN = C.CFUNCTYPE(C.c_int, C.c_void_p, C.c_int, C.c_int, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64))
+VAL_START, VAL_SINGLE, VAL_ROUND, VAL_ANSWER, VAL_FINALS, VAL_COLUMN = range(6)
 
 
 def had2_protocol_drive(tx: "Transcript", v: int, values) -> bytes:
@@ -111,14 +113,14 @@ def had2_protocol_drive(tx: "Transcript", v: int, values) -> bytes:
 
     def cb(_user, kind, t, inp, out):
         try:
-            if kind == EXT_START:
+            if kind == VAL_START:
                 values.start([(int(inp[2 * i]), int(inp[2 * i + 1])) for i in range(t)])
                 return 0
-            if kind == EXT_ANSWER:
+            if kind == VAL_ANSWER:
                 values.answer(t, (int(inp[0]), int(inp[1])))
                 return 0
-            res = {EXT_SINGLE: values.single, EXT_FINALS: values.finals}.get(kind)
-            res = values.round(t) if kind == EXT_ROUND else res()
+            res = {VAL_SINGLE: values.single, VAL_FINALS: values.finals}.get(kind)
+            res = values.round(t) if kind == VAL_ROUND else res()
             for i, (a, b) in enumerate(res):
                 out[2 * i] = int(a)
                 out[2 * i + 1] = int(b)
@@ -126,13 +128,57 @@ def had2_protocol_drive(tx: "Transcript", v: int, values) -> bytes:
         except Exception:  # reported to the caller as FP_ERR_ARG
             return 1
 
-    fn = _EXT_VALUES_FN(cb)
+    fn = _VALUES_FN(cb)
     cap = 16 + 64 * v + 32
     buf = C.create_string_buffer(cap)
     ln = C.c_size_t(cap)
     rc = L.fp_had2_protocol_drive(tx.h, v, fn, None, buf, C.byref(ln))
     if rc != 0:
         raise FpError(rc, "fp_had2_protocol_drive failed")
+    return buf.raw[: ln.value]
+
+
+def lhi_protocol_drive(tx: "Transcript", v: int, k: int, m, m_digest: bytes, values) -> bytes:
+    """Run the host half of the helper-inverse LogUp from the multiplicities on, with its
+    device values taken from `values` (no GPU work): values.column(alpha) -> 32-byte digest
+    of the helper column, values.start(z, beta), values.round(t) -> (H(0), H(1), Q(0), Q(1),
+    Q(2)), values.answer(t, rho), values.finals() -> (h~(rho), f~(rho)). m: 2^k counts;
+    m_digest: the digest of their u32 little-endian bytes. tx must have absorbed "lhi_site"."""
+    import numpy as np
+
+    L = lib()
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            if kind == VAL_COLUMN:
+                d = values.column(int(inp[0]))
+                for i in range(4):
+                    out[i] = int.from_bytes(d[8 * i: 8 * i + 8], "little")
+            elif kind == VAL_START:
+                values.start([int(inp[i]) for i in range(t)], int(inp[t]))
+            elif kind == VAL_ANSWER:
+                values.answer(t, int(inp[0]))
+            elif kind == VAL_ROUND:
+                for i, x in enumerate(values.round(t)):
+                    out[i] = int(x)
+            elif kind == VAL_FINALS:
+                for i, x in enumerate(values.finals()):
+                    out[i] = int(x)
+            else:
+                return 1
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _VALUES_FN(cb)
+    mm = np.ascontiguousarray(np.asarray(m, dtype="<u4"))
+    md = C.create_string_buffer(bytes(m_digest), 32)
+    cap = 4 * (1 << k) + 8 + 32 * v + 16
+    buf = C.create_string_buffer(cap)
+    ln = C.c_size_t(cap)
+    rc = L.fp_lhi_protocol_drive(tx.h, v, k, mm.ctypes.data, md, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_lhi_protocol_drive failed")
     return buf.raw[: ln.value]
 
 
@@ -310,6 +356,22 @@ class Context:
         self._check(self._L.sumcheck_prove_hadamard_ext2(self.h, tx.h, _ptr(s), _ptr(u), n, buf, C.byref(ln),
                                                          _stream(stream)), "sumcheck_prove_hadamard_ext2")
         return buf.raw[: ln.value]
+
+    def prove_helper_inverse(self, tx: Transcript, r, k: int, stream=None):
+        """Helper-inverse LogUp proof that every entry of the device int32 tensor r lies in
+        the remainder table R_k; continues tx. Returns (proof bytes, status): status 1 means
+        some key lies outside the table."""
+        n = int(r.numel())
+        v = 0
+        while (1 << v) < n:
+            v += 1
+        v = max(v, 1)
+        cap = 4 * (1 << k) + 8 + 32 * v + 16
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        rc = self._check(self._L.logup_prove_helper_inverse(self.h, tx.h, _ptr(r), n, k, buf, C.byref(ln),
+                                                            _stream(stream)), "logup_prove_helper_inverse")
+        return buf.raw[: ln.value], rc
 
     def reduce_scales(self, tx: Transcript, w, bits: int, scales, M: int, K: int, point: Sequence[int],
                       stream=None) -> bytes:

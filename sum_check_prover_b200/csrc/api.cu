@@ -347,12 +347,26 @@ int64_t fp_kernel_log(fp_ctx* c, fp_launch_rec* out, int64_t cap) {
     return n;
 }
 
+// the degree-3 polynomial through (i, g[i]), i = 0..3, at r: the next claim of a
+// degree-3 sum-check round
+uint64_t fp_lagrange4(const uint64_t g[4], uint64_t r) {
+    static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
+    const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2), r3 = gl_sub(r, 3);
+    // L0 = -(r-1)(r-2)(r-3)/6, L1 = r(r-2)(r-3)/2, L2 = -r(r-1)(r-3)/2, L3 = r(r-1)(r-2)/6
+    const uint64_t l0 = gl_sub(0, gl_mul(gl_mul(gl_mul(r1, r2), r3), inv6));
+    const uint64_t l1 = gl_mul(gl_mul(gl_mul(r, r2), r3), inv2);
+    const uint64_t l2 = gl_sub(0, gl_mul(gl_mul(gl_mul(r, r1), r3), inv2));
+    const uint64_t l3 = gl_mul(gl_mul(gl_mul(r, r1), r2), inv6);
+    return gl_add(gl_add(gl_mul(g[0], l0), gl_mul(g[1], l1)), gl_add(gl_mul(g[2], l2), gl_mul(g[3], l3)));
+}
+
 const char* fp_kernel_name(int k) {
     static const char* names[K_COUNT] = {
         "witness_gemm", "digest_leaf", "digest_node", "digest_final", "eq_build", "partial_acc",
         "partial_fin", "claim", "sc_round", "sc_final", "hist", "keys_gather", "tree_leaf",
         "tree_up", "gkr_round", "gkr_final", "leaf_eval", "reduce", "had_claim", "had_round", "had_final",
-        "silu_hist", "silu_tree", "silu_round", "silu_leaf", "had2_round", "had2_final"};
+        "silu_hist", "silu_tree", "silu_round", "silu_leaf", "had2_round", "had2_final",
+        "lhi_hist", "lhi_column", "lhi_round", "lhi_final"};
     return (k >= 0 && k < K_COUNT) ? names[k] : "?";
 }
 

@@ -41,6 +41,10 @@ enum FpKernel {
     K_SILU_LEAF,
     K_HAD2_ROUND,
     K_HAD2_FINAL,
+    K_LHI_HIST,
+    K_LHI_COLUMN,
+    K_LHI_ROUND,
+    K_LHI_FINAL,
     K_COUNT
 };
 
@@ -187,3 +191,6 @@ static inline size_t fp_align_up(size_t x, size_t a) { return (x + a - 1) / a * 
 
 // little-endian u64 words into a proof buffer (sumcheck.cu)
 void put_u64s(uint8_t* p, const uint64_t* v, size_t n);
+
+// the degree-3 polynomial through (i, g[i]), i = 0..3, at r (api.cu)
+uint64_t fp_lagrange4(const uint64_t g[4], uint64_t r);

@@ -204,18 +204,6 @@ __global__ void __launch_bounds__(HAD_THREADS, 2) prod_session_kernel(ProdArgs<S
     }
 }
 
-// the degree-3 polynomial through (i, g[i]), i = 0..3, at r
-uint64_t lagrange4(const uint64_t g[4], uint64_t r) {
-    static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
-    const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2), r3 = gl_sub(r, 3);
-    // L0 = -(r-1)(r-2)(r-3)/6, L1 = r(r-2)(r-3)/2, L2 = -r(r-1)(r-3)/2, L3 = r(r-1)(r-2)/6
-    const uint64_t l0 = gl_sub(0, gl_mul(gl_mul(gl_mul(r1, r2), r3), inv6));
-    const uint64_t l1 = gl_mul(gl_mul(gl_mul(r, r2), r3), inv2);
-    const uint64_t l2 = gl_sub(0, gl_mul(gl_mul(gl_mul(r, r1), r3), inv2));
-    const uint64_t l3 = gl_mul(gl_mul(gl_mul(r, r1), r2), inv6);
-    return gl_add(gl_add(gl_mul(g[0], l0), gl_mul(g[1], l1)), gl_add(gl_mul(g[2], l2), gl_mul(g[3], l3)));
-}
-
 struct ProdLabels {
     const char* claim;
     const char* round;
@@ -342,7 +330,7 @@ int prod_sumcheck(fp_ctx* c, fp_tx* tx, const Src& src, int64_t len, const FpPoi
             fp_session_expect(c, t < v ? 3 : 2);  // the last challenge triggers the final values
             const uint64_t r = fp_tx_squeeze_one(tx, lab.chal);
             fp_session_post(c, A.seq0 + t, r);
-            claim = lagrange4(g, r);
+            claim = fp_lagrange4(g, r);
             pre = gl_mul(pre, gl_add(gl_mul(zt, r), gl_mul(gl_sub(1, zt), gl_sub(1, r))));
         }
         if (c->stepped) {

@@ -411,7 +411,7 @@ struct Had2Device : Had2Source {
 
 // Round values from a caller's callback (no device).
 struct Had2Callback : Had2Source {
-    fp_ext_values_fn fn;
+    fp_values_fn fn;
     void* user;
     int call(int kind, int t, const uint64_t* in, uint64_t* out) {
         return fn(user, kind, t, in, out) ? FP_ERR_ARG : FP_OK;
@@ -422,11 +422,11 @@ struct Had2Callback : Had2Source {
             in[2 * i] = z[i].a;
             in[2 * i + 1] = z[i].b;
         }
-        return call(FP_EXT_START, v, in, nullptr);
+        return call(FP_VAL_START, v, in, nullptr);
     }
     int single(Ext2& claim, Ext2 fin[2]) override {
         uint64_t out[6] = {0, 0, 0, 0, 0, 0};
-        int rc = call(FP_EXT_SINGLE, 0, nullptr, out);
+        int rc = call(FP_VAL_SINGLE, 0, nullptr, out);
         claim = e2_make(gl_canon(out[0]), gl_canon(out[1]));
         fin[0] = e2_make(gl_canon(out[2]), gl_canon(out[3]));
         fin[1] = e2_make(gl_canon(out[4]), gl_canon(out[5]));
@@ -434,17 +434,17 @@ struct Had2Callback : Had2Source {
     }
     int round(int t, Ext2 h[3]) override {
         uint64_t out[6] = {0, 0, 0, 0, 0, 0};
-        int rc = call(FP_EXT_ROUND, t, nullptr, out);
+        int rc = call(FP_VAL_ROUND, t, nullptr, out);
         for (int i = 0; i < 3; i++) h[i] = e2_make(gl_canon(out[2 * i]), gl_canon(out[2 * i + 1]));
         return rc;
     }
     int answer(int t, Ext2 rho) override {
         const uint64_t in[2] = {rho.a, rho.b};
-        return call(FP_EXT_ANSWER, t, in, nullptr);
+        return call(FP_VAL_ANSWER, t, in, nullptr);
     }
     int finals(Ext2 fin[2]) override {
         uint64_t out[4] = {0, 0, 0, 0};
-        int rc = call(FP_EXT_FINALS, 0, nullptr, out);
+        int rc = call(FP_VAL_FINALS, 0, nullptr, out);
         fin[0] = e2_make(gl_canon(out[0]), gl_canon(out[1]));
         fin[1] = e2_make(gl_canon(out[2]), gl_canon(out[3]));
         return rc;
@@ -483,7 +483,7 @@ int sumcheck_prove_hadamard_ext2(fp_ctx* c, fp_tx* tx, const int8_t* s, const in
     return had2_protocol(c, tx, v, dev, proof, proof_len);
 }
 
-int fp_had2_protocol_drive(fp_tx* tx, int v, fp_ext_values_fn fn, void* user, uint8_t* proof, size_t* proof_len) {
+int fp_had2_protocol_drive(fp_tx* tx, int v, fp_values_fn fn, void* user, uint8_t* proof, size_t* proof_len) {
     if (!tx || !fn || !proof_len) return FP_ERR_ARG;
     if (v < 0 || v > H2_MAX_V) return FP_ERR_SHAPE;
     const size_t need_len = 16 + 64 * (size_t)v + 32;

@@ -831,15 +831,6 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
     // device's h(0), h(2): g(1) follows from the running claim (g(0) + g(1) = claim),
     // h(1) = g(1) / (pre z_t) gives g(3) through h(3) = h(0) - 3 h(1) + 3 h(2).
     // The next claim is g(rho_t) (Lagrange on the nodes 0..3).
-    static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
-    auto lagrange4 = [](const uint64_t g[4], uint64_t r) {
-        const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2), r3 = gl_sub(r, 3);
-        const uint64_t l0 = gl_sub(0, gl_mul(gl_mul(r1, r2), gl_mul(r3, inv6)));
-        const uint64_t l1 = gl_mul(gl_mul(r, r2), gl_mul(r3, inv2));
-        const uint64_t l2 = gl_sub(0, gl_mul(gl_mul(r, r1), gl_mul(r3, inv2)));
-        const uint64_t l3 = gl_mul(gl_mul(r, r1), gl_mul(r2, inv6));
-        return gl_add(gl_add(gl_mul(g[0], l0), gl_mul(g[1], l1)), gl_add(gl_mul(g[2], l2), gl_mul(g[3], l3)));
-    };
     uint64_t prev[8];  // the two-node layer's values, then each layer's child values at its point
     memcpy(prev, hsmall, sizeof prev);
     std::vector<uint64_t> zpt, rhos, zinv;
@@ -910,7 +901,7 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
                 fp_session_expect(c, t < d ? 3 : 8);  // the last challenge triggers the final values
                 const uint64_t r = fp_tx_squeeze_one(tx, "gkr_chal");
                 fp_session_post(c, A.seq0 + t, r);
-                claim = lagrange4(g, r);
+                claim = fp_lagrange4(g, r);
                 pre = gl_mul(pre, gl_add(gl_mul(zt, r), gl_mul(gl_sub(1, zt), gl_sub(1, r))));
                 rhos.push_back(r);
             } else {

@@ -219,17 +219,6 @@ const LookupLabels kSiluLabels = {"silu_site", "silu_gamma", "silu_m", "silu_alp
 const LookupLabels kExpLabels = {"exp_site", "exp_gamma", "exp_m", "exp_alpha", "exp_l1", "exp_mu",
                                  "exp_lambda", "exp_round", "exp_chal", "exp_final", "exp_leaf"};
 
-// the degree-3 polynomial through (i, g[i]), i = 0..3, at r
-uint64_t lagrange4(const uint64_t g[4], uint64_t r) {
-    static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
-    const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2), r3 = gl_sub(r, 3);
-    const uint64_t l0 = gl_sub(0, gl_mul(gl_mul(gl_mul(r1, r2), r3), inv6));
-    const uint64_t l1 = gl_mul(gl_mul(gl_mul(r, r2), r3), inv2);
-    const uint64_t l2 = gl_sub(0, gl_mul(gl_mul(gl_mul(r, r1), r3), inv2));
-    const uint64_t l3 = gl_mul(gl_mul(gl_mul(r, r1), r2), inv6);
-    return gl_add(gl_add(gl_mul(g[0], l0), gl_mul(g[1], l1)), gl_add(gl_mul(g[2], l2), gl_mul(g[3], l3)));
-}
-
 unsigned grid_of(const fp_ctx* c, int64_t work) {
     return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
 }
@@ -418,7 +407,7 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
             const uint64_t r = fp_tx_squeeze_one(tx, lab.chal);
             fp_session_post(c, A.seq0 + t, r);
             rho[t - 1] = r;
-            claim = lagrange4(gr, r);
+            claim = fp_lagrange4(gr, r);
             pre = gl_mul(pre, gl_add(gl_mul(zt, r), gl_mul(gl_sub(1, zt), gl_sub(1, r))));
         }
         if (c->stepped) {

@@ -4,6 +4,8 @@ import sys
 import time
 import types
 
+import pytest
+
 import bench
 
 
@@ -40,3 +42,12 @@ def test_no_reasons(monkeypatch):
     c.start()
     time.sleep(0.02)
     assert c.stop()["reasons"] == []
+
+
+def test_micro_names_are_whole_names():
+    import bench
+    assert bench.micro_names("sc,had2") == {"sc", "had2"}
+    assert "had" not in bench.micro_names("had2,lhi") and "sc" not in bench.micro_names("scl")
+    assert bench.micro_names(bench.MICRO_ALL) == set(bench.MICRO_ALL.split(","))
+    with pytest.raises(ValueError):
+        bench.micro_names("sc,nope")

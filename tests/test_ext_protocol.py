@@ -150,7 +150,7 @@ def test_callback_errors_and_small_buffers(fp):
     L = fp.lib()
     ln = C.c_size_t(10)
     buf = C.create_string_buffer(10)
-    cb = fp._EXT_VALUES_FN(lambda *a: 0)
+    cb = fp._VALUES_FN(lambda *a: 0)
     assert L.fp_had2_protocol_drive(fp.Transcript(0).h, 2, cb, None, buf, C.byref(ln)) != 0
     assert ln.value == 16 + 64 * 2 + 32
     assert L.fp_had2_protocol_drive(fp.Transcript(0).h, 31, cb, None, buf, C.byref(ln)) != 0
