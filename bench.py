@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi"
+MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2"
 
 
 def micro_names(which) -> set:
@@ -206,6 +206,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
       extension (16-byte vector elements: 120 B per pair in round 2, 240 B later).
     lhi_round: the helper-inverse LogUp's sum-check over 2^26 keys of R_12 (round 1 reads
       the helper column and the keys, later rounds fold both: 104 and 120 B per pair).
+    mm2_contract: the extension-field matmul's row contraction of a 16384 x 16384 int4
+      weight (the matrix once; the eq weights are 16-byte extension elements).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
@@ -345,6 +347,19 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
             del rv
         except Exception as e:  # a failure here must not cost the rest of the line
             out["helper_inverse_round_2^26_keys"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    if "mm2" in which:
+        # the extension-field matmul sum-check of a 16384 x 16384 int4 weight (128 MiB) and 256
+        # tokens: its row contraction with 16-byte eq weights, set against partial_acc
+        try:
+            s = workloads.random_site(78, 16384, 16384, 256, 4, 12)
+            st, keep = device.upload(workloads.Workload("mm2", 0, [s]), dev)
+            d = st[0][0]
+            ctx.commit_witness(fp.Transcript(0), [d])
+            measure("ext2_contract_16384x16384_int4", "mm2_contract",
+                    lambda: ctx.prove_matmul_ext2(fp.Transcript(8), d), big=1 << 26)
+            del st, keep, d
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["ext2_contract_16384x16384_int4"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     try:
         torch.cuda.empty_cache()

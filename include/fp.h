@@ -265,7 +265,8 @@ enum {
     FP_VAL_ROUND = 2,   /* round t's device values */
     FP_VAL_ANSWER = 3,  /* round t's challenge */
     FP_VAL_FINALS = 4,  /* the final values */
-    FP_VAL_COLUMN = 5   /* a committed column is formed: its digest */
+    FP_VAL_COLUMN = 5,  /* a committed column is formed: its digest */
+    FP_VAL_CLAIM = 6    /* the claim the rounds start from */
 };
 typedef int (*fp_values_fn)(void* user, int kind, int t, const uint64_t* in, uint64_t* out);
 
@@ -352,6 +353,39 @@ int logup_prove_silu(fp_ctx* ctx, fp_tx* tx, const int16_t* g, const int16_t* s,
  */
 int logup_prove_helper_inverse(fp_ctx* ctx, fp_tx* tx, const int32_t* r, int64_t n, int k, uint8_t* proof,
                                size_t* proof_len, void* stream);
+
+/*
+ * The matmul sum-check of one site with challenges in the quadratic extension
+ * F_p[phi]/(phi^2 - 7) ("How fast can FlashProve go", 2 Background: the matmul
+ * Y = W X reduced by sum-check to claims on its operands; 4, the note on
+ * soundness: challenges from an extension field). site: one fp_site with its
+ * witness (q, r) from fp_commit_witness; device pointers, caller-owned, read
+ * only. The call continues tx:
+ *   absorb "mm2_site" D(W) || D(S) || D(Xt) || D(q) || D(r) (D(W) || D(S) from
+ *   site->w_digest when given); squeeze r_row (ceil(log2 M) extension
+ *   coordinates, "mm2_row") and r_col (ceil(log2 N), "mm2_col"); send
+ *   c = sum_{i,j} eq(r_row, i) eq(r_col, j) (2^k q[j][i] + r[j][i])
+ *   ("mm2_claim"); n = ceil(log2 K) rounds of g(0), g(1), g(2) of
+ *   sum_b A(X, b) B(X, b), A = W_eff~(r_row, .), B = X~(., r_col)
+ *   ("mm2_round"), challenges ("mm2_chal"); send A(rho), B(rho) ("mm2_final").
+ * Proof bytes: 16 + 48 n + 32. Site checks and errors as for
+ * sumcheck_prove_matmul.
+ */
+int sumcheck_prove_matmul_ext2(fp_ctx* ctx, fp_tx* tx, const fp_site* site, uint8_t* proof, size_t* proof_len,
+                               void* stream);
+
+/*
+ * The host half of sumcheck_prove_matmul_ext2 (vM, vN point coordinates, n
+ * rounds); tx must have absorbed "mm2_site". Callback kinds:
+ *   FP_VAL_START: in = r_row then r_col (2 (vM + vN) words), t = vM + vN;
+ *   FP_VAL_CLAIM: out = c (2 words);
+ *   FP_VAL_ROUND: out = g_t(0), g_t(1), g_t(2) (6 words);
+ *   FP_VAL_ANSWER: in = rho_t (2 words);
+ *   FP_VAL_FINALS: out = A(rho), B(rho) (4 words).
+ * The proof and proof_len are as for sumcheck_prove_matmul_ext2.
+ */
+int fp_mm2_protocol_drive(fp_tx* tx, int vM, int vN, int n, fp_values_fn fn, void* user, uint8_t* proof,
+                          size_t* proof_len);
 
 /*
  * The host half of logup_prove_helper_inverse from the multiplicities on (v >= 1

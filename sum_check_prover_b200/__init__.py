@@ -15,7 +15,7 @@ from pathlib import Path
 from typing import Optional, Sequence
 
 __all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P",
-           "had2_protocol_drive", "lhi_protocol_drive"]
+           "had2_protocol_drive", "lhi_protocol_drive", "mm2_protocol_drive"]
 
 P = 0xFFFFFFFF00000001
 LIB_PATH = Path(__file__).resolve().with_name("libfp.so")
@@ -77,6 +77,8 @@ def lib():
     L.sumcheck_prove_hadamard.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.sumcheck_prove_hadamard_ext2.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_had2_protocol_drive.argtypes = [vp, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
+    L.sumcheck_prove_matmul_ext2.argtypes = [vp, vp, C.POINTER(_Site), vp, C.POINTER(sz), vp]
+    L.fp_mm2_protocol_drive.argtypes = [vp, i32, i32, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.logup_prove_helper_inverse.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
     L.fp_lhi_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, C.POINTER(sz), vp]
@@ -101,7 +103,7 @@ def lib():
 
 # int (*)(void* user, int kind, int t, const uint64_t* in, uint64_t* out)
 _VALUES_FN = C.CFUNCTYPE(C.c_int, C.c_void_p, C.c_int, C.c_int, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64))
-VAL_START, VAL_SINGLE, VAL_ROUND, VAL_ANSWER, VAL_FINALS, VAL_COLUMN = range(6)
+VAL_START, VAL_SINGLE, VAL_ROUND, VAL_ANSWER, VAL_FINALS, VAL_COLUMN, VAL_CLAIM = range(7)
 
 
 def had2_protocol_drive(tx: "Transcript", v: int, values) -> bytes:
@@ -135,6 +137,47 @@ def had2_protocol_drive(tx: "Transcript", v: int, values) -> bytes:
     rc = L.fp_had2_protocol_drive(tx.h, v, fn, None, buf, C.byref(ln))
     if rc != 0:
         raise FpError(rc, "fp_had2_protocol_drive failed")
+    return buf.raw[: ln.value]
+
+
+def mm2_protocol_drive(tx: "Transcript", vM: int, vN: int, n: int, values) -> bytes:
+    """Run the host half of the extension-field matmul sum-check with its device values taken
+    from `values` (no GPU work): values.start(r_row, r_col), values.claim() -> c,
+    values.round(t) -> (g(0), g(1), g(2)), values.answer(t, rho), values.finals() -> (A, B),
+    every extension element a pair (a, b). tx must have absorbed "mm2_site"."""
+    L = lib()
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            if kind == VAL_START:
+                pts = [(int(inp[2 * i]), int(inp[2 * i + 1])) for i in range(t)]
+                values.start(pts[:vM], pts[vM:])
+                return 0
+            if kind == VAL_ANSWER:
+                values.answer(t, (int(inp[0]), int(inp[1])))
+                return 0
+            if kind == VAL_CLAIM:
+                res = [values.claim()]
+            elif kind == VAL_ROUND:
+                res = values.round(t)
+            elif kind == VAL_FINALS:
+                res = values.finals()
+            else:
+                return 1
+            for i, (a, b) in enumerate(res):
+                out[2 * i] = int(a)
+                out[2 * i + 1] = int(b)
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _VALUES_FN(cb)
+    cap = 16 + 48 * n + 32
+    buf = C.create_string_buffer(cap)
+    ln = C.c_size_t(cap)
+    rc = L.fp_mm2_protocol_drive(tx.h, vM, vN, n, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_mm2_protocol_drive failed")
     return buf.raw[: ln.value]
 
 
@@ -355,6 +398,20 @@ class Context:
         ln = C.c_size_t(cap)
         self._check(self._L.sumcheck_prove_hadamard_ext2(self.h, tx.h, _ptr(s), _ptr(u), n, buf, C.byref(ln),
                                                          _stream(stream)), "sumcheck_prove_hadamard_ext2")
+        return buf.raw[: ln.value]
+
+    def prove_matmul_ext2(self, tx: Transcript, site: "SiteDesc", stream=None) -> bytes:
+        """The matmul sum-check of one committed site with every challenge and value in the
+        quadratic extension F_p[phi]/(phi^2 - 7); continues tx."""
+        arr, keep = _sites([site])
+        n = 0
+        while (1 << n) < int(site.K):
+            n += 1
+        cap = 16 + 48 * n + 32
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        self._check(self._L.sumcheck_prove_matmul_ext2(self.h, tx.h, arr, buf, C.byref(ln), _stream(stream)),
+                    "sumcheck_prove_matmul_ext2")
         return buf.raw[: ln.value]
 
     def prove_helper_inverse(self, tx: Transcript, r, k: int, stream=None):

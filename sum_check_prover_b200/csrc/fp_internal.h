@@ -45,6 +45,11 @@ enum FpKernel {
     K_LHI_COLUMN,
     K_LHI_ROUND,
     K_LHI_FINAL,
+    K_MM2_EQ,
+    K_MM2_CONTRACT,
+    K_MM2_CLAIM,
+    K_MM2_ROUND,
+    K_MM2_FINAL,
     K_COUNT
 };
 

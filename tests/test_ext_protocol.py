@@ -154,3 +154,112 @@ def test_callback_errors_and_small_buffers(fp):
     assert L.fp_had2_protocol_drive(fp.Transcript(0).h, 2, cb, None, buf, C.byref(ln)) != 0
     assert ln.value == 16 + 64 * 2 + 32
     assert L.fp_had2_protocol_drive(fp.Transcript(0).h, 31, cb, None, buf, C.byref(ln)) != 0
+
+
+# ---- the matmul sum-check over the extension ------------------------------------------
+
+import workloads  # noqa: E402
+
+
+class BruteMm2:
+    """Device values of the extension-field matmul sum-check by their definitions: every
+    MLE a double hypercube sum at an extension point."""
+
+    def __init__(self, site, wit, tamper=None):
+        q, r, _ = wit
+        self.M, self.K, self.N = site.M, site.K, site.N
+        self.vM, self.vN, self.n = bf.log2c(site.M), bf.log2c(site.N), bf.log2c(site.K)
+        self.W = bf.weights(site)
+        self.X = np.asarray(site.xt, np.int64).T
+        self.Y = ((1 << site.k_shift) * np.asarray(q, np.int64) + np.asarray(r, np.int64)).T
+        self.rho = []
+        self.tamper = tamper
+
+    @staticmethod
+    def _bits(x, v):
+        return [((x >> (v - 1 - b)) & 1, 0) for b in range(v)]
+
+    def _A(self, pt):
+        acc = (0, 0)
+        for i in range(self.M):
+            ei = bf.x_eq(self.zr, self._bits(i, self.vM))
+            for k in range(self.K):
+                e = bf.x_mul(ei, bf.x_eq(pt, self._bits(k, self.n)))
+                w = int(self.W[i, k]) % P
+                acc = bf.x_add(acc, (e[0] * w % P, e[1] * w % P))
+        return acc
+
+    def _B(self, pt):
+        acc = (0, 0)
+        for j in range(self.N):
+            ej = bf.x_eq(self.zc, self._bits(j, self.vN))
+            for k in range(self.K):
+                e = bf.x_mul(ej, bf.x_eq(pt, self._bits(k, self.n)))
+                x = int(self.X[k, j]) % P
+                acc = bf.x_add(acc, (e[0] * x % P, e[1] * x % P))
+        return acc
+
+    def start(self, zr, zc):
+        assert len(zr) == self.vM and len(zc) == self.vN
+        self.zr, self.zc = zr, zc
+
+    def claim(self):
+        c = (0, 0)
+        for i in range(self.M):
+            for j in range(self.N):
+                e = bf.x_mul(bf.x_eq(self.zr, self._bits(i, self.vM)), bf.x_eq(self.zc, self._bits(j, self.vN)))
+                y = int(self.Y[i, j]) % P
+                c = bf.x_add(c, (e[0] * y % P, e[1] * y % P))
+        return c
+
+    def round(self, t):
+        rest = self.n - t
+        g = []
+        for X in range(3):
+            acc = (0, 0)
+            for b in range(1 << rest):
+                pt = self.rho + [(X, 0)] + self._bits(b, rest)
+                acc = bf.x_add(acc, bf.x_mul(self._A(pt), self._B(pt)))
+            if self.tamper == (t, X):
+                acc = ((acc[0] + 1) % P, acc[1])
+            g.append(acc)
+        return g
+
+    def answer(self, t, rho):
+        assert t == len(self.rho) + 1
+        self.rho.append(rho)
+
+    def finals(self):
+        return [self._A(self.rho), self._B(self.rho)]
+
+
+def _mm_site(M, K, N, bits, scales, seed):
+    s = workloads.random_site(seed, M, K, N, bits, 6)
+    if scales:
+        s.scales = workloads.group_scales(np.random.default_rng(seed), M, K)
+    return s, oracle.witness(s)
+
+
+def _mm_drive(fp, seed, s, w, vals):
+    tx = fp.Transcript(seed)
+    tx.absorb("mm2_site", bf.site_digests([s], [w])[0][:160])
+    return fp.mm2_protocol_drive(tx, vals.vM, vals.vN, vals.n, vals), tx.state()
+
+
+@pytest.mark.parametrize("M,K,N,bits,scales", [(1, 1, 1, 8, False), (2, 4, 3, 8, False), (3, 5, 2, 4, True),
+                                               (4, 8, 4, 4, False), (5, 3, 6, 8, True)])
+def test_mm2_host_half_matches_oracle(fp, M, K, N, bits, scales):
+    s, w = _mm_site(M, K, N, bits, scales, 100 + M * 7 + K)
+    vals = BruteMm2(s, w)
+    pf, st = _mm_drive(fp, 8, s, w, vals)
+    want, wst = oracle.mm2_prove(8, s, w)
+    assert pf == want
+    assert st == wst
+    assert len(pf) == 16 + 48 * vals.n + 32
+
+
+@pytest.mark.parametrize("t,X", [(1, 0), (1, 1), (2, 1)])
+def test_mm2_inconsistent_round_is_refused(fp, t, X):
+    s, w = _mm_site(2, 4, 2, 8, False, 5)
+    with pytest.raises(fp.FpError):
+        _mm_drive(fp, 1, s, w, BruteMm2(s, w, tamper=(t, X)))
