@@ -211,6 +211,23 @@ void fp_session_post2(fp_ctx* c, uint64_t seq, uint64_t chal, uint64_t chal2) {
 
 void fp_session_post(fp_ctx* c, uint64_t seq, uint64_t chal) { fp_session_post2(c, seq, chal, 0); }
 
+// A session the host stops early (it refused a round's values) leaves its resident
+// kernel waiting; after its bounded wait the kernel would flag the mailbox under the
+// next session. Instead every later wait is answered at once (a sequence number above
+// all, the challenge 0) so the kernel runs to its end; its results are ignored. Then the
+// stream is drained and the mailbox returned to its empty state.
+void fp_session_abandon(fp_ctx* c, cudaStream_t s) {
+    if (!c) return;
+    fp_session_expect(c, 0);
+    fp_session_post2(c, ~0ull - 1, 0, 0);
+    cudaStreamSynchronize(s);
+    volatile FpMailbox* mb = c->mb;
+    _mm_store_si128((__m128i*)(&mb->chal), _mm_set_epi64x(0, 0));  // no kernel runs on the stream now
+    mb->chal2 = 0;
+    mb->err = 0;
+    c->t_result = -1;
+}
+
 const char* fp_last_error(const fp_ctx* c) { return c ? c->err.c_str() : "null context"; }
 
 int fp_reserve(fp_ctx* c, FpArena& a, size_t bytes) {

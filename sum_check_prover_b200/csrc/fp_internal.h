@@ -145,6 +145,8 @@ void fp_session_post(fp_ctx* c, uint64_t seq, uint64_t chal);
 void fp_session_expect(fp_ctx* c, int n);
 void fp_session_post2(fp_ctx* c, uint64_t seq, uint64_t chal, uint64_t chal2);
 int fp_session_begin(fp_ctx* c, cudaStream_t s);
+// Let a resident kernel of a session the host stopped early run to its end, and clear the mailbox.
+void fp_session_abandon(fp_ctx* c, cudaStream_t s);
 
 // transcript (transcript.cu)
 void fp_tx_absorb_raw(fp_tx* t, const char* label, const void* data, uint64_t n);

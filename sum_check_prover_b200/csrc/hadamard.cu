@@ -322,8 +322,10 @@ int prod_sumcheck(fp_ctx* c, fp_tx* tx, const Src& src, int64_t len, const FpPoi
             g[1] = gl_mul(pre, gl_mul(zt, h1));
             g[2] = gl_mul(pre, gl_mul(gl_sub(gl_mul(3, zt), 1), h2));
             g[3] = gl_mul(pre, gl_mul(gl_sub(gl_mul(5, zt), 2), h3));
-            if (gl_add(g[0], g[1]) != claim)
+            if (gl_add(g[0], g[1]) != claim) {
+                fp_session_abandon(c, st);
                 return fp_fail(c, FP_ERR_CUDA, std::string(who) + ": round values inconsistent with the claim");
+            }
             put_u64s(proof + pos, g, 4);
             fp_tx_absorb_raw(tx, lab.round, proof + pos, 32);
             pos += 32;

@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(H2_THREADS, 2) had2_session_kernel(Had2Args A,
 // Where the round values come from. Each call returns FP_OK or an error status.
 struct Had2Source {
     virtual ~Had2Source() {}
+    virtual void abandon() {}  // the host stopped early: let a waiting kernel finish
     virtual int start(const Ext2* z, int v) = 0;         // the point is known
     virtual int single(Ext2& claim, Ext2 fin[2]) = 0;    // v = 0: no rounds
     virtual int round(int t, Ext2 h[3]) = 0;             // h_t(0), h_t(1), h_t(2)
@@ -244,6 +245,7 @@ int had2_protocol(fp_ctx* c, fp_tx* tx, int v, Had2Source& src, uint8_t* proof, 
                 claim = e2_add(g[0], g[1]);
                 e2_send_host(tx, "had2_claim", &claim, 1, proof, pos);
             } else if (!e2_same(e2_add(g[0], g[1]), claim)) {
+                src.abandon();
                 return fp_fail(c, FP_ERR_CUDA, "sumcheck_prove_hadamard_ext2: round values inconsistent with the claim");
             }
             e2_send_host(tx, "had2_round", g, 4, proof, pos);
@@ -290,6 +292,8 @@ struct Had2Device : Had2Source {
         // reads, four factor writes and one E write; later rounds: eight factor reads instead
         return t == 1 ? 20.0 * pairs : (t == 2 ? 120.0 * pairs : 240.0 * pairs);
     }
+
+    void abandon() override { fp_session_abandon(c, st); }
 
     int start(const Ext2* z, int v) override {
         int rc;

@@ -203,6 +203,7 @@ __global__ void __launch_bounds__(LH_THREADS, 2) lhi_session_kernel(LhiArgs A, F
 // Where the device values come from. Each call returns FP_OK or an error status.
 struct LhiSource {
     virtual ~LhiSource() {}
+    virtual void abandon() {}  // the host stopped early: let a waiting kernel finish
     virtual int column(uint64_t alpha, uint8_t digest[32]) = 0;      // commit h, return D(h)
     virtual int start(const uint64_t* z, int v, uint64_t beta) = 0;  // the point is known
     virtual int round(int t, uint64_t vals[5]) = 0;                  // H(0), H(1), Q(0), Q(1), Q(2)
@@ -248,8 +249,10 @@ int lhi_protocol(fp_ctx* c, fp_tx* tx, int v, int k, const uint32_t* m, const ui
         const uint64_t eqX[4] = {gl_sub(1, zt), zt, gl_sub(gl_mul(3, zt), 1), gl_sub(gl_mul(5, zt), 2)};
         uint64_t g[4];
         for (int X = 0; X < 4; X++) g[X] = gl_add(H[X], gl_mul(scale, gl_mul(eqX[X], gl_sub(Q[X], 1))));
-        if (gl_add(g[0], g[1]) != claim)
+        if (gl_add(g[0], g[1]) != claim) {
+            src.abandon();
             return fp_fail(c, FP_ERR_CUDA, "logup_prove_helper_inverse: round values inconsistent with the claim");
+        }
         put_u64s(proof + pos, g, 4);
         fp_tx_absorb_raw(tx, "lhi_round", proof + pos, 32);
         pos += 32;
@@ -306,6 +309,8 @@ struct LhiDevice : LhiSource {
         // rounds read eight folded values instead
         return t == 1 ? 32.0 * pairs : (t == 2 ? 104.0 * pairs : 120.0 * pairs);
     }
+
+    void abandon() override { fp_session_abandon(c, st); }
 
     int column(uint64_t alpha, uint8_t digest[32]) override {
         const int64_t L = 1ll << v, T = 1ll << k;

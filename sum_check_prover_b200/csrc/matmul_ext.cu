@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(M2_THREADS, 2) mm2_session_kernel(Mm2Args P, F
 // Where the device values come from. Each call returns FP_OK or an error status.
 struct Mm2Source {
     virtual ~Mm2Source() {}
+    virtual void abandon() {}  // the host stopped early: let a waiting kernel finish
     virtual int start(const Ext2* zr, int vM, const Ext2* zc, int vN) = 0;  // the point is known
     virtual int claim(Ext2& c) = 0;                                          // Y~(r_row, r_col)
     virtual int round(int t, Ext2 g[3]) = 0;                                 // g_t(0), g_t(1), g_t(2)
@@ -223,8 +224,10 @@ int mm2_protocol(fp_ctx* c, fp_tx* tx, int vM, int vN, int n, Mm2Source& src, ui
     for (int t = 1; t <= n; t++) {
         Ext2 g[3];
         if ((rc = src.round(t, g))) return rc;
-        if (!e2_same(e2_add(g[0], g[1]), claim))
+        if (!e2_same(e2_add(g[0], g[1]), claim)) {
+            src.abandon();
             return fp_fail(c, FP_ERR_CUDA, "sumcheck_prove_matmul_ext2: round values inconsistent with the claim");
+        }
         e2_send_host(tx, "mm2_round", g, 3, proof, pos);
         const Ext2 r = e2_squeeze_host(tx, "mm2_chal");
         if ((rc = src.answer(t, r))) return rc;
@@ -274,6 +277,8 @@ struct Mm2Device : Mm2Source {
         c->launches++;  // two kernels under one timing slot
         return FP_OK;
     }
+
+    void abandon() override { fp_session_abandon(c, st); }
 
     int start(const Ext2* zr, int vM, const Ext2* zc, int vN) override {
         for (int i = 0; i < vM; i++) {

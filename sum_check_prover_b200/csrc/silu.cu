@@ -398,8 +398,10 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
             gr[1] = gl_mul(pre, gl_mul(zt, h1));
             gr[2] = gl_mul(pre, gl_mul(gl_sub(gl_mul(3, zt), 1), h2));
             gr[3] = gl_mul(pre, gl_mul(gl_sub(gl_mul(5, zt), 2), h3));
-            if (gl_add(gr[0], gr[1]) != claim)
+            if (gl_add(gr[0], gr[1]) != claim) {
+                fp_session_abandon(c, st);
                 return fp_fail(c, FP_ERR_CUDA, "logup_prove_silu: round values inconsistent with the claim");
+            }
             put_u64s(proof + pos, gr, 4);
             fp_tx_absorb_raw(tx, lab.round, proof + pos, 32);
             pos += 32;
