@@ -124,6 +124,14 @@ int fp_session_begin(fp_ctx* c, cudaStream_t s) {
     return FP_OK;
 }
 
+// a failed wait: record the error, then let whatever is still resident run out
+// (fp_session_abandon) so the next session starts from an empty mailbox
+static int session_fail(fp_ctx* c, cudaStream_t s, int code, const char* msg) {
+    const int rc = fp_fail(c, code, msg);
+    fp_session_abandon(c, s);
+    return rc;
+}
+
 int fp_session_wait(fp_ctx* c, uint64_t seq, cudaStream_t s) {
     (void)seq;
     const volatile FpMailbox* mb = c->mb;
@@ -143,7 +151,7 @@ int fp_session_wait(fp_ctx* c, uint64_t seq, cudaStream_t s) {
             return FP_OK;
         }
         if ((spin & 255) != 255) continue;
-        if (mb->err) return fp_fail(c, FP_ERR_TIMEOUT, "a persistent kernel stopped waiting for the host");
+        if (mb->err) return session_fail(c, s, FP_ERR_TIMEOUT, "a persistent kernel stopped waiting for the host");
         const auto now = clk::now();
         if (now < next_query) continue;
         // the device may have failed: look at the stream every couple of milliseconds
@@ -153,11 +161,15 @@ int fp_session_wait(fp_ctx* c, uint64_t seq, cudaStream_t s) {
             bool done = true;
             for (int i = 0; i < n; i++) done = done && (mb->res[i] != kEmpty);
             if (done) continue;
-            if (q != cudaSuccess) return fp_cuda_check(c, q, "persistent kernel");
-            return fp_fail(c, FP_ERR_TIMEOUT, "a persistent kernel ended without publishing");
+            if (q != cudaSuccess) {
+                const int rc = fp_cuda_check(c, q, "persistent kernel");
+                fp_session_abandon(c, s);
+                return rc;
+            }
+            return session_fail(c, s, FP_ERR_TIMEOUT, "a persistent kernel ended without publishing");
         }
         if (std::chrono::duration<double>(now - t0).count() > 30.0)
-            return fp_fail(c, FP_ERR_TIMEOUT, "no answer from the device within 30 s");
+            return session_fail(c, s, FP_ERR_TIMEOUT, "no answer from the device within 30 s");
     }
 }
 
