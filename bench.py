@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2"
+MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2,frv"
 
 
 def micro_names(which) -> set:
@@ -208,6 +208,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
       the helper column and the keys, later rounds fold both: 104 and 120 B per pair).
     mm2_contract: the extension-field matmul's row contraction of a 16384 x 16384 int4
       weight (the matrix once; the eq weights are 16-byte extension elements).
+    frv_u: Freivalds' prover, u = X rho^(.) over a 16384-token x 16384 int8 activation
+      (the activation once, plus the powers of rho).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
@@ -360,6 +362,17 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
             del st, keep, d
         except Exception as e:  # a failure here must not cost the rest of the line
             out["ext2_contract_16384x16384_int4"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    if "frv" in which:
+        # Freivalds' prover for 16384 tokens of a 16384-wide activation (256 MiB of Xt)
+        try:
+            s = workloads.random_site(79, 128, 16384, 16384, 4, 12)
+            st, keep = device.upload(workloads.Workload("frv", 0, [s]), dev)
+            d = st[0][0]
+            ctx.commit_witness(fp.Transcript(0), [d])
+            measure("freivalds_u_16384x16384", "frv_u", lambda: ctx.prove_freivalds(fp.Transcript(9), d))
+            del st, keep, d
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["freivalds_u_16384x16384"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     try:
         torch.cuda.empty_cache()

@@ -375,6 +375,22 @@ int sumcheck_prove_matmul_ext2(fp_ctx* ctx, fp_tx* tx, const fp_site* site, uint
                                void* stream);
 
 /*
+ * Freivalds' check of a weight matmul, the prover's side ("Towards Proving
+ * Frontier-Scale LLM Inference", The proof system: the weight matmuls are
+ * checked by Freivalds' algorithm, A (B r) = C r for a random vector r), the
+ * comparison statement for the matmul sum-check. site: one fp_site with its
+ * witness; device pointers, caller-owned, read only. The call continues tx:
+ *   absorb "frv_site" D(W) || D(S) || D(Xt) || D(q) || D(r) (D(W) || D(S) from
+ *   site->w_digest when given); squeeze rho ("frv_rho"); send
+ *   u_k = sum_j X[k][j] rho^j for k < K ("frv_u").
+ * The verifier checks u against X and sum_k W_eff[i][k] u_k =
+ * sum_j (2^k q + r)[j][i] rho^j for every row i. Proof bytes: 8 K. Site checks
+ * and errors as for sumcheck_prove_matmul.
+ */
+int freivalds_prove_matmul(fp_ctx* ctx, fp_tx* tx, const fp_site* site, uint8_t* proof, size_t* proof_len,
+                           void* stream);
+
+/*
  * The host half of sumcheck_prove_matmul_ext2 (vM, vN point coordinates, n
  * rounds); tx must have absorbed "mm2_site". Callback kinds:
  *   FP_VAL_START: in = r_row then r_col (2 (vM + vN) words), t = vM + vN;

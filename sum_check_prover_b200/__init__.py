@@ -78,6 +78,7 @@ def lib():
     L.sumcheck_prove_hadamard_ext2.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_had2_protocol_drive.argtypes = [vp, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.sumcheck_prove_matmul_ext2.argtypes = [vp, vp, C.POINTER(_Site), vp, C.POINTER(sz), vp]
+    L.freivalds_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), vp, C.POINTER(sz), vp]
     L.fp_mm2_protocol_drive.argtypes = [vp, i32, i32, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.logup_prove_helper_inverse.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
     L.fp_lhi_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
@@ -412,6 +413,17 @@ class Context:
         ln = C.c_size_t(cap)
         self._check(self._L.sumcheck_prove_matmul_ext2(self.h, tx.h, arr, buf, C.byref(ln), _stream(stream)),
                     "sumcheck_prove_matmul_ext2")
+        return buf.raw[: ln.value]
+
+    def prove_freivalds(self, tx: Transcript, site: "SiteDesc", stream=None) -> bytes:
+        """Freivalds' check of one committed site, the prover's side: u = X rho^(.) (K field
+        elements); continues tx."""
+        arr, keep = _sites([site])
+        cap = 8 * int(site.K)
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        self._check(self._L.freivalds_prove_matmul(self.h, tx.h, arr, buf, C.byref(ln), _stream(stream)),
+                    "freivalds_prove_matmul")
         return buf.raw[: ln.value]
 
     def prove_helper_inverse(self, tx: Transcript, r, k: int, stream=None):

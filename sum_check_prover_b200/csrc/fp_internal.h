@@ -50,6 +50,7 @@ enum FpKernel {
     K_MM2_CLAIM,
     K_MM2_ROUND,
     K_MM2_FINAL,
+    K_FRV_U,
     K_COUNT
 };
 
@@ -162,6 +163,9 @@ struct FpDigestJob {
     uint64_t len;
 };
 int fp_digest_many(fp_ctx* c, const FpDigestJob* jobs, int njobs, uint8_t* out, cudaStream_t s);
+// D(W) || D(S) || D(Xt) || D(q) || D(r) of one site (D(W) || D(S) from w_digest when given;
+// matmul_ext.cu); synchronises the stream
+int fp_site_digest160(fp_ctx* c, const fp_site& s, uint8_t d[160], cudaStream_t st);
 
 // witness (witness.cu)
 int fp_launch_witness(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t s);

@@ -433,6 +433,22 @@ size_t mm2_proof_len(int n) { return 16 + 48 * (size_t)n + 32; }
 
 }  // namespace
 
+int fp_site_digest160(fp_ctx* c, const fp_site& s, uint8_t d[160], cudaStream_t st) {
+    const uint64_t mn = (uint64_t)s.M * s.N;
+    const uint64_t wb = (uint64_t)s.M * (s.w_bits == 4 ? (uint64_t)((s.K + 1) / 2) : (uint64_t)s.K);
+    const uint64_t sb = s.scales ? (uint64_t)s.M * ((s.K + 63) / 64) : 0;
+    FpDigestJob jobs[5] = {{(const uint8_t*)s.w, wb},
+                           {(const uint8_t*)s.scales, sb},
+                           {(const uint8_t*)s.xt, (uint64_t)s.N * s.K},
+                           {(const uint8_t*)s.q, 4 * mn},
+                           {(const uint8_t*)s.r, 4 * mn}};
+    if (s.w_digest) {
+        memcpy(d, s.w_digest, 64);
+        return fp_digest_many(c, jobs + 2, 3, d + 64, st);  // synchronises the stream
+    }
+    return fp_digest_many(c, jobs, 5, d, st);
+}
+
 int sumcheck_prove_matmul_ext2(fp_ctx* c, fp_tx* tx, const fp_site* site, uint8_t* proof, size_t* proof_len,
                                void* stream) {
     if (!c || !tx || !proof_len || !site) return fp_fail(c, FP_ERR_ARG, "sumcheck_prove_matmul_ext2: null argument");
@@ -448,22 +464,8 @@ int sumcheck_prove_matmul_ext2(fp_ctx* c, fp_tx* tx, const fp_site* site, uint8_
     FP_CUDA(c, cudaSetDevice(c->device));
     cudaStream_t st = (cudaStream_t)stream;
     {
-        // D(W) || D(S) || D(Xt) || D(q) || D(r); the weights' pair from w_digest when given
-        const uint64_t mn = (uint64_t)s.M * s.N;
-        const uint64_t wb = (uint64_t)s.M * (s.w_bits == 4 ? (uint64_t)((s.K + 1) / 2) : (uint64_t)s.K);
-        const uint64_t sb = s.scales ? (uint64_t)s.M * ((s.K + 63) / 64) : 0;
-        FpDigestJob jobs[5] = {{(const uint8_t*)s.w, wb},
-                               {(const uint8_t*)s.scales, sb},
-                               {(const uint8_t*)s.xt, (uint64_t)s.N * s.K},
-                               {(const uint8_t*)s.q, 4 * mn},
-                               {(const uint8_t*)s.r, 4 * mn}};
         uint8_t d[160];
-        if (s.w_digest) {
-            memcpy(d, s.w_digest, 64);
-            if ((rc = fp_digest_many(c, jobs + 2, 3, d + 64, st))) return rc;  // synchronises the stream
-        } else if ((rc = fp_digest_many(c, jobs, 5, d, st))) {
-            return rc;
-        }
+        if ((rc = fp_site_digest160(c, s, d, st))) return rc;
         fp_tx_absorb_raw(tx, "mm2_site", d, 160);
     }
     Mm2Device dev;

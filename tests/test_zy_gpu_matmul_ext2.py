@@ -100,3 +100,34 @@ def test_ffn_projection_verified(env):
     pf, st, d = _prove(env, s, 12)
     assert len(pf) == 16 + 48 * 14 + 32
     assert oracle.mm2_verify(12, s, oracle.witness(s), pf) == ("accept", (0, 0))
+
+
+# ---- Freivalds' check, the prover's side (the comparison statement) ------------------
+
+def _freivalds(env, s, seed, offline_digest=False):
+    torch, fp, ctx = env
+    stages, keep = device.upload(workloads.Workload("frv", 0, [s]))
+    d = stages[0][0]
+    if offline_digest:
+        device.weight_digests(ctx, stages)
+    ctx.commit_witness(fp.Transcript(0), [d])
+    tx = fp.Transcript(seed)
+    pf = ctx.prove_freivalds(tx, d)
+    torch.cuda.synchronize()
+    return pf, tx.state()
+
+
+@pytest.mark.parametrize("M,K,N,bits,scales", [(1, 1, 1, 8, False), (3, 5, 2, 4, True), (64, 256, 300, 8, False),
+                                               (100, 1000, 4097, 4, True)])
+def test_freivalds_matches_oracle(env, M, K, N, bits, scales):
+    s = _site(M, K, N, bits, scales, 700 + M + K + N)
+    w = oracle.witness(s)
+    pf, st = _freivalds(env, s, 2)
+    assert (pf, st) == oracle.frv_prove(2, s, w)
+    assert oracle.frv_verify(2, s, w, pf) == ("accept", (0, 0))
+
+
+def test_freivalds_offline_weight_digest(env):
+    s = _site(32, 640, 48, 4, True, 12)
+    assert _freivalds(env, s, 5) == _freivalds(env, s, 5, offline_digest=True) == oracle.frv_prove(5, s,
+                                                                                                   oracle.witness(s))
