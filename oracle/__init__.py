@@ -62,6 +62,9 @@ REASONS = {
     29: "lhi_round",
     30: "lhi_final",
     31: "lhi_open",
+    34: "route_open",
+    35: "route_round",
+    36: "route_final",
 }
 
 
@@ -159,6 +162,12 @@ def lib():
         L.orc_frv_prove.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, C.POINTER(u64)]
         L.orc_frv_verify.restype = C.c_int
         L.orc_frv_verify.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, vp]
+        L.orc_route_witness.restype = None
+        L.orc_route_witness.argtypes = [vp, u64, C.c_int, vp, vp]
+        L.orc_route_prove.restype = C.c_int
+        L.orc_route_prove.argtypes = [vp, vp, vp, vp, u64, C.c_int, vp, u64, C.POINTER(u64)]
+        L.orc_route_verify.restype = C.c_int
+        L.orc_route_verify.argtypes = [vp, vp, vp, vp, u64, C.c_int, vp, u64, vp]
         L.orc_mm2_prove.restype = C.c_int
         L.orc_mm2_prove.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, C.POINTER(u64)]
         L.orc_mm2_verify.restype = C.c_int
@@ -694,5 +703,53 @@ def _site_verify(fn, seed: int, site, wit, proof: bytes):
     det = np.zeros(2, dtype=np.int64)
     tx = L.orc_tx_new(seed)
     rc = fn(tx, C.byref(cs), C.byref(cw), _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+# ---- MoE routing (top-1, the first argmax of the router logits) ---------------------
+
+def route_witness(l, T: int, E: int):
+    """(H, D): the one-hot first-argmax choice (T x E u8) and D = l[t][e_t] - l[t][e] - [e < e_t]
+    (T x E int32) of the router logits l (T x E int8, token-major)."""
+    L = lib()
+    a = np.ascontiguousarray(np.asarray(l, dtype=np.int8).reshape(-1))
+    H = np.zeros(T * E, dtype=np.uint8)
+    D = np.zeros(T * E, dtype=np.int32)
+    L.orc_route_witness(_ptr(a), T, E, _ptr(H), _ptr(D))
+    return H.reshape(T, E), D.reshape(T, E)
+
+
+def route_prove(seed: int, l, H, D, T: int, E: int):
+    """The routing proof (sum-check tying D to H and l, H one-hot; the range of D by the
+    helper-inverse LogUp) for the given witness; returns (proof bytes, transcript state)."""
+    L = lib()
+    a = np.ascontiguousarray(np.asarray(l, dtype=np.int8).reshape(-1))
+    h = np.ascontiguousarray(np.asarray(H, dtype=np.uint8).reshape(-1))
+    d = np.ascontiguousarray(np.asarray(D, dtype=np.int32).reshape(-1))
+    n = C.c_uint64(0)
+    tx = L.orc_tx_new(seed)
+    L.orc_route_prove(tx, _ptr(a), _ptr(h), _ptr(d), T, E, None, 0, C.byref(n))
+    L.orc_tx_free(tx)
+    buf = np.zeros(max(1, n.value), dtype=np.uint8)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_route_prove(tx, _ptr(a), _ptr(h), _ptr(d), T, E, _ptr(buf), n.value, C.byref(n))
+    st = C.create_string_buffer(32)
+    L.orc_tx_state(tx, st)
+    L.orc_tx_free(tx)
+    if rc != 0:
+        raise ValueError(f"orc_route_prove failed ({rc})")
+    return buf[: n.value].tobytes(), st.raw
+
+
+def route_verify(seed: int, l, H, D, T: int, E: int, proof: bytes):
+    L = lib()
+    a = np.ascontiguousarray(np.asarray(l, dtype=np.int8).reshape(-1))
+    h = np.ascontiguousarray(np.asarray(H, dtype=np.uint8).reshape(-1))
+    d = np.ascontiguousarray(np.asarray(D, dtype=np.int32).reshape(-1))
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_route_verify(tx, _ptr(a), _ptr(h), _ptr(d), T, E, _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

@@ -2420,3 +2420,249 @@ done:
     free(E);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MoE routing (next row f3; "How fast can FlashProve go", 2 Background, the */
+/* note on MoE layers: they also prove the routing computation and each      */
+/* token's choice of expert). Top-1 routing over E experts (E a power of     */
+/* two): token t goes to e_t, the first index of the largest of its router   */
+/* logits l[t][.] (int8, token-major T x E: the router matmul's rescaled      */
+/* outputs). The prover commits the one-hot choice H[t][e] = [e = e_t] (u8)  */
+/* and D[t][e] = l[t][e_t] - l[t][e] - [e < e_t] (int32), which lies in      */
+/* [0, 256) for every e exactly when e_t is the first maximum. All columns   */
+/* are zero-padded from T to 2^vT rows; x = t E + e, the t bits first.       */
+/*   absorb "route_site" D(l) || D(H) || D(D as int32 little-endian);        */
+/*   squeeze z (vT + vE, "route_z"), w (vT + vE, "route_w"), lambda1 and     */
+/*   lambda2 ("route_lambda");                                               */
+/*   send D~(z), l~(z) ("route_open");                                       */
+/*   sum-check over vT + vE variables of                                    */
+/*     F(x) = eq(z_t, t) H(x) (l(x) - G(e)) + lambda1 eq(w, x) H(x) (1 - H(x))*/
+/*            + lambda2 eq(w_t, t) H(x),   G(e) = sum_{e' < e} eq(z_e, e'),   */
+/*   claim D~(z) + l~(z) + lambda2 sum_{t < T} eq(w_t, t): rounds g(0..3)     */
+/*   ("route_round"), "route_chal"; send H~(rho), l~(rho) ("route_final");  */
+/*   then the helper-inverse LogUp of the keys D - 128 on R_8 (the statement */
+/*   of orc_lhi_prove, T E keys, the same transcript).                       */
+/* Why: sum_t eq(z_t, t) (l[t][e_t] - l~(t, z_e) - sum_e eq(z_e, e) [e < e_t])*/
+/* is D~(z), and it equals the first sum minus l~(z) because                 */
+/* sum_e eq(z_e, e) [e < e'] = G(e'); the second term forces H Boolean and   */
+/* the third forces every real row of H to sum to 1 (padded rows to 0), each  */
+/* with high probability over w; the range check then makes e_t the first    */
+/* argmax.                                                                   */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_ROUTE_OPEN = 34,  /* an opened value != the column's MLE; detail[0]: 0 D(z), 1 l(z), 2 H(rho), 3 l(rho) */
+    REJ_ROUTE_ROUND = 35, /* g(0) + g(1) != running claim; detail[0] = round */
+    REJ_ROUTE_FINAL = 36  /* the end does not match F at rho */
+};
+
+/* the honest witness: H and D of the first argmax of every row */
+void orc_route_witness(const int8_t* l, u64 T, int E, uint8_t* H, int32_t* D) {
+    for (u64 t = 0; t < T; t++) {
+        const int8_t* row = l + t * (u64)E;
+        int best = 0;
+        for (int e = 1; e < E; e++)
+            if (row[e] > row[best]) best = e;
+        for (int e = 0; e < E; e++) {
+            H[t * (u64)E + e] = (uint8_t)(e == best);
+            D[t * (u64)E + e] = (int32_t)row[best] - (int32_t)row[e] - (e < best ? 1 : 0);
+        }
+    }
+}
+
+typedef struct {
+    int vT, vE, n;
+    u64 L;
+    u64 *z, *w, lam1, lam2;
+    u64 *Hv, *lv, *Dv; /* lifted, zero-padded, length L */
+} route_ctx;
+
+static int route_begin(orc_tx* t, const int8_t* l, const uint8_t* H, const int32_t* D, u64 T, int E, route_ctx* c) {
+    if (T < 1 || E < 1 || (E & (E - 1)) || E > 4096) return -1;
+    c->vT = orc_log2_ceil(T);
+    c->vE = orc_log2_ceil((u64)E);
+    c->n = c->vT + c->vE;
+    c->L = (u64)1 << c->n;
+    u64 TE = T * (u64)E;
+    uint8_t dg[96];
+    uint8_t* db = (uint8_t*)calloc(4 * TE + 1, 1);
+    for (u64 i = 0; i < TE; i++) put_le(db + 4 * i, (u64)(u32)D[i], 4);
+    orc_tree_digest(l, TE, dg);
+    orc_tree_digest(H, TE, dg + 32);
+    orc_tree_digest(db, 4 * TE, dg + 64);
+    free(db);
+    orc_tx_absorb(t, "route_site", dg, 96);
+    c->z = (u64*)malloc(sizeof(u64) * (c->n + 1));
+    c->w = (u64*)malloc(sizeof(u64) * (c->n + 1));
+    for (int i = 0; i < c->n; i++) c->z[i] = orc_tx_squeeze(t, "route_z");
+    for (int i = 0; i < c->n; i++) c->w[i] = orc_tx_squeeze(t, "route_w");
+    c->lam1 = orc_tx_squeeze(t, "route_lambda");
+    c->lam2 = orc_tx_squeeze(t, "route_lambda");
+    c->Hv = (u64*)calloc(c->L, sizeof(u64));
+    c->lv = (u64*)calloc(c->L, sizeof(u64));
+    c->Dv = (u64*)calloc(c->L, sizeof(u64));
+    for (u64 i = 0; i < TE; i++) {
+        c->Hv[i] = (u64)H[i] % ORC_P;
+        c->lv[i] = orc_fint(l[i]);
+        c->Dv[i] = orc_fint(D[i]);
+    }
+    return 0;
+}
+
+static void route_end(route_ctx* c) {
+    free(c->z);
+    free(c->w);
+    free(c->Hv);
+    free(c->lv);
+    free(c->Dv);
+}
+
+/* G(e) = sum_{e' < e} eq(z_e, e') for e < E */
+static void route_G(const u64* ze, int vE, int E, u64* G) {
+    u64* eq = (u64*)malloc(sizeof(u64) * E);
+    orc_eq_table(ze, vE, eq);
+    u64 acc = 0;
+    for (int e = 0; e < E; e++) {
+        G[e] = acc;
+        acc = orc_fadd(acc, eq[e]);
+    }
+    free(eq);
+}
+
+/* sum_{t < T} eq(w_t, t) */
+static u64 route_rowsum(const u64* wt, int vT, u64 T) {
+    u64* eq = (u64*)malloc(sizeof(u64) * ((u64)1 << vT));
+    orc_eq_table(wt, vT, eq);
+    u64 acc = 0;
+    for (u64 t = 0; t < T; t++) acc = orc_fadd(acc, eq[t]);
+    free(eq);
+    return acc;
+}
+
+/* the keys D - 128 of the range lookup */
+static int32_t* route_keys(const int32_t* D, u64 TE) {
+    int32_t* k = (int32_t*)malloc(sizeof(int32_t) * (TE ? TE : 1));
+    for (u64 i = 0; i < TE; i++) k[i] = (int32_t)((int64_t)D[i] - 128);
+    return k;
+}
+
+int orc_route_prove(void* txh, const int8_t* l, const uint8_t* H, const int32_t* D, u64 T, int E, uint8_t* proof,
+                    u64 cap, u64* len) {
+    orc_tx* t = (orc_tx*)txh;
+    route_ctx c;
+    if (route_begin(t, l, H, D, T, E, &c)) return -1;
+    pbuf pb = {proof, cap, 0, 0};
+    u64 open[2] = {orc_mle_eval(c.Dv, c.L, c.z, c.n), orc_mle_eval(c.lv, c.L, c.z, c.n)};
+    send_fe(t, &pb, "route_open", open, 2);
+    /* the factors as vectors over x: eq(z_t, t), G(e), eq(w, x), eq(w_t, t) */
+    u64 L = c.L;
+    u64* Et = (u64*)malloc(sizeof(u64) * L);
+    u64* Gv = (u64*)malloc(sizeof(u64) * L);
+    u64* Ew = (u64*)malloc(sizeof(u64) * L);
+    u64* Ewt = (u64*)malloc(sizeof(u64) * L);
+    {
+        u64* et = (u64*)malloc(sizeof(u64) * ((u64)1 << c.vT));
+        u64* ewt = (u64*)malloc(sizeof(u64) * ((u64)1 << c.vT));
+        u64* G = (u64*)malloc(sizeof(u64) * E);
+        orc_eq_table(c.z, c.vT, et);
+        orc_eq_table(c.w, c.vT, ewt);
+        orc_eq_table(c.w, c.n, Ew);
+        route_G(c.z + c.vT, c.vE, E, G);
+        for (u64 x = 0; x < L; x++) {
+            Et[x] = et[x >> c.vE];
+            Ewt[x] = ewt[x >> c.vE];
+            Gv[x] = G[x & (u64)(E - 1)];
+        }
+        free(et);
+        free(ewt);
+        free(G);
+    }
+    u64* V[6] = {Et, c.Hv, c.lv, Gv, Ew, Ewt};
+    u64 Lr = L;
+    for (int r = 0; r < c.n; r++) {
+        u64 h = Lr >> 1;
+        u64 g[4] = {0, 0, 0, 0};
+        for (u64 b = 0; b < h; b++)
+            for (u64 X = 0; X < 4; X++) {
+                u64 at[6];
+                for (int k = 0; k < 6; k++) at[k] = orc_fadd(V[k][b], orc_fmul(X, orc_fsub(V[k][h + b], V[k][b])));
+                u64 Hx = at[1];
+                u64 f = orc_fmul(at[0], orc_fmul(Hx, orc_fsub(at[2], at[3])));
+                f = orc_fadd(f, orc_fmul(c.lam1, orc_fmul(at[4], orc_fmul(Hx, orc_fsub(1, Hx)))));
+                f = orc_fadd(f, orc_fmul(c.lam2, orc_fmul(at[5], Hx)));
+                g[X] = orc_fadd(g[X], f);
+            }
+        send_fe(t, &pb, "route_round", g, 4);
+        u64 rho = orc_tx_squeeze(t, "route_chal");
+        for (int k = 0; k < 6; k++)
+            for (u64 b = 0; b < h; b++) V[k][b] = orc_fadd(V[k][b], orc_fmul(rho, orc_fsub(V[k][h + b], V[k][b])));
+        Lr = h;
+    }
+    u64 fin[2] = {c.Hv[0], c.lv[0]};
+    send_fe(t, &pb, "route_final", fin, 2);
+    free(Et);
+    free(Gv);
+    free(Ew);
+    free(Ewt);
+    /* the range of D: the helper-inverse LogUp on R_8, continuing the transcript */
+    u64 TE = T * (u64)E, l2 = 0;
+    int32_t* keys = route_keys(D, TE);
+    int rc = orc_lhi_prove(txh, keys, TE, 8, pb.overflow || !proof ? NULL : proof + pb.len,
+                           pb.overflow || cap < pb.len ? 0 : cap - pb.len, &l2);
+    free(keys);
+    route_end(&c);
+    *len = pb.len + l2;
+    if (rc == -2 || pb.overflow) return -2;
+    return rc;
+}
+
+int orc_route_verify(void* txh, const int8_t* l, const uint8_t* H, const int32_t* D, u64 T, int E,
+                     const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    orc_tx* t = (orc_tx*)txh;
+    route_ctx c;
+    if (route_begin(t, l, H, D, T, E, &c)) return REJ_ARGS;
+    int rc = 0;
+    u64* rho = (u64*)malloc(sizeof(u64) * (c.n + 1));
+    prd rd = {proof, len, 0, 0};
+    u64 open[2];
+    rd_fe(t, &rd, "route_open", open, 2);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    if (open[0] != orc_mle_eval(c.Dv, c.L, c.z, c.n)) FAIL(REJ_ROUTE_OPEN, 0, 0);
+    if (open[1] != orc_mle_eval(c.lv, c.L, c.z, c.n)) FAIL(REJ_ROUTE_OPEN, 1, 0);
+    {
+        u64 claim = orc_fadd(orc_fadd(open[0], open[1]), orc_fmul(c.lam2, route_rowsum(c.w, c.vT, T)));
+        for (int r = 0; r < c.n; r++) {
+            u64 g[4];
+            rd_fe(t, &rd, "route_round", g, 4);
+            if (rd.bad) FAIL(REJ_FORMAT, 1, r);
+            if (orc_fadd(g[0], g[1]) != claim) FAIL(REJ_ROUTE_ROUND, r, 0);
+            rho[r] = orc_tx_squeeze(t, "route_chal");
+            claim = orc_lagrange(g, 4, rho[r]);
+        }
+        u64 fin[2];
+        rd_fe(t, &rd, "route_final", fin, 2);
+        if (rd.bad) FAIL(REJ_FORMAT, 2, 0);
+        if (fin[0] != orc_mle_eval(c.Hv, c.L, rho, c.n)) FAIL(REJ_ROUTE_OPEN, 2, 0);
+        if (fin[1] != orc_mle_eval(c.lv, c.L, rho, c.n)) FAIL(REJ_ROUTE_OPEN, 3, 0);
+        u64* G = (u64*)malloc(sizeof(u64) * E);
+        route_G(c.z + c.vT, c.vE, E, G);
+        u64 Gr = orc_mle_eval(G, (u64)E, rho + c.vT, c.vE);
+        free(G);
+        u64 Hr = fin[0], lr = fin[1];
+        u64 f = orc_fmul(eq_closed(c.z, rho, c.vT), orc_fmul(Hr, orc_fsub(lr, Gr)));
+        f = orc_fadd(f, orc_fmul(c.lam1, orc_fmul(eq_closed(c.w, rho, c.n), orc_fmul(Hr, orc_fsub(1, Hr)))));
+        f = orc_fadd(f, orc_fmul(c.lam2, orc_fmul(eq_closed(c.w, rho, c.vT), Hr)));
+        if (f != claim) FAIL(REJ_ROUTE_FINAL, 0, 0);
+    }
+    {
+        u64 TE = T * (u64)E;
+        int32_t* keys = route_keys(D, TE);
+        rc = orc_lhi_verify(txh, keys, TE, 8, proof + rd.pos, len - rd.pos, detail);
+        free(keys);
+    }
+done:
+    free(rho);
+    route_end(&c);
+    return rc;
+}

@@ -516,6 +516,11 @@ def lookup16_prove(seed: int, g, s, prefix: str, pad_s: int) -> bytes:
 def lhi_prove(seed: int, r, k: int) -> bytes:
     """The helper-inverse LogUp proof from definitions: h by Python modular inverses, every
     round value a hypercube sum of h + beta eq (h (alpha - f) - 1) over MLEs (no folding)."""
+    return lhi_body(Tx(seed), r, k)
+
+
+def lhi_body(tx, r, k: int) -> bytes:
+    """The helper-inverse LogUp proof continuing the transcript tx."""
     r = [int(x) for x in np.asarray(r).reshape(-1)]
     n = len(r)
     v = max(1, log2c(n))
@@ -528,7 +533,6 @@ def lhi_prove(seed: int, r, k: int) -> bytes:
         out.extend(b)
         tx.absorb(label, b)
 
-    tx = Tx(seed)
     tx.absorb("lhi_site", tree_digest(np.asarray(r, "<i4").tobytes()))
     m = np.zeros(1 << k, np.int64)
     for x in r + [0] * (L - n):
@@ -702,3 +706,70 @@ def mm2_prove(seed: int, site, wit) -> bytes:
         rho.append(squeeze_ext("mm2_chal"))
     send("mm2_final", [A_at(rho), B_at(rho)])
     return bytes(out)
+
+
+# ---- MoE routing: the first argmax of every token's router logits ----------------------
+
+def route_witness(l, T: int, E: int):
+    """H (one-hot of the first maximum of every row) and D = l[t][e_t] - l[t][e] - [e < e_t]."""
+    l = np.asarray(l, np.int64).reshape(T, E)
+    H = np.zeros((T, E), np.uint8)
+    D = np.zeros((T, E), np.int64)
+    for t in range(T):
+        best = max(range(E), key=lambda e: (int(l[t, e]), -e))
+        H[t, best] = 1
+        for e in range(E):
+            D[t, e] = int(l[t, best]) - int(l[t, e]) - (1 if e < best else 0)
+    return H, D.astype(np.int32)
+
+
+def route_prove(seed: int, l, H, D, T: int, E: int) -> bytes:
+    """The routing proof from definitions: every round value a hypercube sum of F over the
+    unbound variables, with H, l, G and the eq factors as MLEs at the point (no folding)."""
+    l = np.asarray(l, np.int64).reshape(-1)
+    H = np.asarray(H, np.int64).reshape(-1)
+    D = np.asarray(D, np.int64).reshape(-1)
+    vT, vE = log2c(T), log2c(E)
+    n = vT + vE
+    tx = Tx(seed)
+    tx.absorb("route_site", tree_digest(np.asarray(l, np.int8).tobytes()) + tree_digest(np.asarray(H, np.uint8).tobytes())
+              + tree_digest(np.asarray(D, "<i4").tobytes()))
+    z = [tx.squeeze("route_z") for _ in range(n)]
+    w = [tx.squeeze("route_w") for _ in range(n)]
+    lam1 = tx.squeeze("route_lambda")
+    lam2 = tx.squeeze("route_lambda")
+    out = bytearray()
+
+    def send(label, vals):
+        b = fe_bytes(vals)
+        out.extend(b)
+        tx.absorb(label, b)
+
+    send("route_open", [mle_at(D, z), mle_at(l, z)])
+    # G(e) = sum over e' < e of eq(z_e, e'), as a table over the e bits
+    ze = z[vT:]
+    G = []
+    acc = 0
+    for e in range(E):
+        G.append(acc)
+        acc = (acc + eq_ml(ze, [(e >> (vE - 1 - b)) & 1 for b in range(vE)])) % P
+
+    def F(x):  # the summand at a point x of n coordinates
+        xt, xe = x[:vT], x[vT:]
+        Hx, lx, Gx = mle_at(H, x), mle_at(l, x), mle_at(G, xe)
+        return (eq_ml(z[:vT], xt) * Hx * (lx - Gx) + lam1 * eq_ml(w, x) * Hx * (1 - Hx)
+                + lam2 * eq_ml(w[:vT], xt) * Hx) % P
+
+    rho = []
+    for t in range(n):
+        rest = n - t - 1
+        g = []
+        for X in range(4):
+            s = 0
+            for bb in range(1 << rest):
+                s += F(rho + [X] + [(bb >> (rest - 1 - i)) & 1 for i in range(rest)])
+            g.append(s % P)
+        send("route_round", g)
+        rho.append(tx.squeeze("route_chal"))
+    send("route_final", [mle_at(H, rho), mle_at(l, rho)])
+    return bytes(out) + lhi_body(tx, (D - 128).astype(np.int32), 8)
