@@ -404,6 +404,43 @@ int fp_mm2_protocol_drive(fp_tx* tx, int vM, int vN, int n, fp_values_fn fn, voi
                           size_t* proof_len);
 
 /*
+ * MoE routing, top-1 ("How fast can FlashProve go", 2 Background, the note on MoE
+ * layers: the routing computation and each token's choice of expert are proven).
+ * Token t goes to e_t, the first index of its largest router logit. logits:
+ * device, T x E int8 token-major (the router matmul's rescaled outputs), read
+ * only; E a power of two. H (T x E u8) and D (T x E int32): device, caller-
+ * allocated, written by the call: the committed choice H[t][e] = [e = e_t] and
+ * D[t][e] = l[t][e_t] - l[t][e] - [e < e_t]. With x = t E + e (token bits first,
+ * rows zero-padded to 2^vT, n = vT + log2 E) the call continues tx:
+ *   absorb "route_site" D(logits) || D(H) || D(D as int32 little-endian);
+ *   squeeze z, w (n each, "route_z", "route_w"), lambda1, lambda2
+ *   ("route_lambda"); send D~(z), l~(z) ("route_open"); n rounds of g(0..3)
+ *   ("route_round") and challenges ("route_chal") of the sum-check of
+ *   eq(z_t, t) H (l - G(e)) + lambda1 eq(w, x) H (1 - H) + lambda2 eq(w_t, t) H,
+ *   G(e) = sum_{e' < e} eq(z_e, e'), claim D~(z) + l~(z) + lambda2 sum_{t < T}
+ *   eq(w_t, t); send H~(rho), l~(rho) ("route_final"); then the statement of
+ *   logup_prove_helper_inverse for the keys D - 128 (T E of them) on R_8.
+ * Proof bytes: 16 + 32 n + 16 + the helper-inverse proof (4 * 256 + 8 + 32 v + 16,
+ * v = max(1, ceil(log2 (T E)))). E not a power of two in [1, 4096], T < 1 or
+ * n > 26: FP_ERR_SHAPE; null arguments FP_ERR_ARG; proof / proof_len as for
+ * sumcheck_prove_matmul.
+ */
+int sumcheck_prove_routing(fp_ctx* ctx, fp_tx* tx, const int8_t* logits, int64_t T, int E, uint8_t* H, int32_t* D,
+                           uint8_t* proof, size_t* proof_len, void* stream);
+
+/*
+ * The host half of sumcheck_prove_routing up to "route_final" (n variables);
+ * tx must have absorbed "route_site". Callback kinds:
+ *   FP_VAL_START: in = z_1..z_n, w_1..w_n, lambda1, lambda2 (2 n + 2 words), t = n;
+ *   FP_VAL_CLAIM: out = D~(z), l~(z), sum_{t < T} eq(w_t, t) (3 words);
+ *   FP_VAL_ROUND: out = g_t(0..3) (4 words);
+ *   FP_VAL_ANSWER: in = rho_t (1 word);
+ *   FP_VAL_FINALS: out = H~(rho), l~(rho) (2 words).
+ * The proof holds 16 + 32 n + 16 bytes.
+ */
+int fp_route_protocol_drive(fp_tx* tx, int n, fp_values_fn fn, void* user, uint8_t* proof, size_t* proof_len);
+
+/*
  * The host half of logup_prove_helper_inverse from the multiplicities on (v >= 1
  * variables, table R_k): m (host, 2^k u32) and m_digest (host, 32 bytes: the
  * digest of m's bytes) are given; tx must have absorbed "lhi_site". Callback

@@ -15,7 +15,7 @@ from pathlib import Path
 from typing import Optional, Sequence
 
 __all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P",
-           "had2_protocol_drive", "lhi_protocol_drive", "mm2_protocol_drive"]
+           "had2_protocol_drive", "lhi_protocol_drive", "mm2_protocol_drive", "route_protocol_drive"]
 
 P = 0xFFFFFFFF00000001
 LIB_PATH = Path(__file__).resolve().with_name("libfp.so")
@@ -79,6 +79,8 @@ def lib():
     L.fp_had2_protocol_drive.argtypes = [vp, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.sumcheck_prove_matmul_ext2.argtypes = [vp, vp, C.POINTER(_Site), vp, C.POINTER(sz), vp]
     L.freivalds_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), vp, C.POINTER(sz), vp]
+    L.sumcheck_prove_routing.argtypes = [vp, vp, vp, C.c_int64, i32, vp, vp, vp, C.POINTER(sz), vp]
+    L.fp_route_protocol_drive.argtypes = [vp, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.fp_mm2_protocol_drive.argtypes = [vp, i32, i32, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.logup_prove_helper_inverse.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
     L.fp_lhi_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
@@ -179,6 +181,41 @@ def mm2_protocol_drive(tx: "Transcript", vM: int, vN: int, n: int, values) -> by
     rc = L.fp_mm2_protocol_drive(tx.h, vM, vN, n, fn, None, buf, C.byref(ln))
     if rc != 0:
         raise FpError(rc, "fp_mm2_protocol_drive failed")
+    return buf.raw[: ln.value]
+
+
+def route_protocol_drive(tx: "Transcript", n: int, values) -> bytes:
+    """Run the host half of the routing proof up to "route_final" with its device values
+    taken from `values` (no GPU work): values.start(z, w, lam1, lam2), values.claim() ->
+    (D~(z), l~(z), row-sum weight), values.round(t) -> g(0..3), values.answer(t, rho),
+    values.finals() -> (H~(rho), l~(rho)). tx must have absorbed "route_site"."""
+    L = lib()
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            if kind == VAL_START:
+                vals = [int(inp[i]) for i in range(2 * t + 2)]
+                values.start(vals[:t], vals[t:2 * t], vals[2 * t], vals[2 * t + 1])
+            elif kind == VAL_ANSWER:
+                values.answer(t, int(inp[0]))
+            elif kind in (VAL_CLAIM, VAL_ROUND, VAL_FINALS):
+                res = values.claim() if kind == VAL_CLAIM else (values.round(t) if kind == VAL_ROUND
+                                                                else values.finals())
+                for i, x in enumerate(res):
+                    out[i] = int(x)
+            else:
+                return 1
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _VALUES_FN(cb)
+    cap = 16 + 32 * n + 16
+    buf = C.create_string_buffer(cap)
+    ln = C.c_size_t(cap)
+    rc = L.fp_route_protocol_drive(tx.h, n, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_route_protocol_drive failed")
     return buf.raw[: ln.value]
 
 
@@ -425,6 +462,27 @@ class Context:
         self._check(self._L.freivalds_prove_matmul(self.h, tx.h, arr, buf, C.byref(ln), _stream(stream)),
                     "freivalds_prove_matmul")
         return buf.raw[: ln.value]
+
+    def prove_routing(self, tx: Transcript, logits, T: int, E: int, H, D, stream=None):
+        """Top-1 routing proof of the device int8 router logits (T x E, token-major): writes the
+        committed choice H (T x E uint8) and differences D (T x E int32) into the given device
+        tensors and returns (proof bytes, status); continues tx."""
+        vT = 0
+        while (1 << vT) < T:
+            vT += 1
+        vE = 0
+        while (1 << vE) < E:
+            vE += 1
+        v = 0
+        while (1 << v) < T * E:
+            v += 1
+        v = max(v, 1)
+        cap = 16 + 32 * (vT + vE) + 16 + 4 * 256 + 8 + 32 * v + 16
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        rc = self._check(self._L.sumcheck_prove_routing(self.h, tx.h, _ptr(logits), T, E, _ptr(H), _ptr(D), buf,
+                                                        C.byref(ln), _stream(stream)), "sumcheck_prove_routing")
+        return buf.raw[: ln.value], rc
 
     def prove_helper_inverse(self, tx: Transcript, r, k: int, stream=None):
         """Helper-inverse LogUp proof that every entry of the device int32 tensor r lies in

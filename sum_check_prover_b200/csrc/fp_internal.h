@@ -51,6 +51,11 @@ enum FpKernel {
     K_MM2_ROUND,
     K_MM2_FINAL,
     K_FRV_U,
+    K_ROUTE_WITNESS,
+    K_ROUTE_VECTORS,
+    K_ROUTE_OPEN,
+    K_ROUTE_ROUND,
+    K_ROUTE_FINAL,
     K_COUNT
 };
 
@@ -202,6 +207,15 @@ static inline size_t fp_align_up(size_t x, size_t a) { return (x + a - 1) / a * 
 
 // little-endian u64 words into a proof buffer (sumcheck.cu)
 void put_u64s(uint8_t* p, const uint64_t* v, size_t n);
+
+// The helper-inverse LogUp of an int32 key column on R_k (lhi.cu): its proof length, the
+// device (and host) scratch of fp_lhi_run, and the run itself from "lhi_site" on, which
+// allocates from c->dev and c->host as the caller reserved them (no reset). Returns FP_OK,
+// 1 when some key lies outside the table, or an error.
+size_t fp_lhi_proof_len(int64_t n, int k);
+size_t fp_lhi_scratch(fp_ctx* c, int64_t n, int k, size_t* host_bytes);
+int fp_lhi_run(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n, int k, uint8_t* proof, size_t* proof_len,
+               cudaStream_t st);
 
 // the degree-3 polynomial through (i, g[i]), i = 0..3, at r (api.cu)
 uint64_t fp_lagrange4(const uint64_t g[4], uint64_t r);

@@ -410,20 +410,21 @@ size_t lhi_proof_len(int v, int k) { return 4 * ((size_t)1 << k) + 8 + 32 * (siz
 
 }  // namespace
 
-int logup_prove_helper_inverse(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n, int k, uint8_t* proof,
-                               size_t* proof_len, void* stream) {
-    if (!c || !tx || !proof_len || !r) return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse: null argument");
-    if (k < 1 || k > LH_MAX_K) return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse: need 1 <= k <= 24");
-    if (n < 1 || n > (1ll << LH_MAX_V))
-        return fp_fail(c, FP_ERR_SHAPE, "logup_prove_helper_inverse: need 1 <= n <= 2^30");
+size_t fp_lhi_proof_len(int64_t n, int k) { return lhi_proof_len(std::max(1, fp_log2_ceil((uint64_t)n)), k); }
+
+size_t fp_lhi_scratch(fp_ctx* c, int64_t n, int k, size_t* host_bytes) {
     const int v = std::max(1, fp_log2_ceil((uint64_t)n));
-    const size_t need_len = lhi_proof_len(v, k);
-    if (!proof || *proof_len < need_len) {
-        *proof_len = need_len;
-        return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse: proof buffer too small");
-    }
-    FP_CUDA(c, cudaSetDevice(c->device));
-    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t L = 1ll << v, T = 1ll << k, half = L / 2;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, lhi_session_kernel, LH_THREADS, 0) != cudaSuccess) occ = 2;
+    const size_t part_n = (size_t)5 * std::max(1, occ) * c->num_sms;
+    if (host_bytes) *host_bytes = fp_align_up((size_t)4 * T, 256) + fp_align_up(8 * 64, 256);
+    return fp_align_up((size_t)8 * L, 256) + 3 * fp_align_up((size_t)8 * half, 256) + fp_align_up((size_t)8 * T, 256) +
+           fp_align_up((size_t)4 * T, 256) + fp_align_up(8 * part_n, 256) + 2 * fp_align_up(8 * 64, 256);
+}
+
+int fp_lhi_run(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n, int k, uint8_t* proof, size_t* proof_len,
+               cudaStream_t st) {
     int rc;
     {
         FpDigestJob job = {(const uint8_t*)r, 4 * (uint64_t)n};
@@ -431,6 +432,7 @@ int logup_prove_helper_inverse(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n
         if ((rc = fp_digest_many(c, &job, 1, d, st))) return rc;  // synchronises the stream
         fp_tx_absorb_raw(tx, "lhi_site", d, 32);
     }
+    const int v = std::max(1, fp_log2_ceil((uint64_t)n));
     const int64_t L = 1ll << v, T = 1ll << k, half = L / 2;
     LhiDevice dev;
     dev.c = c;
@@ -443,13 +445,6 @@ int logup_prove_helper_inverse(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n
     FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, lhi_session_kernel, LH_THREADS, 0));
     dev.cap_grid = std::max(1, occ) * c->num_sms;
     const size_t part_n = (size_t)5 * dev.cap_grid;
-    const size_t need = fp_align_up((size_t)8 * L, 256) + 3 * fp_align_up((size_t)8 * half, 256) +
-                        fp_align_up((size_t)8 * T, 256) + fp_align_up((size_t)4 * T, 256) +
-                        fp_align_up(8 * part_n, 256) + 2 * fp_align_up(8 * 64, 256) + 4096;
-    if ((rc = fp_reserve(c, c->dev, need))) return rc;
-    if ((rc = fp_reserve(c, c->host, fp_align_up((size_t)4 * T, 256) + 4096))) return rc;
-    fp_reset(c->dev);
-    fp_reset(c->host);
     dev.hcol = (uint64_t*)fp_alloc(c->dev, (size_t)8 * L);
     uint64_t* Hv = (uint64_t*)fp_alloc(c->dev, (size_t)8 * half);
     uint64_t* Fv = (uint64_t*)fp_alloc(c->dev, (size_t)8 * half);
@@ -462,7 +457,7 @@ int logup_prove_helper_inverse(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n
     uint32_t* hm = (uint32_t*)fp_alloc(c->host, (size_t)4 * T);
     dev.hs = (uint64_t*)fp_alloc(c->host, 8 * 64);
     if (!dev.hcol || !Hv || !Fv || !E || !dev.inv || !m || !dev.part || !dev.small || !outside || !hm || !dev.hs)
-        return fp_fail(c, FP_ERR_OOM, "logup_prove_helper_inverse: scratch exhausted");
+        return fp_fail(c, FP_ERR_OOM, "helper-inverse LogUp: scratch exhausted");
     memset(&dev.A, 0, sizeof dev.A);
     dev.A.r = r;
     dev.A.n = n;
@@ -496,6 +491,29 @@ int logup_prove_helper_inverse(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n
     memcpy(&n_outside, dev.hs, 4);
     if ((rc = lhi_protocol(c, tx, v, k, hm, md, dev, proof, proof_len))) return rc;
     return n_outside ? 1 : FP_OK;
+}
+
+int logup_prove_helper_inverse(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n, int k, uint8_t* proof,
+                               size_t* proof_len, void* stream) {
+    if (!c || !tx || !proof_len || !r) return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse: null argument");
+    if (k < 1 || k > LH_MAX_K) return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse: need 1 <= k <= 24");
+    if (n < 1 || n > (1ll << LH_MAX_V))
+        return fp_fail(c, FP_ERR_SHAPE, "logup_prove_helper_inverse: need 1 <= n <= 2^30");
+    const size_t need_len = fp_lhi_proof_len(n, k);
+    if (!proof || *proof_len < need_len) {
+        *proof_len = need_len;
+        return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse: proof buffer too small");
+    }
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t st = (cudaStream_t)stream;
+    int rc;
+    size_t hb = 0;
+    const size_t need = fp_lhi_scratch(c, n, k, &hb) + 4096;
+    if ((rc = fp_reserve(c, c->dev, need))) return rc;
+    if ((rc = fp_reserve(c, c->host, hb + 4096))) return rc;
+    fp_reset(c->dev);
+    fp_reset(c->host);
+    return fp_lhi_run(c, tx, r, n, k, proof, proof_len, st);
 }
 
 int fp_lhi_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uint8_t* m_digest, fp_values_fn fn,

@@ -160,3 +160,79 @@ def test_callback_errors_and_sizes(fp):
     assert ln.value == 4 * 8 + 8 + 32 * 2 + 16
     assert L.fp_lhi_protocol_drive(fp.Transcript(0).h, 0, 3, m, md, cb, None, buf, C.byref(ln)) != 0
     assert L.fp_lhi_protocol_drive(fp.Transcript(0).h, 2, 25, m, md, cb, None, buf, C.byref(ln)) != 0
+
+
+# ---- the routing proof's sum-check (its range check is the statement above) ------------
+
+class BruteRoute:
+    """Device values of the routing sum-check by their definitions (MLEs by hypercube sums)."""
+
+    def __init__(self, l, T, E, tamper=None):
+        self.T, self.E = T, E
+        self.vT, self.vE = bf.log2c(T), bf.log2c(E)
+        self.n = self.vT + self.vE
+        self.l = np.asarray(l, np.int64).reshape(-1)
+        H, D = bf.route_witness(l, T, E)
+        self.H = H.astype(np.int64).reshape(-1)
+        self.D = D.astype(np.int64).reshape(-1)
+        self.rho = []
+        self.tamper = tamper
+
+    def start(self, z, w, lam1, lam2):
+        self.z, self.w, self.lam1, self.lam2 = z, w, lam1, lam2
+        ze = z[self.vT:]
+        self.G, acc = [], 0
+        for e in range(self.E):
+            self.G.append(acc)
+            acc = (acc + bf.eq_ml(ze, [(e >> (self.vE - 1 - b)) & 1 for b in range(self.vE)])) % P
+
+    def claim(self):
+        rowsum = sum(bf.eq_ml(self.w[:self.vT], [(t >> (self.vT - 1 - b)) & 1 for b in range(self.vT)])
+                     for t in range(self.T)) % P
+        return [bf.mle_at(self.D, self.z), bf.mle_at(self.l, self.z), rowsum]
+
+    def _F(self, x):
+        xt, xe = x[:self.vT], x[self.vT:]
+        Hx, lx, Gx = bf.mle_at(self.H, x), bf.mle_at(self.l, x), bf.mle_at(self.G, xe)
+        return (bf.eq_ml(self.z[:self.vT], xt) * Hx * (lx - Gx) + self.lam1 * bf.eq_ml(self.w, x) * Hx * (1 - Hx)
+                + self.lam2 * bf.eq_ml(self.w[:self.vT], xt) * Hx) % P
+
+    def round(self, t):
+        rest = self.n - t
+        g = [sum(self._F(self.rho + [X] + [(b >> (rest - 1 - i)) & 1 for i in range(rest)])
+                 for b in range(1 << rest)) % P for X in range(4)]
+        if self.tamper == t:
+            g[0] = (g[0] + 1) % P
+        return g
+
+    def answer(self, t, rho):
+        assert t == len(self.rho) + 1
+        self.rho.append(rho)
+
+    def finals(self):
+        return [bf.mle_at(self.H, self.rho), bf.mle_at(self.l, self.rho)]
+
+
+def _route_drive(fp, seed, l, T, E, vals):
+    H, D = bf.route_witness(l, T, E)
+    tx = fp.Transcript(seed)
+    tx.absorb("route_site", bf.tree_digest(np.asarray(l, np.int8).tobytes()) + bf.tree_digest(H.tobytes())
+              + bf.tree_digest(np.asarray(D, "<i4").tobytes()))
+    return fp.route_protocol_drive(tx, vals.n, vals)
+
+
+@pytest.mark.parametrize("T,E,seed", [(1, 1, 0), (1, 2, 1), (3, 4, 2), (2, 8, 3), (5, 2, 4)])
+def test_route_host_half_matches_oracle(fp, T, E, seed):
+    l = np.random.default_rng(seed).integers(-4, 4, (T, E)).astype(np.int8)
+    vals = BruteRoute(l, T, E)
+    pf = _route_drive(fp, seed, l, T, E, vals)
+    H, D = oracle.route_witness(l, T, E)
+    want, _ = oracle.route_prove(seed, l, H, D, T, E)
+    assert len(pf) == 16 + 32 * vals.n + 16
+    assert pf == want[:len(pf)]  # the rest of the oracle's proof is the range LogUp
+
+
+def test_route_inconsistent_round_is_refused(fp):
+    l = np.random.default_rng(9).integers(-4, 4, (3, 4)).astype(np.int8)
+    with pytest.raises(fp.FpError):
+        _route_drive(fp, 1, l, 3, 4, BruteRoute(l, 3, 4, tamper=2))
