@@ -65,6 +65,10 @@ REASONS = {
     34: "route_open",
     35: "route_round",
     36: "route_final",
+    37: "lhi2_sum",
+    38: "lhi2_round",
+    39: "lhi2_final",
+    40: "lhi2_open",
 }
 
 
@@ -162,6 +166,11 @@ def lib():
         L.orc_frv_prove.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, C.POINTER(u64)]
         L.orc_frv_verify.restype = C.c_int
         L.orc_frv_verify.argtypes = [vp, C.POINTER(_Site), C.POINTER(_Wit), vp, u64, vp]
+        for nm in ("orc_lhi2_prove",):
+            getattr(L, nm).restype = C.c_int
+            getattr(L, nm).argtypes = [vp, vp, u64, C.c_int, vp, u64, C.POINTER(u64)]
+        L.orc_lhi2_verify.restype = C.c_int
+        L.orc_lhi2_verify.argtypes = [vp, vp, u64, C.c_int, vp, u64, vp]
         L.orc_route_witness.restype = None
         L.orc_route_witness.argtypes = [vp, u64, C.c_int, vp, vp]
         L.orc_route_prove.restype = C.c_int
@@ -571,6 +580,15 @@ def exp_verify(seed: int, g, s, proof: bytes):
 
 def lhi_prove(seed: int, r, k: int):
     """Helper-inverse LogUp proof that every key r_i lies in the remainder table R_k."""
+    return _lhi_prove(lib().orc_lhi_prove, seed, r, k)
+
+
+def lhi2_prove(seed: int, r, k: int):
+    """The same statement with every challenge and value in the quadratic extension."""
+    return _lhi_prove(lib().orc_lhi2_prove, seed, r, k)
+
+
+def _lhi_prove(fn, seed: int, r, k: int):
     L = lib()
     a = np.ascontiguousarray(np.asarray(r, dtype=np.int32).reshape(-1))
     out = []
@@ -578,26 +596,34 @@ def lhi_prove(seed: int, r, k: int):
         tx = L.orc_tx_new(seed)
         n = C.c_uint64(0)
         buf = np.zeros(max(1, out[0] if out else 1), dtype=np.uint8)
-        rc = L.orc_lhi_prove(tx, _ptr(a), a.size, k, _ptr(buf) if out else None, out[0] if out else 0, C.byref(n))
+        rc = fn(tx, _ptr(a), a.size, k, _ptr(buf) if out else None, out[0] if out else 0, C.byref(n))
         st = C.create_string_buffer(32)
         L.orc_tx_state(tx, st)
         L.orc_tx_free(tx)
         if out:
             if rc != 0:
-                raise ValueError(f"orc_lhi_prove failed ({rc})")
+                raise ValueError(f"helper-inverse prover failed ({rc})")
             return buf[: n.value].tobytes(), st.raw
         if rc not in (0, -2):
-            raise ValueError(f"orc_lhi_prove rejected the statement ({rc})")
+            raise ValueError(f"helper-inverse prover rejected the statement ({rc})")
         out.append(n.value)
 
 
 def lhi_verify(seed: int, r, k: int, proof: bytes):
+    return _lhi_verify(lib().orc_lhi_verify, seed, r, k, proof)
+
+
+def lhi2_verify(seed: int, r, k: int, proof: bytes):
+    return _lhi_verify(lib().orc_lhi2_verify, seed, r, k, proof)
+
+
+def _lhi_verify(fn, seed: int, r, k: int, proof: bytes):
     L = lib()
     a = np.ascontiguousarray(np.asarray(r, dtype=np.int32).reshape(-1))
     pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
     det = np.zeros(2, dtype=np.int64)
     tx = L.orc_tx_new(seed)
-    rc = L.orc_lhi_verify(tx, _ptr(a), a.size, k, _ptr(pb), len(proof), _ptr(det))
+    rc = fn(tx, _ptr(a), a.size, k, _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
 

@@ -2666,3 +2666,202 @@ done:
     route_end(&c);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* The helper-inverse LogUp over the extension (next row f4: challenges in   */
+/* F_p[phi] / (phi^2 - 7), "How fast can FlashProve go", 4, the note on      */
+/* soundness). The statement of orc_lhi_prove with alpha, z, beta, every     */
+/* challenge and every value sent in the extension (16 bytes each); the      */
+/* helper column holds extension elements:                                  */
+/*   absorb "lhi2_site" D(r); send m (2^k u32, digest absorbed, "lhi2_m");   */
+/*   squeeze alpha ("lhi2_alpha"); commit h_i = 1 / (alpha - r_i): absorb    */
+/*   "lhi2_h" D(h as (a, b) u64 little-endian pairs); squeeze z_1..z_v       */
+/*   ("lhi2_z") and beta ("lhi2_beta"); send S = sum_i h_i ("lhi2_sum");     */
+/*   sum-check of h + beta eq(z, x) (h (alpha - f) - 1) over v variables,     */
+/*   claim S: rounds g(0..3) ("lhi2_round"), "lhi2_chal"; send h(rho),       */
+/*   f(rho) ("lhi2_final").                                                  */
+/* The verifier checks as for orc_lhi_verify, in the extension.              */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_LHI2_SUM = 37,    /* S != the table side */
+    REJ_LHI2_ROUND = 38,  /* g(0) + g(1) != running claim */
+    REJ_LHI2_FINAL = 39,  /* the end does not match F at rho */
+    REJ_LHI2_OPEN = 40    /* h(rho) or f(rho) != the columns' MLEs */
+};
+
+/* 1 / (a + b phi) = (a - b phi) / (a^2 - 7 b^2); 0 for 0 */
+static ext2 e2_inv(ext2 x) {
+    u64 nrm = orc_fsub(orc_fmul(x.a, x.a), orc_fmul(7, orc_fmul(x.b, x.b)));
+    u64 ni = orc_finv(nrm);
+    return e2(orc_fmul(x.a, ni), orc_fsub(0, orc_fmul(x.b, ni)));
+}
+
+/* eq(z, rho) = prod_i (z_i rho_i + (1 - z_i)(1 - rho_i)) in the extension */
+static ext2 e2_eq_closed(const ext2* z, const ext2* rho, int v) {
+    ext2 e = e2(1, 0), one = e2(1, 0);
+    for (int i = 0; i < v; i++)
+        e = e2_mul(e, e2_add(e2_mul(z[i], rho[i]), e2_mul(e2_sub(one, z[i]), e2_sub(one, rho[i]))));
+    return e;
+}
+
+static void lhi2_columns(const int32_t* r, u64 n, int v, ext2 alpha, ext2* f, ext2* h) {
+    u64 L = (u64)1 << v;
+    for (u64 i = 0; i < L; i++) {
+        f[i] = e2(i < n ? orc_fint(r[i]) : 0, 0);
+        h[i] = e2_inv(e2_sub(alpha, f[i]));
+    }
+}
+
+static void lhi2_absorb_h(orc_tx* t, const ext2* h, u64 L) {
+    uint8_t* b = (uint8_t*)malloc(16 * L);
+    uint8_t d[32];
+    for (u64 i = 0; i < L; i++) {
+        put_le(b + 16 * i, h[i].a, 8);
+        put_le(b + 16 * i + 8, h[i].b, 8);
+    }
+    orc_tree_digest(b, 16 * L, d);
+    free(b);
+    orc_tx_absorb(t, "lhi2_h", d, 32);
+}
+
+static void lhi2_absorb_site(orc_tx* t, const int32_t* r, u64 n) {
+    uint8_t* b = (uint8_t*)calloc(4 * n, 1);
+    uint8_t d[32];
+    for (u64 i = 0; i < n; i++) put_le(b + 4 * i, (u64)(u32)r[i], 4);
+    orc_tree_digest(b, 4 * n, d);
+    free(b);
+    orc_tx_absorb(t, "lhi2_site", d, 32);
+}
+
+/* F at one point of the three lines: h + beta e (h (alpha - f) - 1) */
+static ext2 lhi2_F(ext2 h, ext2 f, ext2 e, ext2 alpha, ext2 beta) {
+    return e2_add(h, e2_mul(beta, e2_mul(e, e2_sub(e2_mul(h, e2_sub(alpha, f)), e2(1, 0)))));
+}
+
+int orc_lhi2_prove(void* txh, const int32_t* r, u64 n, int k, uint8_t* proof, u64 cap, u64* len) {
+    if (n < 1 || k < 1 || k > 24) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n);
+    if (v < 1) v = 1;
+    u64 L = (u64)1 << v, T = (u64)1 << k;
+    pbuf pb = {proof, cap, 0, 0};
+    lhi2_absorb_site(t, r, n);
+    u32* m = (u32*)malloc(T * sizeof(u32));
+    lhi_mult(r, n, L, k, m);
+    send_mult(t, &pb, "lhi2_m", m, T);
+    ext2 alpha = e2_squeeze(t, "lhi2_alpha");
+    ext2* f = (ext2*)malloc(L * sizeof(ext2));
+    ext2* h = (ext2*)malloc(L * sizeof(ext2));
+    ext2* E = (ext2*)malloc(L * sizeof(ext2));
+    ext2* z = (ext2*)malloc(sizeof(ext2) * v);
+    lhi2_columns(r, n, v, alpha, f, h);
+    lhi2_absorb_h(t, h, L);
+    for (int i = 0; i < v; i++) z[i] = e2_squeeze(t, "lhi2_z");
+    ext2 beta = e2_squeeze(t, "lhi2_beta");
+    ext2 S = e2(0, 0);
+    for (u64 i = 0; i < L; i++) S = e2_add(S, h[i]);
+    e2_send(t, &pb, "lhi2_sum", &S, 1);
+    e2_eq_table(z, v, E);
+    u64 Lr = L;
+    for (int rd = 0; rd < v; rd++) {
+        u64 hh = Lr >> 1;
+        ext2 g[4] = {e2(0, 0), e2(0, 0), e2(0, 0), e2(0, 0)};
+        for (u64 b = 0; b < hh; b++)
+            for (u64 X = 0; X < 4; X++) {
+                ext2 hx = e2_add(h[b], e2_scal(e2_sub(h[hh + b], h[b]), X));
+                ext2 fx = e2_add(f[b], e2_scal(e2_sub(f[hh + b], f[b]), X));
+                ext2 ex = e2_add(E[b], e2_scal(e2_sub(E[hh + b], E[b]), X));
+                g[X] = e2_add(g[X], lhi2_F(hx, fx, ex, alpha, beta));
+            }
+        e2_send(t, &pb, "lhi2_round", g, 4);
+        ext2 rho = e2_squeeze(t, "lhi2_chal");
+        for (u64 b = 0; b < hh; b++) {
+            h[b] = e2_add(h[b], e2_mul(rho, e2_sub(h[hh + b], h[b])));
+            f[b] = e2_add(f[b], e2_mul(rho, e2_sub(f[hh + b], f[b])));
+            E[b] = e2_add(E[b], e2_mul(rho, e2_sub(E[hh + b], E[b])));
+        }
+        Lr = hh;
+    }
+    ext2 fin[2] = {h[0], f[0]};
+    e2_send(t, &pb, "lhi2_final", fin, 2);
+    free(m);
+    free(f);
+    free(h);
+    free(E);
+    free(z);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+int orc_lhi2_verify(void* txh, const int32_t* r, u64 n, int k, const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (n < 1 || k < 1 || k > 24) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n), rc = 0;
+    if (v < 1) v = 1;
+    u64 L = (u64)1 << v, T = (u64)1 << k;
+    prd rd = {proof, len, 0, 0};
+    u32* m = (u32*)malloc(T * sizeof(u32));
+    ext2* f = (ext2*)malloc(L * sizeof(ext2));
+    ext2* h = (ext2*)malloc(L * sizeof(ext2));
+    ext2* E = (ext2*)malloc(L * sizeof(ext2));
+    ext2* z = (ext2*)malloc(sizeof(ext2) * v);
+    ext2* rho = (ext2*)malloc(sizeof(ext2) * v);
+    lhi2_absorb_site(t, r, n);
+    rd_mult(t, &rd, "lhi2_m", m, T);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    ext2 alpha = e2_squeeze(t, "lhi2_alpha");
+    lhi2_columns(r, n, v, alpha, f, h); /* the verifier holds the key column, so h too */
+    lhi2_absorb_h(t, h, L);
+    for (int i = 0; i < v; i++) z[i] = e2_squeeze(t, "lhi2_z");
+    ext2 beta = e2_squeeze(t, "lhi2_beta");
+    ext2 S;
+    e2_read(t, &rd, "lhi2_sum", &S, 1);
+    if (rd.bad) FAIL(REJ_FORMAT, 1, 0);
+    {
+        /* the table side: sum_j m_j / (alpha - t_j) as one fraction P / Q */
+        ext2 P = e2(0, 0), Q = e2(1, 0);
+        for (u64 j = 0; j < T; j++) {
+            ext2 dj = e2_sub(alpha, e2(orc_fint((int64_t)j - ((int64_t)1 << (k - 1))), 0));
+            P = e2_add(e2_mul(P, dj), e2_scal(Q, (u64)m[j]));
+            Q = e2_mul(Q, dj);
+        }
+        ext2 lhs = e2_mul(S, Q);
+        if (lhs.a != P.a || lhs.b != P.b) FAIL(REJ_LHI2_SUM, 0, 0);
+    }
+    {
+        ext2 claim = S;
+        for (int i = 0; i < v; i++) {
+            ext2 g[4];
+            e2_read(t, &rd, "lhi2_round", g, 4);
+            if (rd.bad) FAIL(REJ_FORMAT, 2, i);
+            ext2 s01 = e2_add(g[0], g[1]);
+            if (s01.a != claim.a || s01.b != claim.b) FAIL(REJ_LHI2_ROUND, i, 0);
+            rho[i] = e2_squeeze(t, "lhi2_chal");
+            claim = e2_lagrange4(g, rho[i]);
+        }
+        ext2 fin[2];
+        e2_read(t, &rd, "lhi2_final", fin, 2);
+        if (rd.bad) FAIL(REJ_FORMAT, 3, 0);
+        ext2 want = lhi2_F(fin[0], fin[1], e2_eq_closed(z, rho, v), alpha, beta);
+        if (want.a != claim.a || want.b != claim.b) FAIL(REJ_LHI2_FINAL, 0, 0);
+        e2_eq_table(rho, v, E);
+        ext2 hr = e2(0, 0), fr = e2(0, 0);
+        for (u64 x = 0; x < L; x++) {
+            hr = e2_add(hr, e2_mul(E[x], h[x]));
+            fr = e2_add(fr, e2_mul(E[x], f[x]));
+        }
+        if (hr.a != fin[0].a || hr.b != fin[0].b) FAIL(REJ_LHI2_OPEN, 0, 0);
+        if (fr.a != fin[1].a || fr.b != fin[1].b) FAIL(REJ_LHI2_OPEN, 1, 0);
+    }
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(m);
+    free(f);
+    free(h);
+    free(E);
+    free(z);
+    free(rho);
+    return rc;
+}

@@ -773,3 +773,76 @@ def route_prove(seed: int, l, H, D, T: int, E: int) -> bytes:
         rho.append(tx.squeeze("route_chal"))
     send("route_final", [mle_at(H, rho), mle_at(l, rho)])
     return bytes(out) + lhi_body(tx, (D - 128).astype(np.int32), 8)
+
+
+def x_inv(x):
+    """1 / (a + b phi) = (a - b phi) / (a^2 - 7 b^2), by Python modular inversion."""
+    a, b = x
+    nrm = (a * a - 7 * b * b) % P
+    ni = pow(nrm, P - 2, P)
+    return (a * ni % P, (-b) * ni % P)
+
+
+def lhi2_prove(seed: int, r, k: int) -> bytes:
+    """The helper-inverse LogUp over the extension from definitions: h by extension inverses,
+    every round value a hypercube sum of h + beta eq (h (alpha - f) - 1) over MLEs at
+    extension points (no folding)."""
+    r = [int(x) for x in np.asarray(r).reshape(-1)]
+    n = len(r)
+    v = max(1, log2c(n))
+    L = 1 << v
+    f = [x % P for x in r] + [0] * (L - n)
+    out = bytearray()
+    tx = Tx(seed)
+
+    def send(label, xs):
+        b = fe_bytes([c for x in xs for c in x])
+        out.extend(b)
+        tx.absorb(label, b)
+
+    def sq(label):
+        a = tx.squeeze(label)
+        return (a, tx.squeeze(label))
+
+    tx.absorb("lhi2_site", tree_digest(np.asarray(r, "<i4").tobytes()))
+    m = np.zeros(1 << k, np.int64)
+    for x in r + [0] * (L - n):
+        j = x + (1 << (k - 1))
+        if 0 <= j < (1 << k):
+            m[j] += 1
+    b = m.astype("<u4").tobytes()
+    out.extend(b)
+    tx.absorb("lhi2_m", tree_digest(b))
+    alpha = sq("lhi2_alpha")
+    h = [x_inv(((alpha[0] - x) % P, alpha[1])) for x in f]
+    tx.absorb("lhi2_h", tree_digest(b"".join(struct.pack("<QQ", a, c) for a, c in h)))
+    z = [sq("lhi2_z") for _ in range(v)]
+    beta = sq("lhi2_beta")
+    S = (0, 0)
+    for x in h:
+        S = x_add(S, x)
+    send("lhi2_sum", [S])
+    one = (1, 0)
+    rho = []
+    for t in range(v):
+        rest = v - t - 1
+        g = []
+        for X in range(4):
+            acc = (0, 0)
+            for bb in range(1 << rest):
+                w = rho + [(X, 0)] + [((bb >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                hw = (0, 0)
+                for x in range(L):
+                    e = x_eq(w, [((x >> (v - 1 - i)) & 1, 0) for i in range(v)])
+                    hw = x_add(hw, x_mul(e, h[x]))
+                fw = x_mle(f, w)
+                inner = x_add(x_mul(hw, x_add(alpha, ((-fw[0]) % P, (-fw[1]) % P))), ((-1) % P, 0))
+                acc = x_add(acc, x_add(hw, x_mul(beta, x_mul(x_eq(z, w), inner))))
+            g.append(acc)
+        send("lhi2_round", g)
+        rho.append(sq("lhi2_chal"))
+    hr = (0, 0)
+    for x in range(L):
+        hr = x_add(hr, x_mul(x_eq(rho, [((x >> (v - 1 - i)) & 1, 0) for i in range(v)]), h[x]))
+    send("lhi2_final", [hr, x_mle(f, rho)])
+    return bytes(out)

@@ -112,3 +112,47 @@ def test_mm2_honest_accepted_and_tampering_named(M, K, N, bits, scales):
     q, r, y = (t.copy() for t in w)
     r[1, 2] += 1
     assert oracle.mm2_verify(7, s, (q, r, y), pf)[0] != "accept"
+
+
+# ---- the helper-inverse LogUp over the extension ----------------------------------------
+
+def _keys(n, k, seed):
+    return np.random.default_rng(seed).integers(-(1 << (k - 1)), 1 << (k - 1), n).astype(np.int32)
+
+
+def test_extension_inverse():
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        x = (int(rng.integers(0, P, dtype=np.uint64)), int(rng.integers(0, P, dtype=np.uint64)))
+        assert bf.x_mul(x, bf.x_inv(x)) == (1, 0)
+
+
+@pytest.mark.parametrize("n,k", [(1, 1), (3, 4), (5, 7), (8, 3), (13, 5)])
+def test_lhi2_bytes_match_bruteforce(n, k):
+    r = _keys(n, k, n * 10 + k)
+    pf, _ = oracle.lhi2_prove(2, r, k)
+    assert pf == bf.lhi2_prove(2, r, k)
+
+
+def test_lhi2_accepts_and_names_tampering():
+    k = 7
+    r = _keys(1000, k, 4)
+    pf, _ = oracle.lhi2_prove(6, r, k)
+    assert oracle.lhi2_verify(6, r, k, pf) == ("accept", (0, 0))
+    T = 1 << k
+    off = 4 * T  # S
+    x = struct.unpack("<Q", pf[off:off + 8])[0]
+    assert oracle.lhi2_verify(6, r, k, pf[:off] + struct.pack("<Q", (x + 1) % P) + pf[off + 8:])[0] == "lhi2_sum"
+    off = 4 * T + 16  # round 1, g(0)'s first coordinate
+    x = struct.unpack("<Q", pf[off:off + 8])[0]
+    assert oracle.lhi2_verify(6, r, k, pf[:off] + struct.pack("<Q", (x + 1) % P) + pf[off + 8:]) == ("lhi2_round", (0, 0))
+    off = len(pf) - 32  # h(rho)
+    x = struct.unpack("<Q", pf[off:off + 8])[0]
+    assert oracle.lhi2_verify(6, r, k, pf[:off] + struct.pack("<Q", (x + 1) % P) + pf[off + 8:])[0] == "lhi2_final"
+    r2 = r.copy()
+    r2[17] = 1 << 20  # outside R_7
+    pf2, _ = oracle.lhi2_prove(6, r2, k)
+    assert oracle.lhi2_verify(6, r2, k, pf2)[0] == "lhi2_sum"
+    # the base-field proof of the same keys is another proof
+    base, _ = oracle.lhi_prove(6, r, k)
+    assert oracle.lhi2_verify(6, r, k, base)[0] != "accept"
