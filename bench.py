@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2,frv"
+MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2"
 
 
 def micro_names(which) -> set:
@@ -210,6 +210,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
       weight (the matrix once; the eq weights are 16-byte extension elements).
     frv_u: Freivalds' prover, u = X rho^(.) over a 16384-token x 16384 int8 activation
       (the activation once, plus the powers of rho).
+    lhi2_round: the helper-inverse LogUp's rounds over 2^26 keys with extension challenges
+      (16-byte vectors: 176 B per pair in round 2, 240 B later).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
@@ -373,6 +375,16 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
             del st, keep, d
         except Exception as e:  # a failure here must not cost the rest of the line
             out["freivalds_u_16384x16384"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    if "lhi2" in which:
+        # the helper-inverse LogUp of 2^26 remainders in R_12 with extension-field challenges
+        try:
+            rng = __import__("numpy").random.default_rng(12)
+            rv = torch.from_numpy(rng.integers(-2048, 2048, 1 << 26).astype("int32")).to(dev)
+            measure("helper_inverse_ext2_round_2^26_keys", "lhi2_round",
+                    lambda: ctx.prove_helper_inverse_ext2(fp.Transcript(7), rv, 12))
+            del rv
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["helper_inverse_ext2_round_2^26_keys"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     try:
         torch.cuda.empty_cache()

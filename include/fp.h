@@ -441,6 +441,33 @@ int sumcheck_prove_routing(fp_ctx* ctx, fp_tx* tx, const int8_t* logits, int64_t
 int fp_route_protocol_drive(fp_tx* tx, int n, fp_values_fn fn, void* user, uint8_t* proof, size_t* proof_len);
 
 /*
+ * The helper-inverse LogUp over the quadratic extension F_p[phi]/(phi^2 - 7)
+ * ("How fast can FlashProve go", 4, the note on soundness: challenges from an
+ * extension field): the statement of logup_prove_helper_inverse with alpha, z,
+ * beta, every challenge and every value sent an extension element (16 bytes: a
+ * then b), the helper column the extension inverses 1 / (alpha - r_i) committed
+ * as 16-byte pairs, and the labels "lhi2_site", "lhi2_m", "lhi2_alpha",
+ * "lhi2_h", "lhi2_z", "lhi2_beta", "lhi2_sum", "lhi2_round", "lhi2_chal",
+ * "lhi2_final". Proof bytes: 4 2^k + 16 + 64 v + 32. Same arguments, status and
+ * errors as logup_prove_helper_inverse.
+ */
+int logup_prove_helper_inverse_ext2(fp_ctx* ctx, fp_tx* tx, const int32_t* r, int64_t n, int k, uint8_t* proof,
+                                    size_t* proof_len, void* stream);
+
+/*
+ * The host half of logup_prove_helper_inverse_ext2 from the multiplicities on
+ * (as fp_lhi_protocol_drive, every value an extension element of two words):
+ *   FP_VAL_COLUMN: in = alpha (2 words); out = D(h) (4 words);
+ *   FP_VAL_START: in = z_1..z_v, beta (2 v + 2 words), t = v;
+ *   FP_VAL_ROUND: out = H_t(0), H_t(1), Q_t(0), Q_t(1), Q_t(2) (10 words);
+ *   FP_VAL_ANSWER: in = rho_t (2 words);
+ *   FP_VAL_FINALS: out = h~(rho), f~(rho) (4 words).
+ * The proof holds 4 2^k + 16 + 64 v + 32 bytes.
+ */
+int fp_lhi2_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uint8_t* m_digest, fp_values_fn fn,
+                           void* user, uint8_t* proof, size_t* proof_len);
+
+/*
  * The host half of logup_prove_helper_inverse from the multiplicities on (v >= 1
  * variables, table R_k): m (host, 2^k u32) and m_digest (host, 32 bytes: the
  * digest of m's bytes) are given; tx must have absorbed "lhi_site". Callback

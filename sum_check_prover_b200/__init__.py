@@ -15,7 +15,8 @@ from pathlib import Path
 from typing import Optional, Sequence
 
 __all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P",
-           "had2_protocol_drive", "lhi_protocol_drive", "mm2_protocol_drive", "route_protocol_drive"]
+           "had2_protocol_drive", "lhi_protocol_drive", "mm2_protocol_drive", "route_protocol_drive",
+           "lhi2_protocol_drive"]
 
 P = 0xFFFFFFFF00000001
 LIB_PATH = Path(__file__).resolve().with_name("libfp.so")
@@ -81,6 +82,8 @@ def lib():
     L.freivalds_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), vp, C.POINTER(sz), vp]
     L.sumcheck_prove_routing.argtypes = [vp, vp, vp, C.c_int64, i32, vp, vp, vp, C.POINTER(sz), vp]
     L.fp_route_protocol_drive.argtypes = [vp, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
+    L.logup_prove_helper_inverse_ext2.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
+    L.fp_lhi2_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.fp_mm2_protocol_drive.argtypes = [vp, i32, i32, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.logup_prove_helper_inverse.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
     L.fp_lhi_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
@@ -216,6 +219,48 @@ def route_protocol_drive(tx: "Transcript", n: int, values) -> bytes:
     rc = L.fp_route_protocol_drive(tx.h, n, fn, None, buf, C.byref(ln))
     if rc != 0:
         raise FpError(rc, "fp_route_protocol_drive failed")
+    return buf.raw[: ln.value]
+
+
+def lhi2_protocol_drive(tx: "Transcript", v: int, k: int, m, m_digest: bytes, values) -> bytes:
+    """As lhi_protocol_drive for the statement over the quadratic extension: every challenge and
+    value an extension pair (a, b); values.column(alpha) -> 32-byte digest, values.start(z, beta),
+    values.round(t) -> (H(0), H(1), Q(0), Q(1), Q(2)), values.answer(t, rho), values.finals()."""
+    import numpy as np
+
+    L = lib()
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            if kind == VAL_COLUMN:
+                d = values.column((int(inp[0]), int(inp[1])))
+                for i in range(4):
+                    out[i] = int.from_bytes(d[8 * i: 8 * i + 8], "little")
+            elif kind == VAL_START:
+                pts = [(int(inp[2 * i]), int(inp[2 * i + 1])) for i in range(t + 1)]
+                values.start(pts[:t], pts[t])
+            elif kind == VAL_ANSWER:
+                values.answer(t, (int(inp[0]), int(inp[1])))
+            elif kind in (VAL_ROUND, VAL_FINALS):
+                res = values.round(t) if kind == VAL_ROUND else values.finals()
+                for i, (a, b) in enumerate(res):
+                    out[2 * i] = int(a)
+                    out[2 * i + 1] = int(b)
+            else:
+                return 1
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _VALUES_FN(cb)
+    mm = np.ascontiguousarray(np.asarray(m, dtype="<u4"))
+    md = C.create_string_buffer(bytes(m_digest), 32)
+    cap = 4 * (1 << k) + 16 + 64 * v + 32
+    buf = C.create_string_buffer(cap)
+    ln = C.c_size_t(cap)
+    rc = L.fp_lhi2_protocol_drive(tx.h, v, k, mm.ctypes.data, md, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_lhi2_protocol_drive failed")
     return buf.raw[: ln.value]
 
 
@@ -482,6 +527,20 @@ class Context:
         ln = C.c_size_t(cap)
         rc = self._check(self._L.sumcheck_prove_routing(self.h, tx.h, _ptr(logits), T, E, _ptr(H), _ptr(D), buf,
                                                         C.byref(ln), _stream(stream)), "sumcheck_prove_routing")
+        return buf.raw[: ln.value], rc
+
+    def prove_helper_inverse_ext2(self, tx: Transcript, r, k: int, stream=None):
+        """As prove_helper_inverse with every challenge and value in the quadratic extension."""
+        n = int(r.numel())
+        v = 0
+        while (1 << v) < n:
+            v += 1
+        v = max(v, 1)
+        cap = 4 * (1 << k) + 16 + 64 * v + 32
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        rc = self._check(self._L.logup_prove_helper_inverse_ext2(self.h, tx.h, _ptr(r), n, k, buf, C.byref(ln),
+                                                                 _stream(stream)), "logup_prove_helper_inverse_ext2")
         return buf.raw[: ln.value], rc
 
     def prove_helper_inverse(self, tx: Transcript, r, k: int, stream=None):

@@ -397,7 +397,8 @@ const char* fp_kernel_name(int k) {
         "silu_hist", "silu_tree", "silu_round", "silu_leaf", "had2_round", "had2_final",
         "lhi_hist", "lhi_column", "lhi_round", "lhi_final",
         "mm2_eq", "mm2_contract", "mm2_claim", "mm2_round", "mm2_final", "frv_u",
-        "route_witness", "route_vectors", "route_open", "route_round", "route_final"};
+        "route_witness", "route_vectors", "route_open", "route_round", "route_final",
+        "lhi2_column", "lhi2_round", "lhi2_final"};
     return (k >= 0 && k < K_COUNT) ? names[k] : "?";
 }
 

@@ -56,6 +56,9 @@ enum FpKernel {
     K_ROUTE_OPEN,
     K_ROUTE_ROUND,
     K_ROUTE_FINAL,
+    K_LHI2_COLUMN,
+    K_LHI2_ROUND,
+    K_LHI2_FINAL,
     K_COUNT
 };
 

@@ -33,6 +33,8 @@
 #include <algorithm>
 
 #include "fp_eqchunks.cuh"
+#include "fp_ext2.cuh"
+#include "fp_ext2_host.h"
 #include "fp_internal.h"
 #include "fp_reduce.cuh"
 #include "fp_session.cuh"
@@ -408,6 +410,392 @@ struct LhiCallback : LhiSource {
 
 size_t lhi_proof_len(int v, int k) { return 4 * ((size_t)1 << k) + 8 + 32 * (size_t)v + 16; }
 
+// ---- the same statement over the extension F_p[phi]/(phi^2 - 7) ---------------------
+//
+// alpha, z, beta and every challenge are extension elements, the helper column
+// holds the extension inverses 1 / (alpha - r_i) = (a - b phi) / (a^2 - 7 b^2)
+// (16 bytes each), and every value sent is an extension element; the labels
+// are "lhi2_*". The kernels are the base-field ones with 16-byte vectors: the
+// eq weights of round 1 come from four 2^8-entry chunk tables in shared memory,
+// and the device returns H(0), H(1), Q(0), Q(1), Q(2) as ten words.
+
+constexpr int LH2_CHUNK = 8;
+
+// 1 / x in the extension (0 for 0)
+__device__ __forceinline__ Ext2 e2_inv_dev(Ext2 x) {
+    const uint64_t ni = gl_inv(gl_sub(gl_mul(x.a, x.a), gl_mul7(gl_mul(x.b, x.b))));
+    return e2_make(gl_mul(x.a, ni), gl_sub(0, gl_mul(x.b, ni)));
+}
+
+__global__ void lhi2_inv_kernel(Ext2 alpha, int k, Ext2* __restrict__ inv) {
+    const int64_t T = 1ll << k, half = 1ll << (k - 1);
+    for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < T; j += (int64_t)gridDim.x * blockDim.x)
+        inv[j] = e2_inv_dev(e2_make(gl_sub(alpha.a, gl_from_i64(j - half)), alpha.b));
+}
+
+__global__ void lhi2_column_kernel(const int32_t* __restrict__ r, int64_t n, int64_t L, int k, Ext2 alpha,
+                                   const Ext2* __restrict__ inv, Ext2* __restrict__ h) {
+    const int64_t T = 1ll << k, half = 1ll << (k - 1);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < L; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t key = lh_key(r, n, i), j = key + half;
+        h[i] = (j >= 0 && j < T) ? inv[j] : e2_inv_dev(e2_make(gl_sub(alpha.a, gl_from_i64(key)), alpha.b));
+    }
+}
+
+struct Lhi2Args {
+    const int32_t* r;
+    int64_t n;
+    const Ext2* h;  // the helper column (2^v entries)
+    Ext2* Hv;       // h and f folded, from round 2 on (2^(v-1) entries each)
+    Ext2* Fv;
+    Ext2* E;        // eq(z_>t, .) (2^(v-1) entries)
+    const Ext2* z;  // device copy of z_1..z_v
+    Ext2 alpha;
+    int v;
+    int grid;
+    int per_block;
+    int pad;
+    uint64_t seq0;  // round t publishes seq0 + t, the final values seq0 + v + 1
+    int t_begin;    // rounds run by this launch: [t_begin, t_end]; t_end > v includes the final values
+    int t_end;
+};
+
+// Table j (at tab + 2^8 j): for y < 2^w[j], the product of eq(z_c, bit) over its coordinates
+// (the first on y's top bit); the four tables cover z_2..z_v. Called by every thread of the block.
+__device__ __forceinline__ void lh2_tables(Ext2* tab, const Ext2* zs, int v, int (&w)[4]) {
+    int rest = v - 1;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        w[j] = rest < LH2_CHUNK ? rest : LH2_CHUNK;
+        rest -= w[j];
+    }
+    for (int x = threadIdx.x; x < (4 << LH2_CHUNK); x += blockDim.x) {
+        const int j = x >> LH2_CHUNK, y = x & ((1 << LH2_CHUNK) - 1);
+        if (y >= (1 << w[j])) continue;
+        int first = 1;
+        for (int q = 0; q < j; q++) first += w[q];
+        Ext2 e = e2_make(1, 0);
+        for (int i = 0; i < w[j]; i++) e = e2_mul(e, e2_eq1(zs[first + i], (y >> (w[j] - 1 - i)) & 1));
+        tab[x] = e;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ Ext2 lh2_eq_at(const Ext2* tab, const int (&w)[4], int64_t b) {
+    const int s2 = w[3], s1 = w[3] + w[2], s0 = s1 + w[1];
+    Ext2 e = tab[(int)((b >> s0) & ((1 << w[0]) - 1))];
+    if (w[1]) e = e2_mul(e, tab[(1 << LH2_CHUNK) + (int)((b >> s1) & ((1 << w[1]) - 1))]);
+    if (w[2]) e = e2_mul(e, tab[(2 << LH2_CHUNK) + (int)((b >> s2) & ((1 << w[2]) - 1))]);
+    if (w[3]) e = e2_mul(e, tab[(3 << LH2_CHUNK) + (int)(b & ((1 << w[3]) - 1))]);
+    return e;
+}
+
+// ka + rho (kb - ka) for two keys (any int32)
+__device__ __forceinline__ Ext2 lh2_fold_keys(int64_t ka, int64_t kb, Ext2 rho) {
+    const uint64_t d = gl_from_i64(kb - ka);
+    return e2_make(gl_add(gl_from_i64(ka), gl_mul(rho.a, d)), gl_mul(rho.b, d));
+}
+
+__global__ void __launch_bounds__(LH_THREADS, 2) lhi2_session_kernel(Lhi2Args A, FpMailbox* mb, FpRelay* rl,
+                                                                    uint64_t* part) {
+    __shared__ Ext2 zs[32];
+    __shared__ Ext2 tab[4 << LH2_CHUNK];
+    if (threadIdx.x < A.v) zs[threadIdx.x] = A.z[threadIdx.x];
+    __syncthreads();
+    Ext2 rho = e2_make(0, 0);
+    for (int t = A.t_begin; t <= A.v && t <= A.t_end; t++) {
+        if (t > 1) {
+            uint64_t ra, rb;
+            if (!session_wait2(mb, rl, A.seq0 + t - 1, ra, rb)) return;
+            rho = e2_make(ra, rb);
+        }
+        const int64_t h = 1ll << (A.v - t);
+        const int64_t want = (h + A.per_block - 1) / A.per_block;
+        const unsigned active = (unsigned)(want < 1 ? 1 : (want > A.grid ? A.grid : want));
+        if (blockIdx.x >= active) return;  // no pairs for this block in this or any later round
+        int w[4] = {0, 0, 0, 0};
+        if (t == 1) lh2_tables(tab, zs, A.v, w);
+        GlAcc H0a, H0b, H1a, H1b;
+        E2Acc q0, q1, q2;
+        for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
+            Ext2 h0, h1, f0, f1, e;
+            if (t == 1) {
+                h0 = e2_ldcg(A.h + b);
+                h1 = e2_ldcg(A.h + b + h);
+                f0 = e2_make(gl_from_i64(lh_key(A.r, A.n, b)), 0);
+                f1 = e2_make(gl_from_i64(lh_key(A.r, A.n, b + h)), 0);
+                e = lh2_eq_at(tab, w, b);  // eq(z_2..z_v, b)
+                if (A.v > 1) A.E[b] = e;
+            } else {
+                if (t == 2) {
+                    // the column and the keys (length 4h) folded by rho_1
+                    h0 = e2_fold(e2_ldcg(A.h + b), e2_ldcg(A.h + b + 2 * h), rho);
+                    h1 = e2_fold(e2_ldcg(A.h + b + h), e2_ldcg(A.h + b + 3 * h), rho);
+                    f0 = lh2_fold_keys(lh_key(A.r, A.n, b), lh_key(A.r, A.n, b + 2 * h), rho);
+                    f1 = lh2_fold_keys(lh_key(A.r, A.n, b + h), lh_key(A.r, A.n, b + 3 * h), rho);
+                } else {
+                    h0 = e2_fold(e2_ldcg(A.Hv + b), e2_ldcg(A.Hv + b + 2 * h), rho);
+                    h1 = e2_fold(e2_ldcg(A.Hv + b + h), e2_ldcg(A.Hv + b + 3 * h), rho);
+                    f0 = e2_fold(e2_ldcg(A.Fv + b), e2_ldcg(A.Fv + b + 2 * h), rho);
+                    f1 = e2_fold(e2_ldcg(A.Fv + b + h), e2_ldcg(A.Fv + b + 3 * h), rho);
+                }
+                A.Hv[b] = h0;
+                A.Hv[b + h] = h1;
+                A.Fv[b] = f0;
+                A.Fv[b + h] = f1;
+                e = e2_add(e2_ldcg(A.E + b), e2_ldcg(A.E + b + h));  // eq(z_>t, b)
+                A.E[b] = e;
+            }
+            H0a.add(h0.a);
+            H0b.add(h0.b);
+            H1a.add(h1.a);
+            H1b.add(h1.b);
+            const uint64_t e7 = gl_mul7(e.b);
+            q0.mac(e, e7, e2_mul(h0, e2_sub(A.alpha, f0)));
+            q1.mac(e, e7, e2_mul(h1, e2_sub(A.alpha, f1)));
+            q2.mac(e, e7, e2_mul(e2_at2(h0, h1), e2_sub(A.alpha, e2_at2(f0, f1))));
+        }
+        uint64_t acc[10] = {H0a.value(), H0b.value(), H1a.value(), H1b.value(), q0.a.value(),
+                            q0.b.value(), q1.a.value(), q1.b.value(), q2.a.value(), q2.b.value()};
+        bool last;
+        if (active == 1) {
+            block_sum_gl<10>(acc);
+            last = true;
+        } else {
+            last = grid_sum_gl_n<10>(acc, part, &rl->ticket, active);
+        }
+        if (last && threadIdx.x == 0) session_publish(mb, acc, A.seq0 + t);  // {H(0), H(1), Q(0), Q(1), Q(2)}
+    }
+    // block 0 folds the last pair by the last challenge: h~(rho), f~(rho)
+    if (A.t_end <= A.v || blockIdx.x != 0) return;
+    uint64_t ra, rb;
+    if (!session_wait2(mb, rl, A.seq0 + A.v, ra, rb)) return;
+    rho = e2_make(ra, rb);
+    if (threadIdx.x == 0) {
+        Ext2 hf, ff;
+        if (A.v == 1) {
+            hf = e2_fold(e2_ldcg(A.h), e2_ldcg(A.h + 1), rho);
+            ff = lh2_fold_keys(lh_key(A.r, A.n, 0), lh_key(A.r, A.n, 1), rho);
+        } else {
+            hf = e2_fold(e2_ldcg(A.Hv), e2_ldcg(A.Hv + 1), rho);
+            ff = e2_fold(e2_ldcg(A.Fv), e2_ldcg(A.Fv + 1), rho);
+        }
+        const uint64_t fin[4] = {hf.a, hf.b, ff.a, ff.b};
+        session_publish(mb, fin, A.seq0 + A.v + 1);
+    }
+}
+
+struct Lhi2Source {
+    virtual ~Lhi2Source() {}
+    virtual void abandon() {}  // the host stopped early: let a waiting kernel finish
+    virtual int column(Ext2 alpha, uint8_t digest[32]) = 0;   // commit h, return D(h)
+    virtual int start(const Ext2* z, int v, Ext2 beta) = 0;   // the point is known
+    virtual int round(int t, Ext2 vals[5]) = 0;               // H(0), H(1), Q(0), Q(1), Q(2)
+    virtual int answer(int t, Ext2 rho) = 0;
+    virtual int finals(Ext2 fin[2]) = 0;                      // h~(rho), f~(rho)
+};
+
+// The statement over the extension after "lhi2_site" is absorbed, from the multiplicities on:
+// 4 2^k + 16 + 64 v + 32 proof bytes.
+int lhi2_protocol(fp_ctx* c, fp_tx* tx, int v, int k, const uint32_t* m, const uint8_t m_digest[32],
+                  Lhi2Source& src, uint8_t* proof, size_t* proof_len) {
+    int rc;
+    size_t pos = 0;
+    const size_t T = (size_t)1 << k;
+    for (size_t j = 0; j < T; j++)
+        for (int b = 0; b < 4; b++) proof[4 * j + b] = (uint8_t)(m[j] >> (8 * b));
+    pos += 4 * T;
+    fp_tx_absorb_raw(tx, "lhi2_m", m_digest, 32);
+    const Ext2 alpha = e2_squeeze_host(tx, "lhi2_alpha");
+    {
+        uint8_t hd[32];
+        if ((rc = src.column(alpha, hd))) return rc;
+        fp_tx_absorb_raw(tx, "lhi2_h", hd, 32);
+    }
+    Ext2 z[LH_MAX_V];
+    for (int i = 0; i < v; i++) z[i] = e2_squeeze_host(tx, "lhi2_z");
+    const Ext2 beta = e2_squeeze_host(tx, "lhi2_beta");
+    if ((rc = src.start(z, v, beta))) return rc;
+    const Ext2 one = e2_make(1, 0);
+    Ext2 claim = e2_make(0, 0), pre = one;  // pre = eq(z_<t, rho_<t)
+    for (int t = 1; t <= v; t++) {
+        Ext2 w[5];
+        if ((rc = src.round(t, w))) return rc;
+        if (t == 1) {
+            claim = e2_add(w[0], w[1]);  // S = the sum of h over the whole cube
+            e2_send_host(tx, "lhi2_sum", &claim, 1, proof, pos);
+        }
+        const Ext2 zt = z[t - 1], scale = e2_mul(beta, pre);
+        const Ext2 H[4] = {w[0], w[1], e2_at2(w[0], w[1]), e2_sub(e2_scal(w[1], 3), e2_add(w[0], w[0]))};
+        const Ext2 Q[4] = {w[2], w[3], w[4], e2_add(e2_sub(w[2], e2_scal(w[3], 3)), e2_scal(w[4], 3))};
+        const Ext2 eqX[4] = {e2_sub(one, zt), zt, e2_sub(e2_scal(zt, 3), one), e2_sub(e2_scal(zt, 5), e2_make(2, 0))};
+        Ext2 g[4];
+        for (int X = 0; X < 4; X++) g[X] = e2_add(H[X], e2_mul(scale, e2_mul(eqX[X], e2_sub(Q[X], one))));
+        if (!e2_same(e2_add(g[0], g[1]), claim)) {
+            src.abandon();
+            return fp_fail(c, FP_ERR_CUDA, "logup_prove_helper_inverse_ext2: round values inconsistent with the claim");
+        }
+        e2_send_host(tx, "lhi2_round", g, 4, proof, pos);
+        const Ext2 r = e2_squeeze_host(tx, "lhi2_chal");
+        if ((rc = src.answer(t, r))) return rc;
+        claim = e2_lagrange4(g, r);
+        pre = e2_mul(pre, e2_eq(zt, r));
+    }
+    Ext2 fin[2];
+    if ((rc = src.finals(fin))) return rc;
+    e2_send_host(tx, "lhi2_final", fin, 2, proof, pos);
+    *proof_len = pos;
+    return FP_OK;
+}
+
+struct Lhi2Device : Lhi2Source {
+    fp_ctx* c;
+    cudaStream_t st;
+    const int32_t* r;
+    int64_t n;
+    int k;
+    int v;
+    Ext2* hcol = nullptr;
+    Ext2* inv = nullptr;
+    uint64_t* part = nullptr;
+    uint64_t* small = nullptr;  // device: [8 .. 8 + 2 v) z
+    uint64_t* hs = nullptr;
+    Lhi2Args A;
+    int cap_grid = 1;
+
+    unsigned grid_of(int64_t work) const {
+        return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
+    }
+
+    void abandon() override { fp_session_abandon(c, st); }
+
+    int launch(int t_begin, int t_end, unsigned grid, int kernel, double bytes) {
+        A.t_begin = t_begin;
+        A.t_end = t_end;
+        void* args[] = {&A, &c->mb_dev, &c->relay, &part};
+        int slot;
+        fp_tic(c, st, kernel, bytes, &slot);
+        FP_CUDA(c, cudaLaunchCooperativeKernel((const void*)lhi2_session_kernel, dim3(grid), dim3(LH_THREADS), args,
+                                               0, st));
+        fp_toc(c, st, slot);
+        return FP_OK;
+    }
+
+    double round_bytes(int t) const {
+        const double pairs = (double)(1ll << (v - t));
+        // round 1: two 16-byte column reads, two key reads and one E write per pair; round 2:
+        // four column and four key reads, two E reads, four folded writes, one E write; later
+        // rounds read eight folded values instead
+        return t == 1 ? 56.0 * pairs : (t == 2 ? 176.0 * pairs : 240.0 * pairs);
+    }
+
+    int column(Ext2 alpha, uint8_t digest[32]) override {
+        const int64_t L = 1ll << v, T = 1ll << k;
+        int slot;
+        fp_tic(c, st, K_LHI2_COLUMN, 16.0 * (double)T + 20.0 * (double)L, &slot);
+        lhi2_inv_kernel<<<grid_of(T), 256, 0, st>>>(alpha, k, inv);
+        lhi2_column_kernel<<<grid_of(L), 256, 0, st>>>(r, n, L, k, alpha, inv, hcol);
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+        c->launches++;  // two kernels under one timing slot
+        A.alpha = alpha;
+        FpDigestJob job = {(const uint8_t*)hcol, 16 * (uint64_t)L};
+        return fp_digest_many(c, &job, 1, digest, st);  // synchronises the stream
+    }
+
+    int start(const Ext2* z, int vv, Ext2 beta) override {
+        (void)beta;  // the host alone applies beta
+        int rc;
+        for (int i = 0; i < vv; i++) {
+            hs[8 + 2 * i] = z[i].a;
+            hs[9 + 2 * i] = z[i].b;
+        }
+        FP_CUDA(c, cudaMemcpyAsync(small + 8, hs + 8, 16 * (size_t)vv, cudaMemcpyHostToDevice, st));
+        A.z = (const Ext2*)(small + 8);
+        A.v = vv;
+        A.per_block = LH_THREADS;  // one pair per thread
+        const int64_t half = 1ll << (vv - 1);
+        A.grid = (int)std::max<int64_t>(1, std::min<int64_t>((half + A.per_block - 1) / A.per_block, cap_grid));
+        A.seq0 = fp_seq_reserve(c, (uint64_t)vv + 2);
+        if ((rc = fp_session_begin(c, st))) return rc;
+        fp_session_expect(c, 10);  // before any launch: round 1 publishes without a challenge
+        if (!c->stepped) {
+            double bytes = 0;
+            for (int t = 1; t <= vv; t++) bytes += round_bytes(t);
+            return launch(1, vv + 1, (unsigned)A.grid, K_LHI2_ROUND, bytes);
+        }
+        return FP_OK;
+    }
+
+    int round(int t, Ext2 vals[5]) override {
+        int rc;
+        if (c->stepped && (rc = launch(t, t, (unsigned)A.grid, K_LHI2_ROUND, round_bytes(t)))) return rc;
+        if ((rc = fp_session_wait(c, A.seq0 + t, st))) return rc;
+        for (int i = 0; i < 5; i++) vals[i] = e2_make(c->mb->res[2 * i], c->mb->res[2 * i + 1]);
+        return FP_OK;
+    }
+
+    int answer(int t, Ext2 rho) override {
+        fp_session_expect(c, t < v ? 10 : 4);  // the last challenge triggers the final values
+        fp_session_post2(c, A.seq0 + t, rho.a, rho.b);
+        return FP_OK;
+    }
+
+    int finals(Ext2 fin[2]) override {
+        int rc;
+        if (c->stepped && (rc = launch(v + 1, v + 1, 1, K_LHI2_FINAL, 64.0))) return rc;
+        if ((rc = fp_session_wait(c, A.seq0 + v + 1, st))) return rc;
+        fin[0] = e2_make(c->mb->res[0], c->mb->res[1]);
+        fin[1] = e2_make(c->mb->res[2], c->mb->res[3]);
+        FP_CUDA(c, cudaStreamSynchronize(st));
+        return FP_OK;
+    }
+};
+
+struct Lhi2Callback : Lhi2Source {
+    fp_values_fn fn;
+    void* user;
+    int call(int kind, int t, const uint64_t* in, uint64_t* out) { return fn(user, kind, t, in, out) ? FP_ERR_ARG : FP_OK; }
+    static Ext2 ext(const uint64_t* w) { return e2_make(gl_canon(w[0]), gl_canon(w[1])); }
+    int column(Ext2 alpha, uint8_t digest[32]) override {
+        const uint64_t in[2] = {alpha.a, alpha.b};
+        uint64_t out[4] = {0, 0, 0, 0};
+        const int rc = call(FP_VAL_COLUMN, 0, in, out);
+        for (int i = 0; i < 4; i++)
+            for (int b = 0; b < 8; b++) digest[8 * i + b] = (uint8_t)(out[i] >> (8 * b));
+        return rc;
+    }
+    int start(const Ext2* z, int v, Ext2 beta) override {
+        uint64_t in[2 * LH_MAX_V + 2];
+        for (int i = 0; i < v; i++) {
+            in[2 * i] = z[i].a;
+            in[2 * i + 1] = z[i].b;
+        }
+        in[2 * v] = beta.a;
+        in[2 * v + 1] = beta.b;
+        return call(FP_VAL_START, v, in, nullptr);
+    }
+    int round(int t, Ext2 vals[5]) override {
+        uint64_t out[10] = {0};
+        const int rc = call(FP_VAL_ROUND, t, nullptr, out);
+        for (int i = 0; i < 5; i++) vals[i] = ext(out + 2 * i);
+        return rc;
+    }
+    int answer(int t, Ext2 rho) override {
+        const uint64_t in[2] = {rho.a, rho.b};
+        return call(FP_VAL_ANSWER, t, in, nullptr);
+    }
+    int finals(Ext2 fin[2]) override {
+        uint64_t out[4] = {0, 0, 0, 0};
+        const int rc = call(FP_VAL_FINALS, 0, nullptr, out);
+        fin[0] = ext(out);
+        fin[1] = ext(out + 2);
+        return rc;
+    }
+};
+
+size_t lhi2_proof_len(int v, int k) { return 4 * ((size_t)1 << k) + 16 + 64 * (size_t)v + 32; }
+
 }  // namespace
 
 size_t fp_lhi_proof_len(int64_t n, int k) { return lhi_proof_len(std::max(1, fp_log2_ceil((uint64_t)n)), k); }
@@ -530,4 +918,107 @@ int fp_lhi_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uint
     cb.fn = fn;
     cb.user = user;
     return lhi_protocol(nullptr, tx, v, k, m, m_digest, cb, proof, proof_len);
+}
+
+int logup_prove_helper_inverse_ext2(fp_ctx* c, fp_tx* tx, const int32_t* r, int64_t n, int k, uint8_t* proof,
+                                    size_t* proof_len, void* stream) {
+    if (!c || !tx || !proof_len || !r)
+        return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse_ext2: null argument");
+    if (k < 1 || k > LH_MAX_K) return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse_ext2: need 1 <= k <= 24");
+    if (n < 1 || n > (1ll << LH_MAX_V))
+        return fp_fail(c, FP_ERR_SHAPE, "logup_prove_helper_inverse_ext2: need 1 <= n <= 2^30");
+    const int v = std::max(1, fp_log2_ceil((uint64_t)n));
+    const size_t need_len = lhi2_proof_len(v, k);
+    if (!proof || *proof_len < need_len) {
+        *proof_len = need_len;
+        return fp_fail(c, FP_ERR_ARG, "logup_prove_helper_inverse_ext2: proof buffer too small");
+    }
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t st = (cudaStream_t)stream;
+    int rc;
+    {
+        FpDigestJob job = {(const uint8_t*)r, 4 * (uint64_t)n};
+        uint8_t d[32];
+        if ((rc = fp_digest_many(c, &job, 1, d, st))) return rc;  // synchronises the stream
+        fp_tx_absorb_raw(tx, "lhi2_site", d, 32);
+    }
+    const int64_t L = 1ll << v, T = 1ll << k, half = L / 2;
+    Lhi2Device dev;
+    dev.c = c;
+    dev.st = st;
+    dev.r = r;
+    dev.n = n;
+    dev.k = k;
+    dev.v = v;
+    int occ = 0;
+    FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, lhi2_session_kernel, LH_THREADS, 0));
+    dev.cap_grid = std::max(1, occ) * c->num_sms;
+    const size_t part_n = (size_t)10 * dev.cap_grid;
+    const size_t need = fp_align_up((size_t)16 * L, 256) + 3 * fp_align_up((size_t)16 * half, 256) +
+                        fp_align_up((size_t)16 * T, 256) + fp_align_up((size_t)4 * T, 256) +
+                        fp_align_up(8 * part_n, 256) + 2 * fp_align_up(8 * 128, 256) + 4096;
+    if ((rc = fp_reserve(c, c->dev, need))) return rc;
+    if ((rc = fp_reserve(c, c->host, fp_align_up((size_t)4 * T, 256) + fp_align_up(8 * 128, 256) + 4096))) return rc;
+    fp_reset(c->dev);
+    fp_reset(c->host);
+    dev.hcol = (Ext2*)fp_alloc(c->dev, (size_t)16 * L);
+    Ext2* Hv = (Ext2*)fp_alloc(c->dev, (size_t)16 * half);
+    Ext2* Fv = (Ext2*)fp_alloc(c->dev, (size_t)16 * half);
+    Ext2* E = (Ext2*)fp_alloc(c->dev, (size_t)16 * half);
+    dev.inv = (Ext2*)fp_alloc(c->dev, (size_t)16 * T);
+    uint32_t* m = (uint32_t*)fp_alloc(c->dev, (size_t)4 * T);
+    dev.part = (uint64_t*)fp_alloc(c->dev, 8 * part_n);
+    dev.small = (uint64_t*)fp_alloc(c->dev, 8 * 128);
+    uint32_t* outside = (uint32_t*)fp_alloc(c->dev, 8 * 128);
+    uint32_t* hm = (uint32_t*)fp_alloc(c->host, (size_t)4 * T);
+    dev.hs = (uint64_t*)fp_alloc(c->host, 8 * 128);
+    if (!dev.hcol || !Hv || !Fv || !E || !dev.inv || !m || !dev.part || !dev.small || !outside || !hm || !dev.hs)
+        return fp_fail(c, FP_ERR_OOM, "logup_prove_helper_inverse_ext2: scratch exhausted");
+    memset(&dev.A, 0, sizeof dev.A);
+    dev.A.r = r;
+    dev.A.n = n;
+    dev.A.h = dev.hcol;
+    dev.A.Hv = Hv;
+    dev.A.Fv = Fv;
+    dev.A.E = E;
+    FP_CUDA(c, cudaMemsetAsync(m, 0, (size_t)4 * T, st));
+    FP_CUDA(c, cudaMemsetAsync(outside, 0, 4, st));
+    {
+        const int in_smem = T <= LH_SMEM_BINS;
+        const int smem = in_smem ? 4 * (int)T : 0;
+        if (smem > 48 * 1024)
+            FP_CUDA(c, cudaFuncSetAttribute(lhi_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+        int slot;
+        fp_tic(c, st, K_LHI_HIST, 4.0 * (double)n + 4.0 * (double)T, &slot);
+        lhi_hist_kernel<<<c->num_sms, 1024, smem, st>>>(r, n, L, k, m, outside, in_smem);
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+    }
+    FP_CUDA(c, cudaMemcpyAsync(hm, m, (size_t)4 * T, cudaMemcpyDeviceToHost, st));
+    FP_CUDA(c, cudaMemcpyAsync(dev.hs, outside, 4, cudaMemcpyDeviceToHost, st));
+    uint8_t md[32];
+    {
+        FpDigestJob job = {(const uint8_t*)m, 4 * (uint64_t)T};
+        if ((rc = fp_digest_many(c, &job, 1, md, st))) return rc;  // synchronises the stream
+    }
+    uint32_t n_outside;
+    memcpy(&n_outside, dev.hs, 4);
+    if ((rc = lhi2_protocol(c, tx, v, k, hm, md, dev, proof, proof_len))) return rc;
+    return n_outside ? 1 : FP_OK;
+}
+
+int fp_lhi2_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uint8_t* m_digest, fp_values_fn fn,
+                           void* user, uint8_t* proof, size_t* proof_len) {
+    if (!tx || !fn || !proof_len || !m || !m_digest) return FP_ERR_ARG;
+    if (v < 1 || v > LH_MAX_V) return FP_ERR_SHAPE;
+    if (k < 1 || k > LH_MAX_K) return FP_ERR_ARG;
+    const size_t need_len = lhi2_proof_len(v, k);
+    if (!proof || *proof_len < need_len) {
+        *proof_len = need_len;
+        return FP_ERR_ARG;
+    }
+    Lhi2Callback cb;
+    cb.fn = fn;
+    cb.user = user;
+    return lhi2_protocol(nullptr, tx, v, k, m, m_digest, cb, proof, proof_len);
 }

@@ -263,3 +263,85 @@ def test_mm2_inconsistent_round_is_refused(fp, t, X):
     s, w = _mm_site(2, 4, 2, 8, False, 5)
     with pytest.raises(fp.FpError):
         _mm_drive(fp, 1, s, w, BruteMm2(s, w, tamper=(t, X)))
+
+
+# ---- the helper-inverse LogUp over the extension ------------------------------------------
+
+class BruteLhi2:
+    """Device values of the extension-field helper-inverse LogUp by their definitions."""
+
+    def __init__(self, r, k, tamper=None):
+        self.r = [int(x) for x in r]
+        self.v = max(1, bf.log2c(len(self.r)))
+        L = 1 << self.v
+        self.f = [x % P for x in self.r] + [0] * (L - len(self.r))
+        self.rho = []
+        self.tamper = tamper
+
+    def column(self, alpha):
+        import struct as _s
+        self.alpha = alpha
+        self.h = [bf.x_inv(((alpha[0] - x) % P, alpha[1])) for x in self.f]
+        return bf.tree_digest(b"".join(_s.pack("<QQ", a, b) for a, b in self.h))
+
+    def start(self, z, beta):
+        self.z, self.beta = z, beta
+
+    def _h(self, w):
+        acc = (0, 0)
+        for x in range(len(self.h)):
+            acc = bf.x_add(acc, bf.x_mul(bf.x_eq(w, [((x >> (self.v - 1 - i)) & 1, 0) for i in range(self.v)]),
+                                         self.h[x]))
+        return acc
+
+    def round(self, t):
+        rest = self.v - t
+        H, Q = [], []
+        for X in range(3):
+            hs = qs = (0, 0)
+            for b in range(1 << rest):
+                bits = [((b >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                w = self.rho + [(X, 0)] + bits
+                hw, fw = self._h(w), bf.x_mle(self.f, w)
+                hs = bf.x_add(hs, hw)
+                am = bf.x_add(self.alpha, ((-fw[0]) % P, (-fw[1]) % P))
+                qs = bf.x_add(qs, bf.x_mul(bf.x_eq(self.z[t:], bits), bf.x_mul(hw, am)))
+            H.append(hs)
+            Q.append(qs)
+        out = [H[0], H[1], Q[0], Q[1], Q[2]]
+        if self.tamper == t:
+            out[2] = ((out[2][0] + 1) % P, out[2][1])
+        return out
+
+    def answer(self, t, rho):
+        assert t == len(self.rho) + 1
+        self.rho.append(rho)
+
+    def finals(self):
+        return [self._h(self.rho), bf.x_mle(self.f, self.rho)]
+
+
+def _lhi2_drive(fp, seed, r, k, vals):
+    tx = fp.Transcript(seed)
+    tx.absorb("lhi2_site", bf.tree_digest(np.asarray(r, "<i4").tobytes()))
+    m = np.zeros(1 << k, np.int64)
+    for x in list(r) + [0] * ((1 << vals.v) - len(r)):
+        j = int(x) + (1 << (k - 1))
+        if 0 <= j < (1 << k):
+            m[j] += 1
+    m = m.astype("<u4")
+    return fp.lhi2_protocol_drive(tx, vals.v, k, m, bf.tree_digest(m.tobytes()), vals), tx.state()
+
+
+@pytest.mark.parametrize("n,k", [(1, 1), (3, 4), (5, 7), (8, 3), (13, 5)])
+def test_lhi2_host_half_matches_oracle(fp, n, k):
+    r = np.random.default_rng(n + 50 * k).integers(-(1 << (k - 1)), 1 << (k - 1), n).astype(np.int32)
+    vals = BruteLhi2(r, k)
+    assert _lhi2_drive(fp, 3, r, k, vals) == oracle.lhi2_prove(3, r, k)
+
+
+@pytest.mark.parametrize("t", [1, 2])
+def test_lhi2_inconsistent_round_is_refused(fp, t):
+    r = np.random.default_rng(8).integers(-8, 8, 8).astype(np.int32)
+    with pytest.raises(fp.FpError):
+        _lhi2_drive(fp, 1, r, 4, BruteLhi2(r, 4, tamper=t))

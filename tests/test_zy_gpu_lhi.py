@@ -114,3 +114,36 @@ def test_ffn_projection_remainders_verified(env):
     assert status == 0
     assert len(pf) == 4 * 4096 + 8 + 32 * 24 + 16
     assert oracle.lhi_verify(31, r, 12, pf) == ("accept", (0, 0))
+
+
+# ---- the same statement over the quadratic extension --------------------------------------
+
+def _gpu2(env, seed, r, k):
+    torch, fp, ctx = env
+    tx = fp.Transcript(seed)
+    pf, status = ctx.prove_helper_inverse_ext2(tx, torch.from_numpy(r).cuda(), k)
+    torch.cuda.synchronize()
+    return pf, tx.state(), status
+
+
+@pytest.mark.parametrize("n,k", [(1, 7), (2, 1), (3, 7), (257, 12), (1000, 16), (4097, 8), (65537, 7)])
+def test_ext2_matches_oracle(env, n, k):
+    r = _keys(n, k, 5000 + n + k)
+    pf, st, status = _gpu2(env, 4, r, k)
+    assert status == 0
+    assert (pf, st) == oracle.lhi2_prove(4, r, k)
+
+
+def test_ext2_keys_outside_and_stepped(env):
+    torch, fp, ctx = env
+    r = _keys(70001, 12, 9)
+    r[[3, 60000]] = [5000, -5000]
+    a = _gpu2(env, 2, r, 12)
+    ctx.set_profiling(True)
+    b = _gpu2(env, 2, r, 12)
+    stats = ctx.kernel_stats()
+    ctx.set_profiling(False)
+    assert a == b and a[2] == 1
+    assert stats["lhi2_round"][0] == 17
+    assert (a[0], a[1]) == oracle.lhi2_prove(2, r, 12)
+    assert oracle.lhi2_verify(2, r, 12, a[0])[0] == "lhi2_sum"
