@@ -152,6 +152,12 @@ def lib():
         L.orc_exp_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
         L.orc_exp_verify.restype = C.c_int
         L.orc_exp_verify.argtypes = [vp, vp, vp, u64, vp, u64, vp]
+        for nm in ("orc_silu2_prove", "orc_exp2_prove"):
+            getattr(L, nm).restype = C.c_int
+            getattr(L, nm).argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
+        for nm in ("orc_silu2_verify", "orc_exp2_verify"):
+            getattr(L, nm).restype = C.c_int
+            getattr(L, nm).argtypes = [vp, vp, vp, u64, vp, u64, vp]
         L.orc_lhi_prove.restype = C.c_int
         L.orc_lhi_prove.argtypes = [vp, vp, u64, C.c_int, vp, u64, C.POINTER(u64)]
         L.orc_lhi_verify.restype = C.c_int
@@ -574,6 +580,24 @@ def exp_prove(seed: int, g, s):
 
 def exp_verify(seed: int, g, s, proof: bytes):
     return _lookup16_verify(lib().orc_exp_verify, seed, g, s, proof)
+
+
+def silu2_prove(seed: int, g, s):
+    """The SiLU lookup with every challenge and value in the quadratic extension."""
+    return _lookup16_prove(lib().orc_silu2_prove, seed, g, s)
+
+
+def silu2_verify(seed: int, g, s, proof: bytes):
+    return _lookup16_verify(lib().orc_silu2_verify, seed, g, s, proof)
+
+
+def exp2_prove(seed: int, g, s):
+    """The softmax numerator lookup with every challenge and value in the quadratic extension."""
+    return _lookup16_prove(lib().orc_exp2_prove, seed, g, s)
+
+
+def exp2_verify(seed: int, g, s, proof: bytes):
+    return _lookup16_verify(lib().orc_exp2_verify, seed, g, s, proof)
 
 
 # ---- the helper-inverse LogUp (the variant to set against the GKR tree) -------------

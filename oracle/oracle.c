@@ -2865,3 +2865,227 @@ done:
     free(rho);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* The 16-bit function lookup (the LogUp-GKR tree of lookup16_prove) over    */
+/* the extension (next row f4, "How fast can FlashProve go", 4, the note on  */
+/* soundness): gamma, alpha, mu, lambda, every round challenge and every     */
+/* value sent are extension elements (16 bytes); the tree's fractions live   */
+/* in the extension; labels "<fn>2_*" (silu2_site, silu2_gamma, silu2_m,     */
+/* silu2_alpha, silu2_l1, silu2_mu, silu2_lambda, silu2_round, silu2_chal,   */
+/* silu2_final, silu2_leaf; exp2_* likewise). Keys f = g + gamma s, padded   */
+/* with (0, table(0)); the verifier checks the root against the table side   */
+/* sum_j m_j / (alpha - v_j - gamma table(v_j)) in the extension.            */
+/* ------------------------------------------------------------------------ */
+
+static const lk_labels LK_SILU2 = {"silu2_site", "silu2_gamma", "silu2_m", "silu2_alpha", "silu2_l1", "silu2_mu",
+                                   "silu2_lambda", "silu2_round", "silu2_chal", "silu2_final", "silu2_leaf"};
+static const lk_labels LK_EXP2 = {"exp2_site", "exp2_gamma", "exp2_m", "exp2_alpha", "exp2_l1", "exp2_mu",
+                                  "exp2_lambda", "exp2_round", "exp2_chal", "exp2_final", "exp2_leaf"};
+
+static ext2 x16_F(const ext2 x[4], ext2 lam) { /* pL qR + pR qL + lambda qL qR */
+    return e2_add(e2_add(e2_mul(x[0], x[3]), e2_mul(x[1], x[2])), e2_mul(lam, e2_mul(x[2], x[3])));
+}
+
+/* MLE at an extension point of a base column given as field elements */
+static ext2 x16_mle(const u64* col, u64 L, const ext2* z, int v) {
+    ext2* E = (ext2*)malloc(sizeof(ext2) * L);
+    e2_eq_table(z, v, E);
+    ext2 acc = e2(0, 0);
+    for (u64 x = 0; x < L; x++) acc = e2_add(acc, e2_scal(E[x], col[x]));
+    free(E);
+    return acc;
+}
+
+static void x16_leaf_values(const int16_t* g, const int16_t* s, u64 n, int v, const ext2* z, int32_t pad_s,
+                            ext2 out[2]) {
+    u64 L = (u64)1 << v;
+    u64* col = (u64*)malloc(L * sizeof(u64));
+    for (u64 i = 0; i < L; i++) col[i] = i < n ? orc_fint(g[i]) : 0;
+    out[0] = x16_mle(col, L, z, v);
+    for (u64 i = 0; i < L; i++) col[i] = i < n ? orc_fint(s[i]) : orc_fint(pad_s);
+    out[1] = x16_mle(col, L, z, v);
+    free(col);
+}
+
+static int lookup16x_prove(void* txh, const lk_labels* lab, int32_t pad_s, const int16_t* g, const int16_t* s, u64 n,
+                           uint8_t* proof, u64 cap, u64* len) {
+    if (n < 1) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n);
+    if (v < 1) v = 1;
+    u64 L = (u64)1 << v;
+    pbuf pb = {proof, cap, 0, 0};
+    silu_absorb_site(t, lab, g, s, n);
+    ext2 gamma = e2_squeeze(t, lab->gamma);
+    u32* m = (u32*)malloc(65536 * sizeof(u32));
+    silu_mult(g, n, L, m);
+    send_mult(t, &pb, lab->m, m, 65536);
+    ext2 alpha = e2_squeeze(t, lab->alpha);
+    /* the fraction tree: layer d has 2^d nodes */
+    ext2** Pd = (ext2**)malloc(sizeof(ext2*) * (v + 1));
+    ext2** Qd = (ext2**)malloc(sizeof(ext2*) * (v + 1));
+    Pd[v] = (ext2*)malloc(L * sizeof(ext2));
+    Qd[v] = (ext2*)malloc(L * sizeof(ext2));
+    for (u64 i = 0; i < L; i++) {
+        ext2 f = i < n ? e2_add(e2(orc_fint(g[i]), 0), e2_scal(gamma, orc_fint(s[i]))) : e2_scal(gamma, orc_fint(pad_s));
+        Pd[v][i] = e2(1, 0);
+        Qd[v][i] = e2_sub(alpha, f);
+    }
+    for (int d = v - 1; d >= 0; d--) {
+        u64 c = (u64)1 << d;
+        Pd[d] = (ext2*)malloc(c * sizeof(ext2));
+        Qd[d] = (ext2*)malloc(c * sizeof(ext2));
+        for (u64 x = 0; x < c; x++) {
+            Pd[d][x] = e2_add(e2_mul(Pd[d + 1][2 * x], Qd[d + 1][2 * x + 1]), e2_mul(Pd[d + 1][2 * x + 1], Qd[d + 1][2 * x]));
+            Qd[d][x] = e2_mul(Qd[d + 1][2 * x], Qd[d + 1][2 * x + 1]);
+        }
+    }
+    ext2 l1[4] = {Pd[1][0], Pd[1][1], Qd[1][0], Qd[1][1]};
+    e2_send(t, &pb, lab->l1, l1, 4);
+    ext2* z = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    z[0] = e2_squeeze(t, lab->mu);
+    for (int d = 1; d < v; d++) {
+        ext2 lam = e2_squeeze(t, lab->lambda);
+        u64 c = (u64)1 << d;
+        ext2* V[5]; /* pL, pR, qL, qR (children of layer d), eq(z, .) */
+        for (int i = 0; i < 5; i++) V[i] = (ext2*)malloc(c * sizeof(ext2));
+        for (u64 x = 0; x < c; x++) {
+            V[0][x] = Pd[d + 1][2 * x];
+            V[1][x] = Pd[d + 1][2 * x + 1];
+            V[2][x] = Qd[d + 1][2 * x];
+            V[3][x] = Qd[d + 1][2 * x + 1];
+        }
+        e2_eq_table(z, d, V[4]);
+        ext2* rho = (ext2*)malloc(sizeof(ext2) * d);
+        u64 Lr = c;
+        for (int r = 0; r < d; r++) {
+            u64 h = Lr >> 1;
+            ext2 gr[4] = {e2(0, 0), e2(0, 0), e2(0, 0), e2(0, 0)};
+            for (u64 b = 0; b < h; b++)
+                for (u64 X = 0; X < 4; X++) {
+                    ext2 ev[5];
+                    for (int i = 0; i < 5; i++) ev[i] = e2_add(V[i][b], e2_scal(e2_sub(V[i][h + b], V[i][b]), X));
+                    gr[X] = e2_add(gr[X], e2_mul(ev[4], x16_F(ev, lam)));
+                }
+            e2_send(t, &pb, lab->round, gr, 4);
+            rho[r] = e2_squeeze(t, lab->chal);
+            for (int i = 0; i < 5; i++)
+                for (u64 b = 0; b < h; b++) V[i][b] = e2_add(V[i][b], e2_mul(rho[r], e2_sub(V[i][h + b], V[i][b])));
+            Lr = h;
+        }
+        ext2 fin[4] = {V[0][0], V[1][0], V[2][0], V[3][0]};
+        e2_send(t, &pb, lab->fin, fin, 4);
+        ext2 mu = e2_squeeze(t, lab->mu);
+        for (int r = 0; r < d; r++) z[r] = rho[r];
+        z[d] = mu;
+        for (int i = 0; i < 5; i++) free(V[i]);
+        free(rho);
+    }
+    ext2 leaf[2];
+    x16_leaf_values(g, s, n, v, z, pad_s, leaf);
+    e2_send(t, &pb, lab->leaf, leaf, 2);
+    for (int d = 0; d <= v; d++) {
+        free(Pd[d]);
+        free(Qd[d]);
+    }
+    free(Pd);
+    free(Qd);
+    free(z);
+    free(m);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+static int e2_eqv(ext2 x, ext2 y) { return x.a == y.a && x.b == y.b; }
+
+static int lookup16x_verify(void* txh, const lk_labels* lab, int32_t (*tab)(int32_t), const int16_t* g,
+                            const int16_t* s, u64 n, const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (n < 1) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int v = orc_log2_ceil(n), rc = 0;
+    if (v < 1) v = 1;
+    prd rd = {proof, len, 0, 0};
+    u32* m = (u32*)malloc(65536 * sizeof(u32));
+    ext2* z = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    ext2* rho = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    silu_absorb_site(t, lab, g, s, n);
+    ext2 gamma = e2_squeeze(t, lab->gamma);
+    rd_mult(t, &rd, lab->m, m, 65536);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    ext2 alpha = e2_squeeze(t, lab->alpha);
+    ext2 l1[4];
+    e2_read(t, &rd, lab->l1, l1, 4);
+    if (rd.bad) FAIL(REJ_FORMAT, 1, 0);
+    {
+        /* the table side, sum_j m_j / (alpha - t_j) with t_j = v_j + gamma tab(v_j) */
+        ext2 PT = e2(0, 0), QT = e2(1, 0);
+        for (u64 j = 0; j < 65536; j++) {
+            int32_t vj = (int32_t)j - 32768;
+            ext2 dj = e2_sub(alpha, e2_add(e2(orc_fint(vj), 0), e2_scal(gamma, orc_fint(tab(vj)))));
+            PT = e2_add(e2_mul(PT, dj), e2_scal(QT, (u64)m[j]));
+            QT = e2_mul(QT, dj);
+        }
+        ext2 P0 = e2_add(e2_mul(l1[0], l1[3]), e2_mul(l1[1], l1[2]));
+        ext2 Q0 = e2_mul(l1[2], l1[3]);
+        if ((Q0.a == 0 && Q0.b == 0) || !e2_eqv(e2_mul(P0, QT), e2_mul(Q0, PT))) FAIL(REJ_SILU_ROOT, 0, 0);
+    }
+    ext2 mu = e2_squeeze(t, lab->mu);
+    ext2 cP = e2_add(l1[0], e2_mul(mu, e2_sub(l1[1], l1[0])));
+    ext2 cQ = e2_add(l1[2], e2_mul(mu, e2_sub(l1[3], l1[2])));
+    z[0] = mu;
+    for (int d = 1; d < v; d++) {
+        ext2 lam = e2_squeeze(t, lab->lambda);
+        ext2 claim = e2_add(cP, e2_mul(lam, cQ));
+        for (int r = 0; r < d; r++) {
+            ext2 gr[4];
+            e2_read(t, &rd, lab->round, gr, 4);
+            if (rd.bad) FAIL(REJ_FORMAT, 2, d);
+            if (!e2_eqv(e2_add(gr[0], gr[1]), claim)) FAIL(REJ_SILU_ROUND, d, r);
+            rho[r] = e2_squeeze(t, lab->chal);
+            claim = e2_lagrange4(gr, rho[r]);
+        }
+        ext2 fin[4];
+        e2_read(t, &rd, lab->fin, fin, 4);
+        if (rd.bad) FAIL(REJ_FORMAT, 3, d);
+        if (!e2_eqv(e2_mul(e2_eq_closed(z, rho, d), x16_F(fin, lam)), claim)) FAIL(REJ_SILU_FINAL, d, 0);
+        mu = e2_squeeze(t, lab->mu);
+        cP = e2_add(fin[0], e2_mul(mu, e2_sub(fin[1], fin[0])));
+        cQ = e2_add(fin[2], e2_mul(mu, e2_sub(fin[3], fin[2])));
+        for (int r = 0; r < d; r++) z[r] = rho[r];
+        z[d] = mu;
+    }
+    ext2 leaf[2];
+    e2_read(t, &rd, lab->leaf, leaf, 2);
+    if (rd.bad) FAIL(REJ_FORMAT, 4, 0);
+    if (!e2_eqv(cP, e2(1, 0))) FAIL(REJ_SILU_LEAF, 0, 0);
+    if (!e2_eqv(cQ, e2_sub(alpha, e2_add(leaf[0], e2_mul(gamma, leaf[1]))))) FAIL(REJ_SILU_LEAF, 1, 0);
+    {
+        ext2 want[2];
+        x16_leaf_values(g, s, n, v, z, tab(0), want);
+        if (!e2_eqv(want[0], leaf[0])) FAIL(REJ_SILU_OPEN, 0, 0);
+        if (!e2_eqv(want[1], leaf[1])) FAIL(REJ_SILU_OPEN, 1, 0);
+    }
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(m);
+    free(z);
+    free(rho);
+    return rc;
+}
+
+int orc_silu2_prove(void* txh, const int16_t* g, const int16_t* s, u64 n, uint8_t* proof, u64 cap, u64* len) {
+    return lookup16x_prove(txh, &LK_SILU2, orc_silu_q(0), g, s, n, proof, cap, len);
+}
+int orc_silu2_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const uint8_t* proof, u64 len,
+                     int64_t detail[2]) {
+    return lookup16x_verify(txh, &LK_SILU2, orc_silu_q, g, s, n, proof, len, detail);
+}
+int orc_exp2_prove(void* txh, const int16_t* g, const int16_t* s, u64 n, uint8_t* proof, u64 cap, u64* len) {
+    return lookup16x_prove(txh, &LK_EXP2, orc_exp_q(0), g, s, n, proof, cap, len);
+}
+int orc_exp2_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const uint8_t* proof, u64 len,
+                    int64_t detail[2]) {
+    return lookup16x_verify(txh, &LK_EXP2, orc_exp_q, g, s, n, proof, len, detail);
+}

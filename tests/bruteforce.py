@@ -846,3 +846,80 @@ def lhi2_prove(seed: int, r, k: int) -> bytes:
         hr = x_add(hr, x_mul(x_eq(rho, [((x >> (v - 1 - i)) & 1, 0) for i in range(v)]), h[x]))
     send("lhi2_final", [hr, x_mle(f, rho)])
     return bytes(out)
+
+
+def xv_mle(vals, w):
+    """MLE of extension-valued vals (zero-padded to 2^len(w)) at an extension point w."""
+    v = len(w)
+    acc = (0, 0)
+    for x in range(min(len(vals), 1 << v)):
+        acc = x_add(acc, x_mul(x_eq(w, [((x >> (v - 1 - b)) & 1, 0) for b in range(v)]), vals[x]))
+    return acc
+
+
+def lookup16x_prove(seed: int, g, s, prefix: str, pad_s: int) -> bytes:
+    """The 16-bit function lookup over the extension from definitions: the fraction tree by its
+    recurrence in the extension, every layer round value a hypercube sum of eq times the layer
+    summand over MLEs at extension points (no folding)."""
+    g = [int(x) for x in np.asarray(g).reshape(-1)]
+    s = [int(x) for x in np.asarray(s).reshape(-1)]
+    n = len(g)
+    v = max(1, log2c(n))
+    L = 1 << v
+    gp = g + [0] * (L - n)
+    sp = s + [pad_s] * (L - n)
+    out = bytearray()
+    tx = Tx(seed)
+
+    def send(label, xs):
+        b = fe_bytes([c for x in xs for c in x])
+        out.extend(b)
+        tx.absorb(label, b)
+
+    def sq(label):
+        a = tx.squeeze(label)
+        return (a, tx.squeeze(label))
+
+    def neg(x):
+        return ((-x[0]) % P, (-x[1]) % P)
+
+    tx.absorb(prefix + "_site", tree_digest(np.asarray(g, "<i2").tobytes()) + tree_digest(np.asarray(s, "<i2").tobytes()))
+    gamma = sq(prefix + "_gamma")
+    m = np.zeros(1 << 16, np.int64)
+    for x in gp:
+        m[x + 32768] += 1
+    b = m.astype("<u4").tobytes()
+    out.extend(b)
+    tx.absorb(prefix + "_m", tree_digest(b))
+    alpha = sq(prefix + "_alpha")
+    Pl = [[(1, 0)] * L]
+    Ql = [[x_add(alpha, neg(x_add((a % P, 0), x_mul(gamma, (c % P, 0))))) for a, c in zip(gp, sp)]]
+    for _ in range(v):
+        p, q_ = Pl[0], Ql[0]
+        Pl.insert(0, [x_add(x_mul(p[2 * x], q_[2 * x + 1]), x_mul(p[2 * x + 1], q_[2 * x])) for x in range(len(p) // 2)])
+        Ql.insert(0, [x_mul(q_[2 * x], q_[2 * x + 1]) for x in range(len(p) // 2)])
+    send(prefix + "_l1", [Pl[1][0], Pl[1][1], Ql[1][0], Ql[1][1]])
+    z = [sq(prefix + "_mu")]
+    for d in range(1, v):
+        lam = sq(prefix + "_lambda")
+        Pc, Qc = Pl[d + 1], Ql[d + 1]
+        vecs = ([Pc[2 * x] for x in range(1 << d)], [Pc[2 * x + 1] for x in range(1 << d)],
+                [Qc[2 * x] for x in range(1 << d)], [Qc[2 * x + 1] for x in range(1 << d)])
+        rho_l = []
+        for t in range(d):
+            gr = []
+            for X in range(4):
+                acc = (0, 0)
+                rest = d - t - 1
+                for bb in range(1 << rest):
+                    pt = rho_l + [(X, 0)] + [((bb >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                    pL, pR, qL, qR = (xv_mle(vv, pt) for vv in vecs)
+                    Fv = x_add(x_add(x_mul(pL, qR), x_mul(pR, qL)), x_mul(lam, x_mul(qL, qR)))
+                    acc = x_add(acc, x_mul(x_eq(z, pt), Fv))
+                gr.append(acc)
+            send(prefix + "_round", gr)
+            rho_l.append(sq(prefix + "_chal"))
+        send(prefix + "_final", [xv_mle(vv, rho_l) for vv in vecs])
+        z = rho_l + [sq(prefix + "_mu")]
+    send(prefix + "_leaf", [x_mle(gp, z), x_mle(sp, z)])
+    return bytes(out)

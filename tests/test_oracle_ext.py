@@ -156,3 +156,37 @@ def test_lhi2_accepts_and_names_tampering():
     # the base-field proof of the same keys is another proof
     base, _ = oracle.lhi_prove(6, r, k)
     assert oracle.lhi2_verify(6, r, k, base)[0] != "accept"
+
+
+# ---- the 16-bit function lookups (LogUp-GKR tree) over the extension -----------------------
+
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 8])
+def test_silu2_bytes_match_bruteforce(n):
+    rng = np.random.default_rng(n + 70)
+    g = rng.integers(-32768, 32768, n).astype(np.int16)
+    s = np.array([oracle.silu_q(int(x)) for x in g], np.int16)
+    pf, _ = oracle.silu2_prove(5, g, s)
+    assert pf == bf.lookup16x_prove(5, g, s, "silu2", oracle.silu_q(0))
+
+
+def test_exp2_bytes_match_bruteforce():
+    g = np.array([-5, 0, -300, -1800, 7], np.int16)
+    s = np.array([oracle.exp_q(int(x)) for x in g], np.int16)
+    pf, _ = oracle.exp2_prove(6, g, s)
+    assert pf == bf.lookup16x_prove(6, g, s, "exp2", oracle.exp_q(0))
+
+
+def test_lookup16_over_extension_accepts_and_rejects():
+    rng = np.random.default_rng(71)
+    g = rng.integers(-32768, 32768, 3000).astype(np.int16)
+    s = np.array([oracle.silu_q(int(x)) for x in g], np.int16)
+    pf, _ = oracle.silu2_prove(8, g, s)
+    assert oracle.silu2_verify(8, g, s, pf) == ("accept", (0, 0))
+    bad = s.copy()
+    bad[100] += 1  # an output the table does not hold
+    pf2, _ = oracle.silu2_prove(8, g, bad)
+    assert oracle.silu2_verify(8, g, bad, pf2)[0] == "lookup_root"
+    # the base-field proof and the exponent table's proof are other statements
+    base, _ = oracle.silu_prove(8, g, s)
+    assert oracle.silu2_verify(8, g, s, base)[0] != "accept"
+    assert oracle.exp2_verify(8, g, s, pf)[0] != "accept"
