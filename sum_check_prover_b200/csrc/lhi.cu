@@ -28,6 +28,12 @@
 // The host half (lhi_protocol) takes its device values from a source: the
 // kernels here, or a caller's callback (fp_lhi_protocol_drive), so the transcript
 // order and the round polynomials can be checked without a GPU.
+//
+// The same statement over the quadratic extension ("How fast can FlashProve go",
+// 4, the note on soundness) follows the base-field kernels with 16-byte vectors
+// (lhi2_*, logup_prove_helper_inverse_ext2); fp_lhi_run is the base-field
+// statement from "lhi_site" on, for callers (the MoE routing proof) that reserve
+// the arenas themselves.
 #include <string.h>
 
 #include <algorithm>
