@@ -484,6 +484,40 @@ int fp_lhi2_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uin
 int fp_lhi_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uint8_t* m_digest, fp_values_fn fn,
                           void* user, uint8_t* proof, size_t* proof_len);
 
+/*
+ * The SiLU and softmax numerator lookups over the quadratic extension
+ * F_p[phi]/(phi^2 - 7) ("How fast can FlashProve go", 4, the note on soundness:
+ * challenges from an extension field): the statements of logup_prove_silu and
+ * logup_prove_exp with gamma, alpha, mu, lambda, every round challenge and every
+ * value sent an extension element (16 bytes: a then b), the tree's fractions in
+ * the extension, and the labels "silu2_*" / "exp2_*" (site, gamma, m, alpha, l1,
+ * mu, lambda, round, chal, final, leaf). Proof bytes: 4 * 2^16 + 64 + 32 +
+ * sum_{d=1}^{v-1} (64 d + 64). Same arguments and errors as logup_prove_silu.
+ */
+int logup_prove_silu_ext2(fp_ctx* ctx, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
+                          size_t* proof_len, void* stream);
+int logup_prove_exp_ext2(fp_ctx* ctx, fp_tx* tx, const int16_t* g, const int16_t* s, int64_t n, uint8_t* proof,
+                         size_t* proof_len, void* stream);
+
+/*
+ * The host half of logup_prove_silu_ext2 (table 0) or logup_prove_exp_ext2
+ * (table 1) from the multiplicities on, v >= 1 variables: gamma (2 words, squeezed
+ * by the caller after the site), m (host, 2^16 u32) and m_digest (32 bytes) are
+ * given. Callback kinds:
+ *   FP_VAL_COLUMN: in = gamma, alpha (4 words); out = layer one's P(0), P(1), Q(0),
+ *     Q(1) (8 words);
+ *   FP_VAL_START: layer d begins; in = z_1..z_d, lambda (2 d + 2 words), t = d;
+ *   FP_VAL_ROUND: out = h_t(0), h_t(1), h_t(2) of the current layer (6 words);
+ *   FP_VAL_ANSWER: in = rho_t (2 words);
+ *   FP_VAL_FINALS: out = pL, pR, qL, qR at rho (8 words);
+ *   FP_VAL_CLAIM: in = the leaf point z_1..z_v (2 v words), t = v; out = g~(z), s~(z)
+ *     of the padded columns (4 words).
+ * The proof and proof_len are as for logup_prove_silu_ext2 with 2^v keys.
+ */
+int fp_lookup16x_protocol_drive(fp_tx* tx, int table, int v, const uint64_t* gamma, const uint32_t* m,
+                                const uint8_t* m_digest, fp_values_fn fn, void* user, uint8_t* proof,
+                                size_t* proof_len);
+
 /* The SiLU table's 2^16 entries silu_q(v), v = -2^15 .. 2^15 - 1, into host out (no GPU work). */
 int fp_silu_table(int32_t* out);
 

@@ -16,7 +16,7 @@ from typing import Optional, Sequence
 
 __all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P",
            "had2_protocol_drive", "lhi_protocol_drive", "mm2_protocol_drive", "route_protocol_drive",
-           "lhi2_protocol_drive"]
+           "lhi2_protocol_drive", "lookup16x_protocol_drive"]
 
 P = 0xFFFFFFFF00000001
 LIB_PATH = Path(__file__).resolve().with_name("libfp.so")
@@ -82,6 +82,9 @@ def lib():
     L.freivalds_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), vp, C.POINTER(sz), vp]
     L.sumcheck_prove_routing.argtypes = [vp, vp, vp, C.c_int64, i32, vp, vp, vp, C.POINTER(sz), vp]
     L.fp_route_protocol_drive.argtypes = [vp, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
+    L.logup_prove_silu_ext2.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
+    L.logup_prove_exp_ext2.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
+    L.fp_lookup16x_protocol_drive.argtypes = [vp, i32, i32, C.POINTER(u64), vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.logup_prove_helper_inverse_ext2.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
     L.fp_lhi2_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.fp_mm2_protocol_drive.argtypes = [vp, i32, i32, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
@@ -219,6 +222,59 @@ def route_protocol_drive(tx: "Transcript", n: int, values) -> bytes:
     rc = L.fp_route_protocol_drive(tx.h, n, fn, None, buf, C.byref(ln))
     if rc != 0:
         raise FpError(rc, "fp_route_protocol_drive failed")
+    return buf.raw[: ln.value]
+
+
+def lookup16x_protocol_drive(tx: "Transcript", table: int, v: int, gamma, m, m_digest: bytes, values) -> bytes:
+    """Run the host half of the extension-field 16-bit lookup (table 0: SiLU, 1: exponent) from
+    the multiplicities on, with its device values taken from `values` (no GPU work):
+    values.tree(gamma, alpha) -> layer one's (P0, P1, Q0, Q1), values.layer(d, z, lam),
+    values.round(t) -> (h(0), h(1), h(2)), values.answer(t, rho), values.finals() -> (pL, pR,
+    qL, qR), values.leaf(z) -> (g~(z), s~(z)); extension elements are pairs (a, b). gamma is the
+    pair squeezed after the site."""
+    import numpy as np
+
+    L = lib()
+
+    def pairs(inp, k):
+        return [(int(inp[2 * i]), int(inp[2 * i + 1])) for i in range(k)]
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            res = None
+            if kind == VAL_COLUMN:
+                ga = pairs(inp, 2)
+                res = values.tree(ga[0], ga[1])
+            elif kind == VAL_START:
+                pts = pairs(inp, t + 1)
+                values.layer(t, pts[:t], pts[t])
+            elif kind == VAL_ANSWER:
+                values.answer(t, (int(inp[0]), int(inp[1])))
+            elif kind == VAL_ROUND:
+                res = values.round(t)
+            elif kind == VAL_FINALS:
+                res = values.finals()
+            elif kind == VAL_CLAIM:
+                res = values.leaf(pairs(inp, t))
+            else:
+                return 1
+            for i, (a, b) in enumerate(res or []):
+                out[2 * i] = int(a)
+                out[2 * i + 1] = int(b)
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _VALUES_FN(cb)
+    mm = np.ascontiguousarray(np.asarray(m, dtype="<u4"))
+    md = C.create_string_buffer(bytes(m_digest), 32)
+    gm = (C.c_uint64 * 2)(int(gamma[0]), int(gamma[1]))
+    cap = 4 * 65536 + 64 + 32 + sum(64 * d + 64 for d in range(1, v))
+    buf = C.create_string_buffer(cap)
+    ln = C.c_size_t(cap)
+    rc = L.fp_lookup16x_protocol_drive(tx.h, table, v, gm, mm.ctypes.data, md, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_lookup16x_protocol_drive failed")
     return buf.raw[: ln.value]
 
 
@@ -589,7 +645,15 @@ class Context:
         """As prove_silu, for the softmax numerator table."""
         return self._lookup16(self._L.logup_prove_exp, "prove_exp", tx, g, s, stream)
 
-    def _lookup16(self, fn, what, tx, g, s, stream):
+    def prove_silu_ext2(self, tx: Transcript, g, s, stream=None) -> bytes:
+        """As prove_silu with every challenge and value in the quadratic extension."""
+        return self._lookup16(self._L.logup_prove_silu_ext2, "prove_silu_ext2", tx, g, s, stream, ext=True)
+
+    def prove_exp_ext2(self, tx: Transcript, g, s, stream=None) -> bytes:
+        """As prove_exp with every challenge and value in the quadratic extension."""
+        return self._lookup16(self._L.logup_prove_exp_ext2, "prove_exp_ext2", tx, g, s, stream, ext=True)
+
+    def _lookup16(self, fn, what, tx, g, s, stream, ext=False):
         n = int(g.numel())
         if int(s.numel()) != n:
             raise ValueError(f"{what}: g and s differ in size")
@@ -597,7 +661,8 @@ class Context:
         while (1 << v) < n:
             v += 1
         v = max(v, 1)
-        cap = 4 * 65536 + 32 + 16 + sum(32 * d + 32 for d in range(1, v))
+        w = 2 if ext else 1  # words per value
+        cap = 4 * 65536 + w * (32 + 16) + sum(w * (32 * d + 32) for d in range(1, v))
         buf = C.create_string_buffer(cap)
         ln = C.c_size_t(cap)
         self._check(fn(self.h, tx.h, _ptr(g), _ptr(s), n, buf, C.byref(ln), _stream(stream)), what)

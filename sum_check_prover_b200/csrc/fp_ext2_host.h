@@ -6,14 +6,17 @@
 #include "fp_ext2.cuh"
 #include "fp_internal.h"
 
-inline Ext2 e2_squeeze_host(fp_tx* tx, const char* label) {
+// a + r (b - a): a pair folded by an extension challenge
+static inline Ext2 e2_fold_host(Ext2 a, Ext2 b, Ext2 r) { return e2_add(a, e2_mul(r, e2_sub(b, a))); }
+
+static inline Ext2 e2_squeeze_host(fp_tx* tx, const char* label) {
     const uint64_t a = fp_tx_squeeze_one(tx, label);
     const uint64_t b = fp_tx_squeeze_one(tx, label);
     return e2_make(a, b);
 }
 
 // n <= 4 extension elements into the proof at pos, absorbed under one label
-inline void e2_send_host(fp_tx* tx, const char* label, const Ext2* v, int n, uint8_t* proof, size_t& pos) {
+static inline void e2_send_host(fp_tx* tx, const char* label, const Ext2* v, int n, uint8_t* proof, size_t& pos) {
     uint64_t w[8];
     for (int i = 0; i < n; i++) {
         w[2 * i] = v[i].a;
@@ -26,7 +29,7 @@ inline void e2_send_host(fp_tx* tx, const char* label, const Ext2* v, int n, uin
 
 // the degree-2 polynomial through (i, g[i]), i = 0..2, at r:
 // L0 = (r-1)(r-2)/2, L1 = -r(r-2), L2 = r(r-1)/2
-inline Ext2 e2_lagrange3(const Ext2 g[3], Ext2 r) {
+static inline Ext2 e2_lagrange3(const Ext2 g[3], Ext2 r) {
     static const uint64_t inv2 = gl_inv(2);
     const Ext2 r1 = e2_sub(r, e2_make(1, 0)), r2 = e2_sub(r, e2_make(2, 0));
     const Ext2 l0 = e2_scal(e2_mul(r1, r2), inv2);
@@ -37,7 +40,7 @@ inline Ext2 e2_lagrange3(const Ext2 g[3], Ext2 r) {
 
 // the degree-3 polynomial through (i, g[i]), i = 0..3, at r:
 // L0 = -(r-1)(r-2)(r-3)/6, L1 = r(r-2)(r-3)/2, L2 = -r(r-1)(r-3)/2, L3 = r(r-1)(r-2)/6
-inline Ext2 e2_lagrange4(const Ext2 g[4], Ext2 r) {
+static inline Ext2 e2_lagrange4(const Ext2 g[4], Ext2 r) {
     static const uint64_t inv2 = gl_inv(2), inv6 = gl_inv(6);
     const Ext2 r1 = e2_sub(r, e2_make(1, 0)), r2 = e2_sub(r, e2_make(2, 0)), r3 = e2_sub(r, e2_make(3, 0));
     const Ext2 zero = e2_make(0, 0);

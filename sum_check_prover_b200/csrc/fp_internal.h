@@ -59,6 +59,9 @@ enum FpKernel {
     K_LHI2_COLUMN,
     K_LHI2_ROUND,
     K_LHI2_FINAL,
+    K_X16_TREE,
+    K_X16_ROUND,
+    K_X16_LEAF,
     K_COUNT
 };
 

@@ -345,3 +345,94 @@ def test_lhi2_inconsistent_round_is_refused(fp, t):
     r = np.random.default_rng(8).integers(-8, 8, 8).astype(np.int32)
     with pytest.raises(fp.FpError):
         _lhi2_drive(fp, 1, r, 4, BruteLhi2(r, 4, tamper=t))
+
+
+# ---- the 16-bit function lookups (LogUp-GKR tree) over the extension ----------------------
+
+class BruteLookup16x:
+    """Device values of the extension-field 16-bit lookup by their definitions: the tree by
+    its recurrence, every round value a hypercube sum over MLEs at extension points."""
+
+    def __init__(self, g, s, pad_s, tamper=None):
+        self.g = [int(x) for x in g]
+        self.s = [int(x) for x in s]
+        n = len(self.g)
+        self.v = max(1, bf.log2c(n))
+        L = 1 << self.v
+        self.gp = self.g + [0] * (L - n)
+        self.sp = self.s + [pad_s] * (L - n)
+        self.tamper = tamper
+
+    def tree(self, gamma, alpha):
+        neg = lambda x: ((-x[0]) % P, (-x[1]) % P)  # noqa: E731
+        L = 1 << self.v
+        Pl = [[(1, 0)] * L]
+        Ql = [[bf.x_add(alpha, neg(bf.x_add((a % P, 0), bf.x_mul(gamma, (c % P, 0))))) for a, c in zip(self.gp, self.sp)]]
+        for _ in range(self.v):
+            p, q_ = Pl[0], Ql[0]
+            Pl.insert(0, [bf.x_add(bf.x_mul(p[2 * x], q_[2 * x + 1]), bf.x_mul(p[2 * x + 1], q_[2 * x]))
+                          for x in range(len(p) // 2)])
+            Ql.insert(0, [bf.x_mul(q_[2 * x], q_[2 * x + 1]) for x in range(len(p) // 2)])
+        self.Pl, self.Ql = Pl, Ql
+        return [Pl[1][0], Pl[1][1], Ql[1][0], Ql[1][1]]
+
+    def layer(self, d, z, lam):
+        self.d, self.z, self.lam, self.rho = d, z, lam, []
+        Pc, Qc = self.Pl[d + 1], self.Ql[d + 1]
+        n2 = 1 << d
+        self.vecs = ([Pc[2 * x] for x in range(n2)], [Pc[2 * x + 1] for x in range(n2)],
+                     [Qc[2 * x] for x in range(n2)], [Qc[2 * x + 1] for x in range(n2)])
+
+    def round(self, t):
+        rest = self.d - t
+        h = []
+        for X in range(3):
+            acc = (0, 0)
+            for b in range(1 << rest):
+                bits = [((b >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                pt = self.rho + [(X, 0)] + bits
+                pL, pR, qL, qR = (bf.xv_mle(vv, pt) for vv in self.vecs)
+                F = bf.x_add(bf.x_add(bf.x_mul(pL, qR), bf.x_mul(pR, qL)), bf.x_mul(self.lam, bf.x_mul(qL, qR)))
+                acc = bf.x_add(acc, bf.x_mul(bf.x_eq(self.z[t:self.d], bits), F))
+            h.append(acc)
+        if self.tamper == (self.d, t):
+            h[0] = ((h[0][0] + 1) % P, h[0][1])
+        return h
+
+    def answer(self, t, rho):
+        self.rho.append(rho)
+
+    def finals(self):
+        return [bf.xv_mle(vv, self.rho) for vv in self.vecs]
+
+    def leaf(self, z):
+        return [bf.x_mle(self.gp, z), bf.x_mle(self.sp, z)]
+
+
+def _lk_drive(fp, seed, g, s, table, vals):
+    prefix = "silu2" if table == 0 else "exp2"
+    tx = fp.Transcript(seed)
+    tx.absorb(prefix + "_site", bf.tree_digest(np.asarray(g, "<i2").tobytes()) + bf.tree_digest(np.asarray(s, "<i2").tobytes()))
+    gamma = (tx.squeeze(prefix + "_gamma")[0], tx.squeeze(prefix + "_gamma")[0])
+    m = np.zeros(1 << 16, np.int64)
+    for x in vals.gp:
+        m[x + 32768] += 1
+    m = m.astype("<u4")
+    return fp.lookup16x_protocol_drive(tx, table, vals.v, gamma, m, bf.tree_digest(m.tobytes()), vals), tx.state()
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 8])
+def test_lookup16x_host_half_matches_oracle(fp, n):
+    rng = np.random.default_rng(n + 90)
+    g = rng.integers(-32768, 32768, n).astype(np.int16)
+    s = np.array([oracle.silu_q(int(x)) for x in g], np.int16)
+    vals = BruteLookup16x(g, s, oracle.silu_q(0))
+    assert _lk_drive(fp, 4, g, s, 0, vals) == oracle.silu2_prove(4, g, s)
+
+
+def test_lookup16x_exp_table_and_refusal(fp):
+    g = np.array([-5, 0, -300, -1800, 7], np.int16)
+    s = np.array([oracle.exp_q(int(x)) for x in g], np.int16)
+    assert _lk_drive(fp, 6, g, s, 1, BruteLookup16x(g, s, oracle.exp_q(0))) == oracle.exp2_prove(6, g, s)
+    with pytest.raises(fp.FpError):
+        _lk_drive(fp, 6, g, s, 1, BruteLookup16x(g, s, oracle.exp_q(0), tamper=(2, 2)))
