@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2"
+MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2,silu2"
 
 
 def micro_names(which) -> set:
@@ -212,6 +212,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
       (the activation once, plus the powers of rho).
     lhi2_round: the helper-inverse LogUp's rounds over 2^26 keys with extension challenges
       (16-byte vectors: 176 B per pair in round 2, 240 B later).
+    silu2_round: the SiLU lookup's layer rounds over 2^26 keys with extension challenges
+      (16-byte vectors: 160 and 320 B per pair).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
@@ -385,6 +387,19 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
             del rv
         except Exception as e:  # a failure here must not cost the rest of the line
             out["helper_inverse_ext2_round_2^26_keys"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    if "silu2" in which:
+        # the SiLU lookup of 2^26 gate values with extension-field challenges
+        try:
+            np_ = __import__("numpy")
+            rng = np_.random.default_rng(11)
+            tab = fp.silu_table().astype(np_.int16)
+            gv = rng.integers(-32768, 32768, 1 << 26).astype(np_.int16)
+            gd = torch.from_numpy(gv).to(dev)
+            sd = torch.from_numpy(tab[gv.astype(np_.int64) + 32768]).to(dev)
+            measure("silu_ext2_lookup_round_2^26", "silu2_round", lambda: ctx.prove_silu_ext2(fp.Transcript(6), gd, sd))
+            del gd, sd
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["silu_ext2_lookup_round_2^26"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     try:
         torch.cuda.empty_cache()
