@@ -218,7 +218,7 @@ struct Had2Source {
 
 // The protocol after "had2_site" is absorbed: proof of 16 + 64 v + 32 bytes.
 int had2_protocol(fp_ctx* c, fp_tx* tx, int v, Had2Source& src, uint8_t* proof, size_t* proof_len) {
-    Ext2 z[H2_MAX_V];
+    Ext2 z[H2_MAX_V] = {};
     for (int i = 0; i < v; i++) z[i] = e2_squeeze_host(tx, "had2_z");
     int rc;
     if ((rc = src.start(z, v))) return rc;

@@ -212,7 +212,7 @@ constexpr int M2_MAX_V = 32;
 
 // The protocol after "mm2_site" is absorbed: proof of 16 + 48 n + 32 bytes.
 int mm2_protocol(fp_ctx* c, fp_tx* tx, int vM, int vN, int n, Mm2Source& src, uint8_t* proof, size_t* proof_len) {
-    Ext2 zr[M2_MAX_V], zc[M2_MAX_V];
+    Ext2 zr[M2_MAX_V] = {}, zc[M2_MAX_V] = {};
     for (int i = 0; i < vM; i++) zr[i] = e2_squeeze_host(tx, "mm2_row");
     for (int i = 0; i < vN; i++) zc[i] = e2_squeeze_host(tx, "mm2_col");
     int rc;

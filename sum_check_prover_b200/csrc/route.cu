@@ -215,7 +215,7 @@ struct RouteSource {
 
 // The routing sum-check after "route_site" is absorbed: 16 + 32 n + 16 proof bytes.
 int route_protocol(fp_ctx* c, fp_tx* tx, int n, RouteSource& src, uint8_t* proof, size_t* proof_len) {
-    uint64_t z[RT_MAX_N], w[RT_MAX_N];
+    uint64_t z[RT_MAX_N] = {}, w[RT_MAX_N] = {};
     for (int i = 0; i < n; i++) z[i] = fp_tx_squeeze_one(tx, "route_z");
     for (int i = 0; i < n; i++) w[i] = fp_tx_squeeze_one(tx, "route_w");
     const uint64_t lam1 = fp_tx_squeeze_one(tx, "route_lambda");
