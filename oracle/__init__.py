@@ -177,6 +177,10 @@ def lib():
             getattr(L, nm).argtypes = [vp, vp, u64, C.c_int, vp, u64, C.POINTER(u64)]
         L.orc_lhi2_verify.restype = C.c_int
         L.orc_lhi2_verify.argtypes = [vp, vp, u64, C.c_int, vp, u64, vp]
+        L.orc_lu2_prove.restype = C.c_int
+        L.orc_lu2_prove.argtypes = [vp, vp, C.c_int, vp, vp, u64, C.POINTER(u64)]
+        L.orc_lu2_verify.restype = C.c_int
+        L.orc_lu2_verify.argtypes = [vp, vp, C.c_int, vp, vp, u64, vp]
         L.orc_route_witness.restype = None
         L.orc_route_witness.argtypes = [vp, u64, C.c_int, vp, vp]
         L.orc_route_prove.restype = C.c_int
@@ -801,5 +805,40 @@ def route_verify(seed: int, l, H, D, T: int, E: int, proof: bytes):
     det = np.zeros(2, dtype=np.int64)
     tx = L.orc_tx_new(seed)
     rc = L.orc_route_verify(tx, _ptr(a), _ptr(h), _ptr(d), T, E, _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+# ---- the rescale LogUp over the extension -------------------------------------------
+
+def lu2_prove(seed: int, sites, wits):
+    """The two-table rescale LogUp of the sites' key columns with every challenge and value in
+    the quadratic extension; returns (proof bytes, transcript state)."""
+    L = lib()
+    keep = []
+    cs, cw = _marshal(sites, wits, keep)
+    n = C.c_uint64(0)
+    tx = L.orc_tx_new(seed)
+    L.orc_lu2_prove(tx, cs, len(sites), cw, None, 0, C.byref(n))
+    L.orc_tx_free(tx)
+    buf = np.zeros(max(1, n.value), dtype=np.uint8)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_lu2_prove(tx, cs, len(sites), cw, _ptr(buf), n.value, C.byref(n))
+    st = C.create_string_buffer(32)
+    L.orc_tx_state(tx, st)
+    L.orc_tx_free(tx)
+    if rc != 0:
+        raise ValueError(f"orc_lu2_prove failed ({rc})")
+    return buf[: n.value].tobytes(), st.raw
+
+
+def lu2_verify(seed: int, sites, wits, proof: bytes):
+    L = lib()
+    keep = []
+    cs, cw = _marshal(sites, wits, keep)
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_lu2_verify(tx, cs, len(sites), cw, _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

@@ -3089,3 +3089,277 @@ int orc_exp2_verify(void* txh, const int16_t* g, const int16_t* s, u64 n, const 
                     int64_t detail[2]) {
     return lookup16x_verify(txh, &LK_EXP2, orc_exp_q, g, s, n, proof, len, detail);
 }
+
+/* ------------------------------------------------------------------------ */
+/* The rescale LogUp (the two tables of lu_prove, batched in one GKR) over   */
+/* the extension (next row f4, "How fast can FlashProve go", 4, the note on  */
+/* soundness), as a statement of its own over the sites' key columns:       */
+/*   absorb "lu2_site" D(r) || D(q) (int32 little-endian) || D(y) of the     */
+/*   concatenated, unpadded key columns; send m_rem ("lu2_m_rem"); squeeze    */
+/*   gamma ("lu2_gamma"); send m_clamp ("lu2_m_clamp"); squeeze alpha_0,      */
+/*   alpha_1 ("lu2_alpha"); then lu_prove's layers with every challenge and   */
+/*   value in F_p[phi]/(phi^2 - 7): "lu2_l1" (8 values), "lu2_mu",            */
+/*   "lu2_lambda", "lu2_round", "lu2_chal", "lu2_final" (8 values), and the  */
+/*   leaf claims r~(z), q~(z), y~(z) ("lu2_leaf").                            */
+/* ------------------------------------------------------------------------ */
+
+static void lu2_absorb_site(orc_tx* t, const orc_keys* K) {
+    u64 nk = K->nk;
+    uint8_t* b = (uint8_t*)calloc(4 * nk + 1, 1);
+    uint8_t d[96];
+    for (u64 i = 0; i < nk; i++) put_le(b + 4 * i, (u64)(u32)(int32_t)K->fr[i], 4);
+    orc_tree_digest(b, 4 * nk, d);
+    for (u64 i = 0; i < nk; i++) put_le(b + 4 * i, (u64)(u32)(int32_t)K->fq[i], 4);
+    orc_tree_digest(b, 4 * nk, d + 32);
+    for (u64 i = 0; i < nk; i++) b[i] = (uint8_t)(int8_t)K->fy[i];
+    orc_tree_digest(b, nk, d + 64);
+    free(b);
+    orc_tx_absorb(t, "lu2_site", d, 96);
+}
+
+static ext2 lu2_key(const orc_keys* K, int tab, u64 i, ext2 gamma) {
+    if (tab == 0) return e2(orc_fint(K->fr[i]), 0);
+    return e2_add(e2(orc_fint(K->fq[i]), 0), e2_scal(gamma, orc_fint(K->fy[i])));
+}
+
+/* layer summand: sum over tables tau of lambda^(2 tau) (pL qR + pR qL + lambda qL qR) */
+static ext2 lu2_F(const ext2 v8[8], ext2 lam, ext2 lam2) {
+    ext2 acc = e2(0, 0), w = e2(1, 0);
+    for (int tau = 0; tau < 2; tau++) {
+        const ext2* x = v8 + 4 * tau;
+        ext2 f = e2_add(e2_add(e2_mul(x[0], x[3]), e2_mul(x[1], x[2])), e2_mul(lam, e2_mul(x[2], x[3])));
+        acc = e2_add(acc, e2_mul(w, f));
+        w = lam2;
+    }
+    return acc;
+}
+
+static ext2 lu2_fold(ext2 a, ext2 b, ext2 r) { return e2_add(a, e2_mul(r, e2_sub(b, a))); }
+
+int orc_lu2_prove(void* txh, const orc_site* sites, int ns, const orc_wit* wit, uint8_t* proof, u64 cap, u64* len) {
+    orc_tx* t = (orc_tx*)txh;
+    orc_keys K;
+    if (ns < 1 || keys_build(sites, ns, wit, &K) != 0) return -1;
+    pbuf pb = {proof, cap, 0, 0};
+    int v = K.v;
+    u64 L = (u64)1 << v, Trem = (u64)1 << K.k;
+    lu2_absorb_site(t, &K);
+    u32* mr = (u32*)malloc(Trem * sizeof(u32));
+    u32* mc = (u32*)malloc(65536 * sizeof(u32));
+    mult_rem(&K, mr);
+    send_mult(t, &pb, "lu2_m_rem", mr, Trem);
+    ext2 gamma = e2_squeeze(t, "lu2_gamma");
+    mult_clamp(&K, mc);
+    send_mult(t, &pb, "lu2_m_clamp", mc, 65536);
+    ext2 alpha[2];
+    alpha[0] = e2_squeeze(t, "lu2_alpha");
+    alpha[1] = e2_squeeze(t, "lu2_alpha");
+    /* the two fraction trees: layer d has 2^d nodes */
+    ext2** P[2];
+    ext2** Q[2];
+    for (int tau = 0; tau < 2; tau++) {
+        P[tau] = (ext2**)malloc(sizeof(ext2*) * (v + 1));
+        Q[tau] = (ext2**)malloc(sizeof(ext2*) * (v + 1));
+        P[tau][v] = (ext2*)malloc(L * sizeof(ext2));
+        Q[tau][v] = (ext2*)malloc(L * sizeof(ext2));
+        for (u64 i = 0; i < L; i++) {
+            P[tau][v][i] = e2(1, 0);
+            Q[tau][v][i] = e2_sub(alpha[tau], lu2_key(&K, tau, i, gamma));
+        }
+        for (int d = v - 1; d >= 0; d--) {
+            u64 c = (u64)1 << d;
+            P[tau][d] = (ext2*)malloc(c * sizeof(ext2));
+            Q[tau][d] = (ext2*)malloc(c * sizeof(ext2));
+            for (u64 x = 0; x < c; x++) {
+                ext2 pl = P[tau][d + 1][2 * x], pr = P[tau][d + 1][2 * x + 1];
+                ext2 ql = Q[tau][d + 1][2 * x], qr = Q[tau][d + 1][2 * x + 1];
+                P[tau][d][x] = e2_add(e2_mul(pl, qr), e2_mul(pr, ql));
+                Q[tau][d][x] = e2_mul(ql, qr);
+            }
+        }
+    }
+    ext2 l1[8];
+    for (int tau = 0; tau < 2; tau++) {
+        l1[4 * tau + 0] = P[tau][1][0];
+        l1[4 * tau + 1] = P[tau][1][1];
+        l1[4 * tau + 2] = Q[tau][1][0];
+        l1[4 * tau + 3] = Q[tau][1][1];
+    }
+    e2_send(t, &pb, "lu2_l1", l1, 8);
+    ext2* z = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    z[0] = e2_squeeze(t, "lu2_mu");
+    for (int d = 1; d < v; d++) {
+        ext2 lam = e2_squeeze(t, "lu2_lambda");
+        ext2 lam2 = e2_mul(lam, lam);
+        u64 c = (u64)1 << d;
+        ext2* V[9];
+        for (int i = 0; i < 9; i++) V[i] = (ext2*)malloc(c * sizeof(ext2));
+        for (int tau = 0; tau < 2; tau++)
+            for (u64 x = 0; x < c; x++) {
+                V[4 * tau + 0][x] = P[tau][d + 1][2 * x];
+                V[4 * tau + 1][x] = P[tau][d + 1][2 * x + 1];
+                V[4 * tau + 2][x] = Q[tau][d + 1][2 * x];
+                V[4 * tau + 3][x] = Q[tau][d + 1][2 * x + 1];
+            }
+        e2_eq_table(z, d, V[8]);
+        ext2* rho = (ext2*)malloc(sizeof(ext2) * d);
+        u64 Lr = c;
+        for (int r = 0; r < d; r++) {
+            u64 h = Lr >> 1;
+            ext2 g[4] = {e2(0, 0), e2(0, 0), e2(0, 0), e2(0, 0)};
+            for (u64 b = 0; b < h; b++)
+                for (u64 X = 0; X < 4; X++) {
+                    ext2 ev[9];
+                    for (int i = 0; i < 9; i++) ev[i] = e2_add(V[i][b], e2_scal(e2_sub(V[i][h + b], V[i][b]), X));
+                    g[X] = e2_add(g[X], e2_mul(ev[8], lu2_F(ev, lam, lam2)));
+                }
+            e2_send(t, &pb, "lu2_round", g, 4);
+            rho[r] = e2_squeeze(t, "lu2_chal");
+            for (int i = 0; i < 9; i++)
+                for (u64 b = 0; b < h; b++) V[i][b] = lu2_fold(V[i][b], V[i][h + b], rho[r]);
+            Lr = h;
+        }
+        ext2 fin[8];
+        for (int i = 0; i < 8; i++) fin[i] = V[i][0];
+        e2_send(t, &pb, "lu2_final", fin, 8);
+        ext2 mu = e2_squeeze(t, "lu2_mu");
+        for (int r = 0; r < d; r++) z[r] = rho[r];
+        z[d] = mu;
+        for (int i = 0; i < 9; i++) free(V[i]);
+        free(rho);
+    }
+    {
+        u64* col = (u64*)malloc(L * sizeof(u64));
+        ext2 leaf[3];
+        for (u64 i = 0; i < L; i++) col[i] = orc_fint(K.fr[i]);
+        leaf[0] = x16_mle(col, L, z, v);
+        for (u64 i = 0; i < L; i++) col[i] = orc_fint(K.fq[i]);
+        leaf[1] = x16_mle(col, L, z, v);
+        for (u64 i = 0; i < L; i++) col[i] = orc_fint(K.fy[i]);
+        leaf[2] = x16_mle(col, L, z, v);
+        e2_send(t, &pb, "lu2_leaf", leaf, 3);
+        free(col);
+    }
+    for (int tau = 0; tau < 2; tau++) {
+        for (int d = 0; d <= v; d++) {
+            free(P[tau][d]);
+            free(Q[tau][d]);
+        }
+        free(P[tau]);
+        free(Q[tau]);
+    }
+    free(z);
+    free(mr);
+    free(mc);
+    keys_free(&K);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+/* the table side sum_j m_j / (alpha - t_j) as one extension fraction */
+static void lu2_table(const u32* m, u64 T, int tab, int k, ext2 alpha, ext2 gamma, ext2* num, ext2* den) {
+    ext2 Pn = e2(0, 0), Qd = e2(1, 0);
+    for (u64 j = 0; j < T; j++) {
+        ext2 tj;
+        if (tab == 0) {
+            tj = e2(orc_fint((int64_t)j - ((int64_t)1 << (k - 1))), 0);
+        } else {
+            int64_t vj = (int64_t)j - 32768;
+            int64_t cj = vj < -128 ? -128 : (vj > 127 ? 127 : vj);
+            tj = e2_add(e2(orc_fint(vj), 0), e2_scal(gamma, orc_fint(cj)));
+        }
+        ext2 d = e2_sub(alpha, tj);
+        Pn = e2_add(e2_mul(Pn, d), e2_scal(Qd, (u64)m[j]));
+        Qd = e2_mul(Qd, d);
+    }
+    *num = Pn;
+    *den = Qd;
+}
+
+int orc_lu2_verify(void* txh, const orc_site* sites, int ns, const orc_wit* wit, const uint8_t* proof, u64 len,
+                   int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    orc_tx* t = (orc_tx*)txh;
+    orc_keys K;
+    if (ns < 1 || keys_build(sites, ns, wit, &K) != 0) return REJ_ARGS;
+    int rc = 0, v = K.v;
+    u64 L = (u64)1 << v, Trem = (u64)1 << K.k;
+    prd rd = {proof, len, 0, 0};
+    u32* mr = (u32*)malloc(Trem * sizeof(u32));
+    u32* mc = (u32*)malloc(65536 * sizeof(u32));
+    ext2* z = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    ext2* rho = (ext2*)malloc(sizeof(ext2) * (v + 1));
+    u64* col = NULL;
+    lu2_absorb_site(t, &K);
+    rd_mult(t, &rd, "lu2_m_rem", mr, Trem);
+    ext2 gamma = e2_squeeze(t, "lu2_gamma");
+    rd_mult(t, &rd, "lu2_m_clamp", mc, 65536);
+    if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    ext2 alpha[2];
+    alpha[0] = e2_squeeze(t, "lu2_alpha");
+    alpha[1] = e2_squeeze(t, "lu2_alpha");
+    ext2 l1[8];
+    e2_read(t, &rd, "lu2_l1", l1, 8);
+    if (rd.bad) FAIL(REJ_FORMAT, 1, 0);
+    for (int tau = 0; tau < 2; tau++) {
+        const ext2* x = l1 + 4 * tau;
+        ext2 P0 = e2_add(e2_mul(x[0], x[3]), e2_mul(x[1], x[2])), Q0 = e2_mul(x[2], x[3]), PT, QT;
+        lu2_table(tau == 0 ? mr : mc, tau == 0 ? Trem : 65536, tau, K.k, alpha[tau], gamma, &PT, &QT);
+        if ((Q0.a == 0 && Q0.b == 0) || !e2_eqv(e2_mul(P0, QT), e2_mul(Q0, PT)))
+            FAIL(tau == 0 ? REJ_ROOT_REM : REJ_ROOT_CLAMP, 0, 0);
+    }
+    ext2 mu = e2_squeeze(t, "lu2_mu"), cP[2], cQ[2];
+    for (int tau = 0; tau < 2; tau++) {
+        cP[tau] = lu2_fold(l1[4 * tau], l1[4 * tau + 1], mu);
+        cQ[tau] = lu2_fold(l1[4 * tau + 2], l1[4 * tau + 3], mu);
+    }
+    z[0] = mu;
+    for (int d = 1; d < v; d++) {
+        ext2 lam = e2_squeeze(t, "lu2_lambda");
+        ext2 lam2 = e2_mul(lam, lam), lam3 = e2_mul(lam2, lam);
+        ext2 claim = e2_add(e2_add(cP[0], e2_mul(lam, cQ[0])), e2_add(e2_mul(lam2, cP[1]), e2_mul(lam3, cQ[1])));
+        for (int r = 0; r < d; r++) {
+            ext2 g[4];
+            e2_read(t, &rd, "lu2_round", g, 4);
+            if (rd.bad) FAIL(REJ_FORMAT, 2, d);
+            if (!e2_eqv(e2_add(g[0], g[1]), claim)) FAIL(REJ_GKR_ROUND, d, r);
+            rho[r] = e2_squeeze(t, "lu2_chal");
+            claim = e2_lagrange4(g, rho[r]);
+        }
+        ext2 fin[8];
+        e2_read(t, &rd, "lu2_final", fin, 8);
+        if (rd.bad) FAIL(REJ_FORMAT, 3, d);
+        if (!e2_eqv(e2_mul(e2_eq_closed(z, rho, d), lu2_F(fin, lam, lam2)), claim)) FAIL(REJ_GKR_FINAL, d, 0);
+        mu = e2_squeeze(t, "lu2_mu");
+        for (int tau = 0; tau < 2; tau++) {
+            cP[tau] = lu2_fold(fin[4 * tau], fin[4 * tau + 1], mu);
+            cQ[tau] = lu2_fold(fin[4 * tau + 2], fin[4 * tau + 3], mu);
+        }
+        for (int r = 0; r < d; r++) z[r] = rho[r];
+        z[d] = mu;
+    }
+    {
+        ext2 leaf[3];
+        e2_read(t, &rd, "lu2_leaf", leaf, 3);
+        if (rd.bad) FAIL(REJ_FORMAT, 4, 0);
+        if (!e2_eqv(cP[0], e2(1, 0)) || !e2_eqv(cP[1], e2(1, 0))) FAIL(REJ_LEAF_P, 0, 0);
+        if (!e2_eqv(cQ[0], e2_sub(alpha[0], leaf[0]))) FAIL(REJ_LEAF_Q, 0, 0);
+        if (!e2_eqv(cQ[1], e2_sub(alpha[1], e2_add(leaf[1], e2_mul(gamma, leaf[2]))))) FAIL(REJ_LEAF_Q, 1, 0);
+        col = (u64*)malloc(L * sizeof(u64));
+        for (u64 i = 0; i < L; i++) col[i] = orc_fint(K.fr[i]);
+        if (!e2_eqv(x16_mle(col, L, z, v), leaf[0])) FAIL(REJ_LEAF_OPEN, 0, 0);
+        for (u64 i = 0; i < L; i++) col[i] = orc_fint(K.fq[i]);
+        if (!e2_eqv(x16_mle(col, L, z, v), leaf[1])) FAIL(REJ_LEAF_OPEN, 1, 0);
+        for (u64 i = 0; i < L; i++) col[i] = orc_fint(K.fy[i]);
+        if (!e2_eqv(x16_mle(col, L, z, v), leaf[2])) FAIL(REJ_LEAF_OPEN, 2, 0);
+    }
+    if (rd.pos != rd.len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(col);
+    free(mr);
+    free(mc);
+    free(z);
+    free(rho);
+    keys_free(&K);
+    return rc;
+}

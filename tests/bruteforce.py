@@ -923,3 +923,90 @@ def lookup16x_prove(seed: int, g, s, prefix: str, pad_s: int) -> bytes:
         z = rho_l + [sq(prefix + "_mu")]
     send(prefix + "_leaf", [x_mle(gp, z), x_mle(sp, z)])
     return bytes(out)
+
+
+def lu2_prove(seed: int, sites, wits) -> bytes:
+    """The two-table rescale LogUp over the extension from definitions: both fraction trees by
+    their recurrence, every layer round value a hypercube sum of eq times the batched summand
+    over MLEs at extension points (no folding)."""
+    r = np.concatenate([np.asarray(w[1], np.int64).reshape(-1) for w in wits])
+    q = np.concatenate([np.asarray(w[0], np.int64).reshape(-1) for w in wits])
+    y = np.concatenate([np.asarray(w[2], np.int64).reshape(-1) for w in wits])
+    nk = len(r)
+    v = max(1, log2c(nk))
+    L = 1 << v
+    k = sites[0].k_shift
+    rp = [int(x) for x in r] + [0] * (L - nk)
+    qp = [int(x) for x in q] + [0] * (L - nk)
+    yp = [int(x) for x in y] + [0] * (L - nk)
+    out = bytearray()
+    tx = Tx(seed)
+
+    def send(label, xs):
+        b = fe_bytes([c for x in xs for c in x])
+        out.extend(b)
+        tx.absorb(label, b)
+
+    def sq(label):
+        a = tx.squeeze(label)
+        return (a, tx.squeeze(label))
+
+    def mult(vals, off, T, label):
+        m = np.zeros(T, np.int64)
+        for x in vals:
+            if 0 <= x + off < T:
+                m[x + off] += 1
+        b = m.astype("<u4").tobytes()
+        out.extend(b)
+        tx.absorb(label, tree_digest(b))
+
+    tx.absorb("lu2_site", tree_digest(r.astype("<i4").tobytes()) + tree_digest(q.astype("<i4").tobytes())
+              + tree_digest(y.astype(np.int8).tobytes()))
+    mult(rp, 1 << (k - 1), 1 << k, "lu2_m_rem")
+    gamma = sq("lu2_gamma")
+    mult(qp, 32768, 65536, "lu2_m_clamp")
+    alpha = [sq("lu2_alpha"), sq("lu2_alpha")]
+    neg = lambda x: ((-x[0]) % P, (-x[1]) % P)  # noqa: E731
+    keys = [[(a % P, 0) for a in rp], [x_add((a % P, 0), x_mul(gamma, (c % P, 0))) for a, c in zip(qp, yp)]]
+    trees = []
+    for tau in range(2):
+        Pl = [[(1, 0)] * L]
+        Ql = [[x_add(alpha[tau], neg(f)) for f in keys[tau]]]
+        for _ in range(v):
+            p_, q_ = Pl[0], Ql[0]
+            Pl.insert(0, [x_add(x_mul(p_[2 * x], q_[2 * x + 1]), x_mul(p_[2 * x + 1], q_[2 * x])) for x in range(len(p_) // 2)])
+            Ql.insert(0, [x_mul(q_[2 * x], q_[2 * x + 1]) for x in range(len(p_) // 2)])
+        trees.append((Pl, Ql))
+    send("lu2_l1", [t_[0][1][0] if j == 0 else t_[0][1][1] if j == 1 else t_[1][1][0] if j == 2 else t_[1][1][1]
+                    for t_ in trees for j in range(4)])
+    z = [sq("lu2_mu")]
+    for d in range(1, v):
+        lam = sq("lu2_lambda")
+        lam2 = x_mul(lam, lam)
+        vecs = []
+        for Pl, Ql in trees:
+            Pc, Qc = Pl[d + 1], Ql[d + 1]
+            vecs += [[Pc[2 * x] for x in range(1 << d)], [Pc[2 * x + 1] for x in range(1 << d)],
+                     [Qc[2 * x] for x in range(1 << d)], [Qc[2 * x + 1] for x in range(1 << d)]]
+        rho_l = []
+        for t in range(d):
+            gr = []
+            for X in range(4):
+                acc = (0, 0)
+                rest = d - t - 1
+                for bb in range(1 << rest):
+                    pt = rho_l + [(X, 0)] + [((bb >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                    ev = [xv_mle(vv, pt) for vv in vecs]
+                    F = (0, 0)
+                    for tau, w in ((0, (1, 0)), (1, lam2)):
+                        pL, pR, qL, qR = ev[4 * tau:4 * tau + 4]
+                        f = x_add(x_add(x_mul(pL, qR), x_mul(pR, qL)), x_mul(lam, x_mul(qL, qR)))
+                        F = x_add(F, x_mul(w, f))
+                    acc = x_add(acc, x_mul(x_eq(z, pt), F))
+                gr.append(acc)
+            send("lu2_round", gr)
+            rho_l.append(sq("lu2_chal"))
+        send("lu2_final", [xv_mle(vv, rho_l) for vv in vecs])
+        z = rho_l + [sq("lu2_mu")]
+    send("lu2_leaf", [x_mle(rp, z), x_mle(qp, z), x_mle(yp, z)])
+    return bytes(out)

@@ -190,3 +190,34 @@ def test_lookup16_over_extension_accepts_and_rejects():
     base, _ = oracle.silu_prove(8, g, s)
     assert oracle.silu2_verify(8, g, s, base)[0] != "accept"
     assert oracle.exp2_verify(8, g, s, pf)[0] != "accept"
+
+
+# ---- the two-table rescale LogUp over the extension -------------------------------------
+
+def _lu_sites(shapes, seed, k=6):
+    sites = [workloads.random_site(seed + i, M, K, N, 8, k) for i, (M, K, N) in enumerate(shapes)]
+    return sites, [oracle.witness(s) for s in sites]
+
+
+@pytest.mark.parametrize("shapes", [[(1, 4, 1)], [(2, 8, 1), (1, 8, 1)], [(3, 5, 2)], [(2, 16, 4)]])
+def test_lu2_bytes_match_bruteforce(shapes):
+    sites, wits = _lu_sites(shapes, 30)
+    pf, _ = oracle.lu2_prove(3, sites, wits)
+    assert pf == bf.lu2_prove(3, sites, wits)
+
+
+def test_lu2_accepts_and_rejects():
+    sites, wits = _lu_sites([(32, 64, 16), (16, 64, 8)], 40)
+    pf, _ = oracle.lu2_prove(5, sites, wits)
+    assert oracle.lu2_verify(5, sites, wits, pf) == ("accept", (0, 0))
+    q, r, y = (a.copy() for a in wits[0])
+    r[0, 0] += 1 << 6  # a remainder outside R_6
+    pf2, _ = oracle.lu2_prove(5, sites, [(q, r, y), wits[1]])
+    assert oracle.lu2_verify(5, sites, [(q, r, y), wits[1]], pf2)[0] == "root_rem"
+    q, r, y = (a.copy() for a in wits[1])
+    y[1, 1] = 100 if y[1, 1] != 100 else 99  # an output that is not clamp(q)
+    pf3, _ = oracle.lu2_prove(5, sites, [wits[0], (q, r, y)])
+    assert oracle.lu2_verify(5, sites, [wits[0], (q, r, y)], pf3)[0] == "root_clamp"
+    off = len(pf) - 48  # r~(z)
+    x = struct.unpack("<Q", pf[off:off + 8])[0]
+    assert oracle.lu2_verify(5, sites, wits, pf[:off] + struct.pack("<Q", (x + 1) % P) + pf[off + 8:])[0] == "leaf_Q"
