@@ -518,6 +518,43 @@ int fp_lookup16x_protocol_drive(fp_tx* tx, int table, int v, const uint64_t* gam
                                 const uint8_t* m_digest, fp_values_fn fn, void* user, uint8_t* proof,
                                 size_t* proof_len);
 
+/*
+ * The rescale LogUp over the quadratic extension ("How fast can FlashProve go", 4,
+ * the note on soundness): the remainder table R_k and the clamp table C16 of
+ * logup_prove_rescale batched in one GKR, with every challenge and value an
+ * extension element (16 bytes: a then b), as a statement of its own over the
+ * sites' key columns (q, r, y of every site, concatenated in site order):
+ *   absorb "lu2_site" D(r) || D(q) (int32 little-endian) || D(y); send m_rem
+ *   ("lu2_m_rem"); squeeze gamma ("lu2_gamma"); send m_clamp ("lu2_m_clamp");
+ *   squeeze alpha_0, alpha_1 ("lu2_alpha"); send layer one of both trees
+ *   ("lu2_l1", 8 values); squeeze mu ("lu2_mu"); per layer d = 1..v-1 squeeze
+ *   lambda ("lu2_lambda"), d rounds of g(0..3) ("lu2_round", "lu2_chal") of the
+ *   sum-check of eq(z, x) sum_tau lambda^(2 tau) (pL qR + pR qL + lambda qL qR),
+ *   the eight children at rho ("lu2_final"), squeeze mu; then r~(z), q~(z), y~(z)
+ *   ("lu2_leaf").
+ * Proof bytes: 4 2^k + 4 2^16 + 128 + sum_{d=1}^{v-1} (64 d + 128) + 48. Returns
+ * FP_OK, or 1 when some key lies outside its table (the proof is still written).
+ * Site checks and errors as for logup_prove_rescale.
+ */
+int logup_prove_rescale_ext2(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites, uint8_t* proof,
+                             size_t* proof_len, void* stream);
+
+/*
+ * The host half of logup_prove_rescale_ext2 from the multiplicities on (v >= 1
+ * variables, remainder table R_k): m_rem (2^k u32), m_clamp (2^16 u32) and their
+ * 32-byte digests are given; tx must have absorbed "lu2_site". Callback kinds:
+ *   FP_VAL_COLUMN: in = gamma, alpha_0, alpha_1 (6 words); out = layer one of
+ *     both trees, P(0), P(1), Q(0), Q(1) per table (16 words);
+ *   FP_VAL_START: layer d begins; in = z_1..z_d, lambda (2 d + 2 words), t = d;
+ *   FP_VAL_ROUND: out = h_t(0), h_t(1), h_t(2) (6 words);
+ *   FP_VAL_ANSWER: in = rho_t (2 words);
+ *   FP_VAL_FINALS: out = pL, pR, qL, qR at rho, per table (16 words);
+ *   FP_VAL_CLAIM: in = the leaf point (2 v words), t = v; out = r~(z), q~(z), y~(z)
+ *     (6 words).
+ */
+int fp_lu2_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m_rem, const uint8_t* d_rem, const uint32_t* m_clamp,
+                          const uint8_t* d_clamp, fp_values_fn fn, void* user, uint8_t* proof, size_t* proof_len);
+
 /* The SiLU table's 2^16 entries silu_q(v), v = -2^15 .. 2^15 - 1, into host out (no GPU work). */
 int fp_silu_table(int32_t* out);
 

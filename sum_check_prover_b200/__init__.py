@@ -16,7 +16,7 @@ from typing import Optional, Sequence
 
 __all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P",
            "had2_protocol_drive", "lhi_protocol_drive", "mm2_protocol_drive", "route_protocol_drive",
-           "lhi2_protocol_drive", "lookup16x_protocol_drive"]
+           "lhi2_protocol_drive", "lookup16x_protocol_drive", "lu2_protocol_drive"]
 
 P = 0xFFFFFFFF00000001
 LIB_PATH = Path(__file__).resolve().with_name("libfp.so")
@@ -85,6 +85,8 @@ def lib():
     L.logup_prove_silu_ext2.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.logup_prove_exp_ext2.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_lookup16x_protocol_drive.argtypes = [vp, i32, i32, C.POINTER(u64), vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
+    L.logup_prove_rescale_ext2.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
+    L.fp_lu2_protocol_drive.argtypes = [vp, i32, i32, vp, vp, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.logup_prove_helper_inverse_ext2.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
     L.fp_lhi2_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.fp_mm2_protocol_drive.argtypes = [vp, i32, i32, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
@@ -275,6 +277,60 @@ def lookup16x_protocol_drive(tx: "Transcript", table: int, v: int, gamma, m, m_d
     rc = L.fp_lookup16x_protocol_drive(tx.h, table, v, gm, mm.ctypes.data, md, fn, None, buf, C.byref(ln))
     if rc != 0:
         raise FpError(rc, "fp_lookup16x_protocol_drive failed")
+    return buf.raw[: ln.value]
+
+
+def lu2_protocol_drive(tx: "Transcript", v: int, k: int, m_rem, d_rem: bytes, m_clamp, d_clamp: bytes,
+                       values) -> bytes:
+    """Run the host half of the extension-field rescale LogUp from the multiplicities on, with
+    its device values taken from `values` (no GPU work): values.tree(gamma, alpha0, alpha1) ->
+    layer one of both trees (8 pairs), values.layer(d, z, lam), values.round(t) -> (h(0), h(1),
+    h(2)), values.answer(t, rho), values.finals() -> 8 pairs, values.leaf(z) -> (r~, q~, y~).
+    tx must have absorbed "lu2_site"."""
+    import numpy as np
+
+    L = lib()
+
+    def pairs(inp, k_):
+        return [(int(inp[2 * i]), int(inp[2 * i + 1])) for i in range(k_)]
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            res = None
+            if kind == VAL_COLUMN:
+                ga = pairs(inp, 3)
+                res = values.tree(*ga)
+            elif kind == VAL_START:
+                pts = pairs(inp, t + 1)
+                values.layer(t, pts[:t], pts[t])
+            elif kind == VAL_ANSWER:
+                values.answer(t, (int(inp[0]), int(inp[1])))
+            elif kind == VAL_ROUND:
+                res = values.round(t)
+            elif kind == VAL_FINALS:
+                res = values.finals()
+            elif kind == VAL_CLAIM:
+                res = values.leaf(pairs(inp, t))
+            else:
+                return 1
+            for i, (a, b) in enumerate(res or []):
+                out[2 * i] = int(a)
+                out[2 * i + 1] = int(b)
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _VALUES_FN(cb)
+    mr = np.ascontiguousarray(np.asarray(m_rem, dtype="<u4"))
+    mc = np.ascontiguousarray(np.asarray(m_clamp, dtype="<u4"))
+    dr = C.create_string_buffer(bytes(d_rem), 32)
+    dc = C.create_string_buffer(bytes(d_clamp), 32)
+    cap = 4 * (1 << k) + 4 * 65536 + 128 + 48 + sum(64 * d + 128 for d in range(1, v))
+    buf = C.create_string_buffer(cap)
+    ln = C.c_size_t(cap)
+    rc = L.fp_lu2_protocol_drive(tx.h, v, k, mr.ctypes.data, dr, mc.ctypes.data, dc, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_lu2_protocol_drive failed")
     return buf.raw[: ln.value]
 
 
@@ -583,6 +639,23 @@ class Context:
         ln = C.c_size_t(cap)
         rc = self._check(self._L.sumcheck_prove_routing(self.h, tx.h, _ptr(logits), T, E, _ptr(H), _ptr(D), buf,
                                                         C.byref(ln), _stream(stream)), "sumcheck_prove_routing")
+        return buf.raw[: ln.value], rc
+
+    def prove_logup_ext2(self, tx: Transcript, sites: Sequence["SiteDesc"], stream=None):
+        """The rescale LogUp of the committed sites' keys with every challenge and value in the
+        quadratic extension; returns (proof bytes, status: 1 if some key lies outside its table)."""
+        arr, keep = _sites(sites)
+        nk = sum(int(s.M) * int(s.N) for s in sites)
+        v = 0
+        while (1 << v) < nk:
+            v += 1
+        v = max(v, 1)
+        k = int(sites[0].k_shift)
+        cap = 4 * (1 << k) + 4 * 65536 + 128 + 48 + sum(64 * d + 128 for d in range(1, v))
+        buf = C.create_string_buffer(cap)
+        ln = C.c_size_t(cap)
+        rc = self._check(self._L.logup_prove_rescale_ext2(self.h, tx.h, arr, len(sites), buf, C.byref(ln),
+                                                          _stream(stream)), "logup_prove_rescale_ext2")
         return buf.raw[: ln.value], rc
 
     def prove_helper_inverse_ext2(self, tx: Transcript, r, k: int, stream=None):

@@ -15,9 +15,9 @@ static inline Ext2 e2_squeeze_host(fp_tx* tx, const char* label) {
     return e2_make(a, b);
 }
 
-// n <= 4 extension elements into the proof at pos, absorbed under one label
+// n <= 8 extension elements into the proof at pos, absorbed under one label
 static inline void e2_send_host(fp_tx* tx, const char* label, const Ext2* v, int n, uint8_t* proof, size_t& pos) {
-    uint64_t w[8];
+    uint64_t w[16];
     for (int i = 0; i < n; i++) {
         w[2 * i] = v[i].a;
         w[2 * i + 1] = v[i].b;

@@ -62,6 +62,10 @@ enum FpKernel {
     K_X16_TREE,
     K_X16_ROUND,
     K_X16_LEAF,
+    K_LU2_HIST,
+    K_LU2_TREE,
+    K_LU2_ROUND,
+    K_LU2_LEAF,
     K_COUNT
 };
 

@@ -81,7 +81,8 @@ __global__ void x16_eq_kernel(X16Point p, Ext2* __restrict__ out) {
 }
 
 // out[0..1] = sum_{x < n} eq(z, x) a(x), out[2..3] = sum_{x < n} eq(z, x) (eq split as EH[x >> vl] EL[...])
-__global__ void __launch_bounds__(256) x16_mle_kernel(const int16_t* __restrict__ a, int64_t n,
+template <class T>
+__global__ void __launch_bounds__(256) x16_mle_kernel(const T* __restrict__ a, int64_t n,
                                                       const Ext2* __restrict__ EH, const Ext2* __restrict__ EL, int vl,
                                                       uint64_t* part, unsigned int* ticket, uint64_t* out) {
     E2Acc acc;
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(256) x16_mle_kernel(const int16_t* __restrict_
         const Ext2 e = e2_mul(EH[x >> vl], EL[x & mask]);
         ea.add(e.a);
         eb.add(e.b);
-        const int v = a[x];
+        const int64_t v = (int64_t)a[x];
         if (v != 0) acc.mac_base(e, x16_lift(v));
     }
     uint64_t v[4] = {acc.a.value(), acc.b.value(), ea.value(), eb.value()};
@@ -342,6 +343,301 @@ int x16_protocol(fp_ctx* c, fp_tx* tx, const X16Labels& lab, int v, Ext2 gamma, 
     return FP_OK;
 }
 
+
+// ---- the rescale LogUp over the extension: two trees batched in one GKR ----------------
+//
+// The remainder table R_k (keys r) and the clamp table C16 (keys q + gamma y) as in
+// logup_prove_rescale, every challenge and value in the extension, as a statement of
+// its own over the sites' key columns (labels "lu2_*"). Each layer's summand is
+// sum_tau lambda^(2 tau) (pL qR + pR qL + lambda qL qR) over both trees; a pair's two
+// trees are folded one after the other to keep the live values few.
+
+// m[key + off] += 1 for the keys inside [0, T); the rest counted in *outside
+__global__ void lu2_hist_kernel(const int32_t* __restrict__ keys, int64_t n, int64_t T, int64_t off,
+                                uint32_t* __restrict__ m, uint32_t* __restrict__ outside) {
+    uint32_t out_local = 0;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t j = (int64_t)keys[i] + off;
+        if (j >= 0 && j < T)
+            atomicAdd(m + j, 1u);
+        else
+            out_local++;
+    }
+    if (out_local) atomicAdd(outside, out_local);
+}
+
+// m[q + 2^15] += 1 for q in [-2^15, 2^15); keys outside, and outputs y != clamp(q), counted in *outside
+__global__ void lu2_hist_clamp_kernel(const int32_t* __restrict__ q, const int8_t* __restrict__ y, int64_t n,
+                                      uint32_t* __restrict__ m, uint32_t* __restrict__ outside) {
+    uint32_t out_local = 0;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t qv = q[i], j = qv + 32768;
+        if (j >= 0 && j < 65536)
+            atomicAdd(m + j, 1u);
+        else
+            out_local++;
+        if ((int64_t)y[i] != (qv < -128 ? -128 : (qv > 127 ? 127 : qv))) out_local++;
+    }
+    if (out_local) atomicAdd(outside, out_local);
+}
+
+__global__ void lu2_add_pad_kernel(uint32_t* m_rem, int64_t half, uint32_t* m_clamp, uint32_t pad) {
+    m_rem[half] += pad;
+    m_clamp[32768] += pad;
+}
+
+// leaves of both trees: P = 1, Q_0 = alpha_0 - r, Q_1 = alpha_1 - (q + gamma y); zero keys past n
+__global__ void lu2_leaf_kernel(const int32_t* __restrict__ r, const int32_t* __restrict__ q,
+                                const int8_t* __restrict__ y, int64_t n, int64_t L, Ext2 alpha0, Ext2 alpha1,
+                                Ext2 gamma, Ext2* __restrict__ P0, Ext2* __restrict__ Q0, Ext2* __restrict__ P1,
+                                Ext2* __restrict__ Q1) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < L; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint64_t rv = i < n ? x16_lift(r[i]) : 0, qv = i < n ? x16_lift(q[i]) : 0;
+        const uint64_t yv = i < n ? x16_lift(y[i]) : 0;
+        P0[i] = e2_make(1, 0);
+        P1[i] = e2_make(1, 0);
+        Q0[i] = e2_sub(alpha0, e2_make(rv, 0));
+        Q1[i] = e2_sub(alpha1, e2_make(gl_add(qv, gl_mul(gamma.a, yv)), gl_mul(gamma.b, yv)));
+    }
+}
+
+struct Lu2Layer {
+    const Ext2* P[2];  // tree layer d + 1 of each table: child x of node b is entry 2 b + x
+    const Ext2* Q[2];
+    Ext2* pl[2];       // folded children from round 2 on (2^(d-1) entries each)
+    Ext2* pr[2];
+    Ext2* ql[2];
+    Ext2* qr[2];
+    Ext2* E;           // suffix eq table (2^(d-1) entries)
+    X16Point z;        // the layer's point z_1..z_d
+    Ext2 lam, lam2;
+    int d;
+    int grid;
+    int per_block;
+    int pad;
+    uint64_t seq0;  // round t publishes seq0 + t, the final values seq0 + d + 1
+    int t_begin;    // rounds run by this launch: [t_begin, t_end]; t_end > d includes the final values
+    int t_end;
+};
+
+__global__ void __launch_bounds__(X16_THREADS, 2) lu2_layer_kernel(Lu2Layer A, FpMailbox* mb, FpRelay* rl,
+                                                                  uint64_t* part) {
+    __shared__ Ext2 tab[4 << X16_CHUNK];
+    Ext2 rho = e2_make(0, 0);
+    for (int t = A.t_begin; t <= A.d && t <= A.t_end; t++) {
+        if (t > 1) {
+            uint64_t ra, rb;
+            if (!session_wait2(mb, rl, A.seq0 + t - 1, ra, rb)) return;
+            rho = e2_make(ra, rb);
+        }
+        const int64_t h = 1ll << (A.d - t);
+        const int64_t want = (h + A.per_block - 1) / A.per_block;
+        const unsigned active = (unsigned)(want < 1 ? 1 : (want > A.grid ? A.grid : want));
+        if (blockIdx.x >= active) return;  // no pairs for this block in this or any later round
+        int w[4] = {0, 0, 0, 0};
+        if (t == 1) x16_tables(tab, A.z.z, A.d, w);
+        E2Acc a0, a1, a2;
+        for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
+            Ext2 F[3] = {e2_make(0, 0), e2_make(0, 0), e2_make(0, 0)};
+#pragma unroll 1
+            for (int tau = 0; tau < 2; tau++) {
+                const Ext2* P = A.P[tau];
+                const Ext2* Q = A.Q[tau];
+                Ext2 p0, p1, r0, r1, q0, q1, s0, s1;  // pL, pR, qL, qR at the pair's two points
+                if (t == 1) {
+                    p0 = e2_ldcg(P + 2 * b);
+                    r0 = e2_ldcg(P + 2 * b + 1);
+                    q0 = e2_ldcg(Q + 2 * b);
+                    s0 = e2_ldcg(Q + 2 * b + 1);
+                    p1 = e2_ldcg(P + 2 * (b + h));
+                    r1 = e2_ldcg(P + 2 * (b + h) + 1);
+                    q1 = e2_ldcg(Q + 2 * (b + h));
+                    s1 = e2_ldcg(Q + 2 * (b + h) + 1);
+                } else {
+                    if (t == 2) {
+                        p0 = e2_fold(e2_ldcg(P + 2 * b), e2_ldcg(P + 2 * (b + 2 * h)), rho);
+                        r0 = e2_fold(e2_ldcg(P + 2 * b + 1), e2_ldcg(P + 2 * (b + 2 * h) + 1), rho);
+                        q0 = e2_fold(e2_ldcg(Q + 2 * b), e2_ldcg(Q + 2 * (b + 2 * h)), rho);
+                        s0 = e2_fold(e2_ldcg(Q + 2 * b + 1), e2_ldcg(Q + 2 * (b + 2 * h) + 1), rho);
+                        p1 = e2_fold(e2_ldcg(P + 2 * (b + h)), e2_ldcg(P + 2 * (b + 3 * h)), rho);
+                        r1 = e2_fold(e2_ldcg(P + 2 * (b + h) + 1), e2_ldcg(P + 2 * (b + 3 * h) + 1), rho);
+                        q1 = e2_fold(e2_ldcg(Q + 2 * (b + h)), e2_ldcg(Q + 2 * (b + 3 * h)), rho);
+                        s1 = e2_fold(e2_ldcg(Q + 2 * (b + h) + 1), e2_ldcg(Q + 2 * (b + 3 * h) + 1), rho);
+                    } else {
+                        p0 = e2_fold(e2_ldcg(A.pl[tau] + b), e2_ldcg(A.pl[tau] + b + 2 * h), rho);
+                        r0 = e2_fold(e2_ldcg(A.pr[tau] + b), e2_ldcg(A.pr[tau] + b + 2 * h), rho);
+                        q0 = e2_fold(e2_ldcg(A.ql[tau] + b), e2_ldcg(A.ql[tau] + b + 2 * h), rho);
+                        s0 = e2_fold(e2_ldcg(A.qr[tau] + b), e2_ldcg(A.qr[tau] + b + 2 * h), rho);
+                        p1 = e2_fold(e2_ldcg(A.pl[tau] + b + h), e2_ldcg(A.pl[tau] + b + 3 * h), rho);
+                        r1 = e2_fold(e2_ldcg(A.pr[tau] + b + h), e2_ldcg(A.pr[tau] + b + 3 * h), rho);
+                        q1 = e2_fold(e2_ldcg(A.ql[tau] + b + h), e2_ldcg(A.ql[tau] + b + 3 * h), rho);
+                        s1 = e2_fold(e2_ldcg(A.qr[tau] + b + h), e2_ldcg(A.qr[tau] + b + 3 * h), rho);
+                    }
+                    A.pl[tau][b] = p0;
+                    A.pr[tau][b] = r0;
+                    A.ql[tau][b] = q0;
+                    A.qr[tau][b] = s0;
+                    A.pl[tau][b + h] = p1;
+                    A.pr[tau][b + h] = r1;
+                    A.ql[tau][b + h] = q1;
+                    A.qr[tau][b + h] = s1;
+                }
+                Ext2 f0 = x16_f(p0, r0, q0, s0, A.lam), f1 = x16_f(p1, r1, q1, s1, A.lam);
+                Ext2 f2 = x16_f(e2_at2(p0, p1), e2_at2(r0, r1), e2_at2(q0, q1), e2_at2(s0, s1), A.lam);
+                if (tau == 1) {
+                    f0 = e2_mul(A.lam2, f0);
+                    f1 = e2_mul(A.lam2, f1);
+                    f2 = e2_mul(A.lam2, f2);
+                }
+                F[0] = e2_add(F[0], f0);
+                F[1] = e2_add(F[1], f1);
+                F[2] = e2_add(F[2], f2);
+            }
+            Ext2 e;
+            if (t == 1) {
+                e = x16_eq_at(tab, w, b);  // eq(z_2..z_d, b)
+                if (A.d > 1) A.E[b] = e;
+            } else {
+                e = e2_add(e2_ldcg(A.E + b), e2_ldcg(A.E + b + h));  // eq(z_>t, b)
+                A.E[b] = e;
+            }
+            const uint64_t e7 = gl_mul7(e.b);
+            a0.mac(e, e7, F[0]);
+            a1.mac(e, e7, F[1]);
+            a2.mac(e, e7, F[2]);
+        }
+        uint64_t acc[6] = {a0.a.value(), a0.b.value(), a1.a.value(), a1.b.value(), a2.a.value(), a2.b.value()};
+        bool last;
+        if (active == 1) {
+            block_sum_gl<6>(acc);
+            last = true;
+        } else {
+            last = grid_sum_gl_n<6>(acc, part, &rl->ticket, active);
+        }
+        if (last && threadIdx.x == 0) session_publish(mb, acc, A.seq0 + t);  // {h(0), h(1), h(2)}
+    }
+    // block 0 folds the last pair of each of the eight vectors by the last challenge
+    if (A.t_end <= A.d || blockIdx.x != 0) return;
+    uint64_t ra, rb;
+    if (!session_wait2(mb, rl, A.seq0 + A.d, ra, rb)) return;
+    rho = e2_make(ra, rb);
+    if (threadIdx.x == 0) {
+        uint64_t fin[16];
+        for (int tau = 0; tau < 2; tau++) {
+            Ext2 f[4];
+            if (A.d == 1) {
+                f[0] = e2_fold(e2_ldcg(A.P[tau]), e2_ldcg(A.P[tau] + 2), rho);
+                f[1] = e2_fold(e2_ldcg(A.P[tau] + 1), e2_ldcg(A.P[tau] + 3), rho);
+                f[2] = e2_fold(e2_ldcg(A.Q[tau]), e2_ldcg(A.Q[tau] + 2), rho);
+                f[3] = e2_fold(e2_ldcg(A.Q[tau] + 1), e2_ldcg(A.Q[tau] + 3), rho);
+            } else {
+                f[0] = e2_fold(e2_ldcg(A.pl[tau]), e2_ldcg(A.pl[tau] + 1), rho);
+                f[1] = e2_fold(e2_ldcg(A.pr[tau]), e2_ldcg(A.pr[tau] + 1), rho);
+                f[2] = e2_fold(e2_ldcg(A.ql[tau]), e2_ldcg(A.ql[tau] + 1), rho);
+                f[3] = e2_fold(e2_ldcg(A.qr[tau]), e2_ldcg(A.qr[tau] + 1), rho);
+            }
+            for (int i = 0; i < 4; i++) {
+                fin[8 * tau + 2 * i] = f[i].a;
+                fin[8 * tau + 2 * i + 1] = f[i].b;
+            }
+        }
+        session_publish(mb, fin, A.seq0 + A.d + 1);
+    }
+}
+
+// Where the device values come from. Each call returns FP_OK or an error status.
+struct Lu2Source {
+    virtual ~Lu2Source() {}
+    virtual void abandon() {}
+    virtual int tree(Ext2 gamma, Ext2 alpha0, Ext2 alpha1, Ext2 l1[8]) = 0;  // both trees, layer one
+    virtual int layer(int d, const Ext2* z, Ext2 lam) = 0;
+    virtual int round(int t, Ext2 h[3]) = 0;
+    virtual int answer(int d, int t, Ext2 rho) = 0;
+    virtual int finals(int d, Ext2 fin[8]) = 0;                               // both trees' children at rho
+    virtual int leaf(const Ext2* z, int v, Ext2 out[3]) = 0;                  // r~(z), q~(z), y~(z)
+};
+
+size_t lu2_proof_len(int v, int k) {
+    size_t len = 4 * ((size_t)1 << k) + 4 * 65536 + 128 + 48;
+    for (int d = 1; d < v; d++) len += 64 * (size_t)d + 128;
+    return len;
+}
+
+// The protocol after "lu2_site" is absorbed, from the multiplicities on.
+int lu2_protocol(fp_ctx* c, fp_tx* tx, int v, int k, const uint32_t* m_rem, const uint8_t d_rem[32],
+                 const uint32_t* m_clamp, const uint8_t d_clamp[32], Lu2Source& src, uint8_t* proof,
+                 size_t* proof_len) {
+    int rc;
+    size_t pos = 0;
+    const size_t T = (size_t)1 << k;
+    for (size_t j = 0; j < T; j++)
+        for (int b = 0; b < 4; b++) proof[pos + 4 * j + b] = (uint8_t)(m_rem[j] >> (8 * b));
+    pos += 4 * T;
+    fp_tx_absorb_raw(tx, "lu2_m_rem", d_rem, 32);
+    const Ext2 gamma = e2_squeeze_host(tx, "lu2_gamma");
+    for (size_t j = 0; j < 65536; j++)
+        for (int b = 0; b < 4; b++) proof[pos + 4 * j + b] = (uint8_t)(m_clamp[j] >> (8 * b));
+    pos += 4 * 65536;
+    fp_tx_absorb_raw(tx, "lu2_m_clamp", d_clamp, 32);
+    const Ext2 alpha0 = e2_squeeze_host(tx, "lu2_alpha");
+    const Ext2 alpha1 = e2_squeeze_host(tx, "lu2_alpha");
+    Ext2 l1[8];
+    if ((rc = src.tree(gamma, alpha0, alpha1, l1))) return rc;
+    e2_send_host(tx, "lu2_l1", l1, 8, proof, pos);
+    Ext2 z[X16_MAX_V + 1];
+    z[0] = e2_squeeze_host(tx, "lu2_mu");
+    Ext2 cP[2], cQ[2];
+    for (int tau = 0; tau < 2; tau++) {
+        cP[tau] = e2_fold_host(l1[4 * tau], l1[4 * tau + 1], z[0]);
+        cQ[tau] = e2_fold_host(l1[4 * tau + 2], l1[4 * tau + 3], z[0]);
+    }
+    const Ext2 one = e2_make(1, 0);
+    for (int d = 1; d < v; d++) {
+        const Ext2 lam = e2_squeeze_host(tx, "lu2_lambda");
+        const Ext2 lam2 = e2_mul(lam, lam), lam3 = e2_mul(lam2, lam);
+        Ext2 claim = e2_add(e2_add(cP[0], e2_mul(lam, cQ[0])), e2_add(e2_mul(lam2, cP[1]), e2_mul(lam3, cQ[1])));
+        if ((rc = src.layer(d, z, lam))) return rc;
+        Ext2 pre = one;
+        Ext2 rho[X16_MAX_V];
+        for (int t = 1; t <= d; t++) {
+            Ext2 h[3];
+            if ((rc = src.round(t, h))) return rc;
+            const Ext2 zt = z[t - 1];
+            const Ext2 h3 = e2_add(e2_sub(h[0], e2_scal(h[1], 3)), e2_scal(h[2], 3));
+            Ext2 g[4];
+            g[0] = e2_mul(pre, e2_mul(e2_sub(one, zt), h[0]));
+            g[1] = e2_mul(pre, e2_mul(zt, h[1]));
+            g[2] = e2_mul(pre, e2_mul(e2_sub(e2_scal(zt, 3), one), h[2]));
+            g[3] = e2_mul(pre, e2_mul(e2_sub(e2_scal(zt, 5), e2_make(2, 0)), h3));
+            if (!e2_same(e2_add(g[0], g[1]), claim)) {
+                src.abandon();
+                return fp_fail(c, FP_ERR_CUDA, "logup_prove_rescale_ext2: round values inconsistent with the claim");
+            }
+            e2_send_host(tx, "lu2_round", g, 4, proof, pos);
+            const Ext2 r = e2_squeeze_host(tx, "lu2_chal");
+            if ((rc = src.answer(d, t, r))) return rc;
+            rho[t - 1] = r;
+            claim = e2_lagrange4(g, r);
+            pre = e2_mul(pre, e2_eq(zt, r));
+        }
+        Ext2 fin[8];
+        if ((rc = src.finals(d, fin))) return rc;
+        e2_send_host(tx, "lu2_final", fin, 8, proof, pos);
+        const Ext2 mu = e2_squeeze_host(tx, "lu2_mu");
+        for (int tau = 0; tau < 2; tau++) {
+            cP[tau] = e2_fold_host(fin[4 * tau], fin[4 * tau + 1], mu);
+            cQ[tau] = e2_fold_host(fin[4 * tau + 2], fin[4 * tau + 3], mu);
+        }
+        for (int i = 0; i < d; i++) z[i] = rho[i];
+        z[d] = mu;
+    }
+    Ext2 leaf[3];
+    if ((rc = src.leaf(z, v, leaf))) return rc;
+    e2_send_host(tx, "lu2_leaf", leaf, 3, proof, pos);
+    *proof_len = pos;
+    return FP_OK;
+}
+
 unsigned x16_grid(const fp_ctx* c, int64_t work) {
     return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
 }
@@ -470,8 +766,8 @@ struct X16Device : X16Source {
         fp_tic(c, st, K_X16_LEAF, 4.0 * (double)n, &slot);
         x16_eq_kernel<<<x16_grid(c, 1ll << vh), 256, 0, st>>>(ph, EH);
         x16_eq_kernel<<<x16_grid(c, 1ll << vl), 256, 0, st>>>(pl, EL);
-        x16_mle_kernel<<<blocks, 256, 0, st>>>(g, n, EH, EL, vl, part, c->tickets, small);
-        x16_mle_kernel<<<blocks, 256, 0, st>>>(s, n, EH, EL, vl, part, c->tickets, small + 4);
+        x16_mle_kernel<int16_t><<<blocks, 256, 0, st>>>(g, n, EH, EL, vl, part, c->tickets, small);
+        x16_mle_kernel<int16_t><<<blocks, 256, 0, st>>>(s, n, EH, EL, vl, part, c->tickets, small + 4);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         c->launches += 3;  // four kernels under one timing slot
@@ -538,6 +834,203 @@ struct X16Callback : X16Source {
         const int rc = call(FP_VAL_CLAIM, v, in, out);
         out2[0] = ext(out);
         out2[1] = ext(out + 2);
+        return rc;
+    }
+};
+
+
+// Device values from the kernels above.
+struct Lu2Device : Lu2Source {
+    fp_ctx* c;
+    cudaStream_t st;
+    const int32_t* r;
+    const int32_t* q;
+    const int8_t* y;
+    int64_t n;
+    int v;
+    std::vector<Ext2*> TP[2], TQ[2];
+    Ext2* vec[9];  // pl, pr, ql, qr of table 0, then of table 1, then E
+    Ext2 *EH, *EL;
+    uint64_t *part, *small, *hs;
+    Lu2Layer A;
+    int cap_grid = 1;
+
+    void abandon() override { fp_session_abandon(c, st); }
+
+    int tree(Ext2 gamma, Ext2 alpha0, Ext2 alpha1, Ext2 l1[8]) override {
+        const int64_t L = 1ll << v;
+        int slot;
+        fp_tic(c, st, K_LU2_TREE, 9.0 * (double)n + 128.0 * (double)L, &slot);
+        lu2_leaf_kernel<<<x16_grid(c, L), 256, 0, st>>>(r, q, y, n, L, alpha0, alpha1, gamma, TP[0][v], TQ[0][v],
+                                                         TP[1][v], TQ[1][v]);
+        FP_CUDA(c, cudaGetLastError());
+        for (int tau = 0; tau < 2; tau++)
+            for (int d = v - 1; d >= 1; d--) {
+                x16_level_kernel<<<x16_grid(c, 1ll << d), 256, 0, st>>>(TP[tau][d + 1], TQ[tau][d + 1], 1ll << d,
+                                                                        TP[tau][d], TQ[tau][d]);
+                FP_CUDA(c, cudaGetLastError());
+                c->launches++;
+            }
+        fp_toc(c, st, slot);
+        for (int tau = 0; tau < 2; tau++) {
+            FP_CUDA(c, cudaMemcpyAsync(hs + 8 * tau, TP[tau][1], 32, cudaMemcpyDeviceToHost, st));
+            FP_CUDA(c, cudaMemcpyAsync(hs + 8 * tau + 4, TQ[tau][1], 32, cudaMemcpyDeviceToHost, st));
+        }
+        FP_CUDA(c, cudaStreamSynchronize(st));
+        for (int i = 0; i < 8; i++) l1[i] = e2_make(hs[2 * i], hs[2 * i + 1]);  // P(0), P(1), Q(0), Q(1) per table
+        return FP_OK;
+    }
+
+    double round_bytes(int t) const {
+        const double pairs = (double)(1ll << (A.d - t));
+        return (t == 1 ? 288.0 : 576.0) * pairs;  // eight 16-byte child vectors and the eq table
+    }
+
+    int launch(int t_begin, int t_end, unsigned grid, double bytes) {
+        A.t_begin = t_begin;
+        A.t_end = t_end;
+        void* args[] = {&A, &c->mb_dev, &c->relay, &part};
+        int slot;
+        fp_tic(c, st, K_LU2_ROUND, bytes, &slot);
+        FP_CUDA(c, cudaLaunchCooperativeKernel((const void*)lu2_layer_kernel, dim3(grid), dim3(X16_THREADS), args, 0,
+                                               st));
+        fp_toc(c, st, slot);
+        return FP_OK;
+    }
+
+    int layer(int d, const Ext2* z, Ext2 lam) override {
+        int rc;
+        memset(&A, 0, sizeof A);
+        for (int tau = 0; tau < 2; tau++) {
+            A.P[tau] = TP[tau][d + 1];
+            A.Q[tau] = TQ[tau][d + 1];
+            A.pl[tau] = vec[4 * tau];
+            A.pr[tau] = vec[4 * tau + 1];
+            A.ql[tau] = vec[4 * tau + 2];
+            A.qr[tau] = vec[4 * tau + 3];
+        }
+        A.E = vec[8];
+        for (int i = 0; i < d; i++) A.z.z[i] = z[i];
+        A.z.v = d;
+        A.lam = lam;
+        A.lam2 = e2_mul(lam, lam);
+        A.d = d;
+        A.per_block = X16_THREADS;  // one pair per thread
+        const int64_t half = 1ll << (d - 1);
+        A.grid = (int)std::max<int64_t>(1, std::min<int64_t>((half + A.per_block - 1) / A.per_block, cap_grid));
+        A.seq0 = fp_seq_reserve(c, (uint64_t)d + 2);
+        if ((rc = fp_session_begin(c, st))) return rc;
+        fp_session_expect(c, 6);  // before any launch: round 1 publishes without a challenge
+        if (!c->stepped) {
+            double bytes = 0;
+            for (int t = 1; t <= d; t++) bytes += round_bytes(t);
+            return launch(1, d + 1, (unsigned)A.grid, bytes);
+        }
+        return FP_OK;
+    }
+
+    int round(int t, Ext2 h[3]) override {
+        int rc;
+        if (c->stepped && (rc = launch(t, t, (unsigned)A.grid, round_bytes(t)))) return rc;
+        if ((rc = fp_session_wait(c, A.seq0 + t, st))) return rc;
+        for (int i = 0; i < 3; i++) h[i] = e2_make(c->mb->res[2 * i], c->mb->res[2 * i + 1]);
+        return FP_OK;
+    }
+
+    int answer(int d, int t, Ext2 rho) override {
+        fp_session_expect(c, t < d ? 6 : 16);  // the last challenge triggers the sixteen final words
+        fp_session_post2(c, A.seq0 + t, rho.a, rho.b);
+        return FP_OK;
+    }
+
+    int finals(int d, Ext2 fin[8]) override {
+        int rc;
+        if (c->stepped && (rc = launch(d + 1, d + 1, 1, 256.0))) return rc;
+        if ((rc = fp_session_wait(c, A.seq0 + d + 1, st))) return rc;
+        for (int i = 0; i < 8; i++) fin[i] = e2_make(c->mb->res[2 * i], c->mb->res[2 * i + 1]);
+        FP_CUDA(c, cudaStreamSynchronize(st));
+        return FP_OK;
+    }
+
+    int leaf(const Ext2* z, int vv, Ext2 out[3]) override {
+        const int vl = vv / 2, vh = vv - vl;
+        X16Point ph, pl;
+        memset(&ph, 0, sizeof ph);
+        memset(&pl, 0, sizeof pl);
+        ph.v = vh;
+        pl.v = vl;
+        for (int i = 0; i < vh; i++) ph.z[i] = z[i];
+        for (int i = 0; i < vl; i++) pl.z[i] = z[vh + i];
+        const unsigned blocks =
+            (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 2 * (int64_t)c->num_sms));
+        int slot;
+        fp_tic(c, st, K_LU2_LEAF, 9.0 * (double)n, &slot);
+        x16_eq_kernel<<<x16_grid(c, 1ll << vh), 256, 0, st>>>(ph, EH);
+        x16_eq_kernel<<<x16_grid(c, 1ll << vl), 256, 0, st>>>(pl, EL);
+        x16_mle_kernel<int32_t><<<blocks, 256, 0, st>>>(r, n, EH, EL, vl, part, c->tickets, small);
+        x16_mle_kernel<int32_t><<<blocks, 256, 0, st>>>(q, n, EH, EL, vl, part, c->tickets, small + 4);
+        x16_mle_kernel<int8_t><<<blocks, 256, 0, st>>>(y, n, EH, EL, vl, part, c->tickets, small + 8);
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+        c->launches += 4;  // five kernels under one timing slot
+        FP_CUDA(c, cudaMemcpyAsync(hs, small, 96, cudaMemcpyDeviceToHost, st));
+        FP_CUDA(c, cudaStreamSynchronize(st));
+        // the padding keys are zero in all three columns: no correction
+        for (int i = 0; i < 3; i++) out[i] = e2_make(hs[4 * i], hs[4 * i + 1]);
+        return FP_OK;
+    }
+};
+
+// Device values from a caller's callback (no device).
+struct Lu2Callback : Lu2Source {
+    fp_values_fn fn;
+    void* user;
+    int call(int kind, int t, const uint64_t* in, uint64_t* out) { return fn(user, kind, t, in, out) ? FP_ERR_ARG : FP_OK; }
+    static Ext2 ext(const uint64_t* w) { return e2_make(gl_canon(w[0]), gl_canon(w[1])); }
+    int tree(Ext2 gamma, Ext2 alpha0, Ext2 alpha1, Ext2 l1[8]) override {
+        const uint64_t in[6] = {gamma.a, gamma.b, alpha0.a, alpha0.b, alpha1.a, alpha1.b};
+        uint64_t out[16] = {0};
+        const int rc = call(FP_VAL_COLUMN, 0, in, out);
+        for (int i = 0; i < 8; i++) l1[i] = ext(out + 2 * i);
+        return rc;
+    }
+    int layer(int d, const Ext2* z, Ext2 lam) override {
+        uint64_t in[2 * X16_MAX_V + 4];
+        for (int i = 0; i < d; i++) {
+            in[2 * i] = z[i].a;
+            in[2 * i + 1] = z[i].b;
+        }
+        in[2 * d] = lam.a;
+        in[2 * d + 1] = lam.b;
+        return call(FP_VAL_START, d, in, nullptr);
+    }
+    int round(int t, Ext2 h[3]) override {
+        uint64_t out[6] = {0};
+        const int rc = call(FP_VAL_ROUND, t, nullptr, out);
+        for (int i = 0; i < 3; i++) h[i] = ext(out + 2 * i);
+        return rc;
+    }
+    int answer(int d, int t, Ext2 rho) override {
+        (void)d;
+        const uint64_t in[2] = {rho.a, rho.b};
+        return call(FP_VAL_ANSWER, t, in, nullptr);
+    }
+    int finals(int d, Ext2 fin[8]) override {
+        (void)d;
+        uint64_t out[16] = {0};
+        const int rc = call(FP_VAL_FINALS, 0, nullptr, out);
+        for (int i = 0; i < 8; i++) fin[i] = ext(out + 2 * i);
+        return rc;
+    }
+    int leaf(const Ext2* z, int v, Ext2 out3[3]) override {
+        uint64_t in[2 * X16_MAX_V + 2];
+        for (int i = 0; i < v; i++) {
+            in[2 * i] = z[i].a;
+            in[2 * i + 1] = z[i].b;
+        }
+        uint64_t out[6] = {0};
+        const int rc = call(FP_VAL_CLAIM, v, in, out);
+        for (int i = 0; i < 3; i++) out3[i] = ext(out + 2 * i);
         return rc;
     }
 };
@@ -659,4 +1152,133 @@ int fp_lookup16x_protocol_drive(fp_tx* tx, int table, int v, const uint64_t* gam
     cb.user = user;
     return x16_protocol(nullptr, tx, table == 0 ? kSilu2 : kExp2, v, e2_make(gamma[0], gamma[1]), m, m_digest, cb,
                         proof, proof_len);
+}
+
+int logup_prove_rescale_ext2(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, uint8_t* proof,
+                             size_t* proof_len, void* stream) {
+    if (!c || !tx || !proof_len) return fp_fail(c, FP_ERR_ARG, "logup_prove_rescale_ext2: null argument");
+    int rc;
+    if ((rc = fp_check_sites(c, sites, nsites, true))) return rc;
+    const int k = sites[0].k_shift;
+    int64_t nk = 0;
+    for (int i = 0; i < nsites; i++) {
+        if (sites[i].k_shift != k)
+            return fp_fail(c, FP_ERR_ARG, "logup_prove_rescale_ext2: every site needs the same k_shift");
+        nk += (int64_t)sites[i].M * sites[i].N;
+    }
+    if (nk > (1ll << X16_MAX_V)) return fp_fail(c, FP_ERR_SHAPE, "logup_prove_rescale_ext2: more than 2^30 keys");
+    const int v = std::max(1, fp_log2_ceil((uint64_t)nk));
+    const size_t need_len = lu2_proof_len(v, k);
+    if (!proof || *proof_len < need_len) {
+        *proof_len = need_len;
+        return fp_fail(c, FP_ERR_ARG, "logup_prove_rescale_ext2: proof buffer too small");
+    }
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t L = 1ll << v, T = 1ll << k;
+    Lu2Device dev;
+    dev.c = c;
+    dev.st = st;
+    dev.n = nk;
+    dev.v = v;
+    int occ = 0;
+    FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, lu2_layer_kernel, X16_THREADS, 0));
+    dev.cap_grid = std::max(1, occ) * c->num_sms;
+    const size_t part_n = (size_t)6 * std::max(dev.cap_grid, 4 * c->num_sms);
+    const int64_t hv = v >= 2 ? 1ll << (v - 2) : 1;
+    const int vl = v / 2, vh = v - vl;
+    size_t need = 2 * fp_align_up((size_t)4 * nk, 256) + fp_align_up((size_t)nk, 256) + fp_align_up((size_t)4 * T, 256) +
+                  fp_align_up(4 * 65536, 256) + fp_align_up(8 * part_n, 256) + 2 * fp_align_up(8 * 64, 256) +
+                  fp_align_up((size_t)16 << vh, 256) + fp_align_up((size_t)16 << vl, 256) +
+                  9 * fp_align_up((size_t)16 * hv, 256) + 4096;
+    for (int d = 1; d <= v; d++) need += 4 * fp_align_up((size_t)16 << d, 256);
+    if ((rc = fp_reserve(c, c->dev, need))) return rc;
+    if ((rc = fp_reserve(c, c->host, fp_align_up((size_t)4 * T, 256) + 4 * 65536 + 8192))) return rc;
+    fp_reset(c->dev);
+    fp_reset(c->host);
+    int32_t* r_all = (int32_t*)fp_alloc(c->dev, (size_t)4 * nk);
+    int32_t* q_all = (int32_t*)fp_alloc(c->dev, (size_t)4 * nk);
+    int8_t* y_all = (int8_t*)fp_alloc(c->dev, (size_t)nk);
+    uint32_t* m_rem = (uint32_t*)fp_alloc(c->dev, (size_t)4 * T);
+    uint32_t* m_cl = (uint32_t*)fp_alloc(c->dev, 4 * 65536);
+    dev.part = (uint64_t*)fp_alloc(c->dev, 8 * part_n);
+    dev.small = (uint64_t*)fp_alloc(c->dev, 8 * 64);
+    uint32_t* outside = (uint32_t*)fp_alloc(c->dev, 8 * 64);
+    dev.EH = (Ext2*)fp_alloc(c->dev, (size_t)16 << vh);
+    dev.EL = (Ext2*)fp_alloc(c->dev, (size_t)16 << vl);
+    bool ok = r_all && q_all && y_all && m_rem && m_cl && dev.part && dev.small && outside && dev.EH && dev.EL;
+    for (int i = 0; i < 9; i++) ok = ok && (dev.vec[i] = (Ext2*)fp_alloc(c->dev, (size_t)16 * hv));
+    for (int tau = 0; tau < 2; tau++) {
+        dev.TP[tau].assign(v + 1, nullptr);
+        dev.TQ[tau].assign(v + 1, nullptr);
+        for (int d = 1; d <= v; d++) {
+            ok = ok && (dev.TP[tau][d] = (Ext2*)fp_alloc(c->dev, (size_t)16 << d));
+            ok = ok && (dev.TQ[tau][d] = (Ext2*)fp_alloc(c->dev, (size_t)16 << d));
+        }
+    }
+    uint32_t* hm = (uint32_t*)fp_alloc(c->host, (size_t)4 * T + 4 * 65536);
+    dev.hs = (uint64_t*)fp_alloc(c->host, 8 * 64);
+    if (!ok || !hm || !dev.hs) return fp_fail(c, FP_ERR_OOM, "logup_prove_rescale_ext2: scratch exhausted");
+    dev.r = r_all;
+    dev.q = q_all;
+    dev.y = y_all;
+
+    // ---- the key columns, concatenated in site order ----
+    int64_t o = 0;
+    for (int i = 0; i < nsites; i++) {
+        const int64_t mn = (int64_t)sites[i].M * sites[i].N;
+        FP_CUDA(c, cudaMemcpyAsync(r_all + o, sites[i].r, 4 * (size_t)mn, cudaMemcpyDeviceToDevice, st));
+        FP_CUDA(c, cudaMemcpyAsync(q_all + o, sites[i].q, 4 * (size_t)mn, cudaMemcpyDeviceToDevice, st));
+        FP_CUDA(c, cudaMemcpyAsync(y_all + o, sites[i].y, (size_t)mn, cudaMemcpyDeviceToDevice, st));
+        o += mn;
+    }
+    {
+        FpDigestJob jobs[3] = {{(const uint8_t*)r_all, 4 * (uint64_t)nk}, {(const uint8_t*)q_all, 4 * (uint64_t)nk},
+                               {(const uint8_t*)y_all, (uint64_t)nk}};
+        uint8_t d[96];
+        if ((rc = fp_digest_many(c, jobs, 3, d, st))) return rc;  // synchronises the stream
+        fp_tx_absorb_raw(tx, "lu2_site", d, 96);
+    }
+    // ---- multiplicities ----
+    FP_CUDA(c, cudaMemsetAsync(m_rem, 0, (size_t)4 * T, st));
+    FP_CUDA(c, cudaMemsetAsync(m_cl, 0, 4 * 65536, st));
+    FP_CUDA(c, cudaMemsetAsync(outside, 0, 4, st));
+    {
+        int slot;
+        fp_tic(c, st, K_LU2_HIST, 9.0 * (double)nk, &slot);
+        lu2_hist_kernel<<<x16_grid(c, nk), 256, 0, st>>>(r_all, nk, T, T / 2, m_rem, outside);
+        lu2_hist_clamp_kernel<<<x16_grid(c, nk), 256, 0, st>>>(q_all, y_all, nk, m_cl, outside);
+        if (L > nk) lu2_add_pad_kernel<<<1, 1, 0, st>>>(m_rem, T / 2, m_cl, (uint32_t)(L - nk));
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+        c->launches += L > nk ? 2 : 1;
+    }
+    FP_CUDA(c, cudaMemcpyAsync(hm, m_rem, (size_t)4 * T, cudaMemcpyDeviceToHost, st));
+    FP_CUDA(c, cudaMemcpyAsync(hm + T, m_cl, 4 * 65536, cudaMemcpyDeviceToHost, st));
+    FP_CUDA(c, cudaMemcpyAsync(dev.hs, outside, 4, cudaMemcpyDeviceToHost, st));
+    uint8_t dm[64];
+    {
+        FpDigestJob jobs[2] = {{(const uint8_t*)m_rem, 4 * (uint64_t)T}, {(const uint8_t*)m_cl, 4 * 65536ull}};
+        if ((rc = fp_digest_many(c, jobs, 2, dm, st))) return rc;  // synchronises the stream
+    }
+    uint32_t n_outside;
+    memcpy(&n_outside, dev.hs, 4);
+    if ((rc = lu2_protocol(c, tx, v, k, hm, dm, hm + T, dm + 32, dev, proof, proof_len))) return rc;
+    return n_outside ? 1 : FP_OK;
+}
+
+int fp_lu2_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m_rem, const uint8_t* d_rem, const uint32_t* m_clamp,
+                          const uint8_t* d_clamp, fp_values_fn fn, void* user, uint8_t* proof, size_t* proof_len) {
+    if (!tx || !fn || !proof_len || !m_rem || !d_rem || !m_clamp || !d_clamp) return FP_ERR_ARG;
+    if (v < 1 || v > X16_MAX_V) return FP_ERR_SHAPE;
+    if (k < 1 || k > 20) return FP_ERR_ARG;
+    const size_t need_len = lu2_proof_len(v, k);
+    if (!proof || *proof_len < need_len) {
+        *proof_len = need_len;
+        return FP_ERR_ARG;
+    }
+    Lu2Callback cb;
+    cb.fn = fn;
+    cb.user = user;
+    return lu2_protocol(nullptr, tx, v, k, m_rem, d_rem, m_clamp, d_clamp, cb, proof, proof_len);
 }

@@ -436,3 +436,108 @@ def test_lookup16x_exp_table_and_refusal(fp):
     assert _lk_drive(fp, 6, g, s, 1, BruteLookup16x(g, s, oracle.exp_q(0))) == oracle.exp2_prove(6, g, s)
     with pytest.raises(fp.FpError):
         _lk_drive(fp, 6, g, s, 1, BruteLookup16x(g, s, oracle.exp_q(0), tamper=(2, 2)))
+
+
+# ---- the two-table rescale LogUp over the extension --------------------------------------
+
+class BruteLu2:
+    """Device values of the extension-field rescale LogUp by their definitions."""
+
+    def __init__(self, wits, tamper=None):
+        self.r = [int(x) for w in wits for x in np.asarray(w[1]).reshape(-1)]
+        self.q = [int(x) for w in wits for x in np.asarray(w[0]).reshape(-1)]
+        self.y = [int(x) for w in wits for x in np.asarray(w[2]).reshape(-1)]
+        nk = len(self.r)
+        self.v = max(1, bf.log2c(nk))
+        L = 1 << self.v
+        self.rp, self.qp, self.yp = (c + [0] * (L - nk) for c in (self.r, self.q, self.y))
+        self.tamper = tamper
+
+    def tree(self, gamma, alpha0, alpha1):
+        neg = lambda x: ((-x[0]) % P, (-x[1]) % P)  # noqa: E731
+        keys = [[(a % P, 0) for a in self.rp],
+                [bf.x_add((a % P, 0), bf.x_mul(gamma, (c % P, 0))) for a, c in zip(self.qp, self.yp)]]
+        self.trees = []
+        for tau, alpha in enumerate((alpha0, alpha1)):
+            Pl = [[(1, 0)] * len(keys[tau])]
+            Ql = [[bf.x_add(alpha, neg(f)) for f in keys[tau]]]
+            for _ in range(self.v):
+                p_, q_ = Pl[0], Ql[0]
+                Pl.insert(0, [bf.x_add(bf.x_mul(p_[2 * x], q_[2 * x + 1]), bf.x_mul(p_[2 * x + 1], q_[2 * x]))
+                              for x in range(len(p_) // 2)])
+                Ql.insert(0, [bf.x_mul(q_[2 * x], q_[2 * x + 1]) for x in range(len(p_) // 2)])
+            self.trees.append((Pl, Ql))
+        return [v_ for Pl, Ql in self.trees for v_ in (Pl[1][0], Pl[1][1], Ql[1][0], Ql[1][1])]
+
+    def layer(self, d, z, lam):
+        self.d, self.z, self.lam, self.rho = d, z, lam, []
+        self.lam2 = bf.x_mul(lam, lam)
+        self.vecs = []
+        for Pl, Ql in self.trees:
+            Pc, Qc = Pl[d + 1], Ql[d + 1]
+            self.vecs += [[Pc[2 * x] for x in range(1 << d)], [Pc[2 * x + 1] for x in range(1 << d)],
+                          [Qc[2 * x] for x in range(1 << d)], [Qc[2 * x + 1] for x in range(1 << d)]]
+
+    def round(self, t):
+        rest = self.d - t
+        h = []
+        for X in range(3):
+            acc = (0, 0)
+            for b in range(1 << rest):
+                bits = [((b >> (rest - 1 - i)) & 1, 0) for i in range(rest)]
+                pt = self.rho + [(X, 0)] + bits
+                ev = [bf.xv_mle(vv, pt) for vv in self.vecs]
+                F = (0, 0)
+                for tau, w in ((0, (1, 0)), (1, self.lam2)):
+                    pL, pR, qL, qR = ev[4 * tau:4 * tau + 4]
+                    f = bf.x_add(bf.x_add(bf.x_mul(pL, qR), bf.x_mul(pR, qL)), bf.x_mul(self.lam, bf.x_mul(qL, qR)))
+                    F = bf.x_add(F, bf.x_mul(w, f))
+                acc = bf.x_add(acc, bf.x_mul(bf.x_eq(self.z[t:self.d], bits), F))
+            h.append(acc)
+        if self.tamper == (self.d, t):
+            h[1] = ((h[1][0] + 1) % P, h[1][1])
+        return h
+
+    def answer(self, t, rho):
+        self.rho.append(rho)
+
+    def finals(self):
+        return [bf.xv_mle(vv, self.rho) for vv in self.vecs]
+
+    def leaf(self, z):
+        return [bf.x_mle(self.rp, z), bf.x_mle(self.qp, z), bf.x_mle(self.yp, z)]
+
+
+def _lu2_drive(fp, seed, sites, wits, vals):
+    k = sites[0].k_shift
+    tx = fp.Transcript(seed)
+    r = np.concatenate([np.asarray(w[1], np.int64).reshape(-1) for w in wits])
+    q = np.concatenate([np.asarray(w[0], np.int64).reshape(-1) for w in wits])
+    y = np.concatenate([np.asarray(w[2], np.int64).reshape(-1) for w in wits])
+    tx.absorb("lu2_site", bf.tree_digest(r.astype("<i4").tobytes()) + bf.tree_digest(q.astype("<i4").tobytes())
+              + bf.tree_digest(y.astype(np.int8).tobytes()))
+    mr = np.zeros(1 << k, np.int64)
+    mc = np.zeros(65536, np.int64)
+    for a in vals.rp:
+        if 0 <= a + (1 << (k - 1)) < (1 << k):
+            mr[a + (1 << (k - 1))] += 1
+    for a in vals.qp:
+        if 0 <= a + 32768 < 65536:
+            mc[a + 32768] += 1
+    mr, mc = mr.astype("<u4"), mc.astype("<u4")
+    pf = fp.lu2_protocol_drive(tx, vals.v, k, mr, bf.tree_digest(mr.tobytes()), mc, bf.tree_digest(mc.tobytes()), vals)
+    return pf, tx.state()
+
+
+@pytest.mark.parametrize("shapes", [[(1, 4, 1)], [(2, 8, 1), (1, 8, 1)], [(3, 5, 2)], [(2, 16, 4)]])
+def test_lu2_host_half_matches_oracle(fp, shapes):
+    sites = [workloads.random_site(30 + i, M, K, N, 8, 6) for i, (M, K, N) in enumerate(shapes)]
+    wits = [oracle.witness(s) for s in sites]
+    assert _lu2_drive(fp, 3, sites, wits, BruteLu2(wits)) == oracle.lu2_prove(3, sites, wits)
+
+
+def test_lu2_inconsistent_round_is_refused(fp):
+    sites = [workloads.random_site(31, 2, 16, 4, 8, 6)]
+    wits = [oracle.witness(s) for s in sites]
+    with pytest.raises(fp.FpError):
+        _lu2_drive(fp, 3, sites, wits, BruteLu2(wits, tamper=(2, 1)))
