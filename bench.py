@@ -171,7 +171,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2,silu2"
+MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2,silu2,lu2"
 
 
 def micro_names(which) -> set:
@@ -214,6 +214,8 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
       (16-byte vectors: 176 B per pair in round 2, 240 B later).
     silu2_round: the SiLU lookup's layer rounds over 2^26 keys with extension challenges
       (16-byte vectors: 160 and 320 B per pair).
+    lu2_round: the rescale LogUp's layer rounds over 2^26 keys with extension challenges,
+      both tables in one launch (288 and 576 B per pair).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
     """
@@ -400,6 +402,17 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
             del gd, sd
         except Exception as e:  # a failure here must not cost the rest of the line
             out["silu_ext2_lookup_round_2^26"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    if "lu2" in which:
+        # the rescale LogUp over the extension for the gkr microbench's site (2^26 keys)
+        try:
+            s = workloads.random_site(77, 8192, 64, 8192, 8, 12)
+            st, keep = device.upload(workloads.Workload("lu2", 0, [s]), dev)
+            ctx.commit_witness(fp.Transcript(0), st[0])
+            measure("rescale_logup_ext2_round_2^26_keys", "lu2_round",
+                    lambda: ctx.prove_logup_ext2(fp.Transcript(10), st[0]))
+            del st, keep
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["rescale_logup_ext2_round_2^26_keys"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     try:
         torch.cuda.empty_cache()
