@@ -215,6 +215,13 @@ int fp_claims(fp_ctx* c, const fp_site* sites, int nsites, const uint64_t* const
 
 static inline size_t fp_align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// blocks of 256 threads for a grid-stride loop over `work` items: enough to cover it, at
+// most four per SM
+static inline unsigned fp_grid256(const fp_ctx* c, int64_t work) {
+    const int64_t want = (work + 255) / 256, cap = 4 * (int64_t)c->num_sms;
+    return (unsigned)(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
 // little-endian u64 words into a proof buffer (sumcheck.cu)
 void put_u64s(uint8_t* p, const uint64_t* v, size_t n);
 

@@ -53,10 +53,6 @@ __global__ void frv_finish_kernel(const uint64_t* __restrict__ part, int nchunks
     }
 }
 
-unsigned frv_grid(const fp_ctx* c, int64_t work) {
-    return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
-}
-
 }  // namespace
 
 int freivalds_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* site, uint8_t* proof, size_t* proof_len,
@@ -93,10 +89,10 @@ int freivalds_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* site, uint8_t* p
     if (!pw || !part || !u || !hu) return fp_fail(c, FP_ERR_OOM, "freivalds_prove_matmul: scratch exhausted");
     int slot;
     fp_tic(c, st, K_FRV_U, (double)s.N * s.K + 8.0 * s.K, &slot);
-    frv_pow_kernel<<<frv_grid(c, s.N), 256, 0, st>>>(rho, s.N, pw);
+    frv_pow_kernel<<<fp_grid256(c, s.N), 256, 0, st>>>(rho, s.N, pw);
     frv_contract_kernel<<<dim3((unsigned)((s.K + 255) / 256), (unsigned)nchunks), 256, 0, st>>>(s.xt, s.N, s.K, per,
                                                                                                 pw, part);
-    frv_finish_kernel<<<frv_grid(c, s.K), 256, 0, st>>>(part, nchunks, s.K, u);
+    frv_finish_kernel<<<fp_grid256(c, s.K), 256, 0, st>>>(part, nchunks, s.K, u);
     fp_toc(c, st, slot);
     FP_CUDA(c, cudaGetLastError());
     c->launches += 2;  // three kernels under one timing slot

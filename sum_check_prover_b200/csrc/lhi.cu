@@ -294,10 +294,6 @@ struct LhiDevice : LhiSource {
     LhiArgs A;
     int cap_grid = 1;
 
-    unsigned grid_of(int64_t work) const {
-        return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
-    }
-
     int launch(int t_begin, int t_end, unsigned grid, int kernel, double bytes) {
         A.t_begin = t_begin;
         A.t_end = t_end;
@@ -324,8 +320,8 @@ struct LhiDevice : LhiSource {
         const int64_t L = 1ll << v, T = 1ll << k;
         int slot;
         fp_tic(c, st, K_LHI_COLUMN, 8.0 * (double)T + 12.0 * (double)L, &slot);
-        lhi_inv_kernel<<<grid_of(T), 256, 0, st>>>(alpha, k, inv);
-        lhi_column_kernel<<<grid_of(L), 256, 0, st>>>(r, n, L, k, alpha, inv, hcol);
+        lhi_inv_kernel<<<fp_grid256(c, T), 256, 0, st>>>(alpha, k, inv);
+        lhi_column_kernel<<<fp_grid256(c, L), 256, 0, st>>>(r, n, L, k, alpha, inv, hcol);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         c->launches++;  // two kernels under one timing slot
@@ -669,10 +665,6 @@ struct Lhi2Device : Lhi2Source {
     Lhi2Args A;
     int cap_grid = 1;
 
-    unsigned grid_of(int64_t work) const {
-        return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
-    }
-
     void abandon() override { fp_session_abandon(c, st); }
 
     int launch(int t_begin, int t_end, unsigned grid, int kernel, double bytes) {
@@ -699,8 +691,8 @@ struct Lhi2Device : Lhi2Source {
         const int64_t L = 1ll << v, T = 1ll << k;
         int slot;
         fp_tic(c, st, K_LHI2_COLUMN, 16.0 * (double)T + 20.0 * (double)L, &slot);
-        lhi2_inv_kernel<<<grid_of(T), 256, 0, st>>>(alpha, k, inv);
-        lhi2_column_kernel<<<grid_of(L), 256, 0, st>>>(r, n, L, k, alpha, inv, hcol);
+        lhi2_inv_kernel<<<fp_grid256(c, T), 256, 0, st>>>(alpha, k, inv);
+        lhi2_column_kernel<<<fp_grid256(c, L), 256, 0, st>>>(r, n, L, k, alpha, inv, hcol);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         c->launches++;  // two kernels under one timing slot

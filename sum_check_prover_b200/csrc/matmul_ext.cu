@@ -257,10 +257,6 @@ struct Mm2Device : Mm2Source {
     Mm2Args P;
     int cap_grid = 1;
 
-    unsigned grid_of(int64_t work) const {
-        return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
-    }
-
     // out (length 2^n) = the E-weighted sum of the rows of a rows x cols matrix
     int contract(const void* mat, int bits, const int8_t* scales, int rows, int cols, const Ext2* E, Ext2* out) {
         const int64_t pitch = bits == 4 ? (cols + 1) / 2 : cols;
@@ -271,7 +267,7 @@ struct Mm2Device : Mm2Source {
         fp_tic(c, st, K_MM2_CONTRACT, (double)rows * (double)pitch, &slot);
         e2_contract_kernel<<<grid, M2_THREADS, 0, st>>>((const uint8_t*)mat, bits, scales, rows, cols, pitch, per, E,
                                                         cpart);
-        e2_contract_finish_kernel<<<grid_of(1ll << n), 256, 0, st>>>(cpart, nchunks, cols, 1ll << n, out);
+        e2_contract_finish_kernel<<<fp_grid256(c, 1ll << n), 256, 0, st>>>(cpart, nchunks, cols, 1ll << n, out);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         c->launches++;  // two kernels under one timing slot
@@ -294,8 +290,8 @@ struct Mm2Device : Mm2Source {
         const Ext2* dzc = dzr + vM;
         int slot;
         fp_tic(c, st, K_MM2_EQ, 16.0 * (double)((1ll << vM) + (1ll << vN)), &slot);
-        e2_eq_kernel<<<grid_of(1ll << vM), 256, 0, st>>>(dzr, vM, Erow);
-        e2_eq_kernel<<<grid_of(1ll << vN), 256, 0, st>>>(dzc, vN, Ecol);
+        e2_eq_kernel<<<fp_grid256(c, 1ll << vM), 256, 0, st>>>(dzr, vM, Erow);
+        e2_eq_kernel<<<fp_grid256(c, 1ll << vN), 256, 0, st>>>(dzc, vN, Ecol);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         c->launches++;
@@ -308,7 +304,7 @@ struct Mm2Device : Mm2Source {
         const int64_t total = (int64_t)s->M * s->N;
         int slot;
         fp_tic(c, st, K_MM2_CLAIM, 8.0 * (double)total, &slot);
-        mm2_claim_kernel<<<grid_of(total), M2_THREADS, 0, st>>>(s->q, s->r, s->M, total, s->k_shift, Erow, Ecol, part,
+        mm2_claim_kernel<<<fp_grid256(c, total), M2_THREADS, 0, st>>>(s->q, s->r, s->M, total, s->k_shift, Erow, Ecol, part,
                                                                 c->tickets, small);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());

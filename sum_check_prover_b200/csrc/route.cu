@@ -266,10 +266,6 @@ struct RouteDevice : RouteSource {
     RouteArgs A;
     int cap_grid = 1;
 
-    unsigned grid_of(int64_t work) const {
-        return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
-    }
-
     void abandon() override { fp_session_abandon(c, st); }
 
     int start(const uint64_t* z, const uint64_t* w, int n, uint64_t lam1, uint64_t lam2) override {
@@ -298,12 +294,12 @@ struct RouteDevice : RouteSource {
         int slot;
         fp_tic(c, st, K_ROUTE_VECTORS, 48.0 * (double)L + 9.0 * (double)TE, &slot);
         route_prefix_kernel<<<1, 1, 0, st>>>(eqe, E, G);
-        route_vectors_kernel<<<grid_of(L), 256, 0, st>>>(l, H, TE, vE, L, et, ewt, G, V[0], V[1], V[2], V[3], V[5]);
+        route_vectors_kernel<<<fp_grid256(c, L), 256, 0, st>>>(l, H, TE, vE, L, et, ewt, G, V[0], V[1], V[2], V[3], V[5]);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         c->launches++;  // two kernels under one timing slot
         fp_tic(c, st, K_ROUTE_OPEN, 5.0 * (double)TE, &slot);
-        route_open_kernel<<<grid_of(TE), RT_THREADS, 0, st>>>(D, l, TE, EH, EL, vl, ewt, T, part, c->tickets, small);
+        route_open_kernel<<<fp_grid256(c, TE), RT_THREADS, 0, st>>>(D, l, TE, EH, EL, vl, ewt, T, part, c->tickets, small);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         memset(&A, 0, sizeof A);

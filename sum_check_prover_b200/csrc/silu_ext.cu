@@ -638,10 +638,6 @@ int lu2_protocol(fp_ctx* c, fp_tx* tx, int v, int k, const uint32_t* m_rem, cons
     return FP_OK;
 }
 
-unsigned x16_grid(const fp_ctx* c, int64_t work) {
-    return (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 4 * (int64_t)c->num_sms));
-}
-
 // Device values from the kernels above.
 struct X16Device : X16Source {
     fp_ctx* c;
@@ -664,10 +660,10 @@ struct X16Device : X16Source {
         const int64_t L = 1ll << v;
         int slot;
         fp_tic(c, st, K_X16_TREE, 4.0 * (double)n + 64.0 * (double)L, &slot);
-        x16_leaf_kernel<<<x16_grid(c, L), 256, 0, st>>>(g, s, n, L, alpha, gamma, pad_s, TP[v], TQ[v]);
+        x16_leaf_kernel<<<fp_grid256(c, L), 256, 0, st>>>(g, s, n, L, alpha, gamma, pad_s, TP[v], TQ[v]);
         FP_CUDA(c, cudaGetLastError());
         for (int d = v - 1; d >= 1; d--) {
-            x16_level_kernel<<<x16_grid(c, 1ll << d), 256, 0, st>>>(TP[d + 1], TQ[d + 1], 1ll << d, TP[d], TQ[d]);
+            x16_level_kernel<<<fp_grid256(c, 1ll << d), 256, 0, st>>>(TP[d + 1], TQ[d + 1], 1ll << d, TP[d], TQ[d]);
             FP_CUDA(c, cudaGetLastError());
             c->launches++;
         }
@@ -764,8 +760,8 @@ struct X16Device : X16Source {
             (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 2 * (int64_t)c->num_sms));
         int slot;
         fp_tic(c, st, K_X16_LEAF, 4.0 * (double)n, &slot);
-        x16_eq_kernel<<<x16_grid(c, 1ll << vh), 256, 0, st>>>(ph, EH);
-        x16_eq_kernel<<<x16_grid(c, 1ll << vl), 256, 0, st>>>(pl, EL);
+        x16_eq_kernel<<<fp_grid256(c, 1ll << vh), 256, 0, st>>>(ph, EH);
+        x16_eq_kernel<<<fp_grid256(c, 1ll << vl), 256, 0, st>>>(pl, EL);
         x16_mle_kernel<int16_t><<<blocks, 256, 0, st>>>(g, n, EH, EL, vl, part, c->tickets, small);
         x16_mle_kernel<int16_t><<<blocks, 256, 0, st>>>(s, n, EH, EL, vl, part, c->tickets, small + 4);
         fp_toc(c, st, slot);
@@ -861,12 +857,12 @@ struct Lu2Device : Lu2Source {
         const int64_t L = 1ll << v;
         int slot;
         fp_tic(c, st, K_LU2_TREE, 9.0 * (double)n + 128.0 * (double)L, &slot);
-        lu2_leaf_kernel<<<x16_grid(c, L), 256, 0, st>>>(r, q, y, n, L, alpha0, alpha1, gamma, TP[0][v], TQ[0][v],
+        lu2_leaf_kernel<<<fp_grid256(c, L), 256, 0, st>>>(r, q, y, n, L, alpha0, alpha1, gamma, TP[0][v], TQ[0][v],
                                                          TP[1][v], TQ[1][v]);
         FP_CUDA(c, cudaGetLastError());
         for (int tau = 0; tau < 2; tau++)
             for (int d = v - 1; d >= 1; d--) {
-                x16_level_kernel<<<x16_grid(c, 1ll << d), 256, 0, st>>>(TP[tau][d + 1], TQ[tau][d + 1], 1ll << d,
+                x16_level_kernel<<<fp_grid256(c, 1ll << d), 256, 0, st>>>(TP[tau][d + 1], TQ[tau][d + 1], 1ll << d,
                                                                         TP[tau][d], TQ[tau][d]);
                 FP_CUDA(c, cudaGetLastError());
                 c->launches++;
@@ -965,8 +961,8 @@ struct Lu2Device : Lu2Source {
             (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 2 * (int64_t)c->num_sms));
         int slot;
         fp_tic(c, st, K_LU2_LEAF, 9.0 * (double)n, &slot);
-        x16_eq_kernel<<<x16_grid(c, 1ll << vh), 256, 0, st>>>(ph, EH);
-        x16_eq_kernel<<<x16_grid(c, 1ll << vl), 256, 0, st>>>(pl, EL);
+        x16_eq_kernel<<<fp_grid256(c, 1ll << vh), 256, 0, st>>>(ph, EH);
+        x16_eq_kernel<<<fp_grid256(c, 1ll << vl), 256, 0, st>>>(pl, EL);
         x16_mle_kernel<int32_t><<<blocks, 256, 0, st>>>(r, n, EH, EL, vl, part, c->tickets, small);
         x16_mle_kernel<int32_t><<<blocks, 256, 0, st>>>(q, n, EH, EL, vl, part, c->tickets, small + 4);
         x16_mle_kernel<int8_t><<<blocks, 256, 0, st>>>(y, n, EH, EL, vl, part, c->tickets, small + 8);
@@ -1104,7 +1100,7 @@ int x16_prove(fp_ctx* c, fp_tx* tx, const X16Labels& lab, int64_t pad_s, const i
     {
         int slot;
         fp_tic(c, st, K_SILU_HIST, 2.0 * (double)n, &slot);
-        x16_hist_kernel<<<x16_grid(c, n), 256, 0, st>>>(g, n, m);
+        x16_hist_kernel<<<fp_grid256(c, n), 256, 0, st>>>(g, n, m);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         if (L > n) {
@@ -1246,8 +1242,8 @@ int logup_prove_rescale_ext2(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsi
     {
         int slot;
         fp_tic(c, st, K_LU2_HIST, 9.0 * (double)nk, &slot);
-        lu2_hist_kernel<<<x16_grid(c, nk), 256, 0, st>>>(r_all, nk, T, T / 2, m_rem, outside);
-        lu2_hist_clamp_kernel<<<x16_grid(c, nk), 256, 0, st>>>(q_all, y_all, nk, m_cl, outside);
+        lu2_hist_kernel<<<fp_grid256(c, nk), 256, 0, st>>>(r_all, nk, T, T / 2, m_rem, outside);
+        lu2_hist_clamp_kernel<<<fp_grid256(c, nk), 256, 0, st>>>(q_all, y_all, nk, m_cl, outside);
         if (L > nk) lu2_add_pad_kernel<<<1, 1, 0, st>>>(m_rem, T / 2, m_cl, (uint32_t)(L - nk));
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
