@@ -63,7 +63,8 @@ def _prove(env, s, seed, offline_digest=False):
 
 @pytest.mark.parametrize("M,K,N,bits,scales", [(1, 1, 1, 8, False), (1, 2, 1, 4, False), (3, 5, 2, 4, True),
                                                (64, 256, 32, 8, False), (100, 1000, 37, 4, True),
-                                               (17, 4097, 9, 8, True), (257, 300, 513, 4, False)])
+                                               (17, 1023, 9, 8, True), (17, 4097, 9, 4, True),
+                                               (257, 300, 513, 4, False)])
 def test_matches_oracle(env, M, K, N, bits, scales):
     s = _site(M, K, N, bits, scales, 500 + M + K + N)
     wit = oracle.witness(s)
@@ -72,6 +73,20 @@ def test_matches_oracle(env, M, K, N, bits, scales):
     want, wst = oracle.mm2_prove(6, s, wit)
     assert pf == want
     assert st == wst
+
+
+def test_int8_with_scales_past_the_exact_domain_is_refused(env):
+    # int8 weights times int8 scales reach 128 * 128 * 128 * K; at K = 4097 that passes 2^31, so the
+    # int32 accumulation of the witness could wrap and the call refuses the site as out of domain
+    torch, fp, ctx = env
+    s = _site(17, 4097, 9, 8, True, 41)
+    stages, keep = device.upload(workloads.Workload("mm2", 0, [s]))
+    with pytest.raises(fp.FpError) as e:
+        ctx.commit_witness(fp.Transcript(0), [stages[0][0]])
+    assert e.value.code == -2  # FP_ERR_SHAPE
+    s = _site(17, 1023, 9, 8, True, 41)  # the largest K in the domain for int8 with scales
+    stages, keep = device.upload(workloads.Workload("mm2", 0, [s]))
+    ctx.commit_witness(fp.Transcript(0), [stages[0][0]])
 
 
 def test_offline_weight_digest_gives_the_same_proof(env):
