@@ -400,11 +400,16 @@ def prove(seed: int, sites, wits):
     n = C.c_uint64(0)
     off = C.c_uint64(0)
     states = C.create_string_buffer(96)
-    rc = lib().orc_prove(seed, cs, len(sites), cw, None, 0, C.byref(n), states, C.byref(off))
-    if rc not in (0, -2):
-        raise ValueError(f"orc_prove rejected the statement ({rc})")
-    buf = np.zeros(max(1, n.value), dtype=np.uint8)
-    rc = lib().orc_prove(seed, cs, len(sites), cw, _ptr(buf), n.value, C.byref(n), states, C.byref(off))
+    # a buffer large enough for any statement's proof in one pass (the multiplicities of
+    # the two tables, 32 + 48 bytes per round and site, the layer rounds); the prover runs
+    # again only if it was not, with the size it reported
+    kmax = max(int(s.k_shift) for s in sites)
+    cap = (1 << 22) + 4 * (1 << kmax) + 64 * len(sites)
+    buf = np.zeros(cap, dtype=np.uint8)
+    rc = lib().orc_prove(seed, cs, len(sites), cw, _ptr(buf), cap, C.byref(n), states, C.byref(off))
+    if rc == -2:
+        buf = np.zeros(max(1, n.value), dtype=np.uint8)
+        rc = lib().orc_prove(seed, cs, len(sites), cw, _ptr(buf), n.value, C.byref(n), states, C.byref(off))
     if rc != 0:
         raise ValueError(f"orc_prove failed ({rc})")
     st = states.raw

@@ -667,9 +667,11 @@ typedef struct {
     u64 nk;       /* real keys */
     int v;        /* tree depth */
     int k;        /* rescale shift */
-    int64_t* fr;  /* remainder keys (padded) */
-    int64_t* fq;  /* q component (padded) */
-    int64_t* fy;  /* y component (padded) */
+    /* stored at the witness's own widths (r, q int32, y int8), so the key
+     * columns of the largest layer (2^29 keys) take 9 bytes a key */
+    int32_t* fr;  /* remainder keys (padded) */
+    int32_t* fq;  /* q component (padded) */
+    int8_t* fy;   /* y component (padded) */
 } orc_keys;
 
 static int keys_build(const orc_site* sites, int ns, const orc_wit* wit, orc_keys* K) {
@@ -685,9 +687,9 @@ static int keys_build(const orc_site* sites, int ns, const orc_wit* wit, orc_key
     K->nk = nk;
     K->v = v;
     K->k = k;
-    K->fr = (int64_t*)calloc(L, sizeof(int64_t));
-    K->fq = (int64_t*)calloc(L, sizeof(int64_t));
-    K->fy = (int64_t*)calloc(L, sizeof(int64_t));
+    K->fr = (int32_t*)calloc(L, sizeof(int32_t));
+    K->fq = (int32_t*)calloc(L, sizeof(int32_t));
+    K->fy = (int8_t*)calloc(L, sizeof(int8_t));
     u64 o = 0;
     for (int s = 0; s < ns; s++) {
         u64 mn = (u64)sites[s].M * sites[s].N;
@@ -713,7 +715,7 @@ static void mult_rem(const orc_keys* K, u32* m) {
     int64_t half = (int64_t)1 << (K->k - 1);
     memset(m, 0, T * sizeof(u32));
     for (u64 i = 0; i < L; i++) {
-        int64_t j = K->fr[i] + half;
+        int64_t j = (int64_t)K->fr[i] + half;
         if (j >= 0 && (u64)j < T) m[j]++;
     }
 }
@@ -722,7 +724,7 @@ static void mult_clamp(const orc_keys* K, u32* m) {
     u64 L = (u64)1 << K->v;
     memset(m, 0, 65536 * sizeof(u32));
     for (u64 i = 0; i < L; i++) {
-        int64_t j = K->fq[i] + 32768;
+        int64_t j = (int64_t)K->fq[i] + 32768;
         if (j >= 0 && j < 65536) m[j]++;
     }
 }
@@ -827,14 +829,21 @@ static void lu_prove(orc_tx* t, pbuf* pb, const orc_site* sites, int ns, const o
         u64 n = (u64)1 << d;
         /* vectors: for tau: pL, pR, qL, qR (children of layer d in layer d+1), then eq(z, .) */
         u64* V[9];
-        for (int i = 0; i < 9; i++) V[i] = (u64*)malloc(n * sizeof(u64));
-        for (int tau = 0; tau < 2; tau++)
+        for (int tau = 0; tau < 2; tau++) {
+            for (int i = 0; i < 4; i++) V[4 * tau + i] = (u64*)malloc(n * sizeof(u64));
             for (u64 x = 0; x < n; x++) {
                 V[4 * tau + 0][x] = T[tau].P[d + 1][2 * x];
                 V[4 * tau + 1][x] = T[tau].P[d + 1][2 * x + 1];
                 V[4 * tau + 2][x] = T[tau].Q[d + 1][2 * x];
                 V[4 * tau + 3][x] = T[tau].Q[d + 1][2 * x + 1];
             }
+            /* level d + 1 is read by no later layer: release it now, which keeps
+             * the prover of the largest layer within a workstation's memory */
+            free(T[tau].P[d + 1]);
+            free(T[tau].Q[d + 1]);
+            T[tau].P[d + 1] = T[tau].Q[d + 1] = NULL;
+        }
+        V[8] = (u64*)malloc(n * sizeof(u64));
         orc_eq_table(z, d, V[8]);
         u64 L = n;
         u64* rho = (u64*)malloc(sizeof(u64) * d);
