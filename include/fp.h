@@ -167,16 +167,20 @@ int mle_partial_eval(fp_ctx* ctx, const void* mat, int bits, const int8_t* scale
  *
  * Same arguments and result as mle_partial_eval; `out` (device) receives
  * 2^ceil(log2 cols) values. Scratch is a fixed 16 MiB device array inside the
- * library (held on every GPU that loads it until the process exits), which
+ * library (held by each GPU the entry point has run on, until the process
+ * exits), which
  * limits the shape: ceil(rows / 1024) * cols must not exceed 2^21, and
  * npoint <= 24. Larger shapes return FP_ERR_SHAPE; bad pointers or bits
  * FP_ERR_ARG; a CUDA failure FP_ERR_CUDA. The kernels are queued on `stream`
  * and the call returns without waiting: the result is ready when the stream
  * reaches that point.
  *
- * The first call on each device looks up the scratch array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture. Every call on a device shares the one scratch
+ * Every call looks up the scratch array's device address on the current
+ * device (cudaGetSymbolAddress). The CUDA runtime loads the library's modules
+ * lazily (the default since CUDA 12), so the first call on each device loads
+ * this one and reserves its 16 MiB there: make that first call outside the
+ * context that must not allocate, and before any stream capture. Later calls
+ * allocate nothing. Every call on a device shares the one scratch
  * array and leaves its contents behind; each call overwrites every entry it
  * reads, so nothing needs clearing, but calls whose kernels overlap on the GPU
  * (different streams of the same device) race on the array and must be

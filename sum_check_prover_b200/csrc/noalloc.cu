@@ -7,14 +7,15 @@
 // byte of device memory for other work. mle_partial_eval needs an fp_ctx,
 // whose scratch arena grows with cudaMalloc; this variant needs neither. Its
 // scratch is one file-scope device array of fixed size (kNoallocWords 64-bit
-// words = 16 MiB), which every GPU that loads the library holds until the
-// process exits.
+// words = 16 MiB). The CUDA runtime loads this file's module on a device the
+// first time it is used there (lazy loading, the default since CUDA 12): that
+// first call reserves the 16 MiB, which the device then holds until the
+// process exits. Make the first call on each device outside the context that
+// must not allocate.
 //
 // The caller still passes the matrix, the point and the output buffer. The
 // result is the same as mle_partial_eval's: out[c] = sum_i eq(point, i) *
 // M_eff[i][c], with M_eff = scales[i][c/64] * mat[i][c] when scales are given.
-#include <mutex>
-
 #include "fp_field.cuh"
 #include "fp_internal.h"
 
@@ -24,7 +25,6 @@ constexpr int kNaThreads = 128;
 constexpr int kNaCols = 8;                  // columns per thread
 constexpr int kNaRows = 1024;               // rows per split (block), eq of those rows kept in shared memory
 constexpr uint64_t kNoallocWords = 1u << 21;  // 16 MiB of per-split column partials
-constexpr int kMaxDevices = 64;
 
 // The scratch array. Host code must not pass its name to a kernel (on the host
 // the name is only a stand-in for the device symbol); the entry point passes
@@ -114,24 +114,16 @@ __global__ void pe_noalloc_fin_kernel(const uint64_t* __restrict__ part, int spl
     out[c] = a;
 }
 
-std::mutex g_setup_mu;
-uint64_t* g_scratch_addr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch array on the current device; looked up once per device.
+// Device address of the scratch array in the current device's context. Looked
+// up on every call (once the module is loaded the lookup allocates nothing), so
+// a context that was torn down and created again never gets a stale address.
 int scratch_for_current_device(uint64_t** ptr) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FP_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return FP_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return FP_ERR_CUDA;
-        }
-        g_scratch_addr[dev] = (uint64_t*)p;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return FP_ERR_CUDA;
     }
-    *ptr = g_scratch_addr[dev];
+    *ptr = (uint64_t*)p;
     return FP_OK;
 }
 

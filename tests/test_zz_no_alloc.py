@@ -64,21 +64,52 @@ def _regular(torch, ctx, mat, bits, sc, rows, cols, z):
     return out.cpu().numpy().view(np.uint64)
 
 
-def test_no_alloc_matches_regular_entry_point_twice(env):
+# int4 and int8, with and without per-64 scales (int8 with scales adds the largest offset,
+# 2^14, over up to 1024 rows per split); rows a multiple of 1024 and ragged; columns below
+# and above one block's 1024 and not a multiple of it
+CASES = [(1, 3000, 4096, 4, False), (2, 1500, 1000, 4, True), (3, 70, 517, 8, False),
+         (4, 2048, 1000, 8, True), (5, 1024, 1031, 8, False)]
+
+
+@pytest.mark.parametrize("seed,rows,cols,bits,scaled", CASES)
+def test_no_alloc_matches_regular_entry_point_twice(env, seed, rows, cols, bits, scaled):
     torch, fp, L, ctx = env
-    # two different statements back to back: the first leaves the scratch full
-    cases = [(1, 3000, 4096, 4, False), (2, 1500, 1000, 4, True), (3, 70, 517, 8, False)]
-    for seed, rows, cols, bits, scaled in cases:
-        mat, sc, z = _case(seed, rows, cols, bits, scaled)
-        dm = torch.from_numpy(mat).cuda()
-        ds = None if sc is None else torch.from_numpy(sc).cuda()
-        rc1, a = _noalloc(torch, L, dm, bits, ds, rows, cols, z)
-        want = _regular(torch, ctx, dm, bits, ds, rows, cols, z)
-        assert rc1 == 0
-        assert np.array_equal(a, want)
-        rc2, b = _noalloc(torch, L, dm, bits, ds, rows, cols, z)
-        assert rc2 == 0
-        assert np.array_equal(b, want)
+    mat, sc, z = _case(seed, rows, cols, bits, scaled)
+    dm = torch.from_numpy(mat).cuda()
+    ds = None if sc is None else torch.from_numpy(sc).cuda()
+    rc1, a = _noalloc(torch, L, dm, bits, ds, rows, cols, z)
+    want = _regular(torch, ctx, dm, bits, ds, rows, cols, z)
+    assert rc1 == 0
+    assert np.array_equal(a, want)
+    # the second call in a row finds the first call's partials in the shared scratch
+    rc2, b = _noalloc(torch, L, dm, bits, ds, rows, cols, z)
+    assert rc2 == 0
+    assert np.array_equal(b, want)
+    if rows * cols <= 1 << 21:  # and both equal the CPU oracle's partial evaluation
+        assert np.array_equal(a, oracle.partial_rows(mat, bits, sc, rows, cols, z))
+
+
+def test_no_alloc_allocates_nothing_after_the_first_call(env):
+    torch, fp, L, ctx = env
+    rows, cols, bits = 2000, 3000, 4
+    mat, sc, z = _case(7, rows, cols, bits, True)
+    dm = torch.from_numpy(mat).cuda()
+    ds = torch.from_numpy(sc).cuda()
+    out = torch.zeros((1 << oracle.log2_ceil(cols),), dtype=torch.int64, device="cuda")
+    pt = (C.c_uint64 * len(z))(*z)
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def call():
+        rc = L.mle_partial_eval_noalloc(dm.data_ptr(), bits, ds.data_ptr(), rows, cols, pt, len(z),
+                                        out.data_ptr(), stream)
+        torch.cuda.synchronize()
+        return rc
+
+    assert call() == 0  # the first call on this device loads the module (and its 16 MiB array)
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    assert call() == 0
+    assert call() == 0
+    assert torch.cuda.mem_get_info()[0] == free0 and torch.cuda.memory_allocated() == alloc0
 
 
 def test_no_alloc_rejects_shapes_beyond_its_scratch(env):
