@@ -4,10 +4,12 @@
 One step = one whole proof of one synthetic statement: witness + commitment
 (fp_commit_witness), batched matmul sum-check (sumcheck_prove_matmul) and the
 LogUp rescale/clamp proof (logup_prove_rescale), from a fresh transcript.
-Default workload: one projection, W 4096x4096 int4, X 4096x512 int8
-activations ~ round(N(0,32)), rescale by 2^12 (8.6e9 MACs).
+Default workload (--config 5): the MoE layer, 128 experts of 5120 -> 8192 ->
+5120 int4 (gate, up, down) with 8192 tokens routed top-1 and a shared expert of
+the same shape, rescale by 2^12: 387 sites, 2.06e12 MACs, 3.5e8 lookup keys.
+--config 2 is the single projection (W 4096x4096 int4, X 4096x512, 8.6e9 MACs).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
 
 Prints one JSON line (rank 0). value = proved MACs/s of the whole job with
 inputs resident in HBM; e2e = the same through the public API with the
@@ -37,7 +39,7 @@ sys.path.insert(0, str(ROOT))
 
 METRIC = "proved matmul MACs/s and sum-check Melem/s at 1 B200; HBM GB/s vs peak"
 UNIT = "MAC/s"
-CONFIG = 2
+DEFAULT_CONFIG = 5
 FLUSH_BYTES = 512 << 20  # > 126 MB L2
 
 # kernel -> source file (traffic counters are valid only for the source they were taken on)
@@ -63,6 +65,38 @@ def peaks() -> dict:
         d = json.loads(p.read_text())
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "src": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "src": "fallback"}
+
+
+def host_cpu() -> dict:
+    """The host's logical core count and CPU model (for the oracle baseline)."""
+    model = None
+    try:
+        for ln in Path("/proc/cpuinfo").read_text().splitlines():
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+def cpu_sample(config: int, seed: int, step: int = 0):
+    """A bounded sample of the configuration's statement for the single-threaded oracle
+    (about 10-20 s of CPU work), and what it is. The sample's sites are the workload's
+    own sites, drawn from the same seeds."""
+    import workloads
+    if config in (1, 2):
+        return workloads.build(config, seed=seed), "the whole statement (witness + full proof)"
+    if config == 5:
+        e = [step % 128]
+        wl = workloads.build(5, seed=seed, experts=e, shared=False)
+        return wl, (f"the sites of expert {e[0]} of the MoE layer (gate, up, down: 3 of 387 sites, "
+                    f"{wl.macs:.3g} MACs, {wl.n_keys} keys), witness + full proof of that sub-statement")
+    if config == 3:
+        wl = workloads.build(3, seed=seed, T=128)
+        return wl, "the FFN with 128 of its 4096 tokens (same weights), witness + full proof"
+    wl = workloads.build(4, seed=seed, B=2)
+    return wl, "the decode layer with 2 of its 64 requests (same weights), witness + full proof"
 
 
 def sumcheck_elems(wl) -> int:
@@ -241,7 +275,6 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
         gbs = by / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
         out[name] = {"kernel": kernel, "launches": len(sel), "ms": ms, "bytes": by, "GBps": gbs,
                      "frac": gbs / pk["hbm_gbs"], "peak": pk["hbm_gbs"],
-                     "per_launch": [[round(r[1], 4), r[2]] for r in sel],
                      "all_launches": len(log), "all_ms": sum(r[1] for r in log)}
 
     which = micro_names(which)
@@ -461,34 +494,41 @@ PAGES_CONTEXT = {
 
 
 def run_reference(args):
-    """The CPU oracle as it stands, on a bounded sample of the same workload."""
+    """The CPU oracle as it stands, each step on a bounded sample of the same workload."""
     world, rank, local = dist()
     if rank != 0:
         return
     import oracle
-    import workloads
-    rows = args.ref_rows
-    wl = workloads.build(CONFIG, seed=args.seed, M=rows)
-    macs = wl.macs
-    times = []
+    times, macs_done, label = [], 0, ""
     for i in range(args.warmup + args.steps):
+        wl, label = cpu_sample(args.config, args.seed, i)
         t0 = time.perf_counter()
         R = oracle.resolve(wl)
-        proof, states, _ = oracle.prove(args.seed, R.sites, R.wits)
+        oracle.prove(args.seed, R.sites, R.wits)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
+            macs_done += wl.macs
+    value = macs_done / sum(times)
     per = statistics.mean(times)
-    value = macs / per
-    sample = (f"projection with W {rows}x4096 int4 (rows sampled from the 4096x4096 statement), X 4096x512, "
-              f"k=12: witness + full proof per step, single thread")
+    full = workloads_description(args.config)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
-            "config": {"workload": "projection W 4096x4096 int4, X 4096x512 int8 N(0,32), k=12", "sample_rows": rows},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "config": {"workload": full, "config": args.config, "sample": label},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {label}; single-threaded C", **host_cpu()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def workloads_description(config: int) -> str:
+    return {1: "tiny matmul W 64x64 int8, X 64x16 int8, k=7",
+            2: "projection W 4096x4096 int4, X 4096x512 int8 N(0,32), k=12",
+            3: "dense FFN d=4096 ffn=14336 T=4096 int4 + per-64 int8 scales, k=18 (3 sites)",
+            4: "decode layer d=5120, 40/8 heads x 128, B=64, ctx 2048, MLP 16384, int4, k=12 (1031 sites)",
+            5: "MoE layer: 128 experts 5120->8192->5120 int4 (gate/up/down), T=8192 top-1 routed, "
+               "shared expert, k=12 (387 sites)"}[config]
 
 
 def run_ours(args):
@@ -511,7 +551,7 @@ def run_ours(args):
 
     dev = torch.device(f"cuda:{local}")
     # every rank proves its own independent statement (weak scaling, no data-path collective)
-    wl = workloads.build(CONFIG, seed=args.seed + rank)
+    wl = workloads.build(args.config, seed=args.seed + rank)
     macs = wl.macs
     elems = sumcheck_elems(wl)
     ctx = fp.Context(local)
@@ -587,14 +627,33 @@ def run_ours(args):
                         "GBps": (v[2] / (v[1] * 1e-3) / 1e9) if v[1] > 0 else None} for k, v in sstats.items()}
     dom = max(tstats.items(), key=lambda kv: kv[1][1])
     pk = peaks()
+    # the scope table's HBM-bound rows inside this proof: algorithmic bytes over device time,
+    # each round alone (stepped pass) and as launched in the timed configuration (a resident
+    # sum-check launch spans its rounds and their host exchanges)
+    rows = {}
+    for row, kn in (("a4_claim", "claim"), ("a5_partial_eval", "partial_acc"), ("a7_matmul_rounds", "sc_round"),
+                    ("a8_histogram", "hist"), ("a9_tree", "tree_up"), ("a10_gkr_rounds", "gkr_round"),
+                    ("a11_leaf_claims", "leaf_eval")):
+        if kn not in sstats:
+            continue
+        n_, ms_, by_ = sstats[kn]
+        gbs = by_ / (ms_ * 1e-3) / 1e9 if ms_ > 0 else 0.0
+        ent = {"kernel": kn, "bytes_per_step": by_ / args.prof_steps, "ms_per_step": ms_ / args.prof_steps,
+               "GBps": gbs, "frac": gbs / pk["hbm_gbs"]}
+        if kn in tstats and tstats[kn][1] > 0:
+            ent["GBps_as_launched"] = tstats[kn][2] / (tstats[kn][1] * 1e-3) / 1e9
+        rows[row] = ent
     dname, (dl, dms, dbytes) = dom
     avg_ms = dms / dl
-    traffic = None
+    traffic, traffic_note = None, None
     tf = ROOT / "profiles" / "traffic.json"
     if tf.exists():
         t = json.loads(tf.read_text()).get(dname)
-        if t and t.get("src") == src_hash(dname) and t.get("workload") == "projection":
-            traffic = t.get("bytes_per_launch")
+        if t and t.get("src") == src_hash(dname) and t.get("ratio") is not None:
+            # DRAM bytes over algorithmic bytes, from an ncu capture of the same kernel
+            # source on a smaller case; scaled to this launch's algorithmic bytes
+            traffic = t["ratio"] * dbytes / dl
+            traffic_note = t.get("note")
     if dname == "witness_gemm":
         flops = 2.0 * macs / (dl / args.steps)
         peak = pk["bf16_tflops"] * 2.0
@@ -602,10 +661,13 @@ def run_ours(args):
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": traffic, "kernel": dname,
                 "peak_note": f"int8 = {pk['src']} bf16 x 2 (nominal int8/bf16 ratio)"}
+        if traffic_note:
+            roof["traffic_note"] = traffic_note
     else:
         achieved = (dbytes / dl) / (avg_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "kernel": dname,
+                "traffic_note": traffic_note,
                 "avg_launch_us": avg_ms * 1e3, "bytes_per_launch": dbytes / dl,
                 "peak_note": f"{pk['src']} copy bandwidth",
                 "measured": "CUDA events around each launch, in a pass of the timed steps' inputs and "
@@ -614,7 +676,12 @@ def run_ours(args):
 
     # ---- e2e pass: activations from pinned host memory, layer output read back ----------
     flat = [d for st in stages for d in st]
-    host_x = [(d, d.xt.cpu().pin_memory()) for d in flat]
+    seen = set()
+    host_x = []
+    for d in flat:  # one copy per activation tensor (the gate and up sites share theirs)
+        if d.xt.data_ptr() not in seen:
+            seen.add(d.xt.data_ptr())
+            host_x.append((d, d.xt.cpu().pin_memory()))
     host_y = [(d, torch.empty(d.y.shape, dtype=torch.int8).pin_memory()) for d in flat]
     h2d = sum(x.numel() for _, x in host_x)
     d2h = sum(y.numel() for _, y in host_y) + proof_len
@@ -638,12 +705,13 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
+        swl, label = cpu_sample(args.config, args.seed, 0)
         t0 = time.perf_counter()
-        R = oracle.resolve(wl)
+        R = oracle.resolve(swl)
         oracle.prove(args.seed, R.sites, R.wits)
         dt = time.perf_counter() - t0
-        cpu = {"value": macs / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "the whole statement once (witness + proof), single-threaded C", "seconds": dt}
+        cpu = {"value": swl.macs / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{label}; single-threaded C", "seconds": dt, **host_cpu()}
 
     micro = None
     if rank == 0 and world == 1 and not args.no_micro:
@@ -654,10 +722,12 @@ def run_ours(args):
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "u64", "data": "synthetic",
-                "config": {"workload": "projection W 4096x4096 int4, X 4096x512 int8 N(0,32), k=12",
-                           "M": 4096, "K": 4096, "N": 512, "macs_per_step": macs,
-                           "l2": "flushed between timed steps (512 MiB write)",
+                "config": {"workload": workloads_description(args.config), "config": args.config,
+                           "sites": len(wl.sites), "macs_per_step": macs, "lookup_keys_per_step": wl.n_keys,
+                           "l2": "flushed between timed steps (512 MiB write); inputs also exceed L2"
+                                 if wl.n_keys * 9 > (126 << 20) else "flushed between timed steps (512 MiB write)",
                            "parallelism": f"{world} independent statements, one per GPU"},
+                "rows": rows,
                 "sumcheck_melem_s": world * elems * args.steps / (total_ms / 1e3) / 1e6,
                 "sumcheck_elems_per_step": elems,
                 "roofline": roof,
@@ -687,7 +757,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--prof-steps", type=int, default=3)
-    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5],
+                    help="the statement one step proves (5: the MoE layer, the largest one-GPU configuration)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-micro", action="store_true")
     ap.add_argument("--micro-only", nargs="?", const=MICRO_ALL, default=None,

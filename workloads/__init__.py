@@ -154,25 +154,31 @@ def _dense_ffn(seed: int, d=4096, ffn=14336, T=4096, k=18) -> Workload:
                     description=f"d={d} ffn={ffn} T={T} int4+scales k={k}")
 
 
-def _moe(seed: int, E=128, d=5120, ffn=8192, T=8192, k=12) -> Workload:
-    """Top-1 routed MoE with a shared expert; every matmul its own site."""
+def _moe(seed: int, E=128, d=5120, ffn=8192, T=8192, k=12, experts=None, shared=True) -> Workload:
+    """Top-1 routed MoE with a shared expert; every matmul its own site.
+
+    ``experts`` (a list of expert indices) and ``shared`` keep only those
+    experts' sites: the same tensors, drawn from the same seeds, as in the
+    whole layer (a sample of the layer's sites for a CPU timing)."""
     x = activations(_rng(seed, 100), (T, d))
     route = _rng(seed, 99).integers(0, E, size=T)
+    keep = set(range(E)) if experts is None else set(int(e) for e in experts)
     sites = []
     for e in range(E):
         idx = np.nonzero(route == e)[0]
         ne = len(idx)
-        if ne == 0:
+        if ne == 0 or e not in keep:
             continue
         xe = np.ascontiguousarray(x[idx])
         he = activations(_rng(seed, 1000 + 10 * e), (ne, ffn))
         for j, (nm, M, K, xt) in enumerate([("gate", ffn, d, xe), ("up", ffn, d, xe), ("down", d, ffn, he)]):
             sites.append(Site(f"e{e}.{nm}", M, K, ne, 4, k,
                               w=int4_packed(_rng(seed, 1000 + 10 * e + 1 + j), M, K), xt=xt))
-    hs = activations(_rng(seed, 200), (T, ffn))
-    for j, (nm, M, K, xt) in enumerate([("gate", ffn, d, x), ("up", ffn, d, x), ("down", d, ffn, hs)]):
-        sites.append(Site(f"shared.{nm}", M, K, T, 4, k,
-                          w=int4_packed(_rng(seed, 300 + j), M, K), xt=xt))
+    if shared:
+        hs = activations(_rng(seed, 200), (T, ffn))
+        for j, (nm, M, K, xt) in enumerate([("gate", ffn, d, x), ("up", ffn, d, x), ("down", d, ffn, hs)]):
+            sites.append(Site(f"shared.{nm}", M, K, T, 4, k,
+                              w=int4_packed(_rng(seed, 300 + j), M, K), xt=xt))
     return Workload("moe", seed, sites,
                     description=f"{E} experts d={d} ffn={ffn} T={T} top-1 + shared, k={k}")
 
