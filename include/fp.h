@@ -204,6 +204,54 @@ int sumcheck_prove_matmul(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsit
                           size_t* proof_len, void* stream);
 
 /*
+ * One statement proven by several ranks, one process per GPU ("How fast can
+ * FlashProve go", 4 Tighter Rooflines: the work spread over the GPUs of one
+ * node). The sites are independent until their claims are combined, so rank r
+ * proves the sites [site_lo[r], site_lo[r + 1]) -- their witness, digests,
+ * claims, partial evaluations and their share of every round -- and the ranks
+ * exchange only small values through the caller's all-gather: the 192-byte
+ * site records, the claims, each round's partial g(0), g(2) (16 bytes per
+ * rank), and the final values. Every rank then absorbs the same values in the
+ * same order, so all ranks hold one transcript and write the proof bytes of
+ * the one-rank statement.
+ *
+ * allgather(user, mine, bytes, all): every rank passes `bytes` bytes (the same
+ * count on every rank in every call); `all` (host, world * bytes) receives the
+ * ranks' bytes in rank order. Returns 0, or nonzero to stop the call with
+ * FP_ERR_ARG. Every rank must make the same calls in the same order.
+ * site_lo: host, world + 1 entries, site_lo[0] = 0, site_lo[world] = nsites,
+ * non-decreasing, every rank owning at least one site.
+ */
+typedef int (*fp_allgather_fn)(void* user, const void* mine, size_t bytes, void* all);
+typedef struct {
+    int rank;
+    int world;
+    const int* site_lo;
+    fp_allgather_fn allgather;
+    void* user;
+} fp_shard;
+
+/*
+ * fp_commit_witness for a statement shared among ranks: computes the witness
+ * and the digests of this rank's sites only, gathers every rank's 192-byte
+ * site records and absorbs all of them in site order. sites: all nsites
+ * descriptors; shapes are read for every site, device pointers only for this
+ * rank's sites. Errors as for fp_commit_witness; a failed all-gather returns
+ * FP_ERR_ARG.
+ */
+int fp_commit_witness_shard(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites, const fp_shard* shard,
+                            void* stream);
+
+/*
+ * sumcheck_prove_matmul for a statement shared among ranks: this rank's claims,
+ * partial evaluations and round shares are computed from its own sites; the
+ * proof and the transcript are those of the one-rank call, on every rank.
+ * sites as for fp_commit_witness_shard. Errors as for sumcheck_prove_matmul.
+ */
+int sumcheck_prove_matmul_shard(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites, const fp_shard* shard,
+                                uint8_t* proof, size_t* proof_len, void* stream);
+
+/*
  * LogUp proof of every site's rescale remainder and clamp ("How fast can
  * FlashProve go", 3.1 and 4; "Towards Proving Frontier-Scale LLM Inference",
  * The proof system). Keys: all outputs in storage order, sites concatenated,
@@ -270,7 +318,8 @@ enum {
     FP_VAL_ANSWER = 3,  /* round t's challenge */
     FP_VAL_FINALS = 4,  /* the final values */
     FP_VAL_COLUMN = 5,  /* a committed column is formed: its digest */
-    FP_VAL_CLAIM = 6    /* the claim the rounds start from */
+    FP_VAL_CLAIM = 6,   /* the claim the rounds start from */
+    FP_VAL_WEIGHTS = 7  /* the batching weights of the caller's sites */
 };
 typedef int (*fp_values_fn)(void* user, int kind, int t, const uint64_t* in, uint64_t* out);
 
@@ -406,6 +455,23 @@ int freivalds_prove_matmul(fp_ctx* ctx, fp_tx* tx, const fp_site* site, uint8_t*
  */
 int fp_mm2_protocol_drive(fp_tx* tx, int vM, int vN, int n, fp_values_fn fn, void* user, uint8_t* proof,
                           size_t* proof_len);
+
+/*
+ * The host half of sumcheck_prove_matmul_shard (and, with shard NULL, of
+ * sumcheck_prove_matmul): tx must have absorbed the site records. sites: all
+ * nsites descriptors, only their shapes read. Callback kinds, for this rank's
+ * own sites (own = site_lo[rank + 1] - site_lo[rank], all sites with no shard):
+ *   FP_VAL_START: in = r_row then r_col (vM + vN words), t = vM + vN;
+ *   FP_VAL_CLAIM: out = c_s of the own sites (own words), t = own;
+ *   FP_VAL_WEIGHTS: in = rho_s of the own sites (own words), t = own;
+ *   FP_VAL_ROUND: out = this rank's share of g_t(0), g_t(2) (2 words): the
+ *     sums over its own sites of rho_s sum_b A_s(X, b) B_s(X, b) at X = 0, 2;
+ *   FP_VAL_ANSWER: in = r_t (1 word);
+ *   FP_VAL_FINALS: out = A_s(rho), B_s(rho) of the own sites (2 own words).
+ * The proof and proof_len are as for sumcheck_prove_matmul.
+ */
+int fp_mm_shard_protocol_drive(fp_tx* tx, const fp_site* sites, int nsites, const fp_shard* shard, fp_values_fn fn,
+                               void* user, uint8_t* proof, size_t* proof_len);
 
 /*
  * MoE routing, top-1 ("How fast can FlashProve go", 2 Background, the note on MoE

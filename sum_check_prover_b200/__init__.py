@@ -14,7 +14,8 @@ import ctypes as C
 from pathlib import Path
 from typing import Optional, Sequence
 
-__all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "lib", "LIB_PATH", "kernel_names", "P",
+__all__ = ["FpError", "Context", "Transcript", "SiteDesc", "prove", "prove_shard", "Shard", "lib", "LIB_PATH",
+           "kernel_names", "P",
            "had2_protocol_drive", "lhi_protocol_drive", "mm2_protocol_drive", "route_protocol_drive",
            "lhi2_protocol_drive", "lookup16x_protocol_drive", "lu2_protocol_drive"]
 
@@ -98,6 +99,11 @@ def lib():
     L.logup_prove_exp.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_exp_table.argtypes = [vp]
     L.fp_proof_size.argtypes = [C.POINTER(_Site), i32, C.POINTER(sz), C.POINTER(sz)]
+    L.fp_commit_witness_shard.argtypes = [vp, vp, C.POINTER(_Site), i32, C.POINTER(_Shard), vp]
+    L.sumcheck_prove_matmul_shard.argtypes = [vp, vp, C.POINTER(_Site), i32, C.POINTER(_Shard), vp, C.POINTER(sz),
+                                              vp]
+    L.fp_mm_shard_protocol_drive.argtypes = [vp, C.POINTER(_Site), i32, C.POINTER(_Shard), _VALUES_FN, vp, vp,
+                                             C.POINTER(sz)]
     L.fp_ctx_set_profiling.argtypes = [vp, i32]
     L.fp_session_selftest.argtypes = [vp, vp]
     L.fp_host_stats.argtypes = [vp, C.POINTER(C.c_double)]
@@ -114,7 +120,120 @@ def lib():
 
 # int (*)(void* user, int kind, int t, const uint64_t* in, uint64_t* out)
 _VALUES_FN = C.CFUNCTYPE(C.c_int, C.c_void_p, C.c_int, C.c_int, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64))
-VAL_START, VAL_SINGLE, VAL_ROUND, VAL_ANSWER, VAL_FINALS, VAL_COLUMN, VAL_CLAIM = range(7)
+VAL_START, VAL_SINGLE, VAL_ROUND, VAL_ANSWER, VAL_FINALS, VAL_COLUMN, VAL_CLAIM, VAL_WEIGHTS = range(8)
+
+# int (*)(void* user, const void* mine, size_t bytes, void* all)
+_ALLGATHER_FN = C.CFUNCTYPE(C.c_int, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p)
+
+
+class _Shard(C.Structure):
+    _fields_ = [("rank", C.c_int32), ("world", C.c_int32), ("site_lo", C.POINTER(C.c_int32)),
+                ("allgather", _ALLGATHER_FN), ("user", C.c_void_p)]
+
+
+class Shard:
+    """This rank's share of one statement proven by several ranks: rank r proves the
+    sites [site_lo[r], site_lo[r + 1]). `allgather(data: bytes) -> list of bytes` returns
+    every rank's bytes in rank order (the same length on every rank)."""
+
+    def __init__(self, rank: int, world: int, site_lo: Sequence[int], allgather):
+        self.rank, self.world, self.site_lo = int(rank), int(world), [int(x) for x in site_lo]
+
+        def cb(_user, mine, nbytes, out):
+            try:
+                parts = allgather(C.string_at(mine, nbytes))
+                if len(parts) != world or any(len(p) != nbytes for p in parts):
+                    return 1
+                C.memmove(out, b"".join(parts), nbytes * world)
+                return 0
+            except Exception:  # reported to the caller as FP_ERR_ARG
+                return 1
+
+        self._fn = _ALLGATHER_FN(cb)
+        self._lo = (C.c_int32 * (world + 1))(*self.site_lo)
+        self.c = _Shard(self.rank, self.world, self._lo, self._fn, None)
+
+    @property
+    def own(self) -> range:
+        return range(self.site_lo[self.rank], self.site_lo[self.rank + 1])
+
+
+def torch_allgather(group=None):
+    """An all-gather of small host byte strings over a torch.distributed process group
+    (gloo, or a gloo group beside NCCL): the host-mediated exchange of a shared statement."""
+    import torch
+    import torch.distributed as td
+
+    def ag(data: bytes):
+        world = td.get_world_size(group)
+        mine = torch.frombuffer(bytearray(data), dtype=torch.uint8) if data else torch.zeros(0, dtype=torch.uint8)
+        out = [torch.empty(len(data), dtype=torch.uint8) for _ in range(world)]
+        td.all_gather(out, mine, group=group)
+        return [bytes(t.numpy().tobytes()) for t in out]
+
+    return ag
+
+
+def balance_sites(costs: Sequence[float], world: int) -> list:
+    """Contiguous site ranges, one per rank, with about equal cost each (every rank at
+    least one site): the site_lo array of a Shard."""
+    n = len(costs)
+    if world < 1 or n < world:
+        raise ValueError("balance_sites: need at least one site per rank")
+    total = float(sum(costs))
+    lo, acc, r = [0], 0.0, 1
+    for i, c in enumerate(costs):
+        acc += c
+        # close rank r's range once it holds its share, leaving a site for every later rank
+        while r < world and acc >= total * r / world and i + 1 <= n - (world - r):
+            lo.append(i + 1)
+            r += 1
+    while len(lo) < world:
+        lo.append(n - (world - len(lo)))
+    lo.append(n)
+    return lo
+
+
+def mm_shard_protocol_drive(tx: "Transcript", sites: Sequence["SiteDesc"], shard: Optional[Shard], values) -> bytes:
+    """Run the host half of the (sharded) matmul sum-check with this rank's device values
+    taken from `values` (no GPU work): values.start(r_row, r_col), values.claims() -> the own
+    sites' c_s, values.weights(rho_own), values.round(t) -> (g(0), g(2)) share,
+    values.answer(t, r), values.finals() -> [A_s, B_s, ...] of the own sites. tx must have
+    absorbed the site records. Only the sites' shapes are read."""
+    L = lib()
+    arr, keep = _sites(sites)
+    own = len(sites) if shard is None else len(shard.own)
+    vM = max((s.M - 1).bit_length() for s in sites)
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            if kind == VAL_START:
+                pts = [int(inp[i]) for i in range(t)]
+                values.start(pts[:vM], pts[vM:])
+                return 0
+            if kind == VAL_WEIGHTS:
+                values.weights([int(inp[i]) for i in range(t)])
+                return 0
+            if kind == VAL_ANSWER:
+                values.answer(t, int(inp[0]))
+                return 0
+            res = {VAL_CLAIM: values.claims, VAL_FINALS: values.finals}.get(kind)
+            res = values.round(t) if kind == VAL_ROUND else res()
+            for i, x in enumerate(res):
+                out[i] = int(x) % P
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _VALUES_FN(cb)
+    ln = C.c_size_t(0)
+    sh = None if shard is None else C.byref(shard.c)
+    L.fp_mm_shard_protocol_drive(tx.h, arr, len(sites), sh, fn, None, None, C.byref(ln))
+    buf = C.create_string_buffer(max(1, ln.value))
+    rc = L.fp_mm_shard_protocol_drive(tx.h, arr, len(sites), sh, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_mm_shard_protocol_drive failed")
+    return buf.raw[: ln.value]
 
 
 def had2_protocol_drive(tx: "Transcript", v: int, values) -> bytes:
@@ -563,6 +682,24 @@ class Context:
                     "sumcheck_prove_matmul")
         return buf.raw[: n.value]
 
+    def commit_witness_shard(self, tx: Transcript, sites: Sequence[SiteDesc], shard: Shard, stream=None):
+        """fp_commit_witness for this rank's sites of a shared statement; every rank absorbs
+        all site records. Only this rank's sites need device tensors."""
+        arr, keep = _sites(sites)
+        self._check(self._L.fp_commit_witness_shard(self.h, tx.h, arr, len(sites), C.byref(shard.c),
+                                                    _stream(stream)), "fp_commit_witness_shard")
+
+    def prove_matmul_shard(self, tx: Transcript, sites: Sequence[SiteDesc], shard: Shard, stream=None) -> bytes:
+        """The matmul sum-check of a shared statement: this rank's sites on this GPU, the
+        round sums exchanged; every rank returns the one-rank proof bytes."""
+        arr, keep = _sites(sites)
+        mm, _ = self.proof_size(sites)
+        buf = C.create_string_buffer(max(1, mm))
+        n = C.c_size_t(mm)
+        self._check(self._L.sumcheck_prove_matmul_shard(self.h, tx.h, arr, len(sites), C.byref(shard.c), buf,
+                                                        C.byref(n), _stream(stream)), "sumcheck_prove_matmul_shard")
+        return buf.raw[: n.value]
+
     def prove_hadamard(self, tx: Transcript, s, u, stream=None) -> bytes:
         """Sum-check proof for the gated product of two device int8 tensors of equal size
         (flattened row-major); continues tx."""
@@ -807,6 +944,68 @@ def prove(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], stream=
         return mm + lu, [s0, s1, tx.state()], status
     finally:
         tx.close()
+
+
+def prove_shard(ctx: Context, seed: int, sites: Sequence[SiteDesc], shard: Shard, gather_witness, stream=None):
+    """Prove one layer statement shared among ranks (one stage, sites independent): this
+    rank commits and folds its own sites, the ranks exchange the round sums, then
+    gather_witness(sites) -> sites with every site's q, r, y on this device, and the
+    lookup section runs over all keys. Every rank returns the one-rank proof, states and
+    status."""
+    tx = Transcript(seed)
+    try:
+        ctx.commit_witness_shard(tx, sites, shard, stream)
+        s0 = tx.state()
+        mm = ctx.prove_matmul_shard(tx, sites, shard, stream)
+        s1 = tx.state()
+        full = gather_witness(sites)
+        lu, status = ctx.prove_logup(tx, full, stream)
+        return mm + lu, [s0, s1, tx.state()], status
+    finally:
+        tx.close()
+
+
+def torch_gather_witness(shard: Shard, group=None):
+    """gather_witness for prove_shard over a torch.distributed group whose backend moves
+    device tensors (NCCL): every rank's q, r, y, concatenated per rank, all-gathered into
+    fresh device buffers, and the sites pointed at them."""
+    import torch
+    import torch.distributed as td
+
+    def gather(sites):
+        dev = next(s.q for s in sites[shard.site_lo[shard.rank]:shard.site_lo[shard.rank + 1]]).device
+        sizes = [sum(sites[i].M * sites[i].N for i in range(shard.site_lo[r], shard.site_lo[r + 1]))
+                 for r in range(shard.world)]
+        most = max(sizes)
+        mine_qr = torch.zeros(2 * most, dtype=torch.int32, device=dev)
+        mine_y = torch.zeros(max(1, most), dtype=torch.int8, device=dev)
+        o = 0
+        for i in shard.own:
+            n = sites[i].M * sites[i].N
+            mine_qr[o:o + n] = sites[i].q.reshape(-1)
+            mine_qr[most + o:most + o + n] = sites[i].r.reshape(-1)
+            mine_y[o:o + n] = sites[i].y.reshape(-1)
+            o += n
+        all_qr = torch.empty(shard.world * 2 * most, dtype=torch.int32, device=dev)
+        all_y = torch.empty(shard.world * max(1, most), dtype=torch.int8, device=dev)
+        td.all_gather_into_tensor(all_qr, mine_qr, group=group)
+        td.all_gather_into_tensor(all_y, mine_y, group=group)
+        out = []
+        for r in range(shard.world):
+            o = 0
+            for i in range(shard.site_lo[r], shard.site_lo[r + 1]):
+                s = sites[i]
+                n = s.M * s.N
+                base = r * 2 * most
+                d = SiteDesc(s.w, s.xt, all_qr[base + o:base + o + n].view(s.N, s.M),
+                             all_qr[base + most + o:base + most + o + n].view(s.N, s.M),
+                             all_y[r * max(1, most) + o:r * max(1, most) + o + n].view(s.N, s.M),
+                             s.M, s.K, s.N, s.w_bits, s.k_shift, s.scales, s.w_digest)
+                out.append(d)
+                o += n
+        return out
+
+    return gather
 
 
 def silu_table():

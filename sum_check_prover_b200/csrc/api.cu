@@ -408,6 +408,24 @@ const char* fp_kernel_name(int k) {
 // ---------------------------------------------------------------------------
 
 int fp_check_sites(fp_ctx* c, const fp_site* sites, int nsites, bool need_witness) {
+    int rc = fp_check_shapes(c, sites, nsites);
+    if (rc) return rc;
+    for (int s = 0; s < nsites; s++) {
+        const fp_site& t = sites[s];
+        char buf[160];
+        if (!t.w || !t.xt) {
+            snprintf(buf, sizeof buf, "site %d: null operand", s);
+            return fp_fail(c, FP_ERR_ARG, buf);
+        }
+        if (need_witness && (!t.q || !t.r || !t.y)) {
+            snprintf(buf, sizeof buf, "site %d: null witness buffer", s);
+            return fp_fail(c, FP_ERR_ARG, buf);
+        }
+    }
+    return FP_OK;
+}
+
+int fp_check_shapes(fp_ctx* c, const fp_site* sites, int nsites) {
     if (!sites || nsites < 1) return fp_fail(c, FP_ERR_SHAPE, "need at least one site");
     for (int s = 0; s < nsites; s++) {
         const fp_site& t = sites[s];
@@ -430,14 +448,6 @@ int fp_check_sites(fp_ctx* c, const fp_site* sites, int nsites, bool need_witnes
         if (wmax * 128.0 * (double)t.K >= 2147483648.0) {
             snprintf(buf, sizeof buf, "site %d: K = %d can overflow the int32 accumulator", s, t.K);
             return fp_fail(c, FP_ERR_SHAPE, buf);
-        }
-        if (!t.w || !t.xt) {
-            snprintf(buf, sizeof buf, "site %d: null operand", s);
-            return fp_fail(c, FP_ERR_ARG, buf);
-        }
-        if (need_witness && (!t.q || !t.r || !t.y)) {
-            snprintf(buf, sizeof buf, "site %d: null witness buffer", s);
-            return fp_fail(c, FP_ERR_ARG, buf);
         }
     }
     return FP_OK;
@@ -489,8 +499,10 @@ int fp_digest(fp_ctx* c, const void* dev, size_t nbytes, uint8_t out[32], void* 
     return fp_digest_many(c, &j, 1, out, (cudaStream_t)stream);
 }
 
-int fp_commit_witness(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, void* stream) {
-    if (!c || !tx) return fp_fail(c, FP_ERR_ARG, "fp_commit_witness: null context or transcript");
+namespace {
+
+// the witness and digests of sites[0, nsites): 192-byte site records into rec
+int commit_records(fp_ctx* c, const fp_site* sites, int nsites, void* stream, std::vector<uint8_t>& rec) {
     int rc = fp_check_sites(c, sites, nsites, true);
     if (rc) return rc;
     FP_CUDA(c, cudaSetDevice(c->device));
@@ -527,11 +539,40 @@ int fp_commit_witness(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, vo
     if (rc) return rc;
     if (c->mb->err)  // the digests synchronised the stream
         return fp_fail(c, FP_ERR_TIMEOUT, "witness GEMM: a tensor-core completion wait ran out");
-    std::vector<uint8_t> rec(192 * (size_t)nsites);
+    rec.assign(192 * (size_t)nsites, 0);
     for (int i = 0; i < nsites; i++)
         if (sites[i].w_digest) memcpy(&rec[192 * i], sites[i].w_digest, 64);
     for (size_t j = 0; j < jobs.size(); j++) memcpy(&rec[32 * where[j]], &dg[32 * j], 32);
+    return FP_OK;
+}
+
+}  // namespace
+
+int fp_commit_witness(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, void* stream) {
+    if (!c || !tx) return fp_fail(c, FP_ERR_ARG, "fp_commit_witness: null context or transcript");
+    std::vector<uint8_t> rec;
+    int rc = commit_records(c, sites, nsites, stream, rec);
+    if (rc) return rc;
     for (int i = 0; i < nsites; i++) fp_tx_absorb_raw(tx, "site", &rec[192 * i], 192);
+    return FP_OK;
+}
+
+int fp_commit_witness_shard(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, const fp_shard* shard,
+                            void* stream) {
+    if (!c || !tx || !shard) return fp_fail(c, FP_ERR_ARG, "fp_commit_witness_shard: null argument");
+    FpShardView sh;
+    int rc = fp_shard_view(c, shard, nsites, sh);
+    if (rc) return rc;
+    if ((rc = fp_check_shapes(c, sites, nsites))) return rc;
+    const int lo = sh.lo[sh.rank], own = sh.lo[sh.rank + 1] - lo;
+    std::vector<uint8_t> rec;
+    if ((rc = commit_records(c, sites + lo, own, stream, rec))) return rc;
+    std::vector<uint64_t> mine(24 * (size_t)own), all(24 * (size_t)nsites);
+    memcpy(mine.data(), rec.data(), rec.size());
+    if ((rc = fp_shard_gather(sh, mine.data(), 24, all.data())))
+        return fp_fail(c, rc, "fp_commit_witness_shard: the all-gather failed");
+    const uint8_t* b = (const uint8_t*)all.data();
+    for (int i = 0; i < nsites; i++) fp_tx_absorb_raw(tx, "site", b + 192 * (size_t)i, 192);
     return FP_OK;
 }
 

@@ -210,6 +210,22 @@ size_t fp_partial_host_scratch(const FpPeJob* jobs, int njobs);
 int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s);
 size_t fp_claims_scratch(const fp_site* sites, int nsites);
 // per-site output claims into dev_out[s]
+// A statement's sites shared among ranks: rank r proves sites [lo[r], lo[r + 1]);
+// small values are exchanged through the caller's all-gather.
+struct FpShardView {
+    int rank = 0, world = 1;
+    std::vector<int> lo;
+    fp_allgather_fn ag = nullptr;
+    void* user = nullptr;
+};
+int fp_shard_view(fp_ctx* c, const fp_shard* shard, int nsites, FpShardView& sh);  // NULL: one rank
+// every rank's `per` words for each of its own sites, in site order (all: nsites * per words)
+int fp_shard_gather(const FpShardView& sh, const uint64_t* mine, int per, uint64_t* all);
+// the ranks' n words added mod p, in place
+int fp_shard_sum(const FpShardView& sh, uint64_t* v, int n);
+// shapes, rescale exponents and the int32 domain of every site (no pointers looked at)
+int fp_check_shapes(fp_ctx* c, const fp_site* sites, int nsites);
+
 int fp_claims(fp_ctx* c, const fp_site* sites, int nsites, const uint64_t* const* eq_rows,
               const uint64_t* const* eq_cols, uint64_t* dev_out, cudaStream_t s);
 
