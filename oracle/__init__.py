@@ -69,6 +69,10 @@ REASONS = {
     38: "lhi2_round",
     39: "lhi2_final",
     40: "lhi2_open",
+    41: "lhr_sum",
+    42: "lhr_round",
+    43: "lhr_final",
+    44: "lhr_open",
 }
 
 
@@ -132,6 +136,9 @@ def lib():
         L.orc_verify.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp]
         L.orc_verify_opts.restype = C.c_int
         L.orc_verify_opts.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp, vp, C.c_int]
+        L.orc_prove_hi.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64,
+                                   C.POINTER(u64), vp, C.POINTER(u64)]
+        L.orc_verify_hi.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp]
         L.orc_had_prove.restype = C.c_int
         L.orc_had_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
         L.orc_had_verify.restype = C.c_int
@@ -414,6 +421,39 @@ def prove(seed: int, sites, wits):
         raise ValueError(f"orc_prove failed ({rc})")
     st = states.raw
     return buf[: n.value].tobytes(), [st[0:32], st[32:64], st[64:96]], off.value
+
+
+def prove_hi(seed: int, sites, wits):
+    """The layer proof with the helper-inverse lookup section (orc_prove_hi): the commit and
+    matmul section of prove(), then both rescale tables by two committed helper columns and
+    one sum-check. Returns (proof bytes, [state after commit, after matmul, after lookup],
+    matmul section length)."""
+    keep = []
+    cs, cw = _marshal(sites, wits, keep)
+    n = C.c_uint64(0)
+    off = C.c_uint64(0)
+    states = C.create_string_buffer(96)
+    kmax = max(int(s.k_shift) for s in sites)
+    cap = (1 << 22) + 4 * (1 << kmax) + 64 * len(sites)
+    buf = np.zeros(cap, dtype=np.uint8)
+    rc = lib().orc_prove_hi(seed, cs, len(sites), cw, _ptr(buf), cap, C.byref(n), states, C.byref(off))
+    if rc == -2:
+        buf = np.zeros(max(1, n.value), dtype=np.uint8)
+        rc = lib().orc_prove_hi(seed, cs, len(sites), cw, _ptr(buf), n.value, C.byref(n), states, C.byref(off))
+    if rc != 0:
+        raise ValueError(f"orc_prove_hi failed ({rc})")
+    st = states.raw
+    return buf[: n.value].tobytes(), [st[0:32], st[32:64], st[64:96]], off.value
+
+
+def verify_hi(seed: int, sites, wits, proof: bytes):
+    """Verifier of prove_hi's proofs: (reason name, detail), 'accept' for a valid proof."""
+    keep = []
+    cs, cw = _marshal(sites, wits, keep)
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    rc = lib().orc_verify_hi(seed, cs, len(sites), cw, _ptr(pb), len(proof), _ptr(det))
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
 
 
 def verify(seed: int, sites, wits, proof: bytes, site_mask=None, skip_leaf_open: bool = False):

@@ -3372,3 +3372,238 @@ done:
     keys_free(&K);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* The rescale lookups by helper inverses (next row f3: LogUp after Haboeck  */
+/* 2022, "Towards Proving Frontier-Scale LLM Inference", The proof system,   */
+/* set against the fraction tree of "How fast can FlashProve go", 4 Tighter  */
+/* Rooflines). The lookup section of the layer proof with the same keys and  */
+/* tables as the GKR form (remainder table R_k, clamp table C16), but with   */
+/* the key side as two committed helper columns checked by one sum-check:    */
+/*   m_rem (2^k u32, digest absorbed, "lhr_m_rem"); squeeze gamma            */
+/*   ("lhr_gamma"); m_clamp (2^16 u32, "lhr_m_clamp"); squeeze alpha0 and    */
+/*   alpha1 ("lhr_alpha"); commit h0_i = 1 / (alpha0 - r_i) and              */
+/*   h1_i = 1 / (alpha1 - q_i - gamma y_i): absorb "lhr_h" D(h0) || D(h1)    */
+/*   (u64 little-endian); squeeze z_1..z_v ("lhr_z") and beta ("lhr_beta");  */
+/*   send S0 = sum h0, S1 = sum h1 ("lhr_sum");                              */
+/*   sum-check over v variables of                                           */
+/*     G = h0 + beta h1 + eq(z, .) (beta^2 (h0 (alpha0 - r) - 1)             */
+/*                                  + beta^3 (h1 (alpha1 - q - gamma y) - 1)) */
+/*   with claim S0 + beta S1: rounds g(0..3) ("lhr_round"), "lhr_chal";      */
+/*   send h0, h1, r, q, y at rho ("lhr_final").                               */
+/* The keys are the sites' outputs in storage order, padded to 2^v (v >= 1)  */
+/* with the neutral key (r, q, y) = 0, which the multiplicities count. The   */
+/* verifier checks S0 and S1 against the table fractions, every round, the  */
+/* end against G at rho (eq(z, rho) in closed form), and the five final      */
+/* values against the columns it recomputes (standing in for openings). The  */
+/* zero-check terms force h0 (alpha0 - r) = 1 and h1 (alpha1 - q - gamma y)  */
+/* = 1 on the whole cube (with high probability over z and beta), so S0 and  */
+/* S1 are the key sides of the two LogUp identities. v rounds in all,        */
+/* against the tree's v (v - 1) / 2, for two committed columns (16 bytes a   */
+/* key).                                                                      */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_LHR_SUM = 41,    /* S0 or S1 != its table side (detail: the table) */
+    REJ_LHR_ROUND = 42,  /* g(0) + g(1) != running claim */
+    REJ_LHR_FINAL = 43,  /* the end does not match G at rho */
+    REJ_LHR_OPEN = 44    /* a final value != its column's MLE at rho (detail: which) */
+};
+
+/* the five columns over the padded keys: r, q, y as field elements, h0, h1 */
+static void lhr_columns(const orc_keys* K, u64 a0, u64 a1, u64 gamma, u64* R, u64* Q, u64* Y, u64* H0, u64* H1) {
+    u64 L = (u64)1 << K->v;
+    for (u64 i = 0; i < L; i++) {
+        R[i] = orc_fint(K->fr[i]);
+        Q[i] = orc_fint(K->fq[i]);
+        Y[i] = orc_fint(K->fy[i]);
+        H0[i] = orc_finv(orc_fsub(a0, R[i]));
+        H1[i] = orc_finv(orc_fsub(a1, orc_fadd(Q[i], orc_fmul(gamma, Y[i]))));
+    }
+}
+
+static void lhr_absorb_h(orc_tx* t, const u64* H0, const u64* H1, u64 L) {
+    uint8_t* b = (uint8_t*)malloc(8 * L);
+    uint8_t d[64];
+    for (u64 i = 0; i < L; i++) put_le(b + 8 * i, H0[i], 8);
+    orc_tree_digest(b, 8 * L, d);
+    for (u64 i = 0; i < L; i++) put_le(b + 8 * i, H1[i], 8);
+    orc_tree_digest(b, 8 * L, d + 32);
+    free(b);
+    orc_tx_absorb(t, "lhr_h", d, 64);
+}
+
+/* G at one point, from the five column values and the eq weight there */
+static u64 lhr_G(const u64 c[5], u64 e, u64 a0, u64 a1, u64 gamma, u64 beta) {
+    u64 b2 = orc_fmul(beta, beta), b3 = orc_fmul(b2, beta);
+    u64 t0 = orc_fsub(orc_fmul(c[3], orc_fsub(a0, c[0])), 1);
+    u64 t1 = orc_fsub(orc_fmul(c[4], orc_fsub(a1, orc_fadd(c[1], orc_fmul(gamma, c[2])))), 1);
+    u64 zc = orc_fadd(orc_fmul(b2, t0), orc_fmul(b3, t1));
+    return orc_fadd(orc_fadd(c[3], orc_fmul(beta, c[4])), orc_fmul(e, zc));
+}
+
+static void lhr_prove(orc_tx* t, pbuf* pb, const orc_site* sites, int ns, const orc_wit* wit) {
+    orc_keys K;
+    keys_build(sites, ns, wit, &K);
+    int v = K.v;
+    u64 L = (u64)1 << v, Trem = (u64)1 << K.k;
+    u32* mr = (u32*)malloc(Trem * sizeof(u32));
+    u32* mc = (u32*)malloc(65536 * sizeof(u32));
+    mult_rem(&K, mr);
+    send_mult(t, pb, "lhr_m_rem", mr, Trem);
+    u64 gamma = orc_tx_squeeze(t, "lhr_gamma");
+    mult_clamp(&K, mc);
+    send_mult(t, pb, "lhr_m_clamp", mc, 65536);
+    u64 a0 = orc_tx_squeeze(t, "lhr_alpha");
+    u64 a1 = orc_tx_squeeze(t, "lhr_alpha");
+    /* V[0..4] = r, q, y, h0, h1; V[5] = eq(z, .) */
+    u64* V[6];
+    for (int i = 0; i < 6; i++) V[i] = (u64*)malloc(L * sizeof(u64));
+    lhr_columns(&K, a0, a1, gamma, V[0], V[1], V[2], V[3], V[4]);
+    lhr_absorb_h(t, V[3], V[4], L);
+    u64* z = (u64*)malloc(sizeof(u64) * v);
+    for (int i = 0; i < v; i++) z[i] = orc_tx_squeeze(t, "lhr_z");
+    u64 beta = orc_tx_squeeze(t, "lhr_beta");
+    u64 S[2] = {0, 0};
+    for (u64 i = 0; i < L; i++) {
+        S[0] = orc_fadd(S[0], V[3][i]);
+        S[1] = orc_fadd(S[1], V[4][i]);
+    }
+    send_fe(t, pb, "lhr_sum", S, 2);
+    orc_eq_table(z, v, V[5]);
+    u64 Lr = L;
+    for (int rd = 0; rd < v; rd++) {
+        u64 hh = Lr >> 1;
+        u64 g[4] = {0, 0, 0, 0};
+        for (u64 b = 0; b < hh; b++)
+            for (u64 X = 0; X < 4; X++) {
+                u64 c[6];
+                for (int i = 0; i < 6; i++) c[i] = orc_fadd(V[i][b], orc_fmul(X, orc_fsub(V[i][hh + b], V[i][b])));
+                g[X] = orc_fadd(g[X], lhr_G(c, c[5], a0, a1, gamma, beta));
+            }
+        send_fe(t, pb, "lhr_round", g, 4);
+        u64 rho = orc_tx_squeeze(t, "lhr_chal");
+        for (int i = 0; i < 6; i++)
+            for (u64 b = 0; b < hh; b++) V[i][b] = orc_fadd(V[i][b], orc_fmul(rho, orc_fsub(V[i][hh + b], V[i][b])));
+        Lr = hh;
+    }
+    u64 fin[5] = {V[3][0], V[4][0], V[0][0], V[1][0], V[2][0]};
+    send_fe(t, pb, "lhr_final", fin, 5);
+    for (int i = 0; i < 6; i++) free(V[i]);
+    free(z);
+    free(mr);
+    free(mc);
+    keys_free(&K);
+}
+
+static int lhr_verify(orc_tx* t, prd* rd, const orc_site* sites, int ns, const orc_wit* wit, int64_t* detail) {
+    int rc = 0;
+    orc_keys K;
+    if (keys_build(sites, ns, wit, &K) != 0) {
+        detail[0] = detail[1] = 0;
+        return REJ_ARGS;
+    }
+    int v = K.v;
+    u64 L = (u64)1 << v, Trem = (u64)1 << K.k;
+    u32* mr = (u32*)malloc(Trem * sizeof(u32));
+    u32* mc = (u32*)malloc(65536 * sizeof(u32));
+    u64* z = (u64*)malloc(sizeof(u64) * (v + 1));
+    u64* rho = (u64*)malloc(sizeof(u64) * (v + 1));
+    u64* C[5];
+    for (int i = 0; i < 5; i++) C[i] = (u64*)malloc(L * sizeof(u64));
+    rd_mult(t, rd, "lhr_m_rem", mr, Trem);
+    u64 gamma = orc_tx_squeeze(t, "lhr_gamma");
+    rd_mult(t, rd, "lhr_m_clamp", mc, 65536);
+    if (rd->bad) FAIL(REJ_FORMAT, 8, 0);
+    u64 a0 = orc_tx_squeeze(t, "lhr_alpha");
+    u64 a1 = orc_tx_squeeze(t, "lhr_alpha");
+    lhr_columns(&K, a0, a1, gamma, C[0], C[1], C[2], C[3], C[4]); /* the verifier holds the keys, so h0, h1 too */
+    lhr_absorb_h(t, C[3], C[4], L);
+    for (int i = 0; i < v; i++) z[i] = orc_tx_squeeze(t, "lhr_z");
+    u64 beta = orc_tx_squeeze(t, "lhr_beta");
+    u64 S[2];
+    rd_fe(t, rd, "lhr_sum", S, 2);
+    if (rd->bad) FAIL(REJ_FORMAT, 9, 0);
+    for (int tau = 0; tau < 2; tau++) {
+        u64 PT, QT;
+        table_fraction(tau == 0 ? mr : mc, tau == 0 ? Trem : 65536, tau, K.k, tau == 0 ? a0 : a1, gamma, &PT, &QT);
+        if (orc_fmul(S[tau], QT) != PT) FAIL(REJ_LHR_SUM, tau, 0);
+    }
+    u64 claim = orc_fadd(S[0], orc_fmul(beta, S[1]));
+    for (int i = 0; i < v; i++) {
+        u64 g[4];
+        rd_fe(t, rd, "lhr_round", g, 4);
+        if (rd->bad) FAIL(REJ_FORMAT, 10, i);
+        if (orc_fadd(g[0], g[1]) != claim) FAIL(REJ_LHR_ROUND, i, 0);
+        rho[i] = orc_tx_squeeze(t, "lhr_chal");
+        claim = orc_lagrange(g, 4, rho[i]);
+    }
+    u64 fin[5];
+    rd_fe(t, rd, "lhr_final", fin, 5);
+    if (rd->bad) FAIL(REJ_FORMAT, 11, 0);
+    {
+        /* G at rho from the final values h0, h1, r, q, y */
+        u64 c[5] = {fin[2], fin[3], fin[4], fin[0], fin[1]};
+        if (lhr_G(c, eq_closed(z, rho, v), a0, a1, gamma, beta) != claim) FAIL(REJ_LHR_FINAL, 0, 0);
+    }
+    {
+        const int col[5] = {3, 4, 0, 1, 2}; /* final value i is column col[i]'s MLE */
+        for (int i = 0; i < 5; i++)
+            if (orc_mle_eval(C[col[i]], L, rho, v) != fin[i]) FAIL(REJ_LHR_OPEN, i, 0);
+    }
+done:
+    for (int i = 0; i < 5; i++) free(C[i]);
+    free(mr);
+    free(mc);
+    free(z);
+    free(rho);
+    keys_free(&K);
+    return rc;
+}
+
+/* The layer proof with the helper-inverse lookup section: the commit and the
+ * matmul section of orc_prove, then lhr_prove instead of the fraction tree.
+ * Arguments and results as for orc_prove. */
+int orc_prove_hi(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, uint8_t* proof, u64 cap, u64* len,
+                 uint8_t states[96], u64* sec_off) {
+    if (ns < 1) return -1;
+    for (int s = 0; s < ns; s++)
+        if (sites[s].M < 1 || sites[s].N < 1 || sites[s].K < 1 || sites[s].k_shift < 1 ||
+            sites[s].k_shift > 30 || (sites[s].w_bits != 4 && sites[s].w_bits != 8) ||
+            sites[s].k_shift != sites[0].k_shift)
+            return -1;
+    orc_tx t;
+    pbuf pb = {proof, cap, 0, 0};
+    orc_tx_init(&t, seed);
+    absorb_sites(&t, sites, ns, wit);
+    memcpy(states, t.st, 32);
+    mm_prove(&t, &pb, sites, ns, wit);
+    memcpy(states + 32, t.st, 32);
+    *sec_off = pb.len;
+    lhr_prove(&t, &pb, sites, ns, wit);
+    memcpy(states + 64, t.st, 32);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+int orc_verify_hi(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, const uint8_t* proof, u64 len,
+                  int64_t detail[2]) {
+    g_site_mask = NULL;
+    g_verify_flags = 0;
+    detail[0] = detail[1] = 0;
+    if (ns < 1) return REJ_ARGS;
+    for (int s = 0; s < ns; s++)
+        if (sites[s].M < 1 || sites[s].N < 1 || sites[s].K < 1 || sites[s].k_shift < 1 ||
+            sites[s].k_shift > 30 || sites[s].k_shift != sites[0].k_shift)
+            return REJ_ARGS;
+    orc_tx t;
+    prd rd = {proof, len, 0, 0};
+    orc_tx_init(&t, seed);
+    absorb_sites(&t, sites, ns, wit);
+    int rc = mm_verify(&t, &rd, sites, ns, wit, detail);
+    if (rc) return rc;
+    rc = lhr_verify(&t, &rd, sites, ns, wit, detail);
+    if (rc) return rc;
+    if (rd.pos != rd.len) return REJ_FORMAT;
+    return 0;
+}

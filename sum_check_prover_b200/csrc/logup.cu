@@ -32,10 +32,23 @@
 
 namespace {
 
-constexpr int LU_THREADS = 256;
-// The leaf layer's kernel runs 512-thread blocks (one per SM): its big rounds, read from the key
-// columns, ran about 3% faster that way than as two 256-thread blocks per SM.
-constexpr int LU_LEAF_THREADS = 512;
+// Launch shapes of the layer kernels (block threads; the blocks per SM the register budget is
+// sized for). The leaf layer's kernel runs 512-thread blocks: its big rounds, read from the key
+// columns, ran about 3% faster as one 512-thread block per SM than as two 256-thread blocks.
+#ifndef FP_GKR_THREADS
+#define FP_GKR_THREADS 256
+#endif
+#ifndef FP_GKR_MIN_BLOCKS
+#define FP_GKR_MIN_BLOCKS 2
+#endif
+#ifndef FP_GKR_LEAF_THREADS
+#define FP_GKR_LEAF_THREADS 512
+#endif
+#ifndef FP_GKR_LEAF_MIN_BLOCKS
+#define FP_GKR_LEAF_MIN_BLOCKS 1
+#endif
+constexpr int LU_THREADS = FP_GKR_THREADS;
+constexpr int LU_LEAF_THREADS = FP_GKR_LEAF_THREADS;
 
 struct KeySrc {
     const int32_t* r;
@@ -471,7 +484,7 @@ __device__ __forceinline__ void layer_tail(const GkrLayer& A, const uint64_t* yt
 
 // Rounds [t_begin, t_end] of one layer (t_end > d: and its final child values).
 template <bool LEAF>
-__global__ void __launch_bounds__(LEAF ? LU_LEAF_THREADS : LU_THREADS, LEAF ? 1 : 2) gkr_layer_kernel(GkrLayer A, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
+__global__ void __launch_bounds__(LEAF ? LU_LEAF_THREADS : LU_THREADS, LEAF ? FP_GKR_LEAF_MIN_BLOCKS : FP_GKR_MIN_BLOCKS) gkr_layer_kernel(GkrLayer A, FpMailbox* mb, FpRelay* rl, uint64_t* part) {
     __shared__ uint64_t zs[32];
     __shared__ uint64_t s_lam;
     __shared__ uint64_t eq_tab[3 << kEqChunk];

@@ -117,6 +117,13 @@ def prove(seed: int, sites, wits) -> bytes:
         out.extend(b)
         tx.absorb(label, b)
 
+    commit_and_matmul(tx, send, sites, wits)
+    lookup_gkr(tx, send, out, sites, wits)
+    return bytes(out)
+
+
+def commit_and_matmul(tx, send, sites, wits):
+    """The site records, then the matmul section, by definition."""
     for s, (q, r, y) in zip(sites, wits):
         sc = b"" if s.scales is None else s.scales.tobytes()
         d = tree_digest(s.w.tobytes()) + tree_digest(sc) + tree_digest(s.xt.tobytes()) + \
@@ -164,7 +171,19 @@ def prove(seed: int, sites, wits) -> bytes:
         fin += [A_at(si, chal), B_at(si, chal)]
     send("sc_final", fin)
 
-    # ---- LogUp ----
+
+def lookup_keys(sites, wits):
+    """The padded key columns r, q, y (int64) of the sites' outputs in storage order."""
+    fr = np.concatenate([w[1].reshape(-1) for w in wits]).astype(np.int64)
+    fq = np.concatenate([w[0].reshape(-1) for w in wits]).astype(np.int64)
+    fy = np.concatenate([w[2].reshape(-1) for w in wits]).astype(np.int64)
+    v = max(1, log2c(len(fr)))
+    pad = (1 << v) - len(fr)
+    return [np.concatenate([a, np.zeros(pad, np.int64)]) for a in (fr, fq, fy)] + [v]
+
+
+def lookup_gkr(tx, send, out, sites, wits):
+    """The lookup section as the fraction tree with one sum-check per layer, by definition."""
     k = sites[0].k_shift
     fr = np.concatenate([w[1].reshape(-1) for w in wits]).astype(np.int64)
     fq = np.concatenate([w[0].reshape(-1) for w in wits]).astype(np.int64)
@@ -245,6 +264,64 @@ def prove(seed: int, sites, wits) -> bytes:
         z = rho_l + [tx.squeeze("gkr_mu")]
 
     send("leaf", [mle(fr, z), mle(fq, z), mle(fy, z)])
+
+
+def prove_hi(seed: int, sites, wits) -> bytes:
+    """The layer proof with the helper-inverse lookup section, by definition: the helper
+    columns by Python modular inverses, every round value a hypercube sum of the summand
+    over MLEs evaluated at field points (no folding)."""
+    tx = Tx(seed)
+    out = bytearray()
+
+    def send(label, vals):
+        b = fe_bytes(vals)
+        out.extend(b)
+        tx.absorb(label, b)
+
+    commit_and_matmul(tx, send, sites, wits)
+    k = sites[0].k_shift
+    fr, fq, fy, v = lookup_keys(sites, wits)
+    m_rem = np.zeros(1 << k, np.int64)
+    for x in fr:
+        if 0 <= x + (1 << (k - 1)) < (1 << k):
+            m_rem[x + (1 << (k - 1))] += 1
+    b = m_rem.astype("<u4").tobytes()
+    out.extend(b)
+    tx.absorb("lhr_m_rem", tree_digest(b))
+    gamma = tx.squeeze("lhr_gamma")
+    m_cl = np.zeros(1 << 16, np.int64)
+    for x in fq:
+        if 0 <= x + 32768 < 65536:
+            m_cl[x + 32768] += 1
+    b = m_cl.astype("<u4").tobytes()
+    out.extend(b)
+    tx.absorb("lhr_m_clamp", tree_digest(b))
+    a0, a1 = tx.squeeze("lhr_alpha"), tx.squeeze("lhr_alpha")
+    R = [int(x) % P for x in fr]
+    Q = [int(x) % P for x in fq]
+    Y = [int(x) % P for x in fy]
+    h0 = [pow((a0 - x) % P, P - 2, P) for x in R]
+    h1 = [pow((a1 - q - gamma * y) % P, P - 2, P) for q, y in zip(Q, Y)]
+    pack = lambda col: b"".join(struct.pack("<Q", x) for x in col)  # noqa: E731
+    tx.absorb("lhr_h", tree_digest(pack(h0)) + tree_digest(pack(h1)))
+    z = [tx.squeeze("lhr_z") for _ in range(v)]
+    beta = tx.squeeze("lhr_beta")
+    send("lhr_sum", [sum(h0) % P, sum(h1) % P])
+    rho = []
+    for t in range(v):
+        rest = v - t - 1
+        g = []
+        for X in range(4):
+            acc = 0
+            for bb in range(1 << rest):
+                w = rho + [X] + [(bb >> (rest - 1 - i)) & 1 for i in range(rest)]
+                H0, H1, r_, q_, y_ = (mle_at(c, w) for c in (h0, h1, R, Q, Y))
+                zero = beta ** 2 * (H0 * (a0 - r_) - 1) + beta ** 3 * (H1 * (a1 - q_ - gamma * y_) - 1)
+                acc += H0 + beta * H1 + eq_ml(z, w) * zero
+            g.append(acc % P)
+        send("lhr_round", g)
+        rho.append(tx.squeeze("lhr_chal"))
+    send("lhr_final", [mle_at(c, rho) for c in (h0, h1, R, Q, Y)])
     return bytes(out)
 
 
