@@ -266,6 +266,27 @@ int logup_prove_rescale(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites
                         size_t* proof_len, void* stream);
 
 /*
+ * The lookup section in the helper-inverse form (LogUp after Haboeck 2022,
+ * "Towards Proving Frontier-Scale LLM Inference", The proof system), the
+ * alternative to logup_prove_rescale's fraction tree ("How fast can FlashProve
+ * go", 4 Tighter Rooflines). Same sites, keys, tables and multiplicities; the
+ * key side is two committed helper columns checked by one sum-check of v rounds
+ * (the tree takes v (v - 1) / 2):
+ *   m_rem, "lhr_m_rem"; gamma; m_clamp, "lhr_m_clamp"; alpha0, alpha1;
+ *   absorb "lhr_h" D(h0) || D(h1), h0_i = 1 / (alpha0 - r_i),
+ *   h1_i = 1 / (alpha1 - q_i - gamma y_i); z_1..z_v, beta; send S0 = sum h0,
+ *   S1 = sum h1; rounds of G = h0 + beta h1 + eq(z, .) (beta^2 (h0 (alpha0 - r)
+ *   - 1) + beta^3 (h1 (alpha1 - q - gamma y) - 1)), claim S0 + beta S1; send
+ *   h0, h1, r, q, y at rho.
+ * Proof bytes: m_rem (2^k u32) | m_clamp (2^16 u32) | S0, S1 | v x 4 round
+ * values | 5 final values. Keys up to 2^30. Returns FP_WARN_KEYS_OUTSIDE_TABLE
+ * (proof still written) when some r or q lies outside its table; proof and
+ * proof_len as for sumcheck_prove_matmul; other errors as logup_prove_rescale.
+ */
+int logup_prove_rescale_hi(fp_ctx* ctx, fp_tx* tx, const fp_site* sites, int nsites, uint8_t* proof,
+                           size_t* proof_len, void* stream);
+
+/*
  * Sum-check of a gated product h = s (.) u that is never committed ("How fast
  * can FlashProve go", 3.1 Committing intermediate values: the MLP's gated
  * product is a plain product, so sum-check handles it without committing to
@@ -552,6 +573,24 @@ int fp_lhi2_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uin
  * The proof and proof_len are as for logup_prove_helper_inverse.
  */
 int fp_lhi_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uint8_t* m_digest, fp_values_fn fn,
+                          void* user, uint8_t* proof, size_t* proof_len);
+
+/*
+ * The host half of logup_prove_rescale_hi from the multiplicities on (v
+ * variables, k the rescale shift); tx must have reached the lookup section.
+ * m: host, 2^k u32 of m_rem then 2^16 of m_clamp; m_digests: 64 bytes, their
+ * two tree digests. Callback kinds:
+ *   FP_VAL_COLUMN: in = alpha0, alpha1, gamma; out = D(h0) || D(h1) (8 words,
+ *     little-endian bytes);
+ *   FP_VAL_START: in = z_1..z_v, beta (v + 1 words), t = v;
+ *   FP_VAL_ROUND: out = A0(0), A0(1), A1(0), A1(1), Q0(0..2), Q1(0..2)
+ *     (10 words; A sums of h0 and h1, Q the eq(z_>t)-weighted sums of
+ *     h0 (alpha0 - r) and h1 (alpha1 - q - gamma y));
+ *   FP_VAL_ANSWER: in = rho_t;
+ *   FP_VAL_FINALS: out = h0, h1, r, q, y at rho (5 words).
+ * proof and proof_len as for logup_prove_rescale_hi.
+ */
+int fp_lhr_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m, const uint8_t* m_digests, fp_values_fn fn,
                           void* user, uint8_t* proof, size_t* proof_len);
 
 /*

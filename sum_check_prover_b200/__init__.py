@@ -104,6 +104,8 @@ def lib():
                                               vp]
     L.fp_mm_shard_protocol_drive.argtypes = [vp, C.POINTER(_Site), i32, C.POINTER(_Shard), _VALUES_FN, vp, vp,
                                              C.POINTER(sz)]
+    L.logup_prove_rescale_hi.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
+    L.fp_lhr_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.fp_ctx_set_profiling.argtypes = [vp, i32]
     L.fp_session_selftest.argtypes = [vp, vp]
     L.fp_host_stats.argtypes = [vp, C.POINTER(C.c_double)]
@@ -192,6 +194,47 @@ def balance_sites(costs: Sequence[float], world: int) -> list:
         lo.append(n - (world - len(lo)))
     lo.append(n)
     return lo
+
+
+def lhr_protocol_drive(tx: "Transcript", v: int, k: int, m, m_digests: bytes, values) -> bytes:
+    """Run the host half of the helper-inverse lookup section from the multiplicities on, with
+    its device values taken from `values` (no GPU work): values.column(alpha0, alpha1, gamma)
+    -> D(h0) || D(h1) (64 bytes), values.start(z, beta), values.round(t) -> 10 values,
+    values.answer(t, rho), values.finals() -> 5 values. m: the 2^k + 2^16 multiplicities
+    (m_rem then m_clamp); m_digests: their two tree digests."""
+    import numpy as np
+    L = lib()
+
+    def cb(_user, kind, t, inp, out):
+        try:
+            if kind == VAL_COLUMN:
+                d = values.column(int(inp[0]), int(inp[1]), int(inp[2]))
+                for i in range(8):
+                    out[i] = int.from_bytes(d[8 * i:8 * i + 8], "little")
+                return 0
+            if kind == VAL_START:
+                values.start([int(inp[i]) for i in range(t)], int(inp[t]))
+                return 0
+            if kind == VAL_ANSWER:
+                values.answer(t, int(inp[0]))
+                return 0
+            res = values.round(t) if kind == VAL_ROUND else values.finals()
+            for i, x in enumerate(res):
+                out[i] = int(x) % P
+            return 0
+        except Exception:  # reported to the caller as FP_ERR_ARG
+            return 1
+
+    fn = _VALUES_FN(cb)
+    mm = np.ascontiguousarray(np.asarray(m, dtype=np.uint32))
+    dg = C.create_string_buffer(bytes(m_digests), 64)
+    ln = C.c_size_t(0)
+    L.fp_lhr_protocol_drive(tx.h, v, k, mm.ctypes.data, dg, fn, None, None, C.byref(ln))
+    buf = C.create_string_buffer(max(1, ln.value))
+    rc = L.fp_lhr_protocol_drive(tx.h, v, k, mm.ctypes.data, dg, fn, None, buf, C.byref(ln))
+    if rc != 0:
+        raise FpError(rc, "fp_lhr_protocol_drive failed")
+    return buf.raw[: ln.value]
 
 
 def mm_shard_protocol_drive(tx: "Transcript", sites: Sequence["SiteDesc"], shard: Optional[Shard], values) -> bytes:
@@ -888,6 +931,17 @@ class Context:
                                                      _stream(stream)), "logup_prove_rescale")
         return buf.raw[: n.value], rc
 
+    def prove_logup_hi(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
+        """The lookup section in the helper-inverse form (logup_prove_rescale_hi). Returns (proof
+        bytes, status): status 1 means some key lies outside its table."""
+        arr, keep = _sites(sites)
+        n = C.c_size_t(0)
+        self._L.logup_prove_rescale_hi(self.h, tx.h, arr, len(sites), None, C.byref(n), _stream(stream))
+        buf = C.create_string_buffer(max(1, n.value))
+        rc = self._check(self._L.logup_prove_rescale_hi(self.h, tx.h, arr, len(sites), buf, C.byref(n),
+                                                        _stream(stream)), "logup_prove_rescale_hi")
+        return buf.raw[: n.value], rc
+
     def set_profiling(self, on):
         """False/0: off; True/1: one launch per sum-check round, each timed; 2: time the
         production (resident) launches as they run."""
@@ -927,11 +981,14 @@ class Context:
         return out
 
 
-def prove(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], stream=None):
+def prove(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], stream=None, lookup: str = "gkr"):
     """Prove a layer: commit every stage's witness in order (a later stage may read
     an earlier stage's outputs), then the batched matmul sum-check over all sites,
-    then the LogUp rescale/clamp proof. Returns (proof bytes, transcript states after
+    then the LogUp rescale/clamp proof, as the fraction tree (lookup="gkr") or by
+    helper inverses (lookup="hi"). Returns (proof bytes, transcript states after
     commit / matmul / lookup, lookup status)."""
+    if lookup not in ("gkr", "hi"):
+        raise ValueError("prove: lookup must be 'gkr' or 'hi'")
     tx = Transcript(seed)
     try:
         for st in stages:
@@ -940,7 +997,7 @@ def prove(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], stream=
         s0 = tx.state()
         mm = ctx.prove_matmul(tx, sites, stream)
         s1 = tx.state()
-        lu, status = ctx.prove_logup(tx, sites, stream)
+        lu, status = (ctx.prove_logup if lookup == "gkr" else ctx.prove_logup_hi)(tx, sites, stream)
         return mm + lu, [s0, s1, tx.state()], status
     finally:
         tx.close()

@@ -66,6 +66,9 @@ enum FpKernel {
     K_LU2_TREE,
     K_LU2_ROUND,
     K_LU2_LEAF,
+    K_LHR_COLUMN,
+    K_LHR_ROUND,
+    K_LHR_FINAL,
     K_COUNT
 };
 
@@ -223,6 +226,22 @@ int fp_shard_view(fp_ctx* c, const fp_shard* shard, int nsites, FpShardView& sh)
 int fp_shard_gather(const FpShardView& sh, const uint64_t* mine, int per, uint64_t* all);
 // the ranks' n words added mod p, in place
 int fp_shard_sum(const FpShardView& sh, uint64_t* v, int n);
+// The lookup keys: every site's outputs in storage order, concatenated; indices
+// in [n, 2^v) are the neutral key (r, q, y) = 0.
+struct FpKeyCols {
+    const int32_t* r;
+    const int32_t* q;
+    const int8_t* y;
+    int64_t n;
+};
+// the key columns (the single site's own buffers, or a copy gathered into c->dev)
+size_t fp_lookup_keys_scratch(int nsites, int64_t nk);
+int fp_lookup_keys(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st, FpKeyCols* K);
+// multiplicities of both tables over the keys padded to L (device, c->dev), copied to
+// hm (host: 2^k u32, 2^16 u32, the count of keys outside the tables) with their digests
+size_t fp_lookup_mults_scratch(int k);
+int fp_lookup_mults(fp_ctx* c, const FpKeyCols& K, int k, int64_t L, cudaStream_t st, uint8_t* hm, uint8_t dg_rem[32],
+                    uint8_t dg_cl[32]);
 // shapes, rescale exponents and the int32 domain of every site (no pointers looked at)
 int fp_check_shapes(fp_ctx* c, const fp_site* sites, int nsites);
 

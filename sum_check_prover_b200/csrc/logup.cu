@@ -50,12 +50,7 @@ namespace {
 constexpr int LU_THREADS = FP_GKR_THREADS;
 constexpr int LU_LEAF_THREADS = FP_GKR_LEAF_THREADS;
 
-struct KeySrc {
-    const int32_t* r;
-    const int32_t* q;
-    const int8_t* y;
-    int64_t n;  // real keys; indices in [n, 2^v) are the neutral key 0
-};
+using KeySrc = FpKeyCols;
 
 struct Chal {
     uint64_t alpha0, alpha1, gamma;
@@ -608,6 +603,77 @@ int grid_for(fp_ctx* c, int64_t work, int threads) {
 
 }  // namespace
 
+size_t fp_lookup_keys_scratch(int nsites, int64_t nk) {
+    return nsites > 1 ? fp_align_up(9 * (size_t)nk + 1024, 256) + fp_align_up(sizeof(GatherSite) * nsites, 256) : 0;
+}
+
+int fp_lookup_keys(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st, FpKeyCols* K) {
+    int64_t nk = 0;
+    for (int s = 0; s < nsites; s++) nk += (int64_t)sites[s].M * sites[s].N;
+    K->n = nk;
+    if (nsites == 1) {
+        K->r = sites[0].r;
+        K->q = sites[0].q;
+        K->y = sites[0].y;
+        return FP_OK;
+    }
+    int32_t* r = (int32_t*)fp_alloc(c->dev, 4 * (size_t)nk);
+    int32_t* q = (int32_t*)fp_alloc(c->dev, 4 * (size_t)nk);
+    int8_t* y = (int8_t*)fp_alloc(c->dev, (size_t)nk);
+    GatherSite* dgs = (GatherSite*)fp_alloc(c->dev, sizeof(GatherSite) * nsites);
+    GatherSite* hgs = (GatherSite*)fp_alloc(c->host, sizeof(GatherSite) * nsites);
+    if (!r || !q || !y || !dgs || !hgs) return fp_fail(c, FP_ERR_OOM, "lookup keys: scratch exhausted");
+    int64_t off = 0;
+    for (int s = 0; s < nsites; s++) {
+        hgs[s] = GatherSite{sites[s].q, sites[s].r, sites[s].y, off};
+        off += (int64_t)sites[s].M * sites[s].N;
+    }
+    FP_CUDA(c, cudaMemcpyAsync(dgs, hgs, sizeof(GatherSite) * nsites, cudaMemcpyHostToDevice, st));
+    int slot;
+    fp_tic(c, st, K_KEYS_GATHER, 18.0 * nk, &slot);
+    gather_kernel<<<grid_for(c, nk, 256), 256, 0, st>>>(dgs, nsites, nk, r, q, y);
+    fp_toc(c, st, slot);
+    FP_CUDA(c, cudaGetLastError());
+    K->r = r;
+    K->q = q;
+    K->y = y;
+    return FP_OK;
+}
+
+size_t fp_lookup_mults_scratch(int k) { return fp_align_up(4 * ((size_t)1 << k), 256) + fp_align_up(4 * 65536, 256) + 256; }
+
+int fp_lookup_mults(fp_ctx* c, const FpKeyCols& K, int k, int64_t L, cudaStream_t st, uint8_t* hm, uint8_t dg_rem[32],
+                    uint8_t dg_cl[32]) {
+    const int64_t T = 1ll << k;
+    int rc;
+    uint32_t* m_rem = (uint32_t*)fp_alloc(c->dev, 4 * (size_t)T);
+    uint32_t* m_cl = (uint32_t*)fp_alloc(c->dev, 4 * 65536);
+    uint32_t* outside = (uint32_t*)fp_alloc(c->dev, 256);
+    if (!m_rem || !m_cl || !outside || !hm) return fp_fail(c, FP_ERR_OOM, "lookup multiplicities: scratch exhausted");
+    FP_CUDA(c, cudaMemsetAsync(m_rem, 0, 4 * (size_t)T, st));
+    FP_CUDA(c, cudaMemsetAsync(m_cl, 0, 4 * 65536, st));
+    FP_CUDA(c, cudaMemsetAsync(outside, 0, 4, st));
+    {
+        const int rem_smem = T <= 16384;
+        const int smem = 4 * (2 * HIST_WIN) + (rem_smem ? 4 * (int)T : 0);
+        FP_CUDA(c, cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+        int slot;
+        fp_tic(c, st, K_HIST, 9.0 * K.n, &slot);
+        hist_kernel<<<c->num_sms, 1024, smem, st>>>(K, k, L, m_rem, m_cl, outside, rem_smem);
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+    }
+    FP_CUDA(c, cudaMemcpyAsync(hm, m_rem, 4 * (size_t)T, cudaMemcpyDeviceToHost, st));
+    FP_CUDA(c, cudaMemcpyAsync(hm + 4 * T, m_cl, 4 * 65536, cudaMemcpyDeviceToHost, st));
+    FP_CUDA(c, cudaMemcpyAsync(hm + 4 * T + 4 * 65536, outside, 4, cudaMemcpyDeviceToHost, st));
+    FpDigestJob jobs[2] = {{(const uint8_t*)m_rem, 4 * (uint64_t)T}, {(const uint8_t*)m_cl, 4 * 65536ull}};
+    uint8_t both[64];
+    if ((rc = fp_digest_many(c, jobs, 2, both, st))) return rc;  // synchronises the stream
+    memcpy(dg_rem, both, 32);
+    memcpy(dg_cl, both + 32, 32);
+    return FP_OK;
+}
+
 int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, uint8_t* proof, size_t* proof_len,
                         void* stream) {
     if (!c || !tx || !proof_len) return fp_fail(c, FP_ERR_ARG, "logup_prove_rescale: null argument");
@@ -635,9 +701,7 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
     const int64_t T = 1ll << k;
 
     // ---- scratch ----
-    size_t need = 0;
-    if (nsites > 1) need += fp_align_up(9 * (size_t)nk + 1024, 256) + fp_align_up(sizeof(GatherSite) * nsites, 256);
-    need += fp_align_up(4 * (size_t)T, 256) + fp_align_up(4 * 65536, 256) + 256;
+    size_t need = fp_lookup_keys_scratch(nsites, nk) + fp_lookup_mults_scratch(k);
     size_t tree = 0;
     for (int d = 1; d <= v - 1; d++) tree += 4 * fp_align_up((size_t)8 << d, 256);
     need += tree;
@@ -651,66 +715,12 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
     fp_reset(c->dev);
     fp_reset(c->host);
 
-    // ---- keys ----
+    // ---- keys, multiplicities ----
     KeySrc K;
-    K.n = nk;
-    if (nsites == 1) {
-        K.r = sites[0].r;
-        K.q = sites[0].q;
-        K.y = sites[0].y;
-    } else {
-        int32_t* r = (int32_t*)fp_alloc(c->dev, 4 * (size_t)nk);
-        int32_t* q = (int32_t*)fp_alloc(c->dev, 4 * (size_t)nk);
-        int8_t* y = (int8_t*)fp_alloc(c->dev, (size_t)nk);
-        std::vector<GatherSite> gs(nsites);
-        int64_t off = 0;
-        for (int s = 0; s < nsites; s++) {
-            gs[s] = GatherSite{sites[s].q, sites[s].r, sites[s].y, off};
-            off += (int64_t)sites[s].M * sites[s].N;
-        }
-        GatherSite* dgs = (GatherSite*)fp_alloc(c->dev, sizeof(GatherSite) * nsites);
-        GatherSite* hgs = (GatherSite*)fp_alloc(c->host, sizeof(GatherSite) * nsites);
-        memcpy(hgs, gs.data(), sizeof(GatherSite) * nsites);
-        FP_CUDA(c, cudaMemcpyAsync(dgs, hgs, sizeof(GatherSite) * nsites, cudaMemcpyHostToDevice, st));
-        int slot;
-        fp_tic(c, st, K_KEYS_GATHER, 18.0 * nk, &slot);
-        gather_kernel<<<grid_for(c, nk, 256), 256, 0, st>>>(dgs, nsites, nk, r, q, y);
-        fp_toc(c, st, slot);
-        FP_CUDA(c, cudaGetLastError());
-        K.r = r;
-        K.q = q;
-        K.y = y;
-    }
-
-    // ---- multiplicities ----
-    uint32_t* m_rem = (uint32_t*)fp_alloc(c->dev, 4 * (size_t)T);
-    uint32_t* m_cl = (uint32_t*)fp_alloc(c->dev, 4 * 65536);
-    uint32_t* outside = (uint32_t*)fp_alloc(c->dev, 256);
-    FP_CUDA(c, cudaMemsetAsync(m_rem, 0, 4 * (size_t)T, st));
-    FP_CUDA(c, cudaMemsetAsync(m_cl, 0, 4 * 65536, st));
-    FP_CUDA(c, cudaMemsetAsync(outside, 0, 4, st));
-    {
-        const int rem_smem = T <= 16384;
-        const int smem = 4 * (2 * HIST_WIN) + (rem_smem ? 4 * (int)T : 0);
-        FP_CUDA(c, cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-        int slot;
-        fp_tic(c, st, K_HIST, 9.0 * nk, &slot);
-        hist_kernel<<<c->num_sms, 1024, smem, st>>>(K, k, L, m_rem, m_cl, outside, rem_smem);
-        fp_toc(c, st, slot);
-        FP_CUDA(c, cudaGetLastError());
-    }
+    if ((rc = fp_lookup_keys(c, sites, nsites, st, &K))) return rc;
     uint8_t* hm = (uint8_t*)fp_alloc(c->host, 4 * (size_t)T + 4 * 65536 + 256);
-    FP_CUDA(c, cudaMemcpyAsync(hm, m_rem, 4 * (size_t)T, cudaMemcpyDeviceToHost, st));
-    FP_CUDA(c, cudaMemcpyAsync(hm + 4 * T, m_cl, 4 * 65536, cudaMemcpyDeviceToHost, st));
-    FP_CUDA(c, cudaMemcpyAsync(hm + 4 * T + 4 * 65536, outside, 4, cudaMemcpyDeviceToHost, st));
     uint8_t dg_rem[32], dg_cl[32];
-    {
-        FpDigestJob jobs[2] = {{(const uint8_t*)m_rem, 4 * (uint64_t)T}, {(const uint8_t*)m_cl, 4 * 65536ull}};
-        uint8_t both[64];
-        if ((rc = fp_digest_many(c, jobs, 2, both, st))) return rc;  // synchronises the stream
-        memcpy(dg_rem, both, 32);
-        memcpy(dg_cl, both + 32, 32);
-    }
+    if ((rc = fp_lookup_mults(c, K, k, L, st, hm, dg_rem, dg_cl))) return rc;
     uint32_t n_outside;
     memcpy(&n_outside, hm + 4 * T + 4 * 65536, 4);
     size_t pos = 0;
