@@ -205,7 +205,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-MICRO_ALL = "sc,pe,gkr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2,silu2,lu2"
+MICRO_ALL = "sc,pe,gkr,lhr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2,silu2,lu2"
 
 
 def micro_names(which) -> set:
@@ -353,6 +353,20 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
         device.weight_digests(ctx, st)
         measure("gkr_round_2^26_keys", "gkr_round", lambda: fp.prove(ctx, 2, st))
         del st, keep
+    if "lhr" in which:
+        # the same statement's lookup section by helper inverses: its rounds, and the columns'
+        # formation (table inverses, two gathers; the digests are timed as digest kernels)
+        try:
+            s = workloads.random_site(77, 8192, 64, 8192, 8, 12)
+            st, keep = device.upload(workloads.Workload("lhr", 0, [s]), dev)
+            device.weight_digests(ctx, st)
+            measure("helper_inverse_rescale_round_2^26_keys", "lhr_round",
+                    lambda: fp.prove(ctx, 2, st, lookup="hi"))
+            measure("helper_inverse_rescale_columns_2^26_keys", "lhr_column",
+                    lambda: fp.prove(ctx, 2, st, lookup="hi"))
+            del st, keep
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["helper_inverse_rescale_round_2^26_keys"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     if "silu" in which:
         # the SiLU lookup of an FFN's gate values: 2^26 16-bit inputs and their table entries
         try:
@@ -674,6 +688,32 @@ def run_ours(args):
                             "launch configuration; a resident sum-check launch spans all its rounds, "
                             "host exchanges included"}
 
+    # ---- the same statement with the lookup section by helper inverses (row f3's comparison
+    # with the fraction tree): device time per proof and host round trips ------------------
+    variants = None
+    if not args.no_variants:
+        for i in range(2):
+            fp.prove(ctx, args.seed + 400 + i, stages, stream, lookup="hi")
+        torch.cuda.synchronize()
+        hv0 = ctx.host_stats()
+        hi_ms = []
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            e0.record(stream)
+            hp, _, hstatus = fp.prove(ctx, args.seed + 500 + i, stages, stream, lookup="hi")
+            e1.record(stream)
+            e1.synchronize()
+            hi_ms.append(e0.elapsed_time(e1))
+        hv1 = ctx.host_stats()
+        hi_total = max_over_ranks(sum(hi_ms), pg, dev)
+        variants = {
+            "gkr": {"lookup": "LogUp-GKR fraction tree, one sum-check per layer", "ms_per_step": ms_per_step,
+                    "value": value, "host_round_trips_per_step": host_waits, "proof_bytes": proof_len},
+            "hi": {"lookup": "helper-inverse LogUp: two committed columns, one sum-check",
+                   "ms_per_step": hi_total / args.steps, "value": job_throughput(macs, world, args.steps, hi_total),
+                   "host_round_trips_per_step": (hv1[0] - hv0[0]) / args.steps, "proof_bytes": len(hp),
+                   "status": hstatus}}
+
     # ---- e2e pass: activations from pinned host memory, layer output read back ----------
     flat = [d for st in stages for d in st]
     seen = set()
@@ -740,6 +780,7 @@ def run_ours(args):
                 "clocks": clk,
                 "kernels": kern,
                 "kernels_stepped": kern_stepped,
+                "lookup_variants": variants,
                 "microbench": micro,
                 "proof_bytes": proof_len,
                 "pages_context": PAGES_CONTEXT}
@@ -761,6 +802,7 @@ def main():
                     help="the statement one step proves (5: the MoE layer, the largest one-GPU configuration)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-micro", action="store_true")
+    ap.add_argument("--no-variants", action="store_true", help="skip the helper-inverse lookup timing")
     ap.add_argument("--micro-only", nargs="?", const=MICRO_ALL, default=None,
                     help="run only the kernel measurements at scale (comma list of sc, pe, gkr, gemm)")
     args = ap.parse_args()
