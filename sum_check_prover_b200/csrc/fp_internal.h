@@ -198,6 +198,8 @@ int fp_eq_table(fp_ctx* c, const FpPoint& z, uint64_t* out, cudaStream_t s);
 // Row contractions out[c] = sum_{i<rows} eq(z, i) M_eff[i][c], many per launch
 // (partial.cu). z is host memory (v = ceil(log2 rows) coordinates); out is
 // device memory with out_len >= cols entries, the ones past cols zeroed.
+// out[c] = sum_i w_i M_eff[i][c]: w_i = eq(z, i) for the point z (v coordinates, host), or, when
+// wts is set, w_i = wts[i * wts_stride] (device, canonical; z and v unused)
 struct FpPeJob {
     const void* mat;
     int bits;
@@ -207,6 +209,8 @@ struct FpPeJob {
     int v;
     uint64_t* out;
     int64_t out_len;
+    const uint64_t* wts = nullptr;
+    int wts_stride = 1;
 };
 size_t fp_partial_scratch(const fp_ctx* c, const FpPeJob* jobs, int njobs);
 size_t fp_partial_host_scratch(const FpPeJob* jobs, int njobs);

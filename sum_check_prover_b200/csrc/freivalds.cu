@@ -11,46 +11,20 @@
 // only the activations (N K bytes), the verifier reads the weights.
 //
 // Kernels: the powers rho^j (one exponentiation each), then the row contraction of
-// Xt (N x K int8) with them: one thread per column over a chunk of rows, exact
-// 192-bit sums, then a pass adding the chunks.
+// Xt (N x K int8) with them, which is the partial evaluation's contraction with the
+// powers as its row weights (the tensor-core byte-limb kernel: Xt streamed once by
+// TMA, the weights split into byte limbs).
 #include <string.h>
 
 #include <algorithm>
 
 #include "fp_internal.h"
-#include "fp_reduce.cuh"
 
 namespace {
-
-constexpr int FRV_MAX_CHUNKS = 32;
 
 __global__ void frv_pow_kernel(uint64_t rho, int64_t n, uint64_t* __restrict__ pw) {
     for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n; j += (int64_t)gridDim.x * blockDim.x)
         pw[j] = gl_pow(rho, (uint64_t)j);
-}
-
-// part[chunk][k] = sum over the chunk's rows j of pw[j] xt[j][k]
-__global__ void __launch_bounds__(256) frv_contract_kernel(const int8_t* __restrict__ xt, int N, int K,
-                                                           int rows_per_chunk, const uint64_t* __restrict__ pw,
-                                                           uint64_t* __restrict__ part) {
-    const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (k >= K) return;  // no barrier below
-    const int chunk = blockIdx.y;
-    const int j0 = chunk * rows_per_chunk, j1 = min(N, j0 + rows_per_chunk);
-    GlAcc acc;
-    for (int j = j0; j < j1; j++) {
-        const int x = __ldg(xt + (int64_t)j * K + k);
-        if (x) acc.mac(__ldg(pw + j), gl_from_i64(x));
-    }
-    part[(int64_t)chunk * K + k] = acc.value();
-}
-
-__global__ void frv_finish_kernel(const uint64_t* __restrict__ part, int nchunks, int K, uint64_t* __restrict__ u) {
-    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < K; k += (int64_t)gridDim.x * blockDim.x) {
-        uint64_t s = 0;
-        for (int c = 0; c < nchunks; c++) s = gl_add(s, part[(int64_t)c * K + k]);
-        u[k] = s;
-    }
 }
 
 }  // namespace
@@ -74,28 +48,27 @@ int freivalds_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* site, uint8_t* p
         fp_tx_absorb_raw(tx, "frv_site", d, 160);
     }
     const uint64_t rho = fp_tx_squeeze_one(tx, "frv_rho");
-    const int nchunks = std::min(FRV_MAX_CHUNKS, std::max(1, (s.N + 127) / 128));
-    const int per = (s.N + nchunks - 1) / nchunks;
-    const size_t need = fp_align_up((size_t)8 * s.N, 256) + fp_align_up((size_t)8 * nchunks * s.K, 256) +
-                        fp_align_up((size_t)8 * s.K, 256) + 4096;
+    // u = sum_j rho^j Xt[j][.]: the row contraction of Xt with the powers as row weights
+    FpPeJob job{s.xt, 8, nullptr, s.N, s.K, nullptr, 0, nullptr, (int64_t)s.K};
+    const size_t need = fp_align_up((size_t)8 * s.N, 256) + fp_align_up((size_t)8 * s.K, 256) +
+                        fp_partial_scratch(c, &job, 1) + 4096;
     if ((rc = fp_reserve(c, c->dev, need))) return rc;
-    if ((rc = fp_reserve(c, c->host, fp_align_up((size_t)8 * s.K, 256) + 4096))) return rc;
+    if ((rc = fp_reserve(c, c->host, fp_align_up((size_t)8 * s.K, 256) + fp_partial_host_scratch(&job, 1) + 4096)))
+        return rc;
     fp_reset(c->dev);
     fp_reset(c->host);
     uint64_t* pw = (uint64_t*)fp_alloc(c->dev, (size_t)8 * s.N);
-    uint64_t* part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * nchunks * s.K);
     uint64_t* u = (uint64_t*)fp_alloc(c->dev, (size_t)8 * s.K);
     uint64_t* hu = (uint64_t*)fp_alloc(c->host, (size_t)8 * s.K);
-    if (!pw || !part || !u || !hu) return fp_fail(c, FP_ERR_OOM, "freivalds_prove_matmul: scratch exhausted");
+    if (!pw || !u || !hu) return fp_fail(c, FP_ERR_OOM, "freivalds_prove_matmul: scratch exhausted");
+    job.out = u;
+    job.wts = pw;
     int slot;
     fp_tic(c, st, K_FRV_U, (double)s.N * s.K + 8.0 * s.K, &slot);
     frv_pow_kernel<<<fp_grid256(c, s.N), 256, 0, st>>>(rho, s.N, pw);
-    frv_contract_kernel<<<dim3((unsigned)((s.K + 255) / 256), (unsigned)nchunks), 256, 0, st>>>(s.xt, s.N, s.K, per,
-                                                                                                pw, part);
-    frv_finish_kernel<<<fp_grid256(c, s.K), 256, 0, st>>>(part, nchunks, s.K, u);
-    fp_toc(c, st, slot);
     FP_CUDA(c, cudaGetLastError());
-    c->launches += 2;  // three kernels under one timing slot
+    if ((rc = fp_partial_many(c, &job, 1, st))) return rc;
+    fp_toc(c, st, slot);  // the powers and the contraction's launches under one slot
     FP_CUDA(c, cudaMemcpyAsync(hu, u, (size_t)8 * s.K, cudaMemcpyDeviceToHost, st));
     FP_CUDA(c, cudaStreamSynchronize(st));
     put_u64s(proof, hu, (size_t)s.K);

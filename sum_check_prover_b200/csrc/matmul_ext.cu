@@ -12,11 +12,13 @@
 //   B = X~(., r_col) ("mm2_round"), rho_t ("mm2_chal"); send A(rho), B(rho)
 //   ("mm2_final").
 //
-// An extension point's eq weights are extension elements, so the partial
-// evaluations A[k] = sum_i eq(r_row, i) W_eff[i][k] and B[k] = sum_j eq(r_col, j)
-// Xt[j][k] are row contractions with 16-byte weights: each thread owns one byte
-// of a row (an int8 column or two int4 columns) and sums a chunk of rows exactly
-// (two 192-bit accumulators per column); a second pass adds the chunks. The claim
+// An extension point's eq weights are extension elements e_i = a_i + b_i phi and the
+// matrices hold base-field integers, so each partial evaluation
+// A[k] = sum_i eq(r_row, i) W_eff[i][k] (and B[k] = sum_j eq(r_col, j) Xt[j][k]) is two
+// base-field row contractions, sum_i a_i W_eff[i][k] and sum_i b_i W_eff[i][k]: the
+// partial evaluation's tensor-core kernel with the two coordinate vectors as its row
+// weights (all four contractions of a call in one launch), then a pass pairing the
+// coordinates into extension elements. The claim
 // is a flat eq_row x eq_col weighted sum of 2^k q + r. The rounds run in one
 // resident cooperative launch over the two length-2^n vectors, folding in place
 // as the base-field matmul kernel does.
@@ -26,6 +28,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <vector>
 
 #include "fp_ext2.cuh"
 #include "fp_ext2_host.h"
@@ -36,7 +39,6 @@
 namespace {
 
 constexpr int M2_THREADS = 256;
-constexpr int M2_MAX_CHUNKS = 32;  // row chunks of a contraction (partial sums per column)
 
 // out[x] = eq(z, x) for x < 2^v, z_1 on the most significant bit
 __global__ void e2_eq_kernel(const Ext2* __restrict__ z, int v, Ext2* __restrict__ out) {
@@ -68,59 +70,11 @@ __global__ void __launch_bounds__(M2_THREADS) mm2_claim_kernel(const int32_t* __
     }
 }
 
-// part[chunk][col] = sum over the chunk's rows i of E[i] M_eff[i][col]: one thread per byte of
-// a row (an int8 column, or the two int4 columns of a byte); M_eff = scales[i][col / 64] M
-// when scales are given
-__global__ void __launch_bounds__(M2_THREADS) e2_contract_kernel(const uint8_t* __restrict__ mat, int bits,
-                                                                 const int8_t* __restrict__ scales, int rows, int cols,
-                                                                 int64_t pitch, int rows_per_chunk,
-                                                                 const Ext2* __restrict__ E, Ext2* __restrict__ part) {
-    const int64_t byte = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (byte >= pitch) return;  // no barrier below
-    const int chunk = blockIdx.y;
-    const int row0 = chunk * rows_per_chunk;
-    const int row1 = min(rows, row0 + rows_per_chunk);
-    const int G = (cols + 63) / 64;
-    if (bits == 8) {
-        const int col = (int)byte;
-        E2Acc acc;
-        for (int i = row0; i < row1; i++) {
-            int w = (int)(int8_t)__ldg(mat + (int64_t)i * pitch + byte);
-            if (scales) w *= (int)__ldg(scales + (int64_t)i * G + (col >> 6));
-            if (w) acc.mac_base(E[i], gl_from_i64(w));
-        }
-        part[(int64_t)chunk * cols + col] = e2_make(acc.a.value(), acc.b.value());
-    } else {
-        const int c0 = (int)(2 * byte), c1 = c0 + 1;  // c1 may be the odd K's padding nibble
-        E2Acc a0, a1;
-        for (int i = row0; i < row1; i++) {
-            const int bv = __ldg(mat + (int64_t)i * pitch + byte);
-            int w0 = bv & 15, w1 = bv >> 4;
-            w0 = w0 >= 8 ? w0 - 16 : w0;
-            w1 = w1 >= 8 ? w1 - 16 : w1;
-            if (scales) {
-                const int s = (int)__ldg(scales + (int64_t)i * G + (c0 >> 6));  // c0, c1 share a group
-                w0 *= s;
-                w1 *= s;
-            }
-            const Ext2 e = E[i];
-            if (w0) a0.mac_base(e, gl_from_i64(w0));
-            if (w1) a1.mac_base(e, gl_from_i64(w1));
-        }
-        part[(int64_t)chunk * cols + c0] = e2_make(a0.a.value(), a0.b.value());
-        if (c1 < cols) part[(int64_t)chunk * cols + c1] = e2_make(a1.a.value(), a1.b.value());
-    }
-}
-
-// out[col] = sum over chunks of part[chunk][col] for col < cols, 0 for cols <= col < len
-__global__ void e2_contract_finish_kernel(const Ext2* __restrict__ part, int nchunks, int cols, int64_t len,
-                                          Ext2* __restrict__ out) {
-    for (int64_t col = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; col < len; col += (int64_t)gridDim.x * blockDim.x) {
-        Ext2 s = e2_make(0, 0);
-        if (col < cols)
-            for (int c = 0; c < nchunks; c++) s = e2_add(s, part[(int64_t)c * cols + col]);
-        out[col] = s;
-    }
+// out[k] = (a[k], b[k]): the two coordinates of the contractions paired into extension elements
+__global__ void e2_pair_kernel(const uint64_t* __restrict__ a, const uint64_t* __restrict__ b, int64_t len,
+                               Ext2* __restrict__ out) {
+    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < len; k += (int64_t)gridDim.x * blockDim.x)
+        out[k] = e2_make(a[k], b[k]);
 }
 
 struct Mm2Args {
@@ -250,27 +204,42 @@ struct Mm2Device : Mm2Source {
     Ext2* B = nullptr;
     Ext2* Erow = nullptr;
     Ext2* Ecol = nullptr;
-    Ext2* cpart = nullptr;      // contraction partial sums
+    uint64_t* coord[4] = {nullptr, nullptr, nullptr, nullptr};  // A.a, A.b, B.a, B.b (2^n each)
     uint64_t* part = nullptr;   // reduction partials
     uint64_t* small = nullptr;  // device: [0..2) claim, [8..) the point
     uint64_t* hs = nullptr;     // pinned host staging
     Mm2Args P;
     int cap_grid = 1;
 
-    // out (length 2^n) = the E-weighted sum of the rows of a rows x cols matrix
-    int contract(const void* mat, int bits, const int8_t* scales, int rows, int cols, const Ext2* E, Ext2* out) {
-        const int64_t pitch = bits == 4 ? (cols + 1) / 2 : cols;
-        const int nchunks = std::min(M2_MAX_CHUNKS, std::max(1, (rows + 127) / 128));
-        const int per = (rows + nchunks - 1) / nchunks;
-        const dim3 grid((unsigned)((pitch + M2_THREADS - 1) / M2_THREADS), (unsigned)nchunks);
-        int slot;
-        fp_tic(c, st, K_MM2_CONTRACT, (double)rows * (double)pitch, &slot);
-        e2_contract_kernel<<<grid, M2_THREADS, 0, st>>>((const uint8_t*)mat, bits, scales, rows, cols, pitch, per, E,
-                                                        cpart);
-        e2_contract_finish_kernel<<<fp_grid256(c, 1ll << n), 256, 0, st>>>(cpart, nchunks, cols, 1ll << n, out);
+    // the four base-field contractions: W and Xt, each with the a and the b coordinates of its
+    // eq weights (row i's weight at E[i].a or E[i].b, a stride of two words)
+    std::vector<FpPeJob> jobs() const {
+        const int64_t L = 1ll << n;
+        std::vector<FpPeJob> j(4);
+        for (int h = 0; h < 2; h++) {
+            j[h] = FpPeJob{s->w, s->w_bits, s->scales, s->M, s->K, nullptr, 0, coord[h], L};
+            j[h].wts = reinterpret_cast<const uint64_t*>(Erow) + h;
+            j[h].wts_stride = 2;
+            j[2 + h] = FpPeJob{s->xt, 8, nullptr, s->N, s->K, nullptr, 0, coord[2 + h], L};
+            j[2 + h].wts = reinterpret_cast<const uint64_t*>(Ecol) + h;
+            j[2 + h].wts_stride = 2;
+        }
+        return j;
+    }
+
+    // A and B from the four contractions, in one partial-evaluation launch per kernel variant
+    int contract() {
+        const int64_t L = 1ll << n;
+        const double bytes = (double)s->M * (s->w_bits == 4 ? (s->K + 1) / 2 : s->K) + (double)s->N * s->K;
+        int slot, rc;
+        fp_tic(c, st, K_MM2_CONTRACT, bytes, &slot);
+        const std::vector<FpPeJob> j = jobs();
+        if ((rc = fp_partial_many(c, j.data(), 4, st))) return rc;
+        e2_pair_kernel<<<fp_grid256(c, L), 256, 0, st>>>(coord[0], coord[1], L, A);
+        e2_pair_kernel<<<fp_grid256(c, L), 256, 0, st>>>(coord[2], coord[3], L, B);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
-        c->launches++;  // two kernels under one timing slot
+        c->launches++;  // the two pairing kernels under one slot (the slot counts one)
         return FP_OK;
     }
 
@@ -295,9 +264,7 @@ struct Mm2Device : Mm2Source {
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         c->launches++;
-        int rc;
-        if ((rc = contract(s->w, s->w_bits, s->scales, s->M, s->K, Erow, A))) return rc;
-        return contract(s->xt, 8, nullptr, s->N, s->K, Ecol, B);
+        return contract();
     }
 
     int claim(Ext2& cl) override {
@@ -473,24 +440,26 @@ int sumcheck_prove_matmul_ext2(fp_ctx* c, fp_tx* tx, const fp_site* site, uint8_
     FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, mm2_session_kernel, M2_THREADS, 0));
     dev.cap_grid = std::max(1, occ) * c->num_sms;
     const int64_t L = 1ll << n;
-    const int64_t cmax = (int64_t)M2_MAX_CHUNKS * s.K;  // contraction partials, the larger of the two
     const size_t part_n = (size_t)6 * std::max(dev.cap_grid, 4 * c->num_sms);
+    const std::vector<FpPeJob> pj = dev.jobs();  // shapes only, for the partial evaluation's scratch
     const size_t need = 2 * fp_align_up((size_t)16 * L, 256) + fp_align_up((size_t)16 << vM, 256) +
-                        fp_align_up((size_t)16 << vN, 256) + fp_align_up((size_t)16 * cmax, 256) +
-                        fp_align_up(8 * part_n, 256) + fp_align_up(8 * 160, 256) + 4096;
+                        fp_align_up((size_t)16 << vN, 256) + 4 * fp_align_up((size_t)8 * L, 256) +
+                        fp_partial_scratch(c, pj.data(), 4) + fp_align_up(8 * part_n, 256) +
+                        fp_align_up(8 * 160, 256) + 4096;
     if ((rc = fp_reserve(c, c->dev, need))) return rc;
-    if ((rc = fp_reserve(c, c->host, 4096))) return rc;
+    if ((rc = fp_reserve(c, c->host, fp_partial_host_scratch(pj.data(), 4) + fp_align_up(8 * 160, 256) + 4096)))
+        return rc;
     fp_reset(c->dev);
     fp_reset(c->host);
     dev.A = (Ext2*)fp_alloc(c->dev, (size_t)16 * L);
     dev.B = (Ext2*)fp_alloc(c->dev, (size_t)16 * L);
     dev.Erow = (Ext2*)fp_alloc(c->dev, (size_t)16 << vM);
     dev.Ecol = (Ext2*)fp_alloc(c->dev, (size_t)16 << vN);
-    dev.cpart = (Ext2*)fp_alloc(c->dev, (size_t)16 * cmax);
+    for (int h = 0; h < 4; h++) dev.coord[h] = (uint64_t*)fp_alloc(c->dev, (size_t)8 * L);
     dev.part = (uint64_t*)fp_alloc(c->dev, 8 * part_n);
     dev.small = (uint64_t*)fp_alloc(c->dev, 8 * 160);
     dev.hs = (uint64_t*)fp_alloc(c->host, 8 * 160);
-    if (!dev.A || !dev.B || !dev.Erow || !dev.Ecol || !dev.cpart || !dev.part || !dev.small || !dev.hs)
+    if (!dev.A || !dev.B || !dev.Erow || !dev.Ecol || !dev.coord[3] || !dev.part || !dev.small || !dev.hs)
         return fp_fail(c, FP_ERR_OOM, "sumcheck_prove_matmul_ext2: scratch exhausted");
     return mm2_protocol(c, tx, vM, vN, n, dev, proof, proof_len);
 }

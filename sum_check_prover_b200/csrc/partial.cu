@@ -25,7 +25,10 @@
 //
 // All contractions of a call go into one launch per kernel variant (a job
 // list; the MoE layer has hundreds of sites). eq(z, i) for the block's rows
-// is computed in the block from the point, so no eq table is materialised.
+// is computed in the block from the point, so no eq table is materialised. A
+// job may give its row weights as a device vector instead (the coordinates of
+// extension-field eq weights, the powers of a Freivalds challenge): the same
+// contraction with w_i read per row.
 #include <cuda.h>  // CUtensorMap and its enums; the encoder is fetched through the runtime
 #include <cudaTypedefs.h>
 #include <string.h>
@@ -42,13 +45,14 @@ struct PeJob {
     const uint8_t* mat;
     const int8_t* scales;
     const uint64_t* z;   // device, v coordinates
+    const uint64_t* wts; // device row weights (row i at wts[i * wstride]), or null: eq(z, i)
     uint64_t* part;      // splits x cols block sums
     uint64_t* out;
     int64_t out_len;
     int32_t rows, cols, v, rows_per_block;
     int32_t col_blocks, splits;
     int32_t aligned;
-    int32_t pad;
+    int32_t wstride;
     int64_t first_block;
     // tensor-core path: the matrix as a 2-D byte tensor (rows x pitch), 32-row x 128-byte
     // boxes with 128-byte swizzle, read by TMA from this device copy of the job
@@ -148,7 +152,10 @@ __global__ void __launch_bounds__(PE_THREADS, 3) partial_many_kernel(const PeJob
     for (int k = threadIdx.x; k < nr; k += PE_THREADS) {
         const uint64_t i = (uint64_t)(r0 + k);
         uint64_t e = 1;
-        for (int b = 0; b < J.v; b++) e = gl_mul(e, gl_eq1(J.z[b], (int)((i >> (J.v - 1 - b)) & 1)));
+        if (J.wts)
+            e = __ldg(J.wts + (int64_t)i * J.wstride);
+        else
+            for (int b = 0; b < J.v; b++) e = gl_mul(e, gl_eq1(J.z[b], (int)((i >> (J.v - 1 - b)) & 1)));
         eqs[k] = e;
         es = gl_add(es, e);
     }
@@ -357,7 +364,9 @@ __global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJo
     if (!SCALED) {
         for (int k = threadIdx.x; k < kend; k += PE_THREADS) {
             // with v < 5 the rows are i = n < 2^v and H = {1}
-            const uint64_t e = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
+            const uint64_t e = k >= nr ? 0ull
+                               : J.wts ? __ldg(J.wts + (int64_t)(r0 + k) * J.wstride)
+                                       : gl_mul(htab[k >> 5], ttab[k & 31]);
 #pragma unroll
             for (int l = 0; l < 8; l++) et[l][k] = (uint8_t)(e >> (8 * l));
             es = gl_add(es, e);
@@ -369,7 +378,10 @@ __global__ void __launch_bounds__(PE_TC_THREADS, 3) partial_tc_kernel(const PeJo
 #pragma unroll
         for (int w = 0; w < PE_THREADS / 32; w++) es = gl_add(es, wsum[w]);
     } else {
-        for (int k = threadIdx.x; k < kend; k += PE_THREADS) eqs[k] = k < nr ? gl_mul(htab[k >> 5], ttab[k & 31]) : 0ull;
+        for (int k = threadIdx.x; k < kend; k += PE_THREADS)
+            eqs[k] = k >= nr ? 0ull
+                     : J.wts ? __ldg(J.wts + (int64_t)(r0 + k) * J.wstride)
+                             : gl_mul(htab[k >> 5], ttab[k & 31]);
         pe_consumers_sync();
     }
     // scaled: the scale of row 32 i + lane in the warp's column group, loaded a chunk ahead
@@ -676,7 +688,8 @@ int fp_partial_many(fp_ctx* c, const FpPeJob* jobs, int njobs, cudaStream_t s) {
         // the fast path loads 4 (int4) or 8 (int8) bytes per lane and row
         d.aligned = ((uintptr_t)q.mat % 16 == 0) && (q.cols % PE_COLS == 0) &&
                     (q.bits == 4 ? (pitch % 4 == 0) : (pitch % 8 == 0));
-        d.pad = 0;
+        d.wts = q.wts;
+        d.wstride = q.wts_stride;
         d.first_block = 0;
         d.part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * d.splits * q.cols);
         if (!d.part) return fp_fail(c, FP_ERR_OOM, "partial evaluation: scratch exhausted");
