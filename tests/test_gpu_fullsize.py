@@ -9,9 +9,11 @@
 * FFN: the oracle's verifier also checks the GPU proof against the GPU
   witness in full, and witness entries sampled at random are recomputed one
   by one from W and X;
-* MoE layer (387 sites, 8 GB of int4 weights): every protocol check of the
-  verifier runs, the direct evaluations of W and X for a sample of sites, and
-  sampled witness entries are recomputed one by one.
+* MoE layer (387 sites, 8 GB of int4 weights): the proof, the transcript states
+  and the witness must hash to the oracle's stored digests (byte parity); every
+  protocol check of the verifier runs as well, with the direct evaluations of W
+  and X for a sample of sites, and sampled witness entries are recomputed one
+  by one.
 """
 
 import hashlib
@@ -142,6 +144,10 @@ def test_moe_full_sampled(env):
     assert len(wl.sites) == 387
     proof, states, status, wits, flat = gpu_prove(env, wl, 0)
     assert status == 0
+    g = golden(5)
+    if g is not None:  # byte parity with the oracle's proof of the whole layer
+        assert g["sites"] == len(flat)
+        check_golden(g, proof, states, wits)
     spot_check(wl.sites, wits, n=200)
     rng = np.random.default_rng(5)
     mask = np.zeros(len(wl.sites), np.uint8)
