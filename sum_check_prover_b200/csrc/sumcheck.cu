@@ -316,6 +316,7 @@ struct MmDevice : MmSource {
     ScArgs P;
     const void* kern = nullptr;
     bool session = false;
+    bool weighted = false;  // the statement has more than one site: every site's sums carry its rho_s
 
     int start(const FpPoint& zr, const FpPoint& zc) override {
         std::map<int, uint64_t*> eqr, eqc;  // eq tables by prefix length
@@ -370,7 +371,8 @@ struct MmDevice : MmSource {
         if ((rc = fp_partial_many(c, pe.data(), (int)pe.size(), st))) return rc;
         if (n == 0) return FP_OK;
         int occ = 0;
-        kern = nsites > 1 ? (const void*)sc_session_kernel<true> : (const void*)sc_session_kernel<false>;
+        // a rank that holds one site of a larger statement still weights it by its rho_s
+        kern = weighted ? (const void*)sc_session_kernel<true> : (const void*)sc_session_kernel<false>;
         FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, SC_THREADS, 0));
         P.A[0] = bufA[0];
         P.A[1] = bufA[1];
@@ -556,6 +558,7 @@ int prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, const f
     mm_dims(sites, nsites, vM, vN, n);
     MmDevice dev;
     if ((rc = mm_device_setup(c, sites + lo, own, n, (cudaStream_t)stream, dev))) return rc;
+    dev.weighted = nsites > 1;
     rc = mm_protocol(tx, vM, vN, n, nsites, sh, dev, proof, proof_len);
     if (rc) dev.abandon();
     return rc;
