@@ -159,6 +159,15 @@ struct GlAcc {
             : "+l"(lo), "+l"(hi), "+r"(top)
             : "l"(plo), "l"(phi));
     }
+    // a b for a 64-bit a and a 32-bit b: two 32 x 32 products, a_lo b + 2^32 a_hi b
+    __device__ __forceinline__ void mac32(uint64_t a, uint32_t b) {
+        const uint64_t p0 = (uint64_t)(uint32_t)a * b, p1 = (uint64_t)(uint32_t)(a >> 32) * b;
+        const uint64_t plo = p0 + (p1 << 32);
+        const uint64_t phi = (p1 >> 32) + (plo < p0 ? 1ull : 0ull);
+        asm("add.cc.u64 %0, %0, %3;\n\taddc.cc.u64 %1, %1, %4;\n\taddc.u32 %2, %2, 0;"
+            : "+l"(lo), "+l"(hi), "+r"(top)
+            : "l"(plo), "l"(phi));
+    }
     __device__ __forceinline__ void add(uint64_t a) {
         asm("add.cc.u64 %0, %0, %3;\n\taddc.cc.u64 %1, %1, 0;\n\taddc.u32 %2, %2, 0;"
             : "+l"(lo), "+l"(hi), "+r"(top)
@@ -176,6 +185,14 @@ __device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
     uint32_t lo = (uint32_t)v, hi = (uint32_t)(v >> 32);
     lo = __shfl_xor_sync(0xffffffffu, lo, m);
     hi = __shfl_xor_sync(0xffffffffu, hi, m);
+    return ((uint64_t)hi << 32) | lo;
+}
+
+// lane src's 64-bit value
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+    uint32_t lo = (uint32_t)v, hi = (uint32_t)(v >> 32);
+    lo = __shfl_sync(0xffffffffu, lo, src);
+    hi = __shfl_sync(0xffffffffu, hi, src);
     return ((uint64_t)hi << 32) | lo;
 }
 

@@ -105,23 +105,39 @@ __global__ void __launch_bounds__(1024) hist_kernel(KeySrc K, int k, int64_t L, 
         for (int i = threadIdx.x; i < T; i += blockDim.x) sr[i] = 0;
     __syncthreads();
     uint32_t out_local = 0;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < K.n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t jr = (int64_t)K.r[i] + half;
+    const int lane = threadIdx.x & 31;
+    // the quotients cluster in a few bins (q is the rescaled output): lanes holding the same key
+    // add their count with one atomic, from the lowest of them. Every lane of a warp runs the same
+    // iterations (a lane past the keys matches no lane that holds one), so the matches take the
+    // full warp.
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < K.n; base += stride) {
+        const int64_t i = base + lane;
+        const bool in = i < K.n;
+        const int32_t rv = in ? K.r[i] : 0, qv = in ? K.q[i] : 0;
+        const uint64_t tag = (uint64_t)in << 32;
+        const unsigned same_r = __match_any_sync(0xffffffffu, (unsigned long long)(tag | (uint32_t)rv));
+        const unsigned same_q = __match_any_sync(0xffffffffu, (unsigned long long)(tag | (uint32_t)qv));
+        if (!in) continue;
+        const int64_t jr = (int64_t)rv + half;
         if (jr >= 0 && jr < T) {
-            if (rem_in_smem)
-                atomicAdd(&sr[jr], 1u);
-            else
-                atomicAdd(&m_rem[jr], 1u);
+            if (__ffs(same_r) - 1 == lane) {
+                if (rem_in_smem)
+                    atomicAdd(&sr[jr], (uint32_t)__popc(same_r));
+                else
+                    atomicAdd(&m_rem[jr], (uint32_t)__popc(same_r));
+            }
         } else {
             out_local++;
         }
-        const int64_t q = K.q[i];
-        if (q >= -HIST_WIN && q < HIST_WIN)
-            atomicAdd(&sq[q + HIST_WIN], 1u);
-        else if (q >= -32768 && q < 32768)
-            atomicAdd(&m_clamp[q + 32768], 1u);
-        else
+        const int64_t q = qv;
+        if (q >= -HIST_WIN && q < HIST_WIN) {
+            if (__ffs(same_q) - 1 == lane) atomicAdd(&sq[q + HIST_WIN], (uint32_t)__popc(same_q));
+        } else if (q >= -32768 && q < 32768) {
+            if (__ffs(same_q) - 1 == lane) atomicAdd(&m_clamp[q + 32768], (uint32_t)__popc(same_q));
+        } else {
             out_local++;
+        }
         if ((int32_t)K.y[i] != (q < -128 ? -128 : (q > 127 ? 127 : (int32_t)q))) out_local++;
     }
     if (out_local) atomicAdd(outside, out_local);
@@ -235,6 +251,137 @@ __global__ void __launch_bounds__(512) tree_chunk_kernel(KeySrc K, Chal C, TreeL
                 dst[(2 * tau + 1) * n1 + x] = Q;
             }
         }
+    }
+}
+
+// The first eleven levels above the leaves (v - 1 .. v - 11) from the keys, for v >= 12. A block
+// takes 2048-leaf chunks in turn: each thread builds the three levels above its 8 consecutive
+// leaves in registers, each warp the next five from its lanes' 32 nodes with shuffles, and warp 0
+// the last three from the block's 8 warp nodes; every level is written as it is formed. One
+// barrier per chunk instead of one per level.
+constexpr int kKeyTreeLevels = 11;
+constexpr int kKeyTreeThreads = 256;  // 8 leaves per thread: 2048 leaves per chunk
+
+struct KeyTreeOut {
+    TreeLayer lay[kKeyTreeLevels];  // lay[l]: level v - 1 - l
+};
+
+// (P, Q) of a parent from its children: (pL qR + pR qL, qL qR)
+__device__ __forceinline__ void tree_up(uint64_t pl, uint64_t ql, uint64_t pr, uint64_t qr, uint64_t& p, uint64_t& q) {
+    p = gl_add(gl_mul(pl, qr), gl_mul(pr, ql));
+    q = gl_mul(ql, qr);
+}
+
+__global__ void __launch_bounds__(kKeyTreeThreads) tree_keys_kernel(KeySrc K, Chal C, KeyTreeOut out, int64_t nchunks) {
+    __shared__ uint64_t ytab[256];
+    __shared__ uint64_t wnode[8][4];  // each warp's level v - 8 node: P0, Q0, P1, Q1
+    leaf_ytab_build(C, ytab);
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int64_t ch = blockIdx.x; ch < nchunks; ch += gridDim.x) {
+        const int64_t leaf0 = ch * 2048 + 8 * (int64_t)threadIdx.x;
+        int32_t r[8], q[8], y[8];
+        if (leaf0 + 8 <= K.n) {
+            const int4 r0 = __ldcs(reinterpret_cast<const int4*>(K.r + leaf0));
+            const int4 r1 = __ldcs(reinterpret_cast<const int4*>(K.r + leaf0 + 4));
+            const int4 q0 = __ldcs(reinterpret_cast<const int4*>(K.q + leaf0));
+            const int4 q1 = __ldcs(reinterpret_cast<const int4*>(K.q + leaf0 + 4));
+            const uint2 yv = __ldcs(reinterpret_cast<const uint2*>(K.y + leaf0));
+            r[0] = r0.x; r[1] = r0.y; r[2] = r0.z; r[3] = r0.w; r[4] = r1.x; r[5] = r1.y; r[6] = r1.z; r[7] = r1.w;
+            q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w; q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
+#pragma unroll
+            for (int j = 0; j < 8; j++) y[j] = (int32_t)(int8_t)(((j < 4 ? yv.x : yv.y) >> (8 * (j & 3))) & 0xFF);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; j++) key_at(K, leaf0 + j, r[j], q[j], y[j]);
+        }
+        // level v - 1 (4 nodes per thread), then v - 2 (2) and v - 3 (1), per table
+        uint64_t P[2][4], Q[2][4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const uint64_t a0 = gl_sub(C.alpha0, gl_from_i64(r[2 * j])), b0 = gl_sub(C.alpha0, gl_from_i64(r[2 * j + 1]));
+            const uint64_t a1 = gl_sub(ytab[y[2 * j] + 128], gl_from_i64(q[2 * j]));
+            const uint64_t b1 = gl_sub(ytab[y[2 * j + 1] + 128], gl_from_i64(q[2 * j + 1]));
+            P[0][j] = gl_add(a0, b0);
+            Q[0][j] = gl_mul(a0, b0);
+            P[1][j] = gl_add(a1, b1);
+            Q[1][j] = gl_mul(a1, b1);
+        }
+        const int64_t n1 = ch * 1024 + 4 * (int64_t)threadIdx.x;
+#pragma unroll
+        for (int t = 0; t < 2; t++) {
+            reinterpret_cast<ulonglong2*>(out.lay[0].P[t] + n1)[0] = make_ulonglong2(P[t][0], P[t][1]);
+            reinterpret_cast<ulonglong2*>(out.lay[0].P[t] + n1)[1] = make_ulonglong2(P[t][2], P[t][3]);
+            reinterpret_cast<ulonglong2*>(out.lay[0].Q[t] + n1)[0] = make_ulonglong2(Q[t][0], Q[t][1]);
+            reinterpret_cast<ulonglong2*>(out.lay[0].Q[t] + n1)[1] = make_ulonglong2(Q[t][2], Q[t][3]);
+            tree_up(P[t][0], Q[t][0], P[t][1], Q[t][1], P[t][0], Q[t][0]);
+            tree_up(P[t][2], Q[t][2], P[t][3], Q[t][3], P[t][1], Q[t][1]);
+        }
+        const int64_t n2 = ch * 512 + 2 * (int64_t)threadIdx.x;
+#pragma unroll
+        for (int t = 0; t < 2; t++) {
+            *reinterpret_cast<ulonglong2*>(out.lay[1].P[t] + n2) = make_ulonglong2(P[t][0], P[t][1]);
+            *reinterpret_cast<ulonglong2*>(out.lay[1].Q[t] + n2) = make_ulonglong2(Q[t][0], Q[t][1]);
+            tree_up(P[t][0], Q[t][0], P[t][1], Q[t][1], P[t][0], Q[t][0]);
+            out.lay[2].P[t][ch * 256 + threadIdx.x] = P[t][0];
+            out.lay[2].Q[t][ch * 256 + threadIdx.x] = Q[t][0];
+        }
+        // levels v - 4 .. v - 8 within the warp: lane x of a level takes the nodes of lanes 2x, 2x + 1
+        uint64_t p[2] = {P[0][0], P[1][0]}, qq[2] = {Q[0][0], Q[1][0]};
+#pragma unroll
+        for (int l = 3; l < 8; l++) {
+            const int nl = 32 >> (l - 2);  // nodes of this level in the warp
+            const int src = (2 * lane) & 31;
+#pragma unroll
+            for (int t = 0; t < 2; t++) {
+                const uint64_t pl = shfl_u64(p[t], src), ql = shfl_u64(qq[t], src);
+                const uint64_t pr = shfl_u64(p[t], src + 1), qr = shfl_u64(qq[t], src + 1);
+                uint64_t np, nq;
+                tree_up(pl, ql, pr, qr, np, nq);
+                p[t] = np;
+                qq[t] = nq;
+                if (lane < nl) {
+                    const int64_t g = (ch * 8 + warp) * (int64_t)nl + lane;
+                    out.lay[l].P[t][g] = np;
+                    out.lay[l].Q[t][g] = nq;
+                }
+            }
+        }
+        if (lane == 0) {
+            wnode[warp][0] = p[0];
+            wnode[warp][1] = qq[0];
+            wnode[warp][2] = p[1];
+            wnode[warp][3] = qq[1];
+        }
+        __syncthreads();
+        // levels v - 9 .. v - 11 from the 8 warp nodes, in warp 0
+        if (warp == 0) {
+            uint64_t bp[2], bq[2];
+#pragma unroll
+            for (int t = 0; t < 2; t++) {
+                bp[t] = lane < 8 ? wnode[lane][2 * t] : 0ull;
+                bq[t] = lane < 8 ? wnode[lane][2 * t + 1] : 0ull;
+            }
+#pragma unroll
+            for (int l = 8; l < kKeyTreeLevels; l++) {
+                const int nl = 8 >> (l - 7);
+                const int src = (2 * lane) & 31;
+#pragma unroll
+                for (int t = 0; t < 2; t++) {
+                    const uint64_t pl = shfl_u64(bp[t], src), ql = shfl_u64(bq[t], src);
+                    const uint64_t pr = shfl_u64(bp[t], src + 1), qr = shfl_u64(bq[t], src + 1);
+                    uint64_t np, nq;
+                    tree_up(pl, ql, pr, qr, np, nq);
+                    bp[t] = np;
+                    bq[t] = nq;
+                    if (lane < nl) {
+                        out.lay[l].P[t][ch * nl + lane] = np;
+                        out.lay[l].Q[t][ch * nl + lane] = nq;
+                    }
+                }
+            }
+        }
+        __syncthreads();  // wnode is rewritten by the next chunk
     }
 }
 
@@ -558,19 +705,35 @@ __global__ void __launch_bounds__(LEAF ? LU_LEAF_THREADS : LU_THREADS, LEAF ? FP
 
 // ---- leaf claims: MLEs of the key columns at z (split eq: hi x lo) ----------------
 
+// Leaf claims: the MLEs of the padded key columns at z, sum_x eq(z, x) f(x) with the eq split
+// as eq_hi[x >> lo] eq_lo[x & (2^lo - 1)]. A block takes groups of 2^lo consecutive keys in turn
+// (eq_hi constant within one): each thread sums eq_lo[.] (f + off) exactly over its keys of the
+// group (64 x 32-bit products, f + off >= 0: off = 2^31 for r and q, 128 for y), removes
+// off sum eq_lo, and weights the group's value by eq_hi once. Padding keys are 0 and add nothing.
 __global__ void __launch_bounds__(LU_THREADS) leaf_eval_kernel(KeySrc K, const uint64_t* __restrict__ ehi,
-                                                               const uint64_t* __restrict__ elo, int lo_bits, int64_t L,
+                                                               const uint64_t* __restrict__ elo, int lo_bits,
                                                                uint64_t* part, unsigned int* ticket,
                                                                uint64_t* __restrict__ out) {
-    uint64_t acc[3] = {0, 0, 0};
-    const int64_t mask = (1ll << lo_bits) - 1;
-    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < K.n && x < L;
-         x += (int64_t)gridDim.x * blockDim.x) {
-        const uint64_t e = gl_mul(ehi[x >> lo_bits], elo[x & mask]);
-        acc[0] = gl_add(acc[0], gl_mul(e, gl_from_i64(K.r[x])));
-        acc[1] = gl_add(acc[1], gl_mul(e, gl_from_i64(K.q[x])));
-        acc[2] = gl_add(acc[2], gl_mul(e, gl_from_i64(K.y[x])));
+    const int64_t G = 1ll << lo_bits;
+    const int64_t ngroups = (K.n + G - 1) >> lo_bits;
+    GlAcc tot[3];
+    for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+        const int64_t x0 = g << lo_bits;
+        const int64_t xe = x0 + G < K.n ? x0 + G : K.n;
+        GlAcc a[3], es;
+        for (int64_t x = x0 + threadIdx.x; x < xe; x += blockDim.x) {
+            const uint64_t e = __ldg(elo + (x - x0));
+            a[0].mac32(e, (uint32_t)K.r[x] ^ 0x80000000u);
+            a[1].mac32(e, (uint32_t)K.q[x] ^ 0x80000000u);
+            a[2].mac32(e, (uint32_t)(K.y[x] + 128));
+            es.add(e);
+        }
+        const uint64_t esum = es.value(), eh = __ldg(ehi + g);
+        const uint64_t off[3] = {1ull << 31, 1ull << 31, 128ull};
+#pragma unroll
+        for (int i = 0; i < 3; i++) tot[i].mac(eh, gl_sub(a[i].value(), gl_mul(off[i], esum)));
     }
+    uint64_t acc[3] = {tot[0].value(), tot[1].value(), tot[2].value()};
     if (grid_sum_gl<3>(acc, part, ticket) && threadIdx.x == 0) {
         out[0] = acc[0];
         out[1] = acc[1];
@@ -611,7 +774,15 @@ int fp_lookup_keys(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st,
     int64_t nk = 0;
     for (int s = 0; s < nsites; s++) nk += (int64_t)sites[s].M * sites[s].N;
     K->n = nk;
-    if (nsites == 1) {
+    // the sites' columns already back to back in site order (one site, or buffers laid out so):
+    // read in place, no copy
+    bool in_place = true;
+    int64_t off = 0;
+    for (int s = 0; s < nsites && in_place; s++) {
+        in_place = sites[s].q == sites[0].q + off && sites[s].r == sites[0].r + off && sites[s].y == sites[0].y + off;
+        off += (int64_t)sites[s].M * sites[s].N;
+    }
+    if (in_place) {
         K->r = sites[0].r;
         K->q = sites[0].q;
         K->y = sites[0].y;
@@ -623,7 +794,7 @@ int fp_lookup_keys(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st,
     GatherSite* dgs = (GatherSite*)fp_alloc(c->dev, sizeof(GatherSite) * nsites);
     GatherSite* hgs = (GatherSite*)fp_alloc(c->host, sizeof(GatherSite) * nsites);
     if (!r || !q || !y || !dgs || !hgs) return fp_fail(c, FP_ERR_OOM, "lookup keys: scratch exhausted");
-    int64_t off = 0;
+    off = 0;
     for (int s = 0; s < nsites; s++) {
         hgs[s] = GatherSite{sites[s].q, sites[s].r, sites[s].y, off};
         off += (int64_t)sites[s].M * sites[s].N;
@@ -754,8 +925,26 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
     if (!part || !small || !hsmall || !E || !zb[2]) return fp_fail(c, FP_ERR_OOM, "logup: scratch exhausted");
 
     if (v >= 2) {
-        // layers v-1 .. 1, kTreeLevels per launch
+        // layers v-1 .. 1: the first eleven from the keys in one persistent launch (v >= 12), the
+        // rest kTreeLevels per launch
         int L0 = v;
+        // the vector loads of 8 keys need 16-byte aligned key columns (8-byte for y)
+        const bool keys_aligned = (uintptr_t)K.r % 16 == 0 && (uintptr_t)K.q % 16 == 0 && (uintptr_t)K.y % 8 == 0;
+        if (v >= 12 && keys_aligned) {
+            KeyTreeOut ko;
+            for (int l = 0; l < kKeyTreeLevels; l++) ko.lay[l] = lay[v - 1 - l];
+            const int64_t nchunks = (1ll << v) / 2048;
+            int occ_t = 0;
+            FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_t, tree_keys_kernel, kKeyTreeThreads, 0));
+            const unsigned blocks = (unsigned)std::min<int64_t>(nchunks, (int64_t)std::max(1, occ_t) * c->num_sms);
+            const double nodes = (double)(1ll << v) - (double)(1ll << (v - kKeyTreeLevels));
+            int slot;
+            fp_tic(c, st, K_TREE_LEAF, 9.0 * (double)(1ll << v) + 32.0 * nodes, &slot);
+            tree_keys_kernel<<<blocks, kKeyTreeThreads, 0, st>>>(K, C, ko, nchunks);
+            fp_toc(c, st, slot);
+            FP_CUDA(c, cudaGetLastError());
+            L0 = v - kKeyTreeLevels;
+        }
         while (L0 > 1) {
             const int levels = std::min(kTreeLevels, L0 - 1);
             TreeOut to;
@@ -958,8 +1147,9 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
         if ((rc = fp_eq_table(c, zl, elo, st))) return rc;
         int slot;
         fp_tic(c, st, K_LEAF_EVAL, 9.0 * nk, &slot);
-        leaf_eval_kernel<<<grid_for(c, nk, LU_THREADS), LU_THREADS, 0, st>>>(K, ehi, elo, lo_bits, L, part, c->tickets,
-                                                                             small);
+        const int64_t ngroups = (nk + (1ll << lo_bits) - 1) >> lo_bits;
+        const unsigned lgrid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ngroups, 8ll * c->num_sms));
+        leaf_eval_kernel<<<lgrid, LU_THREADS, 0, st>>>(K, ehi, elo, lo_bits, part, c->tickets, small);
         fp_toc(c, st, slot);
         FP_CUDA(c, cudaGetLastError());
         FP_CUDA(c, cudaMemcpyAsync(hsmall, small, 24, cudaMemcpyDeviceToHost, st));

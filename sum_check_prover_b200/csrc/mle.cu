@@ -50,20 +50,45 @@ __global__ void __launch_bounds__(CL_THREADS)
     const int64_t total = (int64_t)S.M * S.N;
     const int64_t e0 = (b - S.first_block) * CL_ELEMS;
     const int64_t e1 = min(total, e0 + CL_ELEMS);
-    uint64_t acc = 0;
-    for (int64_t e = e0 + threadIdx.x; e < e1; e += CL_THREADS) {
-        int j, i;
-        if (total < (1ll << 32)) {
-            const uint32_t e32 = (uint32_t)e, m32 = (uint32_t)S.M;
-            j = (int)(e32 / m32);
-            i = (int)(e32 - (uint32_t)j * m32);
-        } else {
-            j = (int)(e / S.M);
-            i = (int)(e - (int64_t)j * S.M);
+    // Row j of the N x M output is contiguous: sum_i eq_row[i] (2^k q + r) over a thread's
+    // elements of row j is kept exactly (q + 2^31 and r + 2^31 as 32-bit factors, the offsets
+    // removed with the sum of the weights) and weighted by eq_col[j] once the thread leaves row j.
+    GlAcc tot, aq, ar, es;
+    int64_t e = e0 + threadIdx.x;
+    int64_t j = e / S.M, i = e - j * S.M;
+    int64_t jcur = j;
+    const uint64_t k2 = 1ull << S.k;
+    auto flush = [&]() {
+        const uint64_t w = es.value();
+        const uint64_t off = gl_mul(1ull << 31, w);
+        const uint64_t vq = gl_sub(aq.value(), off), vr = gl_sub(ar.value(), off);
+        tot.mac(__ldg(S.eq_col + jcur), gl_add(gl_mul(k2, vq), vr));
+        aq = GlAcc();
+        ar = GlAcc();
+        es = GlAcc();
+    };
+    for (; e < e1; e += CL_THREADS) {
+        if (j != jcur) {
+            flush();
+            jcur = j;
         }
-        const int64_t yv = ((int64_t)S.q[e] << S.k) + (int64_t)S.r[e];
-        acc = gl_add(acc, gl_mul(gl_mul(S.eq_row[i], S.eq_col[j]), gl_from_i64(yv)));
+        const uint64_t w = __ldg(S.eq_row + i);
+        aq.mac32(w, (uint32_t)S.q[e] ^ 0x80000000u);
+        ar.mac32(w, (uint32_t)S.r[e] ^ 0x80000000u);
+        es.add(w);
+        i += CL_THREADS;
+        if (i >= S.M) {
+            if (S.M >= CL_THREADS) {
+                i -= S.M;
+                j++;
+            } else {
+                j += i / S.M;
+                i %= S.M;
+            }
+        }
     }
+    if (e0 + threadIdx.x < e1) flush();
+    uint64_t acc = tot.value();
     acc = warp_sum_gl(acc);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
     __syncthreads();

@@ -44,6 +44,15 @@ def upload(wl, device: str = "cuda"):
                          r=torch.zeros((n, m), dtype=torch.int32, device=dev),
                          y=torch.zeros((n, m), dtype=torch.int8, device=dev))
     cache = {}
+    # the witness of the sites without a shared output buffer, one tensor per column in site
+    # order, so the lookup section reads its keys in place
+    free = [s for s in wl.sites if s.out_group is None]
+    nfree = sum(s.M * s.N for s in free)
+    col_q = torch.empty(max(1, nfree), dtype=torch.int32, device=dev)
+    col_r = torch.empty(max(1, nfree), dtype=torch.int32, device=dev)
+    col_y = torch.empty(max(1, nfree), dtype=torch.int8, device=dev)
+    keep["columns"] = (col_q, col_r, col_y)
+    foff = 0
 
     def t(a):
         key = id(a)
@@ -66,9 +75,11 @@ def upload(wl, device: str = "cuda"):
             r = gb["r"].view(-1)[off:off + n].view(s.N, s.M)
             y = gb["y"].view(-1)[off:off + n].view(s.N, s.M)
         else:
-            q = torch.empty((s.N, s.M), dtype=torch.int32, device=dev)
-            r = torch.empty((s.N, s.M), dtype=torch.int32, device=dev)
-            y = torch.empty((s.N, s.M), dtype=torch.int8, device=dev)
+            n = s.M * s.N
+            q = col_q[foff:foff + n].view(s.N, s.M)
+            r = col_r[foff:foff + n].view(s.N, s.M)
+            y = col_y[foff:foff + n].view(s.N, s.M)
+            foff += n
         if s.w_link is not None:
             src, off = s.w_link
             w = y_buffer(src)[off:off + s.M * s.K].view(s.M, s.K)
