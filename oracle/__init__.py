@@ -73,6 +73,10 @@ REASONS = {
     42: "lhr_round",
     43: "lhr_final",
     44: "lhr_open",
+    45: "dsp_claim",
+    46: "dsp_round",
+    47: "dsp_final",
+    48: "dsp_open",
 }
 
 
@@ -139,6 +143,10 @@ def lib():
         L.orc_prove_hi.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64,
                                    C.POINTER(u64), vp, C.POINTER(u64)]
         L.orc_verify_hi.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp]
+        L.orc_dsp_prove.restype = C.c_int
+        L.orc_dsp_prove.argtypes = [vp, vp, vp, vp, u64, u64, C.c_int, vp, u64, C.POINTER(u64)]
+        L.orc_dsp_verify.restype = C.c_int
+        L.orc_dsp_verify.argtypes = [vp, vp, vp, vp, u64, u64, C.c_int, vp, u64, vp]
         L.orc_had_prove.restype = C.c_int
         L.orc_had_prove.argtypes = [vp, vp, vp, u64, vp, u64, C.POINTER(u64)]
         L.orc_had_verify.restype = C.c_int
@@ -850,6 +858,50 @@ def route_verify(seed: int, l, H, D, T: int, E: int, proof: bytes):
     det = np.zeros(2, dtype=np.int64)
     tx = L.orc_tx_new(seed)
     rc = L.orc_route_verify(tx, _ptr(a), _ptr(h), _ptr(d), T, E, _ptr(pb), len(proof), _ptr(det))
+    L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+# ---- MoE dispatch: the experts' stacked inputs are the routed permutation of X ----------
+
+def _dsp_args(X, e, D):
+    x = np.ascontiguousarray(np.asarray(X, dtype=np.int8))
+    ev = np.ascontiguousarray(np.asarray(e, dtype=np.int32).reshape(-1))
+    d = np.ascontiguousarray(np.asarray(D, dtype=np.int8))
+    if x.ndim != 2 or d.shape != x.shape or ev.size != x.shape[0]:
+        raise ValueError("dispatch: X and D must be T x K and e of length T")
+    return x, ev, d
+
+
+def dsp_prove(seed: int, X, e, D, E: int):
+    """The dispatch proof (orc_dsp_prove) for token-major X (T x K int8), experts e (T) and the
+    stacked expert inputs D (T x K); returns (proof bytes, transcript state)."""
+    L = lib()
+    x, ev, d = _dsp_args(X, e, D)
+    T, K = x.shape
+    n = C.c_uint64(0)
+    tx = L.orc_tx_new(seed)
+    L.orc_dsp_prove(tx, _ptr(x), _ptr(ev), _ptr(d), T, K, E, None, 0, C.byref(n))
+    L.orc_tx_free(tx)
+    buf = np.zeros(max(1, n.value), dtype=np.uint8)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_dsp_prove(tx, _ptr(x), _ptr(ev), _ptr(d), T, K, E, _ptr(buf), n.value, C.byref(n))
+    st = C.create_string_buffer(32)
+    L.orc_tx_state(tx, st)
+    L.orc_tx_free(tx)
+    if rc != 0:
+        raise ValueError(f"orc_dsp_prove failed ({rc})")
+    return buf[: n.value].tobytes(), st.raw
+
+
+def dsp_verify(seed: int, X, e, D, E: int, proof: bytes):
+    L = lib()
+    x, ev, d = _dsp_args(X, e, D)
+    T, K = x.shape
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    tx = L.orc_tx_new(seed)
+    rc = L.orc_dsp_verify(tx, _ptr(x), _ptr(ev), _ptr(d), T, K, E, _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
 

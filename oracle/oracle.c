@@ -3607,3 +3607,194 @@ int orc_verify_hi(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, c
     if (rd.pos != rd.len) return REJ_FORMAT;
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MoE dispatch (next row f3: "prove the routing computation and the choice  */
+/* of expert", How fast can FlashProve go, 2 Background, the note on MoE      */
+/* layers; the routing proof covers the choice, this statement the moving of */
+/* each token's activations to its expert). With T tokens, X the layer input */
+/* (T x K int8, token-major), e_t the expert of token t (int32, < E) and D   */
+/* the experts' inputs stacked expert by expert (T x K int8: the rows of X    */
+/* routed to expert 0 in token order, then expert 1, ...), D = Pi X for the  */
+/* permutation that sends token t to position                                */
+/*   pos(t) = #{t' : e_t' < e_t} + #{t' < t : e_t' = e_t}.                   */
+/* Row bits first, T and K zero-padded to 2^vT, 2^vK:                        */
+/*   absorb "dsp_site" D(X) || D(e, int32 little-endian) || D(D);            */
+/*   squeeze r_row (vT, "dsp_row") and r_col (vK, "dsp_col");               */
+/*   send c = D~(r_row, r_col) ("dsp_claim");                                */
+/*   sum-check over t of P(t) B(t), P(t) = eq(r_row, pos(t)) and              */
+/*   B(t) = X~(t, r_col) (both 0 on padded t), degree 2: rounds g(0), g(1),  */
+/*   g(2) ("dsp_round"), "dsp_chal"; send P(rho), B(rho) ("dsp_final").      */
+/* Since D~(r, c) = sum_t eq(r, pos(t)) X~(t, c) exactly when D = Pi X (on   */
+/* the cube, hence everywhere), the verifier checks c against D, the rounds, */
+/* the end P(rho) B(rho), and P(rho) = sum_t eq(rho, t) eq(r_row, pos(t)),   */
+/* B(rho) = X~(rho, r_col) from e and X (standing in for openings).          */
+/* ------------------------------------------------------------------------ */
+
+enum {
+    REJ_DSP_CLAIM = 45,  /* c != D~(r_row, r_col) */
+    REJ_DSP_ROUND = 46,  /* g(0) + g(1) != running claim */
+    REJ_DSP_FINAL = 47,  /* the end != P(rho) B(rho) */
+    REJ_DSP_OPEN = 48    /* P(rho) or B(rho) != its recomputation (detail: which) */
+};
+
+static void dsp_absorb_site(orc_tx* t, const int8_t* X, const int32_t* e, const int8_t* D, u64 T, u64 K) {
+    uint8_t d[96];
+    orc_tree_digest(X, T * K, d);
+    uint8_t* b = (uint8_t*)calloc(4 * T + 1, 1);
+    for (u64 i = 0; i < T; i++) put_le(b + 4 * i, (u64)(u32)e[i], 4);
+    orc_tree_digest(b, 4 * T, d + 32);
+    free(b);
+    orc_tree_digest(D, T * K, d + 64);
+    orc_tx_absorb(t, "dsp_site", d, 96);
+}
+
+/* pos(t) of every token; -1 if some e_t is outside [0, E) */
+static int dsp_positions(const int32_t* e, u64 T, int E, u64* pos) {
+    u64* before = (u64*)calloc((size_t)E + 1, sizeof(u64));
+    for (u64 t = 0; t < T; t++) {
+        if (e[t] < 0 || e[t] >= E) {
+            free(before);
+            return -1;
+        }
+        before[e[t] + 1]++;
+    }
+    for (int x = 0; x < E; x++) before[x + 1] += before[x];
+    for (u64 t = 0; t < T; t++) pos[t] = before[e[t]]++;
+    free(before);
+    return 0;
+}
+
+/* P (eq(r_row, pos(t)) for t < T) and B (X~(t, r_col)) over 2^vT entries */
+static void dsp_vectors(const int8_t* X, const u64* pos, u64 T, u64 K, const u64* rr, int vT, const u64* rc, int vK,
+                        u64* P, u64* B) {
+    u64 LT = (u64)1 << vT;
+    u64* er = (u64*)malloc(sizeof(u64) * LT);
+    u64* ec = (u64*)malloc(sizeof(u64) * ((u64)1 << vK));
+    orc_eq_table(rr, vT, er);
+    orc_eq_table(rc, vK, ec);
+    for (u64 t = 0; t < LT; t++) {
+        P[t] = 0;
+        B[t] = 0;
+        if (t >= T) continue;
+        P[t] = er[pos[t]];
+        for (u64 k = 0; k < K; k++) B[t] = orc_fadd(B[t], orc_fmul(ec[k], orc_fint(X[t * K + k])));
+    }
+    free(er);
+    free(ec);
+}
+
+static u64 dsp_claim(const int8_t* D, u64 T, u64 K, const u64* rr, int vT, const u64* rc, int vK) {
+    u64* er = (u64*)malloc(sizeof(u64) * ((u64)1 << vT));
+    u64* ec = (u64*)malloc(sizeof(u64) * ((u64)1 << vK));
+    orc_eq_table(rr, vT, er);
+    orc_eq_table(rc, vK, ec);
+    u64 c = 0;
+    for (u64 p = 0; p < T; p++)
+        for (u64 k = 0; k < K; k++) c = orc_fadd(c, orc_fmul(orc_fmul(er[p], ec[k]), orc_fint(D[p * K + k])));
+    free(er);
+    free(ec);
+    return c;
+}
+
+int orc_dsp_prove(void* txh, const int8_t* X, const int32_t* e, const int8_t* D, u64 T, u64 K, int E, uint8_t* proof,
+                  u64 cap, u64* len) {
+    if (T < 1 || K < 1 || E < 1) return -1;
+    orc_tx* t = (orc_tx*)txh;
+    int vT = orc_log2_ceil(T), vK = orc_log2_ceil(K);
+    u64 LT = (u64)1 << vT;
+    u64* pos = (u64*)malloc(sizeof(u64) * T);
+    if (dsp_positions(e, T, E, pos)) {
+        free(pos);
+        return -1;
+    }
+    pbuf pb = {proof, cap, 0, 0};
+    dsp_absorb_site(t, X, e, D, T, K);
+    u64* rr = (u64*)malloc(sizeof(u64) * (vT + 1));
+    u64* rc = (u64*)malloc(sizeof(u64) * (vK + 1));
+    for (int i = 0; i < vT; i++) rr[i] = orc_tx_squeeze(t, "dsp_row");
+    for (int i = 0; i < vK; i++) rc[i] = orc_tx_squeeze(t, "dsp_col");
+    u64 c = dsp_claim(D, T, K, rr, vT, rc, vK);
+    send_fe(t, &pb, "dsp_claim", &c, 1);
+    u64* P = (u64*)malloc(sizeof(u64) * LT);
+    u64* B = (u64*)malloc(sizeof(u64) * LT);
+    dsp_vectors(X, pos, T, K, rr, vT, rc, vK, P, B);
+    u64 Lr = LT;
+    for (int r = 0; r < vT; r++) {
+        u64 h = Lr >> 1;
+        u64 g[3] = {0, 0, 0};
+        for (u64 b = 0; b < h; b++)
+            for (u64 X_ = 0; X_ < 3; X_++) {
+                u64 p = orc_fadd(P[b], orc_fmul(X_, orc_fsub(P[h + b], P[b])));
+                u64 q = orc_fadd(B[b], orc_fmul(X_, orc_fsub(B[h + b], B[b])));
+                g[X_] = orc_fadd(g[X_], orc_fmul(p, q));
+            }
+        send_fe(t, &pb, "dsp_round", g, 3);
+        u64 rho = orc_tx_squeeze(t, "dsp_chal");
+        for (u64 b = 0; b < h; b++) {
+            P[b] = orc_fadd(P[b], orc_fmul(rho, orc_fsub(P[h + b], P[b])));
+            B[b] = orc_fadd(B[b], orc_fmul(rho, orc_fsub(B[h + b], B[b])));
+        }
+        Lr = h;
+    }
+    u64 fin[2] = {P[0], B[0]};
+    send_fe(t, &pb, "dsp_final", fin, 2);
+    free(pos);
+    free(rr);
+    free(rc);
+    free(P);
+    free(B);
+    *len = pb.len;
+    return pb.overflow ? -2 : 0;
+}
+
+int orc_dsp_verify(void* txh, const int8_t* X, const int32_t* e, const int8_t* D, u64 T, u64 K, int E,
+                   const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    if (T < 1 || K < 1 || E < 1) return REJ_ARGS;
+    orc_tx* t = (orc_tx*)txh;
+    int vT = orc_log2_ceil(T), vK = orc_log2_ceil(K);
+    u64 LT = (u64)1 << vT;
+    u64* pos = (u64*)malloc(sizeof(u64) * T);
+    u64* rr = (u64*)malloc(sizeof(u64) * (vT + 1));
+    u64* rcol = (u64*)malloc(sizeof(u64) * (vK + 1));
+    u64* rho = (u64*)malloc(sizeof(u64) * (vT + 1));
+    u64* P = (u64*)malloc(sizeof(u64) * LT);
+    u64* B = (u64*)malloc(sizeof(u64) * LT);
+    int rc = 0;
+    prd rdd = {proof, len, 0, 0};
+    prd* rd = &rdd;
+    if (dsp_positions(e, T, E, pos)) FAIL(REJ_ARGS, 0, 0);
+    dsp_absorb_site(t, X, e, D, T, K);
+    for (int i = 0; i < vT; i++) rr[i] = orc_tx_squeeze(t, "dsp_row");
+    for (int i = 0; i < vK; i++) rcol[i] = orc_tx_squeeze(t, "dsp_col");
+    u64 c;
+    rd_fe(t, rd, "dsp_claim", &c, 1);
+    if (rd->bad) FAIL(REJ_FORMAT, 12, 0);
+    if (c != dsp_claim(D, T, K, rr, vT, rcol, vK)) FAIL(REJ_DSP_CLAIM, 0, 0);
+    u64 claim = c;
+    for (int i = 0; i < vT; i++) {
+        u64 g[3];
+        rd_fe(t, rd, "dsp_round", g, 3);
+        if (rd->bad) FAIL(REJ_FORMAT, 13, i);
+        if (orc_fadd(g[0], g[1]) != claim) FAIL(REJ_DSP_ROUND, i, 0);
+        rho[i] = orc_tx_squeeze(t, "dsp_chal");
+        claim = orc_lagrange(g, 3, rho[i]);
+    }
+    u64 fin[2];
+    rd_fe(t, rd, "dsp_final", fin, 2);
+    if (rd->bad) FAIL(REJ_FORMAT, 14, 0);
+    if (orc_fmul(fin[0], fin[1]) != claim) FAIL(REJ_DSP_FINAL, 0, 0);
+    dsp_vectors(X, pos, T, K, rr, vT, rcol, vK, P, B);
+    if (orc_mle_eval(P, LT, rho, vT) != fin[0]) FAIL(REJ_DSP_OPEN, 0, 0);
+    if (orc_mle_eval(B, LT, rho, vT) != fin[1]) FAIL(REJ_DSP_OPEN, 1, 0);
+    if (rd->pos != rd->len) FAIL(REJ_FORMAT, -1, 0);
+done:
+    free(pos);
+    free(rr);
+    free(rcol);
+    free(rho);
+    free(P);
+    free(B);
+    return rc;
+}

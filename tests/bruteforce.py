@@ -1087,3 +1087,46 @@ def lu2_prove(seed: int, sites, wits) -> bytes:
         z = rho_l + [sq("lu2_mu")]
     send("lu2_leaf", [x_mle(rp, z), x_mle(qp, z), x_mle(yp, z)])
     return bytes(out)
+
+
+def dsp_prove(seed: int, X, e, D, E: int) -> bytes:
+    """The MoE dispatch proof from definitions: pos(t) by a stable sort of the tokens by
+    expert, every MLE a hypercube sum at field points (no folding)."""
+    X = np.asarray(X, dtype=np.int64)
+    D = np.asarray(D, dtype=np.int64)
+    e = [int(v) for v in np.asarray(e).reshape(-1)]
+    T, K = X.shape
+    vT, vK = log2c(T), log2c(K)
+    order = sorted(range(T), key=lambda t: (e[t], t))  # expert-major, token order within
+    pos = [0] * T
+    for p, t in enumerate(order):
+        pos[t] = p
+    tx = Tx(seed)
+    out = bytearray()
+
+    def send(label, vals):
+        b = fe_bytes(vals)
+        out.extend(b)
+        tx.absorb(label, b)
+
+    tx.absorb("dsp_site", tree_digest(X.astype(np.int8).tobytes()) +
+              tree_digest(np.asarray(e, "<i4").tobytes()) + tree_digest(D.astype(np.int8).tobytes()))
+    rr = [tx.squeeze("dsp_row") for _ in range(vT)]
+    rc = [tx.squeeze("dsp_col") for _ in range(vK)]
+    send("dsp_claim", [mle2(D, rr, rc)])
+    Pv = [eq_point(rr, pos[t]) for t in range(T)]
+    Bv = [mle(X[t], rc) for t in range(T)]
+    rho = []
+    for t in range(vT):
+        rest = vT - t - 1
+        g = []
+        for Xp in range(3):
+            acc = 0
+            for bb in range(1 << rest):
+                w = rho + [Xp] + [(bb >> (rest - 1 - i)) & 1 for i in range(rest)]
+                acc += mle_at(Pv, w) * mle_at(Bv, w)
+            g.append(acc % P)
+        send("dsp_round", g)
+        rho.append(tx.squeeze("dsp_chal"))
+    send("dsp_final", [mle_at(Pv, rho), mle_at(Bv, rho)])
+    return bytes(out)

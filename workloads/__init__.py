@@ -183,6 +183,17 @@ def _moe(seed: int, E=128, d=5120, ffn=8192, T=8192, k=12, experts=None, shared=
                     description=f"{E} experts d={d} ffn={ffn} T={T} top-1 + shared, k={k}")
 
 
+def moe_dispatch(seed: int, E=128, d=5120, T=8192, experts=None):
+    """The MoE layer's dispatch statement: the layer input X (T x d, the tensor the experts'
+    gate and up sites read), the routing e (the expert of every token) and D, the experts'
+    inputs stacked expert by expert (each expert's tokens in token order: the rows of those
+    sites' activations). The same draws as _moe's (seeds 100 and 99)."""
+    x = activations(_rng(seed, 100), (T, d))
+    route = _rng(seed, 99).integers(0, E, size=T)
+    D = np.concatenate([x[route == e] for e in range(E)])
+    return x, route.astype(np.int32), D
+
+
 def _attn_dense(seed: int, d=5120, nq=40, nkv=8, hd=128, B=64, ctx=2048, ffn=16384, k=12) -> Workload:
     """Decode step of a GQA attention + dense MLP layer, B requests x 1 token.
 
