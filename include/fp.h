@@ -520,6 +520,28 @@ int sumcheck_prove_routing(fp_ctx* ctx, fp_tx* tx, const int8_t* logits, int64_t
                            uint8_t* proof, size_t* proof_len, void* stream);
 
 /*
+ * MoE dispatch ("How fast can FlashProve go", 2 Background, the note on MoE
+ * layers: the routing is proven): the experts' inputs D are the rows of the
+ * layer input X moved to their experts. X: device, T x K int8 token-major (the
+ * tensor the layer's gate and up sites read); e: device, T int32, the expert
+ * of every token (the routing proof's choice), each in [0, E); D: device,
+ * T x K int8, the experts' inputs stacked expert by expert, each expert's
+ * tokens in token order. The call continues tx:
+ *   absorb "dsp_site" D(X) || D(e) || D(D); squeeze r_row ("dsp_row",
+ *   ceil(log2 T) coordinates) and r_col ("dsp_col", ceil(log2 K)); send
+ *   c = D~(r_row, r_col) ("dsp_claim"); ceil(log2 T) degree-2 rounds of
+ *   sum_t eq(r_row, pos(t)) X~(t, r_col), pos(t) = #{t' : e_t' < e_t} +
+ *   #{t' < t : e_t' = e_t} ("dsp_round" g(0), g(1), g(2), "dsp_chal"); send
+ *   both factors at rho ("dsp_final").
+ * The verifier checks c against D, the rounds, the end, and the factors
+ * against e and X. Proof bytes: 8 + 24 ceil(log2 T) + 16. 1 <= T, K <= 2^24,
+ * 1 <= E <= 2^20, else FP_ERR_SHAPE; an expert index outside [0, E) gives
+ * FP_ERR_ARG; proof / proof_len as for sumcheck_prove_matmul.
+ */
+int sumcheck_prove_dispatch(fp_ctx* ctx, fp_tx* tx, const int8_t* X, const int32_t* e, const int8_t* D, int64_t T,
+                            int64_t K, int E, uint8_t* proof, size_t* proof_len, void* stream);
+
+/*
  * The host half of sumcheck_prove_routing up to "route_final" (n variables);
  * tx must have absorbed "route_site". Callback kinds:
  *   FP_VAL_START: in = z_1..z_n, w_1..w_n, lambda1, lambda2 (2 n + 2 words), t = n;

@@ -105,6 +105,7 @@ def lib():
     L.fp_mm_shard_protocol_drive.argtypes = [vp, C.POINTER(_Site), i32, C.POINTER(_Shard), _VALUES_FN, vp, vp,
                                              C.POINTER(sz)]
     L.logup_prove_rescale_hi.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
+    L.sumcheck_prove_dispatch.argtypes = [vp, vp, vp, vp, vp, C.c_int64, C.c_int64, i32, vp, C.POINTER(sz), vp]
     L.fp_lhr_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.fp_ctx_set_profiling.argtypes = [vp, i32]
     L.fp_session_selftest.argtypes = [vp, vp]
@@ -941,6 +942,18 @@ class Context:
         rc = self._check(self._L.logup_prove_rescale_hi(self.h, tx.h, arr, len(sites), buf, C.byref(n),
                                                         _stream(stream)), "logup_prove_rescale_hi")
         return buf.raw[: n.value], rc
+
+    def prove_dispatch(self, tx: Transcript, X, e, D, E: int, stream=None) -> bytes:
+        """The MoE dispatch proof: X (T x K int8, the layer input), e (T int32 experts) and D
+        (T x K int8, the experts' inputs stacked expert by expert), device tensors; continues tx."""
+        T, K = int(X.shape[0]), int(X.shape[1])
+        n = C.c_size_t(0)
+        self._L.sumcheck_prove_dispatch(self.h, tx.h, _ptr(X), _ptr(e), _ptr(D), T, K, E, None, C.byref(n),
+                                        _stream(stream))
+        buf = C.create_string_buffer(max(1, n.value))
+        self._check(self._L.sumcheck_prove_dispatch(self.h, tx.h, _ptr(X), _ptr(e), _ptr(D), T, K, E, buf, C.byref(n),
+                                                    _stream(stream)), "sumcheck_prove_dispatch")
+        return buf.raw[: n.value]
 
     def set_profiling(self, on):
         """False/0: off; True/1: one launch per sum-check round, each timed; 2: time the

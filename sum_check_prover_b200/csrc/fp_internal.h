@@ -69,6 +69,8 @@ enum FpKernel {
     K_LHR_COLUMN,
     K_LHR_ROUND,
     K_LHR_FINAL,
+    K_DSP_CLAIM,
+    K_DSP_VECTORS,
     K_COUNT
 };
 
@@ -246,6 +248,14 @@ int fp_lookup_keys(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st,
 size_t fp_lookup_mults_scratch(int k);
 int fp_lookup_mults(fp_ctx* c, const FpKeyCols& K, int k, int64_t L, cudaStream_t st, uint8_t* hm, uint8_t dg_rem[32],
                     uint8_t dg_cl[32]);
+// The rounds of sum_b A(b) B(b) over two device vectors of length 2^n (overwritten) from
+// the given claim: each round's g(0), g(1), g(2) sent under lab_round at proof + *pos, the
+// challenge squeezed under lab_chal; fin = A(rho), B(rho). The matmul sum-check's kernel with
+// one site; scratch from the context's arenas (fp_two_vector_scratch, _host_scratch).
+size_t fp_two_vector_scratch(const fp_ctx* c, int n);
+size_t fp_two_vector_host_scratch();
+int fp_two_vector_sumcheck(fp_ctx* c, fp_tx* tx, uint64_t* A, uint64_t* B, int n, uint64_t claim, const char* lab_round,
+                           const char* lab_chal, uint8_t* proof, size_t* pos, uint64_t fin[2], cudaStream_t st);
 // shapes, rescale exponents and the int32 domain of every site (no pointers looked at)
 int fp_check_shapes(fp_ctx* c, const fp_site* sites, int nsites);
 

@@ -571,6 +571,56 @@ int sumcheck_prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites
     return prove_matmul(c, tx, sites, nsites, nullptr, proof, proof_len, stream);
 }
 
+size_t fp_two_vector_scratch(const fp_ctx* c, int n) {
+    const size_t vec = (size_t)8 << n;
+    return 2 * fp_align_up(vec, 256) + fp_align_up((size_t)8 * 3 * 16 * c->num_sms, 256) + 3 * 256 + 4096;
+}
+
+size_t fp_two_vector_host_scratch() { return 3 * 256 + 8192; }
+
+int fp_two_vector_sumcheck(fp_ctx* c, fp_tx* tx, uint64_t* A, uint64_t* B, int n, uint64_t claim, const char* lab_round,
+                           const char* lab_chal, uint8_t* proof, size_t* pos, uint64_t fin[2], cudaStream_t st) {
+    // the matmul rounds' device source with one site and no batching weight; A and B are the
+    // site's vectors and are overwritten
+    MmDevice d;
+    d.c = c;
+    d.st = st;
+    d.sites = nullptr;
+    d.nsites = 1;
+    d.n = n;
+    d.L = 1ll << n;
+    memset(&d.P, 0, sizeof d.P);
+    d.bufA[0] = A;
+    d.bufB[0] = B;
+    d.bufA[1] = (uint64_t*)fp_alloc(c->dev, (size_t)8 << n);
+    d.bufB[1] = (uint64_t*)fp_alloc(c->dev, (size_t)8 << n);
+    d.part = (uint64_t*)fp_alloc(c->dev, (size_t)8 * 3 * 16 * c->num_sms);
+    d.dfin = (uint64_t*)fp_alloc(c->dev, 16);
+    d.drho = (uint64_t*)fp_alloc(c->dev, 8);
+    d.hrho = (uint64_t*)fp_alloc(c->host, 8);
+    d.hbuf = (uint64_t*)fp_alloc(c->host, 8 * 64);
+    if (!d.bufA[1] || !d.bufB[1] || !d.part || !d.dfin || !d.drho || !d.hrho || !d.hbuf)
+        return fp_fail(c, FP_ERR_OOM, "two-vector sum-check: scratch exhausted");
+    const uint64_t one = 1;
+    int rc;
+    if ((rc = d.rounds(&one))) return rc;
+    static const uint64_t inv2 = gl_inv(2);
+    for (int t = 1; t <= n; t++) {
+        uint64_t g02[2];
+        if ((rc = d.round(t, g02))) return rc;
+        const uint64_t g[3] = {g02[0], gl_sub(claim, g02[0]), g02[1]};
+        put_u64s(proof + *pos, g, 3);
+        fp_tx_absorb_raw(tx, lab_round, proof + *pos, 24);
+        *pos += 24;
+        const uint64_t r = fp_tx_squeeze_one(tx, lab_chal);
+        if ((rc = d.answer(t, r))) return rc;
+        const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2);
+        claim = gl_add(gl_add(gl_mul(g[0], gl_mul(gl_mul(r1, r2), inv2)), gl_sub(0, gl_mul(g[1], gl_mul(r, r2)))),
+                       gl_mul(g[2], gl_mul(gl_mul(r, r1), inv2)));
+    }
+    return d.finals(fin);
+}
+
 int sumcheck_prove_matmul_shard(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, const fp_shard* shard,
                                 uint8_t* proof, size_t* proof_len, void* stream) {
     if (!shard) return fp_fail(c, FP_ERR_ARG, "sumcheck_prove_matmul_shard: null shard");
