@@ -105,39 +105,23 @@ __global__ void __launch_bounds__(1024) hist_kernel(KeySrc K, int k, int64_t L, 
         for (int i = threadIdx.x; i < T; i += blockDim.x) sr[i] = 0;
     __syncthreads();
     uint32_t out_local = 0;
-    const int lane = threadIdx.x & 31;
-    // the quotients cluster in a few bins (q is the rescaled output): lanes holding the same key
-    // add their count with one atomic, from the lowest of them. Every lane of a warp runs the same
-    // iterations (a lane past the keys matches no lane that holds one), so the matches take the
-    // full warp.
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < K.n; base += stride) {
-        const int64_t i = base + lane;
-        const bool in = i < K.n;
-        const int32_t rv = in ? K.r[i] : 0, qv = in ? K.q[i] : 0;
-        const uint64_t tag = (uint64_t)in << 32;
-        const unsigned same_r = __match_any_sync(0xffffffffu, (unsigned long long)(tag | (uint32_t)rv));
-        const unsigned same_q = __match_any_sync(0xffffffffu, (unsigned long long)(tag | (uint32_t)qv));
-        if (!in) continue;
-        const int64_t jr = (int64_t)rv + half;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < K.n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t jr = (int64_t)K.r[i] + half;
         if (jr >= 0 && jr < T) {
-            if (__ffs(same_r) - 1 == lane) {
-                if (rem_in_smem)
-                    atomicAdd(&sr[jr], (uint32_t)__popc(same_r));
-                else
-                    atomicAdd(&m_rem[jr], (uint32_t)__popc(same_r));
-            }
+            if (rem_in_smem)
+                atomicAdd(&sr[jr], 1u);
+            else
+                atomicAdd(&m_rem[jr], 1u);
         } else {
             out_local++;
         }
-        const int64_t q = qv;
-        if (q >= -HIST_WIN && q < HIST_WIN) {
-            if (__ffs(same_q) - 1 == lane) atomicAdd(&sq[q + HIST_WIN], (uint32_t)__popc(same_q));
-        } else if (q >= -32768 && q < 32768) {
-            if (__ffs(same_q) - 1 == lane) atomicAdd(&m_clamp[q + 32768], (uint32_t)__popc(same_q));
-        } else {
+        const int64_t q = K.q[i];
+        if (q >= -HIST_WIN && q < HIST_WIN)
+            atomicAdd(&sq[q + HIST_WIN], 1u);
+        else if (q >= -32768 && q < 32768)
+            atomicAdd(&m_clamp[q + 32768], 1u);
+        else
             out_local++;
-        }
         if ((int32_t)K.y[i] != (q < -128 ? -128 : (q > 127 ? 127 : (int32_t)q))) out_local++;
     }
     if (out_local) atomicAdd(outside, out_local);
