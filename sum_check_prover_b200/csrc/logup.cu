@@ -394,6 +394,9 @@ struct GkrLayer {
     // layer has no p vectors (all ones) and folds its q pairs into a buffer
     ulonglong2* pp[2];
     ulonglong2* qq[2];
+    // leaf layer: the tree's level above the leaves, (dL + dR, dL dR) of every node per table
+    const uint64_t* parP[2];
+    const uint64_t* parQ[2];
     uint64_t* E;       // suffix eq table, kept in place
     KeySrc keys;
     Chal chal;
@@ -452,6 +455,24 @@ __device__ __forceinline__ ulonglong2 fold2(ulonglong2 a, ulonglong2 b, uint64_t
     return make_ulonglong2(gl_fold_fast(a.x, b.x, r), gl_fold_fast(a.y, b.y, r));
 }
 
+// F of a node of the level above the leaves from its stored (P, Q) = (dL + dR, dL dR):
+// sum_tau lambda^(2 tau) (P + lambda Q), weakly reduced
+__device__ __forceinline__ uint64_t parent_F(const GkrLayer& A, int64_t x, uint64_t lam, uint64_t lam2) {
+    const uint64_t f0 = gl_muladd_weak(lam, __ldcg(A.parQ[0] + x), __ldcg(A.parP[0] + x));
+    const uint64_t f1 = gl_muladd_weak(lam, __ldcg(A.parQ[1] + x), __ldcg(A.parP[1] + x));
+    return gl_muladd_weak(lam2, f1, f0);
+}
+
+// The leaf layer's denominators at X = 2 of the pair (b, b + h): the children's keys on the
+// line through b and b + h, 2 k(b + h) - k(b), formed in integers
+__device__ __forceinline__ void leaf_den_at2(const GkrLayer& A, int64_t i0, int64_t i1, uint64_t& d0, uint64_t& d1) {
+    int32_t r0, q0, y0, r1, q1, y1;
+    key_at(A.keys, i0, r0, q0, y0);
+    key_at(A.keys, i1, r1, q1, y1);
+    d0 = gl_sub(A.chal.alpha0, gl_from_i64(2 * (int64_t)r1 - r0));
+    d1 = gl_sub(gl_sub(A.chal.alpha1, gl_mul_small(A.chal.gamma, 2 * y1 - y0)), gl_from_i64(2 * (int64_t)q1 - q0));
+}
+
 // Round t of layer d over the pairs b < h handled by this block.
 // t == 1: the vectors as they are. t >= 2: fold the previous round's vectors
 // (length 4h) by rprev first and store the folded halves in place.
@@ -462,6 +483,19 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* y
                                             bool need1, GlAcc (&acc)[3]) {
     const bool from_keys = LEAF && t <= 2;
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
+        if (LEAF && t == 1) {
+            // X = 0 (and 1) from the stored level above the leaves; X = 2 from four denominators
+            // of integer-extrapolated keys
+            const uint64_t e = eq_chunks_at(EC, eq_tab, b);  // E_1[b] = eq(z_2..z_d, b)
+            if (A.d > 1) A.E[b] = e;
+            acc[0].mac(e, parent_F(A, b, lam, lam2));
+            if (need1) acc[2].mac(e, parent_F(A, b + h, lam, lam2));
+            uint64_t pl[2] = {1, 1}, pr[2] = {1, 1}, ql[2], qr[2];
+            leaf_den_at2(A, 2 * b, 2 * (b + h), ql[0], ql[1]);
+            leaf_den_at2(A, 2 * b + 1, 2 * (b + h) + 1, qr[0], qr[1]);
+            acc[1].mac(e, layer_F<true>(pl, pr, ql, qr, lam, lam2));
+            continue;
+        }
         ulonglong2 c0p[2], c0q[2], c1p[2], c1q[2];
         uint64_t e;
         if (t == 1) {
@@ -727,11 +761,13 @@ __global__ void __launch_bounds__(LU_THREADS) leaf_eval_kernel(KeySrc K, const u
 
 // Algorithmic bytes of round t of a layer with h pairs: the pair vectors
 // (p and q of both tables, 16 B per pair entry; the leaf layer has only q and
-// reads its first two rounds from the keys, 9 B per key), read at 2 (t = 1)
-// or 4 positions and written at 2, plus the suffix eq table.
+// reads its first two rounds from the keys, 9 B per key, and in round 1 the
+// stored level above the leaves, 32 B per node), read at 2 (t = 1) or 4
+// positions and written at 2, plus the suffix eq table.
 double gkr_round_bytes(bool leaf, int t, double h) {
     const double entry = leaf ? 32.0 : 64.0;  // one position of all pair vectors
-    if (t == 1) return (leaf ? 4 * 9.0 : 2 * entry) * h + 8.0 * h;
+    // the leaf layer's round 1 reads the four children's keys and the stored parent of b
+    if (t == 1) return (leaf ? 4 * 9.0 + 32.0 : 2 * entry) * h + 8.0 * h;
     if (leaf && t == 2) return 8 * 9.0 * h + 2 * entry * h + 24.0 * h;
     return 4 * entry * h + 2 * entry * h + 24.0 * h;
 }
@@ -984,6 +1020,8 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
             if (leaf) {
                 A.pp[tau] = nullptr;
                 A.qq[tau] = leafq[tau];
+                A.parP[tau] = lay[d].P[tau];  // the level above the leaves (d = v - 1)
+                A.parQ[tau] = lay[d].Q[tau];
             } else {
                 A.pp[tau] = reinterpret_cast<ulonglong2*>(lay[d + 1].P[tau]);
                 A.qq[tau] = reinterpret_cast<ulonglong2*>(lay[d + 1].Q[tau]);
