@@ -9,6 +9,29 @@
 // a + r (b - a): a pair folded by an extension challenge
 static inline Ext2 e2_fold_host(Ext2 a, Ext2 b, Ext2 r) { return e2_add(a, e2_mul(r, e2_sub(b, a))); }
 
+// 1 / x = (a - b phi) / (a^2 - 7 b^2) (0 for 0)
+static inline Ext2 e2_inv_host(Ext2 x) {
+    const uint64_t ni = gl_inv(gl_sub(gl_mul(x.a, x.a), gl_mul(7, gl_mul(x.b, x.b))));
+    return e2_make(gl_mul(x.a, ni), gl_sub(0, gl_mul(x.b, ni)));
+}
+
+// The round values g(0..3) of a layer round from the device's h(0), h(2) (and h(1), used only
+// when z_t = 0): g(X) = pre eq(z_t, X) h(X), h of degree 2, and g(1) = claim - g(0), so that
+// pre h(1) = g(1) / z_t. With ph = pre h: g(0) = (1 - z_t) ph(0), g(2) = (3 z_t - 1) ph(2),
+// g(3) = (5 z_t - 2) ph(3), ph(3) = ph(0) - 3 ph(1) + 3 ph(2).
+static inline void e2_layer_round_values(const Ext2 h[3], Ext2 pre, Ext2 zt, Ext2 claim, Ext2 g[4]) {
+    const Ext2 one = e2_make(1, 0);
+    const Ext2 ph0 = e2_mul(pre, h[0]), ph2 = e2_mul(pre, h[2]);
+    g[0] = e2_mul(e2_sub(one, zt), ph0);
+    g[1] = e2_sub(claim, g[0]);
+    const bool z0 = zt.a == 0 && zt.b == 0;
+    const Ext2 ph1 = z0 ? e2_mul(pre, h[1]) : e2_mul(g[1], e2_inv_host(zt));
+    if (z0) g[1] = e2_make(0, 0);  // eq(0, 1) = 0
+    g[2] = e2_mul(e2_sub(e2_scal(zt, 3), one), ph2);
+    const Ext2 ph3 = e2_add(e2_sub(ph0, e2_scal(ph1, 3)), e2_scal(ph2, 3));
+    g[3] = e2_mul(e2_sub(e2_scal(zt, 5), e2_make(2, 0)), ph3);
+}
+
 static inline Ext2 e2_squeeze_host(fp_tx* tx, const char* label) {
     const uint64_t a = fp_tx_squeeze_one(tx, label);
     const uint64_t b = fp_tx_squeeze_one(tx, label);

@@ -169,6 +169,8 @@ __global__ void __launch_bounds__(X16_THREADS, 2) x16_layer_kernel(X16Layer A, F
         if (blockIdx.x >= active) return;  // no pairs for this block in this or any later round
         int w[4] = {0, 0, 0, 0};
         if (t == 1) x16_tables(tab, A.z.z, A.d, w);
+        // h(1) only when z_t = 0: otherwise the host takes it from the running claim
+        const bool need1 = A.z.z[t - 1].a == 0 && A.z.z[t - 1].b == 0;
         E2Acc a0, a1, a2;
         for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
             Ext2 p0, p1, r0, r1, q0, q1, s0, s1, e;  // pL, pR, qL, qR at the pair's two points
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(X16_THREADS, 2) x16_layer_kernel(X16Layer A, F
             }
             const uint64_t e7 = gl_mul7(e.b);
             a0.mac(e, e7, x16_f(p0, r0, q0, s0, A.lam));
-            a1.mac(e, e7, x16_f(p1, r1, q1, s1, A.lam));
+            if (need1) a1.mac(e, e7, x16_f(p1, r1, q1, s1, A.lam));
             a2.mac(e, e7, x16_f(e2_at2(p0, p1), e2_at2(r0, r1), e2_at2(q0, q1), e2_at2(s0, s1), A.lam));
         }
         uint64_t acc[6] = {a0.a.value(), a0.b.value(), a1.a.value(), a1.b.value(), a2.a.value(), a2.b.value()};
@@ -310,12 +312,8 @@ int x16_protocol(fp_ctx* c, fp_tx* tx, const X16Labels& lab, int v, Ext2 gamma, 
             Ext2 h[3];
             if ((rc = src.round(d, t, h))) return rc;
             const Ext2 zt = z[t - 1];
-            const Ext2 h3 = e2_add(e2_sub(h[0], e2_scal(h[1], 3)), e2_scal(h[2], 3));
             Ext2 g[4];
-            g[0] = e2_mul(pre, e2_mul(e2_sub(one, zt), h[0]));
-            g[1] = e2_mul(pre, e2_mul(zt, h[1]));
-            g[2] = e2_mul(pre, e2_mul(e2_sub(e2_scal(zt, 3), one), h[2]));
-            g[3] = e2_mul(pre, e2_mul(e2_sub(e2_scal(zt, 5), e2_make(2, 0)), h3));
+            e2_layer_round_values(h, pre, zt, claim, g);  // h(1) only from the device when z_t = 0
             if (!e2_same(e2_add(g[0], g[1]), claim)) {
                 src.abandon();
                 return fp_fail(c, FP_ERR_CUDA, "lookup over the extension: round values inconsistent with the claim");
@@ -436,6 +434,8 @@ __global__ void __launch_bounds__(X16_THREADS, 2) lu2_layer_kernel(Lu2Layer A, F
         if (blockIdx.x >= active) return;  // no pairs for this block in this or any later round
         int w[4] = {0, 0, 0, 0};
         if (t == 1) x16_tables(tab, A.z.z, A.d, w);
+        // h(1) only when z_t = 0: otherwise the host takes it from the running claim
+        const bool need1 = A.z.z[t - 1].a == 0 && A.z.z[t - 1].b == 0;
         E2Acc a0, a1, a2;
         for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
             Ext2 F[3] = {e2_make(0, 0), e2_make(0, 0), e2_make(0, 0)};
@@ -482,11 +482,12 @@ __global__ void __launch_bounds__(X16_THREADS, 2) lu2_layer_kernel(Lu2Layer A, F
                     A.ql[tau][b + h] = q1;
                     A.qr[tau][b + h] = s1;
                 }
-                Ext2 f0 = x16_f(p0, r0, q0, s0, A.lam), f1 = x16_f(p1, r1, q1, s1, A.lam);
+                Ext2 f0 = x16_f(p0, r0, q0, s0, A.lam), f1 = e2_make(0, 0);
+                if (need1) f1 = x16_f(p1, r1, q1, s1, A.lam);
                 Ext2 f2 = x16_f(e2_at2(p0, p1), e2_at2(r0, r1), e2_at2(q0, q1), e2_at2(s0, s1), A.lam);
                 if (tau == 1) {
                     f0 = e2_mul(A.lam2, f0);
-                    f1 = e2_mul(A.lam2, f1);
+                    if (need1) f1 = e2_mul(A.lam2, f1);
                     f2 = e2_mul(A.lam2, f2);
                 }
                 F[0] = e2_add(F[0], f0);
@@ -503,7 +504,7 @@ __global__ void __launch_bounds__(X16_THREADS, 2) lu2_layer_kernel(Lu2Layer A, F
             }
             const uint64_t e7 = gl_mul7(e.b);
             a0.mac(e, e7, F[0]);
-            a1.mac(e, e7, F[1]);
+            if (need1) a1.mac(e, e7, F[1]);
             a2.mac(e, e7, F[2]);
         }
         uint64_t acc[6] = {a0.a.value(), a0.b.value(), a1.a.value(), a1.b.value(), a2.a.value(), a2.b.value()};
@@ -603,12 +604,8 @@ int lu2_protocol(fp_ctx* c, fp_tx* tx, int v, int k, const uint32_t* m_rem, cons
             Ext2 h[3];
             if ((rc = src.round(t, h))) return rc;
             const Ext2 zt = z[t - 1];
-            const Ext2 h3 = e2_add(e2_sub(h[0], e2_scal(h[1], 3)), e2_scal(h[2], 3));
             Ext2 g[4];
-            g[0] = e2_mul(pre, e2_mul(e2_sub(one, zt), h[0]));
-            g[1] = e2_mul(pre, e2_mul(zt, h[1]));
-            g[2] = e2_mul(pre, e2_mul(e2_sub(e2_scal(zt, 3), one), h[2]));
-            g[3] = e2_mul(pre, e2_mul(e2_sub(e2_scal(zt, 5), e2_make(2, 0)), h3));
+            e2_layer_round_values(h, pre, zt, claim, g);  // h(1) only from the device when z_t = 0
             if (!e2_same(e2_add(g[0], g[1]), claim)) {
                 src.abandon();
                 return fp_fail(c, FP_ERR_CUDA, "logup_prove_rescale_ext2: round values inconsistent with the claim");

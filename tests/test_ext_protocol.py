@@ -430,12 +430,17 @@ def test_lookup16x_host_half_matches_oracle(fp, n):
     assert _lk_drive(fp, 4, g, s, 0, vals) == oracle.silu2_prove(4, g, s)
 
 
-def test_lookup16x_exp_table_and_refusal(fp):
+def test_lookup16x_exp_table_and_bad_round_rejected(fp):
     g = np.array([-5, 0, -300, -1800, 7], np.int16)
     s = np.array([oracle.exp_q(int(x)) for x in g], np.int16)
-    assert _lk_drive(fp, 6, g, s, 1, BruteLookup16x(g, s, oracle.exp_q(0))) == oracle.exp2_prove(6, g, s)
-    with pytest.raises(fp.FpError):
-        _lk_drive(fp, 6, g, s, 1, BruteLookup16x(g, s, oracle.exp_q(0), tamper=(2, 2)))
+    honest = _lk_drive(fp, 6, g, s, 1, BruteLookup16x(g, s, oracle.exp_q(0)))
+    assert honest == oracle.exp2_prove(6, g, s)
+    assert oracle.exp2_verify(6, g, s, honest[0])[0] == "accept"
+    # a layer round's h(1) is the running claim minus h(0), so a wrong device value at X = 0
+    # yields a proof (no refusal) that the verifier rejects
+    bad = _lk_drive(fp, 6, g, s, 1, BruteLookup16x(g, s, oracle.exp_q(0), tamper=(2, 2)))
+    assert bad[0] != honest[0]
+    assert oracle.exp2_verify(6, g, s, bad[0])[0] != "accept"
 
 
 # ---- the two-table rescale LogUp over the extension --------------------------------------
@@ -495,7 +500,7 @@ class BruteLu2:
                 acc = bf.x_add(acc, bf.x_mul(bf.x_eq(self.z[t:self.d], bits), F))
             h.append(acc)
         if self.tamper == (self.d, t):
-            h[1] = ((h[1][0] + 1) % P, h[1][1])
+            h[0] = ((h[0][0] + 1) % P, h[0][1])
         return h
 
     def answer(self, t, rho):
@@ -536,8 +541,11 @@ def test_lu2_host_half_matches_oracle(fp, shapes):
     assert _lu2_drive(fp, 3, sites, wits, BruteLu2(wits)) == oracle.lu2_prove(3, sites, wits)
 
 
-def test_lu2_inconsistent_round_is_refused(fp):
+def test_lu2_bad_round_is_rejected(fp):
     sites = [workloads.random_site(31, 2, 16, 4, 8, 6)]
     wits = [oracle.witness(s) for s in sites]
-    with pytest.raises(fp.FpError):
-        _lu2_drive(fp, 3, sites, wits, BruteLu2(wits, tamper=(2, 1)))
+    honest = _lu2_drive(fp, 3, sites, wits, BruteLu2(wits))
+    bad = _lu2_drive(fp, 3, sites, wits, BruteLu2(wits, tamper=(2, 1)))
+    assert bad[0] != honest[0]
+    assert oracle.lu2_verify(3, sites, wits, honest[0])[0] == "accept"
+    assert oracle.lu2_verify(3, sites, wits, bad[0])[0] != "accept"

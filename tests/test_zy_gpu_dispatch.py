@@ -71,15 +71,18 @@ def test_stepped_and_resident(env):
     assert gpu(env, 6, X, e, D, 16) == gpu(env, 6, X, e, D, 16, stepped=True)
 
 
-def test_dishonest_dispatch_is_proven_and_rejected(env):
-    # rows of two experts swapped: the honest prover's proof of the wrong D equals the oracle's,
-    # and the oracle's verifier rejects it
+def test_dishonest_dispatch_is_rejected(env):
+    # rows of two experts swapped. The GPU prover takes each round's g(1) from the running claim,
+    # so for a false statement its rounds stay consistent and the proof fails at its end; the
+    # oracle's prover evaluates g(1) in full and fails at the first round: both are rejected
     X, e, D = statement(10, 200, 96, 6)
     D2 = D.copy()
     D2[[0, -1]] = D2[[-1, 0]]
     pf, st = gpu(env, 7, X, e, D2, 6)
-    assert (pf, st) == oracle.dsp_prove(7, X, e, D2, 6)
-    assert oracle.dsp_verify(7, X, e, D2, 6, pf)[0] == "dsp_round"
+    honest, _ = gpu(env, 7, X, e, D, 6)
+    assert pf != honest
+    assert oracle.dsp_verify(7, X, e, D2, 6, pf)[0] == "dsp_final"
+    assert oracle.dsp_verify(7, X, e, D2, 6, oracle.dsp_prove(7, X, e, D2, 6)[0])[0] == "dsp_round"
 
 
 def test_expert_index_out_of_range(env):
