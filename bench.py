@@ -251,7 +251,9 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
     lu2_round: the rescale LogUp's layer rounds over 2^26 keys with extension challenges,
       both tables in one launch (288 and 576 B per pair).
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
-      epilogue (a Llama-3.1-8B FFN projection), against the tensor peak.
+      epilogue (a Llama-3.1-8B FFN projection), against the tensor peak; and the witness
+      launches of a 16-expert MoE layer (about 64 tokens per expert, the shared expert over
+      1024 tokens), bound by the weight stream, against the copy bandwidth.
     """
     import workloads
     from workloads import device
@@ -326,6 +328,14 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
                                                     "TOPS": tops, "frac": tops / peak, "peak": peak,
                                                     "peak_note": "int8 = measured bf16 x 2 (nominal ratio)"}
         del st, keep
+        # the witness launches of a MoE layer (16 experts of 8192 x 5120 / 5120 x 8192 int4 with
+        # about 64 routed tokens each, and the shared expert over 1024 tokens): bound by the
+        # weight stream, so reported against the copy bandwidth
+        wl = workloads.build(5, 0, E=16, T=1024)
+        st, keep = device.upload(wl, dev)
+        device.weight_digests(ctx, st)
+        measure("witness_gemm_moe_16x3_experts_T1024", "witness_gemm", lambda: fp.prove(ctx, 0, st), big=1 << 20)
+        del st, keep, wl
 
     if "had" in which:
         # the gated product of an FFN's hidden tensor, 2^26 entries per factor

@@ -47,6 +47,9 @@ namespace {
 #ifndef FP_GKR_LEAF_MIN_BLOCKS
 #define FP_GKR_LEAF_MIN_BLOCKS 1
 #endif
+#ifndef FP_TREE_KEYS_MIN_BLOCKS
+#define FP_TREE_KEYS_MIN_BLOCKS 3
+#endif
 constexpr int LU_THREADS = FP_GKR_THREADS;
 constexpr int LU_LEAF_THREADS = FP_GKR_LEAF_THREADS;
 
@@ -238,130 +241,170 @@ __global__ void __launch_bounds__(512) tree_chunk_kernel(KeySrc K, Chal C, TreeL
     }
 }
 
-// The first eleven levels above the leaves (v - 1 .. v - 11) from the keys, for v >= 12. A block
-// takes 2048-leaf chunks in turn: each thread builds the three levels above its 8 consecutive
-// leaves in registers, each warp the next five from its lanes' 32 nodes with shuffles, and warp 0
-// the last three from the block's 8 warp nodes; every level is written as it is formed. One
-// barrier per chunk instead of one per level.
-constexpr int kKeyTreeLevels = 11;
-constexpr int kKeyTreeThreads = 256;  // 8 leaves per thread: 2048 leaves per chunk
+// The first twelve levels above the leaves (v - 1 .. v - 12) from the keys, for v >= 13. A block
+// takes 4096-leaf chunks in turn: each thread builds the four levels above its 16 consecutive
+// leaves in registers, each warp the next five by shuffles (a lane per node and table), and warp
+// 0 the last three from the block's 8 warp nodes; every level is written as it is formed. The
+// kernel is bound by the integer pipes, so the leaves' denominators take a branch-light
+// subtraction and a parent's P one exact two-product sum and a single reduction.
+constexpr int kKeyTreeLevels = 12;
+constexpr int kKeyTreeThreads = 256;  // 16 leaves per thread: 4096 leaves per chunk
 
 struct KeyTreeOut {
     TreeLayer lay[kKeyTreeLevels];  // lay[l]: level v - 1 - l
 };
 
-// (P, Q) of a parent from its children: (pL qR + pR qL, qL qR)
+// alpha - v for a canonical alpha and a signed 32-bit v, canonical
+__device__ __forceinline__ uint64_t sub_i32(uint64_t alpha, int32_t v) {
+    const uint64_t x = alpha - (uint64_t)(int64_t)v;
+    if (v >= 0) return alpha >= (uint64_t)v ? x : x - GL_EPS;  // a borrow is worth + p
+    return x >= GL_P ? x - GL_P : x;                            // alpha + |v| < 2^64
+}
+
+// (P, Q) of a parent from its children: (pL qR + pR qL, qL qR), canonical
 __device__ __forceinline__ void tree_up(uint64_t pl, uint64_t ql, uint64_t pr, uint64_t qr, uint64_t& p, uint64_t& q) {
-    p = gl_add(gl_mul(pl, qr), gl_mul(pr, ql));
+    GlAcc a;
+    a.mac(pl, qr);
+    a.mac(pr, ql);
+    p = a.value();
     q = gl_mul(ql, qr);
 }
 
-__global__ void __launch_bounds__(kKeyTreeThreads) tree_keys_kernel(KeySrc K, Chal C, KeyTreeOut out, int64_t nchunks) {
+// The four levels above a thread's 16 consecutive leaves in one table (v - 1 .. v - 4), each
+// written as it is formed; the level v - 4 node is returned. One table at a time keeps the
+// thread's live values to one table's keys and nodes.
+template <int T>
+__device__ __forceinline__ void key_subtree(const KeySrc& K, const Chal& C, const uint64_t* ytab, const KeyTreeOut& out,
+                                            int64_t ch, int64_t leaf0, uint64_t& p4, uint64_t& q4) {
+    uint64_t P[8], Q[8];
+    if (leaf0 + 16 <= K.n) {
+        int32_t k[16];  // r (table 0) or q (table 1)
+        const int32_t* col = T == 0 ? K.r : K.q;
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const int4 kv = __ldcs(reinterpret_cast<const int4*>(col + leaf0) + u);
+            k[4 * u] = kv.x; k[4 * u + 1] = kv.y; k[4 * u + 2] = kv.z; k[4 * u + 3] = kv.w;
+        }
+        uint32_t yw[4] = {0, 0, 0, 0};
+        if (T == 1) {
+            const uint4 yv = __ldcs(reinterpret_cast<const uint4*>(K.y + leaf0));
+            yw[0] = yv.x; yw[1] = yv.y; yw[2] = yv.z; yw[3] = yv.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            uint64_t a, b;
+            if (T == 0) {
+                a = sub_i32(C.alpha0, k[2 * j]);
+                b = sub_i32(C.alpha0, k[2 * j + 1]);
+            } else {
+                const int ya = (int8_t)((yw[j >> 1] >> (16 * (j & 1))) & 0xFF);
+                const int yb = (int8_t)((yw[j >> 1] >> (16 * (j & 1) + 8)) & 0xFF);
+                a = sub_i32(ytab[ya + 128], k[2 * j]);
+                b = sub_i32(ytab[yb + 128], k[2 * j + 1]);
+            }
+            P[j] = gl_add(a, b);
+            Q[j] = gl_mul(a, b);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            int32_t r0, q0, y0, r1, q1, y1;
+            key_at(K, leaf0 + 2 * j, r0, q0, y0);
+            key_at(K, leaf0 + 2 * j + 1, r1, q1, y1);
+            const uint64_t a = T == 0 ? sub_i32(C.alpha0, r0) : sub_i32(ytab[y0 + 128], q0);
+            const uint64_t b = T == 0 ? sub_i32(C.alpha0, r1) : sub_i32(ytab[y1 + 128], q1);
+            P[j] = gl_add(a, b);
+            Q[j] = gl_mul(a, b);
+        }
+    }
+    // write level l's n (8, 4, 2, 1) consecutive nodes, then form level l + 1
+#pragma unroll
+    for (int l = 0; l < 4; l++) {
+        const int n = 8 >> l;
+        const int64_t g = (ch * 256 + threadIdx.x) * (int64_t)n;  // the thread's first node of level l
+        if (n >= 2) {
+#pragma unroll
+            for (int j = 0; j < n; j += 2) {
+                reinterpret_cast<ulonglong2*>(out.lay[l].P[T] + g)[j / 2] = make_ulonglong2(P[j], P[j + 1]);
+                reinterpret_cast<ulonglong2*>(out.lay[l].Q[T] + g)[j / 2] = make_ulonglong2(Q[j], Q[j + 1]);
+            }
+#pragma unroll
+            for (int j = 0; j < n / 2; j++) tree_up(P[2 * j], Q[2 * j], P[2 * j + 1], Q[2 * j + 1], P[j], Q[j]);
+        } else {
+            out.lay[l].P[T][g] = P[0];
+            out.lay[l].Q[T][g] = Q[0];
+        }
+    }
+    p4 = P[0];
+    q4 = Q[0];
+}
+
+__global__ void __launch_bounds__(kKeyTreeThreads, FP_TREE_KEYS_MIN_BLOCKS) tree_keys_kernel(KeySrc K, Chal C, KeyTreeOut out, int64_t nchunks) {
     __shared__ uint64_t ytab[256];
-    __shared__ uint64_t wnode[8][4];  // each warp's level v - 8 node: P0, Q0, P1, Q1
+    __shared__ uint64_t wnode[2][2][8];  // [table][P, Q][warp]: each warp's level v - 9 node
     leaf_ytab_build(C, ytab);
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int64_t ch = blockIdx.x; ch < nchunks; ch += gridDim.x) {
-        const int64_t leaf0 = ch * 2048 + 8 * (int64_t)threadIdx.x;
-        int32_t r[8], q[8], y[8];
-        if (leaf0 + 8 <= K.n) {
-            const int4 r0 = __ldcs(reinterpret_cast<const int4*>(K.r + leaf0));
-            const int4 r1 = __ldcs(reinterpret_cast<const int4*>(K.r + leaf0 + 4));
-            const int4 q0 = __ldcs(reinterpret_cast<const int4*>(K.q + leaf0));
-            const int4 q1 = __ldcs(reinterpret_cast<const int4*>(K.q + leaf0 + 4));
-            const uint2 yv = __ldcs(reinterpret_cast<const uint2*>(K.y + leaf0));
-            r[0] = r0.x; r[1] = r0.y; r[2] = r0.z; r[3] = r0.w; r[4] = r1.x; r[5] = r1.y; r[6] = r1.z; r[7] = r1.w;
-            q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w; q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
-#pragma unroll
-            for (int j = 0; j < 8; j++) y[j] = (int32_t)(int8_t)(((j < 4 ? yv.x : yv.y) >> (8 * (j & 3))) & 0xFF);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; j++) key_at(K, leaf0 + j, r[j], q[j], y[j]);
+        const int64_t leaf0 = ch * 4096 + 16 * (int64_t)threadIdx.x;
+        uint64_t P[2][1], Q[2][1];  // the thread's level v - 4 node per table
+        key_subtree<0>(K, C, ytab, out, ch, leaf0, P[0][0], Q[0][0]);
+        key_subtree<1>(K, C, ytab, out, ch, leaf0, P[1][0], Q[1][0]);
+        // each lane now holds its level v - 4 node of both tables in P[t][0], Q[t][0]. Levels v - 5 ..
+        // v - 9 in the warp: at level v - 5 lane L forms node x = L & 15 of table L >> 4 from lanes
+        // 2x, 2x + 1; below, a level's items sit on lanes 0 .. 2 nl - 1, table-major
+        uint64_t mp, mq;  // this lane's item of the current level
+        {
+            const int t = lane >> 4, x = lane & 15, src = 2 * x;
+            const uint64_t pl0 = shfl_u64(P[0][0], src), ql0 = shfl_u64(Q[0][0], src);
+            const uint64_t pr0 = shfl_u64(P[0][0], src + 1), qr0 = shfl_u64(Q[0][0], src + 1);
+            const uint64_t pl1 = shfl_u64(P[1][0], src), ql1 = shfl_u64(Q[1][0], src);
+            const uint64_t pr1 = shfl_u64(P[1][0], src + 1), qr1 = shfl_u64(Q[1][0], src + 1);
+            tree_up(t ? pl1 : pl0, t ? ql1 : ql0, t ? pr1 : pr0, t ? qr1 : qr0, mp, mq);
+            const int64_t g = (ch * 8 + warp) * 16 + x;
+            out.lay[4].P[t][g] = mp;
+            out.lay[4].Q[t][g] = mq;
         }
-        // level v - 1 (4 nodes per thread), then v - 2 (2) and v - 3 (1), per table
-        uint64_t P[2][4], Q[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const uint64_t a0 = gl_sub(C.alpha0, gl_from_i64(r[2 * j])), b0 = gl_sub(C.alpha0, gl_from_i64(r[2 * j + 1]));
-            const uint64_t a1 = gl_sub(ytab[y[2 * j] + 128], gl_from_i64(q[2 * j]));
-            const uint64_t b1 = gl_sub(ytab[y[2 * j + 1] + 128], gl_from_i64(q[2 * j + 1]));
-            P[0][j] = gl_add(a0, b0);
-            Q[0][j] = gl_mul(a0, b0);
-            P[1][j] = gl_add(a1, b1);
-            Q[1][j] = gl_mul(a1, b1);
-        }
-        const int64_t n1 = ch * 1024 + 4 * (int64_t)threadIdx.x;
-#pragma unroll
-        for (int t = 0; t < 2; t++) {
-            reinterpret_cast<ulonglong2*>(out.lay[0].P[t] + n1)[0] = make_ulonglong2(P[t][0], P[t][1]);
-            reinterpret_cast<ulonglong2*>(out.lay[0].P[t] + n1)[1] = make_ulonglong2(P[t][2], P[t][3]);
-            reinterpret_cast<ulonglong2*>(out.lay[0].Q[t] + n1)[0] = make_ulonglong2(Q[t][0], Q[t][1]);
-            reinterpret_cast<ulonglong2*>(out.lay[0].Q[t] + n1)[1] = make_ulonglong2(Q[t][2], Q[t][3]);
-            tree_up(P[t][0], Q[t][0], P[t][1], Q[t][1], P[t][0], Q[t][0]);
-            tree_up(P[t][2], Q[t][2], P[t][3], Q[t][3], P[t][1], Q[t][1]);
-        }
-        const int64_t n2 = ch * 512 + 2 * (int64_t)threadIdx.x;
-#pragma unroll
-        for (int t = 0; t < 2; t++) {
-            *reinterpret_cast<ulonglong2*>(out.lay[1].P[t] + n2) = make_ulonglong2(P[t][0], P[t][1]);
-            *reinterpret_cast<ulonglong2*>(out.lay[1].Q[t] + n2) = make_ulonglong2(Q[t][0], Q[t][1]);
-            tree_up(P[t][0], Q[t][0], P[t][1], Q[t][1], P[t][0], Q[t][0]);
-            out.lay[2].P[t][ch * 256 + threadIdx.x] = P[t][0];
-            out.lay[2].Q[t][ch * 256 + threadIdx.x] = Q[t][0];
-        }
-        // levels v - 4 .. v - 8 within the warp: lane x of a level takes the nodes of lanes 2x, 2x + 1
-        uint64_t p[2] = {P[0][0], P[1][0]}, qq[2] = {Q[0][0], Q[1][0]};
-#pragma unroll
-        for (int l = 3; l < 8; l++) {
-            const int nl = 32 >> (l - 2);  // nodes of this level in the warp
-            const int src = (2 * lane) & 31;
-#pragma unroll
-            for (int t = 0; t < 2; t++) {
-                const uint64_t pl = shfl_u64(p[t], src), ql = shfl_u64(qq[t], src);
-                const uint64_t pr = shfl_u64(p[t], src + 1), qr = shfl_u64(qq[t], src + 1);
-                uint64_t np, nq;
-                tree_up(pl, ql, pr, qr, np, nq);
-                p[t] = np;
-                qq[t] = nq;
-                if (lane < nl) {
-                    const int64_t g = (ch * 8 + warp) * (int64_t)nl + lane;
-                    out.lay[l].P[t][g] = np;
-                    out.lay[l].Q[t][g] = nq;
-                }
+        for (int l = 5; l < 9; l++) {
+            const int nl = 16 >> (l - 4);  // nodes per table of level v - 1 - l in the warp
+            const int t = lane / nl, x = lane % nl;
+            const int src = (t * 2 * nl + 2 * x) & 31;  // children: items 2x, 2x + 1 of table t one level down
+            const uint64_t pl = shfl_u64(mp, src), ql = shfl_u64(mq, src);
+            const uint64_t pr = shfl_u64(mp, src + 1), qr = shfl_u64(mq, src + 1);
+            uint64_t np, nq;
+            tree_up(pl, ql, pr, qr, np, nq);
+            mp = np;
+            mq = nq;
+            if (lane < 2 * nl) {
+                const int64_t g = (ch * 8 + warp) * (int64_t)nl + x;
+                out.lay[l].P[t][g] = np;
+                out.lay[l].Q[t][g] = nq;
             }
         }
-        if (lane == 0) {
-            wnode[warp][0] = p[0];
-            wnode[warp][1] = qq[0];
-            wnode[warp][2] = p[1];
-            wnode[warp][3] = qq[1];
+        if (lane < 2) {  // lane t holds the warp's level v - 9 node of table t
+            wnode[lane][0][warp] = mp;
+            wnode[lane][1][warp] = mq;
         }
         __syncthreads();
-        // levels v - 9 .. v - 11 from the 8 warp nodes, in warp 0
+        // levels v - 10 .. v - 12 from the 8 warp nodes per table, in warp 0 (item i = table i >> 3)
         if (warp == 0) {
-            uint64_t bp[2], bq[2];
+            uint64_t bp = lane < 16 ? wnode[lane >> 3][0][lane & 7] : 0ull;
+            uint64_t bq = lane < 16 ? wnode[lane >> 3][1][lane & 7] : 0ull;
 #pragma unroll
-            for (int t = 0; t < 2; t++) {
-                bp[t] = lane < 8 ? wnode[lane][2 * t] : 0ull;
-                bq[t] = lane < 8 ? wnode[lane][2 * t + 1] : 0ull;
-            }
-#pragma unroll
-            for (int l = 8; l < kKeyTreeLevels; l++) {
-                const int nl = 8 >> (l - 7);
-                const int src = (2 * lane) & 31;
-#pragma unroll
-                for (int t = 0; t < 2; t++) {
-                    const uint64_t pl = shfl_u64(bp[t], src), ql = shfl_u64(bq[t], src);
-                    const uint64_t pr = shfl_u64(bp[t], src + 1), qr = shfl_u64(bq[t], src + 1);
-                    uint64_t np, nq;
-                    tree_up(pl, ql, pr, qr, np, nq);
-                    bp[t] = np;
-                    bq[t] = nq;
-                    if (lane < nl) {
-                        out.lay[l].P[t][ch * nl + lane] = np;
-                        out.lay[l].Q[t][ch * nl + lane] = nq;
-                    }
+            for (int l = 9; l < kKeyTreeLevels; l++) {
+                const int nl = 8 >> (l - 8);
+                const int t = lane / nl, x = lane % nl;
+                const int src = (t * 2 * nl + 2 * x) & 31;
+                const uint64_t pl = shfl_u64(bp, src), ql = shfl_u64(bq, src);
+                const uint64_t pr = shfl_u64(bp, src + 1), qr = shfl_u64(bq, src + 1);
+                uint64_t np, nq;
+                tree_up(pl, ql, pr, qr, np, nq);
+                bp = np;
+                bq = nq;
+                if (lane < 2 * nl) {
+                    out.lay[l].P[t][ch * nl + x] = np;
+                    out.lay[l].Q[t][ch * nl + x] = nq;
                 }
             }
         }
@@ -390,8 +433,14 @@ __global__ void l1_from_layer_kernel(TreeLayer one, uint64_t* out) {
 // ---- layer sum-check: one persistent kernel per layer ---------------------------------
 
 struct GkrLayer {
-    // pair vectors (x: left child, y: right child), folded in place; the leaf
-    // layer has no p vectors (all ones) and folds its q pairs into a buffer
+    // pair vectors (x: left child, y: right child): rounds 1 and 2 read the children's level
+    // (sp, sq), round 2 writes the folded halves to pp, qq, later rounds fold pp, qq in place.
+    // pp == sp everywhere except in the layer above the leaf layer, which must leave its
+    // children's level intact (the leaf layer's first round reads it) and folds into the leaf
+    // layer's buffer instead. The leaf layer has no p vectors (all ones), reads its keys in
+    // rounds 1 and 2 and folds its q pairs into a buffer.
+    const ulonglong2* sp[2];
+    const ulonglong2* sq[2];
     ulonglong2* pp[2];
     ulonglong2* qq[2];
     // leaf layer: the tree's level above the leaves, (dL + dR, dL dR) of every node per table
@@ -431,11 +480,12 @@ __device__ __forceinline__ uint64_t layer_F(const uint64_t (&pl)[2], const uint6
     return gl_muladd_weak(lam2, f[1], f[0]);
 }
 
-// pair x of the layer's current vectors: from the key columns, or from pp/qq
+// pair x of the layer's vectors: before any fold (from_src) from the key columns or the
+// children's level, afterwards from the fold buffers pp/qq
 template <bool LEAF>
-__device__ __forceinline__ void layer_pair(const GkrLayer& A, const uint64_t* ytab, bool from_keys, int64_t x,
+__device__ __forceinline__ void layer_pair(const GkrLayer& A, const uint64_t* ytab, bool from_src, int64_t x,
                                            ulonglong2 (&pp)[2], ulonglong2 (&qq)[2]) {
-    if (LEAF && from_keys) {
+    if (LEAF && from_src) {
         uint64_t l0, l1, r0, r1;
         leaf_den_tab(A.keys, A.chal, ytab, 2 * x, l0, l1);
         leaf_den_tab(A.keys, A.chal, ytab, 2 * x + 1, r0, r1);
@@ -445,8 +495,8 @@ __device__ __forceinline__ void layer_pair(const GkrLayer& A, const uint64_t* yt
     } else {
 #pragma unroll
         for (int tau = 0; tau < 2; tau++) {
-            pp[tau] = LEAF ? make_ulonglong2(1, 1) : __ldcg(A.pp[tau] + x);
-            qq[tau] = __ldcg(A.qq[tau] + x);
+            pp[tau] = LEAF ? make_ulonglong2(1, 1) : __ldcg((from_src ? A.sp[tau] : A.pp[tau]) + x);
+            qq[tau] = __ldcg((!LEAF && from_src ? A.sq[tau] : A.qq[tau]) + x);
         }
     }
 }
@@ -481,7 +531,7 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* y
                                             const uint64_t* eq_tab, int t,
                                             int64_t h, unsigned active, uint64_t rprev, uint64_t lam, uint64_t lam2,
                                             bool need1, GlAcc (&acc)[3]) {
-    const bool from_keys = LEAF && t <= 2;
+    const bool from_keys = t <= 2;  // the unfolded vectors (keys or the children's level)
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
         if (LEAF && t == 1) {
             // X = 0 (and 1) from the stored level above the leaves; X = 2 from four denominators
@@ -569,7 +619,7 @@ __device__ __forceinline__ void layer_tail(const GkrLayer& A, const uint64_t* yt
     __shared__ uint64_t Et[kTailPairs];
     const int d = A.d;
     int h = 1 << (d - t0);
-    const bool from_keys = LEAF && t0 <= 2;
+    const bool from_keys = t0 <= 2;  // the unfolded vectors (keys or the children's level)
     for (int x = threadIdx.x; x < 2 * h; x += blockDim.x) {
         ulonglong2 pp[2], qq[2];
         layer_pair<LEAF>(A, ytab, from_keys, x, pp, qq);
@@ -707,8 +757,8 @@ __global__ void __launch_bounds__(LEAF ? LU_LEAF_THREADS : LU_THREADS, LEAF ? FP
     if (threadIdx.x == 0) {
         A.zout[d - 1] = rprev;
         ulonglong2 p0[2], q0[2], p1[2], q1[2];
-        layer_pair<LEAF>(A, ytab, LEAF && d == 1, 0, p0, q0);
-        layer_pair<LEAF>(A, ytab, LEAF && d == 1, 1, p1, q1);
+        layer_pair<LEAF>(A, ytab, d == 1, 0, p0, q0);  // a one-round layer never folded
+        layer_pair<LEAF>(A, ytab, d == 1, 1, p1, q1);
         uint64_t out[8];
 #pragma unroll
         for (int tau = 0; tau < 2; tau++) {
@@ -945,15 +995,15 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
     if (!part || !small || !hsmall || !E || !zb[2]) return fp_fail(c, FP_ERR_OOM, "logup: scratch exhausted");
 
     if (v >= 2) {
-        // layers v-1 .. 1: the first eleven from the keys in one persistent launch (v >= 12), the
+        // layers v-1 .. 1: the first twelve from the keys in one persistent launch (v >= 13), the
         // rest kTreeLevels per launch
         int L0 = v;
-        // the vector loads of 8 keys need 16-byte aligned key columns (8-byte for y)
-        const bool keys_aligned = (uintptr_t)K.r % 16 == 0 && (uintptr_t)K.q % 16 == 0 && (uintptr_t)K.y % 8 == 0;
-        if (v >= 12 && keys_aligned) {
+        // the vector loads of 16 keys need 16-byte aligned key columns
+        const bool keys_aligned = (uintptr_t)K.r % 16 == 0 && (uintptr_t)K.q % 16 == 0 && (uintptr_t)K.y % 16 == 0;
+        if (v >= kKeyTreeLevels + 1 && keys_aligned) {
             KeyTreeOut ko;
             for (int l = 0; l < kKeyTreeLevels; l++) ko.lay[l] = lay[v - 1 - l];
-            const int64_t nchunks = (1ll << v) / 2048;
+            const int64_t nchunks = (1ll << v) / 4096;
             int occ_t = 0;
             FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_t, tree_keys_kernel, kKeyTreeThreads, 0));
             const unsigned blocks = (unsigned)std::min<int64_t>(nchunks, (int64_t)std::max(1, occ_t) * c->num_sms);
@@ -1023,8 +1073,17 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
                 A.parP[tau] = lay[d].P[tau];  // the level above the leaves (d = v - 1)
                 A.parQ[tau] = lay[d].Q[tau];
             } else {
-                A.pp[tau] = reinterpret_cast<ulonglong2*>(lay[d + 1].P[tau]);
-                A.qq[tau] = reinterpret_cast<ulonglong2*>(lay[d + 1].Q[tau]);
+                A.sp[tau] = reinterpret_cast<const ulonglong2*>(lay[d + 1].P[tau]);
+                A.sq[tau] = reinterpret_cast<const ulonglong2*>(lay[d + 1].Q[tau]);
+                if (d == v - 2) {
+                    // keep level v - 1 for the leaf layer: fold into its (not yet used) q buffer,
+                    // 2^(v-3) positions of p and q pairs per table = 16 << (v - 2) bytes
+                    A.pp[tau] = leafq[tau];
+                    A.qq[tau] = leafq[tau] + ((size_t)1 << (v - 3));
+                } else {
+                    A.pp[tau] = reinterpret_cast<ulonglong2*>(lay[d + 1].P[tau]);
+                    A.qq[tau] = reinterpret_cast<ulonglong2*>(lay[d + 1].Q[tau]);
+                }
             }
         }
         A.E = E;
