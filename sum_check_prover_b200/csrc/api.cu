@@ -81,8 +81,11 @@ fp_ctx* fp_ctx_create(int device) {
     const char* st = getenv("FP_STEPPED");
     c->stepped_env = profiler_injected() || (st && st[0] == '1');
     c->stepped = c->stepped_env;
-    const char* tg = getenv("FP_TCGEN05");  // "0": the mma.sync witness kernel for every site
-    c->tc_gemm = !(tg && tg[0] == '0');
+    // witness GEMM kernels: "0" the mma.sync kernel for every site, "1" the single-role tcgen05
+    // kernel for unscaled sites; otherwise the warp-specialised tcgen05 kernel for every site whose
+    // operands TMA can read
+    const char* tg = getenv("FP_TCGEN05");
+    c->tc_gemm = (tg && tg[0] == '0') ? 0 : (tg && tg[0] == '1') ? 1 : 2;
     return c;
 }
 

@@ -116,8 +116,9 @@ struct fp_ctx {
     // sum-check (under a kernel-replaying profiler, and while profiling)
     int stepped = 0;
     int stepped_env = 0;
-    // witness GEMM on the tcgen05 tensor-core path (FP_TCGEN05=0 selects the mma.sync kernel)
-    int tc_gemm = 1;
+    // witness GEMM kernels: 2 warp-specialised tcgen05 (default), 1 single-role tcgen05 for
+    // unscaled sites, 0 mma.sync (FP_TCGEN05 selects 0 or 1)
+    int tc_gemm = 2;
     // timing
     int profiling = 0;
     int64_t launches = 0;  // every kernel launch of the library on this context
@@ -234,6 +235,12 @@ int fp_shard_gather(const FpShardView& sh, const uint64_t* mine, int per, uint64
 int fp_shard_sum(const FpShardView& sh, uint64_t* v, int n);
 // The lookup keys: every site's outputs in storage order, concatenated; indices
 // in [n, 2^v) are the neutral key (r, q, y) = 0.
+// A 2-D byte tensor (rows of `inner` bytes, `pitch` bytes apart) as a TMA tensor map (128 bytes at
+// `tmap`, 64-byte aligned): boxes of box_inner x box_rows, zero fill outside, optional 128-byte
+// swizzle. False if the driver's encoder is unavailable or rejects the shape.
+bool fp_tmap_u8_2d(void* tmap, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch, uint32_t box_inner,
+                   uint32_t box_rows, bool swizzle128);
+
 struct FpKeyCols {
     const int32_t* r;
     const int32_t* q;

@@ -636,6 +636,19 @@ std::vector<PePlan> pe_plan_all(int num_sms, const FpPeJob* jobs, int njobs) {
 
 }  // namespace
 
+bool fp_tmap_u8_2d(void* tmap, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch, uint32_t box_inner,
+                   uint32_t box_rows, bool swizzle128) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tmap_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)pitch};
+    const cuuint32_t box[2] = {box_inner, box_rows}, estr[2] = {1, 1};
+    return enc(reinterpret_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t fp_partial_scratch(const fp_ctx* c, const FpPeJob* jobs, int njobs) {
     size_t need = 4 * fp_align_up(sizeof(PeJob) * (size_t)njobs, 256) + 4096;
     const std::vector<PePlan> P = pe_plan_all(c->num_sms, jobs, njobs);

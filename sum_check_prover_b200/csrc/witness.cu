@@ -16,6 +16,10 @@
 // 64 k, 8 warps (2 x 4), warp tile 64 x 32, m16n8k32 s8.s8.s32, 3-stage
 // cp.async pipeline. All sites of a call share one launch per operand variant
 // (grouped GEMM over a tile list).
+#include <cuda.h>  // CUtensorMap
+#include <string.h>
+
+#include <algorithm>
 #include <vector>
 
 #include "fp_internal.h"
@@ -660,19 +664,495 @@ int launch_variant(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st)
     return FP_OK;
 }
 
+
+// ---- warp-specialised tcgen05 kernel (every site with TMA-readable operands) ---------------
+//
+// D = Xt . W_eff^T on the 5th-generation tensor cores, for unscaled and scaled sites alike. A
+// persistent kernel: one CTA per SM takes tiles of 128 tokens x WS BN weight rows in turn, and
+// its warps split the work, handing stages over on mbarriers:
+//   warp 0 (one lane)  TMA producer: per k-tile (128 bytes of K) the Xt box (128 tokens x 128
+//                      bytes, 128-byte swizzle: the MMA's K-major layout) and the weight box (the
+//                      packed int4 rows, the int8 rows, or for unscaled int8 directly in the MMA
+//                      layout) into ring stage s, once the MMAs that read its last tile are done.
+//   expansion warps    int4 -> int8, or W_eff = s * w split into a high s8 and a low u8 byte limb
+//                      (256 hi + lo), from the loaded box into one of two buffers in the MMA layout.
+//   warp 1 (one lane)  MMA issue: four K = 32 MMAs per k-tile (and four more on the low limb) into
+//                      the tile's tensor-memory accumulator slot; each k-tile commits to the stage
+//                      and buffer it read, a tile's last k-tile to the slot's "full" barrier.
+//   epilogue warps     tcgen05.ld of a slot (two slots: the next tile's MMAs run meanwhile),
+//                      Y = hi 256 + lo for two limbs, the rescale / remainder / clamp, stores.
+// Every wait is bounded; a wait that runs out sets the error word and an abort flag that ends the
+// other roles' waits, and the kernel drains its copies and MMAs before it frees tensor memory.
+constexpr int WS_BM = 128;                  // tokens per tile: MMA M, tensor-memory lanes
+constexpr int WS_BK = 128;                  // bytes of K per k-tile
+constexpr int WS_A_BYTES = WS_BM * WS_BK;   // 16 KB
+constexpr uint32_t WS_WAIT_LIMIT = 1u << 24;
+
+template <bool W4, bool SCALED>
+struct WsCfg {
+    static constexpr bool EXPAND = W4 || SCALED;  // the MMA reads an expanded copy of the weight box
+    static constexpr int BN = SCALED ? 128 : 256;  // weight rows per tile: MMA N
+    static constexpr int LIMBS = SCALED ? 2 : 1;   // accumulators per tile
+    static constexpr int ACC_COLS = LIMBS * BN;    // tensor-memory columns per accumulator slot
+    static constexpr int BP_BYTES = BN * (W4 ? WS_BK / 2 : WS_BK);        // the weight box as loaded
+    static constexpr int X_BYTES = EXPAND ? LIMBS * BN * WS_BK : 0;       // one expanded buffer
+    static constexpr int RING = WS_A_BYTES + BP_BYTES;                    // one ring stage
+    static constexpr int STAGES_FIT = (216 * 1024 - 2 * X_BYTES) / RING;
+    static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+    static constexpr int EXP_WARPS = EXPAND ? 8 : 0;  // two per SM sub-partition: the expansion is latency-bound
+    static constexpr int EPI0 = 2 + EXP_WARPS;     // first epilogue warp (four: lane quarters 2, 3, 0, 1)
+    static constexpr int THREADS = 32 * (EPI0 + 4);
+    static constexpr int SMEM = STAGES * RING + 2 * X_BYTES + 1024;
+    // s32 accumulator, A s8, B s8 (or u8 for the low limb), both K-major, N = BN, M = 128
+    static constexpr uint32_t IDESC_S8 =
+        (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(WS_BM >> 4) << 24);
+    static constexpr uint32_t IDESC_U8 =
+        (2u << 4) | (1u << 7) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(WS_BM >> 4) << 24);
+};
+
+struct alignas(64) SiteWs {
+    CUtensorMap tmA;   // Xt: N rows of K bytes, 128 x 128 boxes, 128-byte swizzle
+    CUtensorMap tmB;   // W: M rows (packed int4 or int8), boxes of one k-tile x BN rows
+    const int8_t* scales;
+    int32_t* q;
+    int32_t* r;
+    int8_t* y;
+    int32_t M, K, N, k_shift;
+    int32_t G;         // scale groups per row, ceil(K / 64)
+    int32_t tiles_i;   // weight-row tiles
+    int32_t nk;        // k-tiles
+    int32_t pad;
+    int64_t tile_base;  // first tile of this site
+};
+
+__device__ __forceinline__ int ws_find_site(const SiteWs* sites, int nsites, int64_t t) {
+    int lo = 0, hi = nsites - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sites[mid].tile_base <= t)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+// one bounded wait on an mbarrier phase; false if it ran out (the kernel is then aborting) or
+// another role has aborted
+__device__ __forceinline__ bool ws_wait(uint32_t mbar, uint32_t parity, volatile int* abort, volatile uint64_t* err) {
+    for (uint32_t it = 0; it < WS_WAIT_LIMIT; it++) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (*abort) return false;
+    }
+    *abort = 1;
+    *err = 3;  // a tensor-core pipeline wait ran out
+    __threadfence_system();
+    return false;
+}
+
+// ws_wait by every lane of a warp, with one answer for the warp (a warp-collective tcgen05.ld and
+// the warp's arrivals stay uniform)
+__device__ __forceinline__ bool ws_wait_warp(uint32_t mbar, uint32_t parity, volatile int* abort, volatile uint64_t* err) {
+    const bool ok = ws_wait(mbar, parity, abort, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// the same without the abort check: draining the copies and MMAs still in flight
+__device__ __forceinline__ void ws_drain(uint32_t mbar, uint32_t parity) {
+    for (uint32_t it = 0; it < WS_WAIT_LIMIT; it++) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (ok) return;
+    }
+}
+
+__device__ __forceinline__ void ws_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(mbar) : "memory");
+}
+
+__device__ __forceinline__ void ws_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(mbar) : "memory");
+}
+
+__device__ __forceinline__ void ws_mma(uint32_t tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t en) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(en));
+}
+
+__device__ __forceinline__ void ws_tma2d(uint32_t dst, const CUtensorMap* tm, int x, int y, uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];\n" ::"r"(dst),
+        "l"(tm), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
+
+// eight packed nibbles (k0..k7, low nibble first) -> eight sign-extended int8 in two words
+__device__ __forceinline__ void nib8_to_s8x8(uint32_t v, uint32_t& o0, uint32_t& o1) {
+    uint32_t lo = v & 0x0F0F0F0Fu, hi = (v >> 4) & 0x0F0F0F0Fu;  // k0 k2 k4 k6 / k1 k3 k5 k7
+    lo |= (lo & 0x08080808u) * 0x1Eu;                            // sign-extend bit 3 of every byte
+    hi |= (hi & 0x08080808u) * 0x1Eu;
+    o0 = __byte_perm(lo, hi, 0x5140);
+    o1 = __byte_perm(lo, hi, 0x7362);
+}
+
+// W_eff = s * w for four signed bytes w (one word): the high s8 limb (W_eff >> 8) and the low u8
+// limb (W_eff & 255), so W_eff = 256 hi + lo exactly (|s w| <= 2^14)
+__device__ __forceinline__ void ws_limbs4(uint32_t w4, int s, uint32_t& hi, uint32_t& lo) {
+    hi = lo = 0;
+#pragma unroll
+    for (int b = 0; b < 4; b++) {
+        const int v = (int)(int8_t)(w4 >> (8 * b)) * s;
+        lo |= ((uint32_t)v & 0xFFu) << (8 * b);
+        hi |= ((uint32_t)(v >> 8) & 0xFFu) << (8 * b);
+    }
+}
+
+// The loaded weight box of k-tile kt -> the expanded buffer(s) in the MMA layout (tc_off). et:
+// this thread's index among the expansion threads.
+template <bool W4, bool SCALED>
+__device__ __forceinline__ void ws_expand(const SiteWs& S, const uint8_t* pk, uint8_t* xb, int i0, int kt, int et) {
+    using C = WsCfg<W4, SCALED>;
+    constexpr int ET = C::EXP_WARPS > 0 ? 32 * C::EXP_WARPS : 32;  // (no expansion warps: never called)
+    if (W4) {
+        // 16-byte packed chunk c: row c >> 2, k values 32 (c & 3) .. + 31 -> two 16-byte chunks
+#pragma unroll
+        for (int u = 0; u < C::BN * 4 / ET; u++) {
+            const int c = et + ET * u, row = c >> 2, kq = c & 3;
+            const uint4 v = *reinterpret_cast<const uint4*>(pk + row * 64 + kq * 16);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[8];
+#pragma unroll
+            for (int q = 0; q < 4; q++) nib8_to_s8x8(w[q], o[2 * q], o[2 * q + 1]);
+            if (SCALED) {
+                const int i = i0 + row, g = (kt * WS_BK + kq * 32) >> 6;
+                const int s = (i < S.M && g < S.G) ? (int)S.scales[(int64_t)i * S.G + g] : 0;
+                uint32_t hi[8], lo[8];
+#pragma unroll
+                for (int q = 0; q < 8; q++) ws_limbs4(o[q], s, hi[q], lo[q]);
+                uint8_t* xl = xb + C::BN * WS_BK;
+                *reinterpret_cast<uint4*>(xb + tc_off(row, 2 * kq)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(xb + tc_off(row, 2 * kq + 1)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+                *reinterpret_cast<uint4*>(xl + tc_off(row, 2 * kq)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                *reinterpret_cast<uint4*>(xl + tc_off(row, 2 * kq + 1)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            } else {
+                *reinterpret_cast<uint4*>(xb + tc_off(row, 2 * kq)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4*>(xb + tc_off(row, 2 * kq + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+        }
+    } else {
+        // scaled int8: 16-byte chunk c: row c >> 3, k values 16 (c & 7) .. + 15
+#pragma unroll
+        for (int u = 0; u < C::BN * 8 / ET; u++) {
+            const int c = et + ET * u, row = c >> 3, kc = c & 7;
+            const uint4 v = *reinterpret_cast<const uint4*>(pk + row * 128 + kc * 16);
+            const int i = i0 + row, g = (kt * WS_BK + kc * 16) >> 6;
+            const int s = (i < S.M && g < S.G) ? (int)S.scales[(int64_t)i * S.G + g] : 0;
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int q = 0; q < 4; q++) ws_limbs4(w[q], s, hi[q], lo[q]);
+            *reinterpret_cast<uint4*>(xb + tc_off(row, kc)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(xb + C::BN * WS_BK + tc_off(row, kc)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    }
+}
+
+// q, r, y of 16 consecutive weight rows i..i+15 of token j from their accumulator values
+__device__ __forceinline__ void ws_store16(const SiteWs& S, int j, int i, const uint32_t (&v)[16]) {
+    const int k = S.k_shift;
+    const int64_t half = (int64_t)1 << (k - 1);
+    int32_t q[16], r[16];
+    uint32_t y[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int e = 0; e < 16; e++) {
+        const int64_t Y = (int32_t)v[e];
+        const int64_t qq = (Y + half) >> k;
+        q[e] = (int32_t)qq;
+        r[e] = (int32_t)(Y - (qq << k));
+        const int32_t yc = qq < -128 ? -128 : (qq > 127 ? 127 : (int32_t)qq);
+        y[e >> 2] |= ((uint32_t)yc & 0xFFu) << (8 * (e & 3));
+    }
+    const int64_t o = (int64_t)j * S.M + i;
+    const bool vec = i + 16 <= S.M && ((reinterpret_cast<uintptr_t>(S.q + o) | reinterpret_cast<uintptr_t>(S.r + o) |
+                                        reinterpret_cast<uintptr_t>(S.y + o)) & 15) == 0;
+    if (vec) {
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+            *reinterpret_cast<int4*>(S.q + o + e) = make_int4(q[e], q[e + 1], q[e + 2], q[e + 3]);
+            *reinterpret_cast<int4*>(S.r + o + e) = make_int4(r[e], r[e + 1], r[e + 2], r[e + 3]);
+        }
+        *reinterpret_cast<uint4*>(S.y + o) = make_uint4(y[0], y[1], y[2], y[3]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; e++) {
+            if (i + e >= S.M) break;
+            S.q[o + e] = q[e];
+            S.r[o + e] = r[e];
+            S.y[o + e] = (int8_t)(y[e >> 2] >> (8 * (e & 3)));
+        }
+    }
+}
+
+__device__ __forceinline__ void ws_ld16(uint32_t a, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(a));
+}
+
+template <bool W4, bool SCALED>
+__global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
+    witness_ws_kernel(const SiteWs* __restrict__ sites, int nsites, int64_t ntiles, volatile uint64_t* err) {
+    using C = WsCfg<W4, SCALED>;
+    constexpr int ST = C::STAGES;
+    extern __shared__ uint8_t ws_smem_raw[];
+    uint8_t* smem = ws_smem_raw + ((1024 - (smem_addr(ws_smem_raw) & 1023)) & 1023);
+    uint8_t* ring = smem;                 // stage s: the Xt box at s RING, the weight box after it
+    uint8_t* xbuf = smem + ST * C::RING;  // two expanded buffers (high limb first)
+    __shared__ __align__(8) uint64_t full[ST], empty[ST], xfull[2], xempty[2], accfull[2], accempty[2], fin;
+    __shared__ uint32_t tmem_base;
+    __shared__ volatile int s_abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < ST; s++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&empty[s])));
+        }
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(&xfull[e])), "r"(32 * C::EXP_WARPS));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&xempty[e])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&accfull[e])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 128;\n" ::"r"(smem_addr(&accempty[e])));
+        }
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&fin)));
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;\n" ::"r"(smem_addr(&tmem_base)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- producer ----
+            uint32_t it = 0;
+            const SiteWs* cur = nullptr;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const SiteWs* S = &sites[ws_find_site(sites, nsites, t)];
+                if (S != cur) {
+                    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(&S->tmA) : "memory");
+                    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(&S->tmB) : "memory");
+                    cur = S;
+                }
+                const int64_t lt = t - S->tile_base;
+                const int j0 = (int)(lt / S->tiles_i) * WS_BM, i0 = (int)(lt % S->tiles_i) * C::BN;
+                for (int kt = 0; kt < S->nk; kt++, it++) {
+                    const int s = (int)(it % ST);
+                    const uint32_t n = it / ST;
+                    if (n > 0 && !ws_wait(smem_addr(&empty[s]), (n - 1) & 1u, &s_abort, err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_addr(&full[s]);
+                    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(fb), "r"(C::RING) : "memory");
+                    ws_tma2d(smem_addr(ring + s * C::RING), &S->tmA, kt * WS_BK, j0, fb);
+                    ws_tma2d(smem_addr(ring + s * C::RING + WS_A_BYTES), &S->tmB, kt * (W4 ? WS_BK / 2 : WS_BK), i0, fb);
+                }
+            }
+            if (!ok) {
+                // let every copy that was issued land before the block ends
+                for (int s = 0; s < ST; s++) {
+                    if (it <= (uint32_t)s) continue;
+                    const uint32_t last = (uint32_t)s + ((it - 1 - (uint32_t)s) / ST) * ST;
+                    ws_drain(smem_addr(&full[s]), (last / ST) & 1u);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---- MMA issue ----
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, tc++) {
+                const SiteWs* S = &sites[ws_find_site(sites, nsites, t)];
+                const uint32_t a = tc & 1u;
+                if (tc >= 2 && !ws_wait(smem_addr(&accempty[a]), ((tc >> 1) - 1) & 1u, &s_abort, err)) break;
+                asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
+                const uint32_t dst = tmem + a * C::ACC_COLS;
+                for (int kt = 0; kt < S->nk; kt++, it++) {
+                    const int s = (int)(it % ST), e = (int)(it & 1u);
+                    if (!ws_wait(smem_addr(&full[s]), (it / ST) & 1u, &s_abort, err) ||
+                        (C::EXPAND && !ws_wait(smem_addr(&xfull[e]), (it >> 1) & 1u, &s_abort, err))) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
+                    const uint32_t a0 = smem_addr(ring + s * C::RING);
+                    const uint32_t b0 = C::EXPAND ? smem_addr(xbuf + e * C::X_BYTES) : smem_addr(ring + s * C::RING + WS_A_BYTES);
+#pragma unroll
+                    for (int kc = 0; kc < WS_BK / 32; kc++) {
+                        const uint32_t en = (kt > 0 || kc > 0) ? 1u : 0u;
+                        ws_mma(dst, tc_desc(a0 + kc * 32), tc_desc(b0 + kc * 32), C::IDESC_S8, en);
+                        if (SCALED)
+                            ws_mma(dst + C::BN, tc_desc(a0 + kc * 32), tc_desc(b0 + C::BN * WS_BK + kc * 32), C::IDESC_U8, en);
+                    }
+                    ws_commit(smem_addr(&empty[s]));
+                    if (C::EXPAND) ws_commit(smem_addr(&xempty[e]));
+                }
+                if (ok) ws_commit(smem_addr(&accfull[a]));
+            }
+            // every MMA issued is complete before the tensor memory is freed
+            ws_commit(smem_addr(&fin));
+            ws_drain(smem_addr(&fin), 0);
+        }
+        __syncwarp();
+    } else if (warp < C::EPI0) {
+        // ---- expansion ----
+        const int et = tid - 64;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const SiteWs* S = &sites[ws_find_site(sites, nsites, t)];
+            const int64_t lt = t - S->tile_base;
+            const int i0 = (int)(lt % S->tiles_i) * C::BN;
+            for (int kt = 0; kt < S->nk; kt++, it++) {
+                const int s = (int)(it % ST), e = (int)(it & 1u);
+                if (!ws_wait_warp(smem_addr(&full[s]), (it / ST) & 1u, &s_abort, err) ||
+                    (it >= 2 && !ws_wait_warp(smem_addr(&xempty[e]), ((it >> 1) - 1) & 1u, &s_abort, err))) {
+                    ok = false;
+                    break;
+                }
+                ws_expand<W4, SCALED>(*S, ring + s * C::RING + WS_A_BYTES, xbuf + e * C::X_BYTES, i0, kt, et);
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic writes -> MMA reads
+                ws_arrive(smem_addr(&xfull[e]));
+            }
+        }
+    } else {
+        // ---- epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (tokens) ----
+        const int qd = warp & 3;
+        uint32_t tc = 0;
+        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, tc++) {
+            const SiteWs* S = &sites[ws_find_site(sites, nsites, t)];
+            const int64_t lt = t - S->tile_base;
+            const int j0 = (int)(lt / S->tiles_i) * WS_BM, i0 = (int)(lt % S->tiles_i) * C::BN;
+            const uint32_t a = tc & 1u;
+            if (!ws_wait_warp(smem_addr(&accfull[a]), (tc >> 1) & 1u, &s_abort, err)) break;
+            asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
+            const int j = j0 + 32 * qd + lane;
+            const uint32_t base = tmem + ((uint32_t)(32 * qd) << 16) + a * C::ACC_COLS;
+#pragma unroll 1
+            for (int c0 = 0; c0 < C::BN; c0 += 16) {
+                uint32_t v[16];
+                ws_ld16(base + (uint32_t)c0, v);
+                if (SCALED) {
+                    uint32_t lo[16];
+                    ws_ld16(base + (uint32_t)(C::BN + c0), lo);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+                    for (int e = 0; e < 16; e++) v[e] = (uint32_t)(int32_t)(256ll * (int32_t)v[e] + (int32_t)lo[e]);
+                } else {
+                    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+                }
+                const int i = i0 + c0;
+                if (j < S->N && i < S->M) ws_store16(*S, j, i, v);
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
+            ws_arrive(smem_addr(&accempty[a]));
+        }
+    }
+    __syncwarp();
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
+    if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;\n" ::"r"(tmem));
+}
+
+template <bool W4, bool SCALED>
+int launch_ws(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
+    if (list.empty()) return FP_OK;
+    using C = WsCfg<W4, SCALED>;
+    std::vector<SiteWs> h(list.size());
+    int64_t tiles = 0;
+    double bytes = 0;
+    for (size_t s = 0; s < list.size(); s++) {
+        const fp_site& t = list[s];
+        SiteWs& d = h[s];
+        memset(&d, 0, sizeof d);
+        const uint64_t pitch = W4 ? (uint64_t)t.K / 2 : (uint64_t)t.K;
+        if (!fp_tmap_u8_2d(&d.tmA, t.xt, (uint64_t)t.K, (uint64_t)t.N, (uint64_t)t.K, WS_BK, WS_BM, true) ||
+            !fp_tmap_u8_2d(&d.tmB, t.w, pitch, (uint64_t)t.M, pitch, W4 ? WS_BK / 2 : WS_BK, C::BN, !C::EXPAND))
+            return fp_fail(c, FP_ERR_CUDA, "witness: tensor map encoding failed");
+        d.scales = t.scales;
+        d.q = t.q;
+        d.r = t.r;
+        d.y = t.y;
+        d.M = t.M;
+        d.K = t.K;
+        d.N = t.N;
+        d.k_shift = t.k_shift;
+        d.G = (t.K + 63) / 64;
+        d.tiles_i = (t.M + C::BN - 1) / C::BN;
+        d.nk = (t.K + WS_BK - 1) / WS_BK;
+        d.tile_base = tiles;
+        tiles += (int64_t)d.tiles_i * ((t.N + WS_BM - 1) / WS_BM);
+        bytes += (double)t.M * pitch + (double)t.N * t.K + 9.0 * t.M * t.N + (t.scales ? (double)t.M * d.G : 0.0);
+    }
+    const size_t sz = sizeof(SiteWs) * h.size();
+    SiteWs* dsites = (SiteWs*)fp_alloc(c->dev, sz);
+    char* hst = (char*)fp_alloc(c->host, sz);
+    if (!dsites || !hst) return fp_fail(c, FP_ERR_OOM, "witness: scratch exhausted");
+    memcpy(hst, h.data(), sz);
+    FP_CUDA(c, cudaMemcpyAsync(dsites, hst, sz, cudaMemcpyHostToDevice, st));
+    auto kern = witness_ws_kernel<W4, SCALED>;
+    FP_CUDA(c, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, (int64_t)c->num_sms);
+    int slot;
+    fp_tic(c, st, K_GEMM, bytes, &slot);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(dsites, (int)h.size(), tiles, &c->mb_dev->err);
+    fp_toc(c, st, slot);
+    FP_CUDA(c, cudaGetLastError());
+    return FP_OK;
+}
+
 }  // namespace
 
 int fp_launch_witness(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st) {
     // group sites by kernel variant: unscaled sites with 16-byte rows go to the tensor-core
     // (tcgen05) kernel, the rest to the mma.sync kernel
-    std::vector<fp_site> v[8], tcv[2];
+    std::vector<fp_site> v[8], tcv[2], wsv[4];
     for (int s = 0; s < nsites; s++) {
         const fp_site& t = sites[s];
         bool w4 = t.w_bits == 4, sc = t.scales != nullptr;
         size_t pitch = w4 ? (size_t)(t.K + 1) / 2 : (size_t)t.K;
         bool al = ((uintptr_t)t.w % 16 == 0) && ((uintptr_t)t.xt % 16 == 0) && (pitch % 16 == 0) &&
                   (t.K % 16 == 0) && (!w4 || t.K % 32 == 0);
-        if (al && !sc && c->tc_gemm)
+        if (al && c->tc_gemm == 2)
+            wsv[(w4 ? 2 : 0) + (sc ? 1 : 0)].push_back(t);
+        else if (al && !sc && c->tc_gemm == 1)
             tcv[w4 ? 1 : 0].push_back(t);
         else
             v[(w4 ? 4 : 0) + (sc ? 2 : 0) + (al ? 1 : 0)].push_back(t);
@@ -680,12 +1160,17 @@ int fp_launch_witness(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t 
     size_t need = 0;
     for (int i = 0; i < 8; i++) need += fp_align_up(sizeof(SiteDev) * v[i].size(), 256) + 256;
     for (int i = 0; i < 2; i++) need += fp_align_up(sizeof(SiteDev) * tcv[i].size(), 256) + 256;
+    for (int i = 0; i < 4; i++) need += fp_align_up(sizeof(SiteWs) * wsv[i].size(), 256) + 256;
     int rc = fp_reserve(c, c->dev, need + (1 << 20));
     if (rc) return rc;
     rc = fp_reserve(c, c->host, need + (1 << 20));
     if (rc) return rc;
     fp_reset(c->dev);
     fp_reset(c->host);
+    if ((rc = launch_ws<false, false>(c, wsv[0], st))) return rc;
+    if ((rc = launch_ws<false, true>(c, wsv[1], st))) return rc;
+    if ((rc = launch_ws<true, false>(c, wsv[2], st))) return rc;
+    if ((rc = launch_ws<true, true>(c, wsv[3], st))) return rc;
     if ((rc = launch_tc<false>(c, tcv[0], st))) return rc;
     if ((rc = launch_tc<true>(c, tcv[1], st))) return rc;
     if ((rc = launch_variant<false, false, false>(c, v[0], st))) return rc;

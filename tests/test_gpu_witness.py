@@ -2,11 +2,12 @@
 against a plain numpy definition: int64 matrix product, floor division with
 round-half-up, remainder, clamp ("How fast can FlashProve go", 3.1).
 
-The tcgen05 kernel takes unscaled sites whose rows are whole 16-byte chunks
-(128-token x 128- or 256-row tiles, 128-byte k-tiles); the mma.sync kernel takes the
-rest, or every site when the context is created with FP_TCGEN05=0. Shapes
-cover partial tiles in every dimension, K below and across k-tiles, and one
-or many tiles per site.
+Three kernels: the warp-specialised tcgen05 kernel (the default) takes every site whose
+operands TMA can read (16-byte rows), scaled ones through two byte limbs of s * w; the
+single-role tcgen05 kernel (FP_TCGEN05=1) takes such sites without scales; the mma.sync
+kernel takes the rest, or every site with FP_TCGEN05=0. Shapes cover partial tiles in
+every dimension, K below and across k-tiles and scale groups, and one or many tiles per
+site.
 """
 
 import numpy as np
@@ -22,6 +23,8 @@ SHAPES = [
     (300, 128, 200, 8, False), (256, 256, 128, 4, False), (513, 96, 130, 4, False), (64, 16, 1, 8, False),
     (1000, 4096, 77, 4, False), (40, 32, 300, 4, False), (257, 160, 129, 8, False), (256, 1024, 512, 4, False),
     (129, 64, 64, 4, True), (77, 48, 33, 8, False), (33, 40, 17, 8, False),
+    # scaled sites across k-tiles and scale groups, int4 and int8 (K < 1024 keeps int8 x scales exact)
+    (300, 1024, 200, 4, True), (257, 768, 129, 8, True), (64, 96, 5, 8, True), (2048, 512, 1280, 4, True),
     # enough 256-row tiles to fill the GPU: the tcgen05 kernel's N = 256 variant
     (4096, 256, 1280, 4, False), (2048, 128, 2560, 8, False),
 ]
@@ -53,7 +56,7 @@ def lib():
     return torch, fp
 
 
-@pytest.mark.parametrize("tcgen05", ["1", "0"])
+@pytest.mark.parametrize("tcgen05", ["2", "1", "0"])
 @pytest.mark.parametrize("shape", SHAPES)
 def test_witness_matches_definition(lib, shape, tcgen05, monkeypatch):
     torch, fp = lib
