@@ -69,26 +69,62 @@ __device__ __forceinline__ void key_at(const KeySrc& K, int64_t i, int32_t& r, i
     }
 }
 
+// alpha - v for a canonical alpha and a signed 32-bit v, canonical
+__device__ __forceinline__ uint64_t sub_i32(uint64_t alpha, int32_t v) {
+    const uint64_t x = alpha - (uint64_t)(int64_t)v;
+    if (v >= 0) return alpha >= (uint64_t)v ? x : x - GL_EPS;  // a borrow is worth + p
+    return x >= GL_P ? x - GL_P : x;                            // alpha + |v| < 2^64
+}
+
+// alpha - v for a canonical alpha and a signed v with |v| < 2^62, canonical
+__device__ __forceinline__ uint64_t sub_i64(uint64_t alpha, int64_t v) {
+    if (v >= 0) {
+        const uint64_t u = (uint64_t)v, x = alpha - u;
+        return alpha >= u ? x : x - GL_EPS;
+    }
+    const uint64_t u = (uint64_t)(-v);
+    uint64_t x = alpha + u;
+    if (x < u) x += GL_EPS;  // the lost 2^64 is worth EPS; the sum is then alpha + u - p < u
+    return x >= GL_P ? x - GL_P : x;
+}
+
 // leaf denominators alpha - f of key i for both tables
 __device__ __forceinline__ void leaf_den(const KeySrc& K, const Chal& C, int64_t i, uint64_t& d0, uint64_t& d1) {
     int32_t r, q, y;
     key_at(K, i, r, q, y);
-    d0 = gl_sub(C.alpha0, gl_from_i64(r));
-    d1 = gl_sub(C.alpha1, gl_add(gl_from_i64(q), gl_mul_small(C.gamma, y)));
-}
-
-// The same with alpha1 - gamma y taken from a 256-entry table (index y + 128)
-__device__ __forceinline__ void leaf_den_tab(const KeySrc& K, const Chal& C, const uint64_t* ytab, int64_t i,
-                                             uint64_t& d0, uint64_t& d1) {
-    int32_t r, q, y;
-    key_at(K, i, r, q, y);
-    d0 = gl_sub(C.alpha0, gl_from_i64(r));
-    d1 = gl_sub(ytab[y + 128], gl_from_i64(q));
+    d0 = sub_i32(C.alpha0, r);
+    d1 = sub_i32(gl_sub(C.alpha1, gl_mul_small(C.gamma, y)), q);
 }
 
 // ytab[y + 128] = alpha1 - gamma y for every int8 y (one block fills it)
 __device__ __forceinline__ void leaf_ytab_build(const Chal& C, uint64_t* ytab) {
     for (int j = threadIdx.x; j < 256; j += blockDim.x) ytab[j] = gl_sub(C.alpha1, gl_mul_small(C.gamma, j - 128));
+}
+
+// The layer sum-check's table: alpha1 - gamma y for y in [-384, 384) at index y + 384, which
+// covers the int8 outputs and their extrapolations 2 y1 - y0 to the point X = 2
+constexpr int kYWide = 768;
+__device__ __forceinline__ void leaf_ytabw_build(const Chal& C, uint64_t* ytab) {
+    for (int j = threadIdx.x; j < kYWide; j += blockDim.x) ytab[j] = gl_sub(C.alpha1, gl_mul_small(C.gamma, j - 384));
+}
+
+// keys 2x and 2x + 1 (one pair position of the leaf layer), with 8-byte loads of r and q and a
+// 2-byte load of y when the columns allow it
+__device__ __forceinline__ void key_pair(const KeySrc& K, bool vec, int64_t x, int32_t (&r)[2], int32_t (&q)[2],
+                                         int32_t (&y)[2]) {
+    const int64_t i = 2 * x;
+    if (vec && i + 1 < K.n) {
+        const int2 rv = __ldcg(reinterpret_cast<const int2*>(K.r + i));
+        const int2 qv = __ldcg(reinterpret_cast<const int2*>(K.q + i));
+        const unsigned short yv = __ldcg(reinterpret_cast<const unsigned short*>(K.y + i));
+        r[0] = rv.x; r[1] = rv.y;
+        q[0] = qv.x; q[1] = qv.y;
+        y[0] = (int8_t)(yv & 0xFF);
+        y[1] = (int8_t)(yv >> 8);
+    } else {
+        key_at(K, i, r[0], q[0], y[0]);
+        key_at(K, i + 1, r[1], q[1], y[1]);
+    }
 }
 
 // ---- histograms --------------------------------------------------------------
@@ -253,13 +289,6 @@ constexpr int kKeyTreeThreads = 256;  // 16 leaves per thread: 4096 leaves per c
 struct KeyTreeOut {
     TreeLayer lay[kKeyTreeLevels];  // lay[l]: level v - 1 - l
 };
-
-// alpha - v for a canonical alpha and a signed 32-bit v, canonical
-__device__ __forceinline__ uint64_t sub_i32(uint64_t alpha, int32_t v) {
-    const uint64_t x = alpha - (uint64_t)(int64_t)v;
-    if (v >= 0) return alpha >= (uint64_t)v ? x : x - GL_EPS;  // a borrow is worth + p
-    return x >= GL_P ? x - GL_P : x;                            // alpha + |v| < 2^64
-}
 
 // (P, Q) of a parent from its children: (pL qR + pR qL, qL qR), canonical
 __device__ __forceinline__ void tree_up(uint64_t pl, uint64_t ql, uint64_t pr, uint64_t qr, uint64_t& p, uint64_t& q) {
@@ -448,6 +477,9 @@ struct GkrLayer {
     const uint64_t* parQ[2];
     uint64_t* E;       // suffix eq table, kept in place
     KeySrc keys;
+    int keys_vec;      // r, q 8-byte and y 2-byte aligned: key pairs by vector loads
+    int piped;         // the leaf layer's rounds 1 and 2 stream their operands through the
+                       // per-warp cp.async stages (16-byte aligned key columns)
     Chal chal;
     // Challenge points by layer parity: layer d reads its point from zin
     // (z_1..z_(d-1) = the previous layer's round challenges, z_d = mu written
@@ -486,11 +518,10 @@ template <bool LEAF>
 __device__ __forceinline__ void layer_pair(const GkrLayer& A, const uint64_t* ytab, bool from_src, int64_t x,
                                            ulonglong2 (&pp)[2], ulonglong2 (&qq)[2]) {
     if (LEAF && from_src) {
-        uint64_t l0, l1, r0, r1;
-        leaf_den_tab(A.keys, A.chal, ytab, 2 * x, l0, l1);
-        leaf_den_tab(A.keys, A.chal, ytab, 2 * x + 1, r0, r1);
-        qq[0] = make_ulonglong2(l0, r0);
-        qq[1] = make_ulonglong2(l1, r1);
+        int32_t r[2], q[2], y[2];
+        key_pair(A.keys, A.keys_vec != 0, x, r, q, y);
+        qq[0] = make_ulonglong2(sub_i32(A.chal.alpha0, r[0]), sub_i32(A.chal.alpha0, r[1]));
+        qq[1] = make_ulonglong2(sub_i32(ytab[y[0] + 384], q[0]), sub_i32(ytab[y[1] + 384], q[1]));
         pp[0] = pp[1] = make_ulonglong2(1, 1);
     } else {
 #pragma unroll
@@ -513,25 +544,219 @@ __device__ __forceinline__ uint64_t parent_F(const GkrLayer& A, int64_t x, uint6
     return gl_muladd_weak(lam2, f1, f0);
 }
 
-// The leaf layer's denominators at X = 2 of the pair (b, b + h): the children's keys on the
-// line through b and b + h, 2 k(b + h) - k(b), formed in integers
-__device__ __forceinline__ void leaf_den_at2(const GkrLayer& A, int64_t i0, int64_t i1, uint64_t& d0, uint64_t& d1) {
-    int32_t r0, q0, y0, r1, q1, y1;
-    key_at(A.keys, i0, r0, q0, y0);
-    key_at(A.keys, i1, r1, q1, y1);
-    d0 = gl_sub(A.chal.alpha0, gl_from_i64(2 * (int64_t)r1 - r0));
-    d1 = gl_sub(gl_sub(A.chal.alpha1, gl_mul_small(A.chal.gamma, 2 * y1 - y0)), gl_from_i64(2 * (int64_t)q1 - q0));
+// The leaf layer's denominators at X = 2 of the pair positions (b, b + h): the children's keys
+// on the line through b and b + h, 2 k(b + h) - k(b), formed in integers (alpha1 - gamma y for
+// the extrapolated y from the wide table). ql, qr: left and right leaf, per table.
+__device__ __forceinline__ void leaf_pair_at2(const GkrLayer& A, const uint64_t* ytab, int64_t b, int64_t h,
+                                              uint64_t (&ql)[2], uint64_t (&qr)[2]) {
+    int32_t r0[2], q0[2], y0[2], r1[2], q1[2], y1[2];
+    key_pair(A.keys, A.keys_vec != 0, b, r0, q0, y0);
+    key_pair(A.keys, A.keys_vec != 0, b + h, r1, q1, y1);
+    uint64_t d[2][2];  // [leaf][table]
+#pragma unroll
+    for (int j = 0; j < 2; j++) {
+        d[j][0] = sub_i64(A.chal.alpha0, 2 * (int64_t)r1[j] - r0[j]);
+        d[j][1] = sub_i64(ytab[2 * y1[j] - y0[j] + 384], 2 * (int64_t)q1[j] - q0[j]);
+    }
+    ql[0] = d[0][0];
+    ql[1] = d[0][1];
+    qr[0] = d[1][0];
+    qr[1] = d[1][1];
+}
+
+// ---- the leaf layer's rounds 1 and 2 through per-warp cp.async stages ------------------------
+//
+// Both rounds read their operands once, from places h pairs apart (the keys of pair positions b,
+// b + h (and b + 2h, b + 3h), the level above the leaves or the eq table at b), with a few field
+// products per pair: the warps are too few (one 512-thread block of 126 registers per SM) to hide
+// the loads' latency by themselves. So each warp streams its 32-pair chunks through three
+// shared-memory stages by cp.async, two chunks ahead of the one it computes on.
+constexpr int kPipeStages = 3;
+constexpr int kPipeStage = 1024 + 4 * 576;  // parents or eq (4 x 256 B), then 4 positions x (r, q, y of 64 keys)
+constexpr int kPipeWarps = LU_LEAF_THREADS / 32;
+constexpr size_t kPipeBytes = (size_t)kPipeWarps * kPipeStages * kPipeStage;
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, int bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+}
+
+// the keys of pair positions x0 .. x0 + 31 (64 keys from 2 x0) into a stage: r and q by 16 lanes
+// each, y by 4 lanes; keys past the column's end read as zero
+__device__ __forceinline__ void pipe_keys(const KeySrc& K, int64_t x0, uint32_t dst, int lane) {
+    const int64_t i0 = 2 * x0;
+    if (lane < 16) {
+        const int64_t i = i0 + 4 * lane;
+        const int64_t left = K.n - i;
+        const int nb = left >= 4 ? 16 : (left > 0 ? (int)left * 4 : 0);
+        cp_async16_zfill(dst + 16 * lane, nb ? (const void*)(K.r + i) : (const void*)K.r, nb);
+    } else {
+        const int64_t i = i0 + 4 * (lane - 16);
+        const int64_t left = K.n - i;
+        const int nb = left >= 4 ? 16 : (left > 0 ? (int)left * 4 : 0);
+        cp_async16_zfill(dst + 256 + 16 * (lane - 16), nb ? (const void*)(K.q + i) : (const void*)K.q, nb);
+    }
+    if (lane < 4) {
+        const int64_t i = i0 + 16 * lane;
+        const int64_t left = K.n - i;
+        const int nb = left >= 16 ? 16 : (left > 0 ? (int)left : 0);
+        cp_async16_zfill(dst + 512 + 16 * lane, nb ? (const void*)(K.y + i) : (const void*)K.y, nb);
+    }
+}
+
+// 32 consecutive 8-byte values from v + x0 into a stage slot (16 lanes, one 16-byte copy each)
+__device__ __forceinline__ void pipe_u64x32(const uint64_t* v, int64_t x0, uint32_t dst, int l16) {
+    cp_async16_zfill(dst + 16 * l16, v + x0 + 2 * l16, 16);
+}
+
+// issue chunk x0's copies for round t into stage address st
+template <int T>
+__device__ __forceinline__ void pipe_issue(const GkrLayer& A, int64_t x0, int64_t h, uint32_t st, int lane) {
+    if (T == 1) {
+        // the level above the leaves at x0: P of table 0 at 0, of table 1 at 256, Q at 512 and 768
+        const int arr = lane >> 4, l16 = lane & 15;
+        pipe_u64x32(arr == 0 ? A.parP[0] : A.parQ[0], x0, st + 512 * arr, l16);
+        pipe_u64x32(arr == 0 ? A.parP[1] : A.parQ[1], x0, st + 256 + 512 * arr, l16);
+        pipe_keys(A.keys, x0, st + 1024, lane);
+        pipe_keys(A.keys, x0 + h, st + 1024 + 576, lane);
+    } else {
+        // the eq table at x0 and x0 + h, then the keys of four positions
+        pipe_u64x32(A.E, x0 + (lane >> 4) * h, st + 256 * (lane >> 4), lane & 15);
+#pragma unroll
+        for (int p = 0; p < 4; p++) pipe_keys(A.keys, x0 + p * h, st + 1024 + 576 * p, lane);
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+// keys 2 lane, 2 lane + 1 of position slot p of a stage
+__device__ __forceinline__ void pipe_key_pair(const uint8_t* st, int p, int lane, int32_t (&r)[2], int32_t (&q)[2],
+                                              int32_t (&y)[2]) {
+    const uint8_t* kb = st + 1024 + 576 * p;
+    const int2 rv = *reinterpret_cast<const int2*>(kb + 8 * lane);
+    const int2 qv = *reinterpret_cast<const int2*>(kb + 256 + 8 * lane);
+    const unsigned short yv = *reinterpret_cast<const unsigned short*>(kb + 512 + 2 * lane);
+    r[0] = rv.x; r[1] = rv.y;
+    q[0] = qv.x; q[1] = qv.y;
+    y[0] = (int8_t)(yv & 0xFF);
+    y[1] = (int8_t)(yv >> 8);
+}
+
+// Rounds 1 and 2 of the leaf layer by the stages (h >= 32: every chunk is 32 whole pairs).
+template <int T>
+__device__ __forceinline__ void leaf_round_piped(const GkrLayer& A, const uint64_t* ytab, uint8_t* pipe,
+                                                 const EqChunks& EC, const uint64_t* eq_tab, int64_t h,
+                                                 unsigned active, uint64_t rprev, uint64_t lam, uint64_t lam2,
+                                                 bool need1, GlAcc (&acc)[3]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t* wbuf = pipe + (size_t)warp * kPipeStages * kPipeStage;
+    const uint32_t wsa = (uint32_t)__cvta_generic_to_shared(wbuf);
+    const int64_t first = (int64_t)blockIdx.x * blockDim.x + 32 * warp, stride = (int64_t)active * blockDim.x;
+    // prologue: chunks 0 .. kPipeStages - 2 in flight (an empty group keeps the count uniform)
+#pragma unroll
+    for (int i = 0; i < kPipeStages - 1; i++) {
+        const int64_t x0 = first + i * stride;
+        if (x0 < h)
+            pipe_issue<T>(A, x0, h, wsa + i * kPipeStage, lane);
+        else
+            asm volatile("cp.async.commit_group;\n" ::: "memory");
+    }
+    int64_t x0 = first;
+    for (int i = 0; x0 < h; i++, x0 += stride) {
+        {
+            const int64_t xn = x0 + (kPipeStages - 1) * stride;
+            const int sn = (i + kPipeStages - 1) % kPipeStages;
+            if (xn < h)
+                pipe_issue<T>(A, xn, h, wsa + sn * kPipeStage, lane);
+            else
+                asm volatile("cp.async.commit_group;\n" ::: "memory");
+        }
+        asm volatile("cp.async.wait_group %0;\n" ::"n"(kPipeStages - 1) : "memory");
+        __syncwarp();  // every lane's copies of chunk i have landed
+        const uint8_t* st = wbuf + (i % kPipeStages) * kPipeStage;
+        const int64_t b = x0 + lane;
+        if (T == 1) {
+            // X = 0 (and 1) from the level above the leaves; X = 2 from the keys extrapolated
+            const uint64_t e = eq_chunks_at(EC, eq_tab, b);  // E_1[b] = eq(z_2..z_d, b)
+            if (A.d > 1) A.E[b] = e;
+            const uint64_t* pv = reinterpret_cast<const uint64_t*>(st);  // P0, P1, Q0, Q1: 32 each
+            const uint64_t f0 = gl_muladd_weak(lam, pv[64 + lane], pv[lane]);
+            const uint64_t f1 = gl_muladd_weak(lam, pv[96 + lane], pv[32 + lane]);
+            acc[0].mac(e, gl_muladd_weak(lam2, f1, f0));
+            if (need1) acc[2].mac(e, parent_F(A, b + h, lam, lam2));
+            int32_t r0[2], q0[2], y0[2], r1[2], q1[2], y1[2];
+            pipe_key_pair(st, 0, lane, r0, q0, y0);
+            pipe_key_pair(st, 1, lane, r1, q1, y1);
+            uint64_t pl[2] = {1, 1}, pr[2] = {1, 1}, ql[2], qr[2];
+            ql[0] = sub_i64(A.chal.alpha0, 2 * (int64_t)r1[0] - r0[0]);
+            ql[1] = sub_i64(ytab[2 * y1[0] - y0[0] + 384], 2 * (int64_t)q1[0] - q0[0]);
+            qr[0] = sub_i64(A.chal.alpha0, 2 * (int64_t)r1[1] - r0[1]);
+            qr[1] = sub_i64(ytab[2 * y1[1] - y0[1] + 384], 2 * (int64_t)q1[1] - q0[1]);
+            acc[1].mac(e, layer_F<true>(pl, pr, ql, qr, lam, lam2));
+        } else {
+            // fold positions (b, b + 2h) and (b + h, b + 3h) by the round-1 challenge
+            uint64_t c0[2][2], c1[2][2];  // [table][leaf] at X = 0 (position b) and X = 1 (b + h)
+#pragma unroll
+            for (int half = 0; half < 2; half++) {
+                int32_t ra[2], qa[2], ya[2], rb[2], qb[2], yb[2];
+                pipe_key_pair(st, half, lane, ra, qa, ya);
+                pipe_key_pair(st, half + 2, lane, rb, qb, yb);
+                uint64_t (&c)[2][2] = half ? c1 : c0;
+#pragma unroll
+                for (int j = 0; j < 2; j++) {
+                    c[0][j] = gl_fold_fast(sub_i32(A.chal.alpha0, ra[j]), sub_i32(A.chal.alpha0, rb[j]), rprev);
+                    c[1][j] = gl_fold_fast(sub_i32(ytab[ya[j] + 384], qa[j]), sub_i32(ytab[yb[j] + 384], qb[j]), rprev);
+                }
+            }
+#pragma unroll
+            for (int tau = 0; tau < 2; tau++) {
+                A.qq[tau][b] = make_ulonglong2(c0[tau][0], c0[tau][1]);
+                A.qq[tau][b + h] = make_ulonglong2(c1[tau][0], c1[tau][1]);
+            }
+            const uint64_t* ev = reinterpret_cast<const uint64_t*>(st);
+            const uint64_t e = gl_add(ev[lane], ev[32 + lane]);
+            A.E[b] = e;
+            uint64_t pl[2] = {1, 1}, pr[2] = {1, 1}, ql[2], qr[2];
+#pragma unroll
+            for (int tau = 0; tau < 2; tau++) {
+                ql[tau] = c0[tau][0];
+                qr[tau] = c0[tau][1];
+            }
+            acc[0].mac(e, layer_F<true>(pl, pr, ql, qr, lam, lam2));
+            if (need1) {
+#pragma unroll
+                for (int tau = 0; tau < 2; tau++) {
+                    ql[tau] = c1[tau][0];
+                    qr[tau] = c1[tau][1];
+                }
+                acc[2].mac(e, layer_F<true>(pl, pr, ql, qr, lam, lam2));
+            }
+#pragma unroll
+            for (int tau = 0; tau < 2; tau++) {
+                ql[tau] = gl_add(gl_sub(c1[tau][0], c0[tau][0]), c1[tau][0]);
+                qr[tau] = gl_add(gl_sub(c1[tau][1], c0[tau][1]), c1[tau][1]);
+            }
+            acc[1].mac(e, layer_F<true>(pl, pr, ql, qr, lam, lam2));
+        }
+        __syncwarp();  // the stage is refilled two chunks on
+    }
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
 
 // Round t of layer d over the pairs b < h handled by this block.
 // t == 1: the vectors as they are. t >= 2: fold the previous round's vectors
 // (length 4h) by rprev first and store the folded halves in place.
 template <bool LEAF>
-__device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* ytab, const EqChunks& EC,
+__device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* ytab, uint8_t* pipe, const EqChunks& EC,
                                             const uint64_t* eq_tab, int t,
                                             int64_t h, unsigned active, uint64_t rprev, uint64_t lam, uint64_t lam2,
                                             bool need1, GlAcc (&acc)[3]) {
     const bool from_keys = t <= 2;  // the unfolded vectors (keys or the children's level)
+    if (LEAF && t <= 2 && A.piped && h >= 32) {
+        if (t == 1)
+            leaf_round_piped<1>(A, ytab, pipe, EC, eq_tab, h, active, rprev, lam, lam2, need1, acc);
+        else
+            leaf_round_piped<2>(A, ytab, pipe, EC, eq_tab, h, active, rprev, lam, lam2, need1, acc);
+        return;
+    }
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
         if (LEAF && t == 1) {
             // X = 0 (and 1) from the stored level above the leaves; X = 2 from four denominators
@@ -541,8 +766,7 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* y
             acc[0].mac(e, parent_F(A, b, lam, lam2));
             if (need1) acc[2].mac(e, parent_F(A, b + h, lam, lam2));
             uint64_t pl[2] = {1, 1}, pr[2] = {1, 1}, ql[2], qr[2];
-            leaf_den_at2(A, 2 * b, 2 * (b + h), ql[0], ql[1]);
-            leaf_den_at2(A, 2 * b + 1, 2 * (b + h) + 1, qr[0], qr[1]);
+            leaf_pair_at2(A, ytab, b, h, ql, qr);
             acc[1].mac(e, layer_F<true>(pl, pr, ql, qr, lam, lam2));
             continue;
         }
@@ -698,9 +922,11 @@ __global__ void __launch_bounds__(LEAF ? LU_LEAF_THREADS : LU_THREADS, LEAF ? FP
     __shared__ uint64_t zs[32];
     __shared__ uint64_t s_lam;
     __shared__ uint64_t eq_tab[3 << kEqChunk];
-    __shared__ uint64_t ytab[LEAF ? 256 : 1];
+    extern __shared__ __align__(16) uint64_t gkr_dyn_smem[];  // the leaf layer's wide y table, then its stages
+    uint64_t* ytab = gkr_dyn_smem;
+    uint8_t* pipe = reinterpret_cast<uint8_t*>(gkr_dyn_smem + kYWide);
     const int d = A.d;
-    if (LEAF) leaf_ytab_build(A.chal, ytab);  // visible after the first barrier below
+    if (LEAF) leaf_ytabw_build(A.chal, ytab);  // visible after the first barrier below
     if (A.t_begin == 1) {
         // the layer's own challenges: mu (last point coordinate) and lambda
         uint64_t mu, lam;
@@ -738,7 +964,7 @@ __global__ void __launch_bounds__(LEAF ? LU_LEAF_THREADS : LU_THREADS, LEAF ? FP
             return;
         }
         GlAcc sums[3];
-        layer_round<LEAF>(A, ytab, EC, eq_tab, t, h, active, rprev, lam, lam2, zs[t - 1] == 0, sums);
+        layer_round<LEAF>(A, ytab, pipe, EC, eq_tab, t, h, active, rprev, lam, lam2, zs[t - 1] == 0, sums);
         uint64_t acc[3] = {sums[0].value(), sums[1].value(), sums[2].value()};
         bool last;
         if (active == 1) {
@@ -1059,8 +1285,12 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
 
     // ---- layer sum-checks: one resident kernel per layer, all queued up front ----
     int occ[2] = {0, 0};
+    // the leaf layer's kernel takes its wide y table as dynamic shared memory (above the 48 KB
+    // of static shared memory a kernel may declare)
+    const size_t leaf_smem = (size_t)8 * kYWide + kPipeBytes;
+    FP_CUDA(c, cudaFuncSetAttribute(gkr_layer_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)leaf_smem));
     FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[0], gkr_layer_kernel<false>, LU_THREADS, 0));
-    FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[1], gkr_layer_kernel<true>, LU_LEAF_THREADS, 0));
+    FP_CUDA(c, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[1], gkr_layer_kernel<true>, LU_LEAF_THREADS, leaf_smem));
     std::vector<GkrLayer> layers(v > 1 ? v - 1 : 0);
     for (int d = 1; d <= v - 1; d++) {
         const bool leaf = (d == v - 1);
@@ -1088,6 +1318,7 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
         }
         A.E = E;
         A.keys = K;
+        A.keys_vec = (uintptr_t)K.r % 8 == 0 && (uintptr_t)K.q % 8 == 0 && (uintptr_t)K.y % 2 == 0;
         A.chal = C;
         A.zin = zb[d & 1];
         A.zout = zb[(d + 1) & 1];
@@ -1097,6 +1328,8 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
         // small layers: fewer threads, so single-block rounds reduce over fewer warps
         A.threads = (int)std::min<int64_t>(leaf ? LU_LEAF_THREADS : LU_THREADS, std::max<int64_t>(64, h1));
         A.per_block = A.threads;  // one pair per thread: the single-block rounds stay short chains
+        A.piped = leaf && (uintptr_t)K.r % 16 == 0 && (uintptr_t)K.q % 16 == 0 && (uintptr_t)K.y % 16 == 0 &&
+                  A.threads == LU_LEAF_THREADS;
         const int64_t want = (h1 + A.per_block - 1) / A.per_block;
         const int cap = std::max(1, occ[leaf ? 1 : 0]) * c->num_sms;
         A.grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
@@ -1116,7 +1349,7 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
             fp_tic(c, st, K_GKR_ROUND, bytes, &slot);
             FP_CUDA(c, cudaLaunchCooperativeKernel(leaf ? (const void*)gkr_layer_kernel<true>
                                                         : (const void*)gkr_layer_kernel<false>,
-                                                   dim3(A.grid), dim3(A.threads), args, 0, st));
+                                                   dim3(A.grid), dim3(A.threads), args, leaf ? leaf_smem : 0, st));
             fp_toc(c, st, slot);
         }
     }
@@ -1173,7 +1406,8 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
                     fp_tic(c, st, K_GKR_ROUND, gkr_round_bytes(leaf, t, (double)h), &slot);
                 else
                     fp_tic(c, st, K_GKR_FINAL, 128.0, &slot);
-                FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(t <= d ? A.grid : 1), dim3(A.threads), args, 0, st));
+                FP_CUDA(c, cudaLaunchCooperativeKernel(kern, dim3(t <= d ? A.grid : 1), dim3(A.threads), args,
+                                                       leaf ? leaf_smem : 0, st));
                 fp_toc(c, st, slot);
             }
             if ((rc = fp_session_wait(c, A.seq0 + t, st))) return rc;
