@@ -683,6 +683,12 @@ int launch_variant(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st)
 //                      Y = hi 256 + lo for two limbs, the rescale / remainder / clamp, stores.
 // Every wait is bounded; a wait that runs out sets the error word and an abort flag that ends the
 // other roles' waits, and the kernel drains its copies and MMAs before it frees tensor memory.
+#ifndef FP_WS_XBUF
+#define FP_WS_XBUF 3
+#endif
+#ifndef FP_WS_EXP_WARPS
+#define FP_WS_EXP_WARPS 12
+#endif
 constexpr int WS_BM = 128;                  // tokens per tile: MMA M, tensor-memory lanes
 constexpr int WS_BK = 128;                  // bytes of K per k-tile
 constexpr int WS_A_BYTES = WS_BM * WS_BK;   // 16 KB
@@ -696,13 +702,22 @@ struct WsCfg {
     static constexpr int ACC_COLS = LIMBS * BN;    // tensor-memory columns per accumulator slot
     static constexpr int BP_BYTES = BN * (W4 ? WS_BK / 2 : WS_BK);        // the weight box as loaded
     static constexpr int X_BYTES = EXPAND ? LIMBS * BN * WS_BK : 0;       // one expanded buffer
-    static constexpr int RING = WS_A_BYTES + BP_BYTES;                    // one ring stage
-    static constexpr int STAGES_FIT = (216 * 1024 - 2 * X_BYTES) / RING;
-    static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-    static constexpr int EXP_WARPS = EXPAND ? 8 : 0;  // two per SM sub-partition: the expansion is latency-bound
-    static constexpr int EPI0 = 2 + EXP_WARPS;     // first epilogue warp (four: lane quarters 2, 3, 0, 1)
+    // Expanded sites: an Xt ring of SA stages (freed by the MMAs that read it), a weight ring of SP
+    // stages (freed by the expansion as soon as it has read the box, so the weight stream runs ahead
+    // of the MMAs) and SX expanded buffers (the expansion runs up to SX k-tiles ahead of the MMAs).
+    // Unscaled int8: one ring of Xt and weight boxes.
+    static constexpr int RING = WS_A_BYTES + BP_BYTES;
+    static constexpr int BUDGET = 208 * 1024;
+    static constexpr int SX = EXPAND ? FP_WS_XBUF : 1;
+    static constexpr int SA_RAW = EXPAND ? (SX > 2 ? 3 : 4) : BUDGET / RING;
+    static constexpr int SA = SA_RAW > 6 ? 6 : SA_RAW;
+    static constexpr int SP_RAW = EXPAND ? (BUDGET - SX * X_BYTES - SA * WS_A_BYTES) / BP_BYTES : 0;
+    static constexpr int SP = SP_RAW > 8 ? 8 : SP_RAW;
+    static constexpr int A_STAGE = EXPAND ? WS_A_BYTES : RING;  // bytes of one Xt-ring stage
+    static constexpr int EXP_WARPS = EXPAND ? FP_WS_EXP_WARPS : 0;  // the expansion is latency-bound: several per sub-partition
+    static constexpr int EPI0 = 3 + EXP_WARPS;     // first epilogue warp (four consecutive: every lane quarter)
     static constexpr int THREADS = 32 * (EPI0 + 4);
-    static constexpr int SMEM = STAGES * RING + 2 * X_BYTES + 1024;
+    static constexpr int SMEM = SA * A_STAGE + SP * BP_BYTES + SX * X_BYTES + 1024;
     // s32 accumulator, A s8, B s8 (or u8 for the low limb), both K-major, N = BN, M = 128
     static constexpr uint32_t IDESC_S8 =
         (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(WS_BM >> 4) << 24);
@@ -724,18 +739,6 @@ struct alignas(64) SiteWs {
     int32_t pad;
     int64_t tile_base;  // first tile of this site
 };
-
-__device__ __forceinline__ int ws_find_site(const SiteWs* sites, int nsites, int64_t t) {
-    int lo = 0, hi = nsites - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (sites[mid].tile_base <= t)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    return lo;
-}
 
 // one bounded wait on an mbarrier phase; false if it ran out (the kernel is then aborting) or
 // another role has aborted
@@ -829,8 +832,9 @@ __device__ __forceinline__ void ws_expand(const SiteWs& S, const uint8_t* pk, ui
     if (W4) {
         // 16-byte packed chunk c: row c >> 2, k values 32 (c & 3) .. + 31 -> two 16-byte chunks
 #pragma unroll
-        for (int u = 0; u < C::BN * 4 / ET; u++) {
+        for (int u = 0; u < (C::BN * 4 + ET - 1) / ET; u++) {
             const int c = et + ET * u, row = c >> 2, kq = c & 3;
+            if ((C::BN * 4) % ET != 0 && c >= C::BN * 4) break;
             const uint4 v = *reinterpret_cast<const uint4*>(pk + row * 64 + kq * 16);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             uint32_t o[8];
@@ -855,8 +859,9 @@ __device__ __forceinline__ void ws_expand(const SiteWs& S, const uint8_t* pk, ui
     } else {
         // scaled int8: 16-byte chunk c: row c >> 3, k values 16 (c & 7) .. + 15
 #pragma unroll
-        for (int u = 0; u < C::BN * 8 / ET; u++) {
+        for (int u = 0; u < (C::BN * 8 + ET - 1) / ET; u++) {
             const int c = et + ET * u, row = c >> 3, kc = c & 7;
+            if ((C::BN * 8) % ET != 0 && c >= C::BN * 8) break;
             const uint4 v = *reinterpret_cast<const uint4*>(pk + row * 128 + kc * 16);
             const int i = i0 + row, g = (kt * WS_BK + kc * 16) >> 6;
             const int s = (i < S.M && g < S.G) ? (int)S.scales[(int64_t)i * S.G + g] : 0;
@@ -916,28 +921,40 @@ __device__ __forceinline__ void ws_ld16(uint32_t a, uint32_t (&v)[16]) {
 
 template <bool W4, bool SCALED>
 __global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
-    witness_ws_kernel(const SiteWs* __restrict__ sites, int nsites, int64_t ntiles, volatile uint64_t* err) {
+    witness_ws_kernel(const SiteWs* __restrict__ sites, const int4* __restrict__ sched, int64_t ntiles,
+                      volatile uint64_t* err) {
     using C = WsCfg<W4, SCALED>;
-    constexpr int ST = C::STAGES;
+    constexpr int SA = C::SA, SP = C::SP > 0 ? C::SP : 1;
     extern __shared__ uint8_t ws_smem_raw[];
     uint8_t* smem = ws_smem_raw + ((1024 - (smem_addr(ws_smem_raw) & 1023)) & 1023);
-    uint8_t* ring = smem;                 // stage s: the Xt box at s RING, the weight box after it
-    uint8_t* xbuf = smem + ST * C::RING;  // two expanded buffers (high limb first)
-    __shared__ __align__(8) uint64_t full[ST], empty[ST], xfull[2], xempty[2], accfull[2], accempty[2], fin;
+    uint8_t* aring = smem;                          // Xt-ring stage s at s A_STAGE (+ the weight box, unexpanded)
+    uint8_t* pring = smem + SA * C::A_STAGE;        // weight-ring stage s at s BP_BYTES (expanded sites)
+    uint8_t* xbuf = pring + C::SP * C::BP_BYTES;    // SX expanded buffers (high limb first)
+    constexpr int SX = C::SX;
+    __shared__ __align__(8) uint64_t afull[SA], aempty[SA], pfull[SP], pempty[SP], xfull[SX], xempty[SX], accfull[2],
+        accempty[2], fin;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int s_abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
 #pragma unroll
-        for (int s = 0; s < ST; s++) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[s])));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&empty[s])));
+        for (int s = 0; s < SA; s++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&afull[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&aempty[s])));
+        }
+#pragma unroll
+        for (int s = 0; s < SP; s++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&pfull[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(&pempty[s])), "r"(32 * C::EXP_WARPS));
+        }
+#pragma unroll
+        for (int e = 0; e < SX; e++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(&xfull[e])), "r"(32 * C::EXP_WARPS));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&xempty[e])));
         }
 #pragma unroll
         for (int e = 0; e < 2; e++) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(&xfull[e])), "r"(32 * C::EXP_WARPS));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&xempty[e])));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&accfull[e])));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 128;\n" ::"r"(smem_addr(&accempty[e])));
         }
@@ -954,40 +971,53 @@ __global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
     const uint32_t tmem = tmem_base;
 
-    if (warp == 0) {
+    if (warp == 0 || (warp == 2 && C::EXPAND)) {
         if (lane == 0) {
-            // ---- producer ----
+            // ---- producers: warp 0 the Xt ring (with the weight boxes when nothing is expanded),
+            // warp 2 the weight ring of expanded sites ----
+            const bool xt = warp == 0;
+            const int NS = xt ? SA : SP;
+            uint64_t* fullb = xt ? afull : pfull;
+            uint64_t* emptyb = xt ? aempty : pempty;
+            const uint32_t bytes = xt ? (uint32_t)C::A_STAGE : (uint32_t)C::BP_BYTES;
             uint32_t it = 0;
             const SiteWs* cur = nullptr;
             bool ok = true;
+            int4 nx = blockIdx.x < ntiles ? sched[blockIdx.x] : make_int4(0, 0, 0, 0);
             for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const SiteWs* S = &sites[ws_find_site(sites, nsites, t)];
+                const int4 e = nx;  // {site, j0, i0, k-tiles}
+                if (t + gridDim.x < ntiles) nx = sched[t + gridDim.x];
+                const SiteWs* S = &sites[e.x];
                 if (S != cur) {
                     asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(&S->tmA) : "memory");
                     asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;\n" ::"l"(&S->tmB) : "memory");
                     cur = S;
                 }
-                const int64_t lt = t - S->tile_base;
-                const int j0 = (int)(lt / S->tiles_i) * WS_BM, i0 = (int)(lt % S->tiles_i) * C::BN;
-                for (int kt = 0; kt < S->nk; kt++, it++) {
-                    const int s = (int)(it % ST);
-                    const uint32_t n = it / ST;
-                    if (n > 0 && !ws_wait(smem_addr(&empty[s]), (n - 1) & 1u, &s_abort, err)) {
+                const int j0 = e.y, i0 = e.z;
+                for (int kt = 0; kt < e.w; kt++, it++) {
+                    const int s = (int)(it % NS);
+                    const uint32_t n = it / NS;
+                    if (n > 0 && !ws_wait(smem_addr(&emptyb[s]), (n - 1) & 1u, &s_abort, err)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = smem_addr(&full[s]);
-                    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(fb), "r"(C::RING) : "memory");
-                    ws_tma2d(smem_addr(ring + s * C::RING), &S->tmA, kt * WS_BK, j0, fb);
-                    ws_tma2d(smem_addr(ring + s * C::RING + WS_A_BYTES), &S->tmB, kt * (W4 ? WS_BK / 2 : WS_BK), i0, fb);
+                    const uint32_t fb = smem_addr(&fullb[s]);
+                    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(fb), "r"(bytes) : "memory");
+                    const int kw = kt * (W4 ? WS_BK / 2 : WS_BK);
+                    if (xt) {
+                        ws_tma2d(smem_addr(aring + s * C::A_STAGE), &S->tmA, kt * WS_BK, j0, fb);
+                        if (!C::EXPAND) ws_tma2d(smem_addr(aring + s * C::A_STAGE + WS_A_BYTES), &S->tmB, kw, i0, fb);
+                    } else {
+                        ws_tma2d(smem_addr(pring + s * C::BP_BYTES), &S->tmB, kw, i0, fb);
+                    }
                 }
             }
             if (!ok) {
                 // let every copy that was issued land before the block ends
-                for (int s = 0; s < ST; s++) {
+                for (int s = 0; s < NS; s++) {
                     if (it <= (uint32_t)s) continue;
-                    const uint32_t last = (uint32_t)s + ((it - 1 - (uint32_t)s) / ST) * ST;
-                    ws_drain(smem_addr(&full[s]), (last / ST) & 1u);
+                    const uint32_t last = (uint32_t)s + ((it - 1 - (uint32_t)s) / NS) * NS;
+                    ws_drain(smem_addr(&fullb[s]), (last / NS) & 1u);
                 }
             }
         }
@@ -997,22 +1027,24 @@ __global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
             // ---- MMA issue ----
             uint32_t it = 0, tc = 0;
             bool ok = true;
+            int4 nx = blockIdx.x < ntiles ? sched[blockIdx.x] : make_int4(0, 0, 0, 0);
             for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, tc++) {
-                const SiteWs* S = &sites[ws_find_site(sites, nsites, t)];
+                const int nk = nx.w;
+                if (t + gridDim.x < ntiles) nx = sched[t + gridDim.x];
                 const uint32_t a = tc & 1u;
                 if (tc >= 2 && !ws_wait(smem_addr(&accempty[a]), ((tc >> 1) - 1) & 1u, &s_abort, err)) break;
                 asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
                 const uint32_t dst = tmem + a * C::ACC_COLS;
-                for (int kt = 0; kt < S->nk; kt++, it++) {
-                    const int s = (int)(it % ST), e = (int)(it & 1u);
-                    if (!ws_wait(smem_addr(&full[s]), (it / ST) & 1u, &s_abort, err) ||
-                        (C::EXPAND && !ws_wait(smem_addr(&xfull[e]), (it >> 1) & 1u, &s_abort, err))) {
+                for (int kt = 0; kt < nk; kt++, it++) {
+                    const int s = (int)(it % SA), e = (int)(it % SX);
+                    if (!ws_wait(smem_addr(&afull[s]), (it / SA) & 1u, &s_abort, err) ||
+                        (C::EXPAND && !ws_wait(smem_addr(&xfull[e]), (it / SX) & 1u, &s_abort, err))) {
                         ok = false;
                         break;
                     }
                     asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
-                    const uint32_t a0 = smem_addr(ring + s * C::RING);
-                    const uint32_t b0 = C::EXPAND ? smem_addr(xbuf + e * C::X_BYTES) : smem_addr(ring + s * C::RING + WS_A_BYTES);
+                    const uint32_t a0 = smem_addr(aring + s * C::A_STAGE);
+                    const uint32_t b0 = C::EXPAND ? smem_addr(xbuf + e * C::X_BYTES) : a0 + WS_A_BYTES;
 #pragma unroll
                     for (int kc = 0; kc < WS_BK / 32; kc++) {
                         const uint32_t en = (kt > 0 || kc > 0) ? 1u : 0u;
@@ -1020,7 +1052,7 @@ __global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
                         if (SCALED)
                             ws_mma(dst + C::BN, tc_desc(a0 + kc * 32), tc_desc(b0 + C::BN * WS_BK + kc * 32), C::IDESC_U8, en);
                     }
-                    ws_commit(smem_addr(&empty[s]));
+                    ws_commit(smem_addr(&aempty[s]));
                     if (C::EXPAND) ws_commit(smem_addr(&xempty[e]));
                 }
                 if (ok) ws_commit(smem_addr(&accfull[a]));
@@ -1030,35 +1062,41 @@ __global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
             ws_drain(smem_addr(&fin), 0);
         }
         __syncwarp();
-    } else if (warp < C::EPI0) {
-        // ---- expansion ----
-        const int et = tid - 64;
+    } else if (warp >= 3 && warp < C::EPI0) {
+        // ---- expansion: the weight box of k-tile it from the weight ring into expanded buffer it % SX,
+        // the ring stage handed back as soon as it is read ----
+        const int et = tid - 96;
         uint32_t it = 0;
         bool ok = true;
+        int4 nx = blockIdx.x < ntiles ? sched[blockIdx.x] : make_int4(0, 0, 0, 0);
         for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const SiteWs* S = &sites[ws_find_site(sites, nsites, t)];
-            const int64_t lt = t - S->tile_base;
-            const int i0 = (int)(lt % S->tiles_i) * C::BN;
-            for (int kt = 0; kt < S->nk; kt++, it++) {
-                const int s = (int)(it % ST), e = (int)(it & 1u);
-                if (!ws_wait_warp(smem_addr(&full[s]), (it / ST) & 1u, &s_abort, err) ||
-                    (it >= 2 && !ws_wait_warp(smem_addr(&xempty[e]), ((it >> 1) - 1) & 1u, &s_abort, err))) {
+            const int4 te = nx;
+            if (t + gridDim.x < ntiles) nx = sched[t + gridDim.x];
+            const SiteWs* S = &sites[te.x];
+            const int i0 = te.z;
+            for (int kt = 0; kt < te.w; kt++, it++) {
+                const int s = (int)(it % SP), e = (int)(it % SX);
+                if (!ws_wait_warp(smem_addr(&pfull[s]), (it / SP) & 1u, &s_abort, err) ||
+                    (it >= SX && !ws_wait_warp(smem_addr(&xempty[e]), ((it / SX) - 1) & 1u, &s_abort, err))) {
                     ok = false;
                     break;
                 }
-                ws_expand<W4, SCALED>(*S, ring + s * C::RING + WS_A_BYTES, xbuf + e * C::X_BYTES, i0, kt, et);
+                ws_expand<W4, SCALED>(*S, pring + s * C::BP_BYTES, xbuf + e * C::X_BYTES, i0, kt, et);
                 asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // generic writes -> MMA reads
                 ws_arrive(smem_addr(&xfull[e]));
+                ws_arrive(smem_addr(&pempty[s]));
             }
         }
-    } else {
+    } else if (warp >= C::EPI0) {
         // ---- epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (tokens) ----
         const int qd = warp & 3;
         uint32_t tc = 0;
+        int4 nx = blockIdx.x < ntiles ? sched[blockIdx.x] : make_int4(0, 0, 0, 0);
         for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, tc++) {
-            const SiteWs* S = &sites[ws_find_site(sites, nsites, t)];
-            const int64_t lt = t - S->tile_base;
-            const int j0 = (int)(lt / S->tiles_i) * WS_BM, i0 = (int)(lt % S->tiles_i) * C::BN;
+            const int4 te = nx;
+            if (t + gridDim.x < ntiles) nx = sched[t + gridDim.x];
+            const SiteWs* S = &sites[te.x];
+            const int j0 = te.y, i0 = te.z;
             const uint32_t a = tc & 1u;
             if (!ws_wait_warp(smem_addr(&accfull[a]), (tc >> 1) & 1u, &s_abort, err)) break;
             asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
@@ -1121,18 +1159,31 @@ int launch_ws(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st) {
         tiles += (int64_t)d.tiles_i * ((t.N + WS_BM - 1) / WS_BM);
         bytes += (double)t.M * pitch + (double)t.N * t.K + 9.0 * t.M * t.N + (t.scales ? (double)t.M * d.G : 0.0);
     }
-    const size_t sz = sizeof(SiteWs) * h.size();
+    // the tile schedule, {site, j0, i0, k-tiles} per tile in site order (a site's tiles sweep its
+    // weight rows for one token block before the next, so a token block's Xt stays in L2)
+    std::vector<int4> sch((size_t)tiles);
+    for (size_t s = 0; s < h.size(); s++) {
+        const SiteWs& d = h[s];
+        const int64_t nt = (int64_t)d.tiles_i * ((d.N + WS_BM - 1) / WS_BM);
+        for (int64_t lt = 0; lt < nt; lt++)
+            sch[(size_t)(d.tile_base + lt)] =
+                make_int4((int)s, (int)(lt / d.tiles_i) * WS_BM, (int)(lt % d.tiles_i) * C::BN, d.nk);
+    }
+    const size_t sz = sizeof(SiteWs) * h.size(), ssz = sizeof(int4) * sch.size();
     SiteWs* dsites = (SiteWs*)fp_alloc(c->dev, sz);
-    char* hst = (char*)fp_alloc(c->host, sz);
-    if (!dsites || !hst) return fp_fail(c, FP_ERR_OOM, "witness: scratch exhausted");
+    int4* dsch = (int4*)fp_alloc(c->dev, ssz);
+    char* hst = (char*)fp_alloc(c->host, sz + ssz);
+    if (!dsites || !dsch || !hst) return fp_fail(c, FP_ERR_OOM, "witness: scratch exhausted");
     memcpy(hst, h.data(), sz);
+    memcpy(hst + sz, sch.data(), ssz);
     FP_CUDA(c, cudaMemcpyAsync(dsites, hst, sz, cudaMemcpyHostToDevice, st));
+    FP_CUDA(c, cudaMemcpyAsync(dsch, hst + sz, ssz, cudaMemcpyHostToDevice, st));
     auto kern = witness_ws_kernel<W4, SCALED>;
     FP_CUDA(c, cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     const unsigned grid = (unsigned)std::min<int64_t>(tiles, (int64_t)c->num_sms);
     int slot;
     fp_tic(c, st, K_GEMM, bytes, &slot);
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(dsites, (int)h.size(), tiles, &c->mb_dev->err);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(dsites, dsch, tiles, &c->mb_dev->err);
     fp_toc(c, st, slot);
     FP_CUDA(c, cudaGetLastError());
     return FP_OK;
@@ -1160,7 +1211,11 @@ int fp_launch_witness(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t 
     size_t need = 0;
     for (int i = 0; i < 8; i++) need += fp_align_up(sizeof(SiteDev) * v[i].size(), 256) + 256;
     for (int i = 0; i < 2; i++) need += fp_align_up(sizeof(SiteDev) * tcv[i].size(), 256) + 256;
-    for (int i = 0; i < 4; i++) need += fp_align_up(sizeof(SiteWs) * wsv[i].size(), 256) + 256;
+    for (int i = 0; i < 4; i++) {
+        size_t tiles = 0;  // the schedule's entries, counted with 128-row tiles (an upper bound)
+        for (const fp_site& t : wsv[i]) tiles += (size_t)((t.M + 127) / 128) * (size_t)((t.N + WS_BM - 1) / WS_BM);
+        need += fp_align_up(sizeof(SiteWs) * wsv[i].size(), 256) + fp_align_up(sizeof(int4) * tiles, 256) + 512;
+    }
     int rc = fp_reserve(c, c->dev, need + (1 << 20));
     if (rc) return rc;
     rc = fp_reserve(c, c->host, need + (1 << 20));
