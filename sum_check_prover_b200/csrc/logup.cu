@@ -144,8 +144,8 @@ __global__ void __launch_bounds__(1024) hist_kernel(KeySrc K, int k, int64_t L, 
         for (int i = threadIdx.x; i < T; i += blockDim.x) sr[i] = 0;
     __syncthreads();
     uint32_t out_local = 0;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < K.n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t jr = (int64_t)K.r[i] + half;
+    auto count = [&](int32_t rv, int32_t qv, int32_t yv) {
+        const int64_t jr = (int64_t)rv + half;
         if (jr >= 0 && jr < T) {
             if (rem_in_smem)
                 atomicAdd(&sr[jr], 1u);
@@ -154,15 +154,49 @@ __global__ void __launch_bounds__(1024) hist_kernel(KeySrc K, int k, int64_t L, 
         } else {
             out_local++;
         }
-        const int64_t q = K.q[i];
+        const int64_t q = qv;
         if (q >= -HIST_WIN && q < HIST_WIN)
             atomicAdd(&sq[q + HIST_WIN], 1u);
         else if (q >= -32768 && q < 32768)
             atomicAdd(&m_clamp[q + 32768], 1u);
         else
             out_local++;
-        if ((int32_t)K.y[i] != (q < -128 ? -128 : (q > 127 ? 127 : (int32_t)q))) out_local++;
+        if (yv != (q < -128 ? -128 : (q > 127 ? 127 : (int32_t)q))) out_local++;
+    };
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t done = 0;  // keys below this index are counted by the vector loop
+    if (((uintptr_t)K.r | (uintptr_t)K.q) % 16 == 0 && (uintptr_t)K.y % 4 == 0) {
+        // four keys per load (r, q as int4, y as one word), two groups in flight per iteration
+        const int64_t ng = K.n / 4;
+        const int4* r4 = reinterpret_cast<const int4*>(K.r);
+        const int4* q4 = reinterpret_cast<const int4*>(K.q);
+        const uint32_t* y4 = reinterpret_cast<const uint32_t*>(K.y);
+        for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < ng; g += 2 * stride) {
+            const bool two = g + stride < ng;
+            const int4 ra = __ldcs(r4 + g), qa = __ldcs(q4 + g);
+            const uint32_t ya = __ldcs(y4 + g);
+            int4 rb = make_int4(0, 0, 0, 0), qb = rb;
+            uint32_t yb = 0;
+            if (two) {
+                rb = __ldcs(r4 + g + stride);
+                qb = __ldcs(q4 + g + stride);
+                yb = __ldcs(y4 + g + stride);
+            }
+            count(ra.x, qa.x, (int8_t)(ya & 0xFF));
+            count(ra.y, qa.y, (int8_t)((ya >> 8) & 0xFF));
+            count(ra.z, qa.z, (int8_t)((ya >> 16) & 0xFF));
+            count(ra.w, qa.w, (int8_t)(ya >> 24));
+            if (two) {
+                count(rb.x, qb.x, (int8_t)(yb & 0xFF));
+                count(rb.y, qb.y, (int8_t)((yb >> 8) & 0xFF));
+                count(rb.z, qb.z, (int8_t)((yb >> 16) & 0xFF));
+                count(rb.w, qb.w, (int8_t)(yb >> 24));
+            }
+        }
+        done = 4 * ng;
     }
+    for (int64_t i = done + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < K.n; i += stride)
+        count(K.r[i], K.q[i], (int32_t)K.y[i]);
     if (out_local) atomicAdd(outside, out_local);
     __syncthreads();
     for (int i = threadIdx.x; i < 2 * HIST_WIN; i += blockDim.x)
@@ -1010,18 +1044,54 @@ __global__ void __launch_bounds__(LU_THREADS) leaf_eval_kernel(KeySrc K, const u
                                                                uint64_t* __restrict__ out) {
     const int64_t G = 1ll << lo_bits;
     const int64_t ngroups = (K.n + G - 1) >> lo_bits;
+    const bool vec = lo_bits >= 2 && ((uintptr_t)K.r | (uintptr_t)K.q | (uintptr_t)elo) % 16 == 0 && (uintptr_t)K.y % 4 == 0;
     GlAcc tot[3];
     for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
         const int64_t x0 = g << lo_bits;
         const int64_t xe = x0 + G < K.n ? x0 + G : K.n;
         GlAcc a[3], es;
-        for (int64_t x = x0 + threadIdx.x; x < xe; x += blockDim.x) {
-            const uint64_t e = __ldg(elo + (x - x0));
-            a[0].mac32(e, (uint32_t)K.r[x] ^ 0x80000000u);
-            a[1].mac32(e, (uint32_t)K.q[x] ^ 0x80000000u);
-            a[2].mac32(e, (uint32_t)(K.y[x] + 128));
+        auto key = [&](uint64_t e, int32_t rv, int32_t qv, int32_t yv) {
+            a[0].mac32(e, (uint32_t)rv ^ 0x80000000u);
+            a[1].mac32(e, (uint32_t)qv ^ 0x80000000u);
+            a[2].mac32(e, (uint32_t)(yv + 128));
             es.add(e);
+        };
+        int64_t xs = x0;  // keys from here on by the scalar loop
+        if (vec) {
+            // quads of keys (r, q as int4, y as one word, the weights as two 16-byte loads), two in flight
+            const int64_t xq = x0 + ((xe - x0) & ~3ll);
+            const int64_t step = 4 * (int64_t)blockDim.x;
+            for (int64_t x = x0 + 4 * threadIdx.x; x < xq; x += 2 * step) {
+                const bool two = x + step < xq;
+                const int4 ra = __ldcs(reinterpret_cast<const int4*>(K.r + x));
+                const int4 qa = __ldcs(reinterpret_cast<const int4*>(K.q + x));
+                const uint32_t ya = __ldcs(reinterpret_cast<const uint32_t*>(K.y + x));
+                const ulonglong2 ea0 = __ldg(reinterpret_cast<const ulonglong2*>(elo + (x - x0)));
+                const ulonglong2 ea1 = __ldg(reinterpret_cast<const ulonglong2*>(elo + (x - x0) + 2));
+                int4 rb = make_int4(0, 0, 0, 0), qb = rb;
+                uint32_t yb = 0;
+                ulonglong2 eb0 = make_ulonglong2(0, 0), eb1 = eb0;
+                if (two) {
+                    rb = __ldcs(reinterpret_cast<const int4*>(K.r + x + step));
+                    qb = __ldcs(reinterpret_cast<const int4*>(K.q + x + step));
+                    yb = __ldcs(reinterpret_cast<const uint32_t*>(K.y + x + step));
+                    eb0 = __ldg(reinterpret_cast<const ulonglong2*>(elo + (x + step - x0)));
+                    eb1 = __ldg(reinterpret_cast<const ulonglong2*>(elo + (x + step - x0) + 2));
+                }
+                key(ea0.x, ra.x, qa.x, (int8_t)(ya & 0xFF));
+                key(ea0.y, ra.y, qa.y, (int8_t)((ya >> 8) & 0xFF));
+                key(ea1.x, ra.z, qa.z, (int8_t)((ya >> 16) & 0xFF));
+                key(ea1.y, ra.w, qa.w, (int8_t)(ya >> 24));
+                if (two) {
+                    key(eb0.x, rb.x, qb.x, (int8_t)(yb & 0xFF));
+                    key(eb0.y, rb.y, qb.y, (int8_t)((yb >> 8) & 0xFF));
+                    key(eb1.x, rb.z, qb.z, (int8_t)((yb >> 16) & 0xFF));
+                    key(eb1.y, rb.w, qb.w, (int8_t)(yb >> 24));
+                }
+            }
+            xs = xq;
         }
+        for (int64_t x = xs + threadIdx.x; x < xe; x += blockDim.x) key(__ldg(elo + (x - x0)), K.r[x], K.q[x], K.y[x]);
         const uint64_t esum = es.value(), eh = __ldg(ehi + g);
         const uint64_t off[3] = {1ull << 31, 1ull << 31, 128ull};
 #pragma unroll

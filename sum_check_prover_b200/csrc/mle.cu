@@ -67,6 +67,80 @@ __global__ void __launch_bounds__(CL_THREADS)
         ar = GlAcc();
         es = GlAcc();
     };
+    const bool vec = S.M % 4 == 0 && S.M >= 8 * CL_THREADS &&
+                     (((uintptr_t)S.q | (uintptr_t)S.r | (uintptr_t)S.eq_row) & 15) == 0;
+    if (vec) {
+        // four consecutive elements (one row: M is a multiple of 4) per step, two steps' loads in
+        // flight: thread t takes elements 4 t .. 4 t + 3 of every 4 CL_THREADS
+        e = e0 + 4 * (int64_t)threadIdx.x;
+        j = e / S.M;
+        i = e - j * S.M;
+        jcur = j;
+        const bool any = e < e1;
+        for (; e < e1; e += 8 * CL_THREADS) {
+            const int64_t eb = e + 4 * CL_THREADS;
+            int64_t jb = j, ib = i + 4 * CL_THREADS;
+            if (ib >= S.M) {
+                ib -= S.M;
+                jb++;
+            }
+            const bool two = eb < e1;
+            const int4 qa = __ldcs(reinterpret_cast<const int4*>(S.q + e));
+            const int4 ra = __ldcs(reinterpret_cast<const int4*>(S.r + e));
+            const ulonglong2 wa0 = __ldg(reinterpret_cast<const ulonglong2*>(S.eq_row + i));
+            const ulonglong2 wa1 = __ldg(reinterpret_cast<const ulonglong2*>(S.eq_row + i + 2));
+            int4 qb = make_int4(0, 0, 0, 0), rb = qb;
+            ulonglong2 wb0 = make_ulonglong2(0, 0), wb1 = wb0;
+            if (two) {
+                qb = __ldcs(reinterpret_cast<const int4*>(S.q + eb));
+                rb = __ldcs(reinterpret_cast<const int4*>(S.r + eb));
+                wb0 = __ldg(reinterpret_cast<const ulonglong2*>(S.eq_row + ib));
+                wb1 = __ldg(reinterpret_cast<const ulonglong2*>(S.eq_row + ib + 2));
+            }
+            if (j != jcur) {
+                flush();
+                jcur = j;
+            }
+            aq.mac32(wa0.x, (uint32_t)qa.x ^ 0x80000000u);
+            aq.mac32(wa0.y, (uint32_t)qa.y ^ 0x80000000u);
+            aq.mac32(wa1.x, (uint32_t)qa.z ^ 0x80000000u);
+            aq.mac32(wa1.y, (uint32_t)qa.w ^ 0x80000000u);
+            ar.mac32(wa0.x, (uint32_t)ra.x ^ 0x80000000u);
+            ar.mac32(wa0.y, (uint32_t)ra.y ^ 0x80000000u);
+            ar.mac32(wa1.x, (uint32_t)ra.z ^ 0x80000000u);
+            ar.mac32(wa1.y, (uint32_t)ra.w ^ 0x80000000u);
+            es.add(wa0.x);
+            es.add(wa0.y);
+            es.add(wa1.x);
+            es.add(wa1.y);
+            if (two) {
+                if (jb != jcur) {
+                    flush();
+                    jcur = jb;
+                }
+                aq.mac32(wb0.x, (uint32_t)qb.x ^ 0x80000000u);
+                aq.mac32(wb0.y, (uint32_t)qb.y ^ 0x80000000u);
+                aq.mac32(wb1.x, (uint32_t)qb.z ^ 0x80000000u);
+                aq.mac32(wb1.y, (uint32_t)qb.w ^ 0x80000000u);
+                ar.mac32(wb0.x, (uint32_t)rb.x ^ 0x80000000u);
+                ar.mac32(wb0.y, (uint32_t)rb.y ^ 0x80000000u);
+                ar.mac32(wb1.x, (uint32_t)rb.z ^ 0x80000000u);
+                ar.mac32(wb1.y, (uint32_t)rb.w ^ 0x80000000u);
+                es.add(wb0.x);
+                es.add(wb0.y);
+                es.add(wb1.x);
+                es.add(wb1.y);
+            }
+            j = jb;
+            i = ib + 4 * CL_THREADS;
+            while (i >= S.M) {
+                i -= S.M;
+                j++;
+            }
+        }
+        if (any) flush();
+        e = e1;  // the scalar loop below has nothing left
+    }
     for (; e < e1; e += CL_THREADS) {
         if (j != jcur) {
             flush();
@@ -87,7 +161,7 @@ __global__ void __launch_bounds__(CL_THREADS)
             }
         }
     }
-    if (e0 + threadIdx.x < e1) flush();
+    if (!vec && e0 + threadIdx.x < e1) flush();
     uint64_t acc = tot.value();
     acc = warp_sum_gl(acc);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;

@@ -683,6 +683,12 @@ int launch_variant(fp_ctx* c, const std::vector<fp_site>& list, cudaStream_t st)
 //                      Y = hi 256 + lo for two limbs, the rescale / remainder / clamp, stores.
 // Every wait is bounded; a wait that runs out sets the error word and an abort flag that ends the
 // other roles' waits, and the kernel drains its copies and MMAs before it frees tensor memory.
+#ifndef FP_WS_EPI_WARPS
+#define FP_WS_EPI_WARPS 4
+#endif
+#ifndef FP_WS_SA
+#define FP_WS_SA 3
+#endif
 #ifndef FP_WS_XBUF
 #define FP_WS_XBUF 3
 #endif
@@ -709,14 +715,16 @@ struct WsCfg {
     static constexpr int RING = WS_A_BYTES + BP_BYTES;
     static constexpr int BUDGET = 208 * 1024;
     static constexpr int SX = EXPAND ? FP_WS_XBUF : 1;
-    static constexpr int SA_RAW = EXPAND ? (SX > 2 ? 3 : 4) : BUDGET / RING;
+    static constexpr int SA_RAW = EXPAND ? FP_WS_SA : BUDGET / RING;
     static constexpr int SA = SA_RAW > 6 ? 6 : SA_RAW;
     static constexpr int SP_RAW = EXPAND ? (BUDGET - SX * X_BYTES - SA * WS_A_BYTES) / BP_BYTES : 0;
     static constexpr int SP = SP_RAW > 8 ? 8 : SP_RAW;
     static constexpr int A_STAGE = EXPAND ? WS_A_BYTES : RING;  // bytes of one Xt-ring stage
     static constexpr int EXP_WARPS = EXPAND ? FP_WS_EXP_WARPS : 0;  // the expansion is latency-bound: several per sub-partition
-    static constexpr int EPI0 = 3 + EXP_WARPS;     // first epilogue warp (four consecutive: every lane quarter)
-    static constexpr int THREADS = 32 * (EPI0 + 4);
+    static constexpr int EPI0 = 3 + EXP_WARPS;     // first epilogue warp
+    // epilogue warps: four consecutive ones cover the four lane quarters; eight split the columns in two
+    static constexpr int EPI_WARPS = FP_WS_EPI_WARPS;
+    static constexpr int THREADS = 32 * (EPI0 + EPI_WARPS);
     static constexpr int SMEM = SA * A_STAGE + SP * BP_BYTES + SX * X_BYTES + 1024;
     // s32 accumulator, A s8, B s8 (or u8 for the low limb), both K-major, N = BN, M = 128
     static constexpr uint32_t IDESC_S8 =
@@ -956,7 +964,7 @@ __global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&accfull[e])));
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 128;\n" ::"r"(smem_addr(&accempty[e])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(&accempty[e])), "r"(32 * C::EPI_WARPS));
         }
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&fin)));
         s_abort = 0;
@@ -1088,8 +1096,10 @@ __global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
             }
         }
     } else if (warp >= C::EPI0) {
-        // ---- epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (tokens) ----
-        const int qd = warp & 3;
+        // ---- epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (tokens), its share of the
+        // columns in chunks of 16, each chunk's load issued before the previous chunk is stored ----
+        constexpr int COLS = C::BN / (C::EPI_WARPS / 4), NCH = COLS / 16;
+        const int qd = warp & 3, cbase = ((warp - C::EPI0) >> 2) * COLS;
         uint32_t tc = 0;
         int4 nx = blockIdx.x < ntiles ? sched[blockIdx.x] : make_int4(0, 0, 0, 0);
         for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, tc++) {
@@ -1101,22 +1111,34 @@ __global__ void __launch_bounds__(WsCfg<W4, SCALED>::THREADS, 1)
             if (!ws_wait_warp(smem_addr(&accfull[a]), (tc >> 1) & 1u, &s_abort, err)) break;
             asm volatile("tcgen05.fence::after_thread_sync;\n" ::);
             const int j = j0 + 32 * qd + lane;
-            const uint32_t base = tmem + ((uint32_t)(32 * qd) << 16) + a * C::ACC_COLS;
+            const bool live = j < S->N;
+            const uint32_t base = tmem + ((uint32_t)(32 * qd) << 16) + a * C::ACC_COLS + (uint32_t)cbase;
+            if (SCALED) {
+                // two limbs per chunk: both loads, then Y = 256 hi + lo (no prefetch: the registers of a
+                // second chunk would spill)
 #pragma unroll 1
-            for (int c0 = 0; c0 < C::BN; c0 += 16) {
-                uint32_t v[16];
-                ws_ld16(base + (uint32_t)c0, v);
-                if (SCALED) {
-                    uint32_t lo[16];
-                    ws_ld16(base + (uint32_t)(C::BN + c0), lo);
+                for (int c = 0; c < NCH; c++) {
+                    uint32_t v[16], lo[16];
+                    ws_ld16(base + (uint32_t)(16 * c), v);
+                    ws_ld16(base + (uint32_t)(C::BN + 16 * c), lo);
                     asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 #pragma unroll
                     for (int e = 0; e < 16; e++) v[e] = (uint32_t)(int32_t)(256ll * (int32_t)v[e] + (int32_t)lo[e]);
-                } else {
+                    const int i = i0 + cbase + 16 * c;
+                    if (live && i < S->M) ws_store16(*S, j, i, v);
+                }
+            } else {
+                uint32_t v[2][16];
+                ws_ld16(base, v[0]);
+                asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+                for (int c = 0; c < NCH; c++) {
+                    const int cur = c & 1, nxt = cur ^ 1;
+                    if (c + 1 < NCH) ws_ld16(base + (uint32_t)(16 * (c + 1)), v[nxt]);  // lands while chunk c is stored
+                    const int i = i0 + cbase + 16 * c;
+                    if (live && i < S->M) ws_store16(*S, j, i, v[cur]);
                     asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
                 }
-                const int i = i0 + c0;
-                if (j < S->N && i < S->M) ws_store16(*S, j, i, v);
             }
             asm volatile("tcgen05.fence::before_thread_sync;\n" ::);
             ws_arrive(smem_addr(&accempty[a]));
