@@ -77,6 +77,7 @@ REASONS = {
     46: "dsp_round",
     47: "dsp_final",
     48: "dsp_open",
+    49: "ffn_link",
 }
 
 
@@ -143,6 +144,12 @@ def lib():
         L.orc_prove_hi.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64,
                                    C.POINTER(u64), vp, C.POINTER(u64)]
         L.orc_verify_hi.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp]
+        L.orc_prove_ffn.restype = C.c_int
+        L.orc_prove_ffn.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), C.c_int, C.c_int, vp, vp, u64,
+                                    C.POINTER(u64), vp]
+        L.orc_verify_ffn.restype = C.c_int
+        L.orc_verify_ffn.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), C.c_int, C.c_int, vp, vp, u64,
+                                     vp]
         L.orc_dsp_prove.restype = C.c_int
         L.orc_dsp_prove.argtypes = [vp, vp, vp, vp, u64, u64, C.c_int, vp, u64, C.POINTER(u64)]
         L.orc_dsp_verify.restype = C.c_int
@@ -938,4 +945,44 @@ def lu2_verify(seed: int, sites, wits, proof: bytes):
     tx = L.orc_tx_new(seed)
     rc = L.orc_lu2_verify(tx, cs, len(sites), cw, _ptr(pb), len(proof), _ptr(det))
     L.orc_tx_free(tx)
+    return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))
+
+
+# ---- the FFN layer statement (the layer proof chained with the scale reductions, the SiLU
+# lookup of the gate outputs and the gated product with the up outputs) ---------------------
+
+def silu_outputs(y) -> np.ndarray:
+    """The committed SiLU outputs for 8-bit inputs: silu_q of every entry, as int16."""
+    tab = np.array([silu_q(v) for v in range(-128, 128)], dtype=np.int16)
+    return tab[np.asarray(y, dtype=np.int64) + 128]
+
+
+def prove_ffn(seed: int, sites, wits, ig: int = 0, iu: int = 1, s16=None):
+    """The FFN statement (orc_prove_ffn): gate = sites[ig], up = sites[iu]; s16 defaults to the
+    honest SiLU outputs of the gate's y. Returns (proof bytes, transcript state after)."""
+    L = lib()
+    keep = []
+    cs, cw = _marshal(sites, wits, keep)
+    s = np.ascontiguousarray(silu_outputs(wits[ig][2]) if s16 is None else s16, dtype=np.int16)
+    n = C.c_uint64(0)
+    st = C.create_string_buffer(32)
+    rc = L.orc_prove_ffn(seed, cs, len(sites), cw, ig, iu, _ptr(s), None, 0, C.byref(n), st)
+    if rc not in (0, -2):
+        raise ValueError(f"orc_prove_ffn rejected the statement ({rc})")
+    buf = np.zeros(max(1, n.value), dtype=np.uint8)
+    rc = L.orc_prove_ffn(seed, cs, len(sites), cw, ig, iu, _ptr(s), _ptr(buf), n.value, C.byref(n), st)
+    if rc != 0:
+        raise ValueError(f"orc_prove_ffn failed ({rc})")
+    return buf[: n.value].tobytes(), st.raw
+
+
+def verify_ffn(seed: int, sites, wits, proof: bytes, ig: int = 0, iu: int = 1, s16=None):
+    """Returns (reason_name, detail); 'accept' for a valid proof."""
+    L = lib()
+    keep = []
+    cs, cw = _marshal(sites, wits, keep)
+    s = np.ascontiguousarray(silu_outputs(wits[ig][2]) if s16 is None else s16, dtype=np.int16)
+    pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
+    det = np.zeros(2, dtype=np.int64)
+    rc = L.orc_verify_ffn(seed, cs, len(sites), cw, ig, iu, _ptr(s), _ptr(pb), len(proof), _ptr(det))
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

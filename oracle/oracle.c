@@ -580,6 +580,27 @@ static int site_dims(const orc_site* sites, int ns, int* vM, int* vN, int* n) {
     return 0;
 }
 
+/* The point where the last matmul section (proven or verified) left its sites: the row
+ * challenges r_row (vM), the round challenges rho (n) and the final values A_s(rho), B_s(rho).
+ * The FFN statement continues from it. (The oracle is single-threaded.) */
+#define MM_PT_MAX 64
+static struct {
+    int vM, n, ns;
+    u64 rr[MM_PT_MAX], rho[MM_PT_MAX];
+    u64* fin; /* 2 ns values */
+} g_mm_pt = {0, 0, 0, {0}, {0}, NULL};
+
+static void mm_pt_record(int vM, const u64* rr, int n, const u64* rho, int ns, const u64* fin) {
+    g_mm_pt.vM = vM;
+    g_mm_pt.n = n;
+    g_mm_pt.ns = ns;
+    for (int i = 0; i < vM && i < MM_PT_MAX; i++) g_mm_pt.rr[i] = rr[i];
+    for (int i = 0; i < n && i < MM_PT_MAX; i++) g_mm_pt.rho[i] = rho[i];
+    free(g_mm_pt.fin);
+    g_mm_pt.fin = (u64*)malloc(sizeof(u64) * 2 * (size_t)ns);
+    for (int i = 0; i < 2 * ns; i++) g_mm_pt.fin[i] = fin[i];
+}
+
 static void mm_prove(orc_tx* t, pbuf* pb, const orc_site* sites, int ns, const orc_wit* wit) {
     int vM, vN, n;
     site_dims(sites, ns, &vM, &vN, &n);
@@ -612,6 +633,7 @@ static void mm_prove(orc_tx* t, pbuf* pb, const orc_site* sites, int ns, const o
         orc_partial_x(&sites[s], rc, nn, B[s]);
     }
 
+    u64* chal = (u64*)malloc(sizeof(u64) * (n + 1));
     for (int t_ = 0; t_ < n; t_++) {
         u64 h = L >> 1;
         u64 g[3] = {0, 0, 0};
@@ -630,6 +652,7 @@ static void mm_prove(orc_tx* t, pbuf* pb, const orc_site* sites, int ns, const o
         }
         send_fe(t, pb, "sc_round", g, 3);
         u64 r = orc_tx_squeeze(t, "sc_chal");
+        chal[t_] = r;
         for (int s = 0; s < ns; s++)
             for (u64 b = 0; b < h; b++) {
                 A[s][b] = orc_fadd(A[s][b], orc_fmul(r, orc_fsub(A[s][h + b], A[s][b])));
@@ -643,11 +666,12 @@ static void mm_prove(orc_tx* t, pbuf* pb, const orc_site* sites, int ns, const o
         fin[2 * s + 1] = B[s][0];
     }
     send_fe(t, pb, "sc_final", fin, 2 * (u64)ns);
+    mm_pt_record(vM, rr, n, chal, ns, fin);
     for (int s = 0; s < ns; s++) {
         free(A[s]);
         free(B[s]);
     }
-    free(A); free(B); free(fin); free(rho); free(c); free(rr); free(rc);
+    free(A); free(B); free(fin); free(rho); free(c); free(rr); free(rc); free(chal);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -1036,6 +1060,7 @@ static int mm_verify(orc_tx* t, prd* rd, const orc_site* sites, int ns, const or
     }
     rd_fe(t, rd, "sc_final", fin, 2 * (u64)ns);
     if (rd->bad) FAIL(REJ_FORMAT, 2, 0);
+    mm_pt_record(vM, rr, n, pt, ns, fin);
     {
         u64 acc = 0;
         for (int s = 0; s < ns; s++) acc = orc_fadd(acc, orc_fmul(rho[s], orc_fmul(fin[2 * s], fin[2 * s + 1])));
@@ -3796,5 +3821,175 @@ done:
     free(rho);
     free(P);
     free(B);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The FFN layer statement ("How fast can FlashProve go", 3.1: the weights'  */
+/* group scales, the SiLU by lookup, the gated product by sum-check): the    */
+/* layer proof of orc_prove over the gate, up and down sites, continued on    */
+/* the same transcript by                                                    */
+/*  - the per-group scale reduction of every site with scales, at the point  */
+/*    where the matmul section left W_eff: (r_row's first vM_s coordinates,   */
+/*    the last vK_s round challenges); the matmul's A_s(rho) is that value    */
+/*    times prod_{j < n - vK_s} (1 - rho_j), since the padded columns of a    */
+/*    narrower site are zero;                                                 */
+/*  - the SiLU lookup with g the gate projection's committed outputs y (as    */
+/*    16-bit inputs) and s its committed 16-bit outputs;                      */
+/*  - the gated product of s (as 8-bit values: SiLU of an 8-bit input lies in */
+/*    [-48, 79]) with the up projection's committed outputs.                  */
+/* The product h = s u is 16-bit and the down projection reads 8-bit          */
+/* activations, so h is not linked to the down site here.                     */
+/* ------------------------------------------------------------------------ */
+
+enum { REJ_FFN_LINK = 49 /* a scale reduction's claim is not the weight value the matmul section left (detail: site) */ };
+
+static int ffn_args_ok(const orc_site* sites, int ns, int ig, int iu) {
+    if (ig < 0 || iu < 0 || ig >= ns || iu >= ns || ig == iu) return 0;
+    return sites[ig].M == sites[iu].M && sites[ig].N == sites[iu].N;
+}
+
+/* the scale reduction's point for site s and the factor prod_{j < n - vK} (1 - rho_j) */
+static u64 ffn_scl_point(const orc_site* st, u64* z) {
+    const int vM = orc_log2_ceil((u64)st->M), vK = orc_log2_ceil((u64)st->K), n = g_mm_pt.n;
+    for (int i = 0; i < vM; i++) z[i] = g_mm_pt.rr[i];
+    for (int i = 0; i < vK; i++) z[vM + i] = g_mm_pt.rho[n - vK + i];
+    u64 f = 1;
+    for (int j = 0; j < n - vK; j++) f = orc_fmul(f, orc_fsub(1, g_mm_pt.rho[j]));
+    return f;
+}
+
+/* s (16-bit SiLU outputs) as the gated product's 8-bit factor; 0 if a value does not fit */
+static int8_t* ffn_s8(const int16_t* s, u64 n) {
+    int8_t* o = (int8_t*)malloc(n ? n : 1);
+    for (u64 i = 0; i < n; i++) {
+        if (s[i] < -128 || s[i] > 127) {
+            free(o);
+            return NULL;
+        }
+        o[i] = (int8_t)s[i];
+    }
+    return o;
+}
+
+static int16_t* ffn_g16(const int8_t* y, u64 n) {
+    int16_t* g = (int16_t*)malloc(sizeof(int16_t) * (n ? n : 1));
+    for (u64 i = 0; i < n; i++) g[i] = y[i];
+    return g;
+}
+
+/* Prover. s16: the committed SiLU outputs (gate's M x N entries, token-major like y).
+ * Returns 0, -1 on bad input (including an s that does not fit 8 bits), -2 if the buffer is
+ * too small (*len then holds the size needed); state: the transcript after the statement. */
+int orc_prove_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, int ig, int iu, const int16_t* s16,
+                  uint8_t* proof, u64 cap, u64* len, uint8_t state[32]) {
+    if (ns < 1 || !ffn_args_ok(sites, ns, ig, iu)) return -1;
+    for (int s = 0; s < ns; s++)
+        if (sites[s].M < 1 || sites[s].N < 1 || sites[s].K < 1 || sites[s].k_shift < 1 ||
+            sites[s].k_shift > 30 || (sites[s].w_bits != 4 && sites[s].w_bits != 8) ||
+            sites[s].k_shift != sites[0].k_shift)
+            return -1;
+    const u64 n = (u64)sites[ig].M * (u64)sites[ig].N;
+    int8_t* s8 = ffn_s8(s16, n);
+    if (!s8) return -1;
+    orc_tx t;
+    pbuf pb = {proof, cap, 0, 0};
+    orc_tx_init(&t, seed);
+    absorb_sites(&t, sites, ns, wit);
+    mm_prove(&t, &pb, sites, ns, wit);
+    lu_prove(&t, &pb, sites, ns, wit);
+    int rc = 0;
+    /* each chained statement writes at the end of the proof so far (a size query once full) */
+#define FFN_SUB(call)                                                                  \
+    do {                                                                               \
+        u64 l_ = 0;                                                                    \
+        uint8_t* at_ = pb.overflow ? NULL : pb.p + pb.len;                            \
+        u64 room_ = pb.overflow ? 0 : pb.cap - pb.len;                                \
+        rc = call;                                                                     \
+        if (rc == -2) {                                                                \
+            pb.overflow = 1;                                                           \
+            rc = 0;                                                                    \
+        } else if (rc) {                                                               \
+            goto out;                                                                  \
+        }                                                                              \
+        pb.len += l_;                                                                  \
+    } while (0)
+    for (int s = 0; s < ns; s++) {
+        if (!sites[s].scales) continue;
+        u64 z[MM_PT_MAX];
+        (void)ffn_scl_point(&sites[s], z);
+        FFN_SUB(orc_scl_prove(&t, sites[s].w, sites[s].w_bits, sites[s].scales, sites[s].M, sites[s].K, z, at_, room_,
+                              &l_));
+    }
+    {
+        int16_t* g16 = ffn_g16(wit[ig].y, n);
+        FFN_SUB(orc_silu_prove(&t, g16, s16, n, at_, room_, &l_));
+        free(g16);
+    }
+    FFN_SUB(orc_had_prove(&t, s8, wit[iu].y, n, at_, room_, &l_));
+#undef FFN_SUB
+    memcpy(state, t.st, 32);
+    *len = pb.len;
+    rc = pb.overflow ? -2 : 0;
+out:
+    free(s8);
+    return rc;
+}
+
+/* Verifier of orc_prove_ffn's statement: the layer proof as orc_verify, then each chained
+ * statement, with the scale reductions' claims tied to the matmul section's final values.
+ * Returns 0 on accept or a reason code (the sub-statements' own codes for their failures). */
+int orc_verify_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, int ig, int iu, const int16_t* s16,
+                   const uint8_t* proof, u64 len, int64_t detail[2]) {
+    detail[0] = detail[1] = 0;
+    g_site_mask = NULL;
+    g_verify_flags = 0;
+    if (ns < 1 || !ffn_args_ok(sites, ns, ig, iu)) return REJ_ARGS;
+    for (int s = 0; s < ns; s++)
+        if (sites[s].M < 1 || sites[s].N < 1 || sites[s].K < 1 || sites[s].k_shift < 1 ||
+            sites[s].k_shift > 30 || sites[s].k_shift != sites[0].k_shift)
+            return REJ_ARGS;
+    const u64 n = (u64)sites[ig].M * (u64)sites[ig].N;
+    int8_t* s8 = ffn_s8(s16, n);
+    if (!s8) return REJ_ARGS;
+    orc_tx t;
+    prd rd = {proof, len, 0, 0};
+    orc_tx_init(&t, seed);
+    absorb_sites(&t, sites, ns, wit);
+    int rc = mm_verify(&t, &rd, sites, ns, wit, detail);
+    if (!rc) rc = lu_verify(&t, &rd, sites, ns, wit, detail);
+    u64 pos = rd.pos;
+    for (int s = 0; s < ns && !rc; s++) {
+        if (!sites[s].scales) continue;
+        const int v = orc_log2_ceil((u64)sites[s].M) + orc_log2_ceil((u64)sites[s].K);
+        const u64 ls = 8 + 32 * (u64)v + 16;
+        if (pos + ls > len) {
+            rc = REJ_FORMAT;
+            break;
+        }
+        u64 z[MM_PT_MAX];
+        const u64 f = ffn_scl_point(&sites[s], z);
+        if (orc_fmul(f, get_le(proof + pos, 8)) != g_mm_pt.fin[2 * s]) {
+            rc = REJ_FFN_LINK;
+            detail[0] = s;
+            break;
+        }
+        rc = orc_scl_verify(&t, sites[s].w, sites[s].w_bits, sites[s].scales, sites[s].M, sites[s].K, z, proof + pos,
+                            ls, detail);
+        pos += ls;
+    }
+    if (!rc) {
+        const u64 lh = 8 + 32 * (u64)orc_log2_ceil(n) + 16;
+        if (pos + lh > len) {
+            rc = REJ_FORMAT;
+        } else {
+            const u64 lsilu = len - pos - lh;
+            int16_t* g16 = ffn_g16(wit[ig].y, n);
+            rc = orc_silu_verify(&t, g16, s16, n, proof + pos, lsilu, detail);
+            free(g16);
+            if (!rc) rc = orc_had_verify(&t, s8, wit[iu].y, n, proof + pos + lsilu, lh, detail);
+        }
+    }
+    free(s8);
     return rc;
 }
