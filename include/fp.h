@@ -689,6 +689,24 @@ int fp_lu2_protocol_drive(fp_tx* tx, int v, int k, const uint32_t* m_rem, const 
 /* The SiLU table's 2^16 entries silu_q(v), v = -2^15 .. 2^15 - 1, into host out (no GPU work). */
 int fp_silu_table(int32_t* out);
 
+/* The SiLU's inputs and outputs for 8-bit inputs ("How fast can FlashProve go", 3.1: the SiLU
+ * output is committed and proven by lookup; here its inputs are the gate projection's committed
+ * outputs). For the n device int8 values y (the gate site's y, token-major): g[i] = y[i] (device
+ * int16), s[i] = silu_q(y[i]) (device int16) and s8[i] = s[i] (device int8: silu_q maps
+ * [-128, 127] into [-48, 79]). All four buffers are the caller's, n entries each, on ctx's
+ * device; the kernel runs on `stream` and nothing is allocated. Returns FP_OK or FP_ERR_ARG. */
+int fp_silu_inputs(fp_ctx* ctx, const int8_t* y, int64_t n, int16_t* g, int16_t* s, int8_t* s8, void* stream);
+
+/* The point where the last matmul section proven with ctx (sumcheck_prove_matmul) left its
+ * sites: the row challenges r_row (v_row of them, into host r_row) and the round challenges
+ * rho_1..rho_n (into host rho). A chained statement continues from it: a site's weight value
+ * A_s(rho) is W_eff's MLE at (r_row's first ceil(log2 M_s) coordinates, the last ceil(log2 K_s)
+ * round challenges) times prod_{j <= n - ceil(log2 K_s)} (1 - rho_j) (the padded columns of a
+ * narrower site are zero), the point of the per-group scale reduction (sumcheck_reduce_scales).
+ * Null buffers query the sizes. Returns FP_ERR_ARG if no matmul section was proven yet or a
+ * buffer is too small. */
+int sumcheck_last_point(fp_ctx* ctx, uint64_t* r_row, int cap_row, int* v_row, uint64_t* rho, int cap_rho, int* n);
+
 /*
  * The softmax numerator by lookup ("Towards Proving Frontier-Scale LLM Inference",
  * The arithmetic: the exponential is a lookup table, the integer softmax has a

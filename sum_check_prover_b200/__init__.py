@@ -96,6 +96,8 @@ def lib():
     L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, C.POINTER(sz), vp]
     L.logup_prove_silu.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_silu_table.argtypes = [vp]
+    L.fp_silu_inputs.argtypes = [vp, vp, C.c_int64, vp, vp, vp, vp]
+    L.sumcheck_last_point.argtypes = [vp, vp, i32, C.POINTER(i32), vp, i32, C.POINTER(i32)]
     L.logup_prove_exp.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_exp_table.argtypes = [vp]
     L.fp_proof_size.argtypes = [C.POINTER(_Site), i32, C.POINTER(sz), C.POINTER(sz)]
@@ -890,6 +892,23 @@ class Context:
                                                    C.byref(ln), _stream(stream)), "sumcheck_reduce_scales")
         return buf.raw[: ln.value]
 
+    def silu_inputs(self, y, g, s, s8, stream=None) -> None:
+        """g = y (int16), s = silu_q(y) (int16), s8 = s (int8) for the device int8 tensor y
+        (the gate projection's outputs); the caller's device buffers of y's size."""
+        self._check(self._L.fp_silu_inputs(self.h, _ptr(y), int(y.numel()), _ptr(g), _ptr(s), _ptr(s8),
+                                           _stream(stream)), "fp_silu_inputs")
+
+    def last_point(self):
+        """(r_row, rho) of the last matmul section proven with this context (host integers)."""
+        vr, n = C.c_int32(0), C.c_int32(0)
+        self._check(self._L.sumcheck_last_point(self.h, None, 0, C.byref(vr), None, 0, C.byref(n)),
+                    "sumcheck_last_point")
+        rr = (C.c_uint64 * max(1, vr.value))()
+        rho = (C.c_uint64 * max(1, n.value))()
+        self._check(self._L.sumcheck_last_point(self.h, rr, vr.value, C.byref(vr), rho, n.value, C.byref(n)),
+                    "sumcheck_last_point")
+        return list(rr[: vr.value]), list(rho[: n.value])
+
     def prove_silu(self, tx: Transcript, g, s, stream=None) -> bytes:
         """LogUp proof that every entry of the device int16 tensor s is the SiLU table's entry
         for the same entry of g (flattened row-major); continues tx."""
@@ -1012,6 +1031,53 @@ def prove(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], stream=
         s1 = tx.state()
         lu, status = (ctx.prove_logup if lookup == "gkr" else ctx.prove_logup_hi)(tx, sites, stream)
         return mm + lu, [s0, s1, tx.state()], status
+    finally:
+        tx.close()
+
+
+def _log2c(x: int) -> int:
+    v = 0
+    while (1 << v) < x:
+        v += 1
+    return v
+
+
+def prove_ffn(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], gate: int = 0, up: int = 1,
+              stream=None):
+    """Prove an FFN layer ("How fast can FlashProve go", 3.1) as one statement on one
+    transcript: the layer proof of prove(); the per-group scale reduction of every site with
+    scales, at the point where the matmul section left its weights (r_row's first ceil(log2 M)
+    coordinates, the last ceil(log2 K) round challenges); the SiLU lookup with the gate site's
+    outputs as its inputs; the gated product of the SiLU outputs with the up site's outputs.
+    gate and up index the sites in stage order. Returns (proof bytes, transcript state after,
+    lookup status)."""
+    import torch
+    tx = Transcript(seed)
+    try:
+        for st in stages:
+            ctx.commit_witness(tx, st, stream)
+        sites = [s for st in stages for s in st]
+        parts = [ctx.prove_matmul(tx, sites, stream)]
+        lu, status = ctx.prove_logup(tx, sites, stream)
+        parts.append(lu)
+        r_row, rho = ctx.last_point()
+        n = len(rho)
+        for d in sites:
+            if d.scales is None:
+                continue
+            vm, vk = _log2c(d.M), _log2c(d.K)
+            parts.append(ctx.reduce_scales(tx, d.w, d.w_bits, d.scales, d.M, d.K, r_row[:vm] + rho[n - vk:], stream))
+        g_site, u_site = sites[gate], sites[up]
+        if (g_site.M, g_site.N) != (u_site.M, u_site.N):
+            raise ValueError("prove_ffn: the gate and up sites differ in shape")
+        y = g_site.y
+        g = torch.empty(y.shape, dtype=torch.int16, device=y.device)
+        s = torch.empty(y.shape, dtype=torch.int16, device=y.device)
+        s8 = torch.empty(y.shape, dtype=torch.int8, device=y.device)
+        ctx.silu_inputs(y, g, s, s8, stream)
+        parts.append(ctx.prove_silu(tx, g, s, stream))
+        parts.append(ctx.prove_hadamard(tx, s8, u_site.y, stream))
+        return b"".join(parts), tx.state(), status
     finally:
         tx.close()
 

@@ -96,6 +96,13 @@ struct FpArena {
     bool pinned_host = false;
 };
 
+// where the last single-GPU matmul section left its sites: the row challenges, the round
+// challenges and the final values A_s(rho), B_s(rho)
+struct FpMmPoint {
+    bool valid = false;
+    std::vector<uint64_t> r_row, rho, fin;
+};
+
 struct fp_ctx {
     int device = 0;
     int num_sms = 148;
@@ -119,6 +126,7 @@ struct fp_ctx {
     // witness GEMM kernels: 2 warp-specialised tcgen05 (default), 1 single-role tcgen05 for
     // unscaled sites, 0 mma.sync (FP_TCGEN05 selects 0 or 1)
     int tc_gemm = 2;
+    FpMmPoint mm_point;
     // timing
     int profiling = 0;
     int64_t launches = 0;  // every kernel launch of the library on this context

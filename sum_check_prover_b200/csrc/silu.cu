@@ -476,6 +476,39 @@ int logup_prove_exp(fp_ctx* c, fp_tx* tx, const int16_t* g, const int16_t* s, in
     return lookup16_prove(c, tx, kExpLabels, exp_q_host(0), g, s, n, proof, proof_len, stream);
 }
 
+namespace {
+
+// The SiLU's inputs and outputs for 8-bit inputs (the gate projection's outputs): g = y widened,
+// s = silu_q(y) as 16-bit and as 8-bit values (silu_q maps [-128, 127] into [-48, 79])
+struct SiluTab8 {
+    int16_t v[256];
+};
+
+__global__ void silu_inputs_kernel(const int8_t* __restrict__ y, int64_t n, SiluTab8 tab, int16_t* __restrict__ g,
+                                   int16_t* __restrict__ s, int8_t* __restrict__ s8) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int v = y[i];
+        const int16_t o = tab.v[v + 128];
+        g[i] = (int16_t)v;
+        s[i] = o;
+        s8[i] = (int8_t)o;
+    }
+}
+
+}  // namespace
+
+int fp_silu_inputs(fp_ctx* c, const int8_t* y, int64_t n, int16_t* g, int16_t* s, int8_t* s8, void* stream) {
+    if (!c || !y || !g || !s || !s8 || n < 1) return fp_fail(c, FP_ERR_ARG, "fp_silu_inputs: bad argument");
+    FP_CUDA(c, cudaSetDevice(c->device));
+    SiluTab8 tab;
+    for (int v = -128; v < 128; v++) tab.v[v + 128] = (int16_t)silu_q_host(v);
+    cudaStream_t st = (cudaStream_t)stream;
+    const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 8ll * c->num_sms);
+    silu_inputs_kernel<<<grid, 256, 0, st>>>(y, n, tab, g, s, s8);
+    FP_CUDA(c, cudaGetLastError());
+    return FP_OK;
+}
+
 int fp_silu_table(int32_t* out) {
     if (!out) return FP_ERR_ARG;
     for (int64_t v = -32768; v < 32768; v++) out[v + 32768] = (int32_t)silu_q_host(v);

@@ -250,7 +250,7 @@ int fp_shard_view(fp_ctx* c, const fp_shard* shard, int nsites, FpShardView& sh)
 namespace {
 
 int mm_protocol(fp_tx* tx, int vM, int vN, int n, int nsites, const FpShardView& sh, MmSource& src, uint8_t* proof,
-                size_t* proof_len) {
+                size_t* proof_len, FpMmPoint* pt_out = nullptr) {
     int rc;
     const int lo = sh.lo[sh.rank], own = sh.lo[sh.rank + 1] - lo;
     FpPoint zr, zc;
@@ -259,6 +259,7 @@ int mm_protocol(fp_tx* tx, int vM, int vN, int n, int nsites, const FpShardView&
     for (int i = 0; i < vM; i++) zr.z[i] = fp_tx_squeeze_one(tx, "r_row");
     for (int i = 0; i < vN; i++) zc.z[i] = fp_tx_squeeze_one(tx, "r_col");
     if ((rc = src.start(zr, zc))) return rc;
+    std::vector<uint64_t> chal;
 
     // claims of every site, in site order
     std::vector<uint64_t> mine(2 * (size_t)std::max(1, own)), all(2 * (size_t)nsites);
@@ -289,6 +290,7 @@ int mm_protocol(fp_tx* tx, int vM, int vN, int n, int nsites, const FpShardView&
         fp_tx_absorb_raw(tx, "sc_round", proof + pos, 24);
         pos += 24;
         const uint64_t r = fp_tx_squeeze_one(tx, "sc_chal");
+        chal.push_back(r);
         if ((rc = src.answer(t, r))) return rc;
         const uint64_t r1 = gl_sub(r, 1), r2 = gl_sub(r, 2);
         claim = gl_add(gl_add(gl_mul(g[0], gl_mul(gl_mul(r1, r2), inv2)), gl_sub(0, gl_mul(g[1], gl_mul(r, r2)))),
@@ -300,6 +302,12 @@ int mm_protocol(fp_tx* tx, int vM, int vN, int n, int nsites, const FpShardView&
     fp_tx_absorb_raw(tx, "sc_final", proof + pos, 16 * (size_t)nsites);
     pos += 16 * (size_t)nsites;
     *proof_len = pos;
+    if (pt_out) {
+        pt_out->r_row.assign(zr.z, zr.z + vM);
+        pt_out->rho = chal;
+        pt_out->fin = all;
+        pt_out->valid = true;
+    }
     return FP_OK;
 }
 
@@ -559,7 +567,8 @@ int prove_matmul(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, const f
     MmDevice dev;
     if ((rc = mm_device_setup(c, sites + lo, own, n, (cudaStream_t)stream, dev))) return rc;
     dev.weighted = nsites > 1;
-    rc = mm_protocol(tx, vM, vN, n, nsites, sh, dev, proof, proof_len);
+    c->mm_point.valid = false;
+    rc = mm_protocol(tx, vM, vN, n, nsites, sh, dev, proof, proof_len, &c->mm_point);
     if (rc) dev.abandon();
     return rc;
 }
@@ -648,4 +657,15 @@ int fp_mm_shard_protocol_drive(fp_tx* tx, const fp_site* sites, int nsites, cons
     cb.own = sh.lo[sh.rank + 1] - sh.lo[sh.rank];
     cb.n = n;
     return mm_protocol(tx, vM, vN, n, nsites, sh, cb, proof, proof_len);
+}
+
+int sumcheck_last_point(fp_ctx* c, uint64_t* r_row, int cap_row, int* v_row, uint64_t* rho, int cap_rho, int* n) {
+    if (!c || !v_row || !n) return FP_ERR_ARG;
+    if (!c->mm_point.valid) return fp_fail(c, FP_ERR_ARG, "sumcheck_last_point: no matmul section proven yet");
+    *v_row = (int)c->mm_point.r_row.size();
+    *n = (int)c->mm_point.rho.size();
+    if ((r_row && cap_row < *v_row) || (rho && cap_rho < *n)) return fp_fail(c, FP_ERR_ARG, "sumcheck_last_point: buffer too small");
+    if (r_row) memcpy(r_row, c->mm_point.r_row.data(), 8 * (size_t)*v_row);
+    if (rho) memcpy(rho, c->mm_point.rho.data(), 8 * (size_t)*n);
+    return FP_OK;
 }
