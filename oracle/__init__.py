@@ -78,6 +78,8 @@ REASONS = {
     47: "dsp_final",
     48: "dsp_open",
     49: "ffn_link",
+    50: "ffn_hidden",
+    51: "ffn_down",
 }
 
 
@@ -145,11 +147,13 @@ def lib():
                                    C.POINTER(u64), vp, C.POINTER(u64)]
         L.orc_verify_hi.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), vp, u64, vp]
         L.orc_prove_ffn.restype = C.c_int
-        L.orc_prove_ffn.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), C.c_int, C.c_int, vp, vp, u64,
-                                    C.POINTER(u64), vp]
+        L.orc_prove_ffn.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), C.c_int, C.c_int, C.c_int,
+                                    C.c_int, vp, vp, vp, vp, vp, u64, C.POINTER(u64), vp]
         L.orc_verify_ffn.restype = C.c_int
-        L.orc_verify_ffn.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), C.c_int, C.c_int, vp, vp, u64,
-                                     vp]
+        L.orc_verify_ffn.argtypes = [u64, C.POINTER(_Site), C.c_int, C.POINTER(_Wit), C.c_int, C.c_int, C.c_int,
+                                     C.c_int, vp, vp, vp, vp, vp, u64, vp]
+        L.orc_ffn_hidden.restype = C.c_int
+        L.orc_ffn_hidden.argtypes = [vp, vp, u64, C.c_int, vp, vp, vp]
         L.orc_dsp_prove.restype = C.c_int
         L.orc_dsp_prove.argtypes = [vp, vp, vp, vp, u64, u64, C.c_int, vp, u64, C.POINTER(u64)]
         L.orc_dsp_verify.restype = C.c_int
@@ -391,6 +395,10 @@ def resolve(wl) -> Resolved:
             if s.xt_link is not None:
                 src, off = out_buffer(s.xt_link[0])
                 s.xt = src[off + s.xt_link[1]: off + s.xt_link[1] + s.N * s.K].reshape(s.N, s.K).copy()
+            if getattr(s, "xt_hidden", None) is not None:
+                ig, iu, kh = s.xt_hidden
+                s16 = silu_outputs(wits[ig][2])
+                s.xt = ffn_hidden(s16.astype(np.int8), wits[iu][2], kh)[2].reshape(s.N, s.K)
             q, r, y = witness(s)
             if s.out_group is not None:
                 g = groups[s.out_group[0]]
@@ -957,32 +965,63 @@ def silu_outputs(y) -> np.ndarray:
     return tab[np.asarray(y, dtype=np.int64) + 128]
 
 
-def prove_ffn(seed: int, sites, wits, ig: int = 0, iu: int = 1, s16=None):
-    """The FFN statement (orc_prove_ffn): gate = sites[ig], up = sites[iu]; s16 defaults to the
-    honest SiLU outputs of the gate's y. Returns (proof bytes, transcript state after)."""
+def ffn_hidden(s, u, kh: int):
+    """The rescaled hidden activations (orc_ffn_hidden) of the products s * u (8-bit SiLU outputs
+    and up outputs, same shape): (q_h, r_h, y_h) with q_h = floor((h + 2^(kh-1)) / 2^kh),
+    r_h = h - 2^kh q_h, y_h = clamp(q_h, -128, 127)."""
+    s = np.ascontiguousarray(s, dtype=np.int8)
+    u = np.ascontiguousarray(u, dtype=np.int8)
+    if s.shape != u.shape:
+        raise ValueError("ffn_hidden: s and u differ in shape")
+    q = np.zeros(s.shape, np.int32)
+    r = np.zeros(s.shape, np.int32)
+    y = np.zeros(s.shape, np.int8)
+    if lib().orc_ffn_hidden(_ptr(s), _ptr(u), s.size, kh, _ptr(q), _ptr(r), _ptr(y)) != 0:
+        raise ValueError(f"ffn_hidden: kh = {kh} outside [1, 16]")
+    return q, r, y
+
+
+def _ffn_inputs(wits, ig, iu, kh, s16, hidden):
+    s = np.ascontiguousarray(silu_outputs(wits[ig][2]) if s16 is None else s16, dtype=np.int16)
+    if hidden is None:
+        if s.min(initial=0) < -128 or s.max(initial=0) > 127:
+            raise ValueError("SiLU outputs do not fit 8 bits")
+        hidden = ffn_hidden(s.astype(np.int8), wits[iu][2], kh)
+    return s, [np.ascontiguousarray(a, dtype=t) for a, t in zip(hidden, (np.int32, np.int32, np.int8))]
+
+
+def prove_ffn(seed: int, sites, wits, ig: int = 0, iu: int = 1, idn: int = 2, kh: int = 7, s16=None,
+              hidden=None):
+    """The FFN statement (orc_prove_ffn): gate = sites[ig], up = sites[iu], down = sites[idn] (its X
+    the rescaled hidden activations); s16 defaults to the honest SiLU outputs of the gate's y and
+    hidden = (q_h, r_h, y_h) to ffn_hidden of those and the up outputs. Returns (proof bytes,
+    transcript state after)."""
     L = lib()
     keep = []
     cs, cw = _marshal(sites, wits, keep)
-    s = np.ascontiguousarray(silu_outputs(wits[ig][2]) if s16 is None else s16, dtype=np.int16)
+    s, (qh, rh, yh) = _ffn_inputs(wits, ig, iu, kh, s16, hidden)
     n = C.c_uint64(0)
     st = C.create_string_buffer(32)
-    rc = L.orc_prove_ffn(seed, cs, len(sites), cw, ig, iu, _ptr(s), None, 0, C.byref(n), st)
+    args = (seed, cs, len(sites), cw, ig, iu, idn, kh, _ptr(s), _ptr(qh), _ptr(rh), _ptr(yh))
+    rc = L.orc_prove_ffn(*args, None, 0, C.byref(n), st)
     if rc not in (0, -2):
         raise ValueError(f"orc_prove_ffn rejected the statement ({rc})")
     buf = np.zeros(max(1, n.value), dtype=np.uint8)
-    rc = L.orc_prove_ffn(seed, cs, len(sites), cw, ig, iu, _ptr(s), _ptr(buf), n.value, C.byref(n), st)
+    rc = L.orc_prove_ffn(*args, _ptr(buf), n.value, C.byref(n), st)
     if rc != 0:
         raise ValueError(f"orc_prove_ffn failed ({rc})")
     return buf[: n.value].tobytes(), st.raw
 
 
-def verify_ffn(seed: int, sites, wits, proof: bytes, ig: int = 0, iu: int = 1, s16=None):
+def verify_ffn(seed: int, sites, wits, proof: bytes, ig: int = 0, iu: int = 1, idn: int = 2, kh: int = 7,
+               s16=None, hidden=None):
     """Returns (reason_name, detail); 'accept' for a valid proof."""
     L = lib()
     keep = []
     cs, cw = _marshal(sites, wits, keep)
-    s = np.ascontiguousarray(silu_outputs(wits[ig][2]) if s16 is None else s16, dtype=np.int16)
+    s, (qh, rh, yh) = _ffn_inputs(wits, ig, iu, kh, s16, hidden)
     pb = np.frombuffer(proof, dtype=np.uint8).copy() if len(proof) else np.zeros(1, np.uint8)
     det = np.zeros(2, dtype=np.int64)
-    rc = L.orc_verify_ffn(seed, cs, len(sites), cw, ig, iu, _ptr(s), _ptr(pb), len(proof), _ptr(det))
+    rc = L.orc_verify_ffn(seed, cs, len(sites), cw, ig, iu, idn, kh, _ptr(s), _ptr(qh), _ptr(rh), _ptr(yh),
+                          _ptr(pb), len(proof), _ptr(det))
     return REASONS.get(rc, str(rc)), (int(det[0]), int(det[1]))

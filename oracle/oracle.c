@@ -1325,6 +1325,14 @@ static u64* had_lift(const int8_t* a, u64 n, int v) {
     return out;
 }
 
+/* The point z and claim c of the last gated product verified; the FFN statement checks c
+ * against the rescaled product it commits. (The oracle is single-threaded.) */
+static struct {
+    int v;
+    u64 z[MM_PT_MAX];
+    u64 c;
+} g_had_pt;
+
 /* Proof into proof[0..cap); *len = bytes needed. Returns 0, -1 on bad input,
  * -2 if cap is too small. tx is an orc_tx_new handle, advanced in place. */
 int orc_had_prove(void* txh, const int8_t* s, const int8_t* u, u64 n, uint8_t* proof, u64 cap, u64* len) {
@@ -1373,6 +1381,9 @@ int orc_had_verify(void* txh, const int8_t* s, const int8_t* u, u64 n, const uin
     u64 c, claim;
     rd_fe(t, &rd, "had_claim", &c, 1);
     if (rd.bad) FAIL(REJ_FORMAT, 0, 0);
+    g_had_pt.v = v;
+    for (int i = 0; i < v && i < MM_PT_MAX; i++) g_had_pt.z[i] = z[i];
+    g_had_pt.c = c;
     {
         u64* P = (u64*)malloc(sz * sizeof(u64));
         for (u64 x = 0; x < sz; x++) P[x] = orc_fmul(S[x], U[x]);
@@ -3834,19 +3845,49 @@ done:
 /*    the last vK_s round challenges); the matmul's A_s(rho) is that value    */
 /*    times prod_{j < n - vK_s} (1 - rho_j), since the padded columns of a    */
 /*    narrower site are zero;                                                 */
+/*  - the hidden activations: h = s u (s the SiLU outputs, u the up          */
+/*    projection's outputs) is 16-bit while the down projection reads 8-bit   */
+/*    activations, so h is rescaled as a matmul output is (3.1's rescale):    */
+/*    q_h = floor((h + 2^(kh-1)) / 2^kh), r_h = h - 2^kh q_h,                 */
+/*    y_h = clamp(q_h, -128, 127), and y_h is the down site's X. The          */
+/*    statement absorbs "ffn_hidden" D(q_h) || D(r_h) || D(y_h) and runs a    */
+/*    second lookup section (the layer proof's, over the keys (r_h, q_h, y_h) */
+/*    with remainder table R_kh) proving r_h in R_kh and y_h = clamp(q_h);    */
 /*  - the SiLU lookup with g the gate projection's committed outputs y (as    */
 /*    16-bit inputs) and s its committed 16-bit outputs;                      */
 /*  - the gated product of s (as 8-bit values: SiLU of an 8-bit input lies in */
-/*    [-48, 79]) with the up projection's committed outputs.                  */
-/* The product h = s u is 16-bit and the down projection reads 8-bit          */
-/* activations, so h is not linked to the down site here.                     */
+/*    [-48, 79]) with the up projection's committed outputs, whose claim      */
+/*    c = h~(z) the verifier ties to the committed rescale:                   */
+/*    c = 2^kh q_h~(z) + r_h~(z). With r_h in R_kh this fixes q_h as the      */
+/*    rounded quotient of h, so the down projection's input is the layer's    */
+/*    own hidden activation.                                                  */
 /* ------------------------------------------------------------------------ */
 
-enum { REJ_FFN_LINK = 49 /* a scale reduction's claim is not the weight value the matmul section left (detail: site) */ };
+enum {
+    REJ_FFN_LINK = 49,   /* a scale reduction's claim is not the weight value the matmul section left (detail: site) */
+    REJ_FFN_HIDDEN = 50, /* the gated product's claim is not 2^kh q_h~(z) + r_h~(z) */
+    REJ_FFN_DOWN = 51    /* the down site's committed X is not y_h */
+};
 
-static int ffn_args_ok(const orc_site* sites, int ns, int ig, int iu) {
-    if (ig < 0 || iu < 0 || ig >= ns || iu >= ns || ig == iu) return 0;
-    return sites[ig].M == sites[iu].M && sites[ig].N == sites[iu].N;
+static int ffn_args_ok(const orc_site* sites, int ns, int ig, int iu, int idn, int kh) {
+    if (ig < 0 || iu < 0 || idn < 0 || ig >= ns || iu >= ns || idn >= ns) return 0;
+    if (ig == iu || idn == ig || idn == iu || kh < 1 || kh > 16) return 0;
+    return sites[ig].M == sites[iu].M && sites[ig].N == sites[iu].N && sites[idn].K == sites[ig].M &&
+           sites[idn].N == sites[ig].N;
+}
+
+/* The rescaled hidden activations of n products s_i u_i, by the rounding every site's
+ * witness uses. Returns 0, or -1 if kh is outside [1, 16]. */
+int orc_ffn_hidden(const int8_t* s, const int8_t* u, u64 n, int kh, int32_t* q, int32_t* r, int8_t* y) {
+    if (kh < 1 || kh > 16) return -1;
+    for (u64 i = 0; i < n; i++) {
+        const int64_t h = (int64_t)s[i] * (int64_t)u[i];
+        const int64_t qq = floordiv_pow2(h + ((int64_t)1 << (kh - 1)), kh);
+        q[i] = (int32_t)qq;
+        r[i] = (int32_t)(h - qq * ((int64_t)1 << kh));
+        y[i] = (int8_t)(qq < -128 ? -128 : (qq > 127 ? 127 : qq));
+    }
+    return 0;
 }
 
 /* the scale reduction's point for site s and the factor prod_{j < n - vK} (1 - rho_j) */
@@ -3878,17 +3919,46 @@ static int16_t* ffn_g16(const int8_t* y, u64 n) {
     return g;
 }
 
-/* Prover. s16: the committed SiLU outputs (gate's M x N entries, token-major like y).
- * Returns 0, -1 on bad input (including an s that does not fit 8 bits), -2 if the buffer is
- * too small (*len then holds the size needed); state: the transcript after the statement. */
-int orc_prove_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, int ig, int iu, const int16_t* s16,
-                  uint8_t* proof, u64 cap, u64* len, uint8_t state[32]) {
-    if (ns < 1 || !ffn_args_ok(sites, ns, ig, iu)) return -1;
+static void ffn_absorb_hidden(orc_tx* t, const int32_t* qh, const int32_t* rh, const int8_t* yh, u64 n) {
+    uint8_t d[96];
+    orc_tree_digest(qh, 4 * n, d);
+    orc_tree_digest(rh, 4 * n, d + 32);
+    orc_tree_digest(yh, n, d + 64);
+    orc_tx_absorb(t, "ffn_hidden", d, 96);
+}
+
+/* the hidden activations as a lookup section's single site: M x N keys, remainder table R_kh */
+static void ffn_hidden_site(const orc_site* gate, int kh, const int32_t* qh, const int32_t* rh, const int8_t* yh,
+                            orc_site* ps, orc_wit* pw) {
+    memset(ps, 0, sizeof *ps);
+    ps->M = gate->M;
+    ps->N = gate->N;
+    ps->K = 1;
+    ps->w_bits = 8;
+    ps->k_shift = kh;
+    pw->q = (int32_t*)qh;
+    pw->r = (int32_t*)rh;
+    pw->y = (int8_t*)yh;
+}
+
+static int ffn_sites_ok(const orc_site* sites, int ns) {
     for (int s = 0; s < ns; s++)
         if (sites[s].M < 1 || sites[s].N < 1 || sites[s].K < 1 || sites[s].k_shift < 1 ||
             sites[s].k_shift > 30 || (sites[s].w_bits != 4 && sites[s].w_bits != 8) ||
             sites[s].k_shift != sites[0].k_shift)
-            return -1;
+            return 0;
+    return 1;
+}
+
+/* Prover. s16: the committed SiLU outputs (gate's M x N entries, token-major like y); qh, rh,
+ * yh: the committed rescale of the hidden activations (same layout), rescaled by 2^kh; the
+ * down site sites[idn] reads yh as its X. Returns 0, -1 on bad input (including an s that
+ * does not fit 8 bits), -2 if the buffer is too small (*len then holds the size needed);
+ * state: the transcript after the statement. */
+int orc_prove_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, int ig, int iu, int idn, int kh,
+                  const int16_t* s16, const int32_t* qh, const int32_t* rh, const int8_t* yh, uint8_t* proof, u64 cap,
+                  u64* len, uint8_t state[32]) {
+    if (ns < 1 || !ffn_args_ok(sites, ns, ig, iu, idn, kh) || !ffn_sites_ok(sites, ns)) return -1;
     const u64 n = (u64)sites[ig].M * (u64)sites[ig].N;
     int8_t* s8 = ffn_s8(s16, n);
     if (!s8) return -1;
@@ -3922,6 +3992,13 @@ int orc_prove_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, i
                               &l_));
     }
     {
+        orc_site ps;
+        orc_wit pw;
+        ffn_hidden_site(&sites[ig], kh, qh, rh, yh, &ps, &pw);
+        ffn_absorb_hidden(&t, qh, rh, yh, n);
+        lu_prove(&t, &pb, &ps, 1, &pw);
+    }
+    {
         int16_t* g16 = ffn_g16(wit[ig].y, n);
         FFN_SUB(orc_silu_prove(&t, g16, s16, n, at_, room_, &l_));
         free(g16);
@@ -3937,18 +4014,16 @@ out:
 }
 
 /* Verifier of orc_prove_ffn's statement: the layer proof as orc_verify, then each chained
- * statement, with the scale reductions' claims tied to the matmul section's final values.
+ * statement, with the scale reductions' claims tied to the matmul section's final values,
+ * the down site's X to y_h and the gated product's claim to the committed rescale.
  * Returns 0 on accept or a reason code (the sub-statements' own codes for their failures). */
-int orc_verify_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, int ig, int iu, const int16_t* s16,
-                   const uint8_t* proof, u64 len, int64_t detail[2]) {
+int orc_verify_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, int ig, int iu, int idn, int kh,
+                   const int16_t* s16, const int32_t* qh, const int32_t* rh, const int8_t* yh, const uint8_t* proof,
+                   u64 len, int64_t detail[2]) {
     detail[0] = detail[1] = 0;
     g_site_mask = NULL;
     g_verify_flags = 0;
-    if (ns < 1 || !ffn_args_ok(sites, ns, ig, iu)) return REJ_ARGS;
-    for (int s = 0; s < ns; s++)
-        if (sites[s].M < 1 || sites[s].N < 1 || sites[s].K < 1 || sites[s].k_shift < 1 ||
-            sites[s].k_shift > 30 || sites[s].k_shift != sites[0].k_shift)
-            return REJ_ARGS;
+    if (ns < 1 || !ffn_args_ok(sites, ns, ig, iu, idn, kh) || !ffn_sites_ok(sites, ns)) return REJ_ARGS;
     const u64 n = (u64)sites[ig].M * (u64)sites[ig].N;
     int8_t* s8 = ffn_s8(s16, n);
     if (!s8) return REJ_ARGS;
@@ -3979,7 +4054,24 @@ int orc_verify_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, 
         pos += ls;
     }
     if (!rc) {
-        const u64 lh = 8 + 32 * (u64)orc_log2_ceil(n) + 16;
+        /* one committed tensor: the down site's X is the y_h the statement rescales */
+        uint8_t dx[32], dy[32];
+        orc_tree_digest(sites[idn].xt, n, dx);
+        orc_tree_digest(yh, n, dy);
+        if (memcmp(dx, dy, 32)) rc = REJ_FFN_DOWN;
+    }
+    if (!rc) {
+        orc_site ps;
+        orc_wit pw;
+        ffn_hidden_site(&sites[ig], kh, qh, rh, yh, &ps, &pw);
+        ffn_absorb_hidden(&t, qh, rh, yh, n);
+        prd rh_rd = {proof, len, pos, 0};
+        rc = lu_verify(&t, &rh_rd, &ps, 1, &pw, detail);
+        pos = rh_rd.pos;
+    }
+    if (!rc) {
+        const int vh = orc_log2_ceil(n);
+        const u64 lh = 8 + 32 * (u64)vh + 16;
         if (pos + lh > len) {
             rc = REJ_FORMAT;
         } else {
@@ -3988,6 +4080,21 @@ int orc_verify_ffn(u64 seed, const orc_site* sites, int ns, const orc_wit* wit, 
             rc = orc_silu_verify(&t, g16, s16, n, proof + pos, lsilu, detail);
             free(g16);
             if (!rc) rc = orc_had_verify(&t, s8, wit[iu].y, n, proof + pos + lsilu, lh, detail);
+        }
+        if (!rc) {
+            /* c = 2^kh q_h~(z) + r_h~(z) at the gated product's point */
+            const u64 sz = (u64)1 << vh;
+            u64* Q = (u64*)calloc(sz, sizeof(u64));
+            u64* R = (u64*)calloc(sz, sizeof(u64));
+            for (u64 i = 0; i < n; i++) {
+                Q[i] = orc_fint(qh[i]);
+                R[i] = orc_fint(rh[i]);
+            }
+            const u64 want = orc_fadd(orc_fmul(orc_fint((int64_t)1 << kh), orc_mle_eval(Q, sz, g_had_pt.z, vh)),
+                                      orc_mle_eval(R, sz, g_had_pt.z, vh));
+            free(Q);
+            free(R);
+            if (want != g_had_pt.c) rc = REJ_FFN_HIDDEN;
         }
     }
     free(s8);

@@ -48,6 +48,10 @@ class Site:
     # (site_index, element_offset) into that site's output *group* buffer.
     w_link: Optional[tuple] = None
     xt_link: Optional[tuple] = None
+    # An FFN's down projection reads the gated product of the SiLU of the gate site's outputs
+    # with the up site's outputs, rescaled by 2^kh: (gate_index, up_index, kh). Only a
+    # declaration: the prover computes these activations from the two outputs.
+    xt_hidden: Optional[tuple] = None
     # Sites whose outputs live inside one shared N x M buffer: (group, offset).
     out_group: Optional[tuple] = None
     stage: int = 0
@@ -140,18 +144,24 @@ def _projection(seed: int, M=4096, K=4096, N=512, k=12) -> Workload:
                     description=f"W {M}x{K} int4, X {K}x{N} int8 N(0,32), k={k}")
 
 
-def _dense_ffn(seed: int, d=4096, ffn=14336, T=4096, k=18) -> Workload:
-    """Llama-3.1-8B-shaped FFN: gate/up d->ffn, down ffn->d, int4 + per-64 int8 scales."""
+def _dense_ffn(seed: int, d=4096, ffn=14336, T=4096, k=18, chained=False, kh=7) -> Workload:
+    """Llama-3.1-8B-shaped FFN: gate/up d->ffn, down ffn->d, int4 + per-64 int8 scales.
+
+    The down projection's activations are a seeded stand-in, or with ``chained`` the layer's
+    own hidden activations (SiLU(gate) * up rescaled by 2^kh), which the FFN statement proves."""
     x = activations(_rng(seed, 100), (T, d))
-    h = activations(_rng(seed, 101), (T, ffn))  # SiLU(gate)*up output: not proven here
+    h = None if chained else activations(_rng(seed, 101), (T, ffn))
     sites = []
     for idx, (nm, M, K, xt) in enumerate([("gate", ffn, d, x), ("up", ffn, d, x), ("down", d, ffn, h)]):
         sites.append(Site(nm, M, K, T, 4, k,
                           w=int4_packed(_rng(seed, 10 * idx + 1), M, K),
                           scales=group_scales(_rng(seed, 10 * idx + 2), M, K),
                           xt=xt))
-    return Workload("dense_ffn", seed, sites,
-                    description=f"d={d} ffn={ffn} T={T} int4+scales k={k}")
+    if chained:
+        sites[2].xt_hidden = (0, 1, kh)
+        sites[2].stage = 1
+    return Workload("dense_ffn_chained" if chained else "dense_ffn", seed, sites,
+                    description=f"d={d} ffn={ffn} T={T} int4+scales k={k}" + (f" chained kh={kh}" if chained else ""))
 
 
 def _moe(seed: int, E=128, d=5120, ffn=8192, T=8192, k=12, experts=None, shared=True) -> Workload:
