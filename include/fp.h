@@ -697,6 +697,16 @@ int fp_silu_table(int32_t* out);
  * device; the kernel runs on `stream` and nothing is allocated. Returns FP_OK or FP_ERR_ARG. */
 int fp_silu_inputs(fp_ctx* ctx, const int8_t* y, int64_t n, int16_t* g, int16_t* s, int8_t* s8, void* stream);
 
+/* The FFN's hidden activations, rescaled for the down projection ("How fast can FlashProve go",
+ * 3.1: the gated product of the SiLU outputs with the up projection's outputs, brought back to
+ * 8 bits as every matmul output is): for the n device int8 SiLU outputs s and up outputs u
+ * (same token-major layout), h = s[i] u[i], q[i] = floor((h + 2^(kh-1)) / 2^kh), r[i] = h -
+ * 2^kh q[i] (device int32 each) and y[i] = clamp(q[i], -128, 127) (device int8; the down site's
+ * activations). kh in [1, 16]. All buffers are the caller's, n entries each, on ctx's device;
+ * the kernel runs on `stream` and nothing is allocated. Returns FP_OK or FP_ERR_ARG. */
+int fp_ffn_hidden(fp_ctx* ctx, const int8_t* s, const int8_t* u, int64_t n, int kh, int32_t* q, int32_t* r, int8_t* y,
+                  void* stream);
+
 /* The point where the last matmul section proven with ctx (sumcheck_prove_matmul) left its
  * sites: the row challenges r_row (v_row of them, into host r_row) and the round challenges
  * rho_1..rho_n (into host rho). A chained statement continues from it: a site's weight value

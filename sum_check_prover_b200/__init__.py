@@ -97,6 +97,7 @@ def lib():
     L.logup_prove_silu.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_silu_table.argtypes = [vp]
     L.fp_silu_inputs.argtypes = [vp, vp, C.c_int64, vp, vp, vp, vp]
+    L.fp_ffn_hidden.argtypes = [vp, vp, vp, C.c_int64, i32, vp, vp, vp, vp]
     L.sumcheck_last_point.argtypes = [vp, vp, i32, C.POINTER(i32), vp, i32, C.POINTER(i32)]
     L.logup_prove_exp.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_exp_table.argtypes = [vp]
@@ -898,6 +899,15 @@ class Context:
         self._check(self._L.fp_silu_inputs(self.h, _ptr(y), int(y.numel()), _ptr(g), _ptr(s), _ptr(s8),
                                            _stream(stream)), "fp_silu_inputs")
 
+    def ffn_hidden(self, s8, u, kh: int, q, r, y, stream=None) -> None:
+        """The FFN's hidden activations rescaled by 2^kh: h = s8 u, q = floor((h + 2^(kh-1)) /
+        2^kh), r = h - 2^kh q (int32), y = clamp(q) (int8), for the device int8 tensors s8 (SiLU
+        outputs) and u (up outputs) of one shape; the caller's device buffers of that size."""
+        if s8.numel() != u.numel() or q.numel() != s8.numel() or r.numel() != s8.numel() or y.numel() != s8.numel():
+            raise ValueError("ffn_hidden: buffers differ in size")
+        self._check(self._L.fp_ffn_hidden(self.h, _ptr(s8), _ptr(u), int(s8.numel()), kh, _ptr(q), _ptr(r),
+                                          _ptr(y), _stream(stream)), "fp_ffn_hidden")
+
     def last_point(self):
         """(r_row, rho) of the last matmul section proven with this context (host integers)."""
         vr, n = C.c_int32(0), C.c_int32(0)
@@ -1043,38 +1053,64 @@ def _log2c(x: int) -> int:
 
 
 def prove_ffn(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], gate: int = 0, up: int = 1,
-              stream=None):
+              down: int = 2, kh: int = 7, stream=None):
     """Prove an FFN layer ("How fast can FlashProve go", 3.1) as one statement on one
-    transcript: the layer proof of prove(); the per-group scale reduction of every site with
-    scales, at the point where the matmul section left its weights (r_row's first ceil(log2 M)
-    coordinates, the last ceil(log2 K) round challenges); the SiLU lookup with the gate site's
-    outputs as its inputs; the gated product of the SiLU outputs with the up site's outputs.
-    gate and up index the sites in stage order. Returns (proof bytes, transcript state after,
-    lookup status)."""
+    transcript: the layer proof of prove(), its down site reading the layer's own hidden
+    activations; the per-group scale reduction of every site with scales, at the point where
+    the matmul section left its weights (r_row's first ceil(log2 M) coordinates, the last
+    ceil(log2 K) round challenges); the commitment of the hidden rescale (q_h, r_h, y_h of
+    SiLU(gate) * up by 2^kh) and its lookup section (r_h in R_kh, y_h = clamp(q_h)); the SiLU
+    lookup with the gate site's outputs as its inputs; the gated product of the SiLU outputs
+    with the up site's outputs. gate, up and down index the sites in stage order; the down
+    site sits in a later stage than gate and up, and its xt buffer (N x M_gate int8) receives
+    y_h before its stage is committed. Returns (proof bytes, transcript state after, lookup
+    status)."""
     import torch
+    sites = [s for st in stages for s in st]
+    g_site, u_site, d_site = sites[gate], sites[up], sites[down]
+    if (g_site.M, g_site.N) != (u_site.M, u_site.N):
+        raise ValueError("prove_ffn: the gate and up sites differ in shape")
+    if (d_site.K, d_site.N) != (g_site.M, g_site.N) or d_site.xt.numel() != g_site.M * g_site.N:
+        raise ValueError("prove_ffn: the down site does not read the gate's M x N outputs")
+    stage_of = {id(s): i for i, st in enumerate(stages) for s in st}
+    if stage_of[id(d_site)] <= max(stage_of[id(g_site)], stage_of[id(u_site)]):
+        raise ValueError("prove_ffn: the down site must sit in a later stage than gate and up")
+    y = g_site.y
+    dev = y.device
+    g = torch.empty(y.shape, dtype=torch.int16, device=dev)
+    s = torch.empty(y.shape, dtype=torch.int16, device=dev)
+    s8 = torch.empty(y.shape, dtype=torch.int8, device=dev)
+    qh = torch.empty(y.shape, dtype=torch.int32, device=dev)
+    rh = torch.empty(y.shape, dtype=torch.int32, device=dev)
+    yh = d_site.xt
+    n = y.numel()
     tx = Transcript(seed)
     try:
-        for st in stages:
+        hidden = False
+        for i, st in enumerate(stages):
+            if not hidden and i == stage_of[id(d_site)]:
+                ctx.silu_inputs(y, g, s, s8, stream)
+                ctx.ffn_hidden(s8, u_site.y, kh, qh, rh, yh, stream)
+                hidden = True
             ctx.commit_witness(tx, st, stream)
-        sites = [s for st in stages for s in st]
         parts = [ctx.prove_matmul(tx, sites, stream)]
         lu, status = ctx.prove_logup(tx, sites, stream)
         parts.append(lu)
         r_row, rho = ctx.last_point()
-        n = len(rho)
+        nr = len(rho)
         for d in sites:
             if d.scales is None:
                 continue
             vm, vk = _log2c(d.M), _log2c(d.K)
-            parts.append(ctx.reduce_scales(tx, d.w, d.w_bits, d.scales, d.M, d.K, r_row[:vm] + rho[n - vk:], stream))
-        g_site, u_site = sites[gate], sites[up]
-        if (g_site.M, g_site.N) != (u_site.M, u_site.N):
-            raise ValueError("prove_ffn: the gate and up sites differ in shape")
-        y = g_site.y
-        g = torch.empty(y.shape, dtype=torch.int16, device=y.device)
-        s = torch.empty(y.shape, dtype=torch.int16, device=y.device)
-        s8 = torch.empty(y.shape, dtype=torch.int8, device=y.device)
-        ctx.silu_inputs(y, g, s, s8, stream)
+            parts.append(ctx.reduce_scales(tx, d.w, d.w_bits, d.scales, d.M, d.K, r_row[:vm] + rho[nr - vk:], stream))
+        tx.absorb("ffn_hidden", ctx.digest(qh, 4 * n, stream) + ctx.digest(rh, 4 * n, stream)
+                  + ctx.digest(yh, n, stream))
+        # the hidden rescale's keys as a lookup section's single site (M x N keys, table R_kh);
+        # w and xt only satisfy the site checks, the lookup reads q, r and y
+        hs = SiteDesc(w=s8, scales=None, xt=u_site.y, q=qh, r=rh, y=yh, M=g_site.M, K=1, N=g_site.N,
+                      w_bits=8, k_shift=kh)
+        lu_h, _ = ctx.prove_logup(tx, [hs], stream)
+        parts.append(lu_h)
         parts.append(ctx.prove_silu(tx, g, s, stream))
         parts.append(ctx.prove_hadamard(tx, s8, u_site.y, stream))
         return b"".join(parts), tx.state(), status

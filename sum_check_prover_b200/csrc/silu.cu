@@ -495,7 +495,64 @@ __global__ void silu_inputs_kernel(const int8_t* __restrict__ y, int64_t n, Silu
     }
 }
 
+// The FFN's hidden activations h = s u rescaled by 2^kh (round half up, as every site's
+// witness): q = floor((h + 2^(kh-1)) / 2^kh) (an arithmetic shift), r = h - 2^kh q,
+// y = clamp(q, -128, 127). Sixteen entries per thread step from 16-byte loads when every
+// buffer is 16-byte aligned; the rest entry by entry.
+__device__ __forceinline__ void hidden_one(int sv, int uv, int kh, int32_t& q, int32_t& r, int8_t& y) {
+    const int h = sv * uv;
+    const int qq = (h + (1 << (kh - 1))) >> kh;
+    q = qq;
+    r = h - qq * (1 << kh);
+    y = (int8_t)(qq < -128 ? -128 : (qq > 127 ? 127 : qq));
+}
+
+__global__ void ffn_hidden_kernel(const int8_t* __restrict__ s, const int8_t* __restrict__ u, int64_t n, int kh,
+                                  int32_t* __restrict__ q, int32_t* __restrict__ r, int8_t* __restrict__ y,
+                                  bool vec) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t done = 0;
+    if (vec) {
+        const int64_t n16 = n / 16;
+        for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n16; j += stride) {
+            const int4 sv = reinterpret_cast<const int4*>(s)[j];
+            const int4 uv = reinterpret_cast<const int4*>(u)[j];
+            const int8_t* sb = reinterpret_cast<const int8_t*>(&sv);
+            const int8_t* ub = reinterpret_cast<const int8_t*>(&uv);
+            int4 qv[4], rv[4], yv;
+            int32_t* qo = reinterpret_cast<int32_t*>(qv);
+            int32_t* ro = reinterpret_cast<int32_t*>(rv);
+            int8_t* yo = reinterpret_cast<int8_t*>(&yv);
+#pragma unroll
+            for (int e = 0; e < 16; e++) hidden_one(sb[e], ub[e], kh, qo[e], ro[e], yo[e]);
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                reinterpret_cast<int4*>(q)[4 * j + w] = qv[w];
+                reinterpret_cast<int4*>(r)[4 * j + w] = rv[w];
+            }
+            reinterpret_cast<int4*>(y)[j] = yv;
+        }
+        done = n16 * 16;
+    }
+    for (int64_t i = done + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        hidden_one(s[i], u[i], kh, q[i], r[i], y[i]);
+}
+
 }  // namespace
+
+int fp_ffn_hidden(fp_ctx* c, const int8_t* s, const int8_t* u, int64_t n, int kh, int32_t* q, int32_t* r, int8_t* y,
+                  void* stream) {
+    if (!c || !s || !u || !q || !r || !y || n < 1) return fp_fail(c, FP_ERR_ARG, "fp_ffn_hidden: bad argument");
+    if (kh < 1 || kh > 16) return fp_fail(c, FP_ERR_ARG, "fp_ffn_hidden: kh outside [1, 16]");
+    FP_CUDA(c, cudaSetDevice(c->device));
+    cudaStream_t st = (cudaStream_t)stream;
+    const bool vec = ((uintptr_t)s | (uintptr_t)u | (uintptr_t)q | (uintptr_t)r | (uintptr_t)y) % 16 == 0;
+    const int64_t items = vec ? std::max<int64_t>(n / 16, 1) : n;
+    const unsigned grid = (unsigned)std::min<int64_t>((items + 255) / 256, 8ll * c->num_sms);
+    ffn_hidden_kernel<<<grid, 256, 0, st>>>(s, u, n, kh, q, r, y, vec);
+    FP_CUDA(c, cudaGetLastError());
+    return FP_OK;
+}
 
 int fp_silu_inputs(fp_ctx* c, const int8_t* y, int64_t n, int16_t* g, int16_t* s, int8_t* s8, void* stream) {
     if (!c || !y || !g || !s || !s8 || n < 1) return fp_fail(c, FP_ERR_ARG, "fp_silu_inputs: bad argument");

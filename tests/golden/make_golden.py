@@ -32,11 +32,13 @@ def witness_digest(wits) -> str:
 
 
 def ffn(cfg: int, data: dict):
-    """The FFN statement (oracle.prove_ffn: the layer proof continued by the scale reductions,
-    the SiLU lookup of the gate outputs and the gated product with the up outputs)."""
+    """The FFN statement (oracle.prove_ffn: the layer proof of the chained FFN, whose down site
+    reads the layer's own hidden activations, continued by the scale reductions, the hidden
+    rescale's lookup, the SiLU lookup of the gate outputs and the gated product with the up
+    outputs)."""
     seed = 0
     t0 = time.time()
-    wl = workloads.build(cfg, seed=seed)
+    wl = workloads.build(cfg, seed=seed, chained=True)
     R = oracle.resolve(wl)
     t1 = time.time()
     proof, state = oracle.prove_ffn(seed, R.sites, R.wits)

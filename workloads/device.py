@@ -2,7 +2,8 @@
 
 Pointer wiring only: uploads the seeded host arrays, allocates the witness
 buffers (q, r, y; N x M token-major), places grouped outputs inside their
-shared buffer, and makes a linked operand a view of the output it reads. No
+shared buffer, makes a linked operand a view of the output it reads, and gives
+an FFN's down site an empty activation buffer for the prover to fill. No
 arithmetic of the proving method lives here.
 """
 
@@ -88,6 +89,9 @@ def upload(wl, device: str = "cuda"):
         if s.xt_link is not None:
             src, off = s.xt_link
             xt = y_buffer(src)[off:off + s.N * s.K].view(s.N, s.K)
+        elif s.xt_hidden is not None:
+            # an FFN's hidden activations: fp.prove_ffn writes them before this stage is committed
+            xt = torch.zeros((s.N, s.K), dtype=torch.int8, device=dev)
         else:
             xt = t(s.xt)
         sc = t(s.scales) if s.scales is not None else None
