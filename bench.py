@@ -205,7 +205,7 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi, every 200 ms"}
 
 
-MICRO_ALL = "sc,pe,gkr,lhr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2,silu2,lu2"
+MICRO_ALL = "sc,pe,gkr,lhr,gemm,had,scl,silu,had2,lhi,mm2,frv,lhi2,silu2,lu2,ffn"
 
 
 def micro_names(which) -> set:
@@ -250,6 +250,11 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
       (16-byte vectors: 160 and 320 B per pair).
     lu2_round: the rescale LogUp's layer rounds over 2^26 keys with extension challenges,
       both tables in one launch (288 and 576 B per pair).
+    ffn: the FFN layer statement (fp.prove_ffn) over the Llama-3.1-8B-shaped FFN (d 4096,
+      ffn 14336, 4096 tokens, int4 weights with per-64 scales, k 18) with the down projection
+      reading the layer's own hidden activations: device time per statement (CUDA events
+      around the call, inputs resident), the per-kernel split from a profiled pass, and the
+      hidden-rescale kernel against the copy bandwidth.
     witness_gemm: one 14336 x 4096 int4 by 4096 x 4096 int8 product with its rescale
       epilogue (a Llama-3.1-8B FFN projection), against the tensor peak; and the witness
       launches of a 16-expert MoE layer (about 64 tokens per expert, the shared expert over
@@ -470,6 +475,42 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
             del st, keep
         except Exception as e:  # a failure here must not cost the rest of the line
             out["rescale_logup_ext2_round_2^26_keys"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+
+    if "ffn" in which:
+        try:
+            wl = workloads.build(3, 0, chained=True)
+            st, keep = device.upload(wl, dev)
+            device.weight_digests(ctx, st)
+            fp.prove_ffn(ctx, 0, st)  # warm: arena growth and module loading
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(3):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                proof, _, _ = fp.prove_ffn(ctx, 0, st)
+                b.record()
+                torch.cuda.synchronize()
+                times.append(a.elapsed_time(b))
+            ctx.set_profiling(True)
+            fp.prove_ffn(ctx, 0, st)
+            torch.cuda.synchronize()
+            ks = ctx.kernel_stats()
+            ctx.set_profiling(False)
+            macs = sum(x.macs for x in wl.sites)
+            ms = statistics.median(times)
+            top = sorted(ks.items(), key=lambda kv: -kv[1][1])[:12]
+            n_h, ms_h, by_h = ks.get("ffn_hidden", (0, 0.0, 0.0))
+            gbs_h = by_h / (ms_h * 1e-3) / 1e9 if ms_h > 0 else 0.0
+            out["ffn_statement_d4096_ffn14336_T4096"] = {
+                "ms": ms, "ms_all": times, "MACs": macs, "MACps": macs / (ms * 1e-3),
+                "keys": sum(x.M * x.N for x in wl.sites) + wl.sites[0].M * wl.sites[0].N,
+                "proof_bytes": len(proof),
+                "kernels_profiled_ms": {k: round(v[1], 3) for k, v in top},
+                "ffn_hidden": {"launches": n_h, "ms": ms_h, "bytes": by_h, "GBps": gbs_h,
+                               "frac": gbs_h / pk["hbm_gbs"], "peak": pk["hbm_gbs"]}}
+            del st, keep, wl
+        except Exception as e:  # a failure here must not cost the rest of the line
+            out["ffn_statement_d4096_ffn14336_T4096"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     try:
         torch.cuda.empty_cache()

@@ -71,6 +71,8 @@ enum FpKernel {
     K_LHR_FINAL,
     K_DSP_CLAIM,
     K_DSP_VECTORS,
+    K_SILU_INPUTS,
+    K_FFN_HIDDEN,
     K_COUNT
 };
 

@@ -26,6 +26,7 @@
 #include <vector>
 
 #include "fp_eqchunks.cuh"
+#include "fp_hist.cuh"
 #include "fp_internal.h"
 #include "fp_reduce.cuh"
 #include "fp_session.cuh"
@@ -211,6 +212,76 @@ __global__ void __launch_bounds__(1024) hist_kernel(KeySrc K, int k, int64_t L, 
         atomicAdd(&m_clamp[32768], pad);
     }
 }
+
+// The same counts for remainder tables of 2^15 to 2^18 rows, too large for one block: a cluster
+// of 2^(k-15) CTAs holds the table in distributed shared memory, 2^15 rows per CTA (each
+// remainder counted on its owner's shared memory), next to a clamp window [-2^12, 2^12) of its
+// own. Every cluster writes its remainder rows to part (row = cluster index, 2^k words) with
+// plain stores; hist_rows_sum_kernel adds the rows (and the padding keys) into m_rem.
+constexpr int HIST_CL_WIN = 1 << 12;
+
+__global__ void __launch_bounds__(1024) hist_cluster_kernel(KeySrc K, int k, int64_t L, uint32_t* __restrict__ part,
+                                                            uint32_t* __restrict__ m_clamp,
+                                                            uint32_t* __restrict__ outside) {
+    extern __shared__ uint32_t sh[];
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    constexpr int SB = fp_hist::kShareBits;
+    const unsigned crank = cl.block_rank(), csize = cl.num_blocks();
+    uint32_t* sr = sh;               // remainder rows [crank 2^15, (crank + 1) 2^15)
+    uint32_t* sq = sh + (1 << SB);   // 2 HIST_CL_WIN clamp rows around q = 0
+    const int64_t T = 1ll << k;
+    const int32_t half = 1 << (k - 1);
+    for (int i = threadIdx.x; i < (1 << SB); i += blockDim.x) sr[i] = 0;
+    for (int i = threadIdx.x; i < 2 * HIST_CL_WIN; i += blockDim.x) sq[i] = 0;
+    cl.sync();  // every CTA's rows are zero before any CTA counts into them
+    uint32_t out_local = 0;
+    auto count = [&](int32_t rv, int32_t qv, int32_t yv) {
+        const int64_t jr = (int64_t)rv + half;
+        if (jr >= 0 && jr < T)
+            atomicAdd(cl.map_shared_rank(sr, (unsigned)(jr >> SB)) + (jr & ((1 << SB) - 1)), 1u);
+        else
+            out_local++;
+        const int64_t q = qv;
+        if (q >= -HIST_CL_WIN && q < HIST_CL_WIN)
+            atomicAdd(&sq[q + HIST_CL_WIN], 1u);
+        else if (q >= -32768 && q < 32768)
+            atomicAdd(&m_clamp[q + 32768], 1u);
+        else
+            out_local++;
+        if (yv != (q < -128 ? -128 : (q > 127 ? 127 : (int32_t)q))) out_local++;
+    };
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t done = 0;
+    if (((uintptr_t)K.r | (uintptr_t)K.q) % 16 == 0 && (uintptr_t)K.y % 4 == 0) {
+        const int64_t ng = K.n / 4;
+        const int4* r4 = reinterpret_cast<const int4*>(K.r);
+        const int4* q4 = reinterpret_cast<const int4*>(K.q);
+        const uint32_t* y4 = reinterpret_cast<const uint32_t*>(K.y);
+        for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < ng; g += stride) {
+            const int4 ra = __ldcs(r4 + g), qa = __ldcs(q4 + g);
+            const uint32_t ya = __ldcs(y4 + g);
+            count(ra.x, qa.x, (int8_t)(ya & 0xFF));
+            count(ra.y, qa.y, (int8_t)((ya >> 8) & 0xFF));
+            count(ra.z, qa.z, (int8_t)((ya >> 16) & 0xFF));
+            count(ra.w, qa.w, (int8_t)(ya >> 24));
+        }
+        done = 4 * ng;
+    }
+    for (int64_t i = done + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < K.n; i += stride)
+        count(K.r[i], K.q[i], (int32_t)K.y[i]);
+    if (out_local) atomicAdd(outside, out_local);
+    cl.sync();  // every count has landed; no CTA leaves while another may still count into it
+    uint32_t* row = part + (size_t)(blockIdx.x / csize) * (size_t)T + ((size_t)crank << SB);
+    for (int i = threadIdx.x; i < (1 << SB); i += blockDim.x) row[i] = sr[i];
+    for (int i = threadIdx.x; i < 2 * HIST_CL_WIN; i += blockDim.x)
+        if (sq[i]) atomicAdd(&m_clamp[i - HIST_CL_WIN + 32768], sq[i]);
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&m_clamp[32768], (uint32_t)(L - K.n));
+}
+
+// remainder tables counted by hist_cluster_kernel, and the partial rows they may write (one
+// per cluster; at most one cluster per SM)
+constexpr int kHistClMinK = 15, kHistClMaxK = 18, kHistClMaxRows = 160;
 
 // ---- key gather (several sites) ---------------------------------------------
 
@@ -1177,7 +1248,11 @@ int fp_lookup_keys(fp_ctx* c, const fp_site* sites, int nsites, cudaStream_t st,
     return FP_OK;
 }
 
-size_t fp_lookup_mults_scratch(int k) { return fp_align_up(4 * ((size_t)1 << k), 256) + fp_align_up(4 * 65536, 256) + 256; }
+size_t fp_lookup_mults_scratch(int k) {
+    size_t b = fp_align_up(4 * ((size_t)1 << k), 256) + fp_align_up(4 * 65536, 256) + 256;
+    if (k >= kHistClMinK && k <= kHistClMaxK) b += fp_align_up((size_t)4 * (kHistClMaxRows << fp_hist::kShareBits), 256);
+    return b;
+}
 
 int fp_lookup_mults(fp_ctx* c, const FpKeyCols& K, int k, int64_t L, cudaStream_t st, uint8_t* hm, uint8_t dg_rem[32],
                     uint8_t dg_cl[32]) {
@@ -1190,7 +1265,29 @@ int fp_lookup_mults(fp_ctx* c, const FpKeyCols& K, int k, int64_t L, cudaStream_
     FP_CUDA(c, cudaMemsetAsync(m_rem, 0, 4 * (size_t)T, st));
     FP_CUDA(c, cudaMemsetAsync(m_cl, 0, 4 * 65536, st));
     FP_CUDA(c, cudaMemsetAsync(outside, 0, 4, st));
-    {
+    bool counted = false;
+    if (k >= kHistClMinK && k <= kHistClMaxK) {
+        // the remainder table over a cluster's shared memory (2^(k-15) CTAs of 2^15 rows)
+        const int csize = 1 << (k - fp_hist::kShareBits);
+        const size_t rows_bytes = (size_t)4 * (kHistClMaxRows << fp_hist::kShareBits);
+        uint32_t* part = (uint32_t*)fp_alloc(c->dev, rows_bytes);
+        if (!part) return fp_fail(c, FP_ERR_OOM, "lookup multiplicities: scratch exhausted");
+        const int smem = 4 * ((1 << fp_hist::kShareBits) + 2 * HIST_CL_WIN);
+        int clusters = 0, slot;
+        fp_tic(c, st, K_HIST, 9.0 * K.n, &slot);
+        if (fp_hist::launch_clusters(hist_cluster_kernel, csize, smem, kHistClMaxRows / csize, st, &clusters, K, k, L,
+                                     part, m_cl, outside) == cudaSuccess) {
+            fp_hist::hist_rows_sum_kernel<<<fp_grid256(c, T), 256, 0, st>>>(part, clusters, T, m_rem, T / 2,
+                                                                            (uint32_t)(L - K.n));
+            c->launches++;
+            counted = true;
+        } else {
+            (void)cudaGetLastError();  // no cluster of that size fits here: the global-atomic path below
+        }
+        fp_toc(c, st, slot);
+        FP_CUDA(c, cudaGetLastError());
+    }
+    if (!counted) {
         const int rem_smem = T <= 16384;
         const int smem = 4 * (2 * HIST_WIN) + (rem_smem ? 4 * (int)T : 0);
         FP_CUDA(c, cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));

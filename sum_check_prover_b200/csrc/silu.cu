@@ -24,6 +24,7 @@
 #include <vector>
 
 #include "fp_eqchunks.cuh"
+#include "fp_hist.cuh"
 #include "fp_internal.h"
 #include "fp_reduce.cuh"
 #include "fp_session.cuh"
@@ -34,14 +35,6 @@ constexpr int SL_THREADS = 256;
 constexpr int SL_MAX_V = 30;
 
 __device__ __forceinline__ uint64_t lift_i(int64_t x) { return x < 0 ? GL_P - (uint64_t)(-x) : (uint64_t)x; }
-
-// m[g + 2^15] += 1 for every entry of g (the padding keys are counted by the host)
-__global__ void silu_hist_kernel(const int16_t* __restrict__ g, int64_t n, uint32_t* __restrict__ m) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        atomicAdd(m + ((int)g[i] + 32768), 1u);
-}
-
-__global__ void silu_add_pad_kernel(uint32_t* m, uint32_t pad) { m[32768] += pad; }
 
 // leaves: P = 1, Q = alpha - (g + gamma s); past n the padding key fpad (the table's row for input 0)
 __global__ void silu_leaf_kernel(const int16_t* __restrict__ g, const int16_t* __restrict__ s, int64_t n, int64_t L,
@@ -271,11 +264,13 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
                   fp_align_up((size_t)8 << vh, 256) + fp_align_up((size_t)8 << vl, 256) +
                   5 * fp_align_up((size_t)8 * hv, 256) + 4096;
     for (int d = 1; d <= v; d++) need += 2 * fp_align_up((size_t)8 << d, 256);
+    need += fp_hist::hist16_scratch();
     if ((rc = fp_reserve(c, c->dev, need))) return rc;
     if ((rc = fp_reserve(c, c->host, 4 * 65536 + 8192))) return rc;
     fp_reset(c->dev);
     fp_reset(c->host);
     uint32_t* m = (uint32_t*)fp_alloc(c->dev, 4 * 65536);
+    uint32_t* hpart = (uint32_t*)fp_alloc(c->dev, fp_hist::hist16_scratch());
     uint64_t* part = (uint64_t*)fp_alloc(c->dev, 8 * part_n);
     uint64_t* small = (uint64_t*)fp_alloc(c->dev, 8 * 64);  // [0..1] leaf values, [8..] the layer's point
     uint64_t* EH = (uint64_t*)fp_alloc(c->dev, (size_t)8 << vh);
@@ -290,19 +285,16 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
     }
     uint8_t* hm = (uint8_t*)fp_alloc(c->host, 4 * 65536);
     uint64_t* hs = (uint64_t*)fp_alloc(c->host, 8 * 64);
-    if (!m || !part || !small || !EH || !EL || !vecs[4] || !hm || !hs)
+    if (!m || !hpart || !part || !small || !EH || !EL || !vecs[4] || !hm || !hs)
         return fp_fail(c, FP_ERR_OOM, "logup_prove_silu: scratch exhausted");
 
     // ---- multiplicities ----
-    FP_CUDA(c, cudaMemsetAsync(m, 0, 4 * 65536, st));
     {
         int slot;
         fp_tic(c, st, K_SILU_HIST, 2.0 * (double)n, &slot);
-        silu_hist_kernel<<<grid_of(c, n), 256, 0, st>>>(g, n, m);
+        rc = fp_hist::hist16(c, g, n, (uint32_t)(L - n), m, hpart, st);
         fp_toc(c, st, slot);
-        FP_CUDA(c, cudaGetLastError());
-        if (L > n) silu_add_pad_kernel<<<1, 1, 0, st>>>(m, (uint32_t)(L - n));
-        FP_CUDA(c, cudaGetLastError());
+        if (rc) return rc;
     }
     FP_CUDA(c, cudaMemcpyAsync(hm, m, 4 * 65536, cudaMemcpyDeviceToHost, st));
     uint8_t dm[32];
@@ -549,7 +541,10 @@ int fp_ffn_hidden(fp_ctx* c, const int8_t* s, const int8_t* u, int64_t n, int kh
     const bool vec = ((uintptr_t)s | (uintptr_t)u | (uintptr_t)q | (uintptr_t)r | (uintptr_t)y) % 16 == 0;
     const int64_t items = vec ? std::max<int64_t>(n / 16, 1) : n;
     const unsigned grid = (unsigned)std::min<int64_t>((items + 255) / 256, 8ll * c->num_sms);
+    int slot;
+    fp_tic(c, st, K_FFN_HIDDEN, 11.0 * (double)n, &slot);  // two int8 factors in, q and r int32 and y out
     ffn_hidden_kernel<<<grid, 256, 0, st>>>(s, u, n, kh, q, r, y, vec);
+    fp_toc(c, st, slot);
     FP_CUDA(c, cudaGetLastError());
     return FP_OK;
 }
@@ -561,7 +556,10 @@ int fp_silu_inputs(fp_ctx* c, const int8_t* y, int64_t n, int16_t* g, int16_t* s
     for (int v = -128; v < 128; v++) tab.v[v + 128] = (int16_t)silu_q_host(v);
     cudaStream_t st = (cudaStream_t)stream;
     const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 8ll * c->num_sms);
+    int slot;
+    fp_tic(c, st, K_SILU_INPUTS, 6.0 * (double)n, &slot);  // y in; g, s (int16) and s8 out
     silu_inputs_kernel<<<grid, 256, 0, st>>>(y, n, tab, g, s, s8);
+    fp_toc(c, st, slot);
     FP_CUDA(c, cudaGetLastError());
     return FP_OK;
 }

@@ -25,6 +25,7 @@
 
 #include "fp_ext2.cuh"
 #include "fp_ext2_host.h"
+#include "fp_hist.cuh"
 #include "fp_internal.h"
 #include "fp_reduce.cuh"
 #include "fp_session.cuh"
@@ -36,13 +37,6 @@ constexpr int X16_MAX_V = 30;
 constexpr int X16_CHUNK = 8;  // four eq chunk tables of at most 2^8 entries (z_2..z_d, d <= 29)
 
 __device__ __forceinline__ uint64_t x16_lift(int64_t x) { return x < 0 ? GL_P - (uint64_t)(-x) : (uint64_t)x; }
-
-__global__ void x16_hist_kernel(const int16_t* __restrict__ g, int64_t n, uint32_t* __restrict__ m) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        atomicAdd(m + ((int)g[i] + 32768), 1u);
-}
-
-__global__ void x16_add_pad_kernel(uint32_t* m, uint32_t pad) { m[32768] += pad; }
 
 // leaves: P = 1, Q = alpha - (g + gamma s); past n the padding key (0, pad_s)
 __global__ void x16_leaf_kernel(const int16_t* __restrict__ g, const int16_t* __restrict__ s, int64_t n, int64_t L,
@@ -1070,11 +1064,13 @@ int x16_prove(fp_ctx* c, fp_tx* tx, const X16Labels& lab, int64_t pad_s, const i
                   fp_align_up((size_t)16 << vh, 256) + fp_align_up((size_t)16 << vl, 256) +
                   5 * fp_align_up((size_t)16 * hv, 256) + 4096;
     for (int d = 1; d <= v; d++) need += 2 * fp_align_up((size_t)16 << d, 256);
+    need += fp_hist::hist16_scratch();
     if ((rc = fp_reserve(c, c->dev, need))) return rc;
     if ((rc = fp_reserve(c, c->host, 4 * 65536 + 8192))) return rc;
     fp_reset(c->dev);
     fp_reset(c->host);
     uint32_t* m = (uint32_t*)fp_alloc(c->dev, 4 * 65536);
+    uint32_t* hpart = (uint32_t*)fp_alloc(c->dev, fp_hist::hist16_scratch());
     dev.part = (uint64_t*)fp_alloc(c->dev, 8 * part_n);
     dev.small = (uint64_t*)fp_alloc(c->dev, 8 * 64);
     dev.EH = (Ext2*)fp_alloc(c->dev, (size_t)16 << vh);
@@ -1089,22 +1085,16 @@ int x16_prove(fp_ctx* c, fp_tx* tx, const X16Labels& lab, int64_t pad_s, const i
     }
     uint32_t* hm = (uint32_t*)fp_alloc(c->host, 4 * 65536);
     dev.hs = (uint64_t*)fp_alloc(c->host, 8 * 64);
-    if (!m || !dev.part || !dev.small || !dev.EH || !dev.EL || !dev.vecs[4] || !hm || !dev.hs)
+    if (!m || !hpart || !dev.part || !dev.small || !dev.EH || !dev.EL || !dev.vecs[4] || !hm || !dev.hs)
         return fp_fail(c, FP_ERR_OOM, std::string(who) + ": scratch exhausted");
 
     // ---- multiplicities ----
-    FP_CUDA(c, cudaMemsetAsync(m, 0, 4 * 65536, st));
     {
         int slot;
         fp_tic(c, st, K_SILU_HIST, 2.0 * (double)n, &slot);
-        x16_hist_kernel<<<fp_grid256(c, n), 256, 0, st>>>(g, n, m);
+        rc = fp_hist::hist16(c, g, n, (uint32_t)(L - n), m, hpart, st);
         fp_toc(c, st, slot);
-        FP_CUDA(c, cudaGetLastError());
-        if (L > n) {
-            x16_add_pad_kernel<<<1, 1, 0, st>>>(m, (uint32_t)(L - n));
-            FP_CUDA(c, cudaGetLastError());
-            c->launches++;
-        }
+        if (rc) return rc;
     }
     FP_CUDA(c, cudaMemcpyAsync(hm, m, 4 * 65536, cudaMemcpyDeviceToHost, st));
     uint8_t dm[32];

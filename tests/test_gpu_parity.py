@@ -147,6 +147,30 @@ def test_random_shapes_and_seeds(env, i):
     check_against_oracle(env, _random_case(i), 77 + i)
 
 
+@pytest.mark.parametrize("k", [14, 15, 16, 17, 18])
+def test_remainder_tables_over_a_cluster(env, k):
+    # k = 15..18: the remainder table is counted in the distributed shared memory of a cluster
+    # of 2^(k-15) blocks; k = 14 is the one-block table. Two sites, one unaligned in size.
+    sites = [workloads.random_site(3000 + k, 257, 513, 200, 4, k, scales=True),
+             workloads.random_site(3100 + k, 130, 160, 9, 8, k)]
+    check_against_oracle(env, workloads.Workload(f"cl{k}", 0, sites), 40 + k)
+
+
+def test_tampered_clamp_over_a_cluster_is_flagged(env):
+    torch, fp, ctx = env
+    s = workloads.random_site(3200, 64, 96, 33, 8, 16)
+    stages, keep = device.upload(workloads.Workload("t16", 0, [s]))
+    tx = fp.Transcript(0)
+    ctx.commit_witness(tx, stages[0])
+    d = stages[0][0]
+    d.y[3, 5] = (int(d.y[3, 5]) + 1) if int(d.y[3, 5]) < 127 else 126
+    torch.cuda.synchronize()
+    ctx.prove_matmul(tx, stages[0])
+    lu, status = ctx.prove_logup(tx, stages[0])
+    assert status == 1
+    tx.close()
+
+
 def test_inline_weight_digests_give_the_same_proof(env):
     wl = workloads.build(3, seed=5, small=True)
     a = run_gpu(env, wl, 5, digests=True)[0]

@@ -66,6 +66,31 @@ def test_matches_oracle(env, n):
         assert oracle.silu_verify(3, g, s, pf) == ("accept", (0, 0))
 
 
+@pytest.mark.parametrize("case", ["int8_inputs", "uniform_large", "unaligned"])
+def test_histogram_shapes(env, case):
+    # the 2^16-row multiplicities over a cluster of two blocks: keys concentrated in a few
+    # rows (a projection's int8 outputs as inputs: the window around zero), keys spread over
+    # the whole table, and an input column that does not start on a 16-byte boundary
+    torch, fp, ctx = env
+    if case == "int8_inputs":
+        g, s = _cols((1 << 20) + 3, 21, -128, 128)
+    else:
+        g, s = _cols((1 << 20) + 5 if case == "uniform_large" else 70001, 22)
+    if case == "unaligned":
+        gb = torch.zeros(len(g) + 3, dtype=torch.int16, device="cuda")
+        sb = torch.zeros(len(g) + 3, dtype=torch.int16, device="cuda")
+        gd, sd = gb[3:], sb[3:]
+        gd.copy_(torch.from_numpy(g))
+        sd.copy_(torch.from_numpy(s))
+        tx = fp.Transcript(3)
+        pf = ctx.prove_silu(tx, gd, sd)
+        torch.cuda.synchronize()
+        st = tx.state()
+    else:
+        pf, st = _gpu(env, 3, g, s)
+    assert (pf, st) == oracle.silu_prove(3, g, s)
+
+
 def test_dishonest_output_same_bytes_rejected(env):
     g, s = _cols(500, 4, -2000, 2000)
     s = s.copy()
