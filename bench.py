@@ -232,8 +232,10 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
     had_round: gated-product sum-check rounds over two 2^26-entry int8 factors
       (round 1 reads the int8 factors and writes the eq table, round 2 folds
       them into field vectors, later rounds read 4 and write 2 values of both
-      factors and fold the eq table: 120 B per pair); and the same rounds reducing a
-      14336 x 4096 int4 weight matrix with per-64 scales to claims on w and S.
+      factors and fold the eq table: 120 B per pair).
+    scale_reduction: the whole scale reduction of a 14336 x 4096 int4 weight matrix with
+      per-64 scales (CUDA events around the call), its per-kernel split, and the group
+      contraction W' (the weights read once) against the copy bandwidth.
     silu_round: the SiLU lookup's layer sum-checks over 2^26 keys (one tree; round 1
       reads the tree layer's children, later rounds fold them: 80 and 160 B per pair).
     had2_round: the gated product over 2^26 entries with challenges in the quadratic
@@ -358,8 +360,29 @@ def run_micro(fp, torch, ctx, dev: str, which: str = MICRO_ALL) -> dict:
         wv = torch.from_numpy(workloads.int4_packed(rng, M, K)).to(dev)
         sv = torch.from_numpy(workloads.group_scales(rng, M, K)).to(dev)
         pt = [int(x) for x in rng.integers(0, fp.P, size=26, dtype="uint64")]
-        measure("scale_reduction_round_14336x4096", "had_round",
-                lambda: ctx.reduce_scales(fp.Transcript(5), wv, 4, sv, M, K, pt))
+        run = lambda: ctx.reduce_scales(fp.Transcript(5), wv, 4, sv, M, K, pt)  # noqa: E731
+        run()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            run()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ctx.set_profiling(True)
+        run()
+        torch.cuda.synchronize()
+        ks = ctx.kernel_stats()
+        ctx.set_profiling(False)
+        n_g, ms_g, by_g = ks.get("scl_group", (0, 0.0, 0.0))
+        gbs = by_g / (ms_g * 1e-3) / 1e9 if ms_g > 0 else 0.0
+        out["scale_reduction_14336x4096"] = {
+            "ms": statistics.median(times), "ms_all": times,
+            "kernels_profiled_ms": {k: round(v[1], 4) for k, v in sorted(ks.items(), key=lambda kv: -kv[1][1])},
+            "scl_group": {"kernel": "scl_group", "ms": ms_g, "bytes": by_g, "GBps": gbs, "frac": gbs / pk["hbm_gbs"],
+                          "peak": pk["hbm_gbs"]}}
         del wv, sv
 
     if "gkr" in which:

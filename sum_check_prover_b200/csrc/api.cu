@@ -403,7 +403,7 @@ const char* fp_kernel_name(int k) {
         "route_witness", "route_vectors", "route_open", "route_round", "route_final",
         "lhi2_column", "lhi2_round", "lhi2_final", "silu2_tree", "silu2_round", "silu2_leaf",
         "lu2_hist", "lu2_tree", "lu2_round", "lu2_leaf", "lhr_column", "lhr_round", "lhr_final", "dsp_claim",
-        "dsp_vectors", "silu_inputs", "ffn_hidden"};
+        "dsp_vectors", "silu_inputs", "ffn_hidden", "scl_group"};
     return (k >= 0 && k < K_COUNT) ? names[k] : "?";
 }
 

@@ -73,6 +73,7 @@ enum FpKernel {
     K_DSP_VECTORS,
     K_SILU_INPUTS,
     K_FFN_HIDDEN,
+    K_SCL_GROUP,
     K_COUNT
 };
 
