@@ -79,13 +79,11 @@ __global__ void __launch_bounds__(256) silu_mle_kernel(const int16_t* __restrict
 }
 
 struct LayerArgs {
-    const uint64_t* P;  // tree layer d + 1 (2^(d+1) entries): child x of node b is entry 2 b + x
-    const uint64_t* Q;
-    uint64_t* pl;       // folded children from round 2 on (2^(d-1) entries each)
-    uint64_t* pr;
-    uint64_t* ql;
-    uint64_t* qr;
-    uint64_t* E;        // suffix eq table (2^(d-1) entries)
+    const ulonglong2* P;  // tree layer d + 1 as child pairs: (pL, pR) of node b at entry b
+    const ulonglong2* Q;  // (qL, qR)
+    ulonglong2* pp;       // the child pairs folded, from round 2 on (2^(d-1) pairs each)
+    ulonglong2* qq;
+    uint64_t* E;          // suffix eq table (2^(d-1) entries)
     const uint64_t* z;  // device copy of the layer's point z_1..z_d
     uint64_t lam;
     int d;
@@ -99,10 +97,17 @@ struct LayerArgs {
 
 __device__ __forceinline__ uint64_t at2(uint64_t a, uint64_t b) { return gl_sub(gl_add(b, b), a); }
 
-// pL qR + pR qL + lambda qL qR
-__device__ __forceinline__ uint64_t layer_f(uint64_t a, uint64_t b, uint64_t c, uint64_t e, uint64_t lam) {
-    return gl_add(gl_add(gl_mul(a, e), gl_mul(b, c)), gl_mul(lam, gl_mul(c, e)));
+// pL qR + pR qL + lambda qL qR = pL qR + qL (pR + lambda qR), weakly reduced (< 2^64, congruent)
+__device__ __forceinline__ uint64_t layer_f(ulonglong2 p, ulonglong2 q, uint64_t lam) {
+    const uint64_t u = gl_add(p.y, gl_mul_weak(lam, q.y));
+    return gl_muladd_weak(q.x, u, gl_mul_weak(p.x, q.y));
 }
+
+__device__ __forceinline__ ulonglong2 fold2(ulonglong2 a, ulonglong2 b, uint64_t r) {
+    return make_ulonglong2(gl_fold_fast(a.x, b.x, r), gl_fold_fast(a.y, b.y, r));
+}
+
+__device__ __forceinline__ ulonglong2 at2v(ulonglong2 a, ulonglong2 b) { return make_ulonglong2(at2(a.x, b.x), at2(a.y, b.y)); }
 
 __global__ void __launch_bounds__(SL_THREADS, 2) silu_layer_kernel(LayerArgs A, FpMailbox* mb, FpRelay* rl,
                                                                   uint64_t* part) {
@@ -119,55 +124,37 @@ __global__ void __launch_bounds__(SL_THREADS, 2) silu_layer_kernel(LayerArgs A, 
         if (blockIdx.x >= active) return;  // no pairs for this block in this or any later round
         EqChunks EC{0, 0, 0};
         if (t == 1) EC = eq_chunks_build(eq_tab, zs, A.d);
+        // h(1) only where the host cannot take it from the running claim (z_t = 0)
+        const bool need1 = zs[t - 1] == 0;
         GlAcc a0, a1, a2;
         for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
-            uint64_t p0, p1, r0, r1, q0, q1, s0, s1, e;  // pL, pR, qL, qR at the pair's two points
+            ulonglong2 p0, p1, q0, q1;  // (pL, pR), (qL, qR) at the pair's two points
+            uint64_t e;
             if (t == 1) {
-                p0 = A.P[2 * b];
-                r0 = A.P[2 * b + 1];
-                q0 = A.Q[2 * b];
-                s0 = A.Q[2 * b + 1];
-                p1 = A.P[2 * (b + h)];
-                r1 = A.P[2 * (b + h) + 1];
-                q1 = A.Q[2 * (b + h)];
-                s1 = A.Q[2 * (b + h) + 1];
+                p0 = __ldcg(A.P + b);
+                q0 = __ldcg(A.Q + b);
+                p1 = __ldcg(A.P + b + h);
+                q1 = __ldcg(A.Q + b + h);
                 e = eq_chunks_at(EC, eq_tab, b);  // eq(z_2..z_d, b)
                 if (A.d > 1) A.E[b] = e;
             } else {
-                if (t == 2) {
-                    // the children vectors (length 4h, read from the tree layer) folded by rho_1
-                    p0 = gl_fold_fast(A.P[2 * b], A.P[2 * (b + 2 * h)], rprev);
-                    r0 = gl_fold_fast(A.P[2 * b + 1], A.P[2 * (b + 2 * h) + 1], rprev);
-                    q0 = gl_fold_fast(A.Q[2 * b], A.Q[2 * (b + 2 * h)], rprev);
-                    s0 = gl_fold_fast(A.Q[2 * b + 1], A.Q[2 * (b + 2 * h) + 1], rprev);
-                    p1 = gl_fold_fast(A.P[2 * (b + h)], A.P[2 * (b + 3 * h)], rprev);
-                    r1 = gl_fold_fast(A.P[2 * (b + h) + 1], A.P[2 * (b + 3 * h) + 1], rprev);
-                    q1 = gl_fold_fast(A.Q[2 * (b + h)], A.Q[2 * (b + 3 * h)], rprev);
-                    s1 = gl_fold_fast(A.Q[2 * (b + h) + 1], A.Q[2 * (b + 3 * h) + 1], rprev);
-                } else {
-                    p0 = gl_fold_fast(__ldcg(A.pl + b), __ldcg(A.pl + b + 2 * h), rprev);
-                    r0 = gl_fold_fast(__ldcg(A.pr + b), __ldcg(A.pr + b + 2 * h), rprev);
-                    q0 = gl_fold_fast(__ldcg(A.ql + b), __ldcg(A.ql + b + 2 * h), rprev);
-                    s0 = gl_fold_fast(__ldcg(A.qr + b), __ldcg(A.qr + b + 2 * h), rprev);
-                    p1 = gl_fold_fast(__ldcg(A.pl + b + h), __ldcg(A.pl + b + 3 * h), rprev);
-                    r1 = gl_fold_fast(__ldcg(A.pr + b + h), __ldcg(A.pr + b + 3 * h), rprev);
-                    q1 = gl_fold_fast(__ldcg(A.ql + b + h), __ldcg(A.ql + b + 3 * h), rprev);
-                    s1 = gl_fold_fast(__ldcg(A.qr + b + h), __ldcg(A.qr + b + 3 * h), rprev);
-                }
-                A.pl[b] = p0;
-                A.pr[b] = r0;
-                A.ql[b] = q0;
-                A.qr[b] = s0;
-                A.pl[b + h] = p1;
-                A.pr[b + h] = r1;
-                A.ql[b + h] = q1;
-                A.qr[b + h] = s1;
+                // the children (the tree layer in round 2, the folded pairs after) folded by rho_(t-1)
+                const ulonglong2* sp = t == 2 ? A.P : A.pp;
+                const ulonglong2* sq = t == 2 ? A.Q : A.qq;
+                p0 = fold2(__ldcg(sp + b), __ldcg(sp + b + 2 * h), rprev);
+                q0 = fold2(__ldcg(sq + b), __ldcg(sq + b + 2 * h), rprev);
+                p1 = fold2(__ldcg(sp + b + h), __ldcg(sp + b + 3 * h), rprev);
+                q1 = fold2(__ldcg(sq + b + h), __ldcg(sq + b + 3 * h), rprev);
+                A.pp[b] = p0;
+                A.qq[b] = q0;
+                A.pp[b + h] = p1;
+                A.qq[b + h] = q1;
                 e = gl_add(__ldcg(A.E + b), __ldcg(A.E + b + h));  // eq(z_>t, b)
                 A.E[b] = e;
             }
-            a0.mac(e, layer_f(p0, r0, q0, s0, A.lam));
-            a1.mac(e, layer_f(p1, r1, q1, s1, A.lam));
-            a2.mac(e, layer_f(at2(p0, p1), at2(r0, r1), at2(q0, q1), at2(s0, s1), A.lam));
+            a0.mac(e, layer_f(p0, q0, A.lam));
+            if (need1) a1.mac(e, layer_f(p1, q1, A.lam));
+            a2.mac(e, layer_f(at2v(p0, p1), at2v(q0, q1), A.lam));
         }
         uint64_t acc[3] = {a0.value(), a1.value(), a2.value()};
         bool last;
@@ -183,20 +170,32 @@ __global__ void __launch_bounds__(SL_THREADS, 2) silu_layer_kernel(LayerArgs A, 
     if (A.t_end <= A.d || blockIdx.x != 0) return;
     if (!session_wait(mb, rl, A.seq0 + A.d, rprev)) return;
     if (threadIdx.x == 0) {
-        uint64_t fin[4];
-        if (A.d == 1) {
-            fin[0] = gl_fold_fast(A.P[0], A.P[2], rprev);
-            fin[1] = gl_fold_fast(A.P[1], A.P[3], rprev);
-            fin[2] = gl_fold_fast(A.Q[0], A.Q[2], rprev);
-            fin[3] = gl_fold_fast(A.Q[1], A.Q[3], rprev);
-        } else {
-            fin[0] = gl_fold_fast(__ldcg(A.pl), __ldcg(A.pl + 1), rprev);
-            fin[1] = gl_fold_fast(__ldcg(A.pr), __ldcg(A.pr + 1), rprev);
-            fin[2] = gl_fold_fast(__ldcg(A.ql), __ldcg(A.ql + 1), rprev);
-            fin[3] = gl_fold_fast(__ldcg(A.qr), __ldcg(A.qr + 1), rprev);
-        }
+        const ulonglong2* sp = A.d == 1 ? A.P : A.pp;
+        const ulonglong2* sq = A.d == 1 ? A.Q : A.qq;
+        const ulonglong2 pf = fold2(__ldcg(sp), __ldcg(sp + 1), rprev), qf = fold2(__ldcg(sq), __ldcg(sq + 1), rprev);
+        const uint64_t fin[4] = {pf.x, pf.y, qf.x, qf.y};
         session_publish(mb, fin, A.seq0 + A.d + 1);
     }
+}
+
+// 1 / z_i for every nonzero coordinate (one inversion for all), 0 where z_i = 0
+std::vector<uint64_t> inverses_or_zero(const uint64_t* z, int n) {
+    std::vector<uint64_t> inv(n, 0);
+    uint64_t run = 1;
+    for (int i = 0; i < n; i++) {
+        inv[i] = run;
+        if (z[i]) run = gl_mul(run, z[i]);
+    }
+    uint64_t r = gl_inv(run);
+    for (int i = n - 1; i >= 0; i--) {
+        if (!z[i]) {
+            inv[i] = 0;
+            continue;
+        }
+        inv[i] = gl_mul(inv[i], r);
+        r = gl_mul(r, z[i]);
+    }
+    return inv;
 }
 
 int64_t silu_q_host(int64_t v) { return (int64_t)floor((double)v / (1.0 + exp(-(double)v / 256.0)) + 0.5); }
@@ -262,7 +261,7 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
     const int vl = v / 2, vh = v - vl;
     size_t need = fp_align_up(4 * 65536, 256) + fp_align_up(8 * part_n, 256) + fp_align_up(8 * 64, 256) +
                   fp_align_up((size_t)8 << vh, 256) + fp_align_up((size_t)8 << vl, 256) +
-                  5 * fp_align_up((size_t)8 * hv, 256) + 4096;
+                  2 * fp_align_up((size_t)16 * hv, 256) + fp_align_up((size_t)8 * hv, 256) + 4096;
     for (int d = 1; d <= v; d++) need += 2 * fp_align_up((size_t)8 << d, 256);
     need += fp_hist::hist16_scratch();
     if ((rc = fp_reserve(c, c->dev, need))) return rc;
@@ -275,8 +274,10 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
     uint64_t* small = (uint64_t*)fp_alloc(c->dev, 8 * 64);  // [0..1] leaf values, [8..] the layer's point
     uint64_t* EH = (uint64_t*)fp_alloc(c->dev, (size_t)8 << vh);
     uint64_t* EL = (uint64_t*)fp_alloc(c->dev, (size_t)8 << vl);
-    uint64_t* vecs[5];
-    for (int i = 0; i < 5; i++) vecs[i] = (uint64_t*)fp_alloc(c->dev, (size_t)8 * hv);
+    // the layer's folded child pairs (p and q: 16 bytes per pair each) and its suffix eq table
+    ulonglong2* fpp = (ulonglong2*)fp_alloc(c->dev, (size_t)16 * hv);
+    ulonglong2* fqq = (ulonglong2*)fp_alloc(c->dev, (size_t)16 * hv);
+    uint64_t* fE = (uint64_t*)fp_alloc(c->dev, (size_t)8 * hv);
     std::vector<uint64_t*> TP(v + 1, nullptr), TQ(v + 1, nullptr);
     for (int d = 1; d <= v; d++) {
         TP[d] = (uint64_t*)fp_alloc(c->dev, (size_t)8 << d);
@@ -285,7 +286,7 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
     }
     uint8_t* hm = (uint8_t*)fp_alloc(c->host, 4 * 65536);
     uint64_t* hs = (uint64_t*)fp_alloc(c->host, 8 * 64);
-    if (!m || !hpart || !part || !small || !EH || !EL || !vecs[4] || !hm || !hs)
+    if (!m || !hpart || !part || !small || !EH || !EL || !fpp || !fqq || !fE || !hm || !hs)
         return fp_fail(c, FP_ERR_OOM, "logup_prove_silu: scratch exhausted");
 
     // ---- multiplicities ----
@@ -341,13 +342,11 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
         FP_CUDA(c, cudaMemcpyAsync(small + 8, hs + 8, 8 * (size_t)d, cudaMemcpyHostToDevice, st));
         LayerArgs A;
         memset(&A, 0, sizeof A);
-        A.P = TP[d + 1];
-        A.Q = TQ[d + 1];
-        A.pl = vecs[0];
-        A.pr = vecs[1];
-        A.ql = vecs[2];
-        A.qr = vecs[3];
-        A.E = vecs[4];
+        A.P = reinterpret_cast<const ulonglong2*>(TP[d + 1]);
+        A.Q = reinterpret_cast<const ulonglong2*>(TQ[d + 1]);
+        A.pp = fpp;
+        A.qq = fqq;
+        A.E = fE;
         A.z = small + 8;
         A.lam = lam;
         A.d = d;
@@ -372,6 +371,7 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
         }
         uint64_t pre = 1;  // eq(z_<t, rho_<t)
         std::vector<uint64_t> rho(d);
+        const std::vector<uint64_t> zinv = inverses_or_zero(z.z, d);
         for (int t = 1; t <= d; t++) {
             if (c->stepped) {
                 A.t_begin = A.t_end = t;
@@ -382,18 +382,16 @@ int lookup16_prove(fp_ctx* c, fp_tx* tx, const LookupLabels& lab, int64_t pad_s,
                 fp_toc(c, st, slot);
             }
             if ((rc = fp_session_wait(c, A.seq0 + t, st))) return rc;
-            const uint64_t h0 = c->mb->res[0], h1 = c->mb->res[1], h2 = c->mb->res[2];
+            // g(X) = pre eq(z_t, X) h(X); g(1) = claim - g(0), and h(1) = g(1) / (pre z_t) gives
+            // h(3) = h(0) - 3 h(1) + 3 h(2) (the device sends h(1) only when z_t = 0)
             const uint64_t zt = z.z[t - 1];
-            const uint64_t h3 = gl_add(gl_sub(h0, gl_mul(3, h1)), gl_mul(3, h2));
+            const uint64_t ph0 = gl_mul(pre, c->mb->res[0]), ph2 = gl_mul(pre, c->mb->res[2]);
             uint64_t gr[4];
-            gr[0] = gl_mul(pre, gl_mul(gl_sub(1, zt), h0));
-            gr[1] = gl_mul(pre, gl_mul(zt, h1));
-            gr[2] = gl_mul(pre, gl_mul(gl_sub(gl_mul(3, zt), 1), h2));
-            gr[3] = gl_mul(pre, gl_mul(gl_sub(gl_mul(5, zt), 2), h3));
-            if (gl_add(gr[0], gr[1]) != claim) {
-                fp_session_abandon(c, st);
-                return fp_fail(c, FP_ERR_CUDA, "logup_prove_silu: round values inconsistent with the claim");
-            }
+            gr[0] = gl_mul(gl_sub(1, zt), ph0);
+            gr[1] = gl_sub(claim, gr[0]);
+            const uint64_t ph1 = zt ? gl_mul(gr[1], zinv[t - 1]) : gl_mul(pre, c->mb->res[1]);
+            gr[2] = gl_mul(gl_sub(gl_mul(3, zt), 1), ph2);
+            gr[3] = gl_mul(gl_sub(gl_mul(5, zt), 2), gl_add(gl_sub(ph0, gl_mul(3, ph1)), gl_mul(3, ph2)));
             put_u64s(proof + pos, gr, 4);
             fp_tx_absorb_raw(tx, lab.round, proof + pos, 32);
             pos += 32;
