@@ -89,6 +89,32 @@ __device__ __forceinline__ uint64_t sub_i64(uint64_t alpha, int64_t v) {
     return x >= GL_P ? x - GL_P : x;
 }
 
+// Round 1 of the leaf layer sends, in place of h(2), the X^2 coefficient of h: the host takes
+// h(2) = 2 h(1) - h(0) + 2 C2 (h has degree 2, h(1) from the running claim or the device). With
+// leaves q = alpha - f and p = 1, the X^2 coefficient of a pair's F is
+// lambda dL0 dR0 + lambda^3 dL1 dR1, d = q(1) - q(0): for the remainder table the integer
+// r(0) - r(1), for the clamp table -((q'(1) - q'(0)) + gamma (y(1) - y(0))). So C2 needs no field
+// product for the remainder table (an exact integer product below 2^64) and one for the clamp.
+// e dL0 dR0 into ca, e dL1 dR1 into cb.
+__device__ __forceinline__ void leaf_c2(uint64_t e, const int32_t (&r0)[2], const int32_t (&q0)[2],
+                                        const int32_t (&y0)[2], const int32_t (&r1)[2], const int32_t (&q1)[2],
+                                        const int32_t (&y1)[2], uint64_t gamma, GlAcc& ca, GlAcc& cb) {
+    const int64_t dl = (int64_t)r0[0] - r1[0], dr = (int64_t)r0[1] - r1[1];
+    const uint64_t u = (uint64_t)(uint32_t)(dl < 0 ? -dl : dl) * (uint32_t)(dr < 0 ? -dr : dr);
+    const uint64_t uc = u >= GL_P ? u - GL_P : u;
+    ca.mac(e, ((dl < 0) != (dr < 0)) ? gl_sub(0, uc) : uc);
+    const uint64_t dL = sub_i64(gl_mul_small(gamma, y1[0] - y0[0]), (int64_t)q0[0] - q1[0]);
+    const uint64_t dR = sub_i64(gl_mul_small(gamma, y1[1] - y0[1]), (int64_t)q0[1] - q1[1]);
+    cb.mac(e, gl_mul_weak(dL, dR));
+}
+
+// lambda ca + lambda^3 cb as this thread's share of C2, in acc (cleared first)
+__device__ __forceinline__ void leaf_c2_close(GlAcc& acc, const GlAcc& cb, uint64_t lam, uint64_t lam2) {
+    const uint64_t a = acc.value(), b = cb.value();
+    acc = GlAcc();
+    acc.add(gl_mul(lam, gl_add(a, gl_mul(lam2, b))));
+}
+
 // leaf denominators alpha - f of key i for both tables
 __device__ __forceinline__ void leaf_den(const KeySrc& K, const Chal& C, int64_t i, uint64_t& d0, uint64_t& d1) {
     int32_t r, q, y;
@@ -752,6 +778,7 @@ __device__ __forceinline__ void leaf_round_piped(const GkrLayer& A, const uint64
                                                  unsigned active, uint64_t rprev, uint64_t lam, uint64_t lam2,
                                                  bool need1, GlAcc (&acc)[3]) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    GlAcc c2b;  // round 1: the clamp table's share of C2
     uint8_t* wbuf = pipe + (size_t)warp * kPipeStages * kPipeStage;
     const uint32_t wsa = (uint32_t)__cvta_generic_to_shared(wbuf);
     const int64_t first = (int64_t)blockIdx.x * blockDim.x + 32 * warp, stride = (int64_t)active * blockDim.x;
@@ -790,12 +817,7 @@ __device__ __forceinline__ void leaf_round_piped(const GkrLayer& A, const uint64
             int32_t r0[2], q0[2], y0[2], r1[2], q1[2], y1[2];
             pipe_key_pair(st, 0, lane, r0, q0, y0);
             pipe_key_pair(st, 1, lane, r1, q1, y1);
-            uint64_t pl[2] = {1, 1}, pr[2] = {1, 1}, ql[2], qr[2];
-            ql[0] = sub_i64(A.chal.alpha0, 2 * (int64_t)r1[0] - r0[0]);
-            ql[1] = sub_i64(ytab[2 * y1[0] - y0[0] + 384], 2 * (int64_t)q1[0] - q0[0]);
-            qr[0] = sub_i64(A.chal.alpha0, 2 * (int64_t)r1[1] - r0[1]);
-            qr[1] = sub_i64(ytab[2 * y1[1] - y0[1] + 384], 2 * (int64_t)q1[1] - q0[1]);
-            acc[1].mac(e, layer_F<true>(pl, pr, ql, qr, lam, lam2));
+            leaf_c2(e, r0, q0, y0, r1, q1, y1, A.chal.gamma, acc[1], c2b);
         } else {
             // fold positions (b, b + 2h) and (b + h, b + 3h) by the round-1 challenge
             uint64_t c0[2][2], c1[2][2];  // [table][leaf] at X = 0 (position b) and X = 1 (b + h)
@@ -844,6 +866,7 @@ __device__ __forceinline__ void leaf_round_piped(const GkrLayer& A, const uint64
         __syncwarp();  // the stage is refilled two chunks on
     }
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    if (T == 1) leaf_c2_close(acc[1], c2b, lam, lam2);
 }
 
 // Round t of layer d over the pairs b < h handled by this block.
@@ -862,17 +885,19 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* y
             leaf_round_piped<2>(A, ytab, pipe, EC, eq_tab, h, active, rprev, lam, lam2, need1, acc);
         return;
     }
+    GlAcc c2b;  // the leaf layer's round 1: the clamp table's share of C2
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < h; b += (int64_t)active * blockDim.x) {
         if (LEAF && t == 1) {
-            // X = 0 (and 1) from the stored level above the leaves; X = 2 from four denominators
-            // of integer-extrapolated keys
+            // X = 0 (and 1) from the stored level above the leaves; the X^2 coefficient C2 from
+            // the keys' differences
             const uint64_t e = eq_chunks_at(EC, eq_tab, b);  // E_1[b] = eq(z_2..z_d, b)
             if (A.d > 1) A.E[b] = e;
             acc[0].mac(e, parent_F(A, b, lam, lam2));
             if (need1) acc[2].mac(e, parent_F(A, b + h, lam, lam2));
-            uint64_t pl[2] = {1, 1}, pr[2] = {1, 1}, ql[2], qr[2];
-            leaf_pair_at2(A, ytab, b, h, ql, qr);
-            acc[1].mac(e, layer_F<true>(pl, pr, ql, qr, lam, lam2));
+            int32_t r0[2], q0[2], y0[2], r1[2], q1[2], y1[2];
+            key_pair(A.keys, A.keys_vec != 0, b, r0, q0, y0);
+            key_pair(A.keys, A.keys_vec != 0, b + h, r1, q1, y1);
+            leaf_c2(e, r0, q0, y0, r1, q1, y1, A.chal.gamma, acc[1], c2b);
             continue;
         }
         ulonglong2 c0p[2], c0q[2], c1p[2], c1q[2];
@@ -932,6 +957,7 @@ __device__ __forceinline__ void layer_round(const GkrLayer& A, const uint64_t* y
         }
         acc[1].mac(e, layer_F<LEAF>(pl, pr, ql, qr, lam, lam2));
     }
+    if (LEAF && t == 1) leaf_c2_close(acc[1], c2b, lam, lam2);
 }
 
 // The rest of a layer once one block holds all its pairs (h <= kTailPairs): the
@@ -997,8 +1023,16 @@ __device__ __forceinline__ void layer_tail(const GkrLayer& A, const uint64_t* yt
                 v[k] = xi == 0 ? c0 : xi == 1 ? gl_add(gl_sub(c1, c0), c1) : c1;
             }
             // v = pL, pR, qL, qR at X
-            const uint64_t u = gl_add(LEAF ? 1ull : v[1], gl_mul_weak(lam, v[3]));
-            uint64_t f = gl_muladd_weak(v[2], u, LEAF ? v[3] : gl_mul_weak(v[0], v[3]));
+            uint64_t f;
+            if (LEAF && t == 1 && xi == 1) {
+                // the leaf layer's round 1 sends C2: lambda (qL(1) - qL(0)) (qR(1) - qR(0))
+                const uint64_t dl = gl_sub(S[4 * tau + 2][b + h], S[4 * tau + 2][b]);
+                const uint64_t dr = gl_sub(S[4 * tau + 3][b + h], S[4 * tau + 3][b]);
+                f = gl_mul_weak(lam, gl_mul(dl, dr));
+            } else {
+                const uint64_t u = gl_add(LEAF ? 1ull : v[1], gl_mul_weak(lam, v[3]));
+                f = gl_muladd_weak(v[2], u, LEAF ? v[3] : gl_mul_weak(v[0], v[3]));
+            }
             if (tau) f = gl_mul_weak(lam2, f);
             if (xi == 0)
                 acc0.mac(Et[b], f);
@@ -1581,11 +1615,14 @@ int logup_prove_rescale(fp_ctx* c, fp_tx* tx, const fp_site* sites, int nsites, 
             if (t <= d) {
                 const uint64_t h0 = c->mb->res[0], h2 = c->mb->res[1], h1 = c->mb->res[2];
                 const uint64_t zt = zpt[t - 1];
-                const uint64_t ph0 = gl_mul(pre, h0), ph2 = gl_mul(pre, h2);
+                const uint64_t ph0 = gl_mul(pre, h0);
                 uint64_t g[4];
                 g[0] = gl_mul(gl_sub(1, zt), ph0);
                 g[1] = gl_sub(claim, g[0]);
                 const uint64_t ph1 = zt ? gl_mul(g[1], zinv[t - 1]) : gl_mul(pre, h1);
+                // the leaf layer's round 1 sends the X^2 coefficient C2: h(2) = 2 h(1) - h(0) + 2 C2
+                const uint64_t ph2 = (leaf && t == 1) ? gl_add(gl_sub(gl_add(ph1, ph1), ph0), gl_mul(pre, gl_add(h2, h2)))
+                                                      : gl_mul(pre, h2);
                 g[2] = gl_mul(gl_sub(gl_add(zt, gl_add(zt, zt)), 1), ph2);                  // eq(z_t, 2) = 3 z_t - 1
                 const uint64_t ph3 = gl_add(gl_sub(ph0, gl_add(ph1, gl_add(ph1, ph1))), gl_add(ph2, gl_add(ph2, ph2)));
                 g[3] = gl_mul(gl_sub(gl_add(gl_add(zt, zt), gl_add(zt, gl_add(zt, zt))), 2), ph3);  // 5 z_t - 2
