@@ -775,14 +775,17 @@ int64_t fp_ctx_launches(const fp_ctx* ctx);
 int fp_host_stats(const fp_ctx* ctx, double out[4]);
 int fp_kernel_stats(fp_ctx* ctx, fp_kernel_stat* out, int cap);
 /* Per-launch records of the same timing, in launch order: {kernel id, 0, device
- * ms of that launch, its algorithmic bytes}. Copies up to `cap` records into
- * `out` (host memory owned by the caller) and returns how many there are;
- * cleared by fp_ctx_set_profiling. */
+ * ms of that launch, its algorithmic bytes, the device ms from the first timed launch
+ * since fp_ctx_set_profiling to this launch's start (a timeline: the gaps between
+ * launches are host work and waits)}. Copies up to `cap` records into `out` (host
+ * memory owned by the caller) and returns how many there are; cleared by
+ * fp_ctx_set_profiling. */
 typedef struct {
     int32_t kernel;
     int32_t reserved;
     double ms;
     double bytes;
+    double start_ms;
 } fp_launch_rec;
 int64_t fp_kernel_log(fp_ctx* ctx, fp_launch_rec* out, int64_t cap);
 const char* fp_kernel_name(int kernel);

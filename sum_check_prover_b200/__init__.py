@@ -44,7 +44,8 @@ class _KStat(C.Structure):
 
 
 class _LRec(C.Structure):
-    _fields_ = [("kernel", C.c_int32), ("reserved", C.c_int32), ("ms", C.c_double), ("bytes", C.c_double)]
+    _fields_ = [("kernel", C.c_int32), ("reserved", C.c_int32), ("ms", C.c_double), ("bytes", C.c_double),
+                ("start_ms", C.c_double)]
 
 
 _lib = None
@@ -627,19 +628,74 @@ class SiteDesc:
         self.w_digest = w_digest
 
 
-def _sites(sites: Sequence[SiteDesc]):
+def _site_records(sites):
+    """The fp_site records of the sites as one numpy buffer laid out like _Site (filled a column
+    at a time: a layer has hundreds of sites), and the buffers they point into."""
+    import numpy as np
+    fields = [f for f, _ in _Site._fields_]
+    dt = np.dtype({"names": fields,
+                   "formats": [np.uint64 if t is C.c_void_p else np.int32 for _, t in _Site._fields_],
+                   "offsets": [getattr(_Site, f).offset for f in fields], "itemsize": C.sizeof(_Site)})
     n = len(sites)
-    arr = (_Site * n)()
-    keep = []
-    for i, s in enumerate(sites):
-        dg = None
-        if s.w_digest is not None:
-            b = C.create_string_buffer(bytes(s.w_digest), 64)
-            keep.append(b)
-            dg = C.addressof(b)
-        arr[i] = _Site(_ptr(s.w), _ptr(s.scales), _ptr(s.xt), _ptr(s.q), _ptr(s.r), _ptr(s.y),
-                       s.w_bits, s.M, s.K, s.N, s.k_shift, dg)
-    return arr, keep
+    rec = np.zeros(max(1, n), dtype=dt)
+    keep = [rec]
+    for f in ("w", "scales", "xt", "q", "r", "y"):
+        rec[f][:n] = [_ptr(getattr(x, f)) or 0 for x in sites]
+    for f in ("w_bits", "M", "K", "N", "k_shift"):
+        rec[f][:n] = [int(getattr(x, f)) for x in sites]
+    dig = [x.w_digest for x in sites]
+    if any(d is not None for d in dig):
+        if any(d is not None and len(bytes(d)) != 64 for d in dig):
+            raise ValueError("a weight digest is 64 bytes: D(W) || D(scales)")
+        buf = C.create_string_buffer(b"".join(bytes(d) if d is not None else bytes(64) for d in dig), 64 * n)
+        keep.append(buf)
+        base = C.addressof(buf)
+        rec["w_digest"][:n] = [base + 64 * i if d is not None else 0 for i, d in enumerate(dig)]
+    return rec, keep
+
+
+class SiteArray:
+    """Sites marshalled once for the C ABI: the device pointers and sizes are read when it is
+    built, so a proof that passes the same sites to several entry points reads them once. It
+    behaves as the list of its sites; build a new one after changing a site."""
+
+    def __init__(self, sites, _rec=None, _keep=None):
+        self.sites = list(sites)
+        if _rec is None:
+            _rec, _keep = _site_records(self.sites)
+        self.rec, self.keep = _rec, _keep
+        self.arr = (_Site * len(_rec)).from_buffer(_rec)
+
+    @staticmethod
+    def concat(parts: Sequence["SiteArray"]) -> "SiteArray":
+        import numpy as np
+        parts = [p for p in parts if len(p)]
+        if not parts:
+            return SiteArray([])
+        rec = np.zeros(sum(len(p) for p in parts), dtype=parts[0].rec.dtype)  # keeps _Site's padding
+        o = 0
+        for p in parts:
+            rec[o:o + len(p)] = p.rec[: len(p)]
+            o += len(p)
+        return SiteArray([x for p in parts for x in p.sites], rec, [k for p in parts for k in p.keep] + [rec])
+
+    def __len__(self):
+        return len(self.sites)
+
+    def __iter__(self):
+        return iter(self.sites)
+
+    def __getitem__(self, i):
+        return self.sites[i]
+
+
+def _as_array(sites) -> "SiteArray":
+    return sites if isinstance(sites, SiteArray) else SiteArray(sites)
+
+
+def _sites(sites: Sequence[SiteDesc]):
+    sites = _as_array(sites)
+    return sites.arr, [sites]
 
 
 class Transcript:
@@ -721,6 +777,7 @@ class Context:
         return a.value, b.value
 
     def prove_matmul(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None) -> bytes:
+        sites = _as_array(sites)
         arr, keep = _sites(sites)
         mm, _ = self.proof_size(sites)
         buf = C.create_string_buffer(max(1, mm))
@@ -739,6 +796,7 @@ class Context:
     def prove_matmul_shard(self, tx: Transcript, sites: Sequence[SiteDesc], shard: Shard, stream=None) -> bytes:
         """The matmul sum-check of a shared statement: this rank's sites on this GPU, the
         round sums exchanged; every rank returns the one-rank proof bytes."""
+        sites = _as_array(sites)
         arr, keep = _sites(sites)
         mm, _ = self.proof_size(sites)
         buf = C.create_string_buffer(max(1, mm))
@@ -953,6 +1011,7 @@ class Context:
 
     def prove_logup(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
         """Returns (proof bytes, status): status 1 means some key lies outside its table."""
+        sites = _as_array(sites)
         arr, keep = _sites(sites)
         _, lu = self.proof_size(sites)
         buf = C.create_string_buffer(max(1, lu))
@@ -1006,11 +1065,12 @@ class Context:
         return int(self._L.fp_ctx_launches(self.h))
 
     def kernel_log(self) -> list:
-        """[(kernel name, device ms, algorithmic bytes)] per timed launch, in launch order."""
+        """[(kernel name, device ms, algorithmic bytes, start ms from the first timed launch)] per
+        timed launch, in launch order."""
         n = self._check(self._L.fp_kernel_log(self.h, None, 0), "fp_kernel_log")
         arr = (_LRec * max(1, n))()
         n = self._check(self._L.fp_kernel_log(self.h, arr, n), "fp_kernel_log")
-        return [(self._L.fp_kernel_name(r.kernel).decode(), r.ms, r.bytes) for r in arr[:n]]
+        return [(self._L.fp_kernel_name(r.kernel).decode(), r.ms, r.bytes, r.start_ms) for r in arr[:n]]
 
     def kernel_stats(self) -> dict:
         """{kernel name: (launches, total ms, algorithmic bytes)} since the last reset."""
@@ -1033,9 +1093,10 @@ def prove(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], stream=
         raise ValueError("prove: lookup must be 'gkr' or 'hi'")
     tx = Transcript(seed)
     try:
-        for st in stages:
+        parts = [SiteArray(st) for st in stages]
+        for st in parts:
             ctx.commit_witness(tx, st, stream)
-        sites = [s for st in stages for s in st]
+        sites = SiteArray.concat(parts)
         s0 = tx.state()
         mm = ctx.prove_matmul(tx, sites, stream)
         s1 = tx.state()
@@ -1087,12 +1148,14 @@ def prove_ffn(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], gat
     tx = Transcript(seed)
     try:
         hidden = False
-        for i, st in enumerate(stages):
+        arrays = [SiteArray(st) for st in stages]
+        for i, st in enumerate(arrays):
             if not hidden and i == stage_of[id(d_site)]:
                 ctx.silu_inputs(y, g, s, s8, stream)
                 ctx.ffn_hidden(s8, u_site.y, kh, qh, rh, yh, stream)
                 hidden = True
             ctx.commit_witness(tx, st, stream)
+        sites = SiteArray.concat(arrays)
         parts = [ctx.prove_matmul(tx, sites, stream)]
         lu, status = ctx.prove_logup(tx, sites, stream)
         parts.append(lu)
@@ -1126,12 +1189,13 @@ def prove_shard(ctx: Context, seed: int, sites: Sequence[SiteDesc], shard: Shard
     status."""
     tx = Transcript(seed)
     try:
-        ctx.commit_witness_shard(tx, sites, shard, stream)
+        sa = SiteArray(sites)
+        ctx.commit_witness_shard(tx, sa, shard, stream)
         s0 = tx.state()
-        mm = ctx.prove_matmul_shard(tx, sites, shard, stream)
+        mm = ctx.prove_matmul_shard(tx, sa, shard, stream)
         s1 = tx.state()
-        full = gather_witness(sites)
-        lu, status = ctx.prove_logup(tx, full, stream)
+        full = gather_witness(list(sites))
+        lu, status = ctx.prove_logup(tx, SiteArray(full), stream)
         return mm + lu, [s0, s1, tx.state()], status
     finally:
         tx.close()

@@ -98,6 +98,7 @@ void fp_ctx_destroy(fp_ctx* c) {
         cudaEventDestroy(p.b);
     }
     for (auto e : c->ev_free) cudaEventDestroy(e);
+    if (c->ev_ref) cudaEventDestroy(c->ev_ref);
     if (c->dev.p) cudaFree(c->dev.p);
     if (c->dig.p) cudaFree(c->dig.p);
     if (c->host.p) cudaFreeHost(c->host.p);
@@ -295,6 +296,11 @@ void fp_tic(fp_ctx* c, cudaStream_t s, int kernel, double bytes, int* slot) {
     *slot = -1;
     c->launches++;
     if (!c->profiling) return;
+    if (!c->ref_set) {
+        if (!c->ev_ref) cudaEventCreate(&c->ev_ref);
+        cudaEventRecord(c->ev_ref, s);
+        c->ref_set = true;
+    }
     FpEvPair p;
     p.a = ev_get(c);
     p.b = ev_get(c);
@@ -313,12 +319,13 @@ void fp_toc(fp_ctx* c, cudaStream_t s, int slot) {
 static void stats_resolve(fp_ctx* c) {
     for (auto& p : c->ev_live) {
         cudaEventSynchronize(p.b);
-        float ms = 0.f;
+        float ms = 0.f, at = 0.f;
         cudaEventElapsedTime(&ms, p.a, p.b);
+        cudaEventElapsedTime(&at, c->ev_ref, p.a);
         c->stats[p.kernel].launches += 1;
         c->stats[p.kernel].ms += ms;
         c->stats[p.kernel].bytes += p.bytes;
-        c->log.push_back(fp_launch_rec{p.kernel, 0, (double)ms, p.bytes});
+        c->log.push_back(fp_launch_rec{p.kernel, 0, (double)ms, p.bytes, (double)at});
         c->ev_free.push_back(p.a);
         c->ev_free.push_back(p.b);
     }
@@ -340,6 +347,7 @@ int fp_ctx_set_profiling(fp_ctx* c, int on) {
     c->stepped = c->profiling == 1 || c->stepped_env;
     for (auto& s : c->stats) s = FpKStat();
     c->log.clear();
+    c->ref_set = false;
     return FP_OK;
 }
 

@@ -140,6 +140,8 @@ struct fp_ctx {
     double t_result = -1;     // arrival time of the last result (steady clock seconds), -1: none pending
     std::vector<FpEvPair> ev_live;
     std::vector<cudaEvent_t> ev_free;
+    cudaEvent_t ev_ref = nullptr;  // recorded before the first timed launch since profiling was set
+    bool ref_set = false;
     FpKStat stats[K_COUNT];
     std::vector<fp_launch_rec> log;  // every timed launch since profiling was switched on
 };
