@@ -132,6 +132,13 @@ int fp_tx_state(const fp_tx* tx, uint8_t out[32]);
 int fp_digest(fp_ctx* ctx, const void* dev, size_t nbytes, uint8_t out[32], void* stream);
 
 /*
+ * fp_digest of n device buffers in one pass (the chunks of all buffers hashed by the same
+ * launches): devs[i] (device, NULL allowed when nbytes[i] == 0) and nbytes[i] (host arrays of
+ * n entries); out: host, 32 n bytes, digest i at out + 32 i. n >= 1, else FP_ERR_ARG.
+ */
+int fp_digests(fp_ctx* ctx, const void* const* devs, const size_t* nbytes, int n, uint8_t* out, void* stream);
+
+/*
  * Witness and commitment of `nsites` products ("How fast can FlashProve go",
  * 3.1). For every site: Y = W_eff . X (exact int32 accumulation),
  * q = floor((Y + 2^(k-1)) / 2^k) (round half up), r = Y - 2^k q,
@@ -373,11 +380,15 @@ int fp_had2_protocol_drive(fp_tx* tx, int v, fp_values_fn fn, void* user, uint8_
  *   send Se~(rho), w~(rho) ("scl_final").
  * Se~(rho) equals S~(rho_row, rho_col_hi), rho_col_hi the first vK - 6 column
  * coordinates (none when vK <= 6). Proof: 8 + 32 (vM + vK) + 16 bytes.
+ * w_digest: host, the 64 bytes D(W) || D(S) when the weights were committed in advance
+ * (as fp_site.w_digest), or null to digest them here; a wrong value gives a proof the
+ * verifier rejects.
  * M, K >= 1 and vM + vK <= 30, else FP_ERR_SHAPE; null or non-canonical
  * arguments FP_ERR_ARG; proof / proof_len as for sumcheck_prove_matmul.
  */
 int sumcheck_reduce_scales(fp_ctx* ctx, fp_tx* tx, const void* w, int w_bits, const int8_t* scales, int M, int K,
-                           const uint64_t* point, uint8_t* proof, size_t* proof_len, void* stream);
+                           const uint64_t* point, const uint8_t* w_digest, uint8_t* proof, size_t* proof_len,
+                           void* stream);
 
 /*
  * SiLU by lookup ("How fast can FlashProve go", 2 Background and 3.1: the SiLU is

@@ -73,6 +73,7 @@ def lib():
     L.fp_tx_squeeze.argtypes = [vp, C.c_char_p, C.POINTER(u64), sz]
     L.fp_tx_state.argtypes = [vp, vp]
     L.fp_digest.argtypes = [vp, vp, sz, vp, vp]
+    L.fp_digests.argtypes = [vp, vp, vp, i32, vp, vp]
     L.fp_commit_witness.argtypes = [vp, vp, C.POINTER(_Site), i32, vp]
     L.mle_partial_eval.argtypes = [vp, vp, i32, vp, i32, i32, C.POINTER(u64), i32, vp, vp]
     L.sumcheck_prove_matmul.argtypes = [vp, vp, C.POINTER(_Site), i32, vp, C.POINTER(sz), vp]
@@ -94,7 +95,7 @@ def lib():
     L.fp_mm2_protocol_drive.argtypes = [vp, i32, i32, i32, _VALUES_FN, vp, vp, C.POINTER(sz)]
     L.logup_prove_helper_inverse.argtypes = [vp, vp, vp, C.c_int64, i32, vp, C.POINTER(sz), vp]
     L.fp_lhi_protocol_drive.argtypes = [vp, i32, i32, vp, vp, _VALUES_FN, vp, vp, C.POINTER(sz)]
-    L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, C.POINTER(sz), vp]
+    L.sumcheck_reduce_scales.argtypes = [vp, vp, vp, i32, vp, i32, i32, C.POINTER(u64), vp, vp, C.POINTER(sz), vp]
     L.logup_prove_silu.argtypes = [vp, vp, vp, vp, C.c_int64, vp, C.POINTER(sz), vp]
     L.fp_silu_table.argtypes = [vp]
     L.fp_silu_inputs.argtypes = [vp, vp, C.c_int64, vp, vp, vp, vp]
@@ -761,6 +762,15 @@ class Context:
         self._check(self._L.fp_digest(self.h, _ptr(dev), nbytes, out, _stream(stream)), "fp_digest")
         return out.raw
 
+    def digest_many(self, bufs: Sequence, stream=None) -> bytes:
+        """The digests of [(device buffer, nbytes), ...] in one pass, concatenated (32 bytes each)."""
+        n = len(bufs)
+        devs = (C.c_void_p * n)(*[_ptr(b) for b, _ in bufs])
+        lens = (C.c_size_t * n)(*[int(m) for _, m in bufs])
+        out = C.create_string_buffer(32 * n)
+        self._check(self._L.fp_digests(self.h, devs, lens, n, out, _stream(stream)), "fp_digests")
+        return out.raw
+
     def commit_witness(self, tx: Transcript, sites: Sequence[SiteDesc], stream=None):
         arr, keep = _sites(sites)
         self._check(self._L.fp_commit_witness(self.h, tx.h, arr, len(sites), _stream(stream)), "fp_commit_witness")
@@ -931,9 +941,14 @@ class Context:
         return buf.raw[: ln.value], rc
 
     def reduce_scales(self, tx: Transcript, w, bits: int, scales, M: int, K: int, point: Sequence[int],
-                      stream=None) -> bytes:
+                      stream=None, w_digest: Optional[bytes] = None) -> bytes:
         """Sum-check reducing a claim on the scaled weights' MLE at point (row coordinates
-        first) to claims on the weights w and the per-64-column scales (device tensors)."""
+        first) to claims on the weights w and the per-64-column scales (device tensors).
+        w_digest: D(W) || D(S) when the weights were committed in advance (64 bytes), else
+        they are digested here."""
+        if w_digest is not None and len(bytes(w_digest)) != 64:
+            raise ValueError("reduce_scales: w_digest is 64 bytes, D(W) || D(S)")
+        dg = C.create_string_buffer(bytes(w_digest), 64) if w_digest is not None else None
         v = 0
         while (1 << v) < M:
             v += 1
@@ -947,7 +962,7 @@ class Context:
         cap = 8 + 32 * v + 16
         buf = C.create_string_buffer(cap)
         ln = C.c_size_t(cap)
-        self._check(self._L.sumcheck_reduce_scales(self.h, tx.h, _ptr(w), bits, _ptr(scales), M, K, pt, buf,
+        self._check(self._L.sumcheck_reduce_scales(self.h, tx.h, _ptr(w), bits, _ptr(scales), M, K, pt, dg, buf,
                                                    C.byref(ln), _stream(stream)), "sumcheck_reduce_scales")
         return buf.raw[: ln.value]
 
@@ -1165,9 +1180,9 @@ def prove_ffn(ctx: Context, seed: int, stages: Sequence[Sequence[SiteDesc]], gat
             if d.scales is None:
                 continue
             vm, vk = _log2c(d.M), _log2c(d.K)
-            parts.append(ctx.reduce_scales(tx, d.w, d.w_bits, d.scales, d.M, d.K, r_row[:vm] + rho[nr - vk:], stream))
-        tx.absorb("ffn_hidden", ctx.digest(qh, 4 * n, stream) + ctx.digest(rh, 4 * n, stream)
-                  + ctx.digest(yh, n, stream))
+            parts.append(ctx.reduce_scales(tx, d.w, d.w_bits, d.scales, d.M, d.K, r_row[:vm] + rho[nr - vk:], stream,
+                                           w_digest=d.w_digest))
+        tx.absorb("ffn_hidden", ctx.digest_many([(qh, 4 * n), (rh, 4 * n), (yh, n)], stream))
         # the hidden rescale's keys as a lookup section's single site (M x N keys, table R_kh);
         # w and xt only satisfy the site checks, the lookup reads q, r and y
         hs = SiteDesc(w=s8, scales=None, xt=u_site.y, q=qh, r=rh, y=yh, M=g_site.M, K=1, N=g_site.N,

@@ -511,6 +511,17 @@ int fp_digest(fp_ctx* c, const void* dev, size_t nbytes, uint8_t out[32], void* 
     return fp_digest_many(c, &j, 1, out, (cudaStream_t)stream);
 }
 
+int fp_digests(fp_ctx* c, const void* const* devs, const size_t* nbytes, int n, uint8_t* out, void* stream) {
+    if (!c || !devs || !nbytes || !out || n < 1) return fp_fail(c, FP_ERR_ARG, "fp_digests: null argument");
+    std::vector<FpDigestJob> jobs((size_t)n);
+    for (int i = 0; i < n; i++) {
+        if (nbytes[i] && !devs[i]) return fp_fail(c, FP_ERR_ARG, "fp_digests: null buffer");
+        jobs[i] = FpDigestJob{(const uint8_t*)devs[i], (uint64_t)nbytes[i]};
+    }
+    FP_CUDA(c, cudaSetDevice(c->device));
+    return fp_digest_many(c, jobs.data(), n, out, (cudaStream_t)stream);
+}
+
 namespace {
 
 // the witness and digests of sites[0, nsites): 192-byte site records into rec

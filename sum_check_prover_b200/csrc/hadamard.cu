@@ -684,7 +684,8 @@ int sumcheck_prove_hadamard(fp_ctx* c, fp_tx* tx, const int8_t* s, const int8_t*
 }
 
 int sumcheck_reduce_scales(fp_ctx* c, fp_tx* tx, const void* w, int w_bits, const int8_t* scales, int M, int K,
-                           const uint64_t* point, uint8_t* proof, size_t* proof_len, void* stream) {
+                           const uint64_t* point, const uint8_t* w_digest, uint8_t* proof, size_t* proof_len,
+                           void* stream) {
     if (!c || !tx || !proof_len || !point) return fp_fail(c, FP_ERR_ARG, "sumcheck_reduce_scales: null argument");
     if (!w || !scales) return fp_fail(c, FP_ERR_ARG, "sumcheck_reduce_scales: null weights or scales");
     if (w_bits != 4 && w_bits != 8) return fp_fail(c, FP_ERR_ARG, "sumcheck_reduce_scales: w_bits must be 4 or 8");
@@ -704,7 +705,9 @@ int sumcheck_reduce_scales(fp_ctx* c, fp_tx* tx, const void* w, int w_bits, cons
     int rc;
     const int64_t pitch = w_bits == 4 ? (K + 1) / 2 : K;
     const int G = (K + 63) / 64;
-    {
+    if (w_digest) {
+        fp_tx_absorb_raw(tx, "scl_site", w_digest, 64);  // committed in advance
+    } else {
         FpDigestJob jobs[2] = {{(const uint8_t*)w, (uint64_t)M * (uint64_t)pitch},
                                {(const uint8_t*)scales, (uint64_t)M * (uint64_t)G}};
         uint8_t d[64];

@@ -92,6 +92,17 @@ PE_SHAPES = [
 ]
 
 
+def test_digests_in_one_pass_match_one_by_one(env):
+    torch, fp, ctx = env
+    rng = np.random.default_rng(8)
+    bufs = [torch.from_numpy(rng.integers(0, 256, n, dtype=np.uint8)).cuda() for n in (1, 1024, 5000, 1 << 20)]
+    pairs = [(b, b.numel()) for b in bufs] + [(bufs[2][7:], bufs[2].numel() - 7), (None, 0)]
+    got = ctx.digest_many(pairs)
+    want = b"".join(ctx.digest(b, n) for b, n in pairs)
+    assert got == want
+    assert got[:32] == oracle.tree_digest(bufs[0].cpu().numpy().tobytes())
+
+
 @pytest.mark.parametrize("shape", PE_SHAPES)
 def test_partial_eval_matches_oracle(env, shape):
     torch, fp, ctx = env

@@ -68,6 +68,21 @@ def test_matches_oracle(env, M, K, bits):
     assert (pf, st) == oracle.scl_prove(6, w, bits, sc, M, K, z)
 
 
+def test_committed_digest_gives_the_same_proof(env):
+    # D(W) || D(S) committed in advance (the site's weight digest) stands in for digesting here
+    torch, fp, ctx = env
+    M, K, bits = 37, 300, 4
+    w, sc, z = _site(M, K, bits, 5)
+    wd = torch.from_numpy(np.ascontiguousarray(w)).cuda()
+    sd = torch.from_numpy(np.ascontiguousarray(sc)).cuda()
+    dg = ctx.digest(wd, wd.numel()) + ctx.digest(sd, sd.numel())
+    tx = fp.Transcript(4)
+    pf = ctx.reduce_scales(tx, wd, bits, sd, M, K, z, w_digest=dg)
+    assert (pf, tx.state()) == oracle.scl_prove(4, w, bits, sc, M, K, z)
+    with pytest.raises(ValueError):
+        ctx.reduce_scales(fp.Transcript(4), wd, bits, sd, M, K, z, w_digest=dg[:32])
+
+
 def test_stepped_and_resident_give_the_same_proof(env):
     torch, fp, ctx = env
     M, K, bits = 500, 3000, 4
