@@ -796,9 +796,12 @@ def run_ours(args):
         if d.xt.data_ptr() not in seen:
             seen.add(d.xt.data_ptr())
             host_x.append((d, d.xt.cpu().pin_memory()))
-    host_y = [(d, torch.empty(d.y.shape, dtype=torch.int8).pin_memory()) for d in flat]
+    # the outputs: the column buffer that holds every ungrouped site's y, and each output group
+    col_y = keep["columns"][2]
+    dev_y = ([col_y] if any(s.out_group is None for s in wl.sites) else []) + [g["y"] for g in keep["groups"].values()]
+    host_y = [(y, torch.empty(y.shape, dtype=torch.int8).pin_memory()) for y in dev_y]
     h2d = sum(x.numel() for _, x in host_x)
-    d2h = sum(y.numel() for _, y in host_y) + proof_len
+    d2h = sum(y.numel() for y, _ in host_y) + proof_len
     e2e_ms = []
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
@@ -806,8 +809,8 @@ def run_ours(args):
         for d, x in host_x:
             d.xt.copy_(x, non_blocking=True)
         step(args.seed + 300 + i)
-        for d, y in host_y:
-            y.copy_(d.y, non_blocking=True)
+        for y, h in host_y:
+            h.copy_(y, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
