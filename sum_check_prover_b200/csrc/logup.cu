@@ -502,10 +502,42 @@ __device__ __forceinline__ void key_subtree(const KeySrc& K, const Chal& C, cons
 __global__ void __launch_bounds__(kKeyTreeThreads, FP_TREE_KEYS_MIN_BLOCKS) tree_keys_kernel(KeySrc K, Chal C, KeyTreeOut out, int64_t nchunks) {
     __shared__ uint64_t ytab[256];
     __shared__ uint64_t wnode[2][2][8];  // [table][P, Q][warp]: each warp's level v - 9 node
+    // every node over padding keys only (the neutral key 0: leaf alpha0, and alpha1 - gamma 0) has
+    // one value per level and table: [level][table][P, Q]
+    __shared__ uint64_t padc[kKeyTreeLevels][2][2];
     leaf_ytab_build(C, ytab);
+    __syncthreads();
+    if (threadIdx.x < 2) {
+        const int t = threadIdx.x;
+        const uint64_t a = t == 0 ? sub_i32(C.alpha0, 0) : sub_i32(ytab[128], 0);
+        uint64_t p = gl_add(a, a), q = gl_mul(a, a);
+        for (int l = 0; l < kKeyTreeLevels; l++) {
+            padc[l][t][0] = p;
+            padc[l][t][1] = q;
+            uint64_t np, nq;
+            tree_up(p, q, p, q, np, nq);
+            p = np;
+            q = nq;
+        }
+    }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int64_t ch = blockIdx.x; ch < nchunks; ch += gridDim.x) {
+        if (ch * 4096 >= K.n) {
+            // a chunk of padding only: every level's nodes are the level's constants (block-uniform)
+#pragma unroll 1
+            for (int l = 0; l < kKeyTreeLevels; l++) {
+                const int nl = 2048 >> l;  // the chunk's nodes at level v - 1 - l
+                const int64_t g0 = ch * nl;
+#pragma unroll
+                for (int t = 0; t < 2; t++)
+                    for (int i = threadIdx.x; i < nl; i += blockDim.x) {
+                        out.lay[l].P[t][g0 + i] = padc[l][t][0];
+                        out.lay[l].Q[t][g0 + i] = padc[l][t][1];
+                    }
+            }
+            continue;
+        }
         const int64_t leaf0 = ch * 4096 + 16 * (int64_t)threadIdx.x;
         uint64_t P[2][1], Q[2][1];  // the thread's level v - 4 node per table
         key_subtree<0>(K, C, ytab, out, ch, leaf0, P[0][0], Q[0][0]);
