@@ -115,7 +115,12 @@ __global__ void had2_single_kernel(const int8_t* s, const int8_t* u, uint64_t* o
     out[5] = 0;
 }
 
-__global__ void __launch_bounds__(H2_THREADS, 2) had2_session_kernel(Had2Args A, FpMailbox* mb, FpRelay* rl,
+// two blocks per SM: bounded to three (80 registers) the extension products spill and the
+// 2^26-entry rounds slow down (3.56 -> 3.74 ms)
+#ifndef FP_HAD2_MIN_BLOCKS
+#define FP_HAD2_MIN_BLOCKS 2
+#endif
+__global__ void __launch_bounds__(H2_THREADS, FP_HAD2_MIN_BLOCKS) had2_session_kernel(Had2Args A, FpMailbox* mb, FpRelay* rl,
                                                                     uint64_t* part) {
     __shared__ Ext2 zs[32];
     __shared__ Ext2 tab[4 << H2_CHUNK];
