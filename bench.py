@@ -855,16 +855,32 @@ def run_ours(args):
                 "host_turnaround_us_per_round": host_turn_us,
                 "host_wait_ms_per_step": host_wait_ms,
                 "clocks": clk,
+                "proof_bytes": proof_len,
+                "pages_context": PAGES_CONTEXT,
                 "kernels": kern,
                 "kernels_stepped": kern_stepped,
                 "lookup_variants": variants,
                 "microbench": micro,
-                "proof_bytes": proof_len,
-                "pages_context": PAGES_CONTEXT}
+                # last, so that a reader who keeps only the end of the output still sees it
+                "summary": compact_summary(rows, micro, kern, variants)}
         print(json.dumps(line), flush=True)
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
+
+
+def compact_summary(rows, micro, kern, variants):
+    """The figures of the long keys in a few hundred bytes: each scope row's fraction of the HBM
+    peak inside the proof, each microbench's time and fraction, the kernels above 0.2 ms per
+    proof and the two lookup variants' times."""
+    def r3(x):
+        return None if x is None else round(float(x), 3)
+    out = {"rows_frac": {k: r3(v.get("frac")) for k, v in (rows or {}).items()},
+           "micro_ms_frac": {k: [r3(v.get("ms")), r3(v.get("frac"))] for k, v in (micro or {}).items()},
+           "kernels_ms": {k: round(v["ms"], 2) for k, v in (kern or {}).items() if v.get("ms", 0) >= 0.2}}
+    if variants:
+        out["lookup_variants_ms"] = {k: r3(v.get("ms_per_step")) for k, v in variants.items()}
+    return out
 
 
 def main():
